@@ -1,0 +1,432 @@
+"""Pins of the CPU oracle to facts fixed outside the oracle itself.
+
+Each test checks an oracle function against something the pages or the mathematics fix:
+a printed example (tests/golden), a closed form, exact rational arithmetic, brute force
+on tiny inputs, an invariant, or a special case that reduces to a textbook rule.  The
+cases are chosen so that a dropped term, a wrong sign or index, a transposed operand or
+a wrong tie rule fails at least one of them.
+"""
+import itertools
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import hinm_inputs as hi
+from oracle import hinm_oracle as O
+
+
+def bf(a):
+    return hi.f32_to_bf16_bits(np.asarray(a, dtype=np.float32))
+
+
+def f32(bits):
+    return hi.bf16_bits_to_f32(bits)
+
+
+# ----------------------------------------------------------------------------- importance
+def test_energy_closed_form_ones():
+    # X = 1 everywhere: s_c = N exactly, I = w^2 * N.
+    K, N = 7, 13
+    X = bf(np.ones((K, N)))
+    assert np.array_equal(O.channel_energy(X), np.full(K, N, dtype=np.float32))
+    W = bf([[0.5, -2.0, 3.0, 0.25, 1.0, -1.5, 0.125]])
+    I = O.importance(W, X)
+    np.testing.assert_array_equal(I[0], np.array([0.25, 4.0, 9.0, 0.0625, 1.0, 2.25, 0.015625],
+                                                 dtype=np.float32) * N)
+
+
+def test_importance_hand_example_not_transposed():
+    # W = [[1, 2], [3, 0.5]], X = [[1, 1, 1], [2, 0, 0]]  ->  s = [3, 4]
+    # I = [[1*3, 4*4], [9*3, 0.25*4]] = [[3, 16], [27, 1]]
+    W = bf([[1.0, 2.0], [3.0, 0.5]])
+    X = bf([[1.0, 1.0, 1.0], [2.0, 0.0, 0.0]])
+    np.testing.assert_array_equal(O.channel_energy(X), np.array([3.0, 4.0], dtype=np.float32))
+    np.testing.assert_array_equal(O.importance(W, X), np.array([[3, 16], [27, 1]], dtype=np.float32))
+
+
+def test_importance_exact_rational():
+    rng = np.random.default_rng(3)
+    M, K, N = 5, 6, 9
+    W = bf(rng.normal(0, 0.3, (M, K)))
+    X = bf(rng.normal(0, 1.0, (K, N)))
+    I = O.importance(W, X)
+    for c in range(K):
+        exact = sum(Fraction(float(x)) ** 2 for x in f32(X[c]))
+        s32 = np.float32(float(exact))          # tiny sums are exact in fp64
+        for i in range(M):
+            w = Fraction(float(f32(W[i, c])))
+            want = np.float32(float(w * w * Fraction(float(s32))))
+            assert I[i, c] == want
+
+
+# ----------------------------------------------------------------------------- counts
+def test_closed_form_triples(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "closed_form_boundaries.json")))
+    for tr in g["triples"]:
+        assert O.partial_sparsity(tr["t_s"], tr["v_s"]) == pytest.approx(tr["p_s"], abs=1e-12)
+        # and the forward form t_s = v_s + (1 - v_s) p_s / 2
+        assert tr["v_s"] + (1 - tr["v_s"]) * tr["p_s"] * 0.5 == pytest.approx(tr["t_s"], abs=1e-12)
+    assert len(O.LEGAL_NIBBLES) == g["patterns_per_group_of_4"] == math.comb(4, 2)
+
+
+@pytest.mark.parametrize("K,t_s,v_s,want", [
+    (256, 0.5, 0.2, (52, 152, 52)),
+    (4096, 0.5, 0.0, (0, 4096, 0)),
+    (4096, 0.75, 0.6, (2458, 1228, 410)),
+    (11008, 0.625, 0.4, (4404, 4952, 1652)),
+    (4096, 0.5, 0.5, (2048, 0, 2048)),      # p_s = 0: pure column pruning
+    (4096, 0.0, 0.0, (0, 0, 4096)),         # dense
+    (4096, 1.0, 1.0, (4096, 0, 0)),         # everything pruned
+])
+def test_counts_table(K, t_s, v_s, want):
+    assert O.counts_from_vs(K, t_s, v_s) == want
+
+
+def test_counts_invariants():
+    for K in (64, 100, 256, 1000, 4096, 11008):
+        for t_s in (0.5, 0.625, 0.75, 0.875):
+            if t_s * K != int(t_s * K):
+                continue
+            for m in range(0, 40):
+                v_s = t_s - m / 32.0
+                if v_s < max(0.0, 2 * t_s - 1):
+                    break
+                try:
+                    n0, n24, n4 = O.counts_from_vs(K, t_s, v_s)
+                except ValueError:
+                    continue
+                assert n0 + n24 + n4 == K
+                assert n24 % 4 == 0
+                # overall sparsity is exactly t_s: kept = n4 + n24/2 = (1 - t_s) K
+                assert n4 * 2 + n24 == 2 * K - 2 * int(t_s * K)
+                if v_s < 1:
+                    p_s = O.partial_sparsity(t_s, v_s)
+                    assert abs(n24 - p_s * (K - n0)) <= 4
+
+
+def test_counts_rejects():
+    with pytest.raises(ValueError):
+        O.counts_from_vs(100, 0.333, 0.1)       # t_s K not whole
+    with pytest.raises(ValueError):
+        O.counts_from_vs(256, 0.75, 0.3)        # v_s < 2 t_s - 1 -> n_4 < 0
+
+
+def test_search_candidates_span():
+    c = O.search_candidates(4096, 0.75, 1 / 32)
+    assert len(c) == 9 and c[0] == (3072, 0, 1024) and c[-1] == (2048, 2048, 0)
+    c = O.search_candidates(4096, 0.5, 1 / 32)
+    assert len(c) == 17 and c[-1] == (0, 4096, 0)
+    c = O.search_candidates(11008, 0.625, 1 / 32)
+    assert len(c) == 13
+
+
+# ----------------------------------------------------------------------------- 2:4 selection
+def brute_pair(v):
+    """Max-sum pair over all C(4,2) pairs, exact sums, ties -> lexicographically smallest."""
+    best = None
+    for a, b in itertools.combinations(range(4), 2):
+        s = Fraction(float(v[a])) + Fraction(float(v[b]))
+        if best is None or s > best[0]:
+            best = (s, (a, b))
+    return best[1]
+
+
+def test_top2_matches_brute_force_all_ties():
+    for v in itertools.product([0.0, 1.0, 2.0], repeat=4):
+        keep = O.top2_keep(np.array(v, dtype=np.float32))
+        assert keep.sum() == 2
+        assert tuple(np.nonzero(keep)[0]) == brute_pair(v)
+
+
+def test_top2_matches_brute_force_random():
+    rng = np.random.default_rng(11)
+    vals = rng.random((5000, 4)).astype(np.float32) ** 3
+    keep = O.top2_keep(vals)
+    assert (keep.sum(axis=1) == 2).all()
+    for r in range(vals.shape[0]):
+        assert tuple(np.nonzero(keep[r])[0]) == brute_pair(vals[r])
+
+
+def test_magnitude_24_special_case():
+    """X = 1: I = w^2 N, and with v_s = 0 (all vectors 2:4) and the identity order the
+    mask is plain magnitude 2:4 along the input dimension (rkmt.cn, section 二)."""
+    rng = np.random.default_rng(5)
+    M, K, N, T = 8, 32, 4, 8
+    W = bf(rng.normal(0, 1, (M, K)))
+    Wf = f32(W)
+    # distinct magnitudes in every group, so no tie rule is involved
+    for i in range(M):
+        for g in range(K // 4):
+            assert len(set(np.abs(Wf[i, 4 * g:4 * g + 4]).tolist())) == 4
+    X = bf(np.ones((K, N)))
+    I = O.importance(W, X)
+    counts = np.tile(np.array(O.counts_from_vs(K, 0.5, 0.0)), (M // T, 1))
+    bm, region = O.mask(I, np.arange(K, dtype=np.int32), T, counts)
+    keep = O.unpack_bits(bm, K)
+    want = np.zeros((M, K), dtype=bool)
+    for i in range(M):
+        for g in range(K // 4):
+            top = np.argsort(-np.abs(Wf[i, 4 * g:4 * g + 4]))[:2]
+            want[i, 4 * g + top] = True
+    assert np.array_equal(keep, want)
+    assert (region == O.REGION_24).all()
+
+
+def test_column_pruning_special_case():
+    """v_s = t_s (p_s = 0): HiNM reduces to whole-column pruning of the lowest vectors."""
+    rng = np.random.default_rng(8)
+    M, K, N, T = 16, 24, 5, 8
+    W = bf(rng.normal(0, 1, (M, K)))
+    X = bf(rng.normal(0, 1, (K, N)))
+    perm = rng.permutation(K).astype(np.int32)
+    I = O.importance(W, X)
+    counts = np.tile(np.array(O.counts_from_vs(K, 0.5, 0.5)), (M // T, 1))
+    bm, region = O.mask(I, perm, T, counts)
+    keep = O.unpack_bits(bm, K)
+    Id = I.astype(np.float64)
+    for t in range(M // T):
+        # independent: sum each channel's importance over the tile, keep the top half
+        score = {c: sum(float(Id[t * T + i, c]) for i in range(T)) for c in range(K)}
+        pos = {int(c): j for j, c in enumerate(perm)}
+        kept = sorted(range(K), key=lambda c: (-score[c], pos[c]))[:K // 2]
+        want = np.zeros(K, dtype=bool)
+        want[kept] = True
+        for i in range(T):
+            assert np.array_equal(keep[t * T + i], want)
+        assert set(np.nonzero(region[t] == O.REGION_DENSE)[0]) == set(kept)
+
+
+def test_structured_pruning_golden(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "structured_pruning_3x3.json")))
+    W = bf(g["W"])
+    # column pruning: the mask drops column 1 entirely
+    keep = np.ones((3, 3), dtype=bool)
+    keep[:, g["pruned_column"]] = False
+    got = O.masked_weight(W, O.pack_bits(keep))
+    np.testing.assert_allclose(got, f32(bf(g["W_pruned_col"])), rtol=0, atol=0)
+    # row pruning
+    keep = np.ones((3, 3), dtype=bool)
+    keep[g["pruned_row"], :] = False
+    np.testing.assert_allclose(O.masked_weight(W, O.pack_bits(keep)), f32(bf(g["W_pruned_row"])),
+                               rtol=0, atol=0)
+    # unstructured magnitude pruning at the printed threshold
+    keep = np.abs(f32(W)) > g["threshold"]
+    np.testing.assert_allclose(O.masked_weight(W, O.pack_bits(keep)),
+                               f32(bf(g["W_pruned_threshold"])), rtol=0, atol=0)
+
+
+# ----------------------------------------------------------------------------- search
+def exact_R(I_tile_w, keep):
+    return sum((Fraction(float(v)) for v in I_tile_w[keep].astype(np.float64)), Fraction(0))
+
+
+def test_fsum_is_exactly_rounded():
+    rng = np.random.default_rng(1)
+    for _ in range(200):
+        vals = (rng.random(50) * 2.0 ** rng.integers(-40, 40, 50)).astype(np.float32).astype(np.float64)
+        ex = sum((Fraction(v) for v in vals), Fraction(0))
+        assert math.fsum(vals.tolist()) == float(ex)
+    vals = [2.0 ** 60] + [1.0] * 1000
+    assert math.fsum(vals) == float(sum(Fraction(v) for v in vals))
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_search_brute_force(seed):
+    rng = np.random.default_rng(seed)
+    M, K, N, T = 16, 64, 6, 8
+    W = bf(rng.normal(0, 1, (M, K)) * rng.random(K) ** 4)      # uneven column magnitudes
+    X = bf(rng.normal(0, 1, (K, N)))
+    perm = rng.permutation(K).astype(np.int32)
+    I = O.importance(W, X)
+    sr = O.boundary_search(I, perm, T, 0.5, 1 / 32)
+    cands = O.search_candidates(K, 0.5, 1 / 32)
+    for t in range(M // T):
+        I_tile_w = I[t * T:(t + 1) * T][:, perm]
+        # independent ranking of working positions by exact tile sums
+        sums = [sum(Fraction(float(I_tile_w[i, j])) for i in range(T)) for j in range(K)]
+        order = sorted(range(K), key=lambda j: (-sums[j], j))
+        R = []
+        for (n0, n24, n4) in cands:
+            keep = np.zeros((T, K), dtype=bool)
+            dense = order[:n4]
+            mid = sorted(order[n4:n4 + n24])
+            keep[:, dense] = True
+            for gi in range(0, len(mid), 4):
+                grp = mid[gi:gi + 4]
+                for i in range(T):
+                    a, b = brute_pair([I_tile_w[i, j] for j in grp])
+                    keep[i, grp[a]] = keep[i, grp[b]] = True
+            R.append(exact_R(I_tile_w, keep))
+        assert [float(r) for r in R] == sr.R[t]
+        first_drop = next((m for m in range(len(R) - 1) if float(R[m + 1]) < float(R[m])),
+                          len(R) - 1)
+        assert sr.m[t] == first_drop
+        assert tuple(sr.counts[t]) == cands[first_drop]
+        assert sr.v_s[t] == 0.5 - first_drop / 32
+        total = sum(Fraction(float(v)) for v in I_tile_w.ravel())
+        assert all(r <= total for r in R)
+
+
+def test_search_first_drop_hand_built():
+    """Hand-built tile (K = 64, t_s = 0.5, alpha = 1/32, X = 1, |w| constant per column).
+
+    Column magnitudes by working position: 0..27 -> 8, 28..29 -> 3, 30..31 -> 2.875,
+    32..33 -> 1.25, 34..35 -> 1, 36..63 -> 0.5 (so rank == position).
+      m=0: dense 0..31                       R0 = 28*64 + 2*9 + 2*8.265625
+      m=1: dense 0..29, 2:4 {30..33}         keeps 30,31 -> R1 == R0 (no strict drop)
+      m=2: dense 0..27, 2:4 {28..31},{32..35} keeps 28,29 and 32,33 -> R2 < R1
+    so the scan stops at m = 1 (v_s = 0.5 - 1/32).  Moving from m=0 to m=1 can never lose
+    importance (the band's per-row top-2 includes the two vectors that left the dense
+    region); only regrouping at m >= 1 can."""
+    K, N, T = 64, 4, 8
+    mags = np.array([8.0] * 28 + [3.0] * 2 + [2.875] * 2 + [1.25] * 2 + [1.0] * 2 + [0.5] * 28)
+    signs = np.where(np.random.default_rng(0).random((T, K)) < 0.5, -1.0, 1.0)
+    W = bf(signs * mags[None, :])
+    X = bf(np.ones((K, N)))
+    I = O.importance(W, X)
+    sr = O.boundary_search(I, np.arange(K, dtype=np.int32), T, 0.5, 1 / 32)
+    R = sr.R[0]
+    unit = T * N
+    assert R[0] == unit * (28 * 64 + 2 * 9 + 2 * 8.265625)
+    assert R[1] == R[0]
+    assert R[2] == unit * (28 * 64 + 2 * 9 + 2 * 1.5625)
+    assert sr.m[0] == 1 and sr.v_s[0] == 0.5 - 1 / 32
+    assert tuple(sr.counts[0]) == (30, 4, 30)
+
+
+def test_search_runs_to_end_gaussian():
+    """Gaussian weights: 2:4 keeps more importance than column pruning, R rises all the
+    way and the scan ends at v_s = max(0, 2 t_s - 1)."""
+    w = hi.custom(256, 256, 16, 64, seed=0, t_s=0.5, v_s=None)
+    I = O.importance(w.W_bits, w.X_bits)
+    sr = O.boundary_search(I, w.perm, 64, 0.5, 1 / 32)
+    assert (sr.m == 16).all() and (sr.v_s == 0.0).all()
+    for R in sr.R:
+        assert all(R[m + 1] >= R[m] for m in range(len(R) - 1))
+
+
+# ----------------------------------------------------------------------------- mask
+@pytest.mark.parametrize("T", [64, 128])
+def test_mask_counts_invariants(T):
+    w = hi.custom(2 * T, 200, 8, T, seed=9, t_s=0.625, v_s=0.4, random_perm=True)
+    I = O.importance(w.W_bits, w.X_bits)
+    counts = np.tile(np.array(O.counts_from_vs(200, 0.625, 0.4)), (2, 1))
+    bm, region = O.mask(I, w.perm, T, counts)
+    keep = O.unpack_bits(bm, 200)
+    n0, n24, n4 = counts[0]
+    assert keep.sum() == (1 - 0.625) * 2 * T * 200
+    assert (bm[:, -1] >> np.uint32(200 % 32) == 0).all()      # bits past K are zero
+    for t in range(2):
+        reg_w = region[t][w.perm]
+        assert (reg_w == O.REGION_DENSE).sum() == n4 and (reg_w == O.REGION_24).sum() == n24
+        kt = keep[t * T:(t + 1) * T][:, w.perm]
+        assert kt[:, reg_w == O.REGION_DENSE].all()
+        assert not kt[:, reg_w == O.REGION_PRUNED].any()
+        g = O.groups_24(reg_w)
+        assert (kt[:, g].sum(axis=-1) == 2).all()
+
+
+def test_permutation_invariance():
+    """Reordering input channels consistently does not change the computation
+    (FlexHiNM-GP notes, 关键设计 2): run(W, X, pi) == run(W[:, pi], X[pi, :], id)."""
+    w = hi.custom(128, 192, 24, 64, seed=12, t_s=0.625, v_s=None, random_perm=True)
+    a = O.hot_path(w.W_bits, w.X_bits, w.perm, 64, 0.625)
+    Wp = np.ascontiguousarray(w.W_bits[:, w.perm])
+    Xp = np.ascontiguousarray(w.X_bits[w.perm, :])
+    b = O.hot_path(Wp, Xp, np.arange(192, dtype=np.int32), 64, 0.625)
+    assert np.array_equal(a["counts"], b["counts"])
+    ka = O.unpack_bits(a["bitmask"], 192)
+    kb = O.unpack_bits(b["bitmask"], 192)
+    assert np.array_equal(ka[:, w.perm], kb)
+    La, Lb = a["layout"], b["layout"]
+    assert np.array_equal(La.vals_dense, Lb.vals_dense)
+    assert np.array_equal(La.vals_sparse, Lb.vals_sparse)
+    assert np.array_equal(La.meta, Lb.meta)
+    assert np.array_equal(La.tile_info, Lb.tile_info)
+    # idx_a = pi[idx_b] on real entries (padding is 0 on both sides)
+    for ia, ib in ((La.idx_dense, Lb.idx_dense), (La.idx_sparse, Lb.idx_sparse)):
+        real = ~((ia == 0) & (ib == 0))
+        assert np.array_equal(ia[real], w.perm[ib[real]])
+    assert np.array_equal(a["y"], b["y"])
+
+
+def test_tile_permutation_permutes_rows():
+    w = hi.custom(192, 128, 8, 64, seed=21, t_s=0.5, v_s=0.25)
+    a = O.hot_path(w.W_bits, w.X_bits, w.perm, 64, 0.5, v_s=0.25)
+    order = [2, 0, 1]
+    rows = np.concatenate([np.arange(t * 64, (t + 1) * 64) for t in order])
+    b = O.hot_path(np.ascontiguousarray(w.W_bits[rows]), w.X_bits, w.perm, 64, 0.5, v_s=0.25)
+    assert np.array_equal(a["y"][rows], b["y"])
+    assert np.array_equal(a["bitmask"][rows], b["bitmask"])
+
+
+# ----------------------------------------------------------------------------- layout
+def test_swizzle_and_meta_bijections():
+    offs = {O.swizzled_offset(r, k) for r in range(128) for k in range(64)}
+    assert offs == set(range(0, 16384, 2))
+    slots = {O.meta_word_index(m, g) for m in range(128) for g in range(32)}
+    assert slots == {(w, 4 * n) for w in range(512) for n in range(8)}
+
+
+@pytest.mark.parametrize("T,K,t_s,v_s,perm", [
+    (64, 256, 0.5, 0.2, False), (128, 200, 0.625, 0.4, True), (64, 96, 0.75, 0.5, True)])
+def test_compress_round_trip(T, K, t_s, v_s, perm):
+    w = hi.custom(2 * T, K, 8, T, seed=3, t_s=t_s, v_s=v_s, random_perm=perm)
+    I = O.importance(w.W_bits, w.X_bits)
+    counts = np.tile(np.array(O.counts_from_vs(K, t_s, v_s)), (2, 1))
+    bm, region = O.mask(I, w.perm, T, counts)
+    L = O.compress(w.W_bits, bm, region, w.perm, counts, T)
+    np.testing.assert_array_equal(L.tile_info[:, 0], -(-counts[:, 2] // 64))
+    np.testing.assert_array_equal(L.tile_info[:, 1], -(-counts[:, 1] // 128))
+    Wm = O.masked_weight(w.W_bits, bm).astype(np.float32)
+    np.testing.assert_array_equal(O.decompress(L), Wm)
+    nib = (L.meta[:, :, None] >> (4 * np.arange(8, dtype=np.uint32))) & np.uint32(0xF)
+    assert set(np.unique(nib).tolist()) <= set(O.LEGAL_NIBBLES)
+    n0, n24, n4 = counts[0]
+    # padded index entries are 0; real entries are distinct channels of the right region
+    for t in range(2):
+        nd, ns, d0, s0 = L.tile_info[t]
+        dense_idx = L.idx_dense[d0:d0 + nd].ravel()[:n4]
+        assert set(dense_idx.tolist()) == set(np.nonzero(region[t] == O.REGION_DENSE)[0].tolist())
+        assert (L.idx_dense[d0:d0 + nd].ravel()[n4:] == 0).all()
+        sp_idx = L.idx_sparse[s0:s0 + ns].ravel()[:n24]
+        assert set(sp_idx.tolist()) == set(np.nonzero(region[t] == O.REGION_24)[0].tolist())
+
+
+# ----------------------------------------------------------------------------- spmm reference
+def test_spmm_identity_x_gives_masked_weight():
+    w = hi.custom(128, 64, 64, 64, seed=2, t_s=0.5, v_s=0.25)
+    I = O.importance(w.W_bits, w.X_bits)
+    counts = np.tile(np.array(O.counts_from_vs(64, 0.5, 0.25)), (2, 1))
+    bm, _ = O.mask(I, w.perm, 64, counts)
+    eye = bf(np.eye(64))
+    y, bound = O.spmm_reference(w.W_bits, bm, eye)
+    np.testing.assert_array_equal(y, O.masked_weight(w.W_bits, bm))
+    np.testing.assert_array_equal(bound, np.abs(O.masked_weight(w.W_bits, bm)))
+
+
+def test_spmm_dense_case_triple_loop():
+    """t_s = 0 keeps everything: y = W X, checked against a plain triple loop."""
+    w = hi.custom(64, 16, 3, 64, seed=6, t_s=0.0, v_s=0.0)
+    r = O.hot_path(w.W_bits, w.X_bits, w.perm, 64, 0.0, v_s=0.0)
+    Wf, Xf = f32(w.W_bits).astype(np.float64), f32(w.X_bits).astype(np.float64)
+    for i in range(64):
+        for n in range(3):
+            acc = Fraction(0)
+            for c in range(16):
+                acc += Fraction(float(Wf[i, c])) * Fraction(float(Xf[c, n]))
+            assert abs(r["y"][i, n] - float(acc)) <= 1e-12 * max(1.0, abs(float(acc)))
+    assert O.unpack_bits(r["bitmask"], 16).all()
+
+
+def test_spmm_integer_exact():
+    w = hi.integer_workload(128, 128, 16, 64, seed=1, t_s=0.5, v_s=0.25, random_perm=True)
+    r = O.hot_path(w.W_bits, w.X_bits, w.perm, 64, 0.5, v_s=0.25)
+    assert np.array_equal(r["y"], np.round(r["y"]))
+    Wm = O.masked_weight(w.W_bits, r["bitmask"]).astype(np.int64)
+    Xi = f32(w.X_bits).astype(np.int64)
+    assert np.array_equal(r["y"].astype(np.int64), Wm @ Xi)
