@@ -1,0 +1,397 @@
+#!/usr/bin/env python
+"""Benchmark of the HiNM hot path on B200: importance -> boundary search -> mask ->
+compress -> SpMM, one pass per step, on the pure 2:4 workload
+(W 4096x4096 bf16 ~N(0,0.02) with 1% x10 outliers, X 4096x2048 bf16 ~N(0,1), tile 128,
+t_s = 0.5, v_s from the search, alpha = 1/32).
+
+Prints ONE JSON line (rank 0).  `value` is the effective (dense-equivalent) TFLOP/s of the
+whole step, 2*M*K*N per step over all ranks / max-over-ranks step time; the per-kernel
+breakdown, the roofline of the dominant kernel, the end-to-end number through host
+buffers and the CPU oracle baseline are extra keys.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {hinm,reference}]
+Multi-GPU: launched with torch.distributed.run, one rank per GPU; every rank runs its own
+seeded shard of the same shape (weak scaling, no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import hinm_inputs as hi  # noqa: E402
+
+METRIC = "HiNM SpMM TFLOP/s (eff.) and HBM GB/s, % of 2:4-sparse/HBM roofline"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks sampling
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in self.rows for k in range(4) if r[5 + k] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+# ------------------------------------------------------------------ workload accounting
+def workload_model(M, K, N, T, counts):
+    """Algorithmic FLOPs and bytes per step from the region counts actually used."""
+    n0, n24, n4 = (int(x) for x in np.asarray(counts).sum(axis=0))  # summed over tiles
+    nt = M // T
+    kept = T * (n4 + n24 // 2)                       # kept weights
+    flops_eff = 2.0 * M * K * N                      # dense-equivalent
+    flops_dense = 2.0 * T * n4 * N                   # real dense-region MACs x2
+    flops_sparse_eq = 2.0 * T * n24 * N              # 2:4 region, dense-equivalent
+    spmm_bytes = (2.0 * kept + T * n24 / 8.0 + 4.0 * (n4 + n24) + 2.0 * K * N + 4.0 * M * N)
+    return dict(
+        flops_eff=flops_eff, flops_actual=2.0 * kept * N, flops_dense=flops_dense,
+        flops_sparse_eq=flops_sparse_eq, kept=kept,
+        bytes=dict(importance=2.0 * M * K + 2.0 * K * N + 4.0 * M * K + 8.0 * K,
+                   search=4.0 * M * K + 4.0 * nt * K,
+                   mask=4.0 * M * K + M * ((K + 31) // 32) * 4.0 + nt * K,
+                   compress=2.0 * M * K + M * ((K + 31) // 32) * 4.0 + nt * K
+                   + 2.0 * kept + T * n24 / 8.0 + 4.0 * (n4 + n24),
+                   spmm=spmm_bytes))
+
+
+def roofline_for(phase, t_s, model, peaks, peak_kind):
+    """(bound, achieved, peak, unit, frac) of one kernel phase."""
+    hbm = peaks["hbm_gbs"]
+    if phase == "spmm":
+        # tensor time at the measured dense bf16 peak and twice it for the 2:4 region
+        # (the nominal 2:4 ratio); report the dense-equivalent rate against the mix.
+        dense_peak = peaks["bf16_tflops"]
+        t_tensor = (model["flops_dense"] / (dense_peak * 1e12)
+                    + model["flops_sparse_eq"] / (2.0 * dense_peak * 1e12))
+        t_hbm = model["bytes"]["spmm"] / (hbm * 1e9)
+        if t_tensor >= t_hbm:
+            eff_peak = (model["flops_dense"] + model["flops_sparse_eq"]) / t_tensor / 1e12
+            achieved = (model["flops_dense"] + model["flops_sparse_eq"]) / t_s / 1e12
+            return "tensor", achieved, eff_peak, "TFLOP/s", achieved / eff_peak
+        achieved = model["bytes"]["spmm"] / t_s / 1e9
+        return "hbm", achieved, hbm, "GB/s", achieved / hbm
+    achieved = model["bytes"][phase] / t_s / 1e9
+    return "hbm", achieved, hbm, "GB/s", achieved / hbm
+
+
+# ------------------------------------------------------------------ reference arm
+def cpu_oracle_sample(w, tiles_n: int):
+    """Run the CPU oracle on `tiles_n` tiles of the workload; returns (seconds, flops_eff)."""
+    from oracle import hinm_oracle as O
+    M, K, N, T = w.M, w.K, w.N, w.T
+    tiles = list(range(tiles_n))
+    rows = np.arange(0, tiles_n * T)
+    t0 = time.perf_counter()
+    s = O.channel_energy(w.X_bits)
+    Wf = hi.bf16_bits_to_f32(w.W_bits[rows])
+    I = np.zeros((M, K), dtype=np.float32)
+    I[rows] = ((Wf * Wf).astype(np.float32) * s[None, :]).astype(np.float32)
+    sr = O.boundary_search(I, w.perm, T, w.t_s, w.alpha, tiles=tiles)
+    bm, reg = O.mask(I, w.perm, T, sr.counts, tiles=tiles)
+    O.compress(w.W_bits, bm, reg, w.perm, sr.counts, T, tiles=tiles)
+    O.spmm_reference(w.W_bits, bm, w.X_bits, rows=rows)
+    dt = time.perf_counter() - t0
+    return dt, 2.0 * len(rows) * K * N
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from threadpoolctl import threadpool_limits
+    cores = cpu_cores()
+    tiles_n = 2
+    with threadpool_limits(limits=cores):
+        for _ in range(args.warmup):
+            cpu_oracle_sample(w, 1)
+        times, flops = [], 0.0
+        for _ in range(args.steps):
+            dt, fl = cpu_oracle_sample(w, tiles_n)
+            times.append(dt)
+            flops = fl
+    t = statistics.mean(times)
+    value = flops / t / 1e12
+    sample = (f"{tiles_n} of {w.M // w.T} tiles ({tiles_n * w.T} output rows) of {w.name} per step: "
+              "channel energies over all of X, then importance, search, mask, compress and the "
+              "fp64 masked product for those rows")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "T": w.T,
+                       "t_s": w.t_s, "alpha": w.alpha},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="hinm", choices=["hinm", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    w = hi.pure24(seed=rank)
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import pruning_hinm_spmm_b200 as H
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    M, K, N, T = w.M, w.K, w.N, w.T
+    dev = torch.device("cuda", local_rank)
+    W = torch.from_numpy(w.W_bits.view(np.int16)).to(dev).view(torch.bfloat16)
+    X = torch.from_numpy(w.X_bits.view(np.int16)).to(dev).view(torch.bfloat16)
+    perm = torch.from_numpy(w.perm).to(dev)
+    hp = H.HotPath(M, K, N, T, w.t_s, w.alpha, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    phases = ["importance", "search", "mask", "compress", "spmm"]
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        H.hinm_importance(W, X, hp.I, hp.ws)
+        if ev is not None:
+            ev[1].record(stream)
+        H.hinm_boundary_search(hp.I, perm, T, w.t_s, w.alpha, hp.counts, hp.vs, hp.rank, hp.ws)
+        if ev is not None:
+            ev[2].record(stream)
+        H.hinm_mask(hp.I, perm, hp.counts, T, hp.rank, hp.bitmask, hp.region, hp.ws)
+        if ev is not None:
+            ev[3].record(stream)
+        H.hinm_compress(W, hp.bitmask, hp.region, perm, hp.counts, T, hp.layout, hp.ws)
+        if ev is not None:
+            ev[4].record(stream)
+        H.hinm_spmm(hp.layout, X, hp.Y, None, hp.c_layout)
+        if ev is not None:
+            ev[5].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = H.hinm_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+    counts = hp.counts.cpu().numpy()
+    vs = hp.vs.cpu().numpy()
+    model = workload_model(M, K, N, T, counts)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    vis = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    sampler = ClockSampler(vis[local_rank].strip() if local_rank < len(vis) else local_rank)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.4)
+    for k in range(args.steps):
+        flush.zero_()                     # evict L2 (256 MB > 126 MB) between timed steps
+        step(evs[k])
+    torch.cuda.synchronize()
+    sampler.stop()
+    if dist:
+        dist.barrier()
+    per_phase = {p: [evs[k][i].elapsed_time(evs[k][i + 1]) * 1e-3 for k in range(args.steps)]
+                 for i, p in enumerate(phases)}
+    step_s = [evs[k][0].elapsed_time(evs[k][5]) * 1e-3 for k in range(args.steps)]
+    t_step = statistics.mean(step_s)
+    if dist:
+        tt = torch.tensor([t_step], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_step = float(tt.item())
+    value = model["flops_eff"] * world / t_step / 1e12
+
+    # ---------------- end to end through the public API with host buffers
+    W_h = torch.from_numpy(w.W_bits.view(np.int16)).pin_memory()
+    X_h = torch.from_numpy(w.X_bits.view(np.int16)).pin_memory()
+    P_h = torch.from_numpy(w.perm).pin_memory()
+    Y_h = torch.empty((M, N), dtype=torch.float32).pin_memory()
+    W_d = torch.empty_like(W)
+    X_d = torch.empty_like(X)
+    P_d = torch.empty_like(perm)
+
+    def e2e_step():
+        W_d.view(torch.int16).copy_(W_h, non_blocking=True)
+        X_d.view(torch.int16).copy_(X_h, non_blocking=True)
+        P_d.copy_(P_h, non_blocking=True)
+        hp.run(W_d, X_d, P_d)
+        Y_h.copy_(hp.Y, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, min(args.steps, 10))
+    if dist:
+        dist.barrier()
+    e_start.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = e_start.elapsed_time(e_end) * 1e-3 / e2e_steps
+    if dist:
+        tt = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_e2e = float(tt.item())
+    h2d = W_h.numel() * 2 + X_h.numel() * 2 + P_h.numel() * 4
+    d2h = Y_h.numel() * 4
+    # the e2e output must match the device-resident path
+    assert torch.equal(Y_h, hp.Y.cpu())
+
+    if dist:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_kind = load_peaks()
+    mean_phase = {p: statistics.mean(v) for p, v in per_phase.items()}
+    kernels = {}
+    for p in phases:
+        bound, ach, pk, unit, frac = roofline_for(p, mean_phase[p], model, peaks, peak_kind)
+        kernels[p] = {"ms": mean_phase[p] * 1e3, "bound": bound, "achieved": ach, "peak": pk,
+                      "unit": unit, "frac": frac}
+    dom = max(phases, key=lambda p: mean_phase[p])
+    traffic = None
+    tr_path = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tr_path):
+        traffic = json.load(open(tr_path)).get(dom)
+    roof = {"bound": kernels[dom]["bound"], "achieved": kernels[dom]["achieved"],
+            "peak": kernels[dom]["peak"], "unit": kernels[dom]["unit"],
+            "frac": kernels[dom]["frac"], "traffic": traffic, "kernel": dom,
+            "peak_source": f"{peak_kind} (MEASURED_PEAKS.json burst; 2:4 = 2x dense bf16)"}
+    spmm_t = mean_phase["spmm"]
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        from threadpoolctl import threadpool_limits
+        cores = cpu_cores()
+        with threadpool_limits(limits=cores):
+            dt, fl = cpu_oracle_sample(w, 8)
+        cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"8 of {M // T} tiles (1024 output rows) of {w.name}: channel energies, "
+                         "importance, search, mask, compress and fp64 masked product",
+               "seconds": dt}
+    clocks = sampler.summary()
+    kernels_per_step = 2 + 4 + 3 + 3 + 1
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "M": M, "K": K, "N": N, "T": T, "t_s": w.t_s,
+                   "alpha": w.alpha, "v_s_found": sorted(set(np.round(vs, 6).tolist())),
+                   "counts_tile0": counts[0].tolist(),
+                   "l2": "flushed between timed steps (256 MB write)",
+                   "step": "importance+search+mask+compress+spmm",
+                   "parallelism": f"{world} independent shard(s), no collective"},
+        "spmm_only": {"ms": spmm_t * 1e3, "tflops_eff": model["flops_eff"] / spmm_t / 1e12,
+                      "tflops_actual": model["flops_actual"] / spmm_t / 1e12,
+                      "gbs": model["bytes"]["spmm"] / spmm_t / 1e9},
+        "kernels": kernels,
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": model["flops_eff"] * world / t_e2e / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": t_e2e * 1e3},
+        "gpu_launches": kernels_per_step * args.steps,
+        "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                   "reasons": clocks["reasons"], "samples": clocks["samples"]},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -27,9 +27,10 @@ import numpy as np
 
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
     """Round fp32 values to bf16 (round-to-nearest-even), returning uint16 bit patterns."""
-    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    lsb = (u >> np.uint64(16)) & np.uint64(1)
-    r = (u + np.uint64(0x7FFF) + lsb) >> np.uint64(16)
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+    lsb = (u >> np.uint32(16)) & np.uint32(1)
+    # finite values stay below 0xFF800000, so the 32-bit sum cannot wrap
+    r = (u + (np.uint32(0x7FFF) + lsb)) >> np.uint32(16)
     return r.astype(np.uint16)
 
 

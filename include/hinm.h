@@ -1,0 +1,203 @@
+/*
+ * hinm.h -- C ABI of the B200 (sm_100a) hierarchical N:M (HiNM) hot path:
+ *
+ *     Y = W_HiNM . X
+ *
+ * W (M x K, bf16) is cut into tiles of T output rows.  In every tile each input channel
+ * restricted to the tile's rows (a "vector") is assigned to one of three regions --
+ * dense 4:4, 2:4, or pruned 0:4 -- and the 2:4 vectors keep 2 of every 4 per row.  The
+ * product runs on the compressed dense values, the compressed 2:4 values with their
+ * 2-bit metadata, and an index of surviving vectors with the input-channel permutation
+ * folded in.
+ *
+ * Sources (page title, section):
+ *   [P1] "FlexHiNM-GP: Flexible Hierarchical Pruning via Region Allocation and Channel
+ *        Permutation" (papernotes.org notes): 整体框架, 关键设计 1 (three regions, closed
+ *        form t_s = v_s + (1 - v_s) p_s / 2, scan of v_s from t_s downward stopping at
+ *        the first drop of retained second-order importance), 关键设计 2 (channel
+ *        permutation folded into the HiNM index), 关键设计 4 (dense part + 2:4 part
+ *        gathered by the precomputed index, summed into one output).
+ *   [P2] "面向Transformer的块稀疏剪枝：N:M稀疏模式在硬件加速上的优势" (rkmt.cn), section 二:
+ *        keep 2 of every 4 consecutive elements along the input dimension.
+ *   [P3] "结构化稀疏与剪枝:2:4 稀疏模式为何能让 GPU 矩阵吞吐翻倍" (geek-doc.cn), section 三:
+ *        2 stored values per group plus 2-bit positions; section 五: layer uses W ⊙ M.
+ *
+ * Conventions shared by every call
+ *   - Matrices are row-major and dense: W is M x K, X is K x N, Y is M x N, I is M x K.
+ *     bf16 arguments are passed as 16-bit bit patterns (const void*).
+ *   - Pointers are DEVICE pointers unless the name ends in _host.  The caller owns all
+ *     memory; the library never allocates, frees or synchronises, except the *_size
+ *     helpers and hinm_counts_from_vs, which run on the host only.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *     Work is enqueued asynchronously on it.
+ *   - Argument checks run on the host before any launch; a failed check returns an error
+ *     status and launches nothing.  hinm_last_error() then describes it.
+ *   - Faults detected on the device (a malformed mask in hinm_compress, a wait that
+ *     timed out inside a kernel) set a library-owned device status word; kernels then
+ *     finish without hanging or trapping.  hinm_device_status() reads and clears it.
+ *   - Supported sizes: T in {64, 128}; M % T == 0; 4 <= K <= 16384 and K % 4 == 0;
+ *     N % 8 == 0 (16-byte rows for the tensor-memory-accelerator copies); all device
+ *     pointers 16-byte aligned; X must be finite (padding multiplies row 0 of X by 0).
+ *   - No exception crosses the ABI.
+ */
+#ifndef HINM_H_
+#define HINM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define HINM_ABI_VERSION 1
+#define HINM_LAYOUT_VERSION 1
+
+typedef enum {
+  HINM_OK = 0,
+  HINM_ERR_INVALID_ARG = 1,      /* null pointer, NaN parameter, bad enum */
+  HINM_ERR_SHAPE = 2,            /* sizes violate the supported-size rules above */
+  HINM_ERR_ALIGNMENT = 3,        /* a device pointer is not 16-byte aligned */
+  HINM_ERR_UNSUPPORTED = 4,      /* a valid request this build does not implement */
+  HINM_ERR_CUDA = 5,             /* a CUDA runtime call failed (launch, memcpy, ...) */
+  HINM_ERR_DEVICE_TIMEOUT = 6,   /* device status: a bounded wait gave up */
+  HINM_ERR_BAD_MASK = 7,         /* device status: a 2:4 group without exactly 2 kept */
+  HINM_ERR_WORKSPACE = 8         /* workspace pointer null or smaller than required */
+} hinm_status;
+
+/* Region codes written by hinm_mask (one int8 per tile and input channel). */
+#define HINM_REGION_PRUNED 0     /* 0:4 -- vector removed */
+#define HINM_REGION_24 1         /* 2:4 -- 2 of every 4 kept per row */
+#define HINM_REGION_DENSE 2      /* 4:4 -- vector kept whole */
+
+/* Static description of the strings/versions. */
+const char* hinm_status_string(int status);
+const char* hinm_last_error(void);          /* detail of the last error on this host thread */
+int hinm_abi_version(void);
+
+/* ---------------------------------------------------------------------------------
+ * a1. Importance  ([P1] 关键设计 1 "二阶重要度", 关键设计 2 "D 是重要度矩阵")
+ *   s_c    = sum_{n=0..N-1} x_cn^2, accumulated in fp64 with n ascending, rounded to fp32
+ *   I[i,c] = fl32( fl32(w_ic^2) * s_c )
+ * W: bf16 [M][K]; X: bf16 [K][N]; I_out: fp32 [M][K] (written in full).
+ * workspace: hinm_importance_workspace_size() bytes (holds s, one fp32 per channel).
+ * -------------------------------------------------------------------------------- */
+hinm_status hinm_importance_workspace_size(int M, int K, int N, size_t* bytes_host);
+hinm_status hinm_importance(const void* W, const void* X, int M, int K, int N,
+                            float* I_out, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * Region counts for a fixed boundary (host only).  ([P1] 关键设计 1, closed form)
+ *   n_24 = 4 * floor(2 (t_s - v_s) K / 4 + 1/2), n_0 = t_s K - n_24 / 2,
+ *   n_4 = K - n_0 - n_24.   t_s K must be whole and every count >= 0.
+ * out_host[3] = { n_0, n_24, n_4 }.
+ * -------------------------------------------------------------------------------- */
+hinm_status hinm_counts_from_vs(int K, double t_s, double v_s, int32_t* out_host);
+
+/* ---------------------------------------------------------------------------------
+ * a2 + a3. Boundary search  ([P1] 整体框架: every tile runs it; 关键设计 1)
+ * Per tile t:
+ *   V[t,j]  = sum over the tile's rows (ascending, fp64) of I[row, perm[j]]
+ *   rank    = working positions ordered by (V descending, j ascending)
+ *   for m = 0..m_max, v_s = t_s - m * alpha, counts from the closed form above;
+ *     m_max = floor((t_s - max(0, 2 t_s - 1)) / alpha), trailing candidates with a
+ *     negative count dropped; dense = first n_4 ranks, 2:4 = next n_24 (grouped by 4 in
+ *     ascending working position, top-2 of I per row, lower position wins ties);
+ *     R(m) = exact sum of the importance of every kept element, rounded once to fp64.
+ *   Result: the first m with R(m+1) < R(m), else m_max.
+ * I: fp32 [M][K]; perm: int32 [K] (NULL = identity), working position j holds channel
+ * perm[j]; counts_out: int32 [M/T][3] = {n_0, n_24, n_4}; vs_out: fp64 [M/T];
+ * rank_out (NULL allowed): int32 [M/T][K], rank of working position j.
+ * alpha > 0, 0 <= t_s <= 1.  workspace: hinm_search_workspace_size() bytes.
+ * -------------------------------------------------------------------------------- */
+hinm_status hinm_search_workspace_size(int M, int K, int T, double t_s, double alpha,
+                                       size_t* bytes_host);
+hinm_status hinm_boundary_search(const float* I, const int32_t* perm, int M, int K, int T,
+                                 double t_s, double alpha, int32_t* counts_out,
+                                 double* vs_out, int32_t* rank_out, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * a4. Mask  ([P1] 亮点与洞察: high -> dense, middle -> 2:4, low -> pruned;
+ *            [P2] 二: 2 of every 4; [P3] 五: M has W's shape)
+ * counts: int32 [M/T][3] (device; n_24 % 4 == 0, n_0 + n_24 + n_4 == K);
+ * rank: int32 [M/T][K] from hinm_boundary_search, or NULL to recompute it from I.
+ * bitmask_out: uint32 [M][ceil(K/32)], bit b of word w of row i = channel 32w+b kept
+ * (bits past K are 0).  region_out: int8 [M/T][K] by original channel (HINM_REGION_*).
+ * workspace: hinm_mask_workspace_size() bytes.
+ * -------------------------------------------------------------------------------- */
+hinm_status hinm_mask_workspace_size(int M, int K, int T, size_t* bytes_host);
+hinm_status hinm_mask(const float* I, const int32_t* perm, const int32_t* counts,
+                      const int32_t* rank, int M, int K, int T, uint32_t* bitmask_out,
+                      int8_t* region_out, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * a5. Compressed HiNM layout  ([P1] 关键设计 2/4, [P3] 三)
+ * Per tile: dense vectors (ascending working position) in blocks of 64, 2:4 vectors in
+ * blocks of 128 (32 groups of 4).  Every block is 128 rows (rows >= T are zero) and is
+ * stored exactly as the tensor cores read it from shared memory:
+ *   value block  16384 B: bf16 (r, k) at r*128 + ((k/8) XOR (r%8))*16 + (k%8)*2
+ *                (dense: k = vector in block; 2:4: k = 2*group + slot, slot 0 = lower
+ *                kept position);
+ *   meta block    2048 B: 128 lanes x 4 uint32 words; word w of lane L, bits
+ *                [16s+4q, 16s+4q+4) = a | b<<2 (a < b, kept positions 0..3) of group
+ *                8w + 4((L/8)%2) + q of row 16(L/16) + 8s + L%8;
+ *   index         int32 per vector = perm[j] (input channel), 0 for padding.
+ * Padding: value 0, nibble 0x4, index 0.
+ * tile_info[t] = { dense blocks, sparse blocks, first dense block, first sparse block }.
+ * -------------------------------------------------------------------------------- */
+typedef struct {
+  int32_t layout_version;     /* must be HINM_LAYOUT_VERSION */
+  int32_t M, K, T, num_tiles; /* num_tiles = M / T */
+  int32_t max_dense_blocks;   /* capacity of vals_dense / idx_dense in blocks */
+  int32_t max_sparse_blocks;  /* capacity of vals_sparse / meta / idx_sparse in blocks */
+  int32_t* tile_info;         /* device int32 [num_tiles][4] (written by hinm_compress) */
+  uint16_t* vals_dense;       /* device bf16 [max_dense_blocks][8192] */
+  uint16_t* vals_sparse;      /* device bf16 [max_sparse_blocks][8192] */
+  uint32_t* meta;             /* device uint32 [max_sparse_blocks][512] */
+  int32_t* idx_dense;         /* device int32 [max_dense_blocks][64] */
+  int32_t* idx_sparse;        /* device int32 [max_sparse_blocks][128] */
+} hinm_layout;
+
+typedef struct {
+  int32_t max_dense_blocks, max_sparse_blocks;
+  size_t tile_info_bytes, vals_dense_bytes, vals_sparse_bytes, meta_bytes,
+      idx_dense_bytes, idx_sparse_bytes;
+} hinm_layout_sizes;
+
+/* Buffer sizes.  counts_host (int32 [M/T][3], host) gives exact sizes; NULL gives the
+ * worst case over all valid counts (ceil(K/64)+1 dense and ceil(K/128)+1 sparse blocks
+ * per tile), which needs no device-to-host copy of the search result. */
+hinm_status hinm_compress_size(const int32_t* counts_host, int M, int K, int T,
+                               hinm_layout_sizes* out_host);
+hinm_status hinm_compress_workspace_size(int M, int K, int T, size_t* bytes_host);
+/* W: bf16 [M][K]; bitmask/region: from hinm_mask; counts: device int32 [M/T][3].
+ * `layout` (host struct) holds caller-allocated device buffers of the sizes above.
+ * A 2:4 group whose row does not have exactly 2 kept bits sets HINM_ERR_BAD_MASK in the
+ * device status word (that group is then packed from its first two kept bits). */
+hinm_status hinm_compress(const void* W, const uint32_t* bitmask, const int8_t* region,
+                          const int32_t* perm, const int32_t* counts, int M, int K, int T,
+                          const hinm_layout* layout, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * a6. SpMM  ([P1] 关键设计 4: Y = dense part + 2:4 part, one output)
+ *   Y[t*T + r, n] = sum over dense vectors v of Wd[r, v] * X[idx_d(v), n]
+ *                 + sum over 2:4 groups of the 2 kept values times their gathered X rows,
+ * accumulated in fp32 on the tensor cores (dense and sparse MMA into one accumulator).
+ * X: bf16 [K][N]; Y_out: fp32 [M][N] (written in full).
+ * -------------------------------------------------------------------------------- */
+hinm_status hinm_spmm(const hinm_layout* layout, const void* X, int N, float* Y_out,
+                      void* stream);
+
+/* Reads the device status word into *status_host (0 = no fault; else an hinm_status)
+ * and clears it.  Synchronises `stream`. */
+hinm_status hinm_device_status(void* stream, int32_t* status_host);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HINM_H_ */

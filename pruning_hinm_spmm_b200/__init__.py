@@ -1,0 +1,317 @@
+"""Python binding of the HiNM C ABI (``include/hinm.h``, ``libhinm.so``).
+
+The binding only marshals arguments: it allocates device buffers with PyTorch, passes
+their raw pointers and the current CUDA stream to the C entry points of the same names,
+and turns error statuses into exceptions.  Every step of the path runs in the library's
+CUDA kernels; there is no CPU fallback.  If ``libhinm.so`` has not been built, importing
+this package raises ImportError.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional, Tuple
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libhinm.so")
+
+HINM_OK = 0
+HINM_ERR_INVALID_ARG = 1
+HINM_ERR_SHAPE = 2
+HINM_ERR_ALIGNMENT = 3
+HINM_ERR_UNSUPPORTED = 4
+HINM_ERR_CUDA = 5
+HINM_ERR_DEVICE_TIMEOUT = 6
+HINM_ERR_BAD_MASK = 7
+HINM_ERR_WORKSPACE = 8
+HINM_LAYOUT_VERSION = 1
+
+REGION_PRUNED, REGION_24, REGION_DENSE = 0, 1, 2
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m pruning_hinm_spmm_b200.build_lib` "
+        "(the HiNM path has no CPU fallback)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_vp, _i32, _f64, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_size_t
+_szp = ctypes.POINTER(ctypes.c_size_t)
+
+
+class hinm_layout(ctypes.Structure):
+    _fields_ = [("layout_version", ctypes.c_int32), ("M", ctypes.c_int32), ("K", ctypes.c_int32),
+                ("T", ctypes.c_int32), ("num_tiles", ctypes.c_int32),
+                ("max_dense_blocks", ctypes.c_int32), ("max_sparse_blocks", ctypes.c_int32),
+                ("tile_info", _vp), ("vals_dense", _vp), ("vals_sparse", _vp), ("meta", _vp),
+                ("idx_dense", _vp), ("idx_sparse", _vp)]
+
+
+class hinm_layout_sizes(ctypes.Structure):
+    _fields_ = [("max_dense_blocks", ctypes.c_int32), ("max_sparse_blocks", ctypes.c_int32),
+                ("tile_info_bytes", _sz), ("vals_dense_bytes", _sz), ("vals_sparse_bytes", _sz),
+                ("meta_bytes", _sz), ("idx_dense_bytes", _sz), ("idx_sparse_bytes", _sz)]
+
+
+_SIGS = {
+    "hinm_status_string": (ctypes.c_char_p, [_i32]),
+    "hinm_last_error": (ctypes.c_char_p, []),
+    "hinm_abi_version": (_i32, []),
+    "hinm_importance_workspace_size": (_i32, [_i32, _i32, _i32, _szp]),
+    "hinm_importance": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _sz, _vp]),
+    "hinm_counts_from_vs": (_i32, [_i32, _f64, _f64, ctypes.POINTER(ctypes.c_int32)]),
+    "hinm_search_workspace_size": (_i32, [_i32, _i32, _i32, _f64, _f64, _szp]),
+    "hinm_boundary_search": (_i32, [_vp, _vp, _i32, _i32, _i32, _f64, _f64, _vp, _vp, _vp, _vp,
+                                    _sz, _vp]),
+    "hinm_mask_workspace_size": (_i32, [_i32, _i32, _i32, _szp]),
+    "hinm_mask": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "hinm_compress_size": (_i32, [_vp, _i32, _i32, _i32, ctypes.POINTER(hinm_layout_sizes)]),
+    "hinm_compress_workspace_size": (_i32, [_i32, _i32, _i32, _szp]),
+    "hinm_compress": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
+                             ctypes.POINTER(hinm_layout), _vp, _sz, _vp]),
+    "hinm_spmm": (_i32, [ctypes.POINTER(hinm_layout), _vp, _i32, _vp, _vp]),
+    "hinm_device_status": (_i32, [_vp, ctypes.POINTER(ctypes.c_int32)]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+class HinmError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.hinm_last_error().decode(errors="replace")
+        name = _lib.hinm_status_string(status).decode()
+        super().__init__(f"{where}: {name}: {msg}")
+
+
+def _check(status: int, where: str) -> None:
+    if status != HINM_OK:
+        raise HinmError(status, where)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream(stream=None) -> int:
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else int(t.data_ptr())
+
+
+def _size(fn, *args) -> int:
+    out = ctypes.c_size_t(0)
+    _check(fn(*args, ctypes.byref(out)), fn.__name__)
+    return int(out.value)
+
+
+def _empty_bytes(nbytes: int, device):
+    torch = _torch()
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+# ----------------------------------------------------------------------------- a1
+def hinm_importance(W, X, I_out=None, workspace=None, stream=None):
+    """I = fl32(fl32(w^2) * s_c), s_c = sum_n x_cn^2 (fp64, ascending).  W [M,K], X [K,N] bf16."""
+    torch = _torch()
+    M, K = W.shape
+    N = X.shape[1]
+    if I_out is None:
+        I_out = torch.empty((M, K), dtype=torch.float32, device=W.device)
+    if workspace is None:
+        workspace = _empty_bytes(_size(_lib.hinm_importance_workspace_size, M, K, N), W.device)
+    _check(_lib.hinm_importance(_ptr(W), _ptr(X), M, K, N, _ptr(I_out), _ptr(workspace),
+                                workspace.numel(), _stream(stream)), "hinm_importance")
+    return I_out
+
+
+# ----------------------------------------------------------------------------- counts
+def hinm_counts_from_vs(K: int, t_s: float, v_s: float) -> Tuple[int, int, int]:
+    out = (ctypes.c_int32 * 3)()
+    _check(_lib.hinm_counts_from_vs(K, t_s, v_s, out), "hinm_counts_from_vs")
+    return int(out[0]), int(out[1]), int(out[2])
+
+
+# ----------------------------------------------------------------------------- a2/a3
+def hinm_search_workspace_size(M, K, T, t_s, alpha) -> int:
+    return _size(_lib.hinm_search_workspace_size, M, K, T, t_s, alpha)
+
+
+def hinm_boundary_search(I, perm, T: int, t_s: float, alpha: float = 1.0 / 32.0,
+                         counts_out=None, vs_out=None, rank_out=None, workspace=None,
+                         want_rank: bool = True, stream=None):
+    """Per-tile first-drop scan of v_s.  Returns (counts int32 [M/T,3], v_s fp64 [M/T], rank)."""
+    torch = _torch()
+    M, K = I.shape
+    nt = M // T
+    dev = I.device
+    if counts_out is None:
+        counts_out = torch.empty((nt, 3), dtype=torch.int32, device=dev)
+    if vs_out is None:
+        vs_out = torch.empty((nt,), dtype=torch.float64, device=dev)
+    if rank_out is None and want_rank:
+        rank_out = torch.empty((nt, K), dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = _empty_bytes(hinm_search_workspace_size(M, K, T, t_s, alpha), dev)
+    _check(_lib.hinm_boundary_search(_ptr(I), _ptr(perm), M, K, T, t_s, alpha, _ptr(counts_out),
+                                     _ptr(vs_out), _ptr(rank_out), _ptr(workspace),
+                                     workspace.numel(), _stream(stream)), "hinm_boundary_search")
+    return counts_out, vs_out, rank_out
+
+
+# ----------------------------------------------------------------------------- a4
+def hinm_mask_workspace_size(M, K, T) -> int:
+    return _size(_lib.hinm_mask_workspace_size, M, K, T)
+
+
+def hinm_mask(I, perm, counts, T: int, rank=None, bitmask_out=None, region_out=None,
+              workspace=None, stream=None):
+    """Bit-packed mask uint32 [M, ceil(K/32)] (as int32) and region int8 [M/T, K]."""
+    torch = _torch()
+    M, K = I.shape
+    dev = I.device
+    words = (K + 31) // 32
+    if bitmask_out is None:
+        bitmask_out = torch.empty((M, words), dtype=torch.int32, device=dev)
+    if region_out is None:
+        region_out = torch.empty((M // T, K), dtype=torch.int8, device=dev)
+    if workspace is None:
+        workspace = _empty_bytes(hinm_mask_workspace_size(M, K, T), dev)
+    _check(_lib.hinm_mask(_ptr(I), _ptr(perm), _ptr(counts), _ptr(rank), M, K, T,
+                          _ptr(bitmask_out), _ptr(region_out), _ptr(workspace), workspace.numel(),
+                          _stream(stream)), "hinm_mask")
+    return bitmask_out, region_out
+
+
+# ----------------------------------------------------------------------------- a5
+def hinm_compress_size(M: int, K: int, T: int, counts_host=None) -> hinm_layout_sizes:
+    out = hinm_layout_sizes()
+    arg = None
+    if counts_host is not None:
+        import numpy as np
+        arr = np.ascontiguousarray(counts_host, dtype=np.int32)
+        arg = arr.ctypes.data
+    _check(_lib.hinm_compress_size(arg, M, K, T, ctypes.byref(out)), "hinm_compress_size")
+    return out
+
+
+@dataclass
+class HinmLayout:
+    """Device buffers of one compressed HiNM weight (caller-owned torch tensors)."""
+    M: int
+    K: int
+    T: int
+    max_dense_blocks: int
+    max_sparse_blocks: int
+    tile_info: object    # int32 [M/T, 4]
+    vals_dense: object   # int16 (bf16 bits) [blocks, 8192]
+    vals_sparse: object  # int16 [blocks, 8192]
+    meta: object         # int32 [blocks, 512]
+    idx_dense: object    # int32 [blocks, 64]
+    idx_sparse: object   # int32 [blocks, 128]
+
+    @classmethod
+    def allocate(cls, M: int, K: int, T: int, device, counts_host=None) -> "HinmLayout":
+        torch = _torch()
+        sz = hinm_compress_size(M, K, T, counts_host)
+        nd, ns = sz.max_dense_blocks, sz.max_sparse_blocks
+        return cls(M=M, K=K, T=T, max_dense_blocks=nd, max_sparse_blocks=ns,
+                   tile_info=torch.zeros((M // T, 4), dtype=torch.int32, device=device),
+                   vals_dense=torch.empty((nd, 8192), dtype=torch.int16, device=device),
+                   vals_sparse=torch.empty((ns, 8192), dtype=torch.int16, device=device),
+                   meta=torch.empty((ns, 512), dtype=torch.int32, device=device),
+                   idx_dense=torch.empty((nd, 64), dtype=torch.int32, device=device),
+                   idx_sparse=torch.empty((ns, 128), dtype=torch.int32, device=device))
+
+    def as_c(self) -> hinm_layout:
+        return hinm_layout(HINM_LAYOUT_VERSION, self.M, self.K, self.T, self.M // self.T,
+                           self.max_dense_blocks, self.max_sparse_blocks,
+                           _ptr(self.tile_info), _ptr(self.vals_dense), _ptr(self.vals_sparse),
+                           _ptr(self.meta), _ptr(self.idx_dense), _ptr(self.idx_sparse))
+
+
+def hinm_compress_workspace_size(M, K, T) -> int:
+    return _size(_lib.hinm_compress_workspace_size, M, K, T)
+
+
+def hinm_compress(W, bitmask, region, perm, counts, T: int, layout: Optional[HinmLayout] = None,
+                  workspace=None, stream=None) -> HinmLayout:
+    M, K = W.shape
+    if layout is None:
+        layout = HinmLayout.allocate(M, K, T, W.device)
+    if workspace is None:
+        workspace = _empty_bytes(hinm_compress_workspace_size(M, K, T), W.device)
+    c = layout.as_c()
+    _check(_lib.hinm_compress(_ptr(W), _ptr(bitmask), _ptr(region), _ptr(perm), _ptr(counts),
+                              M, K, T, ctypes.byref(c), _ptr(workspace), workspace.numel(),
+                              _stream(stream)), "hinm_compress")
+    return layout
+
+
+# ----------------------------------------------------------------------------- a6
+def hinm_spmm(layout: HinmLayout, X, Y_out=None, stream=None, c_layout: Optional[hinm_layout] = None):
+    """Y (fp32 [M, N]) = W_HiNM . X (X bf16 [K, N])."""
+    torch = _torch()
+    N = X.shape[1]
+    if Y_out is None:
+        Y_out = torch.empty((layout.M, N), dtype=torch.float32, device=X.device)
+    c = c_layout if c_layout is not None else layout.as_c()
+    _check(_lib.hinm_spmm(ctypes.byref(c), _ptr(X), N, _ptr(Y_out), _stream(stream)), "hinm_spmm")
+    return Y_out
+
+
+def hinm_device_status(stream=None) -> int:
+    out = ctypes.c_int32(0)
+    _check(_lib.hinm_device_status(_stream(stream), ctypes.byref(out)), "hinm_device_status")
+    return int(out.value)
+
+
+# ----------------------------------------------------------------------------- whole path
+class HotPath:
+    """Preallocated buffers for importance -> search -> mask -> compress -> spmm on one
+    problem shape; run() enqueues the five steps on the current stream with no host sync."""
+
+    def __init__(self, M: int, K: int, N: int, T: int, t_s: float, alpha: float = 1.0 / 32.0,
+                 device="cuda"):
+        torch = _torch()
+        self.M, self.K, self.N, self.T, self.t_s, self.alpha = M, K, N, T, t_s, alpha
+        nt = M // T
+        self.I = torch.empty((M, K), dtype=torch.float32, device=device)
+        self.counts = torch.empty((nt, 3), dtype=torch.int32, device=device)
+        self.vs = torch.empty((nt,), dtype=torch.float64, device=device)
+        self.rank = torch.empty((nt, K), dtype=torch.int32, device=device)
+        self.bitmask = torch.empty((M, (K + 31) // 32), dtype=torch.int32, device=device)
+        self.region = torch.empty((nt, K), dtype=torch.int8, device=device)
+        self.layout = HinmLayout.allocate(M, K, T, device)
+        self.c_layout = self.layout.as_c()
+        self.Y = torch.empty((M, N), dtype=torch.float32, device=device)
+        ws = max(_size(_lib.hinm_importance_workspace_size, M, K, N),
+                 hinm_search_workspace_size(M, K, T, t_s, alpha),
+                 hinm_mask_workspace_size(M, K, T), hinm_compress_workspace_size(M, K, T))
+        self.ws = _empty_bytes(ws, device)
+
+    def run(self, W, X, perm, fixed_counts=None, stream=None):
+        hinm_importance(W, X, self.I, self.ws, stream)
+        if fixed_counts is None:
+            hinm_boundary_search(self.I, perm, self.T, self.t_s, self.alpha, self.counts, self.vs,
+                                 self.rank, self.ws, stream=stream)
+            counts, rank = self.counts, self.rank
+        else:
+            counts, rank = fixed_counts, None
+        hinm_mask(self.I, perm, counts, self.T, rank, self.bitmask, self.region, self.ws, stream)
+        hinm_compress(W, self.bitmask, self.region, perm, counts, self.T, self.layout, self.ws,
+                      stream)
+        hinm_spmm(self.layout, X, self.Y, stream, self.c_layout)
+        return self.Y

@@ -1,0 +1,400 @@
+// C ABI of the HiNM hot path: argument checks, workspace sizing and dispatch to the
+// kernels.  Every entry point returns an hinm_status and never throws.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/hinm.h"
+#include "hinm_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+hinm_status fail(hinm_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+hinm_status ok() {
+  g_last_error.clear();
+  return HINM_OK;
+}
+
+hinm_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(HINM_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define REQUIRE_PTR(p)                                                            \
+  do {                                                                            \
+    if ((p) == nullptr) return fail(HINM_ERR_INVALID_ARG, "%s is NULL", #p);      \
+    if (!aligned16(p)) return fail(HINM_ERR_ALIGNMENT, "%s is not 16-byte aligned", #p); \
+  } while (0)
+
+#define REQUIRE_ALIGNED_OR_NULL(p)                                                \
+  do {                                                                            \
+    if ((p) != nullptr && !aligned16(p))                                          \
+      return fail(HINM_ERR_ALIGNMENT, "%s is not 16-byte aligned", #p);           \
+  } while (0)
+
+hinm_status check_mkt(int M, int K, int T) {
+  if (T != 64 && T != 128) return fail(HINM_ERR_SHAPE, "T=%d: tile height must be 64 or 128", T);
+  if (M <= 0 || M % T != 0) return fail(HINM_ERR_SHAPE, "M=%d must be a positive multiple of T=%d", M, T);
+  if (K < 4 || K > hinm::kMaxK || K % 4 != 0)
+    return fail(HINM_ERR_SHAPE, "K=%d must be a multiple of 4 in [4, %d]", K, hinm::kMaxK);
+  if ((long long)M * (long long)K >= (1ll << 31))
+    return fail(HINM_ERR_SHAPE, "M*K=%lld exceeds 2^31 elements", (long long)M * K);
+  if (M / T > 65535) return fail(HINM_ERR_SHAPE, "M/T=%d tiles exceeds 65535", M / T);
+  return HINM_OK;
+}
+
+hinm_status check_n(int N) {
+  if (N <= 0 || N % 8 != 0) return fail(HINM_ERR_SHAPE, "N=%d must be a positive multiple of 8", N);
+  if (N > (1 << 24)) return fail(HINM_ERR_SHAPE, "N=%d too large", N);
+  return HINM_OK;
+}
+
+hinm_status check_search_params(double t_s, double alpha) {
+  if (!std::isfinite(t_s) || t_s < 0.0 || t_s > 1.0)
+    return fail(HINM_ERR_INVALID_ARG, "t_s=%g must be in [0, 1]", t_s);
+  if (!std::isfinite(alpha) || alpha <= 0.0)
+    return fail(HINM_ERR_INVALID_ARG, "alpha=%g must be a positive finite step", alpha);
+  return HINM_OK;
+}
+
+// One status word per device, resolved with cudaGetSymbolAddress on first use.
+__device__ int g_device_status;
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices];
+std::mutex g_status_mu;
+
+}  // namespace
+
+namespace hinm {
+
+// Closed form of the three region counts (see hinm.h).  Evaluated left to right in
+// double precision with no fused multiply-add (the host build uses -ffp-contract=off).
+bool counts_from_vs_host(int K, double t_s, double v_s, int out[3]) {
+  const double x = 2.0 * (t_s - v_s) * K / 4.0;
+  const double fl = std::floor(x + 0.5);
+  if (!std::isfinite(fl)) return false;
+  const long long n24 = 4ll * (long long)fl;
+  const double tk = t_s * K;
+  if (tk != std::floor(tk)) return false;
+  const long long n0 = (long long)tk - n24 / 2;
+  const long long n4 = (long long)K - n0 - n24;
+  if (n24 < 0 || n0 < 0 || n4 < 0) return false;
+  out[0] = (int)n0;
+  out[1] = (int)n24;
+  out[2] = (int)n4;
+  return true;
+}
+
+int search_candidates_host(int K, double t_s, double alpha, Candidate* out, int cap) {
+  const double lower = std::fmax(0.0, 2.0 * t_s - 1.0);
+  const double mm = std::floor((t_s - lower) / alpha);
+  const long long m_max = (long long)mm;
+  int n = 0;
+  for (long long m = 0; m <= m_max && n < cap; ++m) {
+    const double v_s = t_s - (double)m * alpha;
+    int c[3];
+    if (!counts_from_vs_host(K, t_s, v_s, c)) {
+      if (m == 0) return -1;
+      break;
+    }
+    out[n++] = Candidate{c[0], c[1], c[2]};
+  }
+  return n;
+}
+
+int* device_status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_status_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+}  // namespace hinm
+
+// =====================================================================================
+extern "C" {
+
+const char* hinm_status_string(int st) {
+  switch (st) {
+    case HINM_OK: return "HINM_OK";
+    case HINM_ERR_INVALID_ARG: return "HINM_ERR_INVALID_ARG";
+    case HINM_ERR_SHAPE: return "HINM_ERR_SHAPE";
+    case HINM_ERR_ALIGNMENT: return "HINM_ERR_ALIGNMENT";
+    case HINM_ERR_UNSUPPORTED: return "HINM_ERR_UNSUPPORTED";
+    case HINM_ERR_CUDA: return "HINM_ERR_CUDA";
+    case HINM_ERR_DEVICE_TIMEOUT: return "HINM_ERR_DEVICE_TIMEOUT";
+    case HINM_ERR_BAD_MASK: return "HINM_ERR_BAD_MASK";
+    case HINM_ERR_WORKSPACE: return "HINM_ERR_WORKSPACE";
+    default: return "HINM_ERR_UNKNOWN";
+  }
+}
+
+const char* hinm_last_error(void) { return g_last_error.c_str(); }
+
+int hinm_abi_version(void) { return HINM_ABI_VERSION; }
+
+hinm_status hinm_counts_from_vs(int K, double t_s, double v_s, int32_t* out_host) {
+  if (!out_host) return fail(HINM_ERR_INVALID_ARG, "out_host is NULL");
+  if (K <= 0) return fail(HINM_ERR_SHAPE, "K=%d must be positive", K);
+  if (!std::isfinite(t_s) || !std::isfinite(v_s) || t_s < 0 || t_s > 1 || v_s < 0 || v_s > 1)
+    return fail(HINM_ERR_INVALID_ARG, "t_s=%g, v_s=%g must be finite and in [0, 1]", t_s, v_s);
+  int c[3];
+  if (!hinm::counts_from_vs_host(K, t_s, v_s, c))
+    return fail(HINM_ERR_INVALID_ARG,
+                "boundary (t_s=%g, v_s=%g) gives no valid counts for K=%d (t_s*K must be whole, "
+                "v_s >= 2 t_s - 1)", t_s, v_s, K);
+  out_host[0] = c[0];
+  out_host[1] = c[1];
+  out_host[2] = c[2];
+  return ok();
+}
+
+hinm_status hinm_importance_workspace_size(int M, int K, int N, size_t* bytes_host) {
+  if (!bytes_host) return fail(HINM_ERR_INVALID_ARG, "bytes_host is NULL");
+  if (M <= 0 || K <= 0 || N <= 0) return fail(HINM_ERR_SHAPE, "sizes must be positive");
+  *bytes_host = hinm::importance_workspace_bytes(K);
+  return ok();
+}
+
+hinm_status hinm_importance(const void* W, const void* X, int M, int K, int N, float* I_out,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  REQUIRE_PTR(W);
+  REQUIRE_PTR(X);
+  REQUIRE_PTR(I_out);
+  if (M <= 0 || K <= 0 || K % 4 != 0 || (long long)M * K >= (1ll << 31))
+    return fail(HINM_ERR_SHAPE, "M=%d, K=%d: need M > 0 and K a positive multiple of 4", M, K);
+  hinm_status st = check_n(N);
+  if (st != HINM_OK) return st;
+  const size_t need = hinm::importance_workspace_bytes(K);
+  if (!workspace || workspace_bytes < need)
+    return fail(HINM_ERR_WORKSPACE, "workspace %zu bytes, need %zu", workspace_bytes, need);
+  REQUIRE_PTR(workspace);
+  cudaError_t e = hinm::launch_importance(static_cast<const uint16_t*>(W),
+                                          static_cast<const uint16_t*>(X), M, K, N, I_out,
+                                          static_cast<float*>(workspace),
+                                          static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "hinm_importance launch");
+  return ok();
+}
+
+hinm_status hinm_search_workspace_size(int M, int K, int T, double t_s, double alpha,
+                                       size_t* bytes_host) {
+  if (!bytes_host) return fail(HINM_ERR_INVALID_ARG, "bytes_host is NULL");
+  hinm_status st = check_mkt(M, K, T);
+  if (st != HINM_OK) return st;
+  st = check_search_params(t_s, alpha);
+  if (st != HINM_OK) return st;
+  hinm::Candidate c[hinm::kMaxCandidates];
+  const int n = hinm::search_candidates_host(K, t_s, alpha, c, hinm::kMaxCandidates);
+  if (n < 0) return fail(HINM_ERR_INVALID_ARG, "t_s*K = %g is not a whole number", t_s * K);
+  *bytes_host = hinm::search_workspace_bytes(M, K, T, n);
+  return ok();
+}
+
+hinm_status hinm_boundary_search(const float* I, const int32_t* perm, int M, int K, int T,
+                                 double t_s, double alpha, int32_t* counts_out, double* vs_out,
+                                 int32_t* rank_out, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+  REQUIRE_PTR(I);
+  REQUIRE_ALIGNED_OR_NULL(perm);
+  REQUIRE_PTR(counts_out);
+  REQUIRE_PTR(vs_out);
+  REQUIRE_ALIGNED_OR_NULL(rank_out);
+  hinm_status st = check_mkt(M, K, T);
+  if (st != HINM_OK) return st;
+  st = check_search_params(t_s, alpha);
+  if (st != HINM_OK) return st;
+  hinm::Candidate c[hinm::kMaxCandidates];
+  const int n = hinm::search_candidates_host(K, t_s, alpha, c, hinm::kMaxCandidates);
+  if (n < 0) return fail(HINM_ERR_INVALID_ARG, "t_s*K = %g is not a whole number", t_s * K);
+  const double lower = std::fmax(0.0, 2.0 * t_s - 1.0);
+  if (std::floor((t_s - lower) / alpha) + 1 > hinm::kMaxCandidates && n == hinm::kMaxCandidates)
+    return fail(HINM_ERR_UNSUPPORTED, "alpha=%g gives more than %d candidates", alpha,
+                hinm::kMaxCandidates);
+  const size_t need = hinm::search_workspace_bytes(M, K, T, n);
+  if (!workspace || workspace_bytes < need)
+    return fail(HINM_ERR_WORKSPACE, "workspace %zu bytes, need %zu", workspace_bytes, need);
+  REQUIRE_PTR(workspace);
+  cudaError_t e = hinm::launch_boundary_search(I, perm, M, K, T, t_s, alpha, c, n, counts_out,
+                                               vs_out, rank_out, workspace,
+                                               hinm::device_status_ptr(),
+                                               static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "hinm_boundary_search launch");
+  return ok();
+}
+
+hinm_status hinm_mask_workspace_size(int M, int K, int T, size_t* bytes_host) {
+  if (!bytes_host) return fail(HINM_ERR_INVALID_ARG, "bytes_host is NULL");
+  hinm_status st = check_mkt(M, K, T);
+  if (st != HINM_OK) return st;
+  *bytes_host = hinm::mask_workspace_bytes(M, K, T);
+  return ok();
+}
+
+hinm_status hinm_mask(const float* I, const int32_t* perm, const int32_t* counts,
+                      const int32_t* rank, int M, int K, int T, uint32_t* bitmask_out,
+                      int8_t* region_out, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  REQUIRE_PTR(I);
+  REQUIRE_ALIGNED_OR_NULL(perm);
+  REQUIRE_PTR(counts);
+  REQUIRE_ALIGNED_OR_NULL(rank);
+  REQUIRE_PTR(bitmask_out);
+  REQUIRE_PTR(region_out);
+  hinm_status st = check_mkt(M, K, T);
+  if (st != HINM_OK) return st;
+  const size_t need = hinm::mask_workspace_bytes(M, K, T);
+  if (!workspace || workspace_bytes < need)
+    return fail(HINM_ERR_WORKSPACE, "workspace %zu bytes, need %zu", workspace_bytes, need);
+  REQUIRE_PTR(workspace);
+  cudaError_t e = hinm::launch_mask(I, perm, counts, rank, M, K, T, bitmask_out, region_out,
+                                    workspace, hinm::device_status_ptr(),
+                                    static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "hinm_mask launch");
+  return ok();
+}
+
+hinm_status hinm_compress_size(const int32_t* counts_host, int M, int K, int T,
+                               hinm_layout_sizes* out_host) {
+  if (!out_host) return fail(HINM_ERR_INVALID_ARG, "out_host is NULL");
+  hinm_status st = check_mkt(M, K, T);
+  if (st != HINM_OK) return st;
+  const int nt = M / T;
+  long long nd = 0, ns = 0;
+  if (counts_host) {
+    for (int t = 0; t < nt; ++t) {
+      const int n0 = counts_host[3 * t], n24 = counts_host[3 * t + 1], n4 = counts_host[3 * t + 2];
+      if (n0 < 0 || n24 < 0 || n4 < 0 || n0 + n24 + n4 != K || n24 % 4 != 0)
+        return fail(HINM_ERR_INVALID_ARG, "tile %d: counts (%d, %d, %d) invalid for K=%d", t, n0,
+                    n24, n4, K);
+      nd += (n4 + hinm::kDenseBK - 1) / hinm::kDenseBK;
+      ns += (n24 + hinm::kSparseBK - 1) / hinm::kSparseBK;
+    }
+  } else {
+    nd = (long long)nt * ((K + hinm::kDenseBK - 1) / hinm::kDenseBK + 1);
+    ns = (long long)nt * ((K + hinm::kSparseBK - 1) / hinm::kSparseBK + 1);
+  }
+  if (nd == 0) nd = 1;  // keep every buffer non-empty so pointers can be checked
+  if (ns == 0) ns = 1;
+  out_host->max_dense_blocks = (int32_t)nd;
+  out_host->max_sparse_blocks = (int32_t)ns;
+  out_host->tile_info_bytes = (size_t)nt * 4 * sizeof(int32_t);
+  out_host->vals_dense_bytes = (size_t)nd * hinm::kBlockBytes;
+  out_host->vals_sparse_bytes = (size_t)ns * hinm::kBlockBytes;
+  out_host->meta_bytes = (size_t)ns * hinm::kMetaWords * sizeof(uint32_t);
+  out_host->idx_dense_bytes = (size_t)nd * hinm::kDenseBK * sizeof(int32_t);
+  out_host->idx_sparse_bytes = (size_t)ns * hinm::kSparseBK * sizeof(int32_t);
+  return ok();
+}
+
+hinm_status hinm_compress_workspace_size(int M, int K, int T, size_t* bytes_host) {
+  if (!bytes_host) return fail(HINM_ERR_INVALID_ARG, "bytes_host is NULL");
+  hinm_status st = check_mkt(M, K, T);
+  if (st != HINM_OK) return st;
+  *bytes_host = hinm::compress_workspace_bytes(M, K, T);
+  return ok();
+}
+
+static hinm_status check_layout(const hinm_layout* L) {
+  if (!L) return fail(HINM_ERR_INVALID_ARG, "layout is NULL");
+  if (L->layout_version != HINM_LAYOUT_VERSION)
+    return fail(HINM_ERR_INVALID_ARG, "layout_version %d, expected %d", L->layout_version,
+                HINM_LAYOUT_VERSION);
+  hinm_status st = check_mkt(L->M, L->K, L->T);
+  if (st != HINM_OK) return st;
+  if (L->num_tiles != L->M / L->T)
+    return fail(HINM_ERR_SHAPE, "num_tiles=%d != M/T=%d", L->num_tiles, L->M / L->T);
+  if (L->max_dense_blocks < 1 || L->max_sparse_blocks < 1)
+    return fail(HINM_ERR_SHAPE, "layout capacities must be >= 1 block");
+  REQUIRE_PTR(L->tile_info);
+  REQUIRE_PTR(L->vals_dense);
+  REQUIRE_PTR(L->vals_sparse);
+  REQUIRE_PTR(L->meta);
+  REQUIRE_PTR(L->idx_dense);
+  REQUIRE_PTR(L->idx_sparse);
+  return HINM_OK;
+}
+
+hinm_status hinm_compress(const void* W, const uint32_t* bitmask, const int8_t* region,
+                          const int32_t* perm, const int32_t* counts, int M, int K, int T,
+                          const hinm_layout* layout, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  REQUIRE_PTR(W);
+  REQUIRE_PTR(bitmask);
+  REQUIRE_PTR(region);
+  REQUIRE_ALIGNED_OR_NULL(perm);
+  REQUIRE_PTR(counts);
+  hinm_status st = check_mkt(M, K, T);
+  if (st != HINM_OK) return st;
+  st = check_layout(layout);
+  if (st != HINM_OK) return st;
+  if (layout->M != M || layout->K != K || layout->T != T)
+    return fail(HINM_ERR_SHAPE, "layout is %dx%d T=%d, call is %dx%d T=%d", layout->M, layout->K,
+                layout->T, M, K, T);
+  const size_t need = hinm::compress_workspace_bytes(M, K, T);
+  if (!workspace || workspace_bytes < need)
+    return fail(HINM_ERR_WORKSPACE, "workspace %zu bytes, need %zu", workspace_bytes, need);
+  REQUIRE_PTR(workspace);
+  cudaError_t e = hinm::launch_compress(static_cast<const uint16_t*>(W), bitmask, region, perm,
+                                        counts, M, K, T, *layout, workspace,
+                                        hinm::device_status_ptr(),
+                                        static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "hinm_compress launch");
+  return ok();
+}
+
+hinm_status hinm_spmm(const hinm_layout* layout, const void* X, int N, float* Y_out,
+                      void* stream) {
+  hinm_status st = check_layout(layout);
+  if (st != HINM_OK) return st;
+  REQUIRE_PTR(X);
+  REQUIRE_PTR(Y_out);
+  st = check_n(N);
+  if (st != HINM_OK) return st;
+  cudaError_t e = hinm::launch_spmm(*layout, static_cast<const uint16_t*>(X), N, Y_out,
+                                    hinm::device_status_ptr(), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "hinm_spmm launch");
+  return ok();
+}
+
+hinm_status hinm_device_status(void* stream, int32_t* status_host) {
+  if (!status_host) return fail(HINM_ERR_INVALID_ARG, "status_host is NULL");
+  int* p = hinm::device_status_ptr();
+  if (!p) return fail(HINM_ERR_CUDA, "cannot resolve the device status word");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, p, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess && v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyAsync(p, &zero, sizeof(int), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "hinm_device_status");
+  *status_host = v;
+  return ok();
+}
+
+}  // extern "C"

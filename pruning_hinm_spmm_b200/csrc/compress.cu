@@ -1,0 +1,237 @@
+// a5. Compress W ⊙ M into the HiNM layout (FlexHiNM-GP notes, 关键设计 2/4: dense part and
+// 2:4 part stored apart, the 2:4 part gathered by a precomputed index with the input
+// permutation folded in; geek-doc.cn section 三: 2 values per group plus 2-bit positions).
+//
+//   tile_info_kernel   per tile: dense blocks ceil(n4/64), sparse blocks ceil(n24/128),
+//                      prefix offsets; checks counts and buffer capacity
+//   lists_kernel       per tile: dense and 2:4 working positions in ascending order
+//   pack_kernel        one CTA per (block, tile): writes one 16 KB value block exactly as
+//                      the tensor cores read it from shared memory (128-byte swizzle),
+//                      the 2 KB metadata block in tensor-memory lane order, and the index.
+#include <cuda_runtime.h>
+
+#include "hinm_internal.h"
+#include "ptx.cuh"
+
+namespace hinm {
+
+__global__ void tile_info_kernel(const int32_t* __restrict__ counts, int nt, int K,
+                                 int max_dense, int max_sparse, int32_t* __restrict__ info,
+                                 int* status) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  int d0 = 0, s0 = 0;
+  for (int t = 0; t < nt; ++t) {
+    const int n0 = counts[3 * t], n24 = counts[3 * t + 1], n4 = counts[3 * t + 2];
+    int nd = 0, ns = 0;
+    if (n0 < 0 || n24 < 0 || n4 < 0 || n0 + n24 + n4 != K || (n24 & 3)) {
+      ptx::record_status(status, HINM_ERR_INVALID_ARG);
+    } else {
+      nd = (n4 + kDenseBK - 1) / kDenseBK;
+      ns = (n24 + kSparseBK - 1) / kSparseBK;
+    }
+    if (d0 + nd > max_dense || s0 + ns > max_sparse) {
+      ptx::record_status(status, HINM_ERR_WORKSPACE);
+      nd = ns = 0;
+    }
+    info[4 * t + 0] = nd;
+    info[4 * t + 1] = ns;
+    info[4 * t + 2] = d0;
+    info[4 * t + 3] = s0;
+    d0 += nd;
+    s0 += ns;
+  }
+}
+
+// lists[t][0 .. n_dense) = dense working positions, lists[t][n_dense .. ) = 2:4 ones.
+__global__ void __launch_bounds__(1024) lists_kernel(const int8_t* __restrict__ region,
+                                                     const int32_t* __restrict__ perm,
+                                                     const int32_t* __restrict__ counts, int K,
+                                                     int32_t* __restrict__ lists, int* status) {
+  __shared__ int warp_tot[2][32];
+  const int t = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int8_t* reg = region + (size_t)t * K;
+  const int per = (K + blockDim.x - 1) / blockDim.x;
+  const int j0 = threadIdx.x * per, j1 = min(K, j0 + per);
+  int cd = 0, cs = 0;
+  for (int j = j0; j < j1; ++j) {
+    const int8_t r = reg[ptx::perm_at(perm, j, K)];
+    cd += (r == HINM_REGION_DENSE);
+    cs += (r == HINM_REGION_24);
+  }
+  int id = cd, is = cs;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int a = __shfl_up_sync(0xffffffffu, id, o), b = __shfl_up_sync(0xffffffffu, is, o);
+    if (lane >= o) {
+      id += a;
+      is += b;
+    }
+  }
+  if (lane == 31) {
+    warp_tot[0][warp] = id;
+    warp_tot[1][warp] = is;
+  }
+  __syncthreads();
+  int bd = 0, bs = 0, td = 0, ts = 0;
+  for (int w = 0; w < nw; ++w) {
+    if (w < warp) {
+      bd += warp_tot[0][w];
+      bs += warp_tot[1][w];
+    }
+    td += warp_tot[0][w];
+    ts += warp_tot[1][w];
+  }
+  const int n4 = counts[3 * t + 2], n24 = counts[3 * t + 1];
+  if (threadIdx.x == 0 && (td != n4 || ts != n24)) ptx::record_status(status, HINM_ERR_INVALID_ARG);
+  int pd = bd + id - cd, ps = td + bs + is - cs;
+  int32_t* L = lists + (size_t)t * K;
+  for (int j = j0; j < j1; ++j) {
+    const int8_t r = reg[ptx::perm_at(perm, j, K)];
+    if (r == HINM_REGION_DENSE) L[pd++] = j;
+    else if (r == HINM_REGION_24) L[ps++] = j;
+  }
+}
+
+__device__ __forceinline__ int swz(int r, int k) {  // byte offset of bf16 (r, k) in a block
+  return r * 128 + ((((k >> 3) ^ (r & 7))) << 4) + (k & 7) * 2;
+}
+
+// Working position stored in a list entry, clamped into [0, K) so that inconsistent
+// region / counts arguments (reported in the status word) never index out of bounds.
+__device__ __forceinline__ int list_at(const int32_t* lst, int p, int K) {
+  const int j = lst[p];
+  return (unsigned)j < (unsigned)K ? j : 0;
+}
+
+__device__ __forceinline__ bool mask_bit(const uint32_t* bm, int words, int i, int c) {
+  return (__ldg(bm + (size_t)i * words + (c >> 5)) >> (c & 31)) & 1u;
+}
+
+__global__ void __launch_bounds__(256) pack_kernel(const uint16_t* __restrict__ W,
+                                                   const uint32_t* __restrict__ bitmask,
+                                                   const int32_t* __restrict__ perm,
+                                                   const int32_t* __restrict__ counts,
+                                                   const int32_t* __restrict__ lists, int K, int T,
+                                                   hinm_layout L, int* status) {
+  __shared__ uint8_t nib[128][32];
+  const int t = blockIdx.y;
+  const int b = blockIdx.x;
+  const int nd = L.tile_info[4 * t + 0], ns = L.tile_info[4 * t + 1];
+  const int d0 = L.tile_info[4 * t + 2], s0 = L.tile_info[4 * t + 3];
+  if (b >= nd + ns) return;
+  const int n4 = counts[3 * t + 2], n24 = counts[3 * t + 1];
+  const int words = (K + 31) >> 5;
+  const int32_t* lst = lists + (size_t)t * K;
+  const int row0 = t * T;
+  if (b < nd) {
+    uint8_t* out = reinterpret_cast<uint8_t*>(L.vals_dense + (size_t)(d0 + b) * 8192);
+    for (int item = threadIdx.x; item < 128 * 8; item += blockDim.x) {
+      const int r = item >> 3, ch = item & 7;
+      uint32_t h[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int p = b * kDenseBK + ch * 8 + e;
+        uint32_t v = 0;
+        if (r < T && p < n4) {
+          const int c = ptx::perm_at(perm, list_at(lst, p, K), K);
+          const int i = row0 + r;
+          if (mask_bit(bitmask, words, i, c)) v = __ldg(W + (size_t)i * K + c);
+        }
+        h[e] = v;
+      }
+      uint4 q;
+      q.x = h[0] | (h[1] << 16);
+      q.y = h[2] | (h[3] << 16);
+      q.z = h[4] | (h[5] << 16);
+      q.w = h[6] | (h[7] << 16);
+      *reinterpret_cast<uint4*>(out + r * 128 + ((ch ^ (r & 7)) << 4)) = q;
+    }
+    if (threadIdx.x < kDenseBK) {
+      const int p = b * kDenseBK + threadIdx.x;
+      L.idx_dense[(size_t)(d0 + b) * kDenseBK + threadIdx.x] =
+          p < n4 ? ptx::perm_at(perm, list_at(lst, p, K), K) : 0;
+    }
+    return;
+  }
+  const int sb = b - nd;
+  uint8_t* out = reinterpret_cast<uint8_t*>(L.vals_sparse + (size_t)(s0 + sb) * 8192);
+  for (int item = threadIdx.x; item < 128 * 32; item += blockDim.x) {
+    const int r = item >> 5, g = item & 31;
+    const int q0 = sb * kSparseBK + 4 * g;  // first 2:4 vector of the group
+    uint32_t a = 0, bb = 1, va = 0, vb = 0;
+    if (r < T && q0 < n24) {
+      const int i = row0 + r;
+      int c[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) c[k] = ptx::perm_at(perm, list_at(lst, n4 + q0 + k, K), K);
+      int kept[4], nk = 0, free_[4], nf = 0;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (mask_bit(bitmask, words, i, c[k])) kept[nk++] = k;
+        else free_[nf++] = k;
+      }
+      if (nk != 2) ptx::record_status(status, HINM_ERR_BAD_MASK);
+      int pa, pb;
+      bool use_a, use_b;
+      if (nk >= 2) {
+        pa = kept[0]; pb = kept[1]; use_a = use_b = true;
+      } else if (nk == 1) {
+        pa = kept[0]; pb = free_[0]; use_a = true; use_b = false;
+        if (pb < pa) { const int x = pa; pa = pb; pb = x; use_a = false; use_b = true; }
+      } else {
+        pa = 0; pb = 1; use_a = use_b = false;
+      }
+      a = pa;
+      bb = pb;
+      va = use_a ? __ldg(W + (size_t)i * K + c[pa]) : 0u;
+      vb = use_b ? __ldg(W + (size_t)i * K + c[pb]) : 0u;
+    }
+    *reinterpret_cast<uint32_t*>(out + swz(r, 2 * g)) = va | (vb << 16);
+    nib[r][g] = (uint8_t)(a | (bb << 2));
+  }
+  __syncthreads();
+  uint32_t* meta = L.meta + (size_t)(s0 + sb) * kMetaWords;
+  for (int wi = threadIdx.x; wi < kMetaWords; wi += blockDim.x) {
+    const int lane = wi >> 2, w = wi & 3;
+    const int h = (lane >> 3) & 1;
+    uint32_t word = 0;
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const int m = 16 * (lane >> 4) + 8 * s + (lane & 7);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) word |= uint32_t(nib[m][8 * w + 4 * h + q]) << (16 * s + 4 * q);
+    }
+    meta[wi] = word;
+  }
+  if (threadIdx.x < kSparseBK) {
+    const int p = sb * kSparseBK + threadIdx.x;
+    L.idx_sparse[(size_t)(s0 + sb) * kSparseBK + threadIdx.x] =
+        p < n24 ? ptx::perm_at(perm, list_at(lst, n4 + p, K), K) : 0;
+  }
+}
+
+size_t compress_workspace_bytes(int M, int K, int T) {
+  const int nt = M / T;
+  return (((size_t)nt * K * sizeof(int32_t)) + 255) & ~size_t(255);
+}
+
+cudaError_t launch_compress(const uint16_t* W, const uint32_t* bitmask, const int8_t* region,
+                            const int32_t* perm, const int32_t* counts, int M, int K, int T,
+                            const hinm_layout& L, void* ws, int* status, cudaStream_t s) {
+  const int nt = M / T;
+  int32_t* lists = static_cast<int32_t*>(ws);
+  tile_info_kernel<<<1, 32, 0, s>>>(counts, nt, K, L.max_dense_blocks, L.max_sparse_blocks,
+                                    L.tile_info, status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // lists are read only at positions below the counts, so no clearing is needed
+  lists_kernel<<<nt, 1024, 0, s>>>(region, perm, counts, K, lists, status);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int max_blocks = (K + kDenseBK - 1) / kDenseBK + (K + kSparseBK - 1) / kSparseBK;
+  dim3 g(max_blocks, nt);
+  pack_kernel<<<g, 256, 0, s>>>(W, bitmask, perm, counts, lists, K, T, L, status);
+  return cudaGetLastError();
+}
+
+}  // namespace hinm

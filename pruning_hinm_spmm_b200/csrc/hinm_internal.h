@@ -1,0 +1,79 @@
+// Internal interface between the C ABI (abi.cu) and the kernels of the HiNM hot path.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/hinm.h"
+
+namespace hinm {
+
+// Device status word codes (a subset of hinm_status) written by kernels.
+constexpr int kStatusOk = 0;
+
+// Geometry of the compressed layout (see hinm.h, a5).
+constexpr int kBlockRows = 128;     // rows per compressed block
+constexpr int kDenseBK = 64;        // dense vectors per dense block
+constexpr int kSparseBK = 128;      // 2:4 vectors per sparse block (32 groups)
+constexpr int kBlockBytes = 16384;  // 128 rows x 128 bytes
+constexpr int kMetaWords = 512;     // 128 lanes x 4 words
+constexpr int kMaxK = 16384;        // rank sort runs in one CTA's shared memory
+constexpr int kMaxCandidates = 64;  // boundary-search candidates per call
+
+struct Candidate {
+  int n0, n24, n4;
+};
+
+// Host-side closed form (hinm.h, counts).  Returns false on an invalid boundary.
+bool counts_from_vs_host(int K, double t_s, double v_s, int out[3]);
+// Candidate list of the boundary search; returns the number of candidates (>= 1) or
+// -1 when the start boundary itself is invalid.
+int search_candidates_host(int K, double t_s, double alpha, Candidate* out, int cap);
+
+// Per-device address of the library's status word (resolved once per device).
+int* device_status_ptr();
+
+// Workspace carving helper: 256-byte aligned sub-buffers.
+struct Carve {
+  char* base;
+  size_t off;
+  template <class T>
+  T* take(size_t count) {
+    off = (off + 255) & ~size_t(255);
+    T* p = reinterpret_cast<T*>(base ? base + off : nullptr);
+    off += count * sizeof(T);
+    return p;
+  }
+};
+
+// ---- launchers (all asynchronous on `s`) ----
+size_t importance_workspace_bytes(int K);
+cudaError_t launch_importance(const uint16_t* W, const uint16_t* X, int M, int K, int N,
+                              float* I, float* s_scratch, cudaStream_t s);
+
+size_t search_workspace_bytes(int M, int K, int T, int ncand);
+cudaError_t launch_boundary_search(const float* I, const int32_t* perm, int M, int K, int T,
+                                   double t_s, double alpha, const Candidate* cands, int ncand,
+                                   int32_t* counts_out, double* vs_out, int32_t* rank_out,
+                                   void* ws, int* status, cudaStream_t s);
+
+size_t mask_workspace_bytes(int M, int K, int T);
+cudaError_t launch_mask(const float* I, const int32_t* perm, const int32_t* counts,
+                        const int32_t* rank, int M, int K, int T, uint32_t* bitmask,
+                        int8_t* region, void* ws, int* status, cudaStream_t s);
+
+size_t compress_workspace_bytes(int M, int K, int T);
+cudaError_t launch_compress(const uint16_t* W, const uint32_t* bitmask, const int8_t* region,
+                            const int32_t* perm, const int32_t* counts, int M, int K, int T,
+                            const hinm_layout& L, void* ws, int* status, cudaStream_t s);
+
+cudaError_t launch_spmm(const hinm_layout& L, const uint16_t* X, int N, float* Y,
+                        int* status, cudaStream_t s);
+
+// Shared by the rank users (search and mask): V (fp64 column sums per tile) and the rank
+// of every working position.
+cudaError_t launch_vector_rank(const float* I, const int32_t* perm, int M, int K, int T,
+                               double* V, int32_t* rank, cudaStream_t s);
+
+}  // namespace hinm

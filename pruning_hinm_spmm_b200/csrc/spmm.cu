@@ -1,0 +1,307 @@
+// a6. HiNM SpMM on the sm_100a tensor cores (FlexHiNM-GP notes, 关键设计 4: the dense part
+// and the 2:4 part, the latter gathered by the precomputed index, summed into one output).
+//
+// The pages run two CUDA streams (mma and mma.sp) merged by atomicAdd.  Here one CTA per
+// (tile, N-block) runs both kinds of K-block into ONE tensor-memory accumulator:
+//
+//   warp 0  producer : per K-block, one bulk copy of the pre-swizzled 16 KB A block (and,
+//                      for a 2:4 block, its 2 KB metadata), plus TMA gather4 loads of the
+//                      block's X rows selected by the index (4 rows per instruction,
+//                      swizzled for an MN-major B operand)
+//   warp 1  MMA      : one thread; 2:4 block -> tcgen05.cp of the metadata into tensor
+//                      memory, then 4 x tcgen05.mma.sp (K = 32 each); dense block ->
+//                      4 x tcgen05.mma (K = 16 each); tcgen05.commit frees the stage
+//   warps 2-5 epilogue: tcgen05.ld of the 128 x BN fp32 accumulator, stores to Y
+//
+// Shared memory holds STAGES stages of [A 16 KB | B 128 x BN bf16 | E 2 KB] behind full /
+// empty mbarriers.  Every wait is bounded (2 s), after which the CTA records
+// HINM_ERR_DEVICE_TIMEOUT, drains what it issued and exits.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "hinm_internal.h"
+#include "ptx.cuh"
+
+namespace hinm {
+
+template <int BN>
+struct SpmmCfg {
+  static constexpr int kAtom = BN >= 64 ? 64 : BN;  // B swizzle atom width (elements)
+  static constexpr int kAtomBytes = kAtom * 2;      // 128, 64 or 32 bytes
+  static constexpr int kNumAtoms = BN / kAtom;
+  static constexpr int kABytes = kBlockBytes;
+  static constexpr int kBBytes = 128 * BN * 2;  // 128 K-rows (a 2:4 block); dense uses 64
+  static constexpr int kEBytes = 2048;
+  static constexpr int kStageBytes = kABytes + kBBytes + kEBytes;
+  static constexpr int kStagesRaw = (200 * 1024) / kStageBytes;
+  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  // layout type of the B descriptor: 2 = 128-byte swizzle, 4 = 64-byte, 6 = 32-byte
+  static constexpr uint32_t kBLayout = kAtomBytes == 128 ? 2u : (kAtomBytes == 64 ? 4u : 6u);
+  static constexpr int kTmemNeed = BN + 4 * kStages;
+  static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
+                                   : kTmemNeed <= 256 ? 256 : 512;
+  static constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024 /*align*/ + 256;
+  static_assert(BN == 16 || BN == 32 || BN % 64 == 0, "BN");
+  static_assert(kStages >= 2, "stages");
+  static_assert(kTmemNeed <= 512, "tmem");
+};
+
+struct SpmmArgs {
+  const int32_t* tile_info;
+  const uint16_t* vals_dense;
+  const uint16_t* vals_sparse;
+  const uint32_t* meta;
+  const int32_t* idx_dense;
+  const int32_t* idx_sparse;
+  float* Y;
+  int N, T;
+  int* status;
+};
+
+template <int BN>
+__global__ void __launch_bounds__(192, 1)
+    spmm_kernel(const __grid_constant__ CUtensorMap tmX, const SpmmArgs a) {
+  using C = SpmmCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  // bars[0..S) full, bars[S..2S) empty, bars[2S] accumulator ready, bars[2S+1] drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::kStages + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.y;
+  const int n0 = blockIdx.x * BN;
+  const int4 info = *reinterpret_cast<const int4*>(a.tile_info + 4 * tile);
+  const int nd = info.x, ns = info.y, d0 = info.z, s0 = info.w;
+  const int nblk = nd + ns;
+
+  auto full_bar = [&](int s) { return ptx::smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return ptx::smem_u32(bars + C::kStages + s); };
+  const uint32_t acc_bar = ptx::smem_u32(bars + 2 * C::kStages);
+  const uint32_t drain_bar = ptx::smem_u32(bars + 2 * C::kStages + 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      ptx::mbar_init(full_bar(s), 1);
+      ptx::mbar_init(empty_bar(s), 1);
+    }
+    ptx::mbar_init(acc_bar, 1);
+    ptx::mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), C::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int issued = 0;
+    for (int kb = 0; kb < nblk; ++kb) {
+      const int s = kb % C::kStages;
+      const uint32_t ph = (kb / C::kStages) & 1;
+      if (!ptx::mbar_wait(empty_bar(s), ph ^ 1, a.status, abort_flag)) break;
+      const bool sparse = kb >= nd;
+      const int rows = sparse ? kSparseBK : kDenseBK;
+      uint8_t* st = smem + s * C::kStageBytes;
+      const uint32_t A_s = ptx::smem_u32(st);
+      const uint32_t B_s = A_s + C::kABytes;
+      const uint32_t E_s = B_s + C::kBBytes;
+      const size_t blk = sparse ? (size_t)(s0 + kb - nd) : (size_t)(d0 + kb);
+      if (lane == 0) {
+        const uint32_t bytes =
+            C::kABytes + (sparse ? C::kEBytes : 0) + (uint32_t)rows * BN * 2u;
+        ptx::mbar_arrive_expect_tx(full_bar(s), bytes);
+        ptx::bulk_g2s(A_s, (sparse ? a.vals_sparse : a.vals_dense) + blk * 8192, C::kABytes,
+                      full_bar(s));
+        if (sparse) ptx::bulk_g2s(E_s, a.meta + blk * kMetaWords, C::kEBytes, full_bar(s));
+      }
+      __syncwarp();
+      const int* idx = sparse ? a.idx_sparse + blk * kSparseBK : a.idx_dense + blk * kDenseBK;
+      const int quads = rows / 4;
+      for (int q = lane; q < quads * C::kNumAtoms; q += 32) {
+        const int rq = q % quads, at = q / quads;
+        const int4 r = __ldg(reinterpret_cast<const int4*>(idx) + rq);
+        ptx::tma_gather4(B_s + at * (128 * C::kAtomBytes) + rq * 4 * C::kAtomBytes, &tmX,
+                         n0 + at * C::kAtom, r.x, r.y, r.z, r.w, full_bar(s));
+      }
+      ++issued;
+    }
+    __syncwarp();
+    if (*abort_flag && lane == 0) {
+      // wait (bounded) for the copies this warp issued and nobody consumed
+      for (int kb = (issued > C::kStages ? issued - C::kStages : 0); kb < issued; ++kb)
+        ptx::mbar_wait(full_bar(kb % C::kStages), (kb / C::kStages) & 1, a.status, nullptr);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_d = ptx::idesc_bf16(BN, 1, 0);
+      const uint32_t idesc_s = ptx::idesc_bf16(BN, 1, 1);
+      bool any = false;
+      for (int kb = 0; kb < nblk; ++kb) {
+        const int s = kb % C::kStages;
+        const uint32_t ph = (kb / C::kStages) & 1;
+        if (!ptx::mbar_wait(full_bar(s), ph, a.status, abort_flag)) break;
+        ptx::tc_fence_after();
+        const bool sparse = kb >= nd;
+        const uint32_t A_s = ptx::smem_u32(smem + s * C::kStageBytes);
+        const uint32_t B_s = A_s + C::kABytes;
+        const uint32_t E_s = B_s + C::kBBytes;
+        if (sparse) {
+          const uint32_t e_col = tmem + BN + 4 * s;
+          // 128 lanes x 16 bytes, rows 16 B apart: core matrices of 8 rows, 128 B apart
+          ptx::tc_cp_128x128b(e_col, ptx::smem_desc(E_s, 2048, 128, 0));
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t ad = ptx::smem_desc(A_s + 32 * k, 16, 1024, 2);
+            const uint64_t bd = ptx::smem_desc(B_s + 32 * k * C::kAtomBytes, 128 * C::kAtomBytes,
+                                               8 * C::kAtomBytes, C::kBLayout);
+            const uint32_t e = e_col + k;
+            ptx::mma_sp_bf16(tmem, ad, bd, e & ~1u, idesc_s | (e & 1u), any ? 1u : 0u);
+            any = true;
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t ad = ptx::smem_desc(A_s + 32 * k, 16, 1024, 2);
+            const uint64_t bd = ptx::smem_desc(B_s + 16 * k * C::kAtomBytes, 128 * C::kAtomBytes,
+                                               8 * C::kAtomBytes, C::kBLayout);
+            ptx::mma_bf16(tmem, ad, bd, idesc_d, any ? 1u : 0u);
+            any = true;
+          }
+        }
+        ptx::tc_commit(empty_bar(s));
+      }
+      if (nblk > 0) ptx::tc_commit(acc_bar);
+      // every tcgen05 operation issued above has completed once drain_bar flips
+      ptx::tc_commit(drain_bar);
+      ptx::mbar_wait(drain_bar, 0, a.status, nullptr);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;  // tensor-memory lane quadrant this warp may access
+    const int row = q * 32 + lane;
+    bool have = nblk > 0;
+    if (have) {
+      have = ptx::mbar_wait(acc_bar, 0, a.status, abort_flag);
+      ptx::tc_fence_after();
+    }
+    const bool row_ok = row < a.T;
+    float* yrow = a.Y + (size_t)(tile * a.T + row) * a.N;
+    constexpr int kChunk = BN >= 32 ? 32 : 16;
+    for (int col = 0; col < BN; col += kChunk) {
+      uint32_t v[32];
+      if (have) {
+        const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)col;
+        if constexpr (kChunk == 32) {
+          ptx::tmem_ld_32x32b_x32(taddr, v);
+        } else {
+          ptx::tmem_ld_32x32b_x16(taddr, v);
+        }
+        ptx::tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0u;
+      }
+      if (row_ok && !(*abort_flag)) {
+        const int gc = n0 + col;
+        if (gc + kChunk <= a.N) {
+#pragma unroll
+          for (int i = 0; i < kChunk; i += 4) {
+            float4 o = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                                   __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+            *reinterpret_cast<float4*>(yrow + gc + i) = o;
+          }
+        } else {
+          for (int i = 0; i < kChunk; ++i)
+            if (gc + i < a.N) yrow[gc + i] = __uint_as_float(v[i]);
+        }
+      }
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// X (K rows x N bf16, row-major) as a 2-D tensor map whose box is one row of `atom`
+// elements, swizzled like the B operand (atom * 2 bytes per swizzle row).
+bool make_x_map(CUtensorMap* m, const uint16_t* X, int K, int N, int atom) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)K};
+  cuuint64_t strides[1] = {(cuuint64_t)N * 2};
+  cuuint32_t box[2] = {(cuuint32_t)atom, 1};
+  cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw = atom == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : atom == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                             : CU_TENSOR_MAP_SWIZZLE_32B;
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN>
+cudaError_t run(const hinm_layout& L, const uint16_t* X, int N, float* Y, int* status,
+                cudaStream_t s) {
+  using C = SpmmCfg<BN>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(spmm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)C::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  CUtensorMap map;
+  if (!make_x_map(&map, X, L.K, N, C::kAtom)) return cudaErrorInvalidValue;
+  SpmmArgs a{L.tile_info, L.vals_dense, L.vals_sparse, L.meta, L.idx_dense, L.idx_sparse,
+             Y,           N,            L.T,           status};
+  dim3 grid((N + BN - 1) / BN, L.num_tiles);
+  spmm_kernel<BN><<<grid, 192, C::kSmemBytes, s>>>(map, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_spmm(const hinm_layout& L, const uint16_t* X, int N, float* Y, int* status,
+                        cudaStream_t s) {
+  if (N <= 16) return run<16>(L, X, N, Y, status, s);
+  if (N <= 32) return run<32>(L, X, N, Y, status, s);
+  if (N <= 64) return run<64>(L, X, N, Y, status, s);
+  return run<128>(L, X, N, Y, status, s);
+}
+
+}  // namespace hinm

@@ -1,0 +1,116 @@
+"""Host-only checks of the C ABI: the library loads without a GPU, exports every entry
+point include/hinm.h declares, computes the closed-form counts and layout sizes the
+oracle predicts, and rejects bad arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import hinm_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def H():
+    from pruning_hinm_spmm_b200 import build_lib
+    build_lib.build()
+    import pruning_hinm_spmm_b200 as H
+    return H
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(hinm_\w+)\s*\(", src))
+    return names
+
+
+def test_exports_every_declared_symbol(H):
+    names = declared_functions()
+    assert {"hinm_importance", "hinm_boundary_search", "hinm_mask", "hinm_compress",
+            "hinm_spmm"} <= names
+    lib = ctypes.CDLL(H.LIB_PATH)
+    for n in sorted(names):
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+
+
+def test_versions_and_strings(H):
+    lib = H.lib()
+    assert lib.hinm_abi_version() == 1
+    assert lib.hinm_status_string(0) == b"HINM_OK"
+    assert lib.hinm_status_string(7) == b"HINM_ERR_BAD_MASK"
+
+
+@pytest.mark.parametrize("K", [64, 100, 200, 256, 4096, 11008])
+@pytest.mark.parametrize("t_s", [0.0, 0.5, 0.625, 0.75, 1.0])
+def test_counts_match_oracle(H, K, t_s):
+    for m in range(0, 40):
+        v_s = t_s - m / 32
+        if v_s < 0:
+            break
+        try:
+            want = O.counts_from_vs(K, t_s, v_s)
+        except ValueError:
+            with pytest.raises(H.HinmError):
+                H.hinm_counts_from_vs(K, t_s, v_s)
+            continue
+        assert H.hinm_counts_from_vs(K, t_s, v_s) == want
+
+
+def test_compress_size_matches_oracle(H):
+    for K, t_s, v_s in [(256, 0.5, 0.2), (4096, 0.75, 0.6), (11008, 0.625, 0.4), (4096, 0.5, 0.0)]:
+        c = np.array(O.counts_from_vs(K, t_s, v_s), dtype=np.int32)
+        counts = np.tile(c, (4, 1))
+        sz = H.hinm_compress_size(512, K, 128, counts)
+        info = O.tile_blocks(counts)
+        assert sz.max_dense_blocks == max(1, info[:, 0].sum())
+        assert sz.max_sparse_blocks == max(1, info[:, 1].sum())
+        worst = H.hinm_compress_size(512, K, 128, None)
+        assert worst.max_dense_blocks >= sz.max_dense_blocks
+        assert worst.max_sparse_blocks >= sz.max_sparse_blocks
+        assert worst.vals_dense_bytes == worst.max_dense_blocks * 16384
+
+
+def test_validation_rejects_before_launch(H):
+    lib = H.lib()
+    fake = 0x10000  # never dereferenced: every call below fails its host checks first
+    ws = ctypes.c_size_t(0)
+    # bad tile height / shapes
+    assert lib.hinm_search_workspace_size(256, 256, 32, 0.5, 1 / 32, ctypes.byref(ws)) == H.HINM_ERR_SHAPE
+    assert lib.hinm_search_workspace_size(200, 256, 64, 0.5, 1 / 32, ctypes.byref(ws)) == H.HINM_ERR_SHAPE
+    assert lib.hinm_search_workspace_size(256, 258, 64, 0.5, 1 / 32, ctypes.byref(ws)) == H.HINM_ERR_SHAPE
+    assert lib.hinm_search_workspace_size(256, 256, 64, 1.5, 1 / 32, ctypes.byref(ws)) == H.HINM_ERR_INVALID_ARG
+    assert lib.hinm_search_workspace_size(256, 256, 64, 0.5, 0.0, ctypes.byref(ws)) == H.HINM_ERR_INVALID_ARG
+    assert lib.hinm_search_workspace_size(256, 256, 64, 0.5, 1 / 32, ctypes.byref(ws)) == H.HINM_OK
+    assert ws.value > 0
+    # null / misaligned pointers
+    assert lib.hinm_importance(None, fake, 64, 64, 16, fake, fake, 1 << 20, None) == H.HINM_ERR_INVALID_ARG
+    assert lib.hinm_importance(fake + 2, fake, 64, 64, 16, fake, fake, 1 << 20, None) == H.HINM_ERR_ALIGNMENT
+    assert lib.hinm_importance(fake, fake, 64, 64, 12, fake, fake, 1 << 20, None) == H.HINM_ERR_SHAPE
+    assert lib.hinm_importance(fake, fake, 64, 64, 16, fake, fake, 0, None) == H.HINM_ERR_WORKSPACE
+    assert b"workspace" in lib.hinm_last_error()
+    # workspace too small for the search
+    cnt = ctypes.c_void_p(fake)
+    assert lib.hinm_boundary_search(fake, None, 256, 256, 64, 0.5, 1 / 32, fake, fake, None, fake, 16,
+                                    None) == H.HINM_ERR_WORKSPACE
+    # t_s * K not whole
+    assert lib.hinm_boundary_search(fake, None, 256, 100, 64, 0.333, 1 / 32, fake, fake, None, fake,
+                                    1 << 30, None) == H.HINM_ERR_INVALID_ARG
+    # layout checks
+    L = H.hinm_layout(H.HINM_LAYOUT_VERSION + 1, 256, 256, 64, 4, 1, 1, fake, fake, fake, fake, fake, fake)
+    assert lib.hinm_spmm(ctypes.byref(L), fake, 16, fake, None) == H.HINM_ERR_INVALID_ARG
+    L = H.hinm_layout(H.HINM_LAYOUT_VERSION, 256, 256, 64, 3, 1, 1, fake, fake, fake, fake, fake, fake)
+    assert lib.hinm_spmm(ctypes.byref(L), fake, 16, fake, None) == H.HINM_ERR_SHAPE
+    L = H.hinm_layout(H.HINM_LAYOUT_VERSION, 256, 256, 64, 4, 1, 1, fake, fake, fake, fake, fake, fake)
+    assert lib.hinm_spmm(ctypes.byref(L), fake, 20, fake, None) == H.HINM_ERR_SHAPE
+    assert lib.hinm_spmm(ctypes.byref(L), fake + 8, 16, fake, None) == H.HINM_ERR_ALIGNMENT
+    # compress size rejects inconsistent counts
+    bad = (ctypes.c_int32 * 3)(10, 11, 235)
+    out = H.hinm_layout_sizes()
+    assert lib.hinm_compress_size(bad, 64, 256, 64, ctypes.byref(out)) == H.HINM_ERR_INVALID_ARG

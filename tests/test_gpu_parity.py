@@ -1,0 +1,226 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle, element by element.
+
+Integer / index / byte results (masks, regions, counts, ranks, layout bytes, the
+importance bits) must match exactly.  The fp32 product must satisfy
+|y - y_ref| <= 1e-3 * sum|w||x| + 1e-5 (bf16 inputs, fp32 accumulation); where every
+partial sum is an exact integer it must match bitwise.
+"""
+import numpy as np
+import pytest
+
+import hinm_inputs as hi
+from oracle import hinm_oracle as O
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+TOL_REL, TOL_ABS = 1e-3, 1e-5
+
+
+@pytest.fixture(scope="module")
+def H():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import pruning_hinm_spmm_b200 as H
+    return H
+
+
+def dev_bf16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def dev_i32(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
+
+
+def status_ok(H):
+    assert H.hinm_device_status() == 0
+
+
+def layout_equal(L_gpu, L_ref, tiles=None):
+    info = L_gpu.tile_info.cpu().numpy()
+    np.testing.assert_array_equal(info if tiles is None else info[tiles],
+                                  L_ref.tile_info if tiles is None else L_ref.tile_info[tiles])
+    vd = L_gpu.vals_dense.cpu().numpy().view(np.uint8).reshape(-1, 16384)
+    vs = L_gpu.vals_sparse.cpu().numpy().view(np.uint8).reshape(-1, 16384)
+    me = L_gpu.meta.cpu().numpy().view(np.uint32)
+    idd = L_gpu.idx_dense.cpu().numpy()
+    ids = L_gpu.idx_sparse.cpu().numpy()
+    for t in (range(info.shape[0]) if tiles is None else tiles):
+        nd, ns, d0, s0 = info[t]
+        nd_r, ns_r, d0_r, s0_r = L_ref.tile_info[t]
+        assert (nd, ns) == (nd_r, ns_r)
+        np.testing.assert_array_equal(vd[d0:d0 + nd], L_ref.vals_dense[d0_r:d0_r + nd])
+        np.testing.assert_array_equal(vs[s0:s0 + ns], L_ref.vals_sparse[s0_r:s0_r + ns])
+        np.testing.assert_array_equal(me[s0:s0 + ns], L_ref.meta[s0_r:s0_r + ns])
+        np.testing.assert_array_equal(idd[d0:d0 + nd], L_ref.idx_dense[d0_r:d0_r + nd])
+        np.testing.assert_array_equal(ids[s0:s0 + ns], L_ref.idx_sparse[s0_r:s0_r + ns])
+
+
+def check_y(y_gpu, y_ref, bound, rows=None):
+    y = y_gpu if rows is None else y_gpu[rows]
+    err = np.abs(y.astype(np.float64) - y_ref)
+    lim = TOL_REL * bound + TOL_ABS
+    bad = err > lim
+    assert not bad.any(), f"{bad.sum()} outputs out of tolerance; worst {(err - lim).max():.3e}"
+
+
+def run_path(H, w, v_s=None, N=None):
+    """GPU path step by step; returns every intermediate as numpy."""
+    M, K, T = w.M, w.K, w.T
+    W, X = dev_bf16(w.W_bits), dev_bf16(w.X_bits)
+    perm = dev_i32(w.perm)
+    I = H.hinm_importance(W, X)
+    counts, vs, rank = H.hinm_boundary_search(I, perm, T, w.t_s, w.alpha)
+    if v_s is not None:
+        c = np.array(H.hinm_counts_from_vs(K, w.t_s, v_s), dtype=np.int32)
+        counts_used = dev_i32(np.tile(c, (M // T, 1)))
+        rank_used = None
+    else:
+        counts_used, rank_used = counts, rank
+    bm, region = H.hinm_mask(I, perm, counts_used, T, rank_used)
+    L = H.hinm_compress(W, bm, region, perm, counts_used, T)
+    Y = H.hinm_spmm(L, X)
+    torch.cuda.synchronize()
+    status_ok(H)
+    return dict(I=I.cpu().numpy(), counts=counts.cpu().numpy(), vs=vs.cpu().numpy(),
+                rank=rank.cpu().numpy(), counts_used=counts_used.cpu().numpy(),
+                bitmask=bm.cpu().numpy().view(np.uint32), region=region.cpu().numpy(), layout=L,
+                Y=Y.cpu().numpy())
+
+
+CASES = [
+    # name, workload factory, fixed v_s (None = searched)
+    ("tiny_hinm_T64", lambda: hi.tiny_hinm(0), 0.2),
+    ("tiny_searched", lambda: hi.tiny_hinm(0), None),
+    ("ragged_K200_N24_perm", lambda: hi.custom(256, 200, 24, 128, seed=3, t_s=0.625, v_s=None,
+                                              random_perm=True), 0.4),
+    ("ragged_K196_N40_T64", lambda: hi.custom(192, 196, 40, 64, seed=4, t_s=0.5, v_s=None,
+                                             random_perm=True), 0.25),
+    ("pure24_small_outliers", lambda: hi.custom(256, 256, 136, 128, seed=5, t_s=0.5, v_s=None,
+                                                outlier_frac=0.01), 0.0),
+    ("column_pruning_only", lambda: hi.custom(128, 192, 16, 64, seed=6, t_s=0.5, v_s=None), 0.5),
+    ("dense_ts0", lambda: hi.custom(128, 128, 32, 128, seed=7, t_s=0.0, v_s=None), 0.0),
+    ("all_pruned_ts1", lambda: hi.custom(128, 128, 16, 64, seed=8, t_s=1.0, v_s=None), 1.0),
+    ("multi_block_K640_N264", lambda: hi.custom(384, 640, 264, 128, seed=9, t_s=0.75, v_s=None,
+                                               random_perm=True), 0.6),
+]
+
+
+@pytest.mark.parametrize("name,make,v_s", CASES, ids=[c[0] for c in CASES])
+def test_path_matches_oracle(H, name, make, v_s):
+    w = make()
+    g = run_path(H, w, v_s)
+    # a1 importance: bit-exact
+    I_ref = O.importance(w.W_bits, w.X_bits)
+    np.testing.assert_array_equal(g["I"].view(np.uint32), I_ref.view(np.uint32))
+    # a2/a3 search: counts, v_s, rank bit-exact
+    sr = O.boundary_search(I_ref, w.perm, w.T, w.t_s, w.alpha)
+    np.testing.assert_array_equal(g["counts"], sr.counts)
+    np.testing.assert_array_equal(g["vs"], sr.v_s)
+    np.testing.assert_array_equal(g["rank"], sr.rank)
+    counts = g["counts_used"]
+    # a4 mask
+    bm_ref, reg_ref = O.mask(I_ref, w.perm, w.T, counts)
+    np.testing.assert_array_equal(g["region"], reg_ref)
+    np.testing.assert_array_equal(g["bitmask"], bm_ref)
+    # a5 layout bytes
+    L_ref = O.compress(w.W_bits, bm_ref, reg_ref, w.perm, counts, w.T)
+    layout_equal(g["layout"], L_ref)
+    # a6 product
+    y_ref, bound = O.spmm_reference(w.W_bits, bm_ref, w.X_bits)
+    check_y(g["Y"], y_ref, bound)
+
+
+def test_identity_x_reproduces_masked_weight(H):
+    """X = I_K (N = K): Y must equal W ⊙ M exactly, which pins the value layout, the
+    metadata placement and the gather to the tensor cores' reading of them."""
+    w = hi.custom(256, 256, 256, 128, seed=11, t_s=0.625, v_s=None, random_perm=True)
+    w.X_bits = hi.f32_to_bf16_bits(np.eye(256, dtype=np.float32))
+    w.N = 256
+    g = run_path(H, w, v_s=0.375)
+    Wm = O.masked_weight(w.W_bits, g["bitmask"])
+    np.testing.assert_array_equal(g["Y"], Wm.astype(np.float32))
+
+
+@pytest.mark.parametrize("T,N,perm", [(64, 16, False), (128, 48, True), (128, 264, True)])
+def test_integer_product_bitwise(H, T, N, perm):
+    w = hi.integer_workload(2 * T, 384, N, T, seed=2, t_s=0.625, v_s=None, random_perm=perm)
+    g = run_path(H, w, v_s=0.375)
+    Wm = O.masked_weight(w.W_bits, g["bitmask"]).astype(np.int64)
+    Xi = hi.bf16_bits_to_f32(w.X_bits).astype(np.int64)
+    np.testing.assert_array_equal(g["Y"].astype(np.int64), Wm @ Xi)
+    assert np.array_equal(g["Y"], np.round(g["Y"]))
+
+
+def test_hand_built_first_drop(H):
+    """The hand-built tile where regrouping makes R drop at m = 2: the GPU scan stops at m=1."""
+    K, N, T = 64, 8, 64
+    mags = np.array([8.0] * 28 + [3.0] * 2 + [2.875] * 2 + [1.25] * 2 + [1.0] * 2 + [0.5] * 28)
+    signs = np.where(np.random.default_rng(0).random((T, K)) < 0.5, -1.0, 1.0)
+    W = hi.f32_to_bf16_bits((signs * mags[None, :]).astype(np.float32))
+    X = hi.f32_to_bf16_bits(np.ones((K, N), dtype=np.float32))
+    I = H.hinm_importance(dev_bf16(W), dev_bf16(X))
+    counts, vs, _ = H.hinm_boundary_search(I, None, T, 0.5, 1 / 32)
+    assert tuple(counts.cpu().numpy()[0]) == (30, 4, 30)
+    assert vs.cpu().numpy()[0] == 0.5 - 1 / 32
+
+
+def test_bad_mask_is_reported_not_faulted(H):
+    """A 2:4 group with 3 kept bits sets HINM_ERR_BAD_MASK in the device status word."""
+    w = hi.custom(128, 128, 16, 128, seed=1, t_s=0.5, v_s=None)
+    W, X = dev_bf16(w.W_bits), dev_bf16(w.X_bits)
+    I = H.hinm_importance(W, X)
+    c = dev_i32(np.array([H.hinm_counts_from_vs(128, 0.5, 0.0)], dtype=np.int32))
+    bm, region = H.hinm_mask(I, None, c, 128)
+    bm = bm.clone()
+    bm[0, 0] = -1  # all 32 channels of row 0 kept: 8 groups with 4 kept bits
+    H.hinm_compress(W, bm, region, None, c, 128)
+    torch.cuda.synchronize()
+    assert H.hinm_device_status() == H.HINM_ERR_BAD_MASK
+    assert H.hinm_device_status() == 0  # cleared by the read
+
+
+# ---------------------------------------------------------------- full-size workloads
+FULL = [("pure24_4096x4096x2048", hi.pure24, 0.0),
+        ("hinm_up_11008x4096x4096", hi.hinm_up_proj, 0.6),
+        ("decode_down_4096x11008x16", hi.decode_down_proj, 0.4)]
+
+
+@pytest.mark.parametrize("name,make,v_s", FULL, ids=[f[0] for f in FULL])
+def test_full_size_sampled(H, name, make, v_s):
+    """Full-size workloads in the launch configuration the benchmark times; the oracle
+    checks sampled tiles (importance rows, search, mask, layout bytes, output rows)."""
+    w = make()
+    M, K, N, T = w.M, w.K, w.N, w.T
+    nt = M // T
+    W, X, perm = dev_bf16(w.W_bits), dev_bf16(w.X_bits), dev_i32(w.perm)
+    hp = H.HotPath(M, K, N, T, w.t_s, w.alpha)
+    c = np.array(H.hinm_counts_from_vs(K, w.t_s, v_s), dtype=np.int32)
+    fixed = dev_i32(np.tile(c, (nt, 1)))
+    Y = hp.run(W, X, perm, fixed_counts=fixed)
+    torch.cuda.synchronize()
+    status_ok(H)
+    tiles = sorted({0, nt // 2, nt - 1})
+    rows = np.concatenate([np.arange(t * T, (t + 1) * T) for t in tiles])
+    s = O.channel_energy(w.X_bits)
+    Wf = hi.bf16_bits_to_f32(w.W_bits[rows])
+    I_rows = ((Wf * Wf).astype(np.float32) * s[None, :]).astype(np.float32)
+    np.testing.assert_array_equal(hp.I[rows].cpu().numpy(), I_rows)
+    # search on the sampled tiles (the GPU's own search, not the fixed counts)
+    counts_s, vs_s, rank_s = H.hinm_boundary_search(hp.I, perm, T, w.t_s, w.alpha)
+    I_full_rows = np.zeros((M, K), dtype=np.float32)
+    I_full_rows[rows] = I_rows
+    sr = O.boundary_search(I_full_rows, w.perm, T, w.t_s, w.alpha, tiles=tiles)
+    np.testing.assert_array_equal(counts_s.cpu().numpy()[tiles], sr.counts[tiles])
+    np.testing.assert_array_equal(rank_s.cpu().numpy()[tiles], sr.rank[tiles])
+    # mask + layout + product on the sampled tiles with the fixed counts
+    counts = np.tile(c, (nt, 1))
+    bm_ref, reg_ref = O.mask(I_full_rows, w.perm, T, counts, tiles=tiles)
+    bm = hp.bitmask.cpu().numpy().view(np.uint32)
+    np.testing.assert_array_equal(bm[rows], bm_ref[rows])
+    np.testing.assert_array_equal(hp.region.cpu().numpy()[tiles], reg_ref[tiles])
+    L_ref = O.compress(w.W_bits, bm_ref, reg_ref, w.perm, counts, T, tiles=tiles)
+    layout_equal(hp.layout, L_ref, tiles=tiles)
+    y_ref, bound = O.spmm_reference(w.W_bits, bm_ref, w.X_bits, rows=rows)
+    check_y(Y.cpu().numpy(), y_ref, bound, rows=rows)
