@@ -51,7 +51,7 @@ extern "C" {
 #endif
 
 #define HINM_ABI_VERSION 1
-#define HINM_LAYOUT_VERSION 1
+#define HINM_LAYOUT_VERSION 2
 
 typedef enum {
   HINM_OK = 0,
@@ -109,14 +109,17 @@ hinm_status hinm_counts_from_vs(int K, double t_s, double v_s, int32_t* out_host
  * I: fp32 [M][K]; perm: int32 [K] (NULL = identity), working position j holds channel
  * perm[j]; counts_out: int32 [M/T][3] = {n_0, n_24, n_4}; vs_out: fp64 [M/T];
  * rank_out (NULL allowed): int32 [M/T][K], rank of working position j.
+ * retained_out (NULL allowed): fp64 [M/T][n_cand], R(m) of every tile and candidate
+ * (n_cand from hinm_search_num_candidates).
  * alpha > 0, 0 <= t_s <= 1.  workspace: hinm_search_workspace_size() bytes.
  * -------------------------------------------------------------------------------- */
+hinm_status hinm_search_num_candidates(int K, double t_s, double alpha, int32_t* n_host);
 hinm_status hinm_search_workspace_size(int M, int K, int T, double t_s, double alpha,
                                        size_t* bytes_host);
 hinm_status hinm_boundary_search(const float* I, const int32_t* perm, int M, int K, int T,
                                  double t_s, double alpha, int32_t* counts_out,
-                                 double* vs_out, int32_t* rank_out, void* workspace,
-                                 size_t workspace_bytes, void* stream);
+                                 double* vs_out, int32_t* rank_out, double* retained_out,
+                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------
  * a4. Mask  ([P1] 亮点与洞察: high -> dense, middle -> 2:4, low -> pruned;
@@ -144,7 +147,9 @@ hinm_status hinm_mask(const float* I, const int32_t* perm, const int32_t* counts
  *   meta block    2048 B: 128 lanes x 4 uint32 words; word w of lane L, bits
  *                [16s+4q, 16s+4q+4) = a | b<<2 (a < b, kept positions 0..3) of group
  *                8w + 4((L/8)%2) + q of row 16(L/16) + 8s + L%8;
- *   index         int32 per vector = perm[j] (input channel), 0 for padding.
+ *   index         int32 per vector = perm[j] (input channel), 0 for padding;
+ *   run           int32 per block = index[0] if the block's indices are one ascending
+ *                 run index[0], index[0]+1, ..., else -1 (such blocks of X load as a tile).
  * Padding: value 0, nibble 0x4, index 0.
  * tile_info[t] = { dense blocks, sparse blocks, first dense block, first sparse block }.
  * -------------------------------------------------------------------------------- */
@@ -159,12 +164,14 @@ typedef struct {
   uint32_t* meta;             /* device uint32 [max_sparse_blocks][512] */
   int32_t* idx_dense;         /* device int32 [max_dense_blocks][64] */
   int32_t* idx_sparse;        /* device int32 [max_sparse_blocks][128] */
+  int32_t* run_dense;         /* device int32 [max_dense_blocks] */
+  int32_t* run_sparse;        /* device int32 [max_sparse_blocks] */
 } hinm_layout;
 
 typedef struct {
   int32_t max_dense_blocks, max_sparse_blocks;
   size_t tile_info_bytes, vals_dense_bytes, vals_sparse_bytes, meta_bytes,
-      idx_dense_bytes, idx_sparse_bytes;
+      idx_dense_bytes, idx_sparse_bytes, run_dense_bytes, run_sparse_bytes;
 } hinm_layout_sizes;
 
 /* Buffer sizes.  counts_host (int32 [M/T][3], host) gives exact sizes; NULL gives the

@@ -393,6 +393,8 @@ class Layout:
     meta: np.ndarray            # uint32 [ns_total, 512]
     idx_dense: np.ndarray       # int32 [nd_total, 64]
     idx_sparse: np.ndarray      # int32 [ns_total, 128]
+    run_dense: np.ndarray       # int32 [nd_total]: idx[0] if idx[v] == idx[0] + v for all v, else -1
+    run_sparse: np.ndarray      # int32 [ns_total]
 
 
 def tile_blocks(counts: np.ndarray) -> np.ndarray:
@@ -483,7 +485,19 @@ def compress(W_bits: np.ndarray, bitmask: np.ndarray, region: np.ndarray, perm: 
             vals_sparse[s0 + b] = blk
             meta[s0 + b] = mw.astype(np.uint32)
     return Layout(M=M, K=K, T=T, tile_info=info, vals_dense=vals_dense,
-                  vals_sparse=vals_sparse, meta=meta, idx_dense=idx_dense, idx_sparse=idx_sparse)
+                  vals_sparse=vals_sparse, meta=meta, idx_dense=idx_dense, idx_sparse=idx_sparse,
+                  run_dense=contiguous_runs(idx_dense), run_sparse=contiguous_runs(idx_sparse))
+
+
+def contiguous_runs(idx: np.ndarray) -> np.ndarray:
+    """Per block: the first index if the block's indices are one ascending run
+    (idx[v] = idx[0] + v), else -1.  Lets the product load such blocks of X as one tile."""
+    out = np.full(idx.shape[0], -1, dtype=np.int32)
+    if idx.shape[0]:
+        steps = idx - idx[:, :1]
+        run = (steps == np.arange(idx.shape[1], dtype=np.int32)[None, :]).all(axis=1)
+        out[run] = idx[run, 0]
+    return out
 
 
 def decompress(L: Layout) -> np.ndarray:

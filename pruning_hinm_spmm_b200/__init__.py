@@ -25,13 +25,13 @@ HINM_ERR_CUDA = 5
 HINM_ERR_DEVICE_TIMEOUT = 6
 HINM_ERR_BAD_MASK = 7
 HINM_ERR_WORKSPACE = 8
-HINM_LAYOUT_VERSION = 1
+HINM_LAYOUT_VERSION = 2
 
 REGION_PRUNED, REGION_24, REGION_DENSE = 0, 1, 2
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m pruning_hinm_spmm_b200.build_lib` "
+        f"{LIB_PATH} is missing: build it with `python pruning_hinm_spmm_b200/build_lib.py` "
         "(the HiNM path has no CPU fallback)")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -45,13 +45,14 @@ class hinm_layout(ctypes.Structure):
                 ("T", ctypes.c_int32), ("num_tiles", ctypes.c_int32),
                 ("max_dense_blocks", ctypes.c_int32), ("max_sparse_blocks", ctypes.c_int32),
                 ("tile_info", _vp), ("vals_dense", _vp), ("vals_sparse", _vp), ("meta", _vp),
-                ("idx_dense", _vp), ("idx_sparse", _vp)]
+                ("idx_dense", _vp), ("idx_sparse", _vp), ("run_dense", _vp), ("run_sparse", _vp)]
 
 
 class hinm_layout_sizes(ctypes.Structure):
     _fields_ = [("max_dense_blocks", ctypes.c_int32), ("max_sparse_blocks", ctypes.c_int32),
                 ("tile_info_bytes", _sz), ("vals_dense_bytes", _sz), ("vals_sparse_bytes", _sz),
-                ("meta_bytes", _sz), ("idx_dense_bytes", _sz), ("idx_sparse_bytes", _sz)]
+                ("meta_bytes", _sz), ("idx_dense_bytes", _sz), ("idx_sparse_bytes", _sz),
+                ("run_dense_bytes", _sz), ("run_sparse_bytes", _sz)]
 
 
 _SIGS = {
@@ -61,9 +62,10 @@ _SIGS = {
     "hinm_importance_workspace_size": (_i32, [_i32, _i32, _i32, _szp]),
     "hinm_importance": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _sz, _vp]),
     "hinm_counts_from_vs": (_i32, [_i32, _f64, _f64, ctypes.POINTER(ctypes.c_int32)]),
+    "hinm_search_num_candidates": (_i32, [_i32, _f64, _f64, ctypes.POINTER(ctypes.c_int32)]),
     "hinm_search_workspace_size": (_i32, [_i32, _i32, _i32, _f64, _f64, _szp]),
     "hinm_boundary_search": (_i32, [_vp, _vp, _i32, _i32, _i32, _f64, _f64, _vp, _vp, _vp, _vp,
-                                    _sz, _vp]),
+                                    _vp, _sz, _vp]),
     "hinm_mask_workspace_size": (_i32, [_i32, _i32, _i32, _szp]),
     "hinm_mask": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
     "hinm_compress_size": (_i32, [_vp, _i32, _i32, _i32, ctypes.POINTER(hinm_layout_sizes)]),
@@ -149,10 +151,18 @@ def hinm_search_workspace_size(M, K, T, t_s, alpha) -> int:
     return _size(_lib.hinm_search_workspace_size, M, K, T, t_s, alpha)
 
 
+def hinm_search_num_candidates(K: int, t_s: float, alpha: float = 1.0 / 32.0) -> int:
+    out = ctypes.c_int32(0)
+    _check(_lib.hinm_search_num_candidates(K, t_s, alpha, ctypes.byref(out)),
+           "hinm_search_num_candidates")
+    return int(out.value)
+
+
 def hinm_boundary_search(I, perm, T: int, t_s: float, alpha: float = 1.0 / 32.0,
                          counts_out=None, vs_out=None, rank_out=None, workspace=None,
-                         want_rank: bool = True, stream=None):
-    """Per-tile first-drop scan of v_s.  Returns (counts int32 [M/T,3], v_s fp64 [M/T], rank)."""
+                         want_rank: bool = True, retained_out=None, stream=None):
+    """Per-tile first-drop scan of v_s.  Returns (counts int32 [M/T,3], v_s fp64 [M/T], rank).
+    ``retained_out`` (fp64 [M/T, n_cand]) optionally receives R(m) of every candidate."""
     torch = _torch()
     M, K = I.shape
     nt = M // T
@@ -166,8 +176,9 @@ def hinm_boundary_search(I, perm, T: int, t_s: float, alpha: float = 1.0 / 32.0,
     if workspace is None:
         workspace = _empty_bytes(hinm_search_workspace_size(M, K, T, t_s, alpha), dev)
     _check(_lib.hinm_boundary_search(_ptr(I), _ptr(perm), M, K, T, t_s, alpha, _ptr(counts_out),
-                                     _ptr(vs_out), _ptr(rank_out), _ptr(workspace),
-                                     workspace.numel(), _stream(stream)), "hinm_boundary_search")
+                                     _ptr(vs_out), _ptr(rank_out), _ptr(retained_out),
+                                     _ptr(workspace), workspace.numel(), _stream(stream)),
+           "hinm_boundary_search")
     return counts_out, vs_out, rank_out
 
 
@@ -221,6 +232,8 @@ class HinmLayout:
     meta: object         # int32 [blocks, 512]
     idx_dense: object    # int32 [blocks, 64]
     idx_sparse: object   # int32 [blocks, 128]
+    run_dense: object    # int32 [blocks]
+    run_sparse: object   # int32 [blocks]
 
     @classmethod
     def allocate(cls, M: int, K: int, T: int, device, counts_host=None) -> "HinmLayout":
@@ -233,13 +246,16 @@ class HinmLayout:
                    vals_sparse=torch.empty((ns, 8192), dtype=torch.int16, device=device),
                    meta=torch.empty((ns, 512), dtype=torch.int32, device=device),
                    idx_dense=torch.empty((nd, 64), dtype=torch.int32, device=device),
-                   idx_sparse=torch.empty((ns, 128), dtype=torch.int32, device=device))
+                   idx_sparse=torch.empty((ns, 128), dtype=torch.int32, device=device),
+                   run_dense=torch.empty((nd,), dtype=torch.int32, device=device),
+                   run_sparse=torch.empty((ns,), dtype=torch.int32, device=device))
 
     def as_c(self) -> hinm_layout:
         return hinm_layout(HINM_LAYOUT_VERSION, self.M, self.K, self.T, self.M // self.T,
                            self.max_dense_blocks, self.max_sparse_blocks,
                            _ptr(self.tile_info), _ptr(self.vals_dense), _ptr(self.vals_sparse),
-                           _ptr(self.meta), _ptr(self.idx_dense), _ptr(self.idx_sparse))
+                           _ptr(self.meta), _ptr(self.idx_dense), _ptr(self.idx_sparse),
+                           _ptr(self.run_dense), _ptr(self.run_sparse))
 
 
 def hinm_compress_workspace_size(M, K, T) -> int:

@@ -1,6 +1,8 @@
 """Build the HiNM C-ABI shared library (libhinm.so) for sm_100a with nvcc, in-tree.
 
-Usage: python -m pruning_hinm_spmm_b200.build_lib   (or build() from __graft_entry__)
+Usage: python pruning_hinm_spmm_b200/build_lib.py [-v] [-f]
+It is loaded by file path (see load_builder in __graft_entry__ and tests/conftest.py)
+because importing the package itself requires the library to exist already.
 """
 from __future__ import annotations
 

@@ -199,6 +199,18 @@ hinm_status hinm_importance(const void* W, const void* X, int M, int K, int N, f
   return ok();
 }
 
+hinm_status hinm_search_num_candidates(int K, double t_s, double alpha, int32_t* n_host) {
+  if (!n_host) return fail(HINM_ERR_INVALID_ARG, "n_host is NULL");
+  if (K < 4 || K > hinm::kMaxK) return fail(HINM_ERR_SHAPE, "K=%d out of range", K);
+  hinm_status st = check_search_params(t_s, alpha);
+  if (st != HINM_OK) return st;
+  hinm::Candidate c[hinm::kMaxCandidates];
+  const int n = hinm::search_candidates_host(K, t_s, alpha, c, hinm::kMaxCandidates);
+  if (n < 0) return fail(HINM_ERR_INVALID_ARG, "t_s*K = %g is not a whole number", t_s * K);
+  *n_host = n;
+  return ok();
+}
+
 hinm_status hinm_search_workspace_size(int M, int K, int T, double t_s, double alpha,
                                        size_t* bytes_host) {
   if (!bytes_host) return fail(HINM_ERR_INVALID_ARG, "bytes_host is NULL");
@@ -215,13 +227,14 @@ hinm_status hinm_search_workspace_size(int M, int K, int T, double t_s, double a
 
 hinm_status hinm_boundary_search(const float* I, const int32_t* perm, int M, int K, int T,
                                  double t_s, double alpha, int32_t* counts_out, double* vs_out,
-                                 int32_t* rank_out, void* workspace, size_t workspace_bytes,
-                                 void* stream) {
+                                 int32_t* rank_out, double* retained_out, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
   REQUIRE_PTR(I);
   REQUIRE_ALIGNED_OR_NULL(perm);
   REQUIRE_PTR(counts_out);
   REQUIRE_PTR(vs_out);
   REQUIRE_ALIGNED_OR_NULL(rank_out);
+  REQUIRE_ALIGNED_OR_NULL(retained_out);
   hinm_status st = check_mkt(M, K, T);
   if (st != HINM_OK) return st;
   st = check_search_params(t_s, alpha);
@@ -238,7 +251,7 @@ hinm_status hinm_boundary_search(const float* I, const int32_t* perm, int M, int
     return fail(HINM_ERR_WORKSPACE, "workspace %zu bytes, need %zu", workspace_bytes, need);
   REQUIRE_PTR(workspace);
   cudaError_t e = hinm::launch_boundary_search(I, perm, M, K, T, t_s, alpha, c, n, counts_out,
-                                               vs_out, rank_out, workspace,
+                                               vs_out, rank_out, retained_out, workspace,
                                                hinm::device_status_ptr(),
                                                static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "hinm_boundary_search launch");
@@ -306,6 +319,8 @@ hinm_status hinm_compress_size(const int32_t* counts_host, int M, int K, int T,
   out_host->meta_bytes = (size_t)ns * hinm::kMetaWords * sizeof(uint32_t);
   out_host->idx_dense_bytes = (size_t)nd * hinm::kDenseBK * sizeof(int32_t);
   out_host->idx_sparse_bytes = (size_t)ns * hinm::kSparseBK * sizeof(int32_t);
+  out_host->run_dense_bytes = (size_t)nd * sizeof(int32_t);
+  out_host->run_sparse_bytes = (size_t)ns * sizeof(int32_t);
   return ok();
 }
 
@@ -334,6 +349,8 @@ static hinm_status check_layout(const hinm_layout* L) {
   REQUIRE_PTR(L->meta);
   REQUIRE_PTR(L->idx_dense);
   REQUIRE_PTR(L->idx_sparse);
+  REQUIRE_PTR(L->run_dense);
+  REQUIRE_PTR(L->run_sparse);
   return HINM_OK;
 }
 

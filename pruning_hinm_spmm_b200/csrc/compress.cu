@@ -114,6 +114,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint16_t* __restrict__ 
                                                    const int32_t* __restrict__ lists, int K, int T,
                                                    hinm_layout L, int* status) {
   __shared__ uint8_t nib[128][32];
+  __shared__ int idx_s[kSparseBK];
   const int t = blockIdx.y;
   const int b = blockIdx.x;
   const int nd = L.tile_info[4 * t + 0], ns = L.tile_info[4 * t + 1];
@@ -146,11 +147,17 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint16_t* __restrict__ 
       q.w = h[6] | (h[7] << 16);
       *reinterpret_cast<uint4*>(out + r * 128 + ((ch ^ (r & 7)) << 4)) = q;
     }
+    int v = 0;
     if (threadIdx.x < kDenseBK) {
       const int p = b * kDenseBK + threadIdx.x;
-      L.idx_dense[(size_t)(d0 + b) * kDenseBK + threadIdx.x] =
-          p < n4 ? ptx::perm_at(perm, list_at(lst, p, K), K) : 0;
+      v = p < n4 ? ptx::perm_at(perm, list_at(lst, p, K), K) : 0;
+      L.idx_dense[(size_t)(d0 + b) * kDenseBK + threadIdx.x] = v;
+      idx_s[threadIdx.x] = v;
     }
+    __syncthreads();
+    const bool step_ok = threadIdx.x >= kDenseBK || v == idx_s[0] + (int)threadIdx.x;
+    const bool run = __syncthreads_and(step_ok);
+    if (threadIdx.x == 0) L.run_dense[d0 + b] = run ? idx_s[0] : -1;
     return;
   }
   const int sb = b - nd;
@@ -203,11 +210,17 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint16_t* __restrict__ 
     }
     meta[wi] = word;
   }
+  int v = 0;
   if (threadIdx.x < kSparseBK) {
     const int p = sb * kSparseBK + threadIdx.x;
-    L.idx_sparse[(size_t)(s0 + sb) * kSparseBK + threadIdx.x] =
-        p < n24 ? ptx::perm_at(perm, list_at(lst, n4 + p, K), K) : 0;
+    v = p < n24 ? ptx::perm_at(perm, list_at(lst, n4 + p, K), K) : 0;
+    L.idx_sparse[(size_t)(s0 + sb) * kSparseBK + threadIdx.x] = v;
+    idx_s[threadIdx.x] = v;
   }
+  __syncthreads();
+  const bool step_ok = threadIdx.x >= kSparseBK || v == idx_s[0] + (int)threadIdx.x;
+  const bool run = __syncthreads_and(step_ok);
+  if (threadIdx.x == 0) L.run_sparse[s0 + sb] = run ? idx_s[0] : -1;
 }
 
 size_t compress_workspace_bytes(int M, int K, int T) {

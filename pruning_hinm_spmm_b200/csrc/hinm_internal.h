@@ -56,7 +56,7 @@ size_t search_workspace_bytes(int M, int K, int T, int ncand);
 cudaError_t launch_boundary_search(const float* I, const int32_t* perm, int M, int K, int T,
                                    double t_s, double alpha, const Candidate* cands, int ncand,
                                    int32_t* counts_out, double* vs_out, int32_t* rank_out,
-                                   void* ws, int* status, cudaStream_t s);
+                                   double* retained_out, void* ws, int* status, cudaStream_t s);
 
 size_t mask_workspace_bytes(int M, int K, int T);
 cudaError_t launch_mask(const float* I, const int32_t* perm, const int32_t* counts,
@@ -73,7 +73,8 @@ cudaError_t launch_spmm(const hinm_layout& L, const uint16_t* X, int N, float* Y
 
 // Shared by the rank users (search and mask): V (fp64 column sums per tile) and the rank
 // of every working position.
+// tile_pmax (int [M/T]) receives each tile's largest fp32 exponent.
 cudaError_t launch_vector_rank(const float* I, const int32_t* perm, int M, int K, int T,
-                               double* V, int32_t* rank, cudaStream_t s);
+                               double* V, int32_t* rank, int* tile_pmax, cudaStream_t s);
 
 }  // namespace hinm

@@ -153,6 +153,7 @@ size_t mask_workspace_bytes(int M, int K, int T) {
   c.take<int32_t>((size_t)K);       // inverse permutation
   c.take<int32_t>((size_t)nt * K);  // pos24
   c.take<int32_t>((size_t)nt * K);  // member
+  c.take<int>((size_t)nt);          // tile max exponent (by-product of the ranking)
   return (c.off + 255) & ~size_t(255);
 }
 
@@ -166,9 +167,10 @@ cudaError_t launch_mask(const float* I, const int32_t* perm, const int32_t* coun
   int32_t* pinv = cv.take<int32_t>((size_t)K);
   int32_t* pos24 = cv.take<int32_t>((size_t)nt * K);
   int32_t* member = cv.take<int32_t>((size_t)nt * K);
+  int* pmax = cv.take<int>((size_t)nt);
   cudaError_t e;
   if (!rank) {
-    e = launch_vector_rank(I, perm, M, K, T, V, rank_ws, s);
+    e = launch_vector_rank(I, perm, M, K, T, V, rank_ws, pmax, s);
     if (e != cudaSuccess) return e;
     rank = rank_ws;
   }

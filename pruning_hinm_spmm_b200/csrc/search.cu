@@ -19,15 +19,94 @@
 namespace hinm {
 
 // ------------------------------------------------------------------ vector scores
+// Exact sums.  Every non-negative finite fp32 value is m * 2^(p - 149) with an integer
+// mantissa m < 2^24 and p = max(biased exponent, 1) - 1 in [0, 253].  Within a tile the
+// sums are kept as 128-bit integers in units of 2^(lsb - 149), lsb = max(P - 83, 0),
+// P = the tile's largest p: a value then needs at most 107 bits and 2^21 of them (128
+// rows x 16384 columns) still fit.  A value more than 2^83 below the tile's largest
+// (p < lsb) would lose bits there, so it goes to 64-bit exponent buckets instead.
+constexpr int kHeadroomShift = 83;
+
+__device__ __forceinline__ void split_f32(float v, uint32_t& m, int& p) {
+  const uint32_t u = __float_as_uint(v);
+  const uint32_t e = (u >> 23) & 0xFF;
+  m = (u & 0x7FFFFF) | (e ? 0x800000u : 0u);
+  p = (e ? (int)e : 1) - 1;
+}
+
+struct U128 {
+  unsigned long long lo, hi;
+};
+
+// a += m * 2^sh, 0 <= sh <= 104
+__device__ __forceinline__ void add_shifted(U128& a, uint32_t m, int sh) {
+  unsigned long long lo, hi;
+  if (sh < 64) {
+    lo = (unsigned long long)m << sh;
+    hi = sh > 40 ? ((unsigned long long)m >> (64 - sh)) : 0ull;
+  } else {
+    lo = 0ull;
+    hi = (unsigned long long)m << (sh - 64);
+  }
+  a.lo += lo;
+  a.hi += hi + (a.lo < lo ? 1ull : 0ull);
+}
+
+__device__ __forceinline__ void add128(U128& a, const U128& b) {
+  a.lo += b.lo;
+  a.hi += b.hi + (a.lo < b.lo ? 1ull : 0ull);
+}
+
+__device__ __forceinline__ int tile_lsb(int pmax) {
+  return pmax > kHeadroomShift ? pmax - kHeadroomShift : 0;
+}
+
+// Pass 1, thread per (tile, channel): V[t, c] = sum over the tile's rows, ascending, of
+// I (fp64), and the tile's largest exponent P.
 __global__ void vector_score_kernel(const float* __restrict__ I, int K, int T,
-                                    double* __restrict__ Vc) {
+                                    double* __restrict__ Vc, int* __restrict__ tile_pmax) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  const int t = blockIdx.y;
+  int pm = 0;
+  if (c < K) {
+    const float* p = I + (size_t)t * T * K + c;
+    double acc = 0.0;
+    for (int i = 0; i < T; ++i) {
+      const float v = __ldg(p + (size_t)i * K);
+      acc = __dadd_rn(acc, (double)v);
+      uint32_t m;
+      int e;
+      split_f32(v, m, e);
+      if (m) pm = max(pm, e);
+    }
+    Vc[(size_t)t * K + c] = acc;
+  }
+  for (int o = 16; o > 0; o >>= 1) pm = max(pm, __shfl_xor_sync(0xffffffffu, pm, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(tile_pmax + t, pm);
+}
+
+// Pass 2, thread per (tile, channel): the column's exact sum at the tile's scale, and a
+// flag when some of its values fell below that scale (summed exactly elsewhere).
+__global__ void column_sum_kernel(const float* __restrict__ I, int K, int T,
+                                  const int* __restrict__ tile_pmax, U128* __restrict__ colsum,
+                                  unsigned char* __restrict__ coltiny) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   const int t = blockIdx.y;
   if (c >= K) return;
+  const int lsb = tile_lsb(tile_pmax[t]);
   const float* p = I + (size_t)t * T * K + c;
-  double acc = 0.0;
-  for (int i = 0; i < T; ++i) acc = __dadd_rn(acc, (double)__ldg(p + (size_t)i * K));
-  Vc[(size_t)t * K + c] = acc;
+  U128 acc{0ull, 0ull};
+  unsigned char tiny = 0;
+  for (int i = 0; i < T; ++i) {
+    uint32_t m;
+    int e;
+    split_f32(__ldg(p + (size_t)i * K), m, e);
+    if (!m) continue;
+    if (e >= lsb) add_shifted(acc, m, e - lsb);
+    else tiny = 1;
+  }
+  colsum[(size_t)t * K + c] = acc;
+  coltiny[(size_t)t * K + c] = tiny;
 }
 
 // ------------------------------------------------------------------ rank sort
@@ -77,11 +156,13 @@ __global__ void __launch_bounds__(1024) rank_sort_kernel(const double* __restric
 }
 
 cudaError_t launch_vector_rank(const float* I, const int32_t* perm, int M, int K, int T,
-                               double* V, int32_t* rank, cudaStream_t s) {
+                               double* V, int32_t* rank, int* tile_pmax, cudaStream_t s) {
   const int nt = M / T;
+  cudaError_t e = cudaMemsetAsync(tile_pmax, 0, (size_t)nt * sizeof(int), s);
+  if (e != cudaSuccess) return e;
   dim3 g1((K + 255) / 256, nt);
-  vector_score_kernel<<<g1, 256, 0, s>>>(I, K, T, V);
-  cudaError_t e = cudaGetLastError();
+  vector_score_kernel<<<g1, 256, 0, s>>>(I, K, T, V, tile_pmax);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   int Kp = 1;
   while (Kp < K) Kp <<= 1;
@@ -95,23 +176,6 @@ cudaError_t launch_vector_rank(const float* I, const int32_t* perm, int M, int K
   }
   rank_sort_kernel<<<nt, 1024, smem, s>>>(V, perm, K, Kp, rank);
   return cudaGetLastError();
-}
-
-// ------------------------------------------------------------------ exact sums
-// Exact sum of non-negative finite fp32 values: every value is m * 2^(b - 150) with an
-// integer mantissa m < 2^24 and b = max(biased exponent, 1); bucket[b] accumulates m in
-// 64-bit integers (at most 2^24 values per sum keeps every bucket below 2^48).
-// Called by all 32 lanes of a warp together (v = 0 contributes nothing).
-__device__ __forceinline__ void bucket_add(unsigned long long* buckets, float v) {
-  const uint32_t u = __float_as_uint(v);
-  const uint32_t e = (u >> 23) & 0xFF;
-  const uint32_t m = (u & 0x7FFFFF) | (e ? 0x800000u : 0u);
-  const uint32_t b = e ? e : 1u;
-  // lanes with the same bucket are summed first (mantissas < 2^24, 32 lanes < 2^29)
-  const unsigned peers = __match_any_sync(0xffffffffu, b);
-  const unsigned sum = __reduce_add_sync(peers, m);
-  if ((__ffs(peers) - 1) == (int)(threadIdx.x & 31) && sum != 0u)
-    atomicAdd(buckets + b, (unsigned long long)sum);
 }
 
 // Adds v * 2^sh (v < 2^64) into the little-endian multi-limb integer z[0..5].
@@ -134,12 +198,14 @@ __device__ __forceinline__ void big_add_shifted(unsigned long long* z, unsigned 
   }
 }
 
-// Z = sum_b bucket[b] * 2^(b-1) (bucket[b] < 2^48, so Z < 2^303), value = Z * 2^-149,
+// value = Z * 2^-149 with Z = main * 2^lsb + sum_p bucket[p] * 2^p (a 384-bit integer),
 // rounded to the nearest fp64, ties to even.
-__device__ double buckets_to_double(const unsigned long long* bucket) {
+__device__ double exact_to_double(U128 main, int lsb, const unsigned long long* bucket) {
   unsigned long long z[6] = {0, 0, 0, 0, 0, 0};
-  for (int b = 1; b < 256; ++b)
-    if (bucket[b]) big_add_shifted(z, bucket[b], b - 1);
+  if (main.lo) big_add_shifted(z, main.lo, lsb);
+  if (main.hi) big_add_shifted(z, main.hi, lsb + 64);
+  for (int p = 0; p < 254; ++p)
+    if (bucket[p]) big_add_shifted(z, bucket[p], p);
   int top = -1;
   for (int l = 5; l >= 0 && top < 0; --l)
     if (z[l]) top = l * 64 + 63 - __clzll((long long)z[l]);
@@ -172,103 +238,111 @@ struct CandidateList {
 };
 
 // blockIdx.x = candidate m, blockIdx.y = tile.  512 threads.
-// Shared memory: 16 warps x 256 buckets (32 KB) + group members (K int16).
-__global__ void __launch_bounds__(512) candidate_kernel(const float* __restrict__ I,
-                                                        const int32_t* __restrict__ perm,
-                                                        const int32_t* __restrict__ rank, int K,
-                                                        int T, CandidateList cl,
-                                                        double* __restrict__ R, int ncand) {
+// R(m) = sum of the column sums of the dense vectors + sum over the 2:4 groups of the
+// top-2 of every row, all exact (128-bit per thread at the tile's scale, exponent buckets
+// for values below it), rounded once to fp64.
+__global__ void __launch_bounds__(512) candidate_kernel(
+    const float* __restrict__ I, const int32_t* __restrict__ perm, const int32_t* __restrict__ rank,
+    const int* __restrict__ tile_pmax, const U128* __restrict__ colsum,
+    const unsigned char* __restrict__ coltiny, int K, int T, CandidateList cl,
+    double* __restrict__ R, int ncand) {
   extern __shared__ __align__(16) unsigned char smem[];
-  unsigned long long* buckets = reinterpret_cast<unsigned long long*>(smem);  // [16][256]
-  unsigned short* member = reinterpret_cast<unsigned short*>(buckets + 16 * 256);  // [K]
+  unsigned long long* bucket = reinterpret_cast<unsigned long long*>(smem);  // [256]
+  unsigned short* member = reinterpret_cast<unsigned short*>(bucket + 256);   // [K]
   __shared__ int warp_tot[16];
+  __shared__ U128 warp_acc[16];
 
   const int m = blockIdx.x, t = blockIdx.y;
   const Candidate cand = cl.c[m];
   const int n4 = cand.n4, n24 = cand.n24;
   const int32_t* rk = rank + (size_t)t * K;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int lsb = tile_lsb(tile_pmax[t]);
+  const float* It = I + (size_t)t * T * K;
 
-  for (int i = threadIdx.x; i < 16 * 256; i += blockDim.x) buckets[i] = 0;
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) bucket[i] = 0;
+  U128 acc{0ull, 0ull};
 
-  // 2:4 members in ascending working position: block-wide prefix count over j.
+  // pass over the working positions: dense column sums, and the 2:4 members in
+  // ascending working position (block-wide prefix count)
   const int per = (K + blockDim.x - 1) / blockDim.x;
-  const int j0 = threadIdx.x * per;
+  const int j0 = threadIdx.x * per, j1 = min(K, j0 + per);
   int cnt = 0;
-  for (int j = j0; j < min(K, j0 + per); ++j) {
+  for (int j = j0; j < j1; ++j) {
     const int r = __ldg(rk + j);
     cnt += (r >= n4 && r < n4 + n24);
   }
-  // exclusive scan of cnt over the block
   int incl = cnt;
   for (int o = 1; o < 32; o <<= 1) {
     const int v = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += v;
   }
   if (lane == 31) warp_tot[warp] = incl;
-  __syncthreads();
-  int wbase = 0;
-  for (int w = 0; w < warp; ++w) wbase += warp_tot[w];
-  int pos = wbase + incl - cnt;
-  for (int j = j0; j < min(K, j0 + per); ++j) {
+  __syncthreads();  // also publishes the cleared buckets
+  int pos = incl - cnt;
+  for (int w = 0; w < warp; ++w) pos += warp_tot[w];
+  for (int j = j0; j < j1; ++j) {
     const int r = __ldg(rk + j);
-    if (r >= n4 && r < n4 + n24) member[pos++] = (unsigned short)j;
+    if (r < n4) {
+      const int c = ptx::perm_at(perm, j, K);
+      add128(acc, colsum[(size_t)t * K + c]);
+      if (coltiny[(size_t)t * K + c]) {  // values below the tile's scale: exact buckets
+        for (int i = 0; i < T; ++i) {
+          uint32_t mm;
+          int e;
+          split_f32(__ldg(It + (size_t)i * K + c), mm, e);
+          if (mm && e < lsb) atomicAdd(bucket + e, (unsigned long long)mm);
+        }
+      }
+    } else if (r < n4 + n24) {
+      member[pos++] = (unsigned short)j;
+    }
   }
   __syncthreads();
 
-  unsigned long long* my = buckets + warp * 256;
-  const float* It = I + (size_t)t * T * K;
-  // dense vectors: every element kept.  Loops advance whole warps together so every
-  // lane takes part in the warp-aggregated bucket adds.
-  const int total_d = T * K;
-  for (int base = threadIdx.x - lane; base < total_d; base += blockDim.x) {
-    const int q = base + lane;
-    float v = 0.0f;
-    if (q < total_d) {
-      const int i = q / K, j = q - (q / K) * K;
-      if (__ldg(rk + j) < n4) {
-        const int c = ptx::perm_at(perm, j, K);
-        v = __ldg(It + (size_t)i * K + c);
-      }
-    }
-    bucket_add(my, v);
-  }
   // 2:4 groups: top-2 of 4 per row (lower position wins ties)
   const int ng = n24 / 4;
   const int total_s = T * ng;
-  for (int base = threadIdx.x - lane; base < total_s; base += blockDim.x) {
-    const int q = base + lane;
-    float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    bool keep[4] = {false, false, false, false};
-    if (q < total_s) {
-      const int i = q / ng, g = q - (q / ng) * ng;
+  for (int q = threadIdx.x; q < total_s; q += blockDim.x) {
+    const int i = q / ng, g = q - (q / ng) * ng;
+    float v[4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        int j = member[4 * g + k];
-        j = j < K ? j : 0;
-        const int c = ptx::perm_at(perm, j, K);
-        v[k] = __ldg(It + (size_t)i * K + c);
-      }
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        int beats = 0;
-#pragma unroll
-        for (int l = 0; l < 4; ++l) beats += (v[l] > v[k]) || (v[l] == v[k] && l < k);
-        keep[k] = beats < 2;
-      }
+    for (int k = 0; k < 4; ++k) {
+      int j = member[4 * g + k];
+      j = j < K ? j : 0;
+      v[k] = __ldg(It + (size_t)i * K + ptx::perm_at(perm, j, K));
     }
 #pragma unroll
-    for (int k = 0; k < 4; ++k) bucket_add(my, keep[k] ? v[k] : 0.0f);
+    for (int k = 0; k < 4; ++k) {
+      int beats = 0;
+#pragma unroll
+      for (int l = 0; l < 4; ++l) beats += (v[l] > v[k]) || (v[l] == v[k] && l < k);
+      if (beats < 2) {
+        uint32_t mm;
+        int e;
+        split_f32(v[k], mm, e);
+        if (mm) {
+          if (e >= lsb) add_shifted(acc, mm, e - lsb);
+          else atomicAdd(bucket + e, (unsigned long long)mm);
+        }
+      }
+    }
   }
-  __syncthreads();
-  // fold the 16 warp copies into copy 0
-  for (int b = threadIdx.x; b < 256; b += blockDim.x) {
-    unsigned long long s = 0;
-    for (int w = 0; w < 16; ++w) s += buckets[w * 256 + b];
-    buckets[b] = s;
+
+  // block reduction of the 128-bit partial sums (integer adds: order-independent)
+  for (int o = 16; o > 0; o >>= 1) {
+    U128 other;
+    other.lo = __shfl_xor_sync(0xffffffffu, acc.lo, o);
+    other.hi = __shfl_xor_sync(0xffffffffu, acc.hi, o);
+    add128(acc, other);
   }
+  if (lane == 0) warp_acc[warp] = acc;
   __syncthreads();
-  if (threadIdx.x == 0) R[(size_t)t * ncand + m] = buckets_to_double(buckets);
+  if (threadIdx.x == 0) {
+    U128 tot{0ull, 0ull};
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) add128(tot, warp_acc[w]);
+    R[(size_t)t * ncand + m] = exact_to_double(tot, lsb, bucket);
+  }
 }
 
 __global__ void select_kernel(const double* __restrict__ R, int nt, int ncand, CandidateList cl,
@@ -293,37 +367,48 @@ __global__ void select_kernel(const double* __restrict__ R, int nt, int ncand, C
 size_t search_workspace_bytes(int M, int K, int T, int ncand) {
   const int nt = M / T;
   Carve c{nullptr, 0};
-  c.take<double>((size_t)nt * K);      // V
-  c.take<int32_t>((size_t)nt * K);     // rank (when the caller passes none)
-  c.take<double>((size_t)nt * ncand);  // R
+  c.take<double>((size_t)nt * K);         // V
+  c.take<int32_t>((size_t)nt * K);        // rank (when the caller passes none)
+  c.take<double>((size_t)nt * ncand);     // R
+  c.take<int>((size_t)nt);                // tile max exponent
+  c.take<U128>((size_t)nt * K);           // exact column sums
+  c.take<unsigned char>((size_t)nt * K);  // column has values below the tile scale
   return (c.off + 255) & ~size_t(255);
 }
 
 cudaError_t launch_boundary_search(const float* I, const int32_t* perm, int M, int K, int T,
                                    double t_s, double alpha, const Candidate* cands, int ncand,
                                    int32_t* counts_out, double* vs_out, int32_t* rank_out,
-                                   void* ws, int* status, cudaStream_t s) {
+                                   double* retained_out, void* ws, int* status, cudaStream_t s) {
   (void)status;
   const int nt = M / T;
   Carve c{static_cast<char*>(ws), 0};
   double* V = c.take<double>((size_t)nt * K);
   int32_t* rank_ws = c.take<int32_t>((size_t)nt * K);
-  double* R = c.take<double>((size_t)nt * ncand);
+  double* R_ws = c.take<double>((size_t)nt * ncand);
+  double* R = retained_out ? retained_out : R_ws;
+  int* pmax = c.take<int>((size_t)nt);
+  U128* colsum = c.take<U128>((size_t)nt * K);
+  unsigned char* coltiny = c.take<unsigned char>((size_t)nt * K);
   int32_t* rank = rank_out ? rank_out : rank_ws;
-  cudaError_t e = launch_vector_rank(I, perm, M, K, T, V, rank, s);
+  cudaError_t e = launch_vector_rank(I, perm, M, K, T, V, rank, pmax, s);
+  if (e != cudaSuccess) return e;
+  dim3 gc((K + 255) / 256, nt);
+  column_sum_kernel<<<gc, 256, 0, s>>>(I, K, T, pmax, colsum, coltiny);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CandidateList cl;
   for (int i = 0; i < kMaxCandidates; ++i) cl.c[i] = i < ncand ? cands[i] : Candidate{0, 0, 0};
-  const size_t smem = 16 * 256 * sizeof(unsigned long long) + (size_t)K * sizeof(unsigned short);
+  const size_t smem = 256 * sizeof(unsigned long long) + (size_t)K * sizeof(unsigned short);
   static bool attr_set = false;
   if (!attr_set) {
     e = cudaFuncSetAttribute(candidate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(16 * 256 * sizeof(unsigned long long) + kMaxK * 2));
+                             (int)(256 * sizeof(unsigned long long) + kMaxK * 2));
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   dim3 g(ncand, nt);
-  candidate_kernel<<<g, 512, smem, s>>>(I, perm, rank, K, T, cl, R, ncand);
+  candidate_kernel<<<g, 512, smem, s>>>(I, perm, rank, pmax, colsum, coltiny, K, T, cl, R, ncand);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   select_kernel<<<(nt + 127) / 128, 128, 0, s>>>(R, nt, ncand, cl, t_s, alpha, counts_out, vs_out);

@@ -4,18 +4,21 @@
 // The pages run two CUDA streams (mma and mma.sp) merged by atomicAdd.  Here one CTA per
 // (tile, N-block) runs both kinds of K-block into ONE tensor-memory accumulator:
 //
-//   warp 0  producer : per K-block, one bulk copy of the pre-swizzled 16 KB A block (and,
-//                      for a 2:4 block, its 2 KB metadata), plus TMA gather4 loads of the
-//                      block's X rows selected by the index (4 rows per instruction,
-//                      swizzled for an MN-major B operand)
-//   warp 1  MMA      : one thread; 2:4 block -> tcgen05.cp of the metadata into tensor
-//                      memory, then 4 x tcgen05.mma.sp (K = 32 each); dense block ->
-//                      4 x tcgen05.mma (K = 16 each); tcgen05.commit frees the stage
-//   warps 2-5 epilogue: tcgen05.ld of the 128 x BN fp32 accumulator, stores to Y
+//   warps 0-3 producers: per K-block, thread 0 bulk-copies the pre-swizzled 16 KB A block
+//                 (and, for a 2:4 block, its 2 KB metadata); the X rows the block's index
+//                 selects are copied by all 128 threads with 16-byte cp.async into the
+//                 swizzled MN-major B tile (coalesced 2*BN-byte row segments), or, when the
+//                 index is one contiguous run, by thread 0 as 2-D tiled TMA boxes.  Every
+//                 producer thread arrives on the stage's full barrier when its copies land.
+//   warp 4       MMA: one thread; 2:4 block -> tcgen05.cp of the metadata into tensor
+//                 memory, then 4 x tcgen05.mma.sp (K = 32 each); dense block -> 4 x
+//                 tcgen05.mma (K = 16 each); tcgen05.commit frees the stage.  Then the warp
+//                 joins the epilogue.
+//   warps 4-7    epilogue: tcgen05.ld of the 128 x BN fp32 accumulator, stores to Y.
 //
-// Shared memory holds STAGES stages of [A 16 KB | B 128 x BN bf16 | E 2 KB] behind full /
-// empty mbarriers.  Every wait is bounded (2 s), after which the CTA records
-// HINM_ERR_DEVICE_TIMEOUT, drains what it issued and exits.
+// Shared memory holds STAGES stages of [A 16 KB | B 128 x BN bf16 | E 2 KB].  Every wait is
+// bounded (2 s), after which the CTA records HINM_ERR_DEVICE_TIMEOUT, drains what it
+// issued, frees tensor memory and returns.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -31,7 +34,9 @@ template <int BN>
 struct SpmmCfg {
   static constexpr int kAtom = BN >= 64 ? 64 : BN;  // B swizzle atom width (elements)
   static constexpr int kAtomBytes = kAtom * 2;      // 128, 64 or 32 bytes
-  static constexpr int kNumAtoms = BN / kAtom;
+  static constexpr int kSwzBits = kAtomBytes == 128 ? 3 : (kAtomBytes == 64 ? 2 : 1);
+  static constexpr int kChunksPerAtom = kAtomBytes / 16;
+  static constexpr int kChunksPerRow = BN / 8;
   static constexpr int kABytes = kBlockBytes;
   static constexpr int kBBytes = 128 * BN * 2;  // 128 K-rows (a 2:4 block); dense uses 64
   static constexpr int kEBytes = 2048;
@@ -44,6 +49,8 @@ struct SpmmCfg {
   static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                    : kTmemNeed <= 256 ? 256 : 512;
   static constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024 /*align*/ + 256;
+  static constexpr int kProducers = 128;
+  static constexpr int kThreads = 256;
   static_assert(BN == 16 || BN == 32 || BN % 64 == 0, "BN");
   static_assert(kStages >= 2, "stages");
   static_assert(kTmemNeed <= 512, "tmem");
@@ -56,13 +63,27 @@ struct SpmmArgs {
   const uint32_t* meta;
   const int32_t* idx_dense;
   const int32_t* idx_sparse;
+  const int32_t* run_dense;
+  const int32_t* run_sparse;
+  const uint16_t* X;
   float* Y;
   int N, T;
   int* status;
 };
 
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 template <int BN>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(256, 1)
     spmm_kernel(const __grid_constant__ CUtensorMap tmX, const SpmmArgs a) {
   using C = SpmmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -87,7 +108,7 @@ __global__ void __launch_bounds__(192, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      ptx::mbar_init(full_bar(s), 1);
+      ptx::mbar_init(full_bar(s), 1 + C::kProducers);  // expect_tx arrival + one per producer
       ptx::mbar_init(empty_bar(s), 1);
     }
     ptx::mbar_init(acc_bar, 1);
@@ -95,7 +116,7 @@ __global__ void __launch_bounds__(192, 1)
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == 4) {
     ptx::tmem_alloc(ptx::smem_u32(tmem_slot), C::kTmemCols);
     ptx::tmem_relinquish();
   }
@@ -104,8 +125,9 @@ __global__ void __launch_bounds__(192, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp < 4) {
+    // ------------------------------------------------------------ producers
+    const int ptid = threadIdx.x;
     int issued = 0;
     for (int kb = 0; kb < nblk; ++kb) {
       const int s = kb % C::kStages;
@@ -113,84 +135,102 @@ __global__ void __launch_bounds__(192, 1)
       if (!ptx::mbar_wait(empty_bar(s), ph ^ 1, a.status, abort_flag)) break;
       const bool sparse = kb >= nd;
       const int rows = sparse ? kSparseBK : kDenseBK;
-      uint8_t* st = smem + s * C::kStageBytes;
-      const uint32_t A_s = ptx::smem_u32(st);
+      const uint32_t A_s = ptx::smem_u32(smem + s * C::kStageBytes);
       const uint32_t B_s = A_s + C::kABytes;
       const uint32_t E_s = B_s + C::kBBytes;
       const size_t blk = sparse ? (size_t)(s0 + kb - nd) : (size_t)(d0 + kb);
-      if (lane == 0) {
-        const uint32_t bytes =
-            C::kABytes + (sparse ? C::kEBytes : 0) + (uint32_t)rows * BN * 2u;
+      const int run = __ldg(sparse ? a.run_sparse + blk : a.run_dense + blk);
+      if (ptid == 0) {
+        const uint32_t bytes = C::kABytes + (sparse ? C::kEBytes : 0) +
+                               (run >= 0 ? (uint32_t)rows * BN * 2u : 0u);
         ptx::mbar_arrive_expect_tx(full_bar(s), bytes);
         ptx::bulk_g2s(A_s, (sparse ? a.vals_sparse : a.vals_dense) + blk * 8192, C::kABytes,
                       full_bar(s));
         if (sparse) ptx::bulk_g2s(E_s, a.meta + blk * kMetaWords, C::kEBytes, full_bar(s));
+        if (run >= 0) {
+          // one ascending run of X rows: 2-D tiled boxes of 64 rows x kAtom columns
+#pragma unroll 1
+          for (int at = 0; at < BN / C::kAtom; ++at)
+#pragma unroll 1
+            for (int h = 0; h < rows / 64; ++h)
+              ptx::tma_load_2d(B_s + at * (128 * C::kAtomBytes) + h * 64 * C::kAtomBytes, &tmX,
+                               n0 + at * C::kAtom, run + h * 64, full_bar(s));
+        }
       }
-      __syncwarp();
-      const int* idx = sparse ? a.idx_sparse + blk * kSparseBK : a.idx_dense + blk * kDenseBK;
-      const int quads = rows / 4;
-      for (int q = lane; q < quads * C::kNumAtoms; q += 32) {
-        const int rq = q % quads, at = q / quads;
-        const int4 r = __ldg(reinterpret_cast<const int4*>(idx) + rq);
-        ptx::tma_gather4(B_s + at * (128 * C::kAtomBytes) + rq * 4 * C::kAtomBytes, &tmX,
-                         n0 + at * C::kAtom, r.x, r.y, r.z, r.w, full_bar(s));
+      if (run < 0) {
+        const int* idx = sparse ? a.idx_sparse + blk * kSparseBK : a.idx_dense + blk * kDenseBK;
+        const int chunks = rows * C::kChunksPerRow;
+        for (int q = ptid; q < chunks; q += C::kProducers) {
+          const int r = q / C::kChunksPerRow, cc = q - r * C::kChunksPerRow;
+          const int at = cc / C::kChunksPerAtom, c = cc - at * C::kChunksPerAtom;
+          const int col = n0 + cc * 8;
+          const int xr = __ldg(idx + r);
+          const bool ok = col < a.N;
+          const uint16_t* src = ok ? a.X + (size_t)xr * a.N + col : a.X;
+          uint32_t off = at * (128 * C::kAtomBytes) + r * C::kAtomBytes + c * 16;
+          off ^= ((off >> 7) & ((1u << C::kSwzBits) - 1u)) << 4;  // shared-memory swizzle
+          cp_async_16(B_s + off, src, ok ? 16u : 0u);
+        }
       }
+      cp_async_arrive_noinc(full_bar(s));
       ++issued;
     }
-    __syncwarp();
-    if (*abort_flag && lane == 0) {
-      // wait (bounded) for the copies this warp issued and nobody consumed
+    cp_async_wait_all();
+    if (*abort_flag && ptid == 0) {
+      // wait (bounded) for the bulk / tensor copies issued and never consumed
       for (int kb = (issued > C::kStages ? issued - C::kStages : 0); kb < issued; ++kb)
         ptx::mbar_wait(full_bar(kb % C::kStages), (kb / C::kStages) & 1, a.status, nullptr);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc_d = ptx::idesc_bf16(BN, 1, 0);
-      const uint32_t idesc_s = ptx::idesc_bf16(BN, 1, 1);
-      bool any = false;
-      for (int kb = 0; kb < nblk; ++kb) {
-        const int s = kb % C::kStages;
-        const uint32_t ph = (kb / C::kStages) & 1;
-        if (!ptx::mbar_wait(full_bar(s), ph, a.status, abort_flag)) break;
-        ptx::tc_fence_after();
-        const bool sparse = kb >= nd;
-        const uint32_t A_s = ptx::smem_u32(smem + s * C::kStageBytes);
-        const uint32_t B_s = A_s + C::kABytes;
-        const uint32_t E_s = B_s + C::kBBytes;
-        if (sparse) {
-          const uint32_t e_col = tmem + BN + 4 * s;
-          // 128 lanes x 16 bytes, rows 16 B apart: core matrices of 8 rows, 128 B apart
-          ptx::tc_cp_128x128b(e_col, ptx::smem_desc(E_s, 2048, 128, 0));
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t ad = ptx::smem_desc(A_s + 32 * k, 16, 1024, 2);
-            const uint64_t bd = ptx::smem_desc(B_s + 32 * k * C::kAtomBytes, 128 * C::kAtomBytes,
-                                               8 * C::kAtomBytes, C::kBLayout);
-            const uint32_t e = e_col + k;
-            ptx::mma_sp_bf16(tmem, ad, bd, e & ~1u, idesc_s | (e & 1u), any ? 1u : 0u);
-            any = true;
-          }
-        } else {
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t ad = ptx::smem_desc(A_s + 32 * k, 16, 1024, 2);
-            const uint64_t bd = ptx::smem_desc(B_s + 16 * k * C::kAtomBytes, 128 * C::kAtomBytes,
-                                               8 * C::kAtomBytes, C::kBLayout);
-            ptx::mma_bf16(tmem, ad, bd, idesc_d, any ? 1u : 0u);
-            any = true;
-          }
-        }
-        ptx::tc_commit(empty_bar(s));
-      }
-      if (nblk > 0) ptx::tc_commit(acc_bar);
-      // every tcgen05 operation issued above has completed once drain_bar flips
-      ptx::tc_commit(drain_bar);
-      ptx::mbar_wait(drain_bar, 0, a.status, nullptr);
-    }
-    __syncwarp();
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2..5)
+    if (warp == 4) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        const uint32_t idesc_d = ptx::idesc_bf16(BN, 1, 0);
+        const uint32_t idesc_s = ptx::idesc_bf16(BN, 1, 1);
+        bool any = false;
+        for (int kb = 0; kb < nblk; ++kb) {
+          const int s = kb % C::kStages;
+          const uint32_t ph = (kb / C::kStages) & 1;
+          if (!ptx::mbar_wait(full_bar(s), ph, a.status, abort_flag)) break;
+          ptx::fence_proxy_async_smem();  // cp.async (generic proxy) -> tensor-core reads
+          ptx::tc_fence_after();
+          const bool sparse = kb >= nd;
+          const uint32_t A_s = ptx::smem_u32(smem + s * C::kStageBytes);
+          const uint32_t B_s = A_s + C::kABytes;
+          const uint32_t E_s = B_s + C::kBBytes;
+          if (sparse) {
+            const uint32_t e_col = tmem + BN + 4 * s;
+            // 128 lanes x 16 bytes, rows 16 B apart: core matrices of 8 rows, 128 B apart
+            ptx::tc_cp_128x128b(e_col, ptx::smem_desc(E_s, 2048, 128, 0));
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint64_t ad = ptx::smem_desc(A_s + 32 * k, 16, 1024, 2);
+              const uint64_t bd = ptx::smem_desc(B_s + 32 * k * C::kAtomBytes, 128 * C::kAtomBytes,
+                                                 8 * C::kAtomBytes, C::kBLayout);
+              const uint32_t e = e_col + k;
+              ptx::mma_sp_bf16(tmem, ad, bd, e & ~1u, idesc_s | (e & 1u), any ? 1u : 0u);
+              any = true;
+            }
+          } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint64_t ad = ptx::smem_desc(A_s + 32 * k, 16, 1024, 2);
+              const uint64_t bd = ptx::smem_desc(B_s + 16 * k * C::kAtomBytes, 128 * C::kAtomBytes,
+                                                 8 * C::kAtomBytes, C::kBLayout);
+              ptx::mma_bf16(tmem, ad, bd, idesc_d, any ? 1u : 0u);
+              any = true;
+            }
+          }
+          ptx::tc_commit(empty_bar(s));
+        }
+        if (nblk > 0) ptx::tc_commit(acc_bar);
+        // every tcgen05 operation issued above has completed once drain_bar flips
+        ptx::tc_commit(drain_bar);
+        ptx::mbar_wait(drain_bar, 0, a.status, nullptr);
+      }
+      __syncwarp();
+    }
+    // ------------------------------------------------------------ epilogue (warps 4..7)
     const int q = warp & 3;  // tensor-memory lane quadrant this warp may access
     const int row = q * 32 + lane;
     bool have = nblk > 0;
@@ -198,6 +238,7 @@ __global__ void __launch_bounds__(192, 1)
       have = ptx::mbar_wait(acc_bar, 0, a.status, abort_flag);
       ptx::tc_fence_after();
     }
+    have = __all_sync(0xffffffffu, have);
     const bool row_ok = row < a.T;
     float* yrow = a.Y + (size_t)(tile * a.T + row) * a.N;
     constexpr int kChunk = BN >= 32 ? 32 : 16;
@@ -233,7 +274,7 @@ __global__ void __launch_bounds__(192, 1)
   }
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 4) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::kTmemCols);
   }
@@ -256,14 +297,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// X (K rows x N bf16, row-major) as a 2-D tensor map whose box is one row of `atom`
-// elements, swizzled like the B operand (atom * 2 bytes per swizzle row).
+// X (K rows x N bf16, row-major) as a 2-D tensor map with a box of 64 rows x `atom`
+// columns, swizzled like the B operand (atom * 2 bytes per swizzle row).
 bool make_x_map(CUtensorMap* m, const uint16_t* X, int K, int N, int atom) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)K};
   cuuint64_t strides[1] = {(cuuint64_t)N * 2};
-  cuuint32_t box[2] = {(cuuint32_t)atom, 1};
+  cuuint32_t box[2] = {(cuuint32_t)atom, (cuuint32_t)(K < 64 ? K : 64)};
   cuuint32_t estr[2] = {1, 1};
   const CUtensorMapSwizzle sw = atom == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
                                 : atom == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
@@ -288,9 +329,10 @@ cudaError_t run(const hinm_layout& L, const uint16_t* X, int N, float* Y, int* s
   CUtensorMap map;
   if (!make_x_map(&map, X, L.K, N, C::kAtom)) return cudaErrorInvalidValue;
   SpmmArgs a{L.tile_info, L.vals_dense, L.vals_sparse, L.meta, L.idx_dense, L.idx_sparse,
-             Y,           N,            L.T,           status};
+             L.run_dense, L.run_sparse, X,      Y,           N,           L.T,
+             status};
   dim3 grid((N + BN - 1) / BN, L.num_tiles);
-  spmm_kernel<BN><<<grid, 192, C::kSmemBytes, s>>>(map, a);
+  spmm_kernel<BN><<<grid, C::kThreads, C::kSmemBytes, s>>>(map, a);
   return cudaGetLastError();
 }
 

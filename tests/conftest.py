@@ -15,3 +15,14 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def golden_dir():
     return os.path.join(ROOT, "tests", "golden")
+
+
+def build_library():
+    """Compile libhinm.so if a source is newer (loaded by path: importing the package
+    needs the library to exist)."""
+    import importlib.util
+    path = os.path.join(ROOT, "pruning_hinm_spmm_b200", "build_lib.py")
+    spec = importlib.util.spec_from_file_location("hinm_build_lib", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()

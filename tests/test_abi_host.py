@@ -15,8 +15,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def H():
-    from pruning_hinm_spmm_b200 import build_lib
-    build_lib.build()
+    from conftest import build_library
+    build_library()
     import pruning_hinm_spmm_b200 as H
     return H
 
@@ -97,17 +97,20 @@ def test_validation_rejects_before_launch(H):
     assert b"workspace" in lib.hinm_last_error()
     # workspace too small for the search
     cnt = ctypes.c_void_p(fake)
-    assert lib.hinm_boundary_search(fake, None, 256, 256, 64, 0.5, 1 / 32, fake, fake, None, fake, 16,
-                                    None) == H.HINM_ERR_WORKSPACE
+    assert lib.hinm_boundary_search(fake, None, 256, 256, 64, 0.5, 1 / 32, fake, fake, None, None,
+                                    fake, 16, None) == H.HINM_ERR_WORKSPACE
     # t_s * K not whole
-    assert lib.hinm_boundary_search(fake, None, 256, 100, 64, 0.333, 1 / 32, fake, fake, None, fake,
-                                    1 << 30, None) == H.HINM_ERR_INVALID_ARG
+    assert lib.hinm_boundary_search(fake, None, 256, 100, 64, 0.333, 1 / 32, fake, fake, None, None,
+                                    fake, 1 << 30, None) == H.HINM_ERR_INVALID_ARG
+    n = ctypes.c_int32(0)
+    assert lib.hinm_search_num_candidates(4096, 0.75, 1 / 32, ctypes.byref(n)) == H.HINM_OK
+    assert n.value == len(O.search_candidates(4096, 0.75, 1 / 32))
     # layout checks
-    L = H.hinm_layout(H.HINM_LAYOUT_VERSION + 1, 256, 256, 64, 4, 1, 1, fake, fake, fake, fake, fake, fake)
+    L = H.hinm_layout(H.HINM_LAYOUT_VERSION + 1, 256, 256, 64, 4, 1, 1, fake, fake, fake, fake, fake, fake, fake, fake)
     assert lib.hinm_spmm(ctypes.byref(L), fake, 16, fake, None) == H.HINM_ERR_INVALID_ARG
-    L = H.hinm_layout(H.HINM_LAYOUT_VERSION, 256, 256, 64, 3, 1, 1, fake, fake, fake, fake, fake, fake)
+    L = H.hinm_layout(H.HINM_LAYOUT_VERSION, 256, 256, 64, 3, 1, 1, fake, fake, fake, fake, fake, fake, fake, fake)
     assert lib.hinm_spmm(ctypes.byref(L), fake, 16, fake, None) == H.HINM_ERR_SHAPE
-    L = H.hinm_layout(H.HINM_LAYOUT_VERSION, 256, 256, 64, 4, 1, 1, fake, fake, fake, fake, fake, fake)
+    L = H.hinm_layout(H.HINM_LAYOUT_VERSION, 256, 256, 64, 4, 1, 1, fake, fake, fake, fake, fake, fake, fake, fake)
     assert lib.hinm_spmm(ctypes.byref(L), fake, 20, fake, None) == H.HINM_ERR_SHAPE
     assert lib.hinm_spmm(ctypes.byref(L), fake + 8, 16, fake, None) == H.HINM_ERR_ALIGNMENT
     # compress size rejects inconsistent counts

@@ -46,6 +46,8 @@ def layout_equal(L_gpu, L_ref, tiles=None):
     me = L_gpu.meta.cpu().numpy().view(np.uint32)
     idd = L_gpu.idx_dense.cpu().numpy()
     ids = L_gpu.idx_sparse.cpu().numpy()
+    rd = L_gpu.run_dense.cpu().numpy()
+    rs = L_gpu.run_sparse.cpu().numpy()
     for t in (range(info.shape[0]) if tiles is None else tiles):
         nd, ns, d0, s0 = info[t]
         nd_r, ns_r, d0_r, s0_r = L_ref.tile_info[t]
@@ -55,6 +57,8 @@ def layout_equal(L_gpu, L_ref, tiles=None):
         np.testing.assert_array_equal(me[s0:s0 + ns], L_ref.meta[s0_r:s0_r + ns])
         np.testing.assert_array_equal(idd[d0:d0 + nd], L_ref.idx_dense[d0_r:d0_r + nd])
         np.testing.assert_array_equal(ids[s0:s0 + ns], L_ref.idx_sparse[s0_r:s0_r + ns])
+        np.testing.assert_array_equal(rd[d0:d0 + nd], L_ref.run_dense[d0_r:d0_r + nd])
+        np.testing.assert_array_equal(rs[s0:s0 + ns], L_ref.run_sparse[s0_r:s0_r + ns])
 
 
 def check_y(y_gpu, y_ref, bound, rows=None):
@@ -71,7 +75,9 @@ def run_path(H, w, v_s=None, N=None):
     W, X = dev_bf16(w.W_bits), dev_bf16(w.X_bits)
     perm = dev_i32(w.perm)
     I = H.hinm_importance(W, X)
-    counts, vs, rank = H.hinm_boundary_search(I, perm, T, w.t_s, w.alpha)
+    nc = H.hinm_search_num_candidates(K, w.t_s, w.alpha)
+    R = torch.empty((M // T, nc), dtype=torch.float64, device="cuda")
+    counts, vs, rank = H.hinm_boundary_search(I, perm, T, w.t_s, w.alpha, retained_out=R)
     if v_s is not None:
         c = np.array(H.hinm_counts_from_vs(K, w.t_s, v_s), dtype=np.int32)
         counts_used = dev_i32(np.tile(c, (M // T, 1)))
@@ -84,6 +90,7 @@ def run_path(H, w, v_s=None, N=None):
     torch.cuda.synchronize()
     status_ok(H)
     return dict(I=I.cpu().numpy(), counts=counts.cpu().numpy(), vs=vs.cpu().numpy(),
+                R=R.cpu().numpy(),
                 rank=rank.cpu().numpy(), counts_used=counts_used.cpu().numpy(),
                 bitmask=bm.cpu().numpy().view(np.uint32), region=region.cpu().numpy(), layout=L,
                 Y=Y.cpu().numpy())
@@ -119,6 +126,7 @@ def test_path_matches_oracle(H, name, make, v_s):
     np.testing.assert_array_equal(g["counts"], sr.counts)
     np.testing.assert_array_equal(g["vs"], sr.v_s)
     np.testing.assert_array_equal(g["rank"], sr.rank)
+    np.testing.assert_array_equal(g["R"], np.array(sr.R))  # exact sums, rounded once
     counts = g["counts_used"]
     # a4 mask
     bm_ref, reg_ref = O.mask(I_ref, w.perm, w.T, counts)

@@ -395,6 +395,21 @@ def test_compress_round_trip(T, K, t_s, v_s, perm):
         assert (L.idx_dense[d0:d0 + nd].ravel()[n4:] == 0).all()
         sp_idx = L.idx_sparse[s0:s0 + ns].ravel()[:n24]
         assert set(sp_idx.tolist()) == set(np.nonzero(region[t] == O.REGION_24)[0].tolist())
+    # contiguous-run flags: a block is flagged iff its indices are one ascending run
+    for idx, run in ((L.idx_dense, L.run_dense), (L.idx_sparse, L.run_sparse)):
+        for b in range(idx.shape[0]):
+            is_run = all(int(idx[b, v]) == int(idx[b, 0]) + v for v in range(idx.shape[1]))
+            assert run[b] == (idx[b, 0] if is_run else -1)
+
+
+def test_contiguous_runs_identity_pure24():
+    """Pure 2:4 with the identity order: every 2:4 block is one run of 128 channels."""
+    w = hi.custom(128, 256, 8, 128, seed=1, t_s=0.5, v_s=None)
+    I = O.importance(w.W_bits, w.X_bits)
+    counts = np.array([O.counts_from_vs(256, 0.5, 0.0)])
+    bm, region = O.mask(I, w.perm, 128, counts)
+    L = O.compress(w.W_bits, bm, region, w.perm, counts, 128)
+    np.testing.assert_array_equal(L.run_sparse, [0, 128])
 
 
 # ----------------------------------------------------------------------------- spmm reference
