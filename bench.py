@@ -31,6 +31,12 @@ sys.path.insert(0, ROOT)
 import hinm_inputs as hi  # noqa: E402
 
 METRIC = "HiNM SpMM TFLOP/s (eff.) and HBM GB/s, % of 2:4-sparse/HBM roofline"
+WORKLOADS = {  # name -> seeded generator (rank r draws seed r)
+    "pure24": lambda r: hi.pure24(seed=r),
+    "tiny": lambda r: hi.tiny_hinm(seed=r),
+    "up": lambda r: hi.hinm_up_proj(seed=r),
+    "decode": lambda r: hi.decode_down_proj(seed=r),
+}
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -212,6 +218,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="hinm", choices=["hinm", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="pure24", choices=sorted(WORKLOADS),
+                    help="synthetic workload (default: the pure 2:4 4096x4096x2048 benchmark)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -219,7 +227,7 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
-    w = hi.pure24(seed=rank)
+    w = WORKLOADS[args.workload](rank)
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -243,6 +251,13 @@ def main():
     stream = torch.cuda.current_stream()
 
     phases = ["importance", "search", "mask", "compress", "spmm"]
+    # Workloads specified with a fixed boundary v_s use its closed-form counts; the search
+    # still runs every step (its ranking feeds the mask).  Otherwise the search's counts.
+    fixed = None
+    if w.v_s is not None:
+        c = H.hinm_counts_from_vs(K, w.t_s, w.v_s)
+        fixed = torch.tensor([c] * (M // T), dtype=torch.int32, device=dev)
+    counts_used = fixed if fixed is not None else hp.counts
 
     def step(ev=None):
         if ev is not None:
@@ -253,10 +268,10 @@ def main():
         H.hinm_boundary_search(hp.I, perm, T, w.t_s, w.alpha, hp.counts, hp.vs, hp.rank, hp.ws)
         if ev is not None:
             ev[2].record(stream)
-        H.hinm_mask(hp.I, perm, hp.counts, T, hp.rank, hp.bitmask, hp.region, hp.ws)
+        H.hinm_mask(hp.I, perm, counts_used, T, hp.rank, hp.bitmask, hp.region, hp.ws)
         if ev is not None:
             ev[3].record(stream)
-        H.hinm_compress(W, hp.bitmask, hp.region, perm, hp.counts, T, hp.layout, hp.ws)
+        H.hinm_compress(W, hp.bitmask, hp.region, perm, counts_used, T, hp.layout, hp.ws)
         if ev is not None:
             ev[4].record(stream)
         H.hinm_spmm(hp.layout, X, hp.Y, None, hp.c_layout)
@@ -269,7 +284,7 @@ def main():
     st = H.hinm_device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} after warm-up")
-    counts = hp.counts.cpu().numpy()
+    counts = counts_used.cpu().numpy()
     vs = hp.vs.cpu().numpy()
     model = workload_model(M, K, N, T, counts)
 
@@ -310,7 +325,7 @@ def main():
         W_d.view(torch.int16).copy_(W_h, non_blocking=True)
         X_d.view(torch.int16).copy_(X_h, non_blocking=True)
         P_d.copy_(P_h, non_blocking=True)
-        hp.run(W_d, X_d, P_d)
+        hp.run(W_d, X_d, P_d, fixed_counts=fixed)
         Y_h.copy_(hp.Y, non_blocking=True)
 
     for _ in range(2):
@@ -375,7 +390,8 @@ def main():
         "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "M": M, "K": K, "N": N, "T": T, "t_s": w.t_s,
-                   "alpha": w.alpha, "v_s_found": sorted(set(np.round(vs, 6).tolist())),
+                   "alpha": w.alpha, "v_s_searched": sorted(set(np.round(vs, 6).tolist())),
+                   "v_s_used": w.v_s if w.v_s is not None else "searched",
                    "counts_tile0": counts[0].tolist(),
                    "l2": "flushed between timed steps (256 MB write)",
                    "step": "importance+search+mask+compress+spmm",

@@ -319,14 +319,14 @@ class HotPath:
         self.ws = _empty_bytes(ws, device)
 
     def run(self, W, X, perm, fixed_counts=None, stream=None):
+        """One pass of the path.  The search always runs (its ranking feeds the mask);
+        ``fixed_counts`` (int32 [M/T, 3]) replaces its counts when given."""
         hinm_importance(W, X, self.I, self.ws, stream)
-        if fixed_counts is None:
-            hinm_boundary_search(self.I, perm, self.T, self.t_s, self.alpha, self.counts, self.vs,
-                                 self.rank, self.ws, stream=stream)
-            counts, rank = self.counts, self.rank
-        else:
-            counts, rank = fixed_counts, None
-        hinm_mask(self.I, perm, counts, self.T, rank, self.bitmask, self.region, self.ws, stream)
+        hinm_boundary_search(self.I, perm, self.T, self.t_s, self.alpha, self.counts, self.vs,
+                             self.rank, self.ws, stream=stream)
+        counts = self.counts if fixed_counts is None else fixed_counts
+        hinm_mask(self.I, perm, counts, self.T, self.rank, self.bitmask, self.region, self.ws,
+                  stream)
         hinm_compress(W, self.bitmask, self.region, perm, counts, self.T, self.layout, self.ws,
                       stream)
         hinm_spmm(self.layout, X, self.Y, stream, self.c_layout)

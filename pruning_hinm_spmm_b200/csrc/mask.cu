@@ -3,12 +3,12 @@
 // rkmt.cn section 二: keep 2 of every 4 consecutive; geek-doc.cn section 五: the mask has
 // W's shape).
 //
-//   inverse_perm_kernel   pinv[perm[j]] = j
-//   classify_kernel       one CTA per tile: region of every working position, prefix
-//                         count of the 2:4 vectors -> pos24[t][j] and member[t][q]
-//   bitmask_kernel        one warp per 32-channel word of a row: dense -> 1, pruned -> 0,
-//                         2:4 -> top-2 of the group's 4 importances; __ballot_sync packs
-//                         the word, so every word is written once, coalesced.
+//   inverse_perm_kernel   pinv[perm[j]] = j (checks that perm is a permutation)
+//   classify_kernel       one CTA per tile: region of every working position and the
+//                         2:4 members in ascending working position (member[t][q])
+//   bitmask_kernel        one CTA per (tile, 16 rows): dense words by ballot over the
+//                         region, 2:4 groups top-2 of 4 per row, words assembled in shared
+//                         memory and written once, coalesced.
 #include <cuda_runtime.h>
 
 #include "hinm_internal.h"
@@ -61,7 +61,6 @@ __global__ void __launch_bounds__(1024) classify_kernel(const int32_t* __restric
                                                         const int32_t* __restrict__ perm,
                                                         const int32_t* __restrict__ counts, int K,
                                                         int8_t* __restrict__ region,
-                                                        int32_t* __restrict__ pos24,
                                                         int32_t* __restrict__ member,
                                                         int* status) {
   __shared__ int warp_tot[32];
@@ -83,7 +82,6 @@ __global__ void __launch_bounds__(1024) classify_kernel(const int32_t* __restric
   }
   int pos = block_exclusive_scan(cnt, warp_tot, &total);
   int8_t* reg = region + (size_t)t * K;
-  int32_t* p24 = pos24 + (size_t)t * K;
   int32_t* mem = member + (size_t)t * K;
   for (int j = j0; j < j1; ++j) {
     const int r = rk[j];
@@ -91,58 +89,76 @@ __global__ void __launch_bounds__(1024) classify_kernel(const int32_t* __restric
     int8_t cls = HINM_REGION_PRUNED;
     if (r < n4) {
       cls = HINM_REGION_DENSE;
-      p24[j] = -1;
     } else if (r < n4 + n24) {
       cls = HINM_REGION_24;
-      mem[pos] = j;
-      p24[j] = pos++;
-    } else {
-      p24[j] = -1;
+      mem[pos++] = j;
     }
     reg[c] = cls;
   }
 }
 
-__global__ void bitmask_kernel(const float* __restrict__ I, const int32_t* __restrict__ perm,
-                               const int32_t* __restrict__ pinv, const int8_t* __restrict__ region,
-                               const int32_t* __restrict__ pos24, const int32_t* __restrict__ member,
-                               int M, int K, int T, uint32_t* __restrict__ bitmask) {
+// One CTA per (tile, kMaskRows rows): the rows' mask words are assembled in shared memory.
+// Dense bits are the same in every row of the tile (one ballot per word over the region
+// array); each 2:4 group is handled by one thread for all the CTA's rows.
+constexpr int kMaskRows = 16;
+
+__global__ void __launch_bounds__(256) bitmask_kernel(
+    const float* __restrict__ I, const int32_t* __restrict__ perm,
+    const int8_t* __restrict__ region, const int32_t* __restrict__ counts,
+    const int32_t* __restrict__ member, int M, int K, int T, uint32_t* __restrict__ bitmask) {
+  extern __shared__ uint32_t words_s[];  // [kMaskRows][words]
   const int words = (K + 31) >> 5;
-  const int w = blockIdx.y * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int i = blockIdx.x;
-  const int lane = threadIdx.x & 31;
-  if (w >= words) return;
-  const int t = i / T;
-  const int c = w * 32 + lane;
-  bool keep = false;
-  if (c < K) {
-    const int8_t reg = __ldg(region + (size_t)t * K + c);
-    if (reg == HINM_REGION_DENSE) {
-      keep = true;
-    } else if (reg == HINM_REGION_24) {
-      const int j = __ldg(pinv + c);
-      const int p = ((unsigned)j < (unsigned)K) ? __ldg(pos24 + (size_t)t * K + j) : -1;
-      if (p >= 0) {
-        const int g = p >> 2, slot = p & 3;
-        const float* Ii = I + (size_t)i * K;
-        const int32_t* mem = member + (size_t)t * K + 4 * g;
-        const float v = __ldg(Ii + c);
-        int beats = 0;
+  const int t = blockIdx.y;
+  const int r0 = blockIdx.x * kMaskRows;  // first row of the chunk within the tile
+  const int rows = min(kMaskRows, T - r0);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int8_t* reg = region + (size_t)t * K;
+
+  // dense bits: warp per word, lane = bit
+  for (int w = warp; w < words; w += nwarps) {
+    const int c = w * 32 + lane;
+    const bool dense = c < K && __ldg(reg + c) == HINM_REGION_DENSE;
+    const uint32_t bits = __ballot_sync(0xffffffffu, dense);
+    if (lane < rows) words_s[lane * words + w] = bits;
+  }
+  __syncthreads();
+
+  int n24 = counts[3 * t + 1];
+  const int n0 = counts[3 * t], n4 = counts[3 * t + 2];
+  if (n0 < 0 || n24 < 0 || n4 < 0 || n0 + n24 + n4 != K || (n24 & 3)) n24 = 0;
+  const int ng = n24 / 4;
+  const int32_t* mem = member + (size_t)t * K;
+  const float* I0 = I + ((size_t)t * T + r0) * K;
+  for (int g = threadIdx.x; g < ng; g += blockDim.x) {
+    int c[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          if (k == slot) continue;
-          int jk = __ldg(mem + k);
-          jk = ((unsigned)jk < (unsigned)K) ? jk : 0;  // never index outside perm / I
-          const int ck = ptx::perm_at(perm, jk, K);
-          const float vk = __ldg(Ii + ck);
-          beats += (vk > v) || (vk == v && k < slot);
+    for (int k = 0; k < 4; ++k) {
+      int j = __ldg(mem + 4 * g + k);
+      j = ((unsigned)j < (unsigned)K) ? j : 0;  // never index outside perm / I
+      c[k] = ptx::perm_at(perm, j, K);
+    }
+    const float* row = I0;
+    for (int r = 0; r < rows; ++r, row += K) {
+      float v[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) v[k] = __ldg(row + c[k]);
+      // beats[k]: members ranked above k (greater value, or equal value at a lower position)
+      int beats[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int l = k + 1; l < 4; ++l) {
+          if (v[l] > v[k]) ++beats[k];
+          else ++beats[l];  // v[k] >= v[l]: k (lower position) ranks above l
         }
-        keep = beats < 2;
-      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (beats[k] < 2) atomicOr(words_s + r * words + (c[k] >> 5), 1u << (c[k] & 31));
     }
   }
-  const unsigned word = __ballot_sync(0xffffffffu, keep);
-  if (lane == 0) bitmask[(size_t)i * words + w] = word;
+  __syncthreads();
+  uint32_t* out = bitmask + ((size_t)t * T + r0) * words;
+  for (int x = threadIdx.x; x < rows * words; x += blockDim.x) out[x] = words_s[x];
 }
 
 size_t mask_workspace_bytes(int M, int K, int T) {
@@ -151,7 +167,6 @@ size_t mask_workspace_bytes(int M, int K, int T) {
   c.take<double>((size_t)nt * K);   // V (only when no rank is passed)
   c.take<int32_t>((size_t)nt * K);  // rank (only when no rank is passed)
   c.take<int32_t>((size_t)K);       // inverse permutation
-  c.take<int32_t>((size_t)nt * K);  // pos24
   c.take<int32_t>((size_t)nt * K);  // member
   c.take<int>((size_t)nt);          // tile max exponent (by-product of the ranking)
   return (c.off + 255) & ~size_t(255);
@@ -165,7 +180,6 @@ cudaError_t launch_mask(const float* I, const int32_t* perm, const int32_t* coun
   double* V = cv.take<double>((size_t)nt * K);
   int32_t* rank_ws = cv.take<int32_t>((size_t)nt * K);
   int32_t* pinv = cv.take<int32_t>((size_t)K);
-  int32_t* pos24 = cv.take<int32_t>((size_t)nt * K);
   int32_t* member = cv.take<int32_t>((size_t)nt * K);
   int* pmax = cv.take<int>((size_t)nt);
   cudaError_t e;
@@ -179,12 +193,20 @@ cudaError_t launch_mask(const float* I, const int32_t* perm, const int32_t* coun
   inverse_perm_kernel<<<(K + 255) / 256, 256, 0, s>>>(perm, K, pinv, status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  classify_kernel<<<nt, 1024, 0, s>>>(rank, perm, counts, K, region, pos24, member, status);
+  classify_kernel<<<nt, 1024, 0, s>>>(rank, perm, counts, K, region, member, status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int words = (K + 31) / 32;
-  dim3 g(M, (words + 7) / 8);
-  bitmask_kernel<<<g, 256, 0, s>>>(I, perm, pinv, region, pos24, member, M, K, T, bitmask);
+  const size_t smem = (size_t)kMaskRows * words * sizeof(uint32_t);
+  static bool attr_set = false;
+  if (!attr_set) {
+    e = cudaFuncSetAttribute(bitmask_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(kMaskRows * ((kMaxK + 31) / 32) * sizeof(uint32_t)));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  dim3 g((T + kMaskRows - 1) / kMaskRows, nt);
+  bitmask_kernel<<<g, 256, smem, s>>>(I, perm, region, counts, member, M, K, T, bitmask);
   return cudaGetLastError();
 }
 

@@ -57,6 +57,25 @@ __device__ __forceinline__ void add128(U128& a, const U128& b) {
   a.hi += b.hi + (a.lo < b.lo ? 1ull : 0ull);
 }
 
+// acc += v (a non-negative finite fp32) exactly: at the tile's scale when v >= 2^lsb-ish,
+// else into the exponent buckets.
+__device__ __forceinline__ void acc_value(U128& acc, float v, int lsb, unsigned long long* bucket) {
+  const uint32_t u = __float_as_uint(v);
+  const uint32_t e = u >> 23;
+  const uint32_t m = (u & 0x7FFFFFu) | (e ? 0x800000u : 0u);
+  const int sh = (int)(e ? e : 1u) - 1 - lsb;
+  if (sh >= 0) {
+    const unsigned long long x = m;
+    const unsigned long long lo = sh < 64 ? (x << sh) : 0ull;
+    const unsigned long long hi =
+        sh >= 64 ? (x << (sh - 64)) : (sh > 40 ? (x >> (64 - sh)) : 0ull);
+    acc.lo += lo;
+    acc.hi += hi + (acc.lo < lo ? 1ull : 0ull);
+  } else if (m) {
+    atomicAdd(bucket + (sh + lsb), (unsigned long long)m);
+  }
+}
+
 __device__ __forceinline__ int tile_lsb(int pmax) {
   return pmax > kHeadroomShift ? pmax - kHeadroomShift : 0;
 }
@@ -300,32 +319,26 @@ __global__ void __launch_bounds__(512) candidate_kernel(
   }
   __syncthreads();
 
-  // 2:4 groups: top-2 of 4 per row (lower position wins ties)
+  // 2:4 groups: the two largest of the four importances of every row are kept (which of
+  // two equal values is kept does not change the sum).  One thread per group walks all
+  // rows, so the group's channels are looked up once.
   const int ng = n24 / 4;
-  const int total_s = T * ng;
-  for (int q = threadIdx.x; q < total_s; q += blockDim.x) {
-    const int i = q / ng, g = q - (q / ng) * ng;
-    float v[4];
+  for (int g = threadIdx.x; g < ng; g += blockDim.x) {
+    int c[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       int j = member[4 * g + k];
       j = j < K ? j : 0;
-      v[k] = __ldg(It + (size_t)i * K + ptx::perm_at(perm, j, K));
+      c[k] = ptx::perm_at(perm, j, K);
     }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      int beats = 0;
-#pragma unroll
-      for (int l = 0; l < 4; ++l) beats += (v[l] > v[k]) || (v[l] == v[k] && l < k);
-      if (beats < 2) {
-        uint32_t mm;
-        int e;
-        split_f32(v[k], mm, e);
-        if (mm) {
-          if (e >= lsb) add_shifted(acc, mm, e - lsb);
-          else atomicAdd(bucket + e, (unsigned long long)mm);
-        }
-      }
+    const float* row = It;
+    for (int i = 0; i < T; ++i, row += K) {
+      const float v0 = __ldg(row + c[0]), v1 = __ldg(row + c[1]);
+      const float v2 = __ldg(row + c[2]), v3 = __ldg(row + c[3]);
+      const float a = fmaxf(v0, v1), b = fminf(v0, v1);
+      const float cc = fmaxf(v2, v3), d = fminf(v2, v3);
+      acc_value(acc, fmaxf(a, cc), lsb, bucket);
+      acc_value(acc, fmaxf(fminf(a, cc), fmaxf(b, d)), lsb, bucket);
     }
   }
 

@@ -1,24 +1,25 @@
 // a6. HiNM SpMM on the sm_100a tensor cores (FlexHiNM-GP notes, 关键设计 4: the dense part
 // and the 2:4 part, the latter gathered by the precomputed index, summed into one output).
 //
-// The pages run two CUDA streams (mma and mma.sp) merged by atomicAdd.  Here one CTA per
-// (tile, N-block) runs both kinds of K-block into ONE tensor-memory accumulator:
+// The pages run two CUDA streams (mma and mma.sp) merged by atomicAdd.  Here a persistent
+// kernel (one CTA per SM) walks work units (tile, BN-column block); in each unit both kinds
+// of K-block accumulate into ONE tensor-memory accumulator, double-buffered so the
+// epilogue of a unit overlaps the main loop of the next.
 //
-//   warps 0-3 producers: per K-block, thread 0 bulk-copies the pre-swizzled 16 KB A block
-//                 (and, for a 2:4 block, its 2 KB metadata); the X rows the block's index
-//                 selects are copied by all 128 threads with 16-byte cp.async into the
-//                 swizzled MN-major B tile (coalesced 2*BN-byte row segments), or, when the
-//                 index is one contiguous run, by thread 0 as 2-D tiled TMA boxes.  Every
-//                 producer thread arrives on the stage's full barrier when its copies land.
-//   warp 4       MMA: one thread; 2:4 block -> tcgen05.cp of the metadata into tensor
-//                 memory, then 4 x tcgen05.mma.sp (K = 32 each); dense block -> 4 x
-//                 tcgen05.mma (K = 16 each); tcgen05.commit frees the stage.  Then the warp
-//                 joins the epilogue.
-//   warps 4-7    epilogue: tcgen05.ld of the 128 x BN fp32 accumulator, stores to Y.
+//   warps 0-3  producers: per K-block, thread 0 bulk-copies the pre-swizzled 16 KB A block
+//              (and, for a 2:4 block, its 2 KB metadata); the X rows the block's index
+//              selects are copied by all 128 threads with 16-byte cp.async into the
+//              swizzled MN-major B tile (coalesced 2*BN-byte row segments), or, when the
+//              index is one contiguous run, by thread 0 as 2-D tiled TMA boxes.
+//   warp 4     MMA: one thread; 2:4 block -> tcgen05.cp of the metadata into tensor memory,
+//              then 4 x tcgen05.mma.sp (K = 32 each); dense block -> 4 x tcgen05.mma
+//              (K = 16 each); tcgen05.commit frees the stage / publishes the accumulator.
+//   warps 5-8  epilogue: tcgen05.ld of the 128 x BN fp32 accumulator, stores to Y.
 //
-// Shared memory holds STAGES stages of [A 16 KB | B 128 x BN bf16 | E 2 KB].  Every wait is
-// bounded (2 s), after which the CTA records HINM_ERR_DEVICE_TIMEOUT, drains what it
-// issued, frees tensor memory and returns.
+// Shared memory holds STAGES stages of [A 16 KB | B 128 x BN bf16 | E 2 KB]; the stage ring
+// runs across work units.  Every wait is bounded (2 s), after which the CTA records
+// HINM_ERR_DEVICE_TIMEOUT, stops all roles, drains what it issued, frees tensor memory and
+// returns.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -45,12 +46,14 @@ struct SpmmCfg {
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
   // layout type of the B descriptor: 2 = 128-byte swizzle, 4 = 64-byte, 6 = 32-byte
   static constexpr uint32_t kBLayout = kAtomBytes == 128 ? 2u : (kAtomBytes == 64 ? 4u : 6u);
-  static constexpr int kTmemNeed = BN + 4 * kStages;
+  static constexpr int kAccCols = BN < 32 ? 32 : BN;  // accumulator buffer stride (columns)
+  static constexpr int kTmemNeed = 2 * kAccCols + 4 * kStages;
   static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                    : kTmemNeed <= 256 ? 256 : 512;
-  static constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024 /*align*/ + 256;
+  static constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024 /*align*/ + 512;
   static constexpr int kProducers = 128;
-  static constexpr int kThreads = 256;
+  static constexpr int kMmaWarp = 4;
+  static constexpr int kThreads = 288;  // 9 warps: 4 producers, 1 MMA, 4 epilogue
   static_assert(BN == 16 || BN == 32 || BN % 64 == 0, "BN");
   static_assert(kStages >= 2, "stages");
   static_assert(kTmemNeed <= 512, "tmem");
@@ -68,6 +71,7 @@ struct SpmmArgs {
   const uint16_t* X;
   float* Y;
   int N, T;
+  int num_tiles, nblk_n, num_units;
   int* status;
 };
 
@@ -82,41 +86,69 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
+// X rows idx[0..ROWS) (columns n0 .. n0+BN) -> the swizzled MN-major B tile, 16 bytes per
+// cp.async; consecutive threads copy consecutive 16-byte pieces of a row (coalesced).
+template <class C, int ROWS>
+struct Gather {
+  static constexpr int kPer = ROWS * C::kChunksPerRow / C::kProducers;
+  static_assert(kPer * C::kProducers == ROWS * C::kChunksPerRow, "chunks per producer");
+  int xr[kPer];
+  __device__ __forceinline__ void load_index(const int* __restrict__ idx, int ptid) {
+#pragma unroll
+    for (int i = 0; i < kPer; ++i)
+      xr[i] = __ldg(idx + (ptid + C::kProducers * i) / C::kChunksPerRow);
+  }
+  __device__ __forceinline__ void copy(uint32_t B_s, const uint16_t* __restrict__ X, int N,
+                                       int n0, int ptid) const {
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int q = ptid + C::kProducers * i;
+      const int r = q / C::kChunksPerRow, cc = q - r * C::kChunksPerRow;
+      const int at = cc / C::kChunksPerAtom, c = cc - at * C::kChunksPerAtom;
+      const int col = n0 + cc * 8;
+      const bool ok = col < N;
+      const uint16_t* src = ok ? X + (size_t)xr[i] * N + col : X;
+      uint32_t off = at * (128 * C::kAtomBytes) + r * C::kAtomBytes + c * 16;
+      off ^= ((off >> 7) & ((1u << C::kSwzBits) - 1u)) << 4;  // shared-memory swizzle
+      cp_async_16(B_s + off, src, ok ? 16u : 0u);
+    }
+  }
+};
+
 template <int BN>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(288, 1)
     spmm_kernel(const __grid_constant__ CUtensorMap tmX, const SpmmArgs a) {
   using C = SpmmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
-  // bars[0..S) full, bars[S..2S) empty, bars[2S] accumulator ready, bars[2S+1] drain
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::kStages + 2);
+  // [0,S) full, [S,2S) empty, 2S+{0,1} accumulator full, 2S+{2,3} accumulator empty,
+  // 2S+4 drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::kStages + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = blockIdx.y;
-  const int n0 = blockIdx.x * BN;
-  const int4 info = *reinterpret_cast<const int4*>(a.tile_info + 4 * tile);
-  const int nd = info.x, ns = info.y, d0 = info.z, s0 = info.w;
-  const int nblk = nd + ns;
-
   auto full_bar = [&](int s) { return ptx::smem_u32(bars + s); };
   auto empty_bar = [&](int s) { return ptx::smem_u32(bars + C::kStages + s); };
-  const uint32_t acc_bar = ptx::smem_u32(bars + 2 * C::kStages);
-  const uint32_t drain_bar = ptx::smem_u32(bars + 2 * C::kStages + 1);
+  auto accf_bar = [&](int b) { return ptx::smem_u32(bars + 2 * C::kStages + b); };
+  auto acce_bar = [&](int b) { return ptx::smem_u32(bars + 2 * C::kStages + 2 + b); };
+  const uint32_t drain_bar = ptx::smem_u32(bars + 2 * C::kStages + 4);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       ptx::mbar_init(full_bar(s), 1 + C::kProducers);  // expect_tx arrival + one per producer
       ptx::mbar_init(empty_bar(s), 1);
     }
-    ptx::mbar_init(acc_bar, 1);
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(accf_bar(b), 1);
+      ptx::mbar_init(acce_bar(b), 4);  // one arrival per epilogue warp
+    }
     ptx::mbar_init(drain_bar, 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == C::kMmaWarp) {
     ptx::tmem_alloc(ptx::smem_u32(tmem_slot), C::kTmemCols);
     ptx::tmem_relinquish();
   }
@@ -124,82 +156,98 @@ __global__ void __launch_bounds__(256, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const uint32_t meta_col0 = 2 * C::kAccCols;
 
   if (warp < 4) {
     // ------------------------------------------------------------ producers
     const int ptid = threadIdx.x;
-    int issued = 0;
-    for (int kb = 0; kb < nblk; ++kb) {
-      const int s = kb % C::kStages;
-      const uint32_t ph = (kb / C::kStages) & 1;
-      if (!ptx::mbar_wait(empty_bar(s), ph ^ 1, a.status, abort_flag)) break;
-      const bool sparse = kb >= nd;
-      const int rows = sparse ? kSparseBK : kDenseBK;
-      const uint32_t A_s = ptx::smem_u32(smem + s * C::kStageBytes);
-      const uint32_t B_s = A_s + C::kABytes;
-      const uint32_t E_s = B_s + C::kBBytes;
-      const size_t blk = sparse ? (size_t)(s0 + kb - nd) : (size_t)(d0 + kb);
-      const int run = __ldg(sparse ? a.run_sparse + blk : a.run_dense + blk);
-      if (ptid == 0) {
-        const uint32_t bytes = C::kABytes + (sparse ? C::kEBytes : 0) +
-                               (run >= 0 ? (uint32_t)rows * BN * 2u : 0u);
-        ptx::mbar_arrive_expect_tx(full_bar(s), bytes);
-        ptx::bulk_g2s(A_s, (sparse ? a.vals_sparse : a.vals_dense) + blk * 8192, C::kABytes,
-                      full_bar(s));
-        if (sparse) ptx::bulk_g2s(E_s, a.meta + blk * kMetaWords, C::kEBytes, full_bar(s));
-        if (run >= 0) {
-          // one ascending run of X rows: 2-D tiled boxes of 64 rows x kAtom columns
+    uint32_t it = 0;  // K-blocks issued by this CTA (stage ring position)
+    bool stop = false;
+    for (int u = blockIdx.x; u < a.num_units && !stop; u += gridDim.x) {
+      const int tile = u / a.nblk_n, n0 = (u - tile * a.nblk_n) * BN;
+      const int4 info = __ldg(reinterpret_cast<const int4*>(a.tile_info) + tile);
+      const int nd = info.x, nblk = info.x + info.y;
+      for (int kb = 0; kb < nblk; ++kb, ++it) {
+        const bool sparse = kb >= nd;
+        const size_t blk = sparse ? (size_t)(info.w + kb - nd) : (size_t)(info.z + kb);
+        // index loads are issued before the wait so their latency hides behind it
+        const int run = __ldg(sparse ? a.run_sparse + blk : a.run_dense + blk);
+        Gather<C, kSparseBK> gs;
+        Gather<C, kDenseBK> gd;
+        if (run < 0) {
+          if (sparse) gs.load_index(a.idx_sparse + blk * kSparseBK, ptid);
+          else gd.load_index(a.idx_dense + blk * kDenseBK, ptid);
+        }
+        const int s = it % C::kStages;
+        const uint32_t ph = (it / C::kStages) & 1;
+        if (!ptx::mbar_wait(empty_bar(s), ph ^ 1, a.status, abort_flag)) {
+          stop = true;
+          break;
+        }
+        const uint32_t A_s = ptx::smem_u32(smem + s * C::kStageBytes);
+        const uint32_t B_s = A_s + C::kABytes;
+        const uint32_t E_s = B_s + C::kBBytes;
+        const int rows = sparse ? kSparseBK : kDenseBK;
+        if (ptid == 0) {
+          const uint32_t bytes = C::kABytes + (sparse ? C::kEBytes : 0) +
+                                 (run >= 0 ? (uint32_t)rows * BN * 2u : 0u);
+          ptx::mbar_arrive_expect_tx(full_bar(s), bytes);
+          ptx::bulk_g2s(A_s, (sparse ? a.vals_sparse : a.vals_dense) + blk * 8192, C::kABytes,
+                        full_bar(s));
+          if (sparse) ptx::bulk_g2s(E_s, a.meta + blk * kMetaWords, C::kEBytes, full_bar(s));
+          if (run >= 0) {
+            // one ascending run of X rows: 2-D tiled boxes of 64 rows x kAtom columns
 #pragma unroll 1
-          for (int at = 0; at < BN / C::kAtom; ++at)
+            for (int at = 0; at < BN / C::kAtom; ++at)
 #pragma unroll 1
-            for (int h = 0; h < rows / 64; ++h)
-              ptx::tma_load_2d(B_s + at * (128 * C::kAtomBytes) + h * 64 * C::kAtomBytes, &tmX,
-                               n0 + at * C::kAtom, run + h * 64, full_bar(s));
+              for (int h = 0; h < rows / 64; ++h)
+                ptx::tma_load_2d(B_s + at * (128 * C::kAtomBytes) + h * 64 * C::kAtomBytes, &tmX,
+                                 n0 + at * C::kAtom, run + h * 64, full_bar(s));
+            ptx::mbar_arrive_count(full_bar(s), C::kProducers);  // on behalf of all producers
+          }
+        }
+        if (run < 0) {
+          if (sparse) gs.copy(B_s, a.X, a.N, n0, ptid);
+          else gd.copy(B_s, a.X, a.N, n0, ptid);
+          cp_async_arrive_noinc(full_bar(s));
         }
       }
-      if (run < 0) {
-        const int* idx = sparse ? a.idx_sparse + blk * kSparseBK : a.idx_dense + blk * kDenseBK;
-        const int chunks = rows * C::kChunksPerRow;
-        for (int q = ptid; q < chunks; q += C::kProducers) {
-          const int r = q / C::kChunksPerRow, cc = q - r * C::kChunksPerRow;
-          const int at = cc / C::kChunksPerAtom, c = cc - at * C::kChunksPerAtom;
-          const int col = n0 + cc * 8;
-          const int xr = __ldg(idx + r);
-          const bool ok = col < a.N;
-          const uint16_t* src = ok ? a.X + (size_t)xr * a.N + col : a.X;
-          uint32_t off = at * (128 * C::kAtomBytes) + r * C::kAtomBytes + c * 16;
-          off ^= ((off >> 7) & ((1u << C::kSwzBits) - 1u)) << 4;  // shared-memory swizzle
-          cp_async_16(B_s + off, src, ok ? 16u : 0u);
-        }
-      }
-      cp_async_arrive_noinc(full_bar(s));
-      ++issued;
     }
     cp_async_wait_all();
     if (*abort_flag && ptid == 0) {
-      // wait (bounded) for the bulk / tensor copies issued and never consumed
-      for (int kb = (issued > C::kStages ? issued - C::kStages : 0); kb < issued; ++kb)
-        ptx::mbar_wait(full_bar(kb % C::kStages), (kb / C::kStages) & 1, a.status, nullptr);
+      // wait (bounded) for the bulk / tensor copies of the last stages
+      for (uint32_t k = (it > (uint32_t)C::kStages ? it - C::kStages : 0u); k < it; ++k)
+        ptx::mbar_wait(full_bar(k % C::kStages), (k / C::kStages) & 1, a.status, nullptr);
     }
-  } else {
-    if (warp == 4) {
-      // ------------------------------------------------------------ MMA issuer
-      if (lane == 0) {
-        const uint32_t idesc_d = ptx::idesc_bf16(BN, 1, 0);
-        const uint32_t idesc_s = ptx::idesc_bf16(BN, 1, 1);
-        bool any = false;
-        for (int kb = 0; kb < nblk; ++kb) {
-          const int s = kb % C::kStages;
-          const uint32_t ph = (kb / C::kStages) & 1;
-          if (!ptx::mbar_wait(full_bar(s), ph, a.status, abort_flag)) break;
+  } else if (warp == C::kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_d = ptx::idesc_bf16(BN, 1, 0);
+      const uint32_t idesc_s = ptx::idesc_bf16(BN, 1, 1);
+      uint32_t it = 0, lu = 0;
+      bool stop = false;
+      for (int u = blockIdx.x; u < a.num_units && !stop; u += gridDim.x, ++lu) {
+        const int tile = u / a.nblk_n;
+        const int4 info = __ldg(reinterpret_cast<const int4*>(a.tile_info) + tile);
+        const int nd = info.x, nblk = info.x + info.y;
+        const int b = lu & 1;
+        if (!ptx::mbar_wait(acce_bar(b), ((lu >> 1) & 1) ^ 1, a.status, abort_flag)) break;
+        ptx::tc_fence_after();
+        const uint32_t acc = tmem + b * C::kAccCols;
+        for (int kb = 0; kb < nblk; ++kb, ++it) {
+          const int s = it % C::kStages;
+          const uint32_t ph = (it / C::kStages) & 1;
+          if (!ptx::mbar_wait(full_bar(s), ph, a.status, abort_flag)) {
+            stop = true;
+            break;
+          }
           ptx::fence_proxy_async_smem();  // cp.async (generic proxy) -> tensor-core reads
           ptx::tc_fence_after();
-          const bool sparse = kb >= nd;
           const uint32_t A_s = ptx::smem_u32(smem + s * C::kStageBytes);
           const uint32_t B_s = A_s + C::kABytes;
           const uint32_t E_s = B_s + C::kBBytes;
-          if (sparse) {
-            const uint32_t e_col = tmem + BN + 4 * s;
+          if (kb >= nd) {
+            const uint32_t e_col = tmem + meta_col0 + 4 * s;
             // 128 lanes x 16 bytes, rows 16 B apart: core matrices of 8 rows, 128 B apart
             ptx::tc_cp_128x128b(e_col, ptx::smem_desc(E_s, 2048, 128, 0));
 #pragma unroll
@@ -208,8 +256,7 @@ __global__ void __launch_bounds__(256, 1)
               const uint64_t bd = ptx::smem_desc(B_s + 32 * k * C::kAtomBytes, 128 * C::kAtomBytes,
                                                  8 * C::kAtomBytes, C::kBLayout);
               const uint32_t e = e_col + k;
-              ptx::mma_sp_bf16(tmem, ad, bd, e & ~1u, idesc_s | (e & 1u), any ? 1u : 0u);
-              any = true;
+              ptx::mma_sp_bf16(acc, ad, bd, e & ~1u, idesc_s | (e & 1u), (kb | k) ? 1u : 0u);
             }
           } else {
 #pragma unroll
@@ -217,64 +264,74 @@ __global__ void __launch_bounds__(256, 1)
               const uint64_t ad = ptx::smem_desc(A_s + 32 * k, 16, 1024, 2);
               const uint64_t bd = ptx::smem_desc(B_s + 16 * k * C::kAtomBytes, 128 * C::kAtomBytes,
                                                  8 * C::kAtomBytes, C::kBLayout);
-              ptx::mma_bf16(tmem, ad, bd, idesc_d, any ? 1u : 0u);
-              any = true;
+              ptx::mma_bf16(acc, ad, bd, idesc_d, (kb | k) ? 1u : 0u);
             }
           }
           ptx::tc_commit(empty_bar(s));
         }
-        if (nblk > 0) ptx::tc_commit(acc_bar);
-        // every tcgen05 operation issued above has completed once drain_bar flips
-        ptx::tc_commit(drain_bar);
-        ptx::mbar_wait(drain_bar, 0, a.status, nullptr);
+        if (stop) break;
+        ptx::tc_commit(accf_bar(b));  // accumulator b ready (immediately if no K-blocks)
       }
-      __syncwarp();
+      // every tcgen05 operation issued above has completed once drain_bar flips
+      ptx::tc_commit(drain_bar);
+      ptx::mbar_wait(drain_bar, 0, a.status, nullptr);
     }
-    // ------------------------------------------------------------ epilogue (warps 4..7)
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 5..8)
     const int q = warp & 3;  // tensor-memory lane quadrant this warp may access
     const int row = q * 32 + lane;
-    bool have = nblk > 0;
-    if (have) {
-      have = ptx::mbar_wait(acc_bar, 0, a.status, abort_flag);
-      ptx::tc_fence_after();
-    }
-    have = __all_sync(0xffffffffu, have);
-    const bool row_ok = row < a.T;
-    float* yrow = a.Y + (size_t)(tile * a.T + row) * a.N;
     constexpr int kChunk = BN >= 32 ? 32 : 16;
-    for (int col = 0; col < BN; col += kChunk) {
-      uint32_t v[32];
-      if (have) {
-        const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)col;
-        if constexpr (kChunk == 32) {
-          ptx::tmem_ld_32x32b_x32(taddr, v);
-        } else {
-          ptx::tmem_ld_32x32b_x16(taddr, v);
-        }
-        ptx::tmem_ld_wait();
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = 0u;
-      }
-      if (row_ok && !(*abort_flag)) {
-        const int gc = n0 + col;
-        if (gc + kChunk <= a.N) {
-#pragma unroll
-          for (int i = 0; i < kChunk; i += 4) {
-            float4 o = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
-                                   __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
-            *reinterpret_cast<float4*>(yrow + gc + i) = o;
+    uint32_t lu = 0;
+    for (int u = blockIdx.x; u < a.num_units; u += gridDim.x, ++lu) {
+      const int tile = u / a.nblk_n, n0 = (u - tile * a.nblk_n) * BN;
+      const int4 info = __ldg(reinterpret_cast<const int4*>(a.tile_info) + tile);
+      const int nblk = info.x + info.y;
+      const int b = lu & 1;
+      bool ok = ptx::mbar_wait(accf_bar(b), (lu >> 1) & 1, a.status, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      const bool row_ok = row < a.T;
+      float* yrow = a.Y + (size_t)(tile * a.T + row) * a.N;
+      for (int col = 0; col < BN; col += kChunk) {
+        uint32_t v[32];
+        if (nblk > 0) {
+          const uint32_t taddr =
+              tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::kAccCols + col);
+          if constexpr (kChunk == 32) {
+            ptx::tmem_ld_32x32b_x32(taddr, v);
+          } else {
+            ptx::tmem_ld_32x32b_x16(taddr, v);
           }
+          ptx::tmem_ld_wait();
         } else {
-          for (int i = 0; i < kChunk; ++i)
-            if (gc + i < a.N) yrow[gc + i] = __uint_as_float(v[i]);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0u;
+        }
+        if (row_ok) {
+          const int gc = n0 + col;
+          if (gc + kChunk <= a.N) {
+#pragma unroll
+            for (int i = 0; i < kChunk; i += 4) {
+              float4 o = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                                     __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+              *reinterpret_cast<float4*>(yrow + gc + i) = o;
+            }
+          } else {
+            for (int i = 0; i < kChunk; ++i)
+              if (gc + i < a.N) yrow[gc + i] = __uint_as_float(v[i]);
+          }
         }
       }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(acce_bar(b));  // accumulator b may be overwritten
     }
   }
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == C::kMmaWarp) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::kTmemCols);
   }
@@ -315,6 +372,17 @@ bool make_x_map(CUtensorMap* m, const uint16_t* X, int K, int N, int atom) {
   return r == CUDA_SUCCESS;
 }
 
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
 template <int BN>
 cudaError_t run(const hinm_layout& L, const uint16_t* X, int N, float* Y, int* status,
                 cudaStream_t s) {
@@ -328,10 +396,12 @@ cudaError_t run(const hinm_layout& L, const uint16_t* X, int N, float* Y, int* s
   if (attr_err != cudaSuccess) return attr_err;
   CUtensorMap map;
   if (!make_x_map(&map, X, L.K, N, C::kAtom)) return cudaErrorInvalidValue;
-  SpmmArgs a{L.tile_info, L.vals_dense, L.vals_sparse, L.meta, L.idx_dense, L.idx_sparse,
-             L.run_dense, L.run_sparse, X,      Y,           N,           L.T,
-             status};
-  dim3 grid((N + BN - 1) / BN, L.num_tiles);
+  const int nblk_n = (N + BN - 1) / BN;
+  const int units = L.num_tiles * nblk_n;
+  SpmmArgs a{L.tile_info, L.vals_dense, L.vals_sparse, L.meta,   L.idx_dense, L.idx_sparse,
+             L.run_dense, L.run_sparse, X,             Y,        N,           L.T,
+             L.num_tiles, nblk_n,       units,         status};
+  const int grid = units < num_sms() ? units : num_sms();
   spmm_kernel<BN><<<grid, C::kThreads, C::kSmemBytes, s>>>(map, a);
   return cudaGetLastError();
 }
