@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint16_t* __restrict__ 
                                                    const int32_t* __restrict__ lists, int K, int T,
                                                    hinm_layout L, int* status) {
   __shared__ uint8_t nib[128][32];
-  __shared__ int idx_s[kSparseBK];
+  __shared__ int chan[kSparseBK];  // input channel of every vector of the block, -1 = padding
   const int t = blockIdx.y;
   const int b = blockIdx.x;
   const int nd = L.tile_info[4 * t + 0], ns = L.tile_info[4 * t + 1];
@@ -124,21 +124,50 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint16_t* __restrict__ 
   const int words = (K + 31) >> 5;
   const int32_t* lst = lists + (size_t)t * K;
   const int row0 = t * T;
-  if (b < nd) {
+  const bool sparse = b >= nd;
+  const int sb = b - nd;
+  const int nvec = sparse ? kSparseBK : kDenseBK;
+  if (threadIdx.x < nvec) {
+    const int p = sparse ? sb * kSparseBK + threadIdx.x : b * kDenseBK + threadIdx.x;
+    const int lim = sparse ? n24 : n4;
+    chan[threadIdx.x] = p < lim ? ptx::perm_at(perm, list_at(lst, (sparse ? n4 : 0) + p, K), K) : -1;
+  }
+  __syncthreads();
+  // index and contiguous-run flag
+  if (threadIdx.x < nvec) {
+    const int v = chan[threadIdx.x] < 0 ? 0 : chan[threadIdx.x];
+    if (sparse) L.idx_sparse[(size_t)(s0 + sb) * kSparseBK + threadIdx.x] = v;
+    else L.idx_dense[(size_t)(d0 + b) * kDenseBK + threadIdx.x] = v;
+  }
+  const int c0 = chan[0] < 0 ? 0 : chan[0];
+  const bool step_ok = threadIdx.x >= nvec || chan[threadIdx.x] == c0 + (int)threadIdx.x;
+  const bool run = __syncthreads_and(step_ok);
+  if (threadIdx.x == 0) {
+    if (sparse) L.run_sparse[s0 + sb] = run ? c0 : -1;
+    else L.run_dense[d0 + b] = run ? c0 : -1;
+  }
+
+  if (!sparse) {
     uint8_t* out = reinterpret_cast<uint8_t*>(L.vals_dense + (size_t)(d0 + b) * 8192);
+#pragma unroll 2
     for (int item = threadIdx.x; item < 128 * 8; item += blockDim.x) {
       const int r = item >> 3, ch = item & 7;
       uint32_t h[8];
+      if (r < T) {
+        const int i = row0 + r;
+        const uint16_t* Wi = W + (size_t)i * K;
+        const uint32_t* bmi = bitmask + (size_t)i * words;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int p = b * kDenseBK + ch * 8 + e;
-        uint32_t v = 0;
-        if (r < T && p < n4) {
-          const int c = ptx::perm_at(perm, list_at(lst, p, K), K);
-          const int i = row0 + r;
-          if (mask_bit(bitmask, words, i, c)) v = __ldg(W + (size_t)i * K + c);
+        for (int e = 0; e < 8; ++e) {
+          const int c = chan[ch * 8 + e];
+          const int cc = c < 0 ? 0 : c;
+          const uint32_t w = __ldg(Wi + cc);
+          const uint32_t bit = (__ldg(bmi + (cc >> 5)) >> (cc & 31)) & 1u;
+          h[e] = (c >= 0 && bit) ? w : 0u;
         }
-        h[e] = v;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) h[e] = 0u;
       }
       uint4 q;
       q.x = h[0] | (h[1] << 16);
@@ -147,51 +176,45 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint16_t* __restrict__ 
       q.w = h[6] | (h[7] << 16);
       *reinterpret_cast<uint4*>(out + r * 128 + ((ch ^ (r & 7)) << 4)) = q;
     }
-    int v = 0;
-    if (threadIdx.x < kDenseBK) {
-      const int p = b * kDenseBK + threadIdx.x;
-      v = p < n4 ? ptx::perm_at(perm, list_at(lst, p, K), K) : 0;
-      L.idx_dense[(size_t)(d0 + b) * kDenseBK + threadIdx.x] = v;
-      idx_s[threadIdx.x] = v;
-    }
-    __syncthreads();
-    const bool step_ok = threadIdx.x >= kDenseBK || v == idx_s[0] + (int)threadIdx.x;
-    const bool run = __syncthreads_and(step_ok);
-    if (threadIdx.x == 0) L.run_dense[d0 + b] = run ? idx_s[0] : -1;
     return;
   }
-  const int sb = b - nd;
+
   uint8_t* out = reinterpret_cast<uint8_t*>(L.vals_sparse + (size_t)(s0 + sb) * 8192);
+#pragma unroll 2
   for (int item = threadIdx.x; item < 128 * 32; item += blockDim.x) {
     const int r = item >> 5, g = item & 31;
-    const int q0 = sb * kSparseBK + 4 * g;  // first 2:4 vector of the group
     uint32_t a = 0, bb = 1, va = 0, vb = 0;
-    if (r < T && q0 < n24) {
+    if (r < T && chan[4 * g] >= 0) {
       const int i = row0 + r;
-      int c[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) c[k] = ptx::perm_at(perm, list_at(lst, n4 + q0 + k, K), K);
-      int kept[4], nk = 0, free_[4], nf = 0;
+      const uint16_t* Wi = W + (size_t)i * K;
+      const uint32_t* bmi = bitmask + (size_t)i * words;
+      uint32_t w[4], kept = 0;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        if (mask_bit(bitmask, words, i, c[k])) kept[nk++] = k;
-        else free_[nf++] = k;
+        const int c = chan[4 * g + k];
+        w[k] = __ldg(Wi + c);
+        kept |= ((__ldg(bmi + (c >> 5)) >> (c & 31)) & 1u) << k;
       }
+      const int nk = __popc(kept);
       if (nk != 2) ptx::record_status(status, HINM_ERR_BAD_MASK);
-      int pa, pb;
-      bool use_a, use_b;
-      if (nk >= 2) {
-        pa = kept[0]; pb = kept[1]; use_a = use_b = true;
-      } else if (nk == 1) {
-        pa = kept[0]; pb = free_[0]; use_a = true; use_b = false;
-        if (pb < pa) { const int x = pa; pa = pb; pb = x; use_a = false; use_b = true; }
+      // the two kept positions, lowest first; a missing one is taken from the unkept
+      // positions with value 0 so that the pair stays a legal (a < b) pattern
+      int pos[2], np = 0;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (((kept >> k) & 1u) && np < 2) pos[np++] = k;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (!((kept >> k) & 1u) && np < 2) pos[np++] = -1 - k;  // filler, value 0
+      const int pa = pos[0] < 0 ? -1 - pos[0] : pos[0];
+      const int pb = pos[1] < 0 ? -1 - pos[1] : pos[1];
+      const bool ua = pos[0] >= 0, ub = pos[1] >= 0;
+      // order the pair by position
+      if (pa < pb) {
+        a = pa; bb = pb; va = ua ? w[pa] : 0u; vb = ub ? w[pb] : 0u;
       } else {
-        pa = 0; pb = 1; use_a = use_b = false;
+        a = pb; bb = pa; va = ub ? w[pb] : 0u; vb = ua ? w[pa] : 0u;
       }
-      a = pa;
-      bb = pb;
-      va = use_a ? __ldg(W + (size_t)i * K + c[pa]) : 0u;
-      vb = use_b ? __ldg(W + (size_t)i * K + c[pb]) : 0u;
     }
     *reinterpret_cast<uint32_t*>(out + swz(r, 2 * g)) = va | (vb << 16);
     nib[r][g] = (uint8_t)(a | (bb << 2));
@@ -210,17 +233,6 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint16_t* __restrict__ 
     }
     meta[wi] = word;
   }
-  int v = 0;
-  if (threadIdx.x < kSparseBK) {
-    const int p = sb * kSparseBK + threadIdx.x;
-    v = p < n24 ? ptx::perm_at(perm, list_at(lst, n4 + p, K), K) : 0;
-    L.idx_sparse[(size_t)(s0 + sb) * kSparseBK + threadIdx.x] = v;
-    idx_s[threadIdx.x] = v;
-  }
-  __syncthreads();
-  const bool step_ok = threadIdx.x >= kSparseBK || v == idx_s[0] + (int)threadIdx.x;
-  const bool run = __syncthreads_and(step_ok);
-  if (threadIdx.x == 0) L.run_sparse[s0 + sb] = run ? idx_s[0] : -1;
 }
 
 size_t compress_workspace_bytes(int M, int K, int T) {

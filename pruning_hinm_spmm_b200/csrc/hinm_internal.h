@@ -73,8 +73,11 @@ cudaError_t launch_spmm(const hinm_layout& L, const uint16_t* X, int N, float* Y
 
 // Shared by the rank users (search and mask): V (fp64 column sums per tile) and the rank
 // of every working position.
-// tile_pmax (int [M/T]) receives each tile's largest fp32 exponent.
+// tile_pmax (int [M/T]) receives each tile's largest fp32 exponent; scratch holds
+// rank_scratch_bytes() bytes.
+size_t rank_scratch_bytes(int M, int K, int T);
 cudaError_t launch_vector_rank(const float* I, const int32_t* perm, int M, int K, int T,
-                               double* V, int32_t* rank, int* tile_pmax, cudaStream_t s);
+                               double* V, int32_t* rank, int* tile_pmax, void* scratch,
+                               cudaStream_t s);
 
 }  // namespace hinm

@@ -16,7 +16,8 @@ __device__ __forceinline__ double bf16_to_f64(uint32_t bits16) {
   return static_cast<double>(__uint_as_float(bits16 << 16));
 }
 
-// One thread per channel c: sequential fp64 sum over n = 0..N-1 (N % 8 == 0).
+// One thread per channel c: sequential fp64 sum over n = 0..N-1 (N % 8 == 0).  Up to 8
+// 16-byte loads are in flight before they are summed, in order.
 __global__ void channel_energy_kernel(const uint16_t* __restrict__ X, int K, int N,
                                       float* __restrict__ s) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
@@ -24,14 +25,32 @@ __global__ void channel_energy_kernel(const uint16_t* __restrict__ X, int K, int
   const uint4* row = reinterpret_cast<const uint4*>(X + (size_t)c * N);
   double acc = 0.0;
   const int nv = N / 8;
-  for (int v = 0; v < nv; ++v) {
-    const uint4 q = __ldg(row + v);
+  constexpr int kBatch = 8;
+  int v0 = 0;
+  for (; v0 + kBatch <= nv; v0 += kBatch) {
+    uint4 q[kBatch];
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) q[k] = __ldg(row + v0 + k);
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      const uint32_t w[4] = {q[k].x, q[k].y, q[k].z, q[k].w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const double a = bf16_to_f64(w[h] & 0xFFFFu);
+        const double b = bf16_to_f64(w[h] >> 16);
+        acc = __dadd_rn(acc, __dmul_rn(a, a));  // x^2 of a bf16 is exact in fp64
+        acc = __dadd_rn(acc, __dmul_rn(b, b));
+      }
+    }
+  }
+  for (; v0 < nv; ++v0) {
+    const uint4 q = __ldg(row + v0);
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
       const double a = bf16_to_f64(w[h] & 0xFFFFu);
       const double b = bf16_to_f64(w[h] >> 16);
-      acc = __dadd_rn(acc, __dmul_rn(a, a));  // x^2 of a bf16 is exact in fp64
+      acc = __dadd_rn(acc, __dmul_rn(a, a));
       acc = __dadd_rn(acc, __dmul_rn(b, b));
     }
   }
@@ -76,7 +95,7 @@ size_t importance_workspace_bytes(int K) { return ((size_t)K * sizeof(float) + 2
 
 cudaError_t launch_importance(const uint16_t* W, const uint16_t* X, int M, int K, int N,
                               float* I, float* s_scratch, cudaStream_t st) {
-  channel_energy_kernel<<<(K + 127) / 128, 128, 0, st>>>(X, K, N, s_scratch);
+  channel_energy_kernel<<<(K + 63) / 64, 64, 0, st>>>(X, K, N, s_scratch);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const long long total4 = (long long)M * K / 4;

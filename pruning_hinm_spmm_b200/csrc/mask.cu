@@ -138,6 +138,7 @@ __global__ void __launch_bounds__(256) bitmask_kernel(
       c[k] = ptx::perm_at(perm, j, K);
     }
     const float* row = I0;
+#pragma unroll 4
     for (int r = 0; r < rows; ++r, row += K) {
       float v[4];
 #pragma unroll
@@ -169,6 +170,7 @@ size_t mask_workspace_bytes(int M, int K, int T) {
   c.take<int32_t>((size_t)K);       // inverse permutation
   c.take<int32_t>((size_t)nt * K);  // member
   c.take<int>((size_t)nt);          // tile max exponent (by-product of the ranking)
+  c.take<char>(rank_scratch_bytes(M, K, T));
   return (c.off + 255) & ~size_t(255);
 }
 
@@ -182,9 +184,10 @@ cudaError_t launch_mask(const float* I, const int32_t* perm, const int32_t* coun
   int32_t* pinv = cv.take<int32_t>((size_t)K);
   int32_t* member = cv.take<int32_t>((size_t)nt * K);
   int* pmax = cv.take<int>((size_t)nt);
+  char* rank_scratch = cv.take<char>(rank_scratch_bytes(M, K, T));
   cudaError_t e;
   if (!rank) {
-    e = launch_vector_rank(I, perm, M, K, T, V, rank_ws, pmax, s);
+    e = launch_vector_rank(I, perm, M, K, T, V, rank_ws, pmax, rank_scratch, s);
     if (e != cudaSuccess) return e;
     rank = rank_ws;
   }

@@ -4,13 +4,19 @@
 // R_total = R_dense + R_24; 亮点与洞察: high -> dense, middle -> 2:4, low -> pruned).
 //
 // Kernels:
-//   vector_score_kernel   V[t, c] = sum of I over the tile's rows, ascending, fp64
-//   rank_sort_kernel      one CTA per tile: bitonic sort of (V desc, j asc) in shared
-//                         memory; writes rank[t][j]
-//   candidate_kernel      one CTA per (candidate m, tile): regions, 2:4 groups, top-2,
-//                         and the EXACT sum of the kept importance (integer exponent
-//                         buckets), rounded once to fp64 -> R[t][m]
-//   select_kernel         first m with R(m+1) < R(m), else the last candidate
+//   vector_score_kernel   V[t, c] = sum of I over the tile's rows, ascending, fp64, and
+//                         each tile's largest exponent
+//   chunk_sort_kernel,    rank[t][j] of (V desc, j asc): bitonic sort of 1024-position
+//   merge_rank_kernel     chunks, then a binary-search count over the sorted chunks
+//   column_sum_kernel     exact column sums (128-bit integers at the tile's scale)
+//   candidate_lists_kernel  one CTA per (candidate m, tile): the 2:4 band's channels in
+//                         ascending working position and the exact sum of the dense
+//                         vectors' column sums
+//   band_sum_kernel       one CTA per (tile, chunk of rows): the rows are staged in shared
+//                         memory once and every candidate's groups are evaluated from there
+//                         (top-2 of 4 per row, exact 128-bit partial sums)
+//   finalize_kernel       per tile: R(m) = exact total rounded once to fp64; the first m
+//                         with R(m+1) < R(m), else the last candidate
 #include <cuda_runtime.h>
 
 #include "hinm_internal.h"
@@ -76,6 +82,30 @@ __device__ __forceinline__ void acc_value(U128& acc, float v, int lsb, unsigned 
   }
 }
 
+// acc += t1 + t2 (t1 >= t2 >= 0, fp32) exactly.  When their fp64 sum is exact (Fast2Sum
+// error 0) and at or above the tile's scale it is added once (a 53-bit mantissa shifted by
+// at most 56 bits); otherwise each value goes through acc_value.
+__device__ __forceinline__ void acc_pair(U128& acc, float t1, float t2, int lsb,
+                                         unsigned long long* bucket) {
+  const double a = t1, b = t2;
+  const double s = __dadd_rn(a, b);
+  const double err = __dsub_rn(b, __dsub_rn(s, a));
+  if (err == 0.0 && s != 0.0) {
+    const unsigned long long bits = (unsigned long long)__double_as_longlong(s);
+    const int sh = (int)(bits >> 52) - 926 - lsb;  // s = m53 * 2^sh in units of 2^(lsb-149)
+    if (sh >= 0) {
+      const unsigned long long m = (bits & 0xFFFFFFFFFFFFFull) | (1ull << 52);
+      const unsigned long long lo = m << sh;
+      const unsigned long long hi = sh ? (m >> (64 - sh)) : 0ull;
+      acc.lo += lo;
+      acc.hi += hi + (acc.lo < lo ? 1ull : 0ull);
+      return;
+    }
+  }
+  acc_value(acc, t1, lsb, bucket);
+  acc_value(acc, t2, lsb, bucket);
+}
+
 __device__ __forceinline__ int tile_lsb(int pmax) {
   return pmax > kHeadroomShift ? pmax - kHeadroomShift : 0;
 }
@@ -90,13 +120,19 @@ __global__ void vector_score_kernel(const float* __restrict__ I, int K, int T,
   if (c < K) {
     const float* p = I + (size_t)t * T * K + c;
     double acc = 0.0;
-    for (int i = 0; i < T; ++i) {
-      const float v = __ldg(p + (size_t)i * K);
-      acc = __dadd_rn(acc, (double)v);
-      uint32_t m;
-      int e;
-      split_f32(v, m, e);
-      if (m) pm = max(pm, e);
+    constexpr int kBatch = 16;  // loads in flight per thread (T is a multiple of 16)
+    for (int i0 = 0; i0 < T; i0 += kBatch) {
+      float v[kBatch];
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) v[k] = __ldg(p + (size_t)(i0 + k) * K);
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) {  // rows ascending
+        acc = __dadd_rn(acc, (double)v[k]);
+        uint32_t m;
+        int e;
+        split_f32(v[k], m, e);
+        if (m) pm = max(pm, e);
+      }
     }
     Vc[(size_t)t * K + c] = acc;
   }
@@ -116,50 +152,65 @@ __global__ void column_sum_kernel(const float* __restrict__ I, int K, int T,
   const float* p = I + (size_t)t * T * K + c;
   U128 acc{0ull, 0ull};
   unsigned char tiny = 0;
-  for (int i = 0; i < T; ++i) {
-    uint32_t m;
-    int e;
-    split_f32(__ldg(p + (size_t)i * K), m, e);
-    if (!m) continue;
-    if (e >= lsb) add_shifted(acc, m, e - lsb);
-    else tiny = 1;
+  constexpr int kBatch = 16;
+  for (int i0 = 0; i0 < T; i0 += kBatch) {
+    float v[kBatch];
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) v[k] = __ldg(p + (size_t)(i0 + k) * K);
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      uint32_t m;
+      int e;
+      split_f32(v[k], m, e);
+      if (!m) continue;
+      if (e >= lsb) add_shifted(acc, m, e - lsb);
+      else tiny = 1;
+    }
   }
   colsum[(size_t)t * K + c] = acc;
   coltiny[(size_t)t * K + c] = tiny;
 }
 
 // ------------------------------------------------------------------ rank sort
-// Sort key: (~bits(V), j) ascending == (V descending, j ascending); V >= 0 so its bit
-// pattern orders like its value.  Padding entries (j = 0xFFFF) sort last.
-__global__ void __launch_bounds__(1024) rank_sort_kernel(const double* __restrict__ Vc,
+// Order key of working position j: (~bits(V), j) ascending == (V descending, j ascending);
+// V >= 0, so its bit pattern orders like its value.  Every (key, j) pair is distinct.
+// Phase 1 sorts chunks of 1024 positions in shared memory (bitonic); phase 2 gives every
+// position its rank = sum over chunks of the number of smaller pairs (binary search).
+constexpr int kRankChunk = 1024;
+
+__device__ __forceinline__ bool pair_less(unsigned long long ka, unsigned ia,
+                                          unsigned long long kb, unsigned ib) {
+  return ka < kb || (ka == kb && ia < ib);
+}
+
+__global__ void __launch_bounds__(512) chunk_sort_kernel(const double* __restrict__ Vc,
                                                          const int32_t* __restrict__ perm, int K,
-                                                         int Kp, int32_t* __restrict__ rank) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  unsigned long long* key = reinterpret_cast<unsigned long long*>(smem);
-  unsigned short* idx = reinterpret_cast<unsigned short*>(key + Kp);
-  const int t = blockIdx.x;
+                                                         int Kp, unsigned long long* __restrict__ skey,
+                                                         unsigned short* __restrict__ sidx) {
+  __shared__ unsigned long long key[kRankChunk];
+  __shared__ unsigned short idx[kRankChunk];
+  const int t = blockIdx.y, base = blockIdx.x * kRankChunk;
   const double* V = Vc + (size_t)t * K;
-  for (int j = threadIdx.x; j < Kp; j += blockDim.x) {
+  for (int i = threadIdx.x; i < kRankChunk; i += blockDim.x) {
+    const int j = base + i;
     if (j < K) {
-      const int c = ptx::perm_at(perm, j, K);
-      key[j] = ~static_cast<unsigned long long>(__double_as_longlong(__ldg(V + c)));
-      idx[j] = (unsigned short)j;
+      key[i] = ~static_cast<unsigned long long>(__double_as_longlong(__ldg(V + ptx::perm_at(perm, j, K))));
+      idx[i] = (unsigned short)j;
     } else {
-      key[j] = ~0ull;
-      idx[j] = 0xFFFF;
+      key[i] = ~0ull;
+      idx[i] = 0xFFFF;
     }
   }
   __syncthreads();
-  for (int k = 2; k <= Kp; k <<= 1) {
+  for (int k = 2; k <= kRankChunk; k <<= 1) {
     for (int jj = k >> 1; jj > 0; jj >>= 1) {
-      for (int i = threadIdx.x; i < Kp; i += blockDim.x) {
+      for (int i = threadIdx.x; i < kRankChunk; i += blockDim.x) {
         const int l = i ^ jj;
         if (l > i) {
           const unsigned long long ki = key[i], kl = key[l];
           const unsigned short ii = idx[i], il = idx[l];
-          const bool i_gt = (ki > kl) || (ki == kl && ii > il);
-          const bool ascending = (i & k) == 0;
-          if (i_gt == ascending) {
+          const bool i_gt = pair_less(kl, il, ki, ii);
+          if (i_gt == ((i & k) == 0)) {
             key[i] = kl;
             key[l] = ki;
             idx[i] = il;
@@ -170,12 +221,49 @@ __global__ void __launch_bounds__(1024) rank_sort_kernel(const double* __restric
       __syncthreads();
     }
   }
-  int32_t* r = rank + (size_t)t * K;
-  for (int p = threadIdx.x; p < K; p += blockDim.x) r[idx[p]] = p;
+  for (int i = threadIdx.x; i < kRankChunk; i += blockDim.x) {
+    skey[(size_t)t * Kp + base + i] = key[i];
+    sidx[(size_t)t * Kp + base + i] = idx[i];
+  }
+}
+
+__global__ void merge_rank_kernel(const double* __restrict__ Vc, const int32_t* __restrict__ perm,
+                                  const unsigned long long* __restrict__ skey,
+                                  const unsigned short* __restrict__ sidx, int K, int Kp,
+                                  int32_t* __restrict__ rank) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  const int t = blockIdx.y;
+  if (j >= K) return;
+  const unsigned long long kj =
+      ~static_cast<unsigned long long>(__double_as_longlong(__ldg(Vc + (size_t)t * K + ptx::perm_at(perm, j, K))));
+  const unsigned ij = (unsigned)j;
+  int r = 0;
+  for (int base = 0; base < Kp; base += kRankChunk) {
+    const unsigned long long* ck = skey + (size_t)t * Kp + base;
+    const unsigned short* ci = sidx + (size_t)t * Kp + base;
+    int lo = 0, hi = kRankChunk;  // count of pairs < (kj, ij) in this sorted chunk
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (pair_less(__ldg(ck + mid), __ldg(ci + mid), kj, ij)) lo = mid + 1;
+      else hi = mid;
+    }
+    r += lo;
+  }
+  rank[(size_t)t * K + j] = r;
+}
+
+size_t rank_scratch_bytes(int M, int K, int T) {
+  const int nt = M / T;
+  const size_t Kp = (size_t)((K + kRankChunk - 1) / kRankChunk) * kRankChunk;
+  Carve c{nullptr, 0};
+  c.take<unsigned long long>((size_t)nt * Kp);
+  c.take<unsigned short>((size_t)nt * Kp);
+  return (c.off + 255) & ~size_t(255);
 }
 
 cudaError_t launch_vector_rank(const float* I, const int32_t* perm, int M, int K, int T,
-                               double* V, int32_t* rank, int* tile_pmax, cudaStream_t s) {
+                               double* V, int32_t* rank, int* tile_pmax, void* scratch,
+                               cudaStream_t s) {
   const int nt = M / T;
   cudaError_t e = cudaMemsetAsync(tile_pmax, 0, (size_t)nt * sizeof(int), s);
   if (e != cudaSuccess) return e;
@@ -183,17 +271,15 @@ cudaError_t launch_vector_rank(const float* I, const int32_t* perm, int M, int K
   vector_score_kernel<<<g1, 256, 0, s>>>(I, K, T, V, tile_pmax);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  int Kp = 1;
-  while (Kp < K) Kp <<= 1;
-  const size_t smem = (size_t)Kp * (sizeof(unsigned long long) + sizeof(unsigned short));
-  static bool attr_set = false;
-  if (!attr_set) {
-    e = cudaFuncSetAttribute(rank_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)((size_t)kMaxK * 10));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  rank_sort_kernel<<<nt, 1024, smem, s>>>(V, perm, K, Kp, rank);
+  const int nchunk = (K + kRankChunk - 1) / kRankChunk;
+  const int Kp = nchunk * kRankChunk;
+  Carve c{static_cast<char*>(scratch), 0};
+  unsigned long long* skey = c.take<unsigned long long>((size_t)nt * Kp);
+  unsigned short* sidx = c.take<unsigned short>((size_t)nt * Kp);
+  chunk_sort_kernel<<<dim3(nchunk, nt), 512, 0, s>>>(V, perm, K, Kp, skey, sidx);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  merge_rank_kernel<<<dim3((K + 255) / 256, nt), 256, 0, s>>>(V, perm, skey, sidx, K, Kp, rank);
   return cudaGetLastError();
 }
 
@@ -256,21 +342,17 @@ struct CandidateList {
   Candidate c[kMaxCandidates];
 };
 
-// blockIdx.x = candidate m, blockIdx.y = tile.  512 threads.
-// R(m) = sum of the column sums of the dense vectors + sum over the 2:4 groups of the
-// top-2 of every row, all exact (128-bit per thread at the tile's scale, exponent buckets
-// for values below it), rounded once to fp64.
-__global__ void __launch_bounds__(512) candidate_kernel(
+// Per (candidate m, tile), 512 threads: the channels of the 2:4 band in ascending working
+// position (block-wide prefix count) -> band[t][m][q], and the exact sum of the dense
+// vectors' column sums -> rdense[t][m] (values below the tile's scale go to the buckets).
+__global__ void __launch_bounds__(512) candidate_lists_kernel(
     const float* __restrict__ I, const int32_t* __restrict__ perm, const int32_t* __restrict__ rank,
     const int* __restrict__ tile_pmax, const U128* __restrict__ colsum,
-    const unsigned char* __restrict__ coltiny, int K, int T, CandidateList cl,
-    double* __restrict__ R, int ncand) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  unsigned long long* bucket = reinterpret_cast<unsigned long long*>(smem);  // [256]
-  unsigned short* member = reinterpret_cast<unsigned short*>(bucket + 256);   // [K]
+    const unsigned char* __restrict__ coltiny, int K, int T, CandidateList cl, int ncand,
+    unsigned short* __restrict__ band, U128* __restrict__ rdense,
+    unsigned long long* __restrict__ bucket, int* __restrict__ bucket_used) {
   __shared__ int warp_tot[16];
   __shared__ U128 warp_acc[16];
-
   const int m = blockIdx.x, t = blockIdx.y;
   const Candidate cand = cl.c[m];
   const int n4 = cand.n4, n24 = cand.n24;
@@ -278,12 +360,10 @@ __global__ void __launch_bounds__(512) candidate_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int lsb = tile_lsb(tile_pmax[t]);
   const float* It = I + (size_t)t * T * K;
-
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) bucket[i] = 0;
+  unsigned long long* bkt = bucket + ((size_t)t * ncand + m) * 256;
+  unsigned short* out = band + ((size_t)t * ncand + m) * K;
   U128 acc{0ull, 0ull};
 
-  // pass over the working positions: dense column sums, and the 2:4 members in
-  // ascending working position (block-wide prefix count)
   const int per = (K + blockDim.x - 1) / blockDim.x;
   const int j0 = threadIdx.x * per, j1 = min(K, j0 + per);
   int cnt = 0;
@@ -297,52 +377,31 @@ __global__ void __launch_bounds__(512) candidate_kernel(
     if (lane >= o) incl += v;
   }
   if (lane == 31) warp_tot[warp] = incl;
-  __syncthreads();  // also publishes the cleared buckets
+  __syncthreads();
   int pos = incl - cnt;
   for (int w = 0; w < warp; ++w) pos += warp_tot[w];
+  bool used = false;
   for (int j = j0; j < j1; ++j) {
     const int r = __ldg(rk + j);
+    const int c = ptx::perm_at(perm, j, K);
     if (r < n4) {
-      const int c = ptx::perm_at(perm, j, K);
       add128(acc, colsum[(size_t)t * K + c]);
       if (coltiny[(size_t)t * K + c]) {  // values below the tile's scale: exact buckets
         for (int i = 0; i < T; ++i) {
           uint32_t mm;
           int e;
           split_f32(__ldg(It + (size_t)i * K + c), mm, e);
-          if (mm && e < lsb) atomicAdd(bucket + e, (unsigned long long)mm);
+          if (mm && e < lsb) {
+            atomicAdd(bkt + e, (unsigned long long)mm);
+            used = true;
+          }
         }
       }
     } else if (r < n4 + n24) {
-      member[pos++] = (unsigned short)j;
+      out[pos++] = (unsigned short)c;
     }
   }
-  __syncthreads();
-
-  // 2:4 groups: the two largest of the four importances of every row are kept (which of
-  // two equal values is kept does not change the sum).  One thread per group walks all
-  // rows, so the group's channels are looked up once.
-  const int ng = n24 / 4;
-  for (int g = threadIdx.x; g < ng; g += blockDim.x) {
-    int c[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      int j = member[4 * g + k];
-      j = j < K ? j : 0;
-      c[k] = ptx::perm_at(perm, j, K);
-    }
-    const float* row = It;
-    for (int i = 0; i < T; ++i, row += K) {
-      const float v0 = __ldg(row + c[0]), v1 = __ldg(row + c[1]);
-      const float v2 = __ldg(row + c[2]), v3 = __ldg(row + c[3]);
-      const float a = fmaxf(v0, v1), b = fminf(v0, v1);
-      const float cc = fmaxf(v2, v3), d = fminf(v2, v3);
-      acc_value(acc, fmaxf(a, cc), lsb, bucket);
-      acc_value(acc, fmaxf(fminf(a, cc), fmaxf(b, d)), lsb, bucket);
-    }
-  }
-
-  // block reduction of the 128-bit partial sums (integer adds: order-independent)
+  if (used) atomicOr(bucket_used + (size_t)t * ncand + m, 1);
   for (int o = 16; o > 0; o >>= 1) {
     U128 other;
     other.lo = __shfl_xor_sync(0xffffffffu, acc.lo, o);
@@ -354,27 +413,195 @@ __global__ void __launch_bounds__(512) candidate_kernel(
   if (threadIdx.x == 0) {
     U128 tot{0ull, 0ull};
     for (int w = 0; w < (int)(blockDim.x >> 5); ++w) add128(tot, warp_acc[w]);
-    R[(size_t)t * ncand + m] = exact_to_double(tot, lsb, bucket);
+    rdense[(size_t)t * ncand + m] = tot;
   }
 }
 
-__global__ void select_kernel(const double* __restrict__ R, int nt, int ncand, CandidateList cl,
-                              double t_s, double alpha, int32_t* __restrict__ counts,
-                              double* __restrict__ vs) {
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= nt) return;
-  const double* r = R + (size_t)t * ncand;
-  int ms = ncand - 1;
-  for (int m = 0; m + 1 < ncand; ++m) {
-    if (r[m + 1] < r[m]) {
-      ms = m;
-      break;
+// An fp64 value as a 128-bit integer in units of 2^(lsb-149); false when it is not a whole
+// number of units (it then holds values below the tile's scale).
+__device__ __forceinline__ bool f64_to_fixed(double s, int lsb, U128& r) {
+  r = U128{0ull, 0ull};
+  if (s == 0.0) return true;
+  const unsigned long long bits = (unsigned long long)__double_as_longlong(s);
+  const unsigned long long m = (bits & 0xFFFFFFFFFFFFFull) | (1ull << 52);
+  const int sh = (int)(bits >> 52) - 926 - lsb;
+  if (sh >= 64) {
+    r.hi = m << (sh - 64);
+  } else if (sh >= 0) {
+    r.lo = m << sh;
+    r.hi = sh ? (m >> (64 - sh)) : 0ull;
+  } else {
+    if (sh <= -53 || (m & ((1ull << (-sh)) - 1ull))) return false;
+    r.lo = m >> (-sh);
+  }
+  return true;
+}
+
+// acc (fp64) += x (fp64 >= 0); err |= the addition rounded (Fast2Sum on max/min).
+__device__ __forceinline__ void add_checked(double& acc, double x, bool& err) {
+  const double a = fmax(acc, x), b = fmin(acc, x);
+  const double s = __dadd_rn(a, b);
+  err |= __dsub_rn(b, __dsub_rn(s, a)) != 0.0;
+  acc = s;
+}
+
+// Per (tile, chunk of RB rows), 512 threads.  The chunk's rows of I are staged in shared
+// memory once; then, candidate by candidate, each thread takes 2:4 groups g = tid,
+// tid + 512, ... and evaluates the top-2 of every row of the chunk.  A thread sums its
+// values in fp64 with every addition checked for rounding: when nothing rounded (and the
+// sum is a whole number of the tile's fixed-point units) the sum is exact; otherwise the
+// same groups are summed again through the exact integer path.  Warps combine their
+// 128-bit partials with shuffles into per-warp slots; one barrier at the end, then
+// part[t][m][chunk] = the CTA's exact total of candidate m.
+__global__ void __launch_bounds__(512) band_sum_kernel(
+    const float* __restrict__ I, const unsigned short* __restrict__ band,
+    const int* __restrict__ tile_pmax, int K, int T, int RB, CandidateList cl, int ncand,
+    U128* __restrict__ part, unsigned long long* __restrict__ bucket,
+    int* __restrict__ bucket_used) {
+  extern __shared__ __align__(16) float rows_s[];  // [RB][K]
+  // per candidate, the CTA's total as four 32-bit digits held in 64-bit words
+  __shared__ unsigned long long digits[kMaxCandidates][4];
+  const int chunk = blockIdx.x, t = blockIdx.y;
+  const int nchunks = gridDim.x;
+  const int lane = threadIdx.x & 31;
+  for (int x = threadIdx.x; x < kMaxCandidates * 4; x += blockDim.x) (&digits[0][0])[x] = 0ull;
+  const int lsb = tile_lsb(tile_pmax[t]);
+  const float4* src = reinterpret_cast<const float4*>(I + ((size_t)t * T + (size_t)chunk * RB) * K);
+  for (int x = threadIdx.x; x < RB * K / 4; x += blockDim.x)
+    reinterpret_cast<float4*>(rows_s)[x] = __ldg(src + x);
+  __syncthreads();
+
+  for (int m = 0; m < ncand; ++m) {
+    const int ng = cl.c[m].n24 / 4;
+    const unsigned short* bl = band + ((size_t)t * ncand + m) * K;
+    unsigned long long* bkt = bucket + ((size_t)t * ncand + m) * 256;
+    U128 ex{0ull, 0ull};
+    if ((int)threadIdx.x < ng) {
+      // pass 1: checked fp64
+      double acc = 0.0;
+      bool err = false;
+      for (int g = threadIdx.x; g < ng; g += blockDim.x) {
+        const ushort4 cq = __ldg(reinterpret_cast<const ushort4*>(bl) + g);
+        const int c0 = min((int)cq.x, K - 1), c1 = min((int)cq.y, K - 1);
+        const int c2 = min((int)cq.z, K - 1), c3 = min((int)cq.w, K - 1);
+        for (int r = 0; r < RB; ++r) {
+          const float* row = rows_s + r * K;
+          const float v0 = row[c0], v1 = row[c1], v2 = row[c2], v3 = row[c3];
+          const float a = fmaxf(v0, v1), b = fminf(v0, v1);
+          const float cc = fmaxf(v2, v3), d = fminf(v2, v3);
+          const float t1 = fmaxf(a, cc), t2 = fmaxf(fminf(a, cc), fmaxf(b, d));
+          const double p = __dadd_rn((double)t1, (double)t2);  // Fast2Sum, t1 >= t2
+          err |= __dsub_rn((double)t2, __dsub_rn(p, (double)t1)) != 0.0;
+          add_checked(acc, p, err);
+        }
+      }
+      if (!err && !f64_to_fixed(acc, lsb, ex)) err = true;
+      if (err) {
+        // pass 2: exact integers (values below the tile's scale into the buckets)
+        ex = U128{0ull, 0ull};
+        bool used = false;
+        for (int g = threadIdx.x; g < ng; g += blockDim.x) {
+          const ushort4 cq = __ldg(reinterpret_cast<const ushort4*>(bl) + g);
+          const int c0 = min((int)cq.x, K - 1), c1 = min((int)cq.y, K - 1);
+          const int c2 = min((int)cq.z, K - 1), c3 = min((int)cq.w, K - 1);
+          for (int r = 0; r < RB; ++r) {
+            const float* row = rows_s + r * K;
+            const float v0 = row[c0], v1 = row[c1], v2 = row[c2], v3 = row[c3];
+            const float a = fmaxf(v0, v1), b = fminf(v0, v1);
+            const float cc = fmaxf(v2, v3), d = fminf(v2, v3);
+            const float tv[2] = {fmaxf(a, cc), fmaxf(fminf(a, cc), fmaxf(b, d))};
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              uint32_t mm;
+              int e;
+              split_f32(tv[q], mm, e);
+              if (!mm) continue;
+              if (e >= lsb) {
+                add_shifted(ex, mm, e - lsb);
+              } else {
+                atomicAdd(bkt + e, (unsigned long long)mm);
+                used = true;
+              }
+            }
+          }
+        }
+        if (used) atomicOr(bucket_used + (size_t)t * ncand + m, 1);
+      }
+    }
+    __syncwarp();
+    for (int o = 16; o > 0; o >>= 1) {
+      U128 other;
+      other.lo = __shfl_xor_sync(0xffffffffu, ex.lo, o);
+      other.hi = __shfl_xor_sync(0xffffffffu, ex.hi, o);
+      add128(ex, other);
+    }
+    if (lane == 0 && (ex.lo | ex.hi)) {
+      atomicAdd(&digits[m][0], ex.lo & 0xFFFFFFFFull);
+      atomicAdd(&digits[m][1], ex.lo >> 32);
+      atomicAdd(&digits[m][2], ex.hi & 0xFFFFFFFFull);
+      atomicAdd(&digits[m][3], ex.hi >> 32);
     }
   }
-  counts[3 * t + 0] = cl.c[ms].n0;
-  counts[3 * t + 1] = cl.c[ms].n24;
-  counts[3 * t + 2] = cl.c[ms].n4;
-  vs[t] = __dsub_rn(t_s, __dmul_rn((double)ms, alpha));
+  __syncthreads();
+  if ((int)threadIdx.x < ncand) {
+    // fold the digits' carries (each digit word is below 2^37: at most 16 warps add)
+    const unsigned long long* d = digits[threadIdx.x];
+    const unsigned long long d0 = d[0];
+    const unsigned long long d1 = d[1] + (d0 >> 32);
+    const unsigned long long d2 = d[2] + (d1 >> 32);
+    const unsigned long long d3 = d[3] + (d2 >> 32);
+    U128 tot;
+    tot.lo = (d0 & 0xFFFFFFFFull) | (d1 << 32);
+    tot.hi = (d2 & 0xFFFFFFFFull) | (d3 << 32);
+    part[((size_t)t * ncand + threadIdx.x) * nchunks + chunk] = tot;
+  }
+}
+
+// Per tile, one thread per candidate: R(m) = exact total rounded once to fp64; then the
+// first m with R(m+1) < R(m) (else the last candidate) gives the counts and v_s.
+__global__ void finalize_kernel(const U128* __restrict__ rdense, const U128* __restrict__ part,
+                                int nchunks, const unsigned long long* __restrict__ bucket,
+                                const int* __restrict__ bucket_used,
+                                const int* __restrict__ tile_pmax, int ncand, CandidateList cl,
+                                double t_s, double alpha, double* __restrict__ R,
+                                int32_t* __restrict__ counts, double* __restrict__ vs) {
+  __shared__ double Rs[kMaxCandidates];
+  __shared__ unsigned long long zero_bkt[256];
+  const int t = blockIdx.x, m = threadIdx.x;
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) zero_bkt[i] = 0ull;
+  __syncthreads();
+  if (m < ncand) {
+    const size_t tm = (size_t)t * ncand + m;
+    U128 tot = rdense[tm];
+    for (int c = 0; c < nchunks; ++c) add128(tot, part[tm * nchunks + c]);
+    const unsigned long long* bk = bucket_used[tm] ? bucket + tm * 256 : zero_bkt;
+    const double r = exact_to_double(tot, tile_lsb(tile_pmax[t]), bk);
+    Rs[m] = r;
+    R[tm] = r;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ms = ncand - 1;
+    for (int k = 0; k + 1 < ncand; ++k) {
+      if (Rs[k + 1] < Rs[k]) {
+        ms = k;
+        break;
+      }
+    }
+    counts[3 * t + 0] = cl.c[ms].n0;
+    counts[3 * t + 1] = cl.c[ms].n24;
+    counts[3 * t + 2] = cl.c[ms].n4;
+    vs[t] = __dsub_rn(t_s, __dmul_rn((double)ms, alpha));
+  }
+}
+
+// Rows per band_sum CTA: the largest power of two <= 8 whose rows fit in ~96 KB of shared
+// memory, so that two CTAs share an SM (T is a multiple of it).  Wider rows (K > 24576)
+// would need one row of more than 96 KB; K is at most 16384.
+static int band_rows(int K) {
+  int rb = 8;
+  while (rb > 1 && (size_t)rb * K * sizeof(float) > 96u * 1024u) rb >>= 1;
+  return rb;
 }
 
 size_t search_workspace_bytes(int M, int K, int T, int ncand) {
@@ -386,6 +613,13 @@ size_t search_workspace_bytes(int M, int K, int T, int ncand) {
   c.take<int>((size_t)nt);                // tile max exponent
   c.take<U128>((size_t)nt * K);           // exact column sums
   c.take<unsigned char>((size_t)nt * K);  // column has values below the tile scale
+  c.take<char>(rank_scratch_bytes(M, K, T));  // chunk-sorted keys for the ranking
+  const int nchunks = T / band_rows(K);
+  c.take<unsigned short>((size_t)nt * ncand * K);      // band channel lists
+  c.take<U128>((size_t)nt * ncand);                    // dense exact sums
+  c.take<U128>((size_t)nt * ncand * nchunks);          // 2:4 partial sums per row chunk
+  c.take<unsigned long long>((size_t)nt * ncand * 256);  // exponent buckets
+  c.take<int>((size_t)nt * ncand);                     // buckets used
   return (c.off + 255) & ~size_t(255);
 }
 
@@ -403,8 +637,9 @@ cudaError_t launch_boundary_search(const float* I, const int32_t* perm, int M, i
   int* pmax = c.take<int>((size_t)nt);
   U128* colsum = c.take<U128>((size_t)nt * K);
   unsigned char* coltiny = c.take<unsigned char>((size_t)nt * K);
+  char* rank_scratch = c.take<char>(rank_scratch_bytes(M, K, T));
   int32_t* rank = rank_out ? rank_out : rank_ws;
-  cudaError_t e = launch_vector_rank(I, perm, M, K, T, V, rank, pmax, s);
+  cudaError_t e = launch_vector_rank(I, perm, M, K, T, V, rank, pmax, rank_scratch, s);
   if (e != cudaSuccess) return e;
   dim3 gc((K + 255) / 256, nt);
   column_sum_kernel<<<gc, 256, 0, s>>>(I, K, T, pmax, colsum, coltiny);
@@ -412,19 +647,36 @@ cudaError_t launch_boundary_search(const float* I, const int32_t* perm, int M, i
   if (e != cudaSuccess) return e;
   CandidateList cl;
   for (int i = 0; i < kMaxCandidates; ++i) cl.c[i] = i < ncand ? cands[i] : Candidate{0, 0, 0};
-  const size_t smem = 256 * sizeof(unsigned long long) + (size_t)K * sizeof(unsigned short);
+  const int RB = band_rows(K);
+  const int nchunks = T / RB;
+  unsigned short* band = c.take<unsigned short>((size_t)nt * ncand * K);
+  U128* rdense = c.take<U128>((size_t)nt * ncand);
+  U128* part = c.take<U128>((size_t)nt * ncand * nchunks);
+  unsigned long long* bucket = c.take<unsigned long long>((size_t)nt * ncand * 256);
+  int* bucket_used = c.take<int>((size_t)nt * ncand);
+  e = cudaMemsetAsync(bucket, 0, (size_t)nt * ncand * 256 * sizeof(unsigned long long), s);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(bucket_used, 0, (size_t)nt * ncand * sizeof(int), s);
+  if (e != cudaSuccess) return e;
+  candidate_lists_kernel<<<dim3(ncand, nt), 512, 0, s>>>(I, perm, rank, pmax, colsum, coltiny, K, T,
+                                                         cl, ncand, band, rdense, bucket,
+                                                         bucket_used);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem = (size_t)RB * K * sizeof(float);
   static bool attr_set = false;
   if (!attr_set) {
-    e = cudaFuncSetAttribute(candidate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(256 * sizeof(unsigned long long) + kMaxK * 2));
+    e = cudaFuncSetAttribute(band_sum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             96 * 1024);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  dim3 g(ncand, nt);
-  candidate_kernel<<<g, 512, smem, s>>>(I, perm, rank, pmax, colsum, coltiny, K, T, cl, R, ncand);
+  band_sum_kernel<<<dim3(nchunks, nt), 512, smem, s>>>(I, band, pmax, K, T, RB, cl, ncand, part,
+                                                       bucket, bucket_used);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  select_kernel<<<(nt + 127) / 128, 128, 0, s>>>(R, nt, ncand, cl, t_s, alpha, counts_out, vs_out);
+  finalize_kernel<<<nt, 64, 0, s>>>(rdense, part, nchunks, bucket, bucket_used, pmax, ncand, cl,
+                                    t_s, alpha, R, counts_out, vs_out);
   return cudaGetLastError();
 }
 

@@ -232,3 +232,28 @@ def test_full_size_sampled(H, name, make, v_s):
     layout_equal(hp.layout, L_ref, tiles=tiles)
     y_ref, bound = O.spmm_reference(w.W_bits, bm_ref, w.X_bits, rows=rows)
     check_y(Y.cpu().numpy(), y_ref, bound, rows=rows)
+
+
+def test_extreme_dynamic_range_exact_sums(H):
+    """Importances spanning more than 2^83 within a tile (weights near 1e-20 give fp32
+    subnormal importances): the values below the tile's fixed-point window take the exact
+    exponent-bucket path, and R(m), counts, rank and mask still match the oracle bit for bit."""
+    rng = np.random.default_rng(5)
+    M, K, N, T = 256, 256, 16, 128
+    scale = np.where(rng.random(K) < 0.3, 1e-20, 1.0).astype(np.float32)
+    Wf = (rng.standard_normal((M, K)).astype(np.float32) * scale[None, :])
+    Wf[:, :8] *= np.float32(1e-19)  # a few columns entirely in the tiny range
+    w = hi.Workload(name="extreme", M=M, K=K, N=N, T=T, W_bits=hi.f32_to_bf16_bits(Wf),
+                    X_bits=hi.f32_to_bf16_bits(rng.standard_normal((K, N)).astype(np.float32)),
+                    perm=rng.permutation(K).astype(np.int32), t_s=0.5, v_s=None)
+    g = run_path(H, w, None)
+    I_ref = O.importance(w.W_bits, w.X_bits)
+    np.testing.assert_array_equal(g["I"].view(np.uint32), I_ref.view(np.uint32))
+    nz = I_ref[I_ref > 0].astype(np.float64)
+    assert np.log2(nz.max() / nz.min()) > 100   # really exercises the bucket path
+    sr = O.boundary_search(I_ref, w.perm, T, w.t_s, w.alpha)
+    np.testing.assert_array_equal(g["R"], np.array(sr.R))
+    np.testing.assert_array_equal(g["counts"], sr.counts)
+    np.testing.assert_array_equal(g["rank"], sr.rank)
+    bm_ref, reg_ref = O.mask(I_ref, w.perm, T, sr.counts)
+    np.testing.assert_array_equal(g["bitmask"], bm_ref)
