@@ -87,6 +87,21 @@ hinm_status hinm_importance(const void* W, const void* X, int M, int K, int N,
                             float* I_out, void* workspace, size_t workspace_bytes,
                             void* stream);
 
+/* Workspace-free variant of hinm_importance.  The method's description has no counterpart:
+ * this is a deployment convenience for callers that cannot hand the library memory.
+ *   Same arguments, layout and result as hinm_importance, without the workspace.  The
+ *   channel energies s live in a static per-device array of the library (16384 fp32,
+ *   64 KiB); K > 16384 returns HINM_ERR_SHAPE.  The call allocates nothing (no
+ *   cudaMalloc / cudaFree, no allocating library routine).  Nothing in the scratch has
+ *   to start at zero: every s_c is written before it is read, in stream order.
+ *   Calls that overlap on one device (other streams or host threads) share the scratch
+ *   and race: order them.  The first call on each device resolves the scratch address
+ *   (cudaGetSymbolAddress, device current); make that call before any stream capture.
+ *   Errors: as hinm_importance, plus HINM_ERR_CUDA if the address cannot be resolved.
+ */
+hinm_status hinm_importance_noalloc(const void* W, const void* X, int M, int K, int N,
+                                    float* I_out, void* stream);
+
 /* ---------------------------------------------------------------------------------
  * Region counts for a fixed boundary (host only).  ([P1] 关键设计 1, closed form)
  *   n_24 = 4 * floor(2 (t_s - v_s) K / 4 + 1/2), n_0 = t_s K - n_24 / 2,

@@ -61,6 +61,7 @@ _SIGS = {
     "hinm_abi_version": (_i32, []),
     "hinm_importance_workspace_size": (_i32, [_i32, _i32, _i32, _szp]),
     "hinm_importance": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _sz, _vp]),
+    "hinm_importance_noalloc": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp]),
     "hinm_counts_from_vs": (_i32, [_i32, _f64, _f64, ctypes.POINTER(ctypes.c_int32)]),
     "hinm_search_num_candidates": (_i32, [_i32, _f64, _f64, ctypes.POINTER(ctypes.c_int32)]),
     "hinm_search_workspace_size": (_i32, [_i32, _i32, _i32, _f64, _f64, _szp]),
@@ -136,6 +137,16 @@ def hinm_importance(W, X, I_out=None, workspace=None, stream=None):
         workspace = _empty_bytes(_size(_lib.hinm_importance_workspace_size, M, K, N), W.device)
     _check(_lib.hinm_importance(_ptr(W), _ptr(X), M, K, N, _ptr(I_out), _ptr(workspace),
                                 workspace.numel(), _stream(stream)), "hinm_importance")
+    return I_out
+
+
+def hinm_importance_noalloc(W, X, I_out, stream=None):
+    """hinm_importance with its scratch in the library's static per-device array
+    (K <= 16384; overlapping calls on one device race).  I_out is caller-provided."""
+    M, K = W.shape
+    N = X.shape[1]
+    _check(_lib.hinm_importance_noalloc(_ptr(W), _ptr(X), M, K, N, _ptr(I_out),
+                                        _stream(stream)), "hinm_importance_noalloc")
     return I_out
 
 

@@ -199,6 +199,27 @@ hinm_status hinm_importance(const void* W, const void* X, int M, int K, int N, f
   return ok();
 }
 
+hinm_status hinm_importance_noalloc(const void* W, const void* X, int M, int K, int N,
+                                    float* I_out, void* stream) {
+  REQUIRE_PTR(W);
+  REQUIRE_PTR(X);
+  REQUIRE_PTR(I_out);
+  if (M <= 0 || K <= 0 || K % 4 != 0 || (long long)M * K >= (1ll << 31))
+    return fail(HINM_ERR_SHAPE, "M=%d, K=%d: need M > 0 and K a positive multiple of 4", M, K);
+  if (K > hinm::kNoAllocMaxK)
+    return fail(HINM_ERR_SHAPE, "K=%d exceeds the static scratch (%d channels)", K,
+                hinm::kNoAllocMaxK);
+  hinm_status st = check_n(N);
+  if (st != HINM_OK) return st;
+  float* scratch = nullptr;
+  cudaError_t e = hinm::noalloc_energy_scratch(&scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "hinm_importance_noalloc scratch address");
+  e = hinm::launch_importance(static_cast<const uint16_t*>(W), static_cast<const uint16_t*>(X),
+                              M, K, N, I_out, scratch, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "hinm_importance_noalloc launch");
+  return ok();
+}
+
 hinm_status hinm_search_num_candidates(int K, double t_s, double alpha, int32_t* n_host) {
   if (!n_host) return fail(HINM_ERR_INVALID_ARG, "n_host is NULL");
   if (K < 4 || K > hinm::kMaxK) return fail(HINM_ERR_SHAPE, "K=%d out of range", K);

@@ -52,6 +52,11 @@ size_t importance_workspace_bytes(int K);
 cudaError_t launch_importance(const uint16_t* W, const uint16_t* X, int M, int K, int N,
                               float* I, float* s_scratch, cudaStream_t s);
 
+// Workspace-free variant: channel energies in a static per-device array of kNoAllocMaxK
+// floats (64 KiB).
+constexpr int kNoAllocMaxK = 16384;
+cudaError_t noalloc_energy_scratch(float** out);
+
 size_t search_workspace_bytes(int M, int K, int T, int ncand);
 cudaError_t launch_boundary_search(const float* I, const int32_t* perm, int M, int K, int T,
                                    double t_s, double alpha, const Candidate* cands, int ncand,

@@ -7,6 +7,8 @@
 // per thread with 8-byte loads and 16-byte stores, grid-stride over the matrix.
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "hinm_internal.h"
 
 namespace hinm {
@@ -89,7 +91,35 @@ int sm_count() {
   return n;
 }
 
+// Scratch of the workspace-free entry point: the channel energies s_c of one call.  One copy
+// per device; nothing in it has to start at zero (channel_energy_kernel writes s_c for every
+// c < K before importance_kernel reads it, in stream order).
+static __device__ __align__(256) float g_noalloc_energy[kNoAllocMaxK];
+
+constexpr int kMaxNoAllocDevices = 64;
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[kMaxNoAllocDevices] = {};
+
 }  // namespace
+
+// Address of this device's static scratch, resolved once per device (the caller's current
+// device is the one the call runs on).
+cudaError_t noalloc_energy_scratch(float** out) {
+  *out = nullptr;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxNoAllocDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_energy);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return cudaSuccess;
+}
 
 size_t importance_workspace_bytes(int K) { return ((size_t)K * sizeof(float) + 255) & ~size_t(255); }
 
