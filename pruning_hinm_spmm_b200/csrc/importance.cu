@@ -18,45 +18,68 @@ __device__ __forceinline__ double bf16_to_f64(uint32_t bits16) {
   return static_cast<double>(__uint_as_float(bits16 << 16));
 }
 
-// One thread per channel c: sequential fp64 sum over n = 0..N-1 (N % 8 == 0).  Up to 8
-// 16-byte loads are in flight before they are summed, in order.
-__global__ void channel_energy_kernel(const uint16_t* __restrict__ X, int K, int N,
-                                      float* __restrict__ s) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= K) return;
-  const uint4* row = reinterpret_cast<const uint4*>(X + (size_t)c * N);
+// One CTA per 32 channels.  The order of the sum is fixed (n ascending, one fp64 chain per
+// channel), so the sum itself cannot be split; what is parallel is the loading.  All 128
+// threads stage [32 channels x 256 values] chunks of X into shared memory with 16-byte
+// cp.async, double-buffered, while warp 0 runs the 32 chains over the previous chunk
+// (lane = channel; rows padded by 16 bytes so the 16-byte reads are conflict-free).
+constexpr int kEnergyChannels = 32;
+constexpr int kEnergyChunk = 256;                      // values per channel per chunk
+constexpr int kEnergyRowBytes = kEnergyChunk * 2 + 16;  // padded row
+constexpr int kEnergyThreads = 128;
+
+__device__ __forceinline__ void energy_cp16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__global__ void __launch_bounds__(kEnergyThreads) channel_energy_kernel(
+    const uint16_t* __restrict__ X, int K, int N, float* __restrict__ s) {
+  __shared__ __align__(16) uint8_t buf[2][kEnergyChannels * kEnergyRowBytes];
+  const int c0 = blockIdx.x * kEnergyChannels;
+  const int nch = min(kEnergyChannels, K - c0);
+  const int nchunks = (N + kEnergyChunk - 1) / kEnergyChunk;
+  constexpr int kPieces = kEnergyChunk / 8;  // 16-byte pieces per channel per chunk
+
+  auto stage = [&](int chunk, int b) {
+    const int n0 = chunk * kEnergyChunk;
+    const int pieces = min(kPieces, (N - n0) / 8);
+    const uint32_t base = (uint32_t)__cvta_generic_to_shared(buf[b]);
+    for (int q = threadIdx.x; q < kEnergyChannels * kPieces; q += kEnergyThreads) {
+      const int ch = q / kPieces, p = q - ch * kPieces;
+      if (ch < nch && p < pieces)
+        energy_cp16(base + ch * kEnergyRowBytes + p * 16, X + (size_t)(c0 + ch) * N + n0 + p * 8);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+
   double acc = 0.0;
-  const int nv = N / 8;
-  constexpr int kBatch = 8;
-  int v0 = 0;
-  for (; v0 + kBatch <= nv; v0 += kBatch) {
-    uint4 q[kBatch];
+  stage(0, 0);
+  for (int chunk = 0; chunk < nchunks; ++chunk) {
+    if (chunk + 1 < nchunks) {
+      stage(chunk + 1, (chunk + 1) & 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x < nch) {
+      const int vals = min(kEnergyChunk, N - chunk * kEnergyChunk);
+      const uint4* row = reinterpret_cast<const uint4*>(buf[chunk & 1] + threadIdx.x * kEnergyRowBytes);
+      for (int v = 0; v < vals / 8; ++v) {
+        const uint4 q = row[v];
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-    for (int k = 0; k < kBatch; ++k) q[k] = __ldg(row + v0 + k);
-#pragma unroll
-    for (int k = 0; k < kBatch; ++k) {
-      const uint32_t w[4] = {q[k].x, q[k].y, q[k].z, q[k].w};
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const double a = bf16_to_f64(w[h] & 0xFFFFu);
-        const double b = bf16_to_f64(w[h] >> 16);
-        acc = __dadd_rn(acc, __dmul_rn(a, a));  // x^2 of a bf16 is exact in fp64
-        acc = __dadd_rn(acc, __dmul_rn(b, b));
+        for (int h = 0; h < 4; ++h) {
+          const double a = bf16_to_f64(w[h] & 0xFFFFu);
+          const double b = bf16_to_f64(w[h] >> 16);
+          acc = __dadd_rn(acc, __dmul_rn(a, a));  // x^2 of a bf16 is exact in fp64
+          acc = __dadd_rn(acc, __dmul_rn(b, b));
+        }
       }
     }
+    __syncthreads();  // buffer (chunk & 1) is refilled by the next iteration's stage()
   }
-  for (; v0 < nv; ++v0) {
-    const uint4 q = __ldg(row + v0);
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const double a = bf16_to_f64(w[h] & 0xFFFFu);
-      const double b = bf16_to_f64(w[h] >> 16);
-      acc = __dadd_rn(acc, __dmul_rn(a, a));
-      acc = __dadd_rn(acc, __dmul_rn(b, b));
-    }
-  }
-  s[c] = __double2float_rn(acc);
+  if (threadIdx.x < nch) s[c0 + threadIdx.x] = __double2float_rn(acc);
 }
 
 // 4 consecutive elements of one row per thread (K % 4 == 0).
@@ -125,7 +148,8 @@ size_t importance_workspace_bytes(int K) { return ((size_t)K * sizeof(float) + 2
 
 cudaError_t launch_importance(const uint16_t* W, const uint16_t* X, int M, int K, int N,
                               float* I, float* s_scratch, cudaStream_t st) {
-  channel_energy_kernel<<<(K + 63) / 64, 64, 0, st>>>(X, K, N, s_scratch);
+  channel_energy_kernel<<<(K + kEnergyChannels - 1) / kEnergyChannels, kEnergyThreads, 0, st>>>(
+      X, K, N, s_scratch);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const long long total4 = (long long)M * K / 4;

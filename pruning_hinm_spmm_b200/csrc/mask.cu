@@ -97,29 +97,64 @@ __global__ void __launch_bounds__(1024) classify_kernel(const int32_t* __restric
   }
 }
 
-// One CTA per (tile, kMaskRows rows): the rows' mask words are assembled in shared memory.
-// Dense bits are the same in every row of the tile (one ballot per word over the region
-// array); each 2:4 group is handled by one thread for all the CTA's rows.
-constexpr int kMaskRows = 16;
+// One CTA per (tile, RB rows).  The rows of I are staged channel-major in shared memory
+// (the RB values of channel c contiguous).  keep[c] holds one bit per row: all ones for a
+// dense channel, zero for a pruned one, and for a 2:4 channel the rows where it is among
+// the top 2 of its group (ties: the lower working position wins).  Each channel belongs
+// to one group, so every keep byte has one writer.  The mask words are then assembled by
+// warp ballots, 32 words per warp and row, and stored coalesced.
+constexpr int kMaskThreads = 256;
 
-__global__ void __launch_bounds__(256) bitmask_kernel(
+template <int RB>
+__device__ __forceinline__ void mask_load_rows(const float* p, float (&v)[RB]) {
+  if constexpr (RB == 8) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0];
+    const float4 b = reinterpret_cast<const float4*>(p)[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else if constexpr (RB == 4) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  } else if constexpr (RB == 2) {
+    const float2 a = *reinterpret_cast<const float2*>(p);
+    v[0] = a.x; v[1] = a.y;
+  } else {
+    v[0] = *p;
+  }
+}
+
+template <int RB>
+__global__ void __launch_bounds__(kMaskThreads) bitmask_kernel(
     const float* __restrict__ I, const int32_t* __restrict__ perm,
     const int8_t* __restrict__ region, const int32_t* __restrict__ counts,
-    const int32_t* __restrict__ member, int M, int K, int T, uint32_t* __restrict__ bitmask) {
-  extern __shared__ uint32_t words_s[];  // [kMaskRows][words]
+    const int32_t* __restrict__ member, int K, int T, uint32_t* __restrict__ bitmask) {
+  extern __shared__ __align__(16) uint8_t mask_smem[];
+  float* rows_s = reinterpret_cast<float*>(mask_smem);  // [K][RB]
+  uint8_t* keep = mask_smem + (size_t)K * RB * sizeof(float);
   const int words = (K + 31) >> 5;
   const int t = blockIdx.y;
-  const int r0 = blockIdx.x * kMaskRows;  // first row of the chunk within the tile
-  const int rows = min(kMaskRows, T - r0);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int r0 = blockIdx.x * RB;  // first row of the chunk within the tile
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int nwarps = kMaskThreads / 32;
   const int8_t* reg = region + (size_t)t * K;
-
-  // dense bits: warp per word, lane = bit
-  for (int w = warp; w < words; w += nwarps) {
-    const int c = w * 32 + lane;
-    const bool dense = c < K && __ldg(reg + c) == HINM_REGION_DENSE;
-    const uint32_t bits = __ballot_sync(0xffffffffu, dense);
-    if (lane < rows) words_s[lane * words + w] = bits;
+  const float* src = I + ((size_t)t * T + r0) * K;
+  constexpr uint8_t kAll = (uint8_t)((1u << RB) - 1u);
+  for (int c = threadIdx.x; c < K; c += kMaskThreads) {
+    float v[RB];
+#pragma unroll
+    for (int r = 0; r < RB; ++r) v[r] = __ldg(src + (size_t)r * K + c);
+    float* d = rows_s + (size_t)c * RB;
+    if constexpr (RB == 8) {
+      reinterpret_cast<float4*>(d)[0] = make_float4(v[0], v[1], v[2], v[3]);
+      reinterpret_cast<float4*>(d)[1] = make_float4(v[4], v[5], v[6], v[7]);
+    } else if constexpr (RB == 4) {
+      *reinterpret_cast<float4*>(d) = make_float4(v[0], v[1], v[2], v[3]);
+    } else if constexpr (RB == 2) {
+      *reinterpret_cast<float2*>(d) = make_float2(v[0], v[1]);
+    } else {
+      d[0] = v[0];
+    }
+    keep[c] = __ldg(reg + c) == HINM_REGION_DENSE ? kAll : (uint8_t)0;
   }
   __syncthreads();
 
@@ -128,38 +163,65 @@ __global__ void __launch_bounds__(256) bitmask_kernel(
   if (n0 < 0 || n24 < 0 || n4 < 0 || n0 + n24 + n4 != K || (n24 & 3)) n24 = 0;
   const int ng = n24 / 4;
   const int32_t* mem = member + (size_t)t * K;
-  const float* I0 = I + ((size_t)t * T + r0) * K;
-  for (int g = threadIdx.x; g < ng; g += blockDim.x) {
+  for (int g = threadIdx.x; g < ng; g += kMaskThreads) {
+    const int4 jq = __ldg(reinterpret_cast<const int4*>(mem) + g);
+    const int jj[4] = {jq.x, jq.y, jq.z, jq.w};
     int c[4];
+    float v[4][RB];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      int j = __ldg(mem + 4 * g + k);
-      j = ((unsigned)j < (unsigned)K) ? j : 0;  // never index outside perm / I
+      const int j = ((unsigned)jj[k] < (unsigned)K) ? jj[k] : 0;  // never index outside perm / I
       c[k] = ptx::perm_at(perm, j, K);
+      mask_load_rows<RB>(rows_s + (size_t)c[k] * RB, v[k]);
     }
-    const float* row = I0;
-#pragma unroll 4
-    for (int r = 0; r < rows; ++r, row += K) {
-      float v[4];
+    uint32_t kb[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-      for (int k = 0; k < 4; ++k) v[k] = __ldg(row + c[k]);
+    for (int r = 0; r < RB; ++r) {
       // beats[k]: members ranked above k (greater value, or equal value at a lower position)
       int beats[4] = {0, 0, 0, 0};
 #pragma unroll
       for (int k = 0; k < 4; ++k)
 #pragma unroll
         for (int l = k + 1; l < 4; ++l) {
-          if (v[l] > v[k]) ++beats[k];
+          if (v[l][r] > v[k][r]) ++beats[k];
           else ++beats[l];  // v[k] >= v[l]: k (lower position) ranks above l
         }
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        if (beats[k] < 2) atomicOr(words_s + r * words + (c[k] >> 5), 1u << (c[k] & 31));
+      for (int k = 0; k < 4; ++k) kb[k] |= (beats[k] < 2 ? 1u : 0u) << r;
     }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) keep[c[k]] = (uint8_t)kb[k];
   }
   __syncthreads();
+
   uint32_t* out = bitmask + ((size_t)t * T + r0) * words;
-  for (int x = threadIdx.x; x < rows * words; x += blockDim.x) out[x] = words_s[x];
+  for (int wb = warp * 32; wb < words; wb += nwarps * 32) {
+    uint32_t mine[RB];
+#pragma unroll
+    for (int r = 0; r < RB; ++r) mine[r] = 0u;
+    const int nw = min(32, words - wb);
+    for (int i = 0; i < nw; ++i) {
+      const int c = (wb + i) * 32 + lane;
+      const uint32_t kbyte = c < K ? keep[c] : 0u;
+#pragma unroll
+      for (int r = 0; r < RB; ++r) {
+        const uint32_t bits = __ballot_sync(0xffffffffu, (kbyte >> r) & 1u);
+        if (lane == i) mine[r] = bits;
+      }
+    }
+    if (lane < nw) {
+#pragma unroll
+      for (int r = 0; r < RB; ++r) out[(size_t)r * words + wb + lane] = mine[r];
+    }
+  }
+}
+
+// Rows per bitmask CTA: the largest power of two <= 8 whose rows fit in 64 KB of shared
+// memory (T is a multiple of it).
+static int mask_rows(int K) {
+  int rb = 8;
+  while (rb > 1 && (size_t)rb * K * sizeof(float) > 64u * 1024u) rb >>= 1;
+  return rb;
 }
 
 size_t mask_workspace_bytes(int M, int K, int T) {
@@ -199,17 +261,26 @@ cudaError_t launch_mask(const float* I, const int32_t* perm, const int32_t* coun
   classify_kernel<<<nt, 1024, 0, s>>>(rank, perm, counts, K, region, member, status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int words = (K + 31) / 32;
-  const size_t smem = (size_t)kMaskRows * words * sizeof(uint32_t);
+  const int RB = mask_rows(K);
+  const size_t smem = (size_t)RB * K * sizeof(float) + (size_t)K;
   static bool attr_set = false;
   if (!attr_set) {
-    e = cudaFuncSetAttribute(bitmask_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(kMaskRows * ((kMaxK + 31) / 32) * sizeof(uint32_t)));
-    if (e != cudaSuccess) return e;
+    for (auto fn : {bitmask_kernel<1>, bitmask_kernel<2>, bitmask_kernel<4>, bitmask_kernel<8>}) {
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               64 * 1024 + kMaxK);
+      if (e != cudaSuccess) return e;
+    }
     attr_set = true;
   }
-  dim3 g((T + kMaskRows - 1) / kMaskRows, nt);
-  bitmask_kernel<<<g, 256, smem, s>>>(I, perm, region, counts, member, M, K, T, bitmask);
+  const dim3 g(T / RB, nt);
+  if (RB == 8)
+    bitmask_kernel<8><<<g, kMaskThreads, smem, s>>>(I, perm, region, counts, member, K, T, bitmask);
+  else if (RB == 4)
+    bitmask_kernel<4><<<g, kMaskThreads, smem, s>>>(I, perm, region, counts, member, K, T, bitmask);
+  else if (RB == 2)
+    bitmask_kernel<2><<<g, kMaskThreads, smem, s>>>(I, perm, region, counts, member, K, T, bitmask);
+  else
+    bitmask_kernel<1><<<g, kMaskThreads, smem, s>>>(I, perm, region, counts, member, K, T, bitmask);
   return cudaGetLastError();
 }
 

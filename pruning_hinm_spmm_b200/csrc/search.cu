@@ -183,73 +183,82 @@ __device__ __forceinline__ bool pair_less(unsigned long long ka, unsigned ia,
   return ka < kb || (ka == kb && ia < ib);
 }
 
-__global__ void __launch_bounds__(512) chunk_sort_kernel(const double* __restrict__ Vc,
-                                                         const int32_t* __restrict__ perm, int K,
-                                                         int Kp, unsigned long long* __restrict__ skey,
-                                                         unsigned short* __restrict__ sidx) {
-  __shared__ unsigned long long key[kRankChunk];
-  __shared__ unsigned short idx[kRankChunk];
+// Sorts one chunk of kRankChunk working positions of one tile by (key, index) ascending:
+// a bitonic network with one element per thread; compare-exchange stages with partner
+// distance < 32 run on warp shuffles, the wider ones through shared memory.
+__global__ void __launch_bounds__(kRankChunk) chunk_sort_kernel(
+    const double* __restrict__ Vc, const int32_t* __restrict__ perm, int K, int Kp,
+    unsigned long long* __restrict__ skey, unsigned short* __restrict__ sidx) {
+  __shared__ unsigned long long key_s[kRankChunk];
+  __shared__ unsigned short idx_s[kRankChunk];
   const int t = blockIdx.y, base = blockIdx.x * kRankChunk;
-  const double* V = Vc + (size_t)t * K;
-  for (int i = threadIdx.x; i < kRankChunk; i += blockDim.x) {
-    const int j = base + i;
-    if (j < K) {
-      key[i] = ~static_cast<unsigned long long>(__double_as_longlong(__ldg(V + ptx::perm_at(perm, j, K))));
-      idx[i] = (unsigned short)j;
-    } else {
-      key[i] = ~0ull;
-      idx[i] = 0xFFFF;
-    }
+  const int i = threadIdx.x;
+  const int j = base + i;
+  unsigned long long key = ~0ull;
+  unsigned idx = 0xFFFFu;
+  if (j < K) {
+    key = ~static_cast<unsigned long long>(
+        __double_as_longlong(__ldg(Vc + (size_t)t * K + ptx::perm_at(perm, j, K))));
+    idx = (unsigned)j;
   }
-  __syncthreads();
   for (int k = 2; k <= kRankChunk; k <<= 1) {
     for (int jj = k >> 1; jj > 0; jj >>= 1) {
-      for (int i = threadIdx.x; i < kRankChunk; i += blockDim.x) {
-        const int l = i ^ jj;
-        if (l > i) {
-          const unsigned long long ki = key[i], kl = key[l];
-          const unsigned short ii = idx[i], il = idx[l];
-          const bool i_gt = pair_less(kl, il, ki, ii);
-          if (i_gt == ((i & k) == 0)) {
-            key[i] = kl;
-            key[l] = ki;
-            idx[i] = il;
-            idx[l] = ii;
-          }
-        }
+      const int l = i ^ jj;
+      unsigned long long pk;
+      unsigned pi;
+      if (jj >= 32) {
+        key_s[i] = key;
+        idx_s[i] = (unsigned short)idx;
+        __syncthreads();
+        pk = key_s[l];
+        pi = idx_s[l];
+        __syncthreads();
+      } else {
+        pk = __shfl_xor_sync(0xffffffffu, key, jj);
+        pi = __shfl_xor_sync(0xffffffffu, idx, jj);
       }
-      __syncthreads();
+      const bool keep_min = ((i & k) == 0) == (i < l);
+      const bool partner_less = pair_less(pk, pi, key, idx);
+      if (partner_less == keep_min) {
+        key = pk;
+        idx = pi;
+      }
     }
   }
-  for (int i = threadIdx.x; i < kRankChunk; i += blockDim.x) {
-    skey[(size_t)t * Kp + base + i] = key[i];
-    sidx[(size_t)t * Kp + base + i] = idx[i];
-  }
+  skey[(size_t)t * Kp + j] = key;
+  sidx[(size_t)t * Kp + j] = (unsigned short)idx;
 }
 
-__global__ void merge_rank_kernel(const double* __restrict__ Vc, const int32_t* __restrict__ perm,
-                                  const unsigned long long* __restrict__ skey,
-                                  const unsigned short* __restrict__ sidx, int K, int Kp,
-                                  int32_t* __restrict__ rank) {
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+// rank[t][j] = number of (key, index) pairs of the tile below position j's: one binary
+// search per sorted chunk, each chunk staged in shared memory once per CTA.
+__global__ void __launch_bounds__(kRankChunk) merge_rank_kernel(
+    const double* __restrict__ Vc, const int32_t* __restrict__ perm,
+    const unsigned long long* __restrict__ skey, const unsigned short* __restrict__ sidx, int K,
+    int Kp, int32_t* __restrict__ rank) {
+  __shared__ unsigned long long ck[kRankChunk];
+  __shared__ unsigned short ci[kRankChunk];
   const int t = blockIdx.y;
-  if (j >= K) return;
-  const unsigned long long kj =
-      ~static_cast<unsigned long long>(__double_as_longlong(__ldg(Vc + (size_t)t * K + ptx::perm_at(perm, j, K))));
+  const int j = blockIdx.x * kRankChunk + threadIdx.x;
+  unsigned long long kj = 0ull;
+  if (j < K)
+    kj = ~static_cast<unsigned long long>(
+        __double_as_longlong(__ldg(Vc + (size_t)t * K + ptx::perm_at(perm, j, K))));
   const unsigned ij = (unsigned)j;
   int r = 0;
   for (int base = 0; base < Kp; base += kRankChunk) {
-    const unsigned long long* ck = skey + (size_t)t * Kp + base;
-    const unsigned short* ci = sidx + (size_t)t * Kp + base;
+    ck[threadIdx.x] = __ldg(skey + (size_t)t * Kp + base + threadIdx.x);
+    ci[threadIdx.x] = __ldg(sidx + (size_t)t * Kp + base + threadIdx.x);
+    __syncthreads();
     int lo = 0, hi = kRankChunk;  // count of pairs < (kj, ij) in this sorted chunk
     while (lo < hi) {
       const int mid = (lo + hi) >> 1;
-      if (pair_less(__ldg(ck + mid), __ldg(ci + mid), kj, ij)) lo = mid + 1;
+      if (pair_less(ck[mid], ci[mid], kj, ij)) lo = mid + 1;
       else hi = mid;
     }
     r += lo;
+    __syncthreads();
   }
-  rank[(size_t)t * K + j] = r;
+  if (j < K) rank[(size_t)t * K + j] = r;
 }
 
 size_t rank_scratch_bytes(int M, int K, int T) {
@@ -276,10 +285,10 @@ cudaError_t launch_vector_rank(const float* I, const int32_t* perm, int M, int K
   Carve c{static_cast<char*>(scratch), 0};
   unsigned long long* skey = c.take<unsigned long long>((size_t)nt * Kp);
   unsigned short* sidx = c.take<unsigned short>((size_t)nt * Kp);
-  chunk_sort_kernel<<<dim3(nchunk, nt), 512, 0, s>>>(V, perm, K, Kp, skey, sidx);
+  chunk_sort_kernel<<<dim3(nchunk, nt), kRankChunk, 0, s>>>(V, perm, K, Kp, skey, sidx);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  merge_rank_kernel<<<dim3((K + 255) / 256, nt), 256, 0, s>>>(V, perm, skey, sidx, K, Kp, rank);
+  merge_rank_kernel<<<dim3(nchunk, nt), kRankChunk, 0, s>>>(V, perm, skey, sidx, K, Kp, rank);
   return cudaGetLastError();
 }
 
@@ -329,6 +338,32 @@ __device__ double exact_to_double(U128 main, int lsb, const unsigned long long* 
   int ex = lo - 149;
   if (half && (sticky || (mant & 1ull))) {
     mant += 1;
+    if (mant == (1ull << 53)) {
+      mant >>= 1;
+      ex += 1;
+    }
+  }
+  return ldexp((double)mant, ex);
+}
+
+// value = v * 2^(lsb - 149) rounded to the nearest fp64, ties to even (the bucket-free case
+// of exact_to_double, on two 64-bit words).
+__device__ __forceinline__ double u128_to_double(U128 v, int lsb) {
+  if (v.hi == 0ull && v.lo < (1ull << 53)) return ldexp((double)v.lo, lsb - 149);  // exact
+  const int top = v.hi ? 127 - __clzll((long long)v.hi) : 63 - __clzll((long long)v.lo);
+  const int lo = top - 52;  // keep bits [lo, lo + 53); lo >= 1 here
+  unsigned long long mant;
+  if (lo >= 64) mant = v.hi >> (lo - 64);
+  else mant = (v.lo >> lo) | (v.hi << (64 - lo));
+  mant &= (1ull << 53) - 1ull;
+  const int hb = lo - 1;  // rounding bit
+  const bool half = hb >= 64 ? ((v.hi >> (hb - 64)) & 1ull) : ((v.lo >> hb) & 1ull);
+  bool sticky;  // any bit below hb
+  if (hb >= 64) sticky = v.lo != 0ull || (hb > 64 && (v.hi & ((1ull << (hb - 64)) - 1ull)) != 0ull);
+  else sticky = hb > 0 && (v.lo & ((1ull << hb) - 1ull)) != 0ull;
+  int ex = lsb + lo - 149;
+  if (half && (sticky || (mant & 1ull))) {
+    mant += 1ull;
     if (mant == (1ull << 53)) {
       mant >>= 1;
       ex += 1;
@@ -417,129 +452,163 @@ __global__ void __launch_bounds__(512) candidate_lists_kernel(
   }
 }
 
-// An fp64 value as a 128-bit integer in units of 2^(lsb-149); false when it is not a whole
-// number of units (it then holds values below the tile's scale).
-__device__ __forceinline__ bool f64_to_fixed(double s, int lsb, U128& r) {
-  r = U128{0ull, 0ull};
-  if (s == 0.0) return true;
-  const unsigned long long bits = (unsigned long long)__double_as_longlong(s);
-  const unsigned long long m = (bits & 0xFFFFFFFFFFFFFull) | (1ull << 52);
-  const int sh = (int)(bits >> 52) - 926 - lsb;
-  if (sh >= 64) {
-    r.hi = m << (sh - 64);
-  } else if (sh >= 0) {
-    r.lo = m << sh;
-    r.hi = sh ? (m >> (64 - sh)) : 0ull;
+// Loads RB consecutive floats (one channel's rows of the chunk) from shared memory.
+template <int RB>
+__device__ __forceinline__ void load_rows(const float* p, float (&v)[RB]) {
+  if constexpr (RB == 8) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0];
+    const float4 b = reinterpret_cast<const float4*>(p)[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else if constexpr (RB == 4) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  } else if constexpr (RB == 2) {
+    const float2 a = *reinterpret_cast<const float2*>(p);
+    v[0] = a.x; v[1] = a.y;
   } else {
-    if (sh <= -53 || (m & ((1ull << (-sh)) - 1ull))) return false;
-    r.lo = m >> (-sh);
+    v[0] = *p;
   }
-  return true;
 }
 
-// acc (fp64) += x (fp64 >= 0); err |= the addition rounded (Fast2Sum on max/min).
-__device__ __forceinline__ void add_checked(double& acc, double x, bool& err) {
-  const double a = fmax(acc, x), b = fmin(acc, x);
-  const double s = __dadd_rn(a, b);
-  err |= __dsub_rn(b, __dsub_rn(s, a)) != 0.0;
-  acc = s;
+template <int RB>
+__device__ __forceinline__ void store_rows(float* p, const float (&v)[RB]) {
+  if constexpr (RB == 8) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+  } else if constexpr (RB == 4) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  } else if constexpr (RB == 2) {
+    *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+  } else {
+    *p = v[0];
+  }
+}
+
+// Exact sum of a value that missed the fast path (p < eb): to the tile-scale 128-bit sum
+// `ex` when p >= lsb, else to the exponent buckets.
+__device__ __forceinline__ void band_slow(float v, U128& ex, int lsb, unsigned long long* bkt,
+                                          bool& used) {
+  uint32_t m;
+  int p;
+  split_f32(v, m, p);
+  if (!m) return;
+  if (p >= lsb) {
+    add_shifted(ex, m, p - lsb);
+  } else {
+    atomicAdd(bkt + p, (unsigned long long)m);
+    used = true;
+  }
 }
 
 // Per (tile, chunk of RB rows), 512 threads.  The chunk's rows of I are staged in shared
-// memory once; then, candidate by candidate, each thread takes 2:4 groups g = tid,
-// tid + 512, ... and evaluates the top-2 of every row of the chunk.  A thread sums its
-// values in fp64 with every addition checked for rounding: when nothing rounded (and the
-// sum is a whole number of the tile's fixed-point units) the sum is exact; otherwise the
-// same groups are summed again through the exact integer path.  Warps combine their
-// 128-bit partials with shuffles into per-warp slots; one barrier at the end, then
-// part[t][m][chunk] = the CTA's exact total of candidate m.
+// memory channel-major (the RB values of channel c contiguous, one vector load each).
+// Then, candidate by candidate, the candidate's 2:4 groups are dealt round-robin to the
+// threads (the starting thread rotates with the groups dealt so far, so the work stays even
+// over all candidates) and, for every row, the top 2 of the group's 4 values are summed.
+//
+// The sums are exact.  With eb = max(P - 24, lsb) every value with p >= eb is a multiple of
+// u = 2^(eb - 149) below 2^48 u, and a thread adds at most 32 of them, so its fp64 sum never
+// rounds (it stays an integer multiple of u below 2^53 u).  Values with p < eb (rare: 2^24
+// below the tile's largest) go to band_slow.  Per candidate, each warp adds its threads'
+// integer sums with three 21-bit-piece reductions and one shared atomic.
+template <int RB>
 __global__ void __launch_bounds__(512) band_sum_kernel(
     const float* __restrict__ I, const unsigned short* __restrict__ band,
-    const int* __restrict__ tile_pmax, int K, int T, int RB, CandidateList cl, int ncand,
+    const int* __restrict__ tile_pmax, int K, int T, CandidateList cl, int ncand,
     U128* __restrict__ part, unsigned long long* __restrict__ bucket,
     int* __restrict__ bucket_used) {
-  extern __shared__ __align__(16) float rows_s[];  // [RB][K]
-  // per candidate, the CTA's total as four 32-bit digits held in 64-bit words
-  __shared__ unsigned long long digits[kMaxCandidates][4];
+  extern __shared__ __align__(16) float rows_s[];  // [K][RB]
+  __shared__ unsigned long long fast_sum[kMaxCandidates];   // units of 2^(eb - 149)
+  __shared__ unsigned long long digits[kMaxCandidates][4];  // slow path, units of 2^(lsb - 149)
   const int chunk = blockIdx.x, t = blockIdx.y;
   const int nchunks = gridDim.x;
   const int lane = threadIdx.x & 31;
-  for (int x = threadIdx.x; x < kMaxCandidates * 4; x += blockDim.x) (&digits[0][0])[x] = 0ull;
-  const int lsb = tile_lsb(tile_pmax[t]);
-  const float4* src = reinterpret_cast<const float4*>(I + ((size_t)t * T + (size_t)chunk * RB) * K);
-  for (int x = threadIdx.x; x < RB * K / 4; x += blockDim.x)
-    reinterpret_cast<float4*>(rows_s)[x] = __ldg(src + x);
+  constexpr int kThreads = 512;
+  const int pmax = tile_pmax[t];
+  const int lsb = tile_lsb(pmax);
+  const int eb = max(pmax - 24, lsb);
+  const float thr = __uint_as_float((uint32_t)(eb + 1) << 23);  // smallest fp32 with p >= eb
+  for (int x = threadIdx.x; x < kMaxCandidates; x += kThreads) fast_sum[x] = 0ull;
+  for (int x = threadIdx.x; x < kMaxCandidates * 4; x += kThreads) (&digits[0][0])[x] = 0ull;
+  const float* src = I + ((size_t)t * T + (size_t)chunk * RB) * K;
+  for (int c = threadIdx.x; c < K; c += kThreads) {
+    float v[RB];
+#pragma unroll
+    for (int r = 0; r < RB; ++r) v[r] = __ldg(src + (size_t)r * K + c);
+    store_rows<RB>(rows_s + (size_t)c * RB, v);
+  }
   __syncthreads();
 
+  const unsigned short* band_t = band + (size_t)t * ncand * K;
+  auto first_group = [&](int off) {
+    int q = (int)threadIdx.x - off;
+    return q < 0 ? q + kThreads : q;
+  };
+  int off = 0;  // groups dealt before this candidate, mod kThreads
+  int q = first_group(off);
+  ushort4 cq_next = make_ushort4(0, 0, 0, 0);
+  if (ncand > 0 && q < cl.c[0].n24 / 4) cq_next = __ldg(reinterpret_cast<const ushort4*>(band_t) + q);
   for (int m = 0; m < ncand; ++m) {
     const int ng = cl.c[m].n24 / 4;
-    const unsigned short* bl = band + ((size_t)t * ncand + m) * K;
+    const ushort4 cq0 = cq_next;
+    const int q_m = q;
+    off = (off + ng) % kThreads;
+    q = first_group(off);
+    if (m + 1 < ncand && q < cl.c[m + 1].n24 / 4)
+      cq_next = __ldg(reinterpret_cast<const ushort4*>(band_t + (size_t)(m + 1) * K) + q);
+    const bool active = q_m < ng;
+    if (!__any_sync(0xffffffffu, active)) continue;  // warp-uniform
+    const unsigned short* bl = band_t + (size_t)m * K;
     unsigned long long* bkt = bucket + ((size_t)t * ncand + m) * 256;
+    double acc = 0.0;
     U128 ex{0ull, 0ull};
-    if ((int)threadIdx.x < ng) {
-      // pass 1: checked fp64
-      double acc = 0.0;
-      bool err = false;
-      for (int g = threadIdx.x; g < ng; g += blockDim.x) {
-        const ushort4 cq = __ldg(reinterpret_cast<const ushort4*>(bl) + g);
-        const int c0 = min((int)cq.x, K - 1), c1 = min((int)cq.y, K - 1);
-        const int c2 = min((int)cq.z, K - 1), c3 = min((int)cq.w, K - 1);
-        for (int r = 0; r < RB; ++r) {
-          const float* row = rows_s + r * K;
-          const float v0 = row[c0], v1 = row[c1], v2 = row[c2], v3 = row[c3];
-          const float a = fmaxf(v0, v1), b = fminf(v0, v1);
-          const float cc = fmaxf(v2, v3), d = fminf(v2, v3);
-          const float t1 = fmaxf(a, cc), t2 = fmaxf(fminf(a, cc), fmaxf(b, d));
-          const double p = __dadd_rn((double)t1, (double)t2);  // Fast2Sum, t1 >= t2
-          err |= __dsub_rn((double)t2, __dsub_rn(p, (double)t1)) != 0.0;
-          add_checked(acc, p, err);
-        }
-      }
-      if (!err && !f64_to_fixed(acc, lsb, ex)) err = true;
-      if (err) {
-        // pass 2: exact integers (values below the tile's scale into the buckets)
-        ex = U128{0ull, 0ull};
-        bool used = false;
-        for (int g = threadIdx.x; g < ng; g += blockDim.x) {
-          const ushort4 cq = __ldg(reinterpret_cast<const ushort4*>(bl) + g);
-          const int c0 = min((int)cq.x, K - 1), c1 = min((int)cq.y, K - 1);
-          const int c2 = min((int)cq.z, K - 1), c3 = min((int)cq.w, K - 1);
-          for (int r = 0; r < RB; ++r) {
-            const float* row = rows_s + r * K;
-            const float v0 = row[c0], v1 = row[c1], v2 = row[c2], v3 = row[c3];
-            const float a = fmaxf(v0, v1), b = fminf(v0, v1);
-            const float cc = fmaxf(v2, v3), d = fminf(v2, v3);
-            const float tv[2] = {fmaxf(a, cc), fmaxf(fminf(a, cc), fmaxf(b, d))};
+    bool used = false;
+    for (int g = q_m; g < ng; g += kThreads) {
+      const ushort4 cq = g == q_m ? cq0 : __ldg(reinterpret_cast<const ushort4*>(bl) + g);
+      float v0[RB], v1[RB], v2[RB], v3[RB];
+      load_rows<RB>(rows_s + (size_t)min((int)cq.x, K - 1) * RB, v0);
+      load_rows<RB>(rows_s + (size_t)min((int)cq.y, K - 1) * RB, v1);
+      load_rows<RB>(rows_s + (size_t)min((int)cq.z, K - 1) * RB, v2);
+      load_rows<RB>(rows_s + (size_t)min((int)cq.w, K - 1) * RB, v3);
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              uint32_t mm;
-              int e;
-              split_f32(tv[q], mm, e);
-              if (!mm) continue;
-              if (e >= lsb) {
-                add_shifted(ex, mm, e - lsb);
-              } else {
-                atomicAdd(bkt + e, (unsigned long long)mm);
-                used = true;
-              }
-            }
-          }
+      for (int r = 0; r < RB; ++r) {
+        const float a = fmaxf(v0[r], v1[r]), b = fminf(v0[r], v1[r]);
+        const float cc = fmaxf(v2[r], v3[r]), d = fminf(v2[r], v3[r]);
+        const float t1 = fmaxf(a, cc), t2 = fmaxf(fminf(a, cc), fmaxf(b, d));
+        if (t2 >= thr) {
+          acc = __dadd_rn(acc, __dadd_rn((double)t1, (double)t2));
+        } else {
+          if (t1 >= thr) acc = __dadd_rn(acc, (double)t1);
+          else band_slow(t1, ex, lsb, bkt, used);
+          band_slow(t2, ex, lsb, bkt, used);
         }
-        if (used) atomicOr(bucket_used + (size_t)t * ncand + m, 1);
       }
     }
-    __syncwarp();
-    for (int o = 16; o > 0; o >>= 1) {
-      U128 other;
-      other.lo = __shfl_xor_sync(0xffffffffu, ex.lo, o);
-      other.hi = __shfl_xor_sync(0xffffffffu, ex.hi, o);
-      add128(ex, other);
+    if (used) atomicOr(bucket_used + (size_t)t * ncand + m, 1);
+    // this thread's fast sum as an integer number of units (< 2^53)
+    const unsigned long long ai = __double2ull_rz(ldexp(acc, 149 - eb));
+    const unsigned s0 = __reduce_add_sync(0xffffffffu, (unsigned)(ai & 0x1FFFFFull));
+    const unsigned s1 = __reduce_add_sync(0xffffffffu, (unsigned)((ai >> 21) & 0x1FFFFFull));
+    const unsigned s2 = __reduce_add_sync(0xffffffffu, (unsigned)(ai >> 42));
+    if (lane == 0) {
+      const unsigned long long w = (unsigned long long)s0 + ((unsigned long long)s1 << 21) +
+                                   ((unsigned long long)s2 << 42);
+      if (w) atomicAdd(&fast_sum[m], w);
     }
-    if (lane == 0 && (ex.lo | ex.hi)) {
-      atomicAdd(&digits[m][0], ex.lo & 0xFFFFFFFFull);
-      atomicAdd(&digits[m][1], ex.lo >> 32);
-      atomicAdd(&digits[m][2], ex.hi & 0xFFFFFFFFull);
-      atomicAdd(&digits[m][3], ex.hi >> 32);
+    if (__any_sync(0xffffffffu, (ex.lo | ex.hi) != 0ull)) {
+      for (int o = 16; o > 0; o >>= 1) {
+        U128 other;
+        other.lo = __shfl_xor_sync(0xffffffffu, ex.lo, o);
+        other.hi = __shfl_xor_sync(0xffffffffu, ex.hi, o);
+        add128(ex, other);
+      }
+      if (lane == 0) {
+        atomicAdd(&digits[m][0], ex.lo & 0xFFFFFFFFull);
+        atomicAdd(&digits[m][1], ex.lo >> 32);
+        atomicAdd(&digits[m][2], ex.hi & 0xFFFFFFFFull);
+        atomicAdd(&digits[m][3], ex.hi >> 32);
+      }
     }
   }
   __syncthreads();
@@ -553,6 +622,13 @@ __global__ void __launch_bounds__(512) band_sum_kernel(
     U128 tot;
     tot.lo = (d0 & 0xFFFFFFFFull) | (d1 << 32);
     tot.hi = (d2 & 0xFFFFFFFFull) | (d3 << 32);
+    // + fast_sum * 2^(eb - lsb): fast_sum < 2^62 (16 warps x 32 threads x 2^53), eb - lsb <= 59
+    const unsigned long long f = fast_sum[threadIdx.x];
+    const int sh = eb - lsb;
+    U128 fx;
+    fx.lo = f << sh;
+    fx.hi = sh ? (f >> (64 - sh)) : 0ull;
+    add128(tot, fx);
     part[((size_t)t * ncand + threadIdx.x) * nchunks + chunk] = tot;
   }
 }
@@ -566,16 +642,14 @@ __global__ void finalize_kernel(const U128* __restrict__ rdense, const U128* __r
                                 double t_s, double alpha, double* __restrict__ R,
                                 int32_t* __restrict__ counts, double* __restrict__ vs) {
   __shared__ double Rs[kMaxCandidates];
-  __shared__ unsigned long long zero_bkt[256];
   const int t = blockIdx.x, m = threadIdx.x;
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) zero_bkt[i] = 0ull;
-  __syncthreads();
   if (m < ncand) {
     const size_t tm = (size_t)t * ncand + m;
     U128 tot = rdense[tm];
     for (int c = 0; c < nchunks; ++c) add128(tot, part[tm * nchunks + c]);
-    const unsigned long long* bk = bucket_used[tm] ? bucket + tm * 256 : zero_bkt;
-    const double r = exact_to_double(tot, tile_lsb(tile_pmax[t]), bk);
+    const int lsb = tile_lsb(tile_pmax[t]);
+    const double r = bucket_used[tm] ? exact_to_double(tot, lsb, bucket + tm * 256)
+                                     : u128_to_double(tot, lsb);
     Rs[m] = r;
     R[tm] = r;
   }
@@ -666,13 +740,21 @@ cudaError_t launch_boundary_search(const float* I, const int32_t* perm, int M, i
   const size_t smem = (size_t)RB * K * sizeof(float);
   static bool attr_set = false;
   if (!attr_set) {
-    e = cudaFuncSetAttribute(band_sum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             96 * 1024);
-    if (e != cudaSuccess) return e;
+    for (auto fn : {band_sum_kernel<1>, band_sum_kernel<2>, band_sum_kernel<4>, band_sum_kernel<8>}) {
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+      if (e != cudaSuccess) return e;
+    }
     attr_set = true;
   }
-  band_sum_kernel<<<dim3(nchunks, nt), 512, smem, s>>>(I, band, pmax, K, T, RB, cl, ncand, part,
-                                                       bucket, bucket_used);
+  const dim3 gb(nchunks, nt);
+  if (RB == 8)
+    band_sum_kernel<8><<<gb, 512, smem, s>>>(I, band, pmax, K, T, cl, ncand, part, bucket, bucket_used);
+  else if (RB == 4)
+    band_sum_kernel<4><<<gb, 512, smem, s>>>(I, band, pmax, K, T, cl, ncand, part, bucket, bucket_used);
+  else if (RB == 2)
+    band_sum_kernel<2><<<gb, 512, smem, s>>>(I, band, pmax, K, T, cl, ncand, part, bucket, bucket_used);
+  else
+    band_sum_kernel<1><<<gb, 512, smem, s>>>(I, band, pmax, K, T, cl, ncand, part, bucket, bucket_used);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   finalize_kernel<<<nt, 64, 0, s>>>(rdense, part, nchunks, bucket, bucket_used, pmax, ncand, cl,
