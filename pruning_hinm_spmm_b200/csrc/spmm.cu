@@ -31,7 +31,7 @@
 
 namespace hinm {
 
-template <int BN>
+template <int BN, bool SPLIT = false>
 struct SpmmCfg {
   static constexpr int kAtom = BN >= 64 ? 64 : BN;  // B swizzle atom width (elements)
   static constexpr int kAtomBytes = kAtom * 2;      // 128, 64 or 32 bytes
@@ -42,21 +42,29 @@ struct SpmmCfg {
   static constexpr int kBBytes = 128 * BN * 2;  // 128 K-rows (a 2:4 block); dense uses 64
   static constexpr int kEBytes = 2048;
   static constexpr int kStageBytes = kABytes + kBBytes + kEBytes;
-  static constexpr int kStagesRaw = (200 * 1024) / kStageBytes;
+  // split-K: CTAs of a cluster per unit; the leader's reduction buffer holds the others'
+  // 128 x BN fp32 partial accumulators
+  static constexpr int kMaxSplit = !SPLIT ? 1 : (BN <= 16 ? 8 : 4);
+  static constexpr int kRedBytes = (kMaxSplit - 1) * 128 * BN * 4;
+  static constexpr int kStagesRaw = (200 * 1024 - kRedBytes) / kStageBytes;
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
   // layout type of the B descriptor: 2 = 128-byte swizzle, 4 = 64-byte, 6 = 32-byte
   static constexpr uint32_t kBLayout = kAtomBytes == 128 ? 2u : (kAtomBytes == 64 ? 4u : 6u);
   static constexpr int kAccCols = BN < 32 ? 32 : BN;  // accumulator buffer stride (columns)
-  static constexpr int kTmemNeed = 2 * kAccCols + 4 * kStages;
+  // two accumulator buffers (epilogue overlaps the next unit) when tensor memory holds them
+  static constexpr int kAccBufs = 2 * kAccCols + 4 * kStages <= 512 ? 2 : 1;
+  static constexpr int kTmemNeed = kAccBufs * kAccCols + 4 * kStages;
   static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                    : kTmemNeed <= 256 ? 256 : 512;
-  static constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024 /*align*/ + 512;
+  static constexpr size_t kSmemBytes =
+      (size_t)kStages * kStageBytes + 1024 /*align*/ + 512 /*barriers*/ + kRedBytes;
   static constexpr int kProducers = 128;
   static constexpr int kMmaWarp = 4;
   static constexpr int kThreads = 288;  // 9 warps: 4 producers, 1 MMA, 4 epilogue
-  static_assert(BN == 16 || BN == 32 || BN % 64 == 0, "BN");
+  static_assert(BN == 16 || BN == 32 || (BN % 64 == 0 && BN <= 256), "BN");
   static_assert(kStages >= 2, "stages");
   static_assert(kTmemNeed <= 512, "tmem");
+  static_assert(!SPLIT || BN <= 32, "split-K is for narrow N");
 };
 
 struct SpmmArgs {
@@ -72,6 +80,7 @@ struct SpmmArgs {
   float* Y;
   int N, T;
   int num_tiles, nblk_n, num_units;
+  int split;  // CTAs (one cluster) per unit; 1 = persistent, no split
   int* status;
 };
 
@@ -115,10 +124,10 @@ struct Gather {
   }
 };
 
-template <int BN>
+template <int BN, bool SPLIT>
 __global__ void __launch_bounds__(288, 1)
     spmm_kernel(const __grid_constant__ CUtensorMap tmX, const SpmmArgs a) {
-  using C = SpmmCfg<BN>;
+  using C = SpmmCfg<BN, SPLIT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -156,18 +165,34 @@ __global__ void __launch_bounds__(288, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t meta_col0 = 2 * C::kAccCols;
+  const uint32_t meta_col0 = C::kAccBufs * C::kAccCols;
+  float* red = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes + 512);
+  // Work: persistent CTAs stride over the units; split-K CTAs take one unit each and the
+  // K-block range [kb0, kb1) of their cluster rank.
+  const int u_first = SPLIT ? (int)blockIdx.x / a.split : (int)blockIdx.x;
+  const int u_step = SPLIT ? a.num_units : (int)gridDim.x;
+  const int rank = SPLIT ? (int)(blockIdx.x % a.split) : 0;
+  auto k_range = [&](int nblk, int& kb0, int& kb1) {
+    kb0 = SPLIT ? (int)((long long)nblk * rank / a.split) : 0;
+    kb1 = SPLIT ? (int)((long long)nblk * (rank + 1) / a.split) : nblk;
+  };
+
+  // split-K: what the leader's epilogue needs after the cluster barrier
+  bool split_ready = false, split_has = false;
+  int split_tile = 0, split_n0 = 0, split_b = 0;
 
   if (warp < 4) {
     // ------------------------------------------------------------ producers
     const int ptid = threadIdx.x;
     uint32_t it = 0;  // K-blocks issued by this CTA (stage ring position)
     bool stop = false;
-    for (int u = blockIdx.x; u < a.num_units && !stop; u += gridDim.x) {
+    for (int u = u_first; u < a.num_units && !stop; u += u_step) {
       const int tile = u / a.nblk_n, n0 = (u - tile * a.nblk_n) * BN;
       const int4 info = __ldg(reinterpret_cast<const int4*>(a.tile_info) + tile);
       const int nd = info.x, nblk = info.x + info.y;
-      for (int kb = 0; kb < nblk; ++kb, ++it) {
+      int kb0, kb1;
+      k_range(nblk, kb0, kb1);
+      for (int kb = kb0; kb < kb1; ++kb, ++it) {
         const bool sparse = kb >= nd;
         const size_t blk = sparse ? (size_t)(info.w + kb - nd) : (size_t)(info.z + kb);
         // index loads are issued before the wait so their latency hides behind it
@@ -226,17 +251,20 @@ __global__ void __launch_bounds__(288, 1)
       const uint32_t idesc_s = ptx::idesc_bf16(BN, 1, 1);
       uint32_t it = 0, lu = 0;
       bool stop = false;
-      for (int u = blockIdx.x; u < a.num_units && !stop; u += gridDim.x, ++lu) {
+      for (int u = u_first; u < a.num_units && !stop; u += u_step, ++lu) {
         const int tile = u / a.nblk_n;
         const int4 info = __ldg(reinterpret_cast<const int4*>(a.tile_info) + tile);
         const int nd = info.x, nblk = info.x + info.y;
-        const int b = lu & 1;
-        if (!ptx::mbar_wait(acce_bar(b), ((lu >> 1) & 1) ^ 1, a.status, abort_flag)) break;
+        int kb0, kb1;
+        k_range(nblk, kb0, kb1);
+        const int b = (int)(lu % C::kAccBufs);
+        if (!ptx::mbar_wait(acce_bar(b), ((lu / C::kAccBufs) & 1) ^ 1, a.status, abort_flag)) break;
         ptx::tc_fence_after();
         const uint32_t acc = tmem + b * C::kAccCols;
-        for (int kb = 0; kb < nblk; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % C::kStages;
           const uint32_t ph = (it / C::kStages) & 1;
+          const uint32_t accum0 = kb != kb0 ? 1u : 0u;  // first K-block overwrites
           if (!ptx::mbar_wait(full_bar(s), ph, a.status, abort_flag)) {
             stop = true;
             break;
@@ -256,7 +284,7 @@ __global__ void __launch_bounds__(288, 1)
               const uint64_t bd = ptx::smem_desc(B_s + 32 * k * C::kAtomBytes, 128 * C::kAtomBytes,
                                                  8 * C::kAtomBytes, C::kBLayout);
               const uint32_t e = e_col + k;
-              ptx::mma_sp_bf16(acc, ad, bd, e & ~1u, idesc_s | (e & 1u), (kb | k) ? 1u : 0u);
+              ptx::mma_sp_bf16(acc, ad, bd, e & ~1u, idesc_s | (e & 1u), (accum0 | k) ? 1u : 0u);
             }
           } else {
 #pragma unroll
@@ -264,7 +292,7 @@ __global__ void __launch_bounds__(288, 1)
               const uint64_t ad = ptx::smem_desc(A_s + 32 * k, 16, 1024, 2);
               const uint64_t bd = ptx::smem_desc(B_s + 16 * k * C::kAtomBytes, 128 * C::kAtomBytes,
                                                  8 * C::kAtomBytes, C::kBLayout);
-              ptx::mma_bf16(acc, ad, bd, idesc_d, (kb | k) ? 1u : 0u);
+              ptx::mma_bf16(acc, ad, bd, idesc_d, (accum0 | k) ? 1u : 0u);
             }
           }
           ptx::tc_commit(empty_bar(s));
@@ -283,50 +311,134 @@ __global__ void __launch_bounds__(288, 1)
     const int row = q * 32 + lane;
     constexpr int kChunk = BN >= 32 ? 32 : 16;
     uint32_t lu = 0;
-    for (int u = blockIdx.x; u < a.num_units; u += gridDim.x, ++lu) {
+    for (int u = u_first; u < a.num_units; u += u_step, ++lu) {
       const int tile = u / a.nblk_n, n0 = (u - tile * a.nblk_n) * BN;
       const int4 info = __ldg(reinterpret_cast<const int4*>(a.tile_info) + tile);
-      const int nblk = info.x + info.y;
-      const int b = lu & 1;
-      bool ok = ptx::mbar_wait(accf_bar(b), (lu >> 1) & 1, a.status, abort_flag);
+      int kb0, kb1;
+      k_range(info.x + info.y, kb0, kb1);
+      const bool has = kb1 > kb0;  // else the accumulator was never written: zeros
+      const int b = (int)(lu % C::kAccBufs);
+      bool ok = ptx::mbar_wait(accf_bar(b), (lu / C::kAccBufs) & 1, a.status, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       ptx::tc_fence_after();
-      const bool row_ok = row < a.T;
-      float* yrow = a.Y + (size_t)(tile * a.T + row) * a.N;
-      for (int col = 0; col < BN; col += kChunk) {
-        uint32_t v[32];
-        if (nblk > 0) {
-          const uint32_t taddr =
-              tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::kAccCols + col);
-          if constexpr (kChunk == 32) {
-            ptx::tmem_ld_32x32b_x32(taddr, v);
-          } else {
-            ptx::tmem_ld_32x32b_x16(taddr, v);
-          }
-          ptx::tmem_ld_wait();
-        } else {
+      if constexpr (SPLIT) {
+        split_ready = true;
+        split_has = has;
+        split_tile = tile;
+        split_n0 = n0;
+        split_b = b;
+        if (rank != 0) {
+          // this CTA's partial -> the leader's reduction buffer, slot rank - 1
+          const uint32_t dst = ptx::mapa_shared(ptx::smem_u32(red), 0) +
+                               (uint32_t)((((rank - 1) * 128 + row) * BN) * 4);
+          for (int col = 0; col < BN; col += kChunk) {
+            uint32_t v[32];
+            if (has) {
+              const uint32_t taddr =
+                  tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::kAccCols + col);
+              if constexpr (kChunk == 32) ptx::tmem_ld_32x32b_x32(taddr, v);
+              else ptx::tmem_ld_32x32b_x16(taddr, v);
+              ptx::tmem_ld_wait();
+            } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = 0u;
-        }
-        if (row_ok) {
-          const int gc = n0 + col;
-          if (gc + kChunk <= a.N) {
-#pragma unroll
-            for (int i = 0; i < kChunk; i += 4) {
-              float4 o = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
-                                     __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
-              *reinterpret_cast<float4*>(yrow + gc + i) = o;
+              for (int i = 0; i < 32; ++i) v[i] = 0u;
             }
+#pragma unroll
+            for (int i = 0; i < kChunk; i += 4)
+              ptx::st_cluster_v4(dst + (uint32_t)(col + i) * 4u, __uint_as_float(v[i]),
+                                 __uint_as_float(v[i + 1]), __uint_as_float(v[i + 2]),
+                                 __uint_as_float(v[i + 3]));
+          }
+        }
+      } else {
+        const bool row_ok = row < a.T;
+        float* yrow = a.Y + (size_t)(tile * a.T + row) * a.N;
+        for (int col = 0; col < BN; col += kChunk) {
+          uint32_t v[32];
+          if (has) {
+            const uint32_t taddr =
+                tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::kAccCols + col);
+            if constexpr (kChunk == 32) {
+              ptx::tmem_ld_32x32b_x32(taddr, v);
+            } else {
+              ptx::tmem_ld_32x32b_x16(taddr, v);
+            }
+            ptx::tmem_ld_wait();
           } else {
-            for (int i = 0; i < kChunk; ++i)
-              if (gc + i < a.N) yrow[gc + i] = __uint_as_float(v[i]);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0u;
+          }
+          if (row_ok) {
+            const int gc = n0 + col;
+            if (gc + kChunk <= a.N) {
+#pragma unroll
+              for (int i = 0; i < kChunk; i += 4) {
+                float4 o = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                                       __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+                *reinterpret_cast<float4*>(yrow + gc + i) = o;
+              }
+            } else {
+              for (int i = 0; i < kChunk; ++i)
+                if (gc + i < a.N) yrow[gc + i] = __uint_as_float(v[i]);
+            }
           }
         }
       }
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(acce_bar(b));  // accumulator b may be overwritten
+    }
+  }
+  if constexpr (SPLIT) {
+    // the partials of ranks 1.. are in the leader's shared memory after this barrier; the
+    // leader adds them in rank order (deterministic) to its own and stores Y
+    ptx::cluster_sync();
+    if (rank == 0 && warp > C::kMmaWarp && split_ready) {
+      ptx::tc_fence_after();
+      const int q = warp & 3;
+      const int row = q * 32 + lane;
+      constexpr int kChunk = BN >= 32 ? 32 : 16;
+      const bool row_ok = row < a.T;
+      float* yrow = a.Y + (size_t)(split_tile * a.T + row) * a.N;
+      for (int col = 0; col < BN; col += kChunk) {
+        uint32_t v[32];
+        if (split_has) {
+          const uint32_t taddr =
+              tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(split_b * C::kAccCols + col);
+          if constexpr (kChunk == 32) ptx::tmem_ld_32x32b_x32(taddr, v);
+          else ptx::tmem_ld_32x32b_x16(taddr, v);
+          ptx::tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0u;
+        }
+        float o[32];
+#pragma unroll
+        for (int i = 0; i < kChunk; ++i) o[i] = __uint_as_float(v[i]);
+        for (int r = 1; r < a.split; ++r) {
+          const float* src = red + ((size_t)(r - 1) * 128 + row) * BN + col;
+#pragma unroll
+          for (int i = 0; i < kChunk; i += 4) {
+            const float4 pv = *reinterpret_cast<const float4*>(src + i);
+            o[i] = __fadd_rn(o[i], pv.x);
+            o[i + 1] = __fadd_rn(o[i + 1], pv.y);
+            o[i + 2] = __fadd_rn(o[i + 2], pv.z);
+            o[i + 3] = __fadd_rn(o[i + 3], pv.w);
+          }
+        }
+        if (row_ok) {
+          const int gc = split_n0 + col;
+          if (gc + kChunk <= a.N) {
+#pragma unroll
+            for (int i = 0; i < kChunk; i += 4)
+              *reinterpret_cast<float4*>(yrow + gc + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+          } else {
+            for (int i = 0; i < kChunk; ++i)
+              if (gc + i < a.N) yrow[gc + i] = o[i];
+          }
+        }
+      }
     }
   }
   ptx::tc_fence_before();
@@ -383,15 +495,15 @@ int num_sms() {
   return n;
 }
 
-template <int BN>
-cudaError_t run(const hinm_layout& L, const uint16_t* X, int N, float* Y, int* status,
+template <int BN, bool SPLIT>
+cudaError_t run(const hinm_layout& L, const uint16_t* X, int N, float* Y, int split, int* status,
                 cudaStream_t s) {
-  using C = SpmmCfg<BN>;
+  using C = SpmmCfg<BN, SPLIT>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(spmm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)C::kSmemBytes);
+    attr_err = cudaFuncSetAttribute(spmm_kernel<BN, SPLIT>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmemBytes);
   });
   if (attr_err != cudaSuccess) return attr_err;
   CUtensorMap map;
@@ -400,20 +512,52 @@ cudaError_t run(const hinm_layout& L, const uint16_t* X, int N, float* Y, int* s
   const int units = L.num_tiles * nblk_n;
   SpmmArgs a{L.tile_info, L.vals_dense, L.vals_sparse, L.meta,   L.idx_dense, L.idx_sparse,
              L.run_dense, L.run_sparse, X,             Y,        N,           L.T,
-             L.num_tiles, nblk_n,       units,         status};
-  const int grid = units < num_sms() ? units : num_sms();
-  spmm_kernel<BN><<<grid, C::kThreads, C::kSmemBytes, s>>>(map, a);
-  return cudaGetLastError();
+             L.num_tiles, nblk_n,       units,         SPLIT ? split : 1,       status};
+  if constexpr (!SPLIT) {
+    const int grid = units < num_sms() ? units : num_sms();
+    spmm_kernel<BN, false><<<grid, C::kThreads, C::kSmemBytes, s>>>(map, a);
+    return cudaGetLastError();
+  } else {
+    // one cluster of `split` CTAs per unit
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(units * split), 1, 1);
+    cfg.blockDim = dim3(C::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, spmm_kernel<BN, true>, map, a);
+  }
+}
+
+// Split-K when the units (tile x column block) fill less than half of the SMs: each unit's
+// K-blocks are shared by a cluster of up to kMaxSplit CTAs.
+template <int BN>
+cudaError_t run_auto(const hinm_layout& L, const uint16_t* X, int N, float* Y, int* status,
+                     cudaStream_t s) {
+  const int units = L.num_tiles * ((N + BN - 1) / BN);
+  if constexpr (BN <= 32) {
+    int split = units > 0 ? num_sms() / units : 1;
+    if (split > SpmmCfg<BN, true>::kMaxSplit) split = SpmmCfg<BN, true>::kMaxSplit;
+    if (split >= 2) return run<BN, true>(L, X, N, Y, split, status, s);
+  }
+  return run<BN, false>(L, X, N, Y, 1, status, s);
 }
 
 }  // namespace
 
 cudaError_t launch_spmm(const hinm_layout& L, const uint16_t* X, int N, float* Y, int* status,
                         cudaStream_t s) {
-  if (N <= 16) return run<16>(L, X, N, Y, status, s);
-  if (N <= 32) return run<32>(L, X, N, Y, status, s);
-  if (N <= 64) return run<64>(L, X, N, Y, status, s);
-  return run<128>(L, X, N, Y, status, s);
+  if (N <= 16) return run_auto<16>(L, X, N, Y, status, s);
+  if (N <= 32) return run_auto<32>(L, X, N, Y, status, s);
+  if (N <= 64) return run_auto<64>(L, X, N, Y, status, s);
+  if (N < 256) return run_auto<128>(L, X, N, Y, status, s);
+  return run_auto<256>(L, X, N, Y, status, s);
 }
 
 }  // namespace hinm
