@@ -41,6 +41,22 @@ UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest of every rank's x (the job's time is its slowest rank's); x itself on
+    one rank.  Every rank must call it at the same point."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(flops_per_rank: float, world: int, t_max: float) -> float:
+    """Whole-job throughput in TFLOP/s: every rank's shard over the slowest rank's time."""
+    return flops_per_rank * world / t_max / 1e12
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -306,11 +322,8 @@ def main():
                  for i, p in enumerate(phases)}
     step_s = [evs[k][0].elapsed_time(evs[k][5]) * 1e-3 for k in range(args.steps)]
     t_step = statistics.mean(step_s)
-    if dist:
-        tt = torch.tensor([t_step], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_step = float(tt.item())
-    value = model["flops_eff"] * world / t_step / 1e12
+    t_step = max_over_ranks(t_step, dist, dev)
+    value = job_value(model["flops_eff"], world, t_step)
 
     # ---------------- end to end through the public API with host buffers
     W_h = torch.from_numpy(w.W_bits.view(np.int16)).pin_memory()
@@ -342,10 +355,7 @@ def main():
     e_end.record(stream)
     torch.cuda.synchronize()
     t_e2e = e_start.elapsed_time(e_end) * 1e-3 / e2e_steps
-    if dist:
-        tt = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_e2e = float(tt.item())
+    t_e2e = max_over_ranks(t_e2e, dist, dev)
     h2d = W_h.numel() * 2 + X_h.numel() * 2 + P_h.numel() * 4
     d2h = Y_h.numel() * 4
     # the e2e output must match the device-resident path
@@ -406,7 +416,7 @@ def main():
         "kernels": kernels,
         "roofline": roof,
         "cpu_baseline": cpu,
-        "e2e": {"value": model["flops_eff"] * world / t_e2e / 1e12, "unit": UNIT,
+        "e2e": {"value": job_value(model["flops_eff"], world, t_e2e), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": t_e2e * 1e3},
         "gpu_launches": kernels_per_step * args.steps,
