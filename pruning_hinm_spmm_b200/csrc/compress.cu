@@ -195,25 +195,32 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint16_t* __restrict__ 
         w[k] = __ldg(Wi + c);
         kept |= ((__ldg(bmi + (c >> 5)) >> (c & 31)) & 1u) << k;
       }
-      const int nk = __popc(kept);
-      if (nk != 2) ptx::record_status(status, HINM_ERR_BAD_MASK);
-      // the two kept positions, lowest first; a missing one is taken from the unkept
-      // positions with value 0 so that the pair stays a legal (a < b) pattern
-      int pos[2], np = 0;
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        if (((kept >> k) & 1u) && np < 2) pos[np++] = k;
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        if (!((kept >> k) & 1u) && np < 2) pos[np++] = -1 - k;  // filler, value 0
-      const int pa = pos[0] < 0 ? -1 - pos[0] : pos[0];
-      const int pb = pos[1] < 0 ? -1 - pos[1] : pos[1];
-      const bool ua = pos[0] >= 0, ub = pos[1] >= 0;
-      // order the pair by position
-      if (pa < pb) {
-        a = pa; bb = pb; va = ua ? w[pa] : 0u; vb = ub ? w[pb] : 0u;
+      if (__popc(kept) == 2) {
+        // the common case: the two kept positions, lowest first
+        a = (uint32_t)(__ffs(kept) - 1);
+        bb = (uint32_t)(31 - __clz(kept));
+        va = a == 0 ? w[0] : (a == 1 ? w[1] : w[2]);   // a <= 2
+        vb = bb == 1 ? w[1] : (bb == 2 ? w[2] : w[3]);  // b >= 1
       } else {
-        a = pb; bb = pa; va = ub ? w[pb] : 0u; vb = ua ? w[pa] : 0u;
+        ptx::record_status(status, HINM_ERR_BAD_MASK);
+        // the two kept positions, lowest first; a missing one is taken from the unkept
+        // positions with value 0 so that the pair stays a legal (a < b) pattern
+        int pos[2], np = 0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (((kept >> k) & 1u) && np < 2) pos[np++] = k;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (!((kept >> k) & 1u) && np < 2) pos[np++] = -1 - k;  // filler, value 0
+        const int pa = pos[0] < 0 ? -1 - pos[0] : pos[0];
+        const int pb = pos[1] < 0 ? -1 - pos[1] : pos[1];
+        const bool ua = pos[0] >= 0, ub = pos[1] >= 0;
+        // order the pair by position
+        if (pa < pb) {
+          a = pa; bb = pb; va = ua ? w[pa] : 0u; vb = ub ? w[pb] : 0u;
+        } else {
+          a = pb; bb = pa; va = ub ? w[pb] : 0u; vb = ua ? w[pa] : 0u;
+        }
       }
     }
     *reinterpret_cast<uint32_t*>(out + swz(r, 2 * g)) = va | (vb << 16);

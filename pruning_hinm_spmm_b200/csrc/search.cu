@@ -142,14 +142,24 @@ __global__ void vector_score_kernel(const float* __restrict__ I, int K, int T,
 
 // Pass 2, thread per (tile, channel): the column's exact sum at the tile's scale, and a
 // flag when some of its values fell below that scale (summed exactly elsewhere).
+// Two fp64 accumulators carry the common values exactly: level 1 takes p >= e1 =
+// max(P - 22, lsb), level 2 takes p in [e2, e1) with e2 = max(e1 - 22, lsb).  At each level
+// a value is an integer below 2^46 in units of 2^(level - 149), and a column has at most 128
+// values, so the fp64 sums stay integers below 2^53 and never round.  Smaller values take
+// the 128-bit path (p >= lsb) or set the flag.
 __global__ void column_sum_kernel(const float* __restrict__ I, int K, int T,
                                   const int* __restrict__ tile_pmax, U128* __restrict__ colsum,
                                   unsigned char* __restrict__ coltiny) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   const int t = blockIdx.y;
   if (c >= K) return;
-  const int lsb = tile_lsb(tile_pmax[t]);
+  const int pmax = tile_pmax[t];
+  const int lsb = tile_lsb(pmax);
+  const int e1 = max(pmax - 22, lsb), e2 = max(e1 - 22, lsb);
+  const float thr1 = __uint_as_float((uint32_t)(e1 + 1) << 23);  // smallest fp32 with p >= e1
+  const float thr2 = __uint_as_float((uint32_t)(e2 + 1) << 23);
   const float* p = I + (size_t)t * T * K + c;
+  double acc1 = 0.0, acc2 = 0.0;
   U128 acc{0ull, 0ull};
   unsigned char tiny = 0;
   constexpr int kBatch = 16;
@@ -159,14 +169,28 @@ __global__ void column_sum_kernel(const float* __restrict__ I, int K, int T,
     for (int k = 0; k < kBatch; ++k) v[k] = __ldg(p + (size_t)(i0 + k) * K);
 #pragma unroll
     for (int k = 0; k < kBatch; ++k) {
-      uint32_t m;
-      int e;
-      split_f32(v[k], m, e);
-      if (!m) continue;
-      if (e >= lsb) add_shifted(acc, m, e - lsb);
-      else tiny = 1;
+      if (v[k] >= thr1) {
+        acc1 = __dadd_rn(acc1, (double)v[k]);
+      } else if (v[k] >= thr2) {
+        acc2 = __dadd_rn(acc2, (double)v[k]);
+      } else {
+        uint32_t m;
+        int e;
+        split_f32(v[k], m, e);
+        if (!m) continue;
+        if (e >= lsb) add_shifted(acc, m, e - lsb);
+        else tiny = 1;
+      }
     }
   }
+  // acc += acc1 * 2^(e1 - lsb) + acc2 * 2^(e2 - lsb)  (integers < 2^53, shifts <= 61)
+  const unsigned long long a1 = __double2ull_rz(ldexp(acc1, 149 - e1));
+  const unsigned long long a2 = __double2ull_rz(ldexp(acc2, 149 - e2));
+  const int s1 = e1 - lsb, s2 = e2 - lsb;
+  U128 f1{a1 << s1, s1 ? (a1 >> (64 - s1)) : 0ull};
+  U128 f2{a2 << s2, s2 ? (a2 >> (64 - s2)) : 0ull};
+  add128(acc, f1);
+  add128(acc, f2);
   colsum[(size_t)t * K + c] = acc;
   coltiny[(size_t)t * K + c] = tiny;
 }
