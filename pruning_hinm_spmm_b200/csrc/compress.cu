@@ -15,20 +15,90 @@
 
 namespace hinm {
 
-__global__ void tile_info_kernel(const int32_t* __restrict__ counts, int nt, int K,
-                                 int max_dense, int max_sparse, int32_t* __restrict__ info,
-                                 int* status) {
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+// One CTA of 1024 threads: each thread takes a contiguous run of tiles; the block offsets
+// are an exclusive prefix sum over the tiles.  Should the blocks exceed the layout's
+// capacity (the caller sized it for other counts), the tiles are walked in order instead,
+// and a tile that does not fit gets no blocks.
+constexpr int kTileInfoThreads = 1024;
+
+__device__ __forceinline__ void tile_blocks(const int32_t* counts, int t, int K, int& nd, int& ns,
+                                            int* status) {
+  const int n0 = counts[3 * t], n24 = counts[3 * t + 1], n4 = counts[3 * t + 2];
+  nd = ns = 0;
+  if (n0 < 0 || n24 < 0 || n4 < 0 || n0 + n24 + n4 != K || (n24 & 3)) {
+    ptx::record_status(status, HINM_ERR_INVALID_ARG);
+  } else {
+    nd = (n4 + kDenseBK - 1) / kDenseBK;
+    ns = (n24 + kSparseBK - 1) / kSparseBK;
+  }
+}
+
+__global__ void __launch_bounds__(kTileInfoThreads) tile_info_kernel(
+    const int32_t* __restrict__ counts, int nt, int K, int max_dense, int max_sparse,
+    int32_t* __restrict__ info, int* status) {
+  __shared__ int wd[32], ws[32];
+  __shared__ int tot_d, tot_s;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int per = (nt + kTileInfoThreads - 1) / kTileInfoThreads;
+  const int t0 = threadIdx.x * per, t1 = min(nt, t0 + per);
+  int sd = 0, ss = 0;
+  for (int t = t0; t < t1; ++t) {
+    int nd, ns;
+    tile_blocks(counts, t, K, nd, ns, nullptr);
+    sd += nd;
+    ss += ns;
+  }
+  // exclusive block scan of (sd, ss)
+  int id = sd, is = ss;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int xd = __shfl_up_sync(0xffffffffu, id, o), xs = __shfl_up_sync(0xffffffffu, is, o);
+    if (lane >= o) {
+      id += xd;
+      is += xs;
+    }
+  }
+  if (lane == 31) {
+    wd[warp] = id;
+    ws[warp] = is;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int vd = wd[lane], vs = ws[lane];
+    int cd = vd, cs = vs;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int xd = __shfl_up_sync(0xffffffffu, cd, o), xs = __shfl_up_sync(0xffffffffu, cs, o);
+      if (lane >= o) {
+        cd += xd;
+        cs += xs;
+      }
+    }
+    wd[lane] = cd - vd;
+    ws[lane] = cs - vs;
+    if (lane == 31) {
+      tot_d = cd;
+      tot_s = cs;
+    }
+  }
+  __syncthreads();
+  if (tot_d <= max_dense && tot_s <= max_sparse) {
+    int d0 = wd[warp] + id - sd, s0 = ws[warp] + is - ss;
+    for (int t = t0; t < t1; ++t) {
+      int nd, ns;
+      tile_blocks(counts, t, K, nd, ns, status);
+      info[4 * t + 0] = nd;
+      info[4 * t + 1] = ns;
+      info[4 * t + 2] = d0;
+      info[4 * t + 3] = s0;
+      d0 += nd;
+      s0 += ns;
+    }
+    return;
+  }
+  if (threadIdx.x != 0) return;
   int d0 = 0, s0 = 0;
   for (int t = 0; t < nt; ++t) {
-    const int n0 = counts[3 * t], n24 = counts[3 * t + 1], n4 = counts[3 * t + 2];
-    int nd = 0, ns = 0;
-    if (n0 < 0 || n24 < 0 || n4 < 0 || n0 + n24 + n4 != K || (n24 & 3)) {
-      ptx::record_status(status, HINM_ERR_INVALID_ARG);
-    } else {
-      nd = (n4 + kDenseBK - 1) / kDenseBK;
-      ns = (n24 + kSparseBK - 1) / kSparseBK;
-    }
+    int nd, ns;
+    tile_blocks(counts, t, K, nd, ns, status);
     if (d0 + nd > max_dense || s0 + ns > max_sparse) {
       ptx::record_status(status, HINM_ERR_WORKSPACE);
       nd = ns = 0;
@@ -252,8 +322,8 @@ cudaError_t launch_compress(const uint16_t* W, const uint32_t* bitmask, const in
                             const hinm_layout& L, void* ws, int* status, cudaStream_t s) {
   const int nt = M / T;
   int32_t* lists = static_cast<int32_t*>(ws);
-  tile_info_kernel<<<1, 32, 0, s>>>(counts, nt, K, L.max_dense_blocks, L.max_sparse_blocks,
-                                    L.tile_info, status);
+  tile_info_kernel<<<1, kTileInfoThreads, 0, s>>>(counts, nt, K, L.max_dense_blocks,
+                                                  L.max_sparse_blocks, L.tile_info, status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // lists are read only at positions below the counts, so no clearing is needed

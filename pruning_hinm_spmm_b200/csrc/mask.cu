@@ -5,7 +5,8 @@
 //
 //   inverse_perm_kernel   pinv[perm[j]] = j (checks that perm is a permutation)
 //   classify_kernel       one CTA per tile: region of every working position and the
-//                         2:4 members in ascending working position (member[t][q])
+//                         2:4 members' input channels in ascending working position
+//                         (member[t][q])
 //   bitmask_kernel        one CTA per (tile, 16 rows): dense words by ballot over the
 //                         region, 2:4 groups top-2 of 4 per row, words assembled in shared
 //                         memory and written once, coalesced.
@@ -91,7 +92,7 @@ __global__ void __launch_bounds__(1024) classify_kernel(const int32_t* __restric
       cls = HINM_REGION_DENSE;
     } else if (r < n4 + n24) {
       cls = HINM_REGION_24;
-      mem[pos++] = j;
+      mem[pos++] = c;
     }
     reg[c] = cls;
   }
@@ -104,6 +105,13 @@ __global__ void __launch_bounds__(1024) classify_kernel(const int32_t* __restric
 // to one group, so every keep byte has one writer.  The mask words are then assembled by
 // warp ballots, 32 words per warp and row, and stored coalesced.
 constexpr int kMaskThreads = 256;
+
+// Slot of channel c in the channel-major shared rows (rows padded to a multiple of 8
+// channels): within each aligned group of 8 channels the 16-byte bank slot is permuted by
+// higher bits of c, so that strided channels of consecutive groups use different banks.
+__device__ __forceinline__ int mask_chan_slot(int c) {
+  return (c & ~7) | ((c ^ (c >> 3) ^ (c >> 6)) & 7);
+}
 
 template <int RB>
 __device__ __forceinline__ void mask_load_rows(const float* p, float (&v)[RB]) {
@@ -125,12 +133,12 @@ __device__ __forceinline__ void mask_load_rows(const float* p, float (&v)[RB]) {
 
 template <int RB>
 __global__ void __launch_bounds__(kMaskThreads) bitmask_kernel(
-    const float* __restrict__ I, const int32_t* __restrict__ perm,
-    const int8_t* __restrict__ region, const int32_t* __restrict__ counts,
+    const float* __restrict__ I, const int8_t* __restrict__ region, const int32_t* __restrict__ counts,
     const int32_t* __restrict__ member, int K, int T, uint32_t* __restrict__ bitmask) {
   extern __shared__ __align__(16) uint8_t mask_smem[];
-  float* rows_s = reinterpret_cast<float*>(mask_smem);  // [K][RB]
-  uint8_t* keep = mask_smem + (size_t)K * RB * sizeof(float);
+  const int K8 = (K + 7) & ~7;
+  float* rows_s = reinterpret_cast<float*>(mask_smem);  // [K8][RB], mask_chan_slot order
+  uint8_t* keep = mask_smem + (size_t)K8 * RB * sizeof(float);
   const int words = (K + 31) >> 5;
   const int t = blockIdx.y;
   const int r0 = blockIdx.x * RB;  // first row of the chunk within the tile
@@ -143,7 +151,7 @@ __global__ void __launch_bounds__(kMaskThreads) bitmask_kernel(
     float v[RB];
 #pragma unroll
     for (int r = 0; r < RB; ++r) v[r] = __ldg(src + (size_t)r * K + c);
-    float* d = rows_s + (size_t)c * RB;
+    float* d = rows_s + (size_t)mask_chan_slot(c) * RB;
     if constexpr (RB == 8) {
       reinterpret_cast<float4*>(d)[0] = make_float4(v[0], v[1], v[2], v[3]);
       reinterpret_cast<float4*>(d)[1] = make_float4(v[4], v[5], v[6], v[7]);
@@ -164,15 +172,15 @@ __global__ void __launch_bounds__(kMaskThreads) bitmask_kernel(
   const int ng = n24 / 4;
   const int32_t* mem = member + (size_t)t * K;
   for (int g = threadIdx.x; g < ng; g += kMaskThreads) {
-    const int4 jq = __ldg(reinterpret_cast<const int4*>(mem) + g);
-    const int jj[4] = {jq.x, jq.y, jq.z, jq.w};
+    // the group's input channels, in ascending working position (k = 0..3)
+    const int4 cq = __ldg(reinterpret_cast<const int4*>(mem) + g);
+    const int cc[4] = {cq.x, cq.y, cq.z, cq.w};
     int c[4];
     float v[4][RB];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const int j = ((unsigned)jj[k] < (unsigned)K) ? jj[k] : 0;  // never index outside perm / I
-      c[k] = ptx::perm_at(perm, j, K);
-      mask_load_rows<RB>(rows_s + (size_t)c[k] * RB, v[k]);
+      c[k] = ((unsigned)cc[k] < (unsigned)K) ? cc[k] : 0;  // never index outside I
+      mask_load_rows<RB>(rows_s + (size_t)mask_chan_slot(c[k]) * RB, v[k]);
     }
     uint32_t kb[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
@@ -219,8 +227,9 @@ __global__ void __launch_bounds__(kMaskThreads) bitmask_kernel(
 // Rows per bitmask CTA: the largest power of two <= 8 whose rows fit in 64 KB of shared
 // memory (T is a multiple of it).
 static int mask_rows(int K) {
+  const size_t K8 = ((size_t)K + 7) & ~size_t(7);
   int rb = 8;
-  while (rb > 1 && (size_t)rb * K * sizeof(float) > 64u * 1024u) rb >>= 1;
+  while (rb > 1 && (size_t)rb * K8 * sizeof(float) > 64u * 1024u) rb >>= 1;
   return rb;
 }
 
@@ -262,7 +271,7 @@ cudaError_t launch_mask(const float* I, const int32_t* perm, const int32_t* coun
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int RB = mask_rows(K);
-  const size_t smem = (size_t)RB * K * sizeof(float) + (size_t)K;
+  const size_t smem = (size_t)RB * (((size_t)K + 7) & ~size_t(7)) * sizeof(float) + (size_t)K;
   static bool attr_set = false;
   if (!attr_set) {
     for (auto fn : {bitmask_kernel<1>, bitmask_kernel<2>, bitmask_kernel<4>, bitmask_kernel<8>}) {
@@ -274,13 +283,13 @@ cudaError_t launch_mask(const float* I, const int32_t* perm, const int32_t* coun
   }
   const dim3 g(T / RB, nt);
   if (RB == 8)
-    bitmask_kernel<8><<<g, kMaskThreads, smem, s>>>(I, perm, region, counts, member, K, T, bitmask);
+    bitmask_kernel<8><<<g, kMaskThreads, smem, s>>>(I, region, counts, member, K, T, bitmask);
   else if (RB == 4)
-    bitmask_kernel<4><<<g, kMaskThreads, smem, s>>>(I, perm, region, counts, member, K, T, bitmask);
+    bitmask_kernel<4><<<g, kMaskThreads, smem, s>>>(I, region, counts, member, K, T, bitmask);
   else if (RB == 2)
-    bitmask_kernel<2><<<g, kMaskThreads, smem, s>>>(I, perm, region, counts, member, K, T, bitmask);
+    bitmask_kernel<2><<<g, kMaskThreads, smem, s>>>(I, region, counts, member, K, T, bitmask);
   else
-    bitmask_kernel<1><<<g, kMaskThreads, smem, s>>>(I, perm, region, counts, member, K, T, bitmask);
+    bitmask_kernel<1><<<g, kMaskThreads, smem, s>>>(I, region, counts, member, K, T, bitmask);
   return cudaGetLastError();
 }
 

@@ -110,6 +110,11 @@ __device__ __forceinline__ int tile_lsb(int pmax) {
   return pmax > kHeadroomShift ? pmax - kHeadroomShift : 0;
 }
 
+// 2^e as an fp64, -1022 <= e <= 1023 (built from its bits; multiplying by it is exact).
+__device__ __forceinline__ double pow2(int e) {
+  return __longlong_as_double((long long)(1023 + e) << 52);
+}
+
 // Pass 1, thread per (tile, channel): V[t, c] = sum over the tile's rows, ascending, of
 // I (fp64), and the tile's largest exponent P.
 __global__ void vector_score_kernel(const float* __restrict__ I, int K, int T,
@@ -184,8 +189,8 @@ __global__ void column_sum_kernel(const float* __restrict__ I, int K, int T,
     }
   }
   // acc += acc1 * 2^(e1 - lsb) + acc2 * 2^(e2 - lsb)  (integers < 2^53, shifts <= 61)
-  const unsigned long long a1 = __double2ull_rz(ldexp(acc1, 149 - e1));
-  const unsigned long long a2 = __double2ull_rz(ldexp(acc2, 149 - e2));
+  const unsigned long long a1 = __double2ull_rz(__dmul_rn(acc1, pow2(149 - e1)));
+  const unsigned long long a2 = __double2ull_rz(__dmul_rn(acc2, pow2(149 - e2)));
   const int s1 = e1 - lsb, s2 = e2 - lsb;
   U128 f1{a1 << s1, s1 ? (a1 >> (64 - s1)) : 0ull};
   U128 f2{a2 << s2, s2 ? (a2 >> (64 - s2)) : 0ull};
@@ -476,6 +481,13 @@ __global__ void __launch_bounds__(512) candidate_lists_kernel(
   }
 }
 
+// Slot of channel c in the channel-major shared rows: within each aligned group of 8
+// channels, the 16-byte bank slot is permuted by higher bits of c, so that the strided
+// channels of consecutive groups (4, 8, 16, 32 or 64 apart) fall into different banks.
+__device__ __forceinline__ int chan_slot(int c) {
+  return (c & ~7) | ((c ^ (c >> 3) ^ (c >> 6)) & 7);
+}
+
 // Loads RB consecutive floats (one channel's rows of the chunk) from shared memory.
 template <int RB>
 __device__ __forceinline__ void load_rows(const float* p, float (&v)[RB]) {
@@ -536,23 +548,23 @@ __device__ __forceinline__ void band_slow(float v, U128& ex, int lsb, unsigned l
 // rounds (it stays an integer multiple of u below 2^53 u).  Values with p < eb (rare: 2^24
 // below the tile's largest) go to band_slow.  Per candidate, each warp adds its threads'
 // integer sums with three 21-bit-piece reductions and one shared atomic.
-template <int RB>
-__global__ void __launch_bounds__(512) band_sum_kernel(
+template <int RB, int kThreads>
+__global__ void __launch_bounds__(kThreads) band_sum_kernel(
     const float* __restrict__ I, const unsigned short* __restrict__ band,
     const int* __restrict__ tile_pmax, int K, int T, CandidateList cl, int ncand,
     U128* __restrict__ part, unsigned long long* __restrict__ bucket,
     int* __restrict__ bucket_used) {
-  extern __shared__ __align__(16) float rows_s[];  // [K][RB]
+  extern __shared__ __align__(16) float rows_s[];  // [K rounded up to 8][RB], chan_slot order
   __shared__ unsigned long long fast_sum[kMaxCandidates];   // units of 2^(eb - 149)
   __shared__ unsigned long long digits[kMaxCandidates][4];  // slow path, units of 2^(lsb - 149)
   const int chunk = blockIdx.x, t = blockIdx.y;
   const int nchunks = gridDim.x;
   const int lane = threadIdx.x & 31;
-  constexpr int kThreads = 512;
   const int pmax = tile_pmax[t];
   const int lsb = tile_lsb(pmax);
   const int eb = max(pmax - 24, lsb);
   const float thr = __uint_as_float((uint32_t)(eb + 1) << 23);  // smallest fp32 with p >= eb
+  const double unit_scale = pow2(149 - eb);                      // fp64 sum -> integer units
   for (int x = threadIdx.x; x < kMaxCandidates; x += kThreads) fast_sum[x] = 0ull;
   for (int x = threadIdx.x; x < kMaxCandidates * 4; x += kThreads) (&digits[0][0])[x] = 0ull;
   const float* src = I + ((size_t)t * T + (size_t)chunk * RB) * K;
@@ -560,7 +572,7 @@ __global__ void __launch_bounds__(512) band_sum_kernel(
     float v[RB];
 #pragma unroll
     for (int r = 0; r < RB; ++r) v[r] = __ldg(src + (size_t)r * K + c);
-    store_rows<RB>(rows_s + (size_t)c * RB, v);
+    store_rows<RB>(rows_s + (size_t)chan_slot(c) * RB, v);
   }
   __syncthreads();
 
@@ -591,10 +603,10 @@ __global__ void __launch_bounds__(512) band_sum_kernel(
     for (int g = q_m; g < ng; g += kThreads) {
       const ushort4 cq = g == q_m ? cq0 : __ldg(reinterpret_cast<const ushort4*>(bl) + g);
       float v0[RB], v1[RB], v2[RB], v3[RB];
-      load_rows<RB>(rows_s + (size_t)min((int)cq.x, K - 1) * RB, v0);
-      load_rows<RB>(rows_s + (size_t)min((int)cq.y, K - 1) * RB, v1);
-      load_rows<RB>(rows_s + (size_t)min((int)cq.z, K - 1) * RB, v2);
-      load_rows<RB>(rows_s + (size_t)min((int)cq.w, K - 1) * RB, v3);
+      load_rows<RB>(rows_s + (size_t)chan_slot(min((int)cq.x, K - 1)) * RB, v0);
+      load_rows<RB>(rows_s + (size_t)chan_slot(min((int)cq.y, K - 1)) * RB, v1);
+      load_rows<RB>(rows_s + (size_t)chan_slot(min((int)cq.z, K - 1)) * RB, v2);
+      load_rows<RB>(rows_s + (size_t)chan_slot(min((int)cq.w, K - 1)) * RB, v3);
 #pragma unroll
       for (int r = 0; r < RB; ++r) {
         const float a = fmaxf(v0[r], v1[r]), b = fminf(v0[r], v1[r]);
@@ -611,7 +623,7 @@ __global__ void __launch_bounds__(512) band_sum_kernel(
     }
     if (used) atomicOr(bucket_used + (size_t)t * ncand + m, 1);
     // this thread's fast sum as an integer number of units (< 2^53)
-    const unsigned long long ai = __double2ull_rz(ldexp(acc, 149 - eb));
+    const unsigned long long ai = __double2ull_rz(__dmul_rn(acc, unit_scale));
     const unsigned s0 = __reduce_add_sync(0xffffffffu, (unsigned)(ai & 0x1FFFFFull));
     const unsigned s1 = __reduce_add_sync(0xffffffffu, (unsigned)((ai >> 21) & 0x1FFFFFull));
     const unsigned s2 = __reduce_add_sync(0xffffffffu, (unsigned)(ai >> 42));
@@ -637,7 +649,7 @@ __global__ void __launch_bounds__(512) band_sum_kernel(
   }
   __syncthreads();
   if ((int)threadIdx.x < ncand) {
-    // fold the digits' carries (each digit word is below 2^37: at most 16 warps add)
+    // fold the digits' carries (each digit word is below 2^38: at most 32 warps add)
     const unsigned long long* d = digits[threadIdx.x];
     const unsigned long long d0 = d[0];
     const unsigned long long d1 = d[1] + (d0 >> 32);
@@ -646,7 +658,7 @@ __global__ void __launch_bounds__(512) band_sum_kernel(
     U128 tot;
     tot.lo = (d0 & 0xFFFFFFFFull) | (d1 << 32);
     tot.hi = (d2 & 0xFFFFFFFFull) | (d3 << 32);
-    // + fast_sum * 2^(eb - lsb): fast_sum < 2^62 (16 warps x 32 threads x 2^53), eb - lsb <= 59
+    // + fast_sum * 2^(eb - lsb): fast_sum < 2^63 (32 warps x 32 threads x 2^53), eb - lsb <= 59
     const unsigned long long f = fast_sum[threadIdx.x];
     const int sh = eb - lsb;
     U128 fx;
@@ -693,13 +705,18 @@ __global__ void finalize_kernel(const U128* __restrict__ rdense, const U128* __r
   }
 }
 
-// Rows per band_sum CTA: the largest power of two <= 8 whose rows fit in ~96 KB of shared
-// memory, so that two CTAs share an SM (T is a multiple of it).  Wider rows (K > 24576)
-// would need one row of more than 96 KB; K is at most 16384.
-static int band_rows(int K) {
-  int rb = 8;
-  while (rb > 1 && (size_t)rb * K * sizeof(float) > 96u * 1024u) rb >>= 1;
-  return rb;
+// Rows and threads per band_sum CTA: the largest power of two <= 4 rows whose rows fit in
+// 96 KB of shared memory, 512 threads, two CTAs per SM (T is a multiple of the rows; K <=
+// 16384 keeps one row within 96 KB).  A thread then adds at most 32 values per candidate.
+// (8 rows with 1024 threads, one CTA per SM, measured slower on the 4096-channel workload.)
+struct BandCfg {
+  int rows, threads;
+};
+static BandCfg band_config(int K) {
+  const size_t K8 = ((size_t)K + 7) & ~size_t(7);  // chan_slot stays below K rounded up to 8
+  int rb = 4;
+  while (rb > 1 && (size_t)rb * K8 * sizeof(float) > 96u * 1024u) rb >>= 1;
+  return {rb, 512};
 }
 
 size_t search_workspace_bytes(int M, int K, int T, int ncand) {
@@ -712,7 +729,7 @@ size_t search_workspace_bytes(int M, int K, int T, int ncand) {
   c.take<U128>((size_t)nt * K);           // exact column sums
   c.take<unsigned char>((size_t)nt * K);  // column has values below the tile scale
   c.take<char>(rank_scratch_bytes(M, K, T));  // chunk-sorted keys for the ranking
-  const int nchunks = T / band_rows(K);
+  const int nchunks = T / band_config(K).rows;
   c.take<unsigned short>((size_t)nt * ncand * K);      // band channel lists
   c.take<U128>((size_t)nt * ncand);                    // dense exact sums
   c.take<U128>((size_t)nt * ncand * nchunks);          // 2:4 partial sums per row chunk
@@ -745,7 +762,8 @@ cudaError_t launch_boundary_search(const float* I, const int32_t* perm, int M, i
   if (e != cudaSuccess) return e;
   CandidateList cl;
   for (int i = 0; i < kMaxCandidates; ++i) cl.c[i] = i < ncand ? cands[i] : Candidate{0, 0, 0};
-  const int RB = band_rows(K);
+  const BandCfg bc = band_config(K);
+  const int RB = bc.rows;
   const int nchunks = T / RB;
   unsigned short* band = c.take<unsigned short>((size_t)nt * ncand * K);
   U128* rdense = c.take<U128>((size_t)nt * ncand);
@@ -761,24 +779,25 @@ cudaError_t launch_boundary_search(const float* I, const int32_t* perm, int M, i
                                                          bucket_used);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t smem = (size_t)RB * K * sizeof(float);
+  const size_t smem = (size_t)RB * (((size_t)K + 7) & ~size_t(7)) * sizeof(float);
   static bool attr_set = false;
   if (!attr_set) {
-    for (auto fn : {band_sum_kernel<1>, band_sum_kernel<2>, band_sum_kernel<4>, band_sum_kernel<8>}) {
+    for (auto fn : {band_sum_kernel<1, 512>, band_sum_kernel<2, 512>, band_sum_kernel<4, 512>}) {
       e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
       if (e != cudaSuccess) return e;
     }
     attr_set = true;
   }
   const dim3 gb(nchunks, nt);
-  if (RB == 8)
-    band_sum_kernel<8><<<gb, 512, smem, s>>>(I, band, pmax, K, T, cl, ncand, part, bucket, bucket_used);
-  else if (RB == 4)
-    band_sum_kernel<4><<<gb, 512, smem, s>>>(I, band, pmax, K, T, cl, ncand, part, bucket, bucket_used);
+  if (RB == 4)
+    band_sum_kernel<4, 512><<<gb, 512, smem, s>>>(I, band, pmax, K, T, cl, ncand, part, bucket,
+                                                  bucket_used);
   else if (RB == 2)
-    band_sum_kernel<2><<<gb, 512, smem, s>>>(I, band, pmax, K, T, cl, ncand, part, bucket, bucket_used);
+    band_sum_kernel<2, 512><<<gb, 512, smem, s>>>(I, band, pmax, K, T, cl, ncand, part, bucket,
+                                                  bucket_used);
   else
-    band_sum_kernel<1><<<gb, 512, smem, s>>>(I, band, pmax, K, T, cl, ncand, part, bucket, bucket_used);
+    band_sum_kernel<1, 512><<<gb, 512, smem, s>>>(I, band, pmax, K, T, cl, ncand, part, bucket,
+                                                  bucket_used);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   finalize_kernel<<<nt, 64, 0, s>>>(rdense, part, nchunks, bucket, bucket_used, pmax, ncand, cl,
