@@ -39,7 +39,11 @@ struct SpmmCfg {
   static constexpr int kChunksPerAtom = kAtomBytes / 16;
   static constexpr int kChunksPerRow = BN / 8;
   static constexpr int kABytes = kBlockBytes;
-  static constexpr int kBBytes = 128 * BN * 2;  // 128 K-rows (a 2:4 block); dense uses 64
+  // B tile: two halves of 64 K-rows (a 2:4 block uses both, a dense block the first); each
+  // half holds its column atoms one after another, 64 rows x kAtomBytes each
+  static constexpr int kBHalfBytes = 64 * BN * 2;
+  static constexpr int kBBytes = 2 * kBHalfBytes;
+  static constexpr int kBAtomStride = 64 * kAtomBytes;
   static constexpr int kEBytes = 2048;
   static constexpr int kStageBytes = kABytes + kBBytes + kEBytes;
   // split-K: CTAs of a cluster per unit; the leader's reduction buffer holds the others'
@@ -81,6 +85,7 @@ struct SpmmArgs {
   int N, T;
   int num_tiles, nblk_n, num_units;
   int split;  // CTAs (one cluster) per unit; 1 = persistent, no split
+  int x3d;    // the X tensor map is 3-D (columns within an atom, rows, atoms)
   int* status;
 };
 
@@ -117,7 +122,8 @@ struct Gather {
       const int col = n0 + cc * 8;
       const bool ok = col < N;
       const uint16_t* src = ok ? X + (size_t)xr[i] * N + col : X;
-      uint32_t off = at * (128 * C::kAtomBytes) + r * C::kAtomBytes + c * 16;
+      uint32_t off = (r >> 6) * C::kBHalfBytes + at * C::kBAtomStride + (r & 63) * C::kAtomBytes +
+                     c * 16;
       off ^= ((off >> 7) & ((1u << C::kSwzBits) - 1u)) << 4;  // shared-memory swizzle
       cp_async_16(B_s + off, src, ok ? 16u : 0u);
     }
@@ -221,13 +227,20 @@ __global__ void __launch_bounds__(288, 1)
                         full_bar(s));
           if (sparse) ptx::bulk_g2s(E_s, a.meta + blk * kMetaWords, C::kEBytes, full_bar(s));
           if (run >= 0) {
-            // one ascending run of X rows: 2-D tiled boxes of 64 rows x kAtom columns
+            // one ascending run of X rows: per half of 64 rows, one 3-D box over all the
+            // column atoms, or one 2-D box per atom
 #pragma unroll 1
-            for (int at = 0; at < BN / C::kAtom; ++at)
+            for (int h = 0; h < rows / 64; ++h) {
+              if (a.x3d) {
+                ptx::tma_load_3d(B_s + h * C::kBHalfBytes, &tmX, 0, run + h * 64, n0 / C::kAtom,
+                                 full_bar(s));
+              } else {
 #pragma unroll 1
-              for (int h = 0; h < rows / 64; ++h)
-                ptx::tma_load_2d(B_s + at * (128 * C::kAtomBytes) + h * 64 * C::kAtomBytes, &tmX,
-                                 n0 + at * C::kAtom, run + h * 64, full_bar(s));
+                for (int at = 0; at < BN / C::kAtom; ++at)
+                  ptx::tma_load_2d(B_s + h * C::kBHalfBytes + at * C::kBAtomStride, &tmX,
+                                   n0 + at * C::kAtom, run + h * 64, full_bar(s));
+              }
+            }
             ptx::mbar_arrive_count(full_bar(s), C::kProducers);  // on behalf of all producers
           }
         }
@@ -281,8 +294,9 @@ __global__ void __launch_bounds__(288, 1)
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const uint64_t ad = ptx::smem_desc(A_s + 32 * k, 16, 1024, 2);
-              const uint64_t bd = ptx::smem_desc(B_s + 32 * k * C::kAtomBytes, 128 * C::kAtomBytes,
-                                                 8 * C::kAtomBytes, C::kBLayout);
+              const uint64_t bd =
+                  ptx::smem_desc(B_s + (k >> 1) * C::kBHalfBytes + 32 * (k & 1) * C::kAtomBytes,
+                                 C::kBAtomStride, 8 * C::kAtomBytes, C::kBLayout);
               const uint32_t e = e_col + k;
               ptx::mma_sp_bf16(acc, ad, bd, e & ~1u, idesc_s | (e & 1u), (accum0 | k) ? 1u : 0u);
             }
@@ -290,7 +304,7 @@ __global__ void __launch_bounds__(288, 1)
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const uint64_t ad = ptx::smem_desc(A_s + 32 * k, 16, 1024, 2);
-              const uint64_t bd = ptx::smem_desc(B_s + 16 * k * C::kAtomBytes, 128 * C::kAtomBytes,
+              const uint64_t bd = ptx::smem_desc(B_s + 16 * k * C::kAtomBytes, C::kBAtomStride,
                                                  8 * C::kAtomBytes, C::kBLayout);
               ptx::mma_bf16(acc, ad, bd, idesc_d, (accum0 | k) ? 1u : 0u);
             }
@@ -466,11 +480,28 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// X (K rows x N bf16, row-major) as a 2-D tensor map with a box of 64 rows x `atom`
-// columns, swizzled like the B operand (atom * 2 bytes per swizzle row).
-bool make_x_map(CUtensorMap* m, const uint16_t* X, int K, int N, int atom) {
+// X (K rows x N bf16, row-major) as a tensor map swizzled like the B operand (atom * 2
+// bytes per swizzle row).  With 64-column atoms and N a multiple of 64 it is 3-D
+// (column within the atom, row, atom; the atom stride is 128 bytes) with a box of all the
+// unit's atoms for 64 rows, so one load fills a half of the B tile; else 2-D with a box of
+// 64 rows x `atom` columns.
+bool make_x_map(CUtensorMap* m, const uint16_t* X, int K, int N, int atom, int atoms, bool* x3d) {
   auto fn = encode_fn();
   if (!fn) return false;
+  *x3d = false;
+  if (atom == 64 && N % 64 == 0 && K >= 64 && atoms <= 4) {
+    cuuint64_t dims[3] = {64, (cuuint64_t)K, (cuuint64_t)(N / 64)};
+    cuuint64_t strides[2] = {(cuuint64_t)N * 2, 128};
+    cuuint32_t box[3] = {64, 64, (cuuint32_t)atoms};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(X), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r == CUDA_SUCCESS) {
+      *x3d = true;
+      return true;
+    }
+  }
   cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)K};
   cuuint64_t strides[1] = {(cuuint64_t)N * 2};
   cuuint32_t box[2] = {(cuuint32_t)atom, (cuuint32_t)(K < 64 ? K : 64)};
@@ -507,12 +538,14 @@ cudaError_t run(const hinm_layout& L, const uint16_t* X, int N, float* Y, int sp
   });
   if (attr_err != cudaSuccess) return attr_err;
   CUtensorMap map;
-  if (!make_x_map(&map, X, L.K, N, C::kAtom)) return cudaErrorInvalidValue;
+  bool x3d = false;
+  if (!make_x_map(&map, X, L.K, N, C::kAtom, BN / C::kAtom, &x3d)) return cudaErrorInvalidValue;
   const int nblk_n = (N + BN - 1) / BN;
   const int units = L.num_tiles * nblk_n;
   SpmmArgs a{L.tile_info, L.vals_dense, L.vals_sparse, L.meta,   L.idx_dense, L.idx_sparse,
              L.run_dense, L.run_sparse, X,             Y,        N,           L.T,
-             L.num_tiles, nblk_n,       units,         SPLIT ? split : 1,       status};
+             L.num_tiles, nblk_n,       units,         SPLIT ? split : 1,       x3d ? 1 : 0,
+             status};
   if constexpr (!SPLIT) {
     const int grid = units < num_sms() ? units : num_sms();
     spmm_kernel<BN, false><<<grid, C::kThreads, C::kSmemBytes, s>>>(map, a);
