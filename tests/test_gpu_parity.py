@@ -257,3 +257,53 @@ def test_extreme_dynamic_range_exact_sums(H):
     np.testing.assert_array_equal(g["rank"], sr.rank)
     bm_ref, reg_ref = O.mask(I_ref, w.perm, T, sr.counts)
     np.testing.assert_array_equal(g["bitmask"], bm_ref)
+
+
+# ---------------------------------------------------------------- LLaMA-2-7B-shaped sweep
+# The sweep's three linear shapes (q/k/v/o 4096x4096, gate/up 11008x4096, down 4096x11008),
+# each at the three target sparsities with the boundary from the search, N rotating over
+# {16, 512, 4096}: the whole path runs on the GPU; the oracle checks two sampled tiles.
+SWEEP = [("q", 0.5, 512), ("q", 0.625, 4096), ("q", 0.75, 16),
+         ("gate", 0.5, 16), ("gate", 0.625, 512), ("gate", 0.75, 4096),
+         ("down", 0.5, 4096), ("down", 0.625, 16), ("down", 0.75, 512)]
+
+
+@pytest.mark.parametrize("linear,t_s,N", SWEEP, ids=[f"{l}_ts{t}_N{n}" for l, t, n in SWEEP])
+def test_llama_sweep_searched_sampled(H, linear, t_s, N):
+    w = hi.llama_sweep_layer(0, linear, N, t_s)
+    M, K, T = w.M, w.K, w.T
+    nt = M // T
+    W, X, perm = dev_bf16(w.W_bits), dev_bf16(w.X_bits), dev_i32(w.perm)
+    hp = H.HotPath(M, K, N, T, w.t_s, w.alpha)
+    Y = hp.run(W, X, perm)  # counts from the search
+    n_c = H.hinm_search_num_candidates(K, t_s, w.alpha)
+    R_gpu = torch.empty((nt, n_c), dtype=torch.float64, device="cuda")
+    H.hinm_boundary_search(hp.I, perm, T, t_s, w.alpha, want_rank=False, retained_out=R_gpu)
+    torch.cuda.synchronize()
+    status_ok(H)
+    tiles = [0, nt - 1]
+    rows = np.concatenate([np.arange(t * T, (t + 1) * T) for t in tiles])
+    s = O.channel_energy(w.X_bits)
+    Wf = hi.bf16_bits_to_f32(w.W_bits[rows])
+    I_rows = ((Wf * Wf).astype(np.float32) * s[None, :]).astype(np.float32)
+    np.testing.assert_array_equal(hp.I[rows].cpu().numpy().view(np.uint32), I_rows.view(np.uint32))
+    I_full_rows = np.zeros((M, K), dtype=np.float32)
+    I_full_rows[rows] = I_rows
+    sr = O.boundary_search(I_full_rows, w.perm, T, t_s, w.alpha, tiles=tiles)
+    counts = hp.counts.cpu().numpy()
+    np.testing.assert_array_equal(counts[tiles], sr.counts[tiles])
+    np.testing.assert_array_equal(hp.vs.cpu().numpy()[tiles], np.asarray(sr.v_s)[tiles])
+    np.testing.assert_array_equal(hp.rank.cpu().numpy()[tiles], sr.rank[tiles])
+    R_all = R_gpu.cpu().numpy()
+    for t in tiles:  # every candidate's retained importance, bit for bit
+        np.testing.assert_array_equal(R_all[t], np.array(sr.R[t], dtype=np.float64))
+    # mask, layout and product on the sampled tiles; the layout's block offsets depend on
+    # every tile's counts, so the oracle is given the GPU's (checked above where sampled)
+    bm_ref, reg_ref = O.mask(I_full_rows, w.perm, T, counts, tiles=tiles)
+    bm = hp.bitmask.cpu().numpy().view(np.uint32)
+    np.testing.assert_array_equal(bm[rows], bm_ref[rows])
+    np.testing.assert_array_equal(hp.region.cpu().numpy()[tiles], reg_ref[tiles])
+    L_ref = O.compress(w.W_bits, bm_ref, reg_ref, w.perm, counts, T, tiles=tiles)
+    layout_equal(hp.layout, L_ref, tiles=tiles)
+    y_ref, bound = O.spmm_reference(w.W_bits, bm_ref, w.X_bits, rows=rows)
+    check_y(Y.cpu().numpy(), y_ref, bound, rows=rows)
