@@ -258,23 +258,22 @@ __global__ void __launch_bounds__(kRankChunk) chunk_sort_kernel(
   sidx[(size_t)t * Kp + j] = (unsigned short)idx;
 }
 
-// rank[t][j] = number of (key, index) pairs of the tile below position j's: one binary
-// search per sorted chunk, each chunk staged in shared memory once per CTA.
+// rank[t][j] = number of (key, index) pairs of the tile below position j's.  One CTA per
+// (tile, sorted chunk): thread i takes the i-th pair of its own sorted chunk (its rank within
+// the chunk is i) and adds, for every other chunk staged in shared memory, the number of that
+// chunk's pairs below it (binary search; consecutive threads hold increasing pairs, so their
+// searches follow nearly the same path).  The rank is then written at position j.
 __global__ void __launch_bounds__(kRankChunk) merge_rank_kernel(
-    const double* __restrict__ Vc, const int32_t* __restrict__ perm,
     const unsigned long long* __restrict__ skey, const unsigned short* __restrict__ sidx, int K,
     int Kp, int32_t* __restrict__ rank) {
   __shared__ unsigned long long ck[kRankChunk];
   __shared__ unsigned short ci[kRankChunk];
-  const int t = blockIdx.y;
-  const int j = blockIdx.x * kRankChunk + threadIdx.x;
-  unsigned long long kj = 0ull;
-  if (j < K)
-    kj = ~static_cast<unsigned long long>(
-        __double_as_longlong(__ldg(Vc + (size_t)t * K + ptx::perm_at(perm, j, K))));
-  const unsigned ij = (unsigned)j;
-  int r = 0;
+  const int t = blockIdx.y, own = blockIdx.x * kRankChunk;
+  const unsigned long long kj = __ldg(skey + (size_t)t * Kp + own + threadIdx.x);
+  const unsigned ij = __ldg(sidx + (size_t)t * Kp + own + threadIdx.x);
+  int r = threadIdx.x;
   for (int base = 0; base < Kp; base += kRankChunk) {
+    if (base == own) continue;  // uniform over the CTA
     ck[threadIdx.x] = __ldg(skey + (size_t)t * Kp + base + threadIdx.x);
     ci[threadIdx.x] = __ldg(sidx + (size_t)t * Kp + base + threadIdx.x);
     __syncthreads();
@@ -287,7 +286,7 @@ __global__ void __launch_bounds__(kRankChunk) merge_rank_kernel(
     r += lo;
     __syncthreads();
   }
-  if (j < K) rank[(size_t)t * K + j] = r;
+  if (ij < (unsigned)K) rank[(size_t)t * K + ij] = r;  // padding pairs carry index 0xFFFF
 }
 
 size_t rank_scratch_bytes(int M, int K, int T) {
@@ -317,7 +316,7 @@ cudaError_t launch_vector_rank(const float* I, const int32_t* perm, int M, int K
   chunk_sort_kernel<<<dim3(nchunk, nt), kRankChunk, 0, s>>>(V, perm, K, Kp, skey, sidx);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  merge_rank_kernel<<<dim3(nchunk, nt), kRankChunk, 0, s>>>(V, perm, skey, sidx, K, Kp, rank);
+  merge_rank_kernel<<<dim3(nchunk, nt), kRankChunk, 0, s>>>(skey, sidx, K, Kp, rank);
   return cudaGetLastError();
 }
 
@@ -409,7 +408,8 @@ struct CandidateList {
 // Per (candidate m, tile), 512 threads: the channels of the 2:4 band in ascending working
 // position (block-wide prefix count) -> band[t][m][q], and the exact sum of the dense
 // vectors' column sums -> rdense[t][m] (values below the tile's scale go to the buckets).
-__global__ void __launch_bounds__(512) candidate_lists_kernel(
+template <int kPerMax>
+__global__ void __launch_bounds__(512, 2) candidate_lists_kernel(
     const float* __restrict__ I, const int32_t* __restrict__ perm, const int32_t* __restrict__ rank,
     const int* __restrict__ tile_pmax, const U128* __restrict__ colsum,
     const unsigned char* __restrict__ coltiny, int K, int T, CandidateList cl, int ncand,
@@ -428,13 +428,18 @@ __global__ void __launch_bounds__(512) candidate_lists_kernel(
   unsigned short* out = band + ((size_t)t * ncand + m) * K;
   U128 acc{0ull, 0ull};
 
+  // each thread takes up to kPerMax consecutive working positions (kPerMax * 512 >= K);
+  // the ranks stay in registers between the counting pass and the writing pass, and the
+  // dependent loads of the second pass are issued kBatch positions at a time
+  constexpr int kBatch = 4;
   const int per = (K + blockDim.x - 1) / blockDim.x;
   const int j0 = threadIdx.x * per, j1 = min(K, j0 + per);
+  int rr[kPerMax];
+#pragma unroll
+  for (int q = 0; q < kPerMax; ++q) rr[q] = (q < per && j0 + q < j1) ? __ldg(rk + j0 + q) : -1;
   int cnt = 0;
-  for (int j = j0; j < j1; ++j) {
-    const int r = __ldg(rk + j);
-    cnt += (r >= n4 && r < n4 + n24);
-  }
+#pragma unroll
+  for (int q = 0; q < kPerMax; ++q) cnt += (rr[q] >= n4 && rr[q] < n4 + n24);
   int incl = cnt;
   for (int o = 1; o < 32; o <<= 1) {
     const int v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -445,24 +450,40 @@ __global__ void __launch_bounds__(512) candidate_lists_kernel(
   int pos = incl - cnt;
   for (int w = 0; w < warp; ++w) pos += warp_tot[w];
   bool used = false;
-  for (int j = j0; j < j1; ++j) {
-    const int r = __ldg(rk + j);
-    const int c = ptx::perm_at(perm, j, K);
-    if (r < n4) {
-      add128(acc, colsum[(size_t)t * K + c]);
-      if (coltiny[(size_t)t * K + c]) {  // values below the tile's scale: exact buckets
-        for (int i = 0; i < T; ++i) {
-          uint32_t mm;
-          int e;
-          split_f32(__ldg(It + (size_t)i * K + c), mm, e);
-          if (mm && e < lsb) {
-            atomicAdd(bkt + e, (unsigned long long)mm);
-            used = true;
+#pragma unroll
+  for (int qb = 0; qb < kPerMax; qb += kBatch) {
+    if (qb >= per) break;
+    int c[kBatch];
+    U128 cs[kBatch];
+    unsigned char tn[kBatch];
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) c[q] = rr[qb + q] >= 0 ? ptx::perm_at(perm, j0 + qb + q, K) : 0;
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+      const bool dense = rr[qb + q] >= 0 && rr[qb + q] < n4;
+      cs[q] = dense ? colsum[(size_t)t * K + c[q]] : U128{0ull, 0ull};
+      tn[q] = dense ? coltiny[(size_t)t * K + c[q]] : (unsigned char)0;
+    }
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+      const int r = rr[qb + q];
+      if (r < 0) continue;
+      if (r < n4) {
+        add128(acc, cs[q]);
+        if (tn[q]) {  // values below the tile's scale: exact buckets
+          for (int i = 0; i < T; ++i) {
+            uint32_t mm;
+            int e;
+            split_f32(__ldg(It + (size_t)i * K + c[q]), mm, e);
+            if (mm && e < lsb) {
+              atomicAdd(bkt + e, (unsigned long long)mm);
+              used = true;
+            }
           }
         }
+      } else if (r < n4 + n24) {
+        out[pos++] = (unsigned short)c[q];
       }
-    } else if (r < n4 + n24) {
-      out[pos++] = (unsigned short)c;
     }
   }
   if (used) atomicOr(bucket_used + (size_t)t * ncand + m, 1);
@@ -774,9 +795,19 @@ cudaError_t launch_boundary_search(const float* I, const int32_t* perm, int M, i
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(bucket_used, 0, (size_t)nt * ncand * sizeof(int), s);
   if (e != cudaSuccess) return e;
-  candidate_lists_kernel<<<dim3(ncand, nt), 512, 0, s>>>(I, perm, rank, pmax, colsum, coltiny, K, T,
-                                                         cl, ncand, band, rdense, bucket,
-                                                         bucket_used);
+  {
+    const dim3 gl(ncand, nt);
+    const int per = (K + 511) / 512;
+    if (per <= 8)
+      candidate_lists_kernel<8><<<gl, 512, 0, s>>>(I, perm, rank, pmax, colsum, coltiny, K, T, cl,
+                                                   ncand, band, rdense, bucket, bucket_used);
+    else if (per <= 16)
+      candidate_lists_kernel<16><<<gl, 512, 0, s>>>(I, perm, rank, pmax, colsum, coltiny, K, T, cl,
+                                                    ncand, band, rdense, bucket, bucket_used);
+    else
+      candidate_lists_kernel<32><<<gl, 512, 0, s>>>(I, perm, rank, pmax, colsum, coltiny, K, T, cl,
+                                                    ncand, band, rdense, bucket, bucket_used);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t smem = (size_t)RB * (((size_t)K + 7) & ~size_t(7)) * sizeof(float);
