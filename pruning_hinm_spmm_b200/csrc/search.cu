@@ -405,8 +405,16 @@ struct CandidateList {
   Candidate c[kMaxCandidates];
 };
 
+// Slot of channel c in the channel-major shared rows: within each aligned group of 8
+// channels, the 16-byte bank slot is permuted by higher bits of c, so that the strided
+// channels of consecutive groups (4, 8, 16, 32 or 64 apart) fall into different banks.
+__device__ __forceinline__ int chan_slot(int c) {
+  return (c & ~7) | ((c ^ (c >> 3) ^ (c >> 6)) & 7);
+}
+
 // Per (candidate m, tile), 512 threads: the channels of the 2:4 band in ascending working
-// position (block-wide prefix count) -> band[t][m][q], and the exact sum of the dense
+// position (block-wide prefix count), stored as their shared-memory slots chan_slot(c) in
+// band_sum's staged rows -> band[t][m][q], and the exact sum of the dense
 // vectors' column sums -> rdense[t][m] (values below the tile's scale go to the buckets).
 template <int kPerMax>
 __global__ void __launch_bounds__(512, 2) candidate_lists_kernel(
@@ -482,7 +490,7 @@ __global__ void __launch_bounds__(512, 2) candidate_lists_kernel(
           }
         }
       } else if (r < n4 + n24) {
-        out[pos++] = (unsigned short)c[q];
+        out[pos++] = (unsigned short)chan_slot(c[q]);
       }
     }
   }
@@ -502,12 +510,6 @@ __global__ void __launch_bounds__(512, 2) candidate_lists_kernel(
   }
 }
 
-// Slot of channel c in the channel-major shared rows: within each aligned group of 8
-// channels, the 16-byte bank slot is permuted by higher bits of c, so that the strided
-// channels of consecutive groups (4, 8, 16, 32 or 64 apart) fall into different banks.
-__device__ __forceinline__ int chan_slot(int c) {
-  return (c & ~7) | ((c ^ (c >> 3) ^ (c >> 6)) & 7);
-}
 
 // Loads RB consecutive floats (one channel's rows of the chunk) from shared memory.
 template <int RB>
@@ -559,16 +561,17 @@ __device__ __forceinline__ void band_slow(float v, U128& ex, int lsb, unsigned l
 }
 
 // Per (tile, chunk of RB rows), 512 threads.  The chunk's rows of I are staged in shared
-// memory channel-major (the RB values of channel c contiguous, one vector load each).
-// Then, candidate by candidate, the candidate's 2:4 groups are dealt round-robin to the
-// threads (the starting thread rotates with the groups dealt so far, so the work stays even
-// over all candidates) and, for every row, the top 2 of the group's 4 values are summed.
+// memory channel-major (the RB values of channel c contiguous at slot chan_slot(c), one
+// vector load each).  Then, candidate by candidate, the candidate's 2:4 groups are dealt to
+// the warps in chunks (the starting warp rotates, so the work stays even over the scan)
+// and, for every row, the top 2 of the group's 4 values are summed.
 //
 // The sums are exact.  With eb = max(P - 24, lsb) every value with p >= eb is a multiple of
-// u = 2^(eb - 149) below 2^48 u, and a thread adds at most 32 of them, so its fp64 sum never
-// rounds (it stays an integer multiple of u below 2^53 u).  Values with p < eb (rare: 2^24
-// below the tile's largest) go to band_slow.  Per candidate, each warp adds its threads'
-// integer sums with three 21-bit-piece reductions and one shared atomic.
+// u = 2^(eb - 149) below 2^48 u, and a thread adds at most 32 of them per candidate (for any
+// K <= 16384 with the rows per CTA of band_config), so its fp64 sum never rounds (it stays
+// an integer multiple of u below 2^53 u), in any order.  Values with p < eb (rare: 2^24 below
+// the tile's largest) go to band_slow.  Per candidate, each warp adds its threads' integer
+// sums with three 21-bit-piece reductions and one shared atomic.
 template <int RB, int kThreads>
 __global__ void __launch_bounds__(kThreads) band_sum_kernel(
     const float* __restrict__ I, const unsigned short* __restrict__ band,
@@ -581,6 +584,7 @@ __global__ void __launch_bounds__(kThreads) band_sum_kernel(
   const int chunk = blockIdx.x, t = blockIdx.y;
   const int nchunks = gridDim.x;
   const int lane = threadIdx.x & 31;
+  const int K8 = (K + 7) & ~7;
   const int pmax = tile_pmax[t];
   const int lsb = tile_lsb(pmax);
   const int eb = max(pmax - 24, lsb);
@@ -598,47 +602,63 @@ __global__ void __launch_bounds__(kThreads) band_sum_kernel(
   __syncthreads();
 
   const unsigned short* band_t = band + (size_t)t * ncand * K;
-  auto first_group = [&](int off) {
-    int q = (int)threadIdx.x - off;
-    return q < 0 ? q + kThreads : q;
-  };
-  int off = 0;  // groups dealt before this candidate, mod kThreads
-  int q = first_group(off);
-  ushort4 cq_next = make_ushort4(0, 0, 0, 0);
-  if (ncand > 0 && q < cl.c[0].n24 / 4) cq_next = __ldg(reinterpret_cast<const ushort4*>(band_t) + q);
+  // A candidate's groups go out in warp chunks of 32 * kG consecutive groups (kG per thread);
+  // chunk k of candidate m goes to warp (woff + k) mod nwarps, and woff advances by the
+  // candidate's chunk count, so the warps' work stays even over the scan.
+  constexpr int kG = 4;
+  constexpr int nwarps = kThreads / 32;
+  const int warp = threadIdx.x >> 5;
+  int woff = 0;
   for (int m = 0; m < ncand; ++m) {
     const int ng = cl.c[m].n24 / 4;
-    const ushort4 cq0 = cq_next;
-    const int q_m = q;
-    off = (off + ng) % kThreads;
-    q = first_group(off);
-    if (m + 1 < ncand && q < cl.c[m + 1].n24 / 4)
-      cq_next = __ldg(reinterpret_cast<const ushort4*>(band_t + (size_t)(m + 1) * K) + q);
-    const bool active = q_m < ng;
-    if (!__any_sync(0xffffffffu, active)) continue;  // warp-uniform
-    const unsigned short* bl = band_t + (size_t)m * K;
+    const int nchunk = (ng + 32 * kG - 1) / (32 * kG);
+    int k0 = (warp - woff) % nwarps;
+    if (k0 < 0) k0 += nwarps;
+    woff = (woff + nchunk) % nwarps;
+    if (k0 >= nchunk) continue;  // warp-uniform: no chunk of this candidate here
+    const ushort4* bl = reinterpret_cast<const ushort4*>(band_t + (size_t)m * K);
     unsigned long long* bkt = bucket + ((size_t)t * ncand + m) * 256;
     double acc = 0.0;
     U128 ex{0ull, 0ull};
     bool used = false;
-    for (int g = q_m; g < ng; g += kThreads) {
-      const ushort4 cq = g == q_m ? cq0 : __ldg(reinterpret_cast<const ushort4*>(bl) + g);
-      float v0[RB], v1[RB], v2[RB], v3[RB];
-      load_rows<RB>(rows_s + (size_t)chan_slot(min((int)cq.x, K - 1)) * RB, v0);
-      load_rows<RB>(rows_s + (size_t)chan_slot(min((int)cq.y, K - 1)) * RB, v1);
-      load_rows<RB>(rows_s + (size_t)chan_slot(min((int)cq.z, K - 1)) * RB, v2);
-      load_rows<RB>(rows_s + (size_t)chan_slot(min((int)cq.w, K - 1)) * RB, v3);
+    for (int k = k0; k < nchunk; k += nwarps) {
+      const int gb = k * 32 * kG + lane;
+      ushort4 cq[kG];
 #pragma unroll
-      for (int r = 0; r < RB; ++r) {
-        const float a = fmaxf(v0[r], v1[r]), b = fminf(v0[r], v1[r]);
-        const float cc = fmaxf(v2[r], v3[r]), d = fminf(v2[r], v3[r]);
-        const float t1 = fmaxf(a, cc), t2 = fmaxf(fminf(a, cc), fmaxf(b, d));
-        if (t2 >= thr) {
-          acc = __dadd_rn(acc, __dadd_rn((double)t1, (double)t2));
+      for (int j = 0; j < kG; ++j)
+        cq[j] = gb + 32 * j < ng ? __ldg(bl + gb + 32 * j) : make_ushort4(0, 0, 0, 0);
+#pragma unroll
+      for (int j = 0; j < kG; ++j) {
+        if (gb + 32 * j >= ng) break;
+        // the lists hold shared-memory slots (chan_slot of the channel), below K rounded up to 8
+        float v0[RB], v1[RB], v2[RB], v3[RB];
+        load_rows<RB>(rows_s + min((int)cq[j].x, K8 - 1) * RB, v0);
+        load_rows<RB>(rows_s + min((int)cq[j].y, K8 - 1) * RB, v1);
+        load_rows<RB>(rows_s + min((int)cq[j].z, K8 - 1) * RB, v2);
+        load_rows<RB>(rows_s + min((int)cq[j].w, K8 - 1) * RB, v3);
+        float t1[RB], t2[RB];
+        float lo = INFINITY;
+#pragma unroll
+        for (int r = 0; r < RB; ++r) {
+          const float a = fmaxf(v0[r], v1[r]), b = fminf(v0[r], v1[r]);
+          const float cc = fmaxf(v2[r], v3[r]), d = fminf(v2[r], v3[r]);
+          t1[r] = fmaxf(a, cc);
+          t2[r] = fmaxf(fminf(a, cc), fmaxf(b, d));
+          lo = fminf(lo, t2[r]);
+        }
+        if (lo >= thr) {  // every value of the group on the fast path (t1 >= t2 >= thr)
+          double g = 0.0;
+#pragma unroll
+          for (int r = 0; r < RB; ++r) g = __dadd_rn(g, __dadd_rn((double)t1[r], (double)t2[r]));
+          acc = __dadd_rn(acc, g);
         } else {
-          if (t1 >= thr) acc = __dadd_rn(acc, (double)t1);
-          else band_slow(t1, ex, lsb, bkt, used);
-          band_slow(t2, ex, lsb, bkt, used);
+#pragma unroll
+          for (int r = 0; r < RB; ++r) {
+            if (t1[r] >= thr) acc = __dadd_rn(acc, (double)t1[r]);
+            else band_slow(t1[r], ex, lsb, bkt, used);
+            if (t2[r] >= thr) acc = __dadd_rn(acc, (double)t2[r]);
+            else band_slow(t2[r], ex, lsb, bkt, used);
+          }
         }
       }
     }
