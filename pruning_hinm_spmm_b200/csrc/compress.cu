@@ -217,13 +217,29 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint16_t* __restrict__ 
     else L.run_dense[d0 + b] = run ? c0 : -1;
   }
 
+  // a block whose channels are one run c0, c0+1, ...: a group's (or 8 vectors') weights are
+  // consecutive in W's row and their mask bits share one word, so they move with one load each
+  const bool run8 = run && (c0 & 7) == 0 && (K & 7) == 0;  // 16-byte loads of 8 weights
+  const bool run4 = run && (c0 & 3) == 0;                  // 8-byte loads of 4 weights
+
   if (!sparse) {
     uint8_t* out = reinterpret_cast<uint8_t*>(L.vals_dense + (size_t)(d0 + b) * 8192);
 #pragma unroll 2
     for (int item = threadIdx.x; item < 128 * 8; item += blockDim.x) {
       const int r = item >> 3, ch = item & 7;
       uint32_t h[8];
-      if (r < T) {
+      if (r < T && run8) {
+        const int i = row0 + r;
+        const int cb = c0 + ch * 8;
+        const uint4 wv = __ldg(reinterpret_cast<const uint4*>(W + (size_t)i * K + cb));
+        const uint32_t bits = (__ldg(bitmask + (size_t)i * words + (cb >> 5)) >> (cb & 31)) & 0xFFu;
+        const uint32_t wr[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          h[2 * p] = ((bits >> (2 * p)) & 1u) ? (wr[p] & 0xFFFFu) : 0u;
+          h[2 * p + 1] = ((bits >> (2 * p + 1)) & 1u) ? (wr[p] >> 16) : 0u;
+        }
+      } else if (r < T) {
         const int i = row0 + r;
         const uint16_t* Wi = W + (size_t)i * K;
         const uint32_t* bmi = bitmask + (size_t)i * words;
@@ -250,7 +266,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint16_t* __restrict__ 
   }
 
   uint8_t* out = reinterpret_cast<uint8_t*>(L.vals_sparse + (size_t)(s0 + sb) * 8192);
-#pragma unroll 2
+#pragma unroll 4
   for (int item = threadIdx.x; item < 128 * 32; item += blockDim.x) {
     const int r = item >> 5, g = item & 31;
     uint32_t a = 0, bb = 1, va = 0, vb = 0;
@@ -259,11 +275,21 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint16_t* __restrict__ 
       const uint16_t* Wi = W + (size_t)i * K;
       const uint32_t* bmi = bitmask + (size_t)i * words;
       uint32_t w[4], kept = 0;
+      if (run4) {
+        const int cb = c0 + 4 * g;
+        const uint2 wv = __ldg(reinterpret_cast<const uint2*>(Wi + cb));
+        w[0] = wv.x & 0xFFFFu;
+        w[1] = wv.x >> 16;
+        w[2] = wv.y & 0xFFFFu;
+        w[3] = wv.y >> 16;
+        kept = (__ldg(bmi + (cb >> 5)) >> (cb & 31)) & 0xFu;
+      } else {
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int c = chan[4 * g + k];
-        w[k] = __ldg(Wi + c);
-        kept |= ((__ldg(bmi + (c >> 5)) >> (c & 31)) & 1u) << k;
+        for (int k = 0; k < 4; ++k) {
+          const int c = chan[4 * g + k];
+          w[k] = __ldg(Wi + c);
+          kept |= ((__ldg(bmi + (c >> 5)) >> (c & 31)) & 1u) << k;
+        }
       }
       if (__popc(kept) == 2) {
         // the common case: the two kept positions, lowest first

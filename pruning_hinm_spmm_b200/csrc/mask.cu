@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(1024) classify_kernel(const int32_t* __restric
 // the top 2 of its group (ties: the lower working position wins).  Each channel belongs
 // to one group, so every keep byte has one writer.  The mask words are then assembled by
 // warp ballots, 32 words per warp and row, and stored coalesced.
-constexpr int kMaskThreads = 256;
+constexpr int kMaskThreads = 512;
 
 // Slot of channel c in the channel-major shared rows (rows padded to a multiple of 8
 // channels): within each aligned group of 8 channels the 16-byte bank slot is permuted by
