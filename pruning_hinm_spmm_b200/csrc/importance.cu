@@ -82,24 +82,40 @@ __global__ void __launch_bounds__(kEnergyThreads) channel_energy_kernel(
   if (threadIdx.x < nch) s[c0 + threadIdx.x] = __double2float_rn(acc);
 }
 
-// 4 consecutive elements of one row per thread (K % 4 == 0).
+// 4 consecutive elements of one row per quad (K % 4 == 0); each thread takes kQuads quads
+// per pass of the grid-stride loop, their loads issued before any arithmetic.
+constexpr int kQuads = 4;
+
 __global__ void importance_kernel(const uint16_t* __restrict__ W, const float* __restrict__ s,
                                   int M, int K, float* __restrict__ I) {
   const long long total4 = (long long)M * K / 4;
   const int k4 = K / 4;
-  for (long long q = blockIdx.x * (long long)blockDim.x + threadIdx.x; q < total4;
-       q += (long long)gridDim.x * blockDim.x) {
-    const int c = (int)(q % k4) * 4;
-    const uint2 wv = __ldg(reinterpret_cast<const uint2*>(W) + q);
-    const float4 sv = __ldg(reinterpret_cast<const float4*>(s + c));
-    const float w0 = __uint_as_float(wv.x << 16), w1 = __uint_as_float(wv.x & 0xFFFF0000u);
-    const float w2 = __uint_as_float(wv.y << 16), w3 = __uint_as_float(wv.y & 0xFFFF0000u);
-    float4 o;
-    o.x = __fmul_rn(__fmul_rn(w0, w0), sv.x);
-    o.y = __fmul_rn(__fmul_rn(w1, w1), sv.y);
-    o.z = __fmul_rn(__fmul_rn(w2, w2), sv.z);
-    o.w = __fmul_rn(__fmul_rn(w3, w3), sv.w);
-    __stcs(reinterpret_cast<float4*>(I) + q, o);
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long q0 = blockIdx.x * (long long)blockDim.x + threadIdx.x; q0 < total4;
+       q0 += stride * kQuads) {
+    uint2 wv[kQuads];
+    float4 sv[kQuads];
+#pragma unroll
+    for (int u = 0; u < kQuads; ++u) {
+      const long long q = q0 + u * stride;
+      if (q < total4) {
+        wv[u] = __ldg(reinterpret_cast<const uint2*>(W) + q);
+        sv[u] = __ldg(reinterpret_cast<const float4*>(s + (int)(q % k4) * 4));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kQuads; ++u) {
+      const long long q = q0 + u * stride;
+      if (q >= total4) break;
+      const float w0 = __uint_as_float(wv[u].x << 16), w1 = __uint_as_float(wv[u].x & 0xFFFF0000u);
+      const float w2 = __uint_as_float(wv[u].y << 16), w3 = __uint_as_float(wv[u].y & 0xFFFF0000u);
+      float4 o;
+      o.x = __fmul_rn(__fmul_rn(w0, w0), sv[u].x);
+      o.y = __fmul_rn(__fmul_rn(w1, w1), sv[u].y);
+      o.z = __fmul_rn(__fmul_rn(w2, w2), sv[u].z);
+      o.w = __fmul_rn(__fmul_rn(w3, w3), sv[u].w);
+      __stcs(reinterpret_cast<float4*>(I) + q, o);
+    }
   }
 }
 
