@@ -63,18 +63,23 @@ __global__ void __launch_bounds__(kEnergyThreads) channel_energy_kernel(
     }
     __syncthreads();
     if (threadIdx.x < nch) {
-      const int vals = min(kEnergyChunk, N - chunk * kEnergyChunk);
+      const int nv = min(kEnergyChunk, N - chunk * kEnergyChunk) / 8;
       const uint4* row = reinterpret_cast<const uint4*>(buf[chunk & 1] + threadIdx.x * kEnergyRowBytes);
-      for (int v = 0; v < vals / 8; ++v) {
-        const uint4 q = row[v];
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+      uint4 q = row[0];
+      for (int v = 0; v < nv; ++v) {
+        const uint4 cur = q;
+        if (v + 1 < nv) q = row[v + 1];  // next 8 values in flight during this chain
+        const uint32_t w[4] = {cur.x, cur.y, cur.z, cur.w};
+        double sq[8];  // x^2 of a bf16 is exact in fp64; computed off the chain
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
           const double a = bf16_to_f64(w[h] & 0xFFFFu);
           const double b = bf16_to_f64(w[h] >> 16);
-          acc = __dadd_rn(acc, __dmul_rn(a, a));  // x^2 of a bf16 is exact in fp64
-          acc = __dadd_rn(acc, __dmul_rn(b, b));
+          sq[2 * h] = __dmul_rn(a, a);
+          sq[2 * h + 1] = __dmul_rn(b, b);
         }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc = __dadd_rn(acc, sq[e]);  // n ascending
       }
     }
     __syncthreads();  // buffer (chunk & 1) is refilled by the next iteration's stage()

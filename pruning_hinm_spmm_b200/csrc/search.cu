@@ -19,6 +19,8 @@
 //                         with R(m+1) < R(m), else the last candidate
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "hinm_internal.h"
 #include "ptx.cuh"
 
@@ -125,21 +127,30 @@ __global__ void vector_score_kernel(const float* __restrict__ I, int K, int T,
   if (c < K) {
     const float* p = I + (size_t)t * T * K + c;
     double acc = 0.0;
-    constexpr int kBatch = 16;  // loads in flight per thread (T is a multiple of 16)
-    for (int i0 = 0; i0 < T; i0 += kBatch) {
-      float v[kBatch];
+    uint32_t mb = 0;  // largest bit pattern = largest value (non-negative floats)
+    constexpr int kBatch = 16;  // T is a multiple of 16
+    float v[kBatch], nx[kBatch];
 #pragma unroll
-      for (int k = 0; k < kBatch; ++k) v[k] = __ldg(p + (size_t)(i0 + k) * K);
+    for (int k = 0; k < kBatch; ++k) v[k] = __ldg(p + (size_t)k * K);
+    for (int i0 = 0; i0 < T; i0 += kBatch) {
+      // the next batch's loads go out before this batch's dependent chain
+      if (i0 + kBatch < T) {
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) nx[k] = __ldg(p + (size_t)(i0 + kBatch + k) * K);
+      }
 #pragma unroll
       for (int k = 0; k < kBatch; ++k) {  // rows ascending
         acc = __dadd_rn(acc, (double)v[k]);
-        uint32_t m;
-        int e;
-        split_f32(v[k], m, e);
-        if (m) pm = max(pm, e);
+        mb = max(mb, __float_as_uint(v[k]));
       }
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) v[k] = nx[k];
     }
     Vc[(size_t)t * K + c] = acc;
+    if (mb) {
+      uint32_t m;
+      split_f32(__uint_as_float(mb), m, pm);
+    }
   }
   for (int o = 16; o > 0; o >>= 1) pm = max(pm, __shfl_xor_sync(0xffffffffu, pm, o));
   if ((threadIdx.x & 31) == 0) atomicMax(tile_pmax + t, pm);
@@ -168,10 +179,14 @@ __global__ void column_sum_kernel(const float* __restrict__ I, int K, int T,
   U128 acc{0ull, 0ull};
   unsigned char tiny = 0;
   constexpr int kBatch = 16;
-  for (int i0 = 0; i0 < T; i0 += kBatch) {
-    float v[kBatch];
+  float v[kBatch], nx[kBatch];
 #pragma unroll
-    for (int k = 0; k < kBatch; ++k) v[k] = __ldg(p + (size_t)(i0 + k) * K);
+  for (int k = 0; k < kBatch; ++k) v[k] = __ldg(p + (size_t)k * K);
+  for (int i0 = 0; i0 < T; i0 += kBatch) {
+    if (i0 + kBatch < T) {  // next batch in flight during this one
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) nx[k] = __ldg(p + (size_t)(i0 + kBatch + k) * K);
+    }
 #pragma unroll
     for (int k = 0; k < kBatch; ++k) {
       if (v[k] >= thr1) {
@@ -187,6 +202,8 @@ __global__ void column_sum_kernel(const float* __restrict__ I, int K, int T,
         else tiny = 1;
       }
     }
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) v[k] = nx[k];
   }
   // acc += acc1 * 2^(e1 - lsb) + acc2 * 2^(e2 - lsb)  (integers < 2^53, shifts <= 61)
   const unsigned long long a1 = __double2ull_rz(__dmul_rn(acc1, pow2(149 - e1)));
@@ -298,16 +315,24 @@ size_t rank_scratch_bytes(int M, int K, int T) {
   return (c.off + 255) & ~size_t(255);
 }
 
-cudaError_t launch_vector_rank(const float* I, const int32_t* perm, int M, int K, int T,
-                               double* V, int32_t* rank, int* tile_pmax, void* scratch,
-                               cudaStream_t s) {
+namespace {
+
+// V and the tile maxima (one launch after clearing the maxima).
+cudaError_t launch_vector_scores(const float* I, int M, int K, int T, double* V, int* tile_pmax,
+                                 cudaStream_t s) {
   const int nt = M / T;
   cudaError_t e = cudaMemsetAsync(tile_pmax, 0, (size_t)nt * sizeof(int), s);
   if (e != cudaSuccess) return e;
   dim3 g1((K + 255) / 256, nt);
   vector_score_kernel<<<g1, 256, 0, s>>>(I, K, T, V, tile_pmax);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+// The ranking from V: chunk sort, then merge.
+cudaError_t launch_rank_sort(const double* V, const int32_t* perm, int M, int K, int T,
+                             int32_t* rank, void* scratch, cudaStream_t s) {
+  const int nt = M / T;
+  cudaError_t e;
   const int nchunk = (K + kRankChunk - 1) / kRankChunk;
   const int Kp = nchunk * kRankChunk;
   Carve c{static_cast<char*>(scratch), 0};
@@ -318,6 +343,44 @@ cudaError_t launch_vector_rank(const float* I, const int32_t* perm, int M, int K
   if (e != cudaSuccess) return e;
   merge_rank_kernel<<<dim3(nchunk, nt), kRankChunk, 0, s>>>(skey, sidx, K, Kp, rank);
   return cudaGetLastError();
+}
+
+// A second stream per device for work that can run beside the caller's stream (forked and
+// joined with events, so it also works under stream capture).  Created on the first call.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kMaxSideDevices = 64;
+std::mutex g_side_mu;  // also orders the fork / join records of concurrent host threads
+SideStream g_side[kMaxSideDevices];
+
+cudaError_t side_stream(SideStream** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxSideDevices) return cudaErrorInvalidDevice;
+  SideStream& ss = g_side[dev];
+  if (!ss.stream) {
+    e = cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking);
+    if (e != cudaSuccess) return e;
+    e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming);
+    if (e != cudaSuccess) return e;
+    e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming);
+    if (e != cudaSuccess) return e;
+  }
+  *out = &ss;
+  return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_vector_rank(const float* I, const int32_t* perm, int M, int K, int T,
+                               double* V, int32_t* rank, int* tile_pmax, void* scratch,
+                               cudaStream_t s) {
+  cudaError_t e = launch_vector_scores(I, M, K, T, V, tile_pmax, s);
+  if (e != cudaSuccess) return e;
+  return launch_rank_sort(V, perm, M, K, T, rank, scratch, s);
 }
 
 // Adds v * 2^sh (v < 2^64) into the little-endian multi-limb integer z[0..5].
@@ -795,12 +858,30 @@ cudaError_t launch_boundary_search(const float* I, const int32_t* perm, int M, i
   unsigned char* coltiny = c.take<unsigned char>((size_t)nt * K);
   char* rank_scratch = c.take<char>(rank_scratch_bytes(M, K, T));
   int32_t* rank = rank_out ? rank_out : rank_ws;
-  cudaError_t e = launch_vector_rank(I, perm, M, K, T, V, rank, pmax, rank_scratch, s);
+  cudaError_t e = launch_vector_scores(I, M, K, T, V, pmax, s);
   if (e != cudaSuccess) return e;
-  dim3 gc((K + 255) / 256, nt);
-  column_sum_kernel<<<gc, 256, 0, s>>>(I, K, T, pmax, colsum, coltiny);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  {
+    // the exact column sums (which need the tile maxima) run on the side stream while the
+    // ranking (which needs V) runs on the caller's stream; joined before the candidates
+    std::lock_guard<std::mutex> lk(g_side_mu);
+    SideStream* ss = nullptr;
+    e = side_stream(&ss);
+    if (e != cudaSuccess) return e;
+    e = cudaEventRecord(ss->fork, s);
+    if (e != cudaSuccess) return e;
+    e = cudaStreamWaitEvent(ss->stream, ss->fork, 0);
+    if (e != cudaSuccess) return e;
+    dim3 gc((K + 255) / 256, nt);
+    column_sum_kernel<<<gc, 256, 0, ss->stream>>>(I, K, T, pmax, colsum, coltiny);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    e = cudaEventRecord(ss->join, ss->stream);
+    if (e != cudaSuccess) return e;
+    e = launch_rank_sort(V, perm, M, K, T, rank, rank_scratch, s);
+    if (e != cudaSuccess) return e;
+    e = cudaStreamWaitEvent(s, ss->join, 0);
+    if (e != cudaSuccess) return e;
+  }
   CandidateList cl;
   for (int i = 0; i < kMaxCandidates; ++i) cl.c[i] = i < ncand ? cands[i] : Candidate{0, 0, 0};
   const BandCfg bc = band_config(K);
