@@ -177,6 +177,38 @@ __device__ __forceinline__ bool mask_bit(const uint32_t* bm, int words, int i, i
   return (__ldg(bm + (size_t)i * words + (c >> 5)) >> (c & 31)) & 1u;
 }
 
+// The stored pair of one 2:4 group from its 4 weights and kept bits: positions a < b and
+// their values.  The common case has exactly two kept positions.  A malformed group is
+// reported (HINM_ERR_BAD_MASK); its kept positions, lowest first, are completed from the
+// unkept ones with value 0, so the pair stays a legal (a < b) pattern.
+__device__ __forceinline__ void select_pair(const uint32_t (&w)[4], uint32_t kept, uint32_t& a,
+                                            uint32_t& bb, uint32_t& va, uint32_t& vb,
+                                            int* status) {
+  if (__popc(kept) == 2) {
+    a = (uint32_t)(__ffs(kept) - 1);
+    bb = (uint32_t)(31 - __clz(kept));
+    va = a == 0 ? w[0] : (a == 1 ? w[1] : w[2]);   // a <= 2
+    vb = bb == 1 ? w[1] : (bb == 2 ? w[2] : w[3]);  // b >= 1
+    return;
+  }
+  ptx::record_status(status, HINM_ERR_BAD_MASK);
+  int pos[2], np = 0;
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    if (((kept >> k) & 1u) && np < 2) pos[np++] = k;
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    if (!((kept >> k) & 1u) && np < 2) pos[np++] = -1 - k;  // filler, value 0
+  const int pa = pos[0] < 0 ? -1 - pos[0] : pos[0];
+  const int pb = pos[1] < 0 ? -1 - pos[1] : pos[1];
+  const bool ua = pos[0] >= 0, ub = pos[1] >= 0;
+  if (pa < pb) {  // order the pair by position
+    a = pa; bb = pb; va = ua ? w[pa] : 0u; vb = ub ? w[pb] : 0u;
+  } else {
+    a = pb; bb = pa; va = ub ? w[pb] : 0u; vb = ua ? w[pa] : 0u;
+  }
+}
+
 __global__ void __launch_bounds__(256) pack_kernel(const uint16_t* __restrict__ W,
                                                    const uint32_t* __restrict__ bitmask,
                                                    const int32_t* __restrict__ perm,
@@ -266,61 +298,55 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint16_t* __restrict__ 
   }
 
   uint8_t* out = reinterpret_cast<uint8_t*>(L.vals_sparse + (size_t)(s0 + sb) * 8192);
-#pragma unroll 4
-  for (int item = threadIdx.x; item < 128 * 32; item += blockDim.x) {
-    const int r = item >> 5, g = item & 31;
-    uint32_t a = 0, bb = 1, va = 0, vb = 0;
-    if (r < T && chan[4 * g] >= 0) {
-      const int i = row0 + r;
-      const uint16_t* Wi = W + (size_t)i * K;
-      const uint32_t* bmi = bitmask + (size_t)i * words;
-      uint32_t w[4], kept = 0;
-      if (run4) {
+  if (run4) {
+    // contiguous run: per thread, the loads of kU items go out before any is processed
+    constexpr int kU = 4;
+    for (int base = threadIdx.x; base < 128 * 32; base += 256 * kU) {
+      uint2 wv[kU];
+      uint32_t mw[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int item = base + 256 * u;
+        const int r = min(item >> 5, T - 1), g = item & 31;  // rows >= T: any valid row, unused
         const int cb = c0 + 4 * g;
-        const uint2 wv = __ldg(reinterpret_cast<const uint2*>(Wi + cb));
-        w[0] = wv.x & 0xFFFFu;
-        w[1] = wv.x >> 16;
-        w[2] = wv.y & 0xFFFFu;
-        w[3] = wv.y >> 16;
-        kept = (__ldg(bmi + (cb >> 5)) >> (cb & 31)) & 0xFu;
-      } else {
+        wv[u] = __ldg(reinterpret_cast<const uint2*>(W + (size_t)(row0 + r) * K + cb));
+        mw[u] = __ldg(bitmask + (size_t)(row0 + r) * words + (cb >> 5));
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int item = base + 256 * u;
+        const int r = item >> 5, g = item & 31;
+        uint32_t a = 0, bb = 1, va = 0, vb = 0;
+        if (r < T) {
+          const uint32_t w[4] = {wv[u].x & 0xFFFFu, wv[u].x >> 16, wv[u].y & 0xFFFFu,
+                                 wv[u].y >> 16};
+          select_pair(w, (mw[u] >> ((c0 + 4 * g) & 31)) & 0xFu, a, bb, va, vb, status);
+        }
+        *reinterpret_cast<uint32_t*>(out + swz(r, 2 * g)) = va | (vb << 16);
+        nib[r][g] = (uint8_t)(a | (bb << 2));
+      }
+    }
+  } else {
+#pragma unroll 4
+    for (int item = threadIdx.x; item < 128 * 32; item += blockDim.x) {
+      const int r = item >> 5, g = item & 31;
+      uint32_t a = 0, bb = 1, va = 0, vb = 0;
+      if (r < T && chan[4 * g] >= 0) {
+        const int i = row0 + r;
+        const uint16_t* Wi = W + (size_t)i * K;
+        const uint32_t* bmi = bitmask + (size_t)i * words;
+        uint32_t w[4], kept = 0;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const int c = chan[4 * g + k];
           w[k] = __ldg(Wi + c);
           kept |= ((__ldg(bmi + (c >> 5)) >> (c & 31)) & 1u) << k;
         }
+        select_pair(w, kept, a, bb, va, vb, status);
       }
-      if (__popc(kept) == 2) {
-        // the common case: the two kept positions, lowest first
-        a = (uint32_t)(__ffs(kept) - 1);
-        bb = (uint32_t)(31 - __clz(kept));
-        va = a == 0 ? w[0] : (a == 1 ? w[1] : w[2]);   // a <= 2
-        vb = bb == 1 ? w[1] : (bb == 2 ? w[2] : w[3]);  // b >= 1
-      } else {
-        ptx::record_status(status, HINM_ERR_BAD_MASK);
-        // the two kept positions, lowest first; a missing one is taken from the unkept
-        // positions with value 0 so that the pair stays a legal (a < b) pattern
-        int pos[2], np = 0;
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          if (((kept >> k) & 1u) && np < 2) pos[np++] = k;
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          if (!((kept >> k) & 1u) && np < 2) pos[np++] = -1 - k;  // filler, value 0
-        const int pa = pos[0] < 0 ? -1 - pos[0] : pos[0];
-        const int pb = pos[1] < 0 ? -1 - pos[1] : pos[1];
-        const bool ua = pos[0] >= 0, ub = pos[1] >= 0;
-        // order the pair by position
-        if (pa < pb) {
-          a = pa; bb = pb; va = ua ? w[pa] : 0u; vb = ub ? w[pb] : 0u;
-        } else {
-          a = pb; bb = pa; va = ub ? w[pb] : 0u; vb = ua ? w[pa] : 0u;
-        }
-      }
+      *reinterpret_cast<uint32_t*>(out + swz(r, 2 * g)) = va | (vb << 16);
+      nib[r][g] = (uint8_t)(a | (bb << 2));
     }
-    *reinterpret_cast<uint32_t*>(out + swz(r, 2 * g)) = va | (vb << 16);
-    nib[r][g] = (uint8_t)(a | (bb << 2));
   }
   __syncthreads();
   uint32_t* meta = L.meta + (size_t)(s0 + sb) * kMetaWords;

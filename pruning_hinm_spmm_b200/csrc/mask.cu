@@ -182,21 +182,23 @@ __global__ void __launch_bounds__(kMaskThreads) bitmask_kernel(
       c[k] = ((unsigned)cc[k] < (unsigned)K) ? cc[k] : 0;  // never index outside I
       mask_load_rows<RB>(rows_s + (size_t)mask_chan_slot(c[k]) * RB, v[k]);
     }
-    uint32_t kb[4] = {0u, 0u, 0u, 0u};
+    // g_kl bit r: member l beats member k (k < l) in row r, i.e. v_l > v_k (equal values:
+    // the lower position k wins).  Member k is kept iff at most one member beats it: the
+    // negated majority of its three "beaten by" words, all rows at once.
+    uint32_t g01 = 0u, g02 = 0u, g03 = 0u, g12 = 0u, g13 = 0u, g23 = 0u;
 #pragma unroll
     for (int r = 0; r < RB; ++r) {
-      // beats[k]: members ranked above k (greater value, or equal value at a lower position)
-      int beats[4] = {0, 0, 0, 0};
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-#pragma unroll
-        for (int l = k + 1; l < 4; ++l) {
-          if (v[l][r] > v[k][r]) ++beats[k];
-          else ++beats[l];  // v[k] >= v[l]: k (lower position) ranks above l
-        }
-#pragma unroll
-      for (int k = 0; k < 4; ++k) kb[k] |= (beats[k] < 2 ? 1u : 0u) << r;
+      g01 |= (uint32_t)(v[1][r] > v[0][r]) << r;
+      g02 |= (uint32_t)(v[2][r] > v[0][r]) << r;
+      g03 |= (uint32_t)(v[3][r] > v[0][r]) << r;
+      g12 |= (uint32_t)(v[2][r] > v[1][r]) << r;
+      g13 |= (uint32_t)(v[3][r] > v[1][r]) << r;
+      g23 |= (uint32_t)(v[3][r] > v[2][r]) << r;
     }
+    auto maj = [](uint32_t a, uint32_t b, uint32_t c) { return (a & b) | (a & c) | (b & c); };
+    constexpr uint32_t kRows = (1u << RB) - 1u;
+    const uint32_t kb[4] = {~maj(g01, g02, g03) & kRows, ~maj(~g01, g12, g13) & kRows,
+                            ~maj(~g02, ~g12, g23) & kRows, ~maj(~g03, ~g13, ~g23) & kRows};
 #pragma unroll
     for (int k = 0; k < 4; ++k) keep[c[k]] = (uint8_t)kb[k];
   }
