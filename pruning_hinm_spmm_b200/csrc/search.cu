@@ -773,7 +773,7 @@ __global__ void __launch_bounds__(kThreads) band_sum_kernel(
   }
 }
 
-// Per tile, one thread per candidate: R(m) = exact total rounded once to fp64; then the
+// Per tile, one warp per candidate: R(m) = exact total rounded once to fp64; then the
 // first m with R(m+1) < R(m) (else the last candidate) gives the counts and v_s.
 __global__ void finalize_kernel(const U128* __restrict__ rdense, const U128* __restrict__ part,
                                 int nchunks, const unsigned long long* __restrict__ bucket,
@@ -782,16 +782,27 @@ __global__ void finalize_kernel(const U128* __restrict__ rdense, const U128* __r
                                 double t_s, double alpha, double* __restrict__ R,
                                 int32_t* __restrict__ counts, double* __restrict__ vs) {
   __shared__ double Rs[kMaxCandidates];
-  const int t = blockIdx.x, m = threadIdx.x;
-  if (m < ncand) {
+  const int t = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  for (int m = warp; m < ncand; m += nwarps) {  // one warp per candidate
     const size_t tm = (size_t)t * ncand + m;
-    U128 tot = rdense[tm];
-    for (int c = 0; c < nchunks; ++c) add128(tot, part[tm * nchunks + c]);
-    const int lsb = tile_lsb(tile_pmax[t]);
-    const double r = bucket_used[tm] ? exact_to_double(tot, lsb, bucket + tm * 256)
-                                     : u128_to_double(tot, lsb);
-    Rs[m] = r;
-    R[tm] = r;
+    U128 tot{0ull, 0ull};
+    for (int c = lane; c < nchunks; c += 32) add128(tot, part[tm * nchunks + c]);
+    for (int o = 16; o > 0; o >>= 1) {
+      U128 other;
+      other.lo = __shfl_xor_sync(0xffffffffu, tot.lo, o);
+      other.hi = __shfl_xor_sync(0xffffffffu, tot.hi, o);
+      add128(tot, other);
+    }
+    if (lane == 0) {
+      add128(tot, rdense[tm]);
+      const int lsb = tile_lsb(tile_pmax[t]);
+      const double r = bucket_used[tm] ? exact_to_double(tot, lsb, bucket + tm * 256)
+                                       : u128_to_double(tot, lsb);
+      Rs[m] = r;
+      R[tm] = r;
+    }
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -932,7 +943,7 @@ cudaError_t launch_boundary_search(const float* I, const int32_t* perm, int M, i
                                                   bucket_used);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  finalize_kernel<<<nt, 64, 0, s>>>(rdense, part, nchunks, bucket, bucket_used, pmax, ncand, cl,
+  finalize_kernel<<<nt, 1024, 0, s>>>(rdense, part, nchunks, bucket, bucket_used, pmax, ncand, cl,
                                     t_s, alpha, R, counts_out, vs_out);
   return cudaGetLastError();
 }

@@ -45,12 +45,15 @@ struct SpmmCfg {
   static constexpr int kBBytes = 2 * kBHalfBytes;
   static constexpr int kBAtomStride = 64 * kAtomBytes;
   static constexpr int kEBytes = 2048;
+  // a stage is a multiple of 1024 bytes (the 128-byte swizzle atoms stay aligned); each
+  // stage's vector indices (gathered blocks) live in a separate region after the stages
   static constexpr int kStageBytes = kABytes + kBBytes + kEBytes;
+  static constexpr int kIdxBytes = 512;
   // split-K: CTAs of a cluster per unit; the leader's reduction buffer holds the others'
   // 128 x BN fp32 partial accumulators
   static constexpr int kMaxSplit = !SPLIT ? 1 : (BN <= 16 ? 8 : 4);
   static constexpr int kRedBytes = (kMaxSplit - 1) * 128 * BN * 4;
-  static constexpr int kStagesRaw = (200 * 1024 - kRedBytes) / kStageBytes;
+  static constexpr int kStagesRaw = (210 * 1024 - kRedBytes) / (kStageBytes + kIdxBytes);
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
   // layout type of the B descriptor: 2 = 128-byte swizzle, 4 = 64-byte, 6 = 32-byte
   static constexpr uint32_t kBLayout = kAtomBytes == 128 ? 2u : (kAtomBytes == 64 ? 4u : 6u);
@@ -60,11 +63,12 @@ struct SpmmCfg {
   static constexpr int kTmemNeed = kAccBufs * kAccCols + 4 * kStages;
   static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                    : kTmemNeed <= 256 ? 256 : 512;
-  static constexpr size_t kSmemBytes =
-      (size_t)kStages * kStageBytes + 1024 /*align*/ + 512 /*barriers*/ + kRedBytes;
+  static constexpr size_t kSmemBytes = (size_t)kStages * (kStageBytes + kIdxBytes) +
+                                       1024 /*align*/ + 512 /*barriers*/ + kRedBytes;
   static constexpr int kProducers = 128;
   static constexpr int kMmaWarp = 4;
-  static constexpr int kThreads = 288;  // 9 warps: 4 producers, 1 MMA, 4 epilogue
+  static constexpr int kBulkWarp = 9;
+  static constexpr int kThreads = 320;  // 10 warps: 4 gather, 1 MMA, 4 epilogue, 1 bulk copies
   static_assert(BN == 16 || BN == 32 || (BN % 64 == 0 && BN <= 256), "BN");
   static_assert(kStages >= 2, "stages");
   static_assert(kTmemNeed <= 512, "tmem");
@@ -107,10 +111,10 @@ struct Gather {
   static constexpr int kPer = ROWS * C::kChunksPerRow / C::kProducers;
   static_assert(kPer * C::kProducers == ROWS * C::kChunksPerRow, "chunks per producer");
   int xr[kPer];
-  __device__ __forceinline__ void load_index(const int* __restrict__ idx, int ptid) {
+  // the block's indices, brought into the stage by the bulk-copy warp
+  __device__ __forceinline__ void load_index(const int* idx_s, int ptid) {
 #pragma unroll
-    for (int i = 0; i < kPer; ++i)
-      xr[i] = __ldg(idx + (ptid + C::kProducers * i) / C::kChunksPerRow);
+    for (int i = 0; i < kPer; ++i) xr[i] = idx_s[(ptid + C::kProducers * i) / C::kChunksPerRow];
   }
   __device__ __forceinline__ void copy(uint32_t B_s, const uint16_t* __restrict__ X, int N,
                                        int n0, int ptid) const {
@@ -131,17 +135,20 @@ struct Gather {
 };
 
 template <int BN, bool SPLIT>
-__global__ void __launch_bounds__(288, 1)
+__global__ void __launch_bounds__(320, 1)
     spmm_kernel(const __grid_constant__ CUtensorMap tmX, const SpmmArgs a) {
   using C = SpmmCfg<BN, SPLIT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint8_t* idx_region = smem + C::kStages * C::kStageBytes;  // [S][kIdxBytes]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(idx_region + C::kStages * C::kIdxBytes);
   // [0,S) full, [S,2S) empty, 2S+{0,1} accumulator full, 2S+{2,3} accumulator empty,
-  // 2S+4 drain
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::kStages + 5);
+  // 2S+4 drain, [2S+5, 3S+5) index ready; then the TMEM address, the abort flag and one run
+  // flag per stage (at most 272 bytes of the 512 reserved)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * C::kStages + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* run_s = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto full_bar = [&](int s) { return ptx::smem_u32(bars + s); };
@@ -149,11 +156,13 @@ __global__ void __launch_bounds__(288, 1)
   auto accf_bar = [&](int b) { return ptx::smem_u32(bars + 2 * C::kStages + b); };
   auto acce_bar = [&](int b) { return ptx::smem_u32(bars + 2 * C::kStages + 2 + b); };
   const uint32_t drain_bar = ptx::smem_u32(bars + 2 * C::kStages + 4);
+  auto idx_bar = [&](int s) { return ptx::smem_u32(bars + 2 * C::kStages + 5 + s); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       ptx::mbar_init(full_bar(s), 1 + C::kProducers);  // expect_tx arrival + one per producer
       ptx::mbar_init(empty_bar(s), 1);
+      ptx::mbar_init(idx_bar(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(accf_bar(b), 1);
@@ -172,7 +181,7 @@ __global__ void __launch_bounds__(288, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t meta_col0 = C::kAccBufs * C::kAccCols;
-  float* red = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes + 512);
+  float* red = reinterpret_cast<float*>(idx_region + C::kStages * C::kIdxBytes + 512);
   // Work: persistent CTAs stride over the units; split-K CTAs take one unit each and the
   // K-block range [kb0, kb1) of their cluster rank.
   const int u_first = SPLIT ? (int)blockIdx.x / a.split : (int)blockIdx.x;
@@ -188,9 +197,14 @@ __global__ void __launch_bounds__(288, 1)
   int split_tile = 0, split_n0 = 0, split_b = 0;
 
   if (warp < 4) {
-    // ------------------------------------------------------------ producers
+    // ------------------------------------------------------------ gather producers
+    // Per K-block: wait until the bulk-copy warp has the stage (its index-ready barrier),
+    // then either gather the X rows the block's index selects (16-byte cp.async, arrival
+    // when they land) or, for a contiguous run it moves by TMA, just arrive.  Every thread
+    // arrives on the stage's full barrier once per block, after its last read of the
+    // stage's run flag and indices, so the stage cannot be recycled under it.
     const int ptid = threadIdx.x;
-    uint32_t it = 0;  // K-blocks issued by this CTA (stage ring position)
+    uint32_t it = 0;  // K-blocks handled by this CTA (stage ring position)
     bool stop = false;
     for (int u = u_first; u < a.num_units && !stop; u += u_step) {
       const int tile = u / a.nblk_n, n0 = (u - tile * a.nblk_n) * BN;
@@ -200,26 +214,71 @@ __global__ void __launch_bounds__(288, 1)
       k_range(nblk, kb0, kb1);
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
         const bool sparse = kb >= nd;
-        const size_t blk = sparse ? (size_t)(info.w + kb - nd) : (size_t)(info.z + kb);
-        // index loads are issued before the wait so their latency hides behind it
-        const int run = __ldg(sparse ? a.run_sparse + blk : a.run_dense + blk);
-        Gather<C, kSparseBK> gs;
-        Gather<C, kDenseBK> gd;
-        if (run < 0) {
-          if (sparse) gs.load_index(a.idx_sparse + blk * kSparseBK, ptid);
-          else gd.load_index(a.idx_dense + blk * kDenseBK, ptid);
-        }
         const int s = it % C::kStages;
         const uint32_t ph = (it / C::kStages) & 1;
-        if (!ptx::mbar_wait(empty_bar(s), ph ^ 1, a.status, abort_flag)) {
+        if (!ptx::mbar_wait(idx_bar(s), ph, a.status, abort_flag)) {
           stop = true;
           break;
         }
+        const int run = run_s[s];
         const uint32_t A_s = ptx::smem_u32(smem + s * C::kStageBytes);
         const uint32_t B_s = A_s + C::kABytes;
-        const uint32_t E_s = B_s + C::kBBytes;
-        const int rows = sparse ? kSparseBK : kDenseBK;
-        if (ptid == 0) {
+        const int* idx_s = reinterpret_cast<const int*>(idx_region + s * C::kIdxBytes);
+        if (run < 0) {
+          if (sparse) {
+            Gather<C, kSparseBK> gs;
+            gs.load_index(idx_s, ptid);
+            gs.copy(B_s, a.X, a.N, n0, ptid);
+          } else {
+            Gather<C, kDenseBK> gd;
+            gd.load_index(idx_s, ptid);
+            gd.copy(B_s, a.X, a.N, n0, ptid);
+          }
+          cp_async_arrive_noinc(full_bar(s));
+        } else {
+          ptx::mbar_arrive(full_bar(s));
+        }
+      }
+    }
+    cp_async_wait_all();
+  } else if (warp == C::kBulkWarp) {
+    // ------------------------------------------------------------ bulk copies
+    // One thread runs ahead of the gather warps by up to a full ring: per K-block, once the
+    // stage is free, it publishes the block's run flag and index list (index-ready barrier)
+    // and bulk-copies the pre-swizzled A block, its metadata and, for a contiguous run, the
+    // X rows by TMA (full barrier).
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool stop = false;
+      for (int u = u_first; u < a.num_units && !stop; u += u_step) {
+        const int tile = u / a.nblk_n, n0 = (u - tile * a.nblk_n) * BN;
+        const int4 info = __ldg(reinterpret_cast<const int4*>(a.tile_info) + tile);
+        const int nd = info.x, nblk = info.x + info.y;
+        int kb0, kb1;
+        k_range(nblk, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const bool sparse = kb >= nd;
+          const size_t blk = sparse ? (size_t)(info.w + kb - nd) : (size_t)(info.z + kb);
+          const int run = __ldg(sparse ? a.run_sparse + blk : a.run_dense + blk);
+          const int s = it % C::kStages;
+          const uint32_t ph = (it / C::kStages) & 1;
+          if (!ptx::mbar_wait(empty_bar(s), ph ^ 1, a.status, abort_flag)) {
+            stop = true;
+            break;
+          }
+          const uint32_t A_s = ptx::smem_u32(smem + s * C::kStageBytes);
+          const uint32_t B_s = A_s + C::kABytes;
+          const uint32_t E_s = B_s + C::kBBytes;
+          const uint32_t I_s = ptx::smem_u32(idx_region + s * C::kIdxBytes);
+          const int rows = sparse ? kSparseBK : kDenseBK;
+          run_s[s] = run;  // published by the arrive below (release)
+          if (run < 0) {
+            ptx::mbar_arrive_expect_tx(idx_bar(s), (uint32_t)rows * 4u);
+            ptx::bulk_g2s(I_s, sparse ? a.idx_sparse + blk * kSparseBK : a.idx_dense + blk * kDenseBK,
+                          (uint32_t)rows * 4u, idx_bar(s));
+          } else {
+            ptx::mbar_arrive(idx_bar(s));
+          }
           const uint32_t bytes = C::kABytes + (sparse ? C::kEBytes : 0) +
                                  (run >= 0 ? (uint32_t)rows * BN * 2u : 0u);
           ptx::mbar_arrive_expect_tx(full_bar(s), bytes);
@@ -241,22 +300,18 @@ __global__ void __launch_bounds__(288, 1)
                                    n0 + at * C::kAtom, run + h * 64, full_bar(s));
               }
             }
-            ptx::mbar_arrive_count(full_bar(s), C::kProducers);  // on behalf of all producers
           }
         }
-        if (run < 0) {
-          if (sparse) gs.copy(B_s, a.X, a.N, n0, ptid);
-          else gd.copy(B_s, a.X, a.N, n0, ptid);
-          cp_async_arrive_noinc(full_bar(s));
+      }
+      if (*abort_flag) {
+        // wait (bounded) for the bulk / tensor copies of the last stages
+        for (uint32_t k = (it > (uint32_t)C::kStages ? it - C::kStages : 0u); k < it; ++k) {
+          ptx::mbar_wait(idx_bar(k % C::kStages), (k / C::kStages) & 1, a.status, nullptr);
+          ptx::mbar_wait(full_bar(k % C::kStages), (k / C::kStages) & 1, a.status, nullptr);
         }
       }
     }
-    cp_async_wait_all();
-    if (*abort_flag && ptid == 0) {
-      // wait (bounded) for the bulk / tensor copies of the last stages
-      for (uint32_t k = (it > (uint32_t)C::kStages ? it - C::kStages : 0u); k < it; ++k)
-        ptx::mbar_wait(full_bar(k % C::kStages), (k / C::kStages) & 1, a.status, nullptr);
-    }
+    __syncwarp();
   } else if (warp == C::kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
