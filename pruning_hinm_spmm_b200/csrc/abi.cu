@@ -131,6 +131,30 @@ int* device_status_ptr() {
   return g_status_ptr[dev];
 }
 
+namespace {
+struct SmemAttr {
+  int dev;
+  const void* fn;
+};
+std::mutex g_attr_mu;
+SmemAttr g_attr_done[1024];
+int g_attr_count = 0;
+}  // namespace
+
+cudaError_t set_max_dynamic_smem(const void* fn, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  for (int i = 0; i < g_attr_count; ++i)
+    if (g_attr_done[i].dev == dev && g_attr_done[i].fn == fn) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  if (g_attr_count < (int)(sizeof(g_attr_done) / sizeof(g_attr_done[0])))
+    g_attr_done[g_attr_count++] = SmemAttr{dev, fn};
+  return cudaSuccess;
+}
+
 }  // namespace hinm
 
 // =====================================================================================

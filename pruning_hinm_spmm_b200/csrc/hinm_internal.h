@@ -34,6 +34,11 @@ int search_candidates_host(int K, double t_s, double alpha, Candidate* out, int 
 // Per-device address of the library's status word (resolved once per device).
 int* device_status_ptr();
 
+// Sets kernel `fn`'s maximum dynamic shared memory to `bytes` on the current device, once per
+// (device, kernel): the attribute belongs to the device, and a process may drive several.
+// Thread-safe; call it before the first launch on each device (and before stream capture).
+cudaError_t set_max_dynamic_smem(const void* fn, int bytes);
+
 // Workspace carving helper: 256-byte aligned sub-buffers.
 struct Carve {
   char* base;

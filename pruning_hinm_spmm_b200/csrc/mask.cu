@@ -3,7 +3,6 @@
 // rkmt.cn section 二: keep 2 of every 4 consecutive; geek-doc.cn section 五: the mask has
 // W's shape).
 //
-//   inverse_perm_kernel   pinv[perm[j]] = j (checks that perm is a permutation)
 //   classify_kernel       one CTA per tile: region of every working position and the
 //                         2:4 members' input channels in ascending working position
 //                         (member[t][q])
@@ -16,20 +15,6 @@
 #include "ptx.cuh"
 
 namespace hinm {
-
-// pinv must be preset to -1.  A repeated or out-of-range channel is reported as
-// HINM_ERR_INVALID_ARG (the permutation is then not a permutation of 0..K-1).
-__global__ void inverse_perm_kernel(const int32_t* __restrict__ perm, int K,
-                                    int32_t* __restrict__ pinv, int* status) {
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= K) return;
-  const int c = perm ? __ldg(perm + j) : j;
-  if (c < 0 || c >= K) {
-    ptx::record_status(status, HINM_ERR_INVALID_ARG);
-    return;
-  }
-  if (atomicExch(pinv + c, j) != -1) ptx::record_status(status, HINM_ERR_INVALID_ARG);
-}
 
 // Block-wide exclusive scan of one int per thread (blockDim.x <= 1024).
 __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* total) {
@@ -66,7 +51,23 @@ __global__ void __launch_bounds__(1024) classify_kernel(const int32_t* __restric
                                                         int* status) {
   __shared__ int warp_tot[32];
   __shared__ int total;
+  __shared__ uint32_t seen[kMaxK / 32];  // tile 0: which channels perm has named
   const int t = blockIdx.x;
+  if (t == 0 && perm) {
+    // the permutation must name every channel 0..K-1 once: a repeated or out-of-range
+    // entry is reported as HINM_ERR_INVALID_ARG (perm_at keeps every access in range)
+    for (int w = threadIdx.x; w < kMaxK / 32; w += blockDim.x) seen[w] = 0u;
+    __syncthreads();
+    for (int j = threadIdx.x; j < K; j += blockDim.x) {
+      const int c = __ldg(perm + j);
+      if (c < 0 || c >= K) {
+        ptx::record_status(status, HINM_ERR_INVALID_ARG);
+      } else {
+        const uint32_t bit = 1u << (c & 31);
+        if (atomicOr(seen + (c >> 5), bit) & bit) ptx::record_status(status, HINM_ERR_INVALID_ARG);
+      }
+    }
+  }
   int n0 = counts[3 * t], n24 = counts[3 * t + 1], n4 = counts[3 * t + 2];
   if (n0 < 0 || n24 < 0 || n4 < 0 || n0 + n24 + n4 != K || (n24 & 3)) {
     if (threadIdx.x == 0) ptx::record_status(status, HINM_ERR_INVALID_ARG);
@@ -240,7 +241,6 @@ size_t mask_workspace_bytes(int M, int K, int T) {
   Carve c{nullptr, 0};
   c.take<double>((size_t)nt * K);   // V (only when no rank is passed)
   c.take<int32_t>((size_t)nt * K);  // rank (only when no rank is passed)
-  c.take<int32_t>((size_t)K);       // inverse permutation
   c.take<int32_t>((size_t)nt * K);  // member
   c.take<int>((size_t)nt);          // tile max exponent (by-product of the ranking)
   c.take<char>(rank_scratch_bytes(M, K, T));
@@ -254,7 +254,6 @@ cudaError_t launch_mask(const float* I, const int32_t* perm, const int32_t* coun
   Carve cv{static_cast<char*>(ws), 0};
   double* V = cv.take<double>((size_t)nt * K);
   int32_t* rank_ws = cv.take<int32_t>((size_t)nt * K);
-  int32_t* pinv = cv.take<int32_t>((size_t)K);
   int32_t* member = cv.take<int32_t>((size_t)nt * K);
   int* pmax = cv.take<int>((size_t)nt);
   char* rank_scratch = cv.take<char>(rank_scratch_bytes(M, K, T));
@@ -264,24 +263,15 @@ cudaError_t launch_mask(const float* I, const int32_t* perm, const int32_t* coun
     if (e != cudaSuccess) return e;
     rank = rank_ws;
   }
-  e = cudaMemsetAsync(pinv, 0xFF, (size_t)K * sizeof(int32_t), s);
-  if (e != cudaSuccess) return e;
-  inverse_perm_kernel<<<(K + 255) / 256, 256, 0, s>>>(perm, K, pinv, status);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
   classify_kernel<<<nt, 1024, 0, s>>>(rank, perm, counts, K, region, member, status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int RB = mask_rows(K);
   const size_t smem = (size_t)RB * (((size_t)K + 7) & ~size_t(7)) * sizeof(float) + (size_t)K;
-  static bool attr_set = false;
-  if (!attr_set) {
-    for (auto fn : {bitmask_kernel<1>, bitmask_kernel<2>, bitmask_kernel<4>, bitmask_kernel<8>}) {
-      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               64 * 1024 + kMaxK);
-      if (e != cudaSuccess) return e;
-    }
-    attr_set = true;
+  for (const void* fn : {(const void*)bitmask_kernel<1>, (const void*)bitmask_kernel<2>,
+                         (const void*)bitmask_kernel<4>, (const void*)bitmask_kernel<8>}) {
+    e = set_max_dynamic_smem(fn, 64 * 1024 + kMaxK);
+    if (e != cudaSuccess) return e;
   }
   const dim3 g(T / RB, nt);
   if (RB == 8)

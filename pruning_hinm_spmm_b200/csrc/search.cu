@@ -923,13 +923,10 @@ cudaError_t launch_boundary_search(const float* I, const int32_t* perm, int M, i
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t smem = (size_t)RB * (((size_t)K + 7) & ~size_t(7)) * sizeof(float);
-  static bool attr_set = false;
-  if (!attr_set) {
-    for (auto fn : {band_sum_kernel<1, 512>, band_sum_kernel<2, 512>, band_sum_kernel<4, 512>}) {
-      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
-      if (e != cudaSuccess) return e;
-    }
-    attr_set = true;
+  for (const void* fn : {(const void*)band_sum_kernel<1, 512>, (const void*)band_sum_kernel<2, 512>,
+                         (const void*)band_sum_kernel<4, 512>}) {
+    e = set_max_dynamic_smem(fn, 96 * 1024);
+    if (e != cudaSuccess) return e;
   }
   const dim3 gb(nchunks, nt);
   if (RB == 4)

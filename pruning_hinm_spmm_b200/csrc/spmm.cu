@@ -585,12 +585,8 @@ template <int BN, bool SPLIT>
 cudaError_t run(const hinm_layout& L, const uint16_t* X, int N, float* Y, int split, int* status,
                 cudaStream_t s) {
   using C = SpmmCfg<BN, SPLIT>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(spmm_kernel<BN, SPLIT>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmemBytes);
-  });
+  cudaError_t attr_err =
+      set_max_dynamic_smem((const void*)spmm_kernel<BN, SPLIT>, (int)C::kSmemBytes);
   if (attr_err != cudaSuccess) return attr_err;
   CUtensorMap map;
   bool x3d = false;

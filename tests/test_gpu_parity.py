@@ -307,3 +307,25 @@ def test_llama_sweep_searched_sampled(H, linear, t_s, N):
     layout_equal(hp.layout, L_ref, tiles=tiles)
     y_ref, bound = O.spmm_reference(w.W_bits, bm_ref, w.X_bits, rows=rows)
     check_y(Y.cpu().numpy(), y_ref, bound, rows=rows)
+
+
+def test_invalid_permutation_reported(H):
+    """A permutation with a repeated or an out-of-range channel is reported on the device
+    status word (every access stays clamped inside the matrices)."""
+    w = hi.custom(128, 256, 16, 64, seed=5, t_s=0.5, v_s=0.25)
+    W, X = dev_bf16(w.W_bits), dev_bf16(w.X_bits)
+    I = H.hinm_importance(W, X)
+    c = dev_i32(np.array([H.hinm_counts_from_vs(w.K, w.t_s, w.v_s)] * (w.M // w.T), dtype=np.int32))
+    good = np.arange(w.K, dtype=np.int32)
+    H.hinm_mask(I, dev_i32(good), c, w.T)
+    torch.cuda.synchronize()
+    assert H.hinm_device_status() == 0
+    dup = good.copy()
+    dup[7] = dup[3]
+    oob = good.copy()
+    oob[11] = w.K + 5
+    for bad in (dup, oob):
+        H.hinm_mask(I, dev_i32(bad), c, w.T)
+        torch.cuda.synchronize()
+        assert H.hinm_device_status() == H.HINM_ERR_INVALID_ARG
+        assert H.hinm_device_status() == 0  # cleared by the read
