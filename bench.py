@@ -226,6 +226,78 @@ def run_reference(args, w):
     return 0
 
 
+# ------------------------------------------------------------------ LLaMA-shaped sweep
+SWEEP_SHAPES = (("q", 4), ("gate", 2), ("down", 1))  # distinct shapes, linears per layer
+
+
+def run_sweep(args):
+    """The LLaMA-2-7B-shaped layer sweep on one GPU: the three distinct linear shapes of
+    layer 0 (q/k/v/o 4096x4096, gate/up 11008x4096, down 4096x11008), each at every
+    N in {16, 512, 4096} and t_s in {0.5, 0.625, 0.75} with the boundary from the search.
+    Each case times K graph-replayed steps (L2 flushed between them); a layer's time is
+    4 x q + 2 x gate + 1 x down.  `value` = the layers' dense-equivalent FLOPs over their
+    total time."""
+    import torch
+    import pruning_hinm_spmm_b200 as H
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(0)
+    sampler.start()
+    rows, tot_flops, tot_s = [], 0.0, 0.0
+    for t_s in (0.5, 0.625, 0.75):
+        for N in (16, 512, 4096):
+            layer_s, layer_flops, per = 0.0, 0.0, {}
+            for name, mult in SWEEP_SHAPES:
+                w = hi.llama_sweep_layer(0, name, N, t_s)
+                M, K, T = w.M, w.K, w.T
+                W = torch.from_numpy(w.W_bits.view(np.int16)).to(dev).view(torch.bfloat16)
+                X = torch.from_numpy(w.X_bits.view(np.int16)).to(dev).view(torch.bfloat16)
+                perm = torch.from_numpy(w.perm).to(dev)
+                hp = H.HotPath(M, K, N, T, w.t_s, w.alpha, device=dev)
+                for _ in range(args.warmup):
+                    hp.run(W, X, perm)
+                torch.cuda.synchronize()
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph):
+                    hp.run(W, X, perm)
+                torch.cuda.synchronize()
+                ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                      for _ in range(args.steps)]
+                for k in range(args.steps):
+                    flush.zero_()
+                    ev[k][0].record(stream)
+                    graph.replay()
+                    ev[k][1].record(stream)
+                torch.cuda.synchronize()
+                if H.hinm_device_status() != 0:
+                    raise RuntimeError(f"device status after {w.name}")
+                t = statistics.mean(e[0].elapsed_time(e[1]) * 1e-3 for e in ev)
+                del graph
+                per[name] = {"M": M, "K": K, "ms": t * 1e3,
+                             "v_s_searched": sorted(set(np.round(hp.vs.cpu().numpy(), 6).tolist()))}
+                layer_s += mult * t
+                layer_flops += mult * 2.0 * M * K * N
+            rows.append({"t_s": t_s, "N": N, "layer_ms": layer_s * 1e3,
+                         "layer_tflops_eff": layer_flops / layer_s / 1e12, "by_shape": per})
+            tot_flops += layer_flops
+            tot_s += layer_s
+    sampler.stop()
+    line = {"metric": METRIC, "value": tot_flops / tot_s / 1e12, "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": tot_s * 1e3 / len(rows), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "llama7b_layer0_sweep",
+                       "step": "importance+search+mask+compress+spmm per linear, searched v_s",
+                       "layer": "4 x (4096x4096) + 2 x (11008x4096) + 1 x (4096x11008)",
+                       "l2": "flushed between timed steps (256 MB write)",
+                       "step_exec": "CUDA graph replay"},
+            "sweep": rows, "clocks": sampler.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # ------------------------------------------------------------------ GPU arm
 def main():
     ap = argparse.ArgumentParser()
@@ -234,8 +306,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="hinm", choices=["hinm", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="pure24", choices=sorted(WORKLOADS),
-                    help="synthetic workload (default: the pure 2:4 4096x4096x2048 benchmark)")
+    ap.add_argument("--workload", default="pure24", choices=sorted(WORKLOADS) + ["sweep"],
+                    help="synthetic workload (default: the pure 2:4 4096x4096x2048 benchmark); "
+                         "'sweep' times the LLaMA-2-7B-shaped layer sweep")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -243,6 +316,10 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
+    if args.workload == "sweep":
+        if world > 1 or args.impl == "reference":
+            raise SystemExit("--workload sweep runs on one GPU with the CUDA arm only")
+        return run_sweep(args)
     w = WORKLOADS[args.workload](rank)
     if args.impl == "reference":
         return run_reference(args, w)

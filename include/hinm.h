@@ -214,6 +214,13 @@ hinm_status hinm_compress(const void* W, const uint32_t* bitmask, const int8_t* 
 hinm_status hinm_spmm(const hinm_layout* layout, const void* X, int N, float* Y_out,
                       void* stream);
 
+/* Diagnostic with no counterpart in the pages: launches one small kernel whose bounded
+ * wait cannot complete (it waits on an mbarrier nothing arrives at), so that after about
+ * limit_ns nanoseconds it records HINM_ERR_DEVICE_TIMEOUT and returns, exercising the
+ * timeout path of every pipelined kernel.  0 < limit_ns <= 2e9, else HINM_ERR_INVALID_ARG.
+ * Read the result with hinm_device_status(); the context stays usable. */
+hinm_status hinm_selftest_wait_timeout(unsigned long long limit_ns, void* stream);
+
 /* Reads the device status word into *status_host (0 = no fault; else an hinm_status)
  * and clears it.  Synchronises `stream`. */
 hinm_status hinm_device_status(void* stream, int32_t* status_host);

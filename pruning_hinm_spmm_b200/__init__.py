@@ -62,6 +62,7 @@ _SIGS = {
     "hinm_importance_workspace_size": (_i32, [_i32, _i32, _i32, _szp]),
     "hinm_importance": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _sz, _vp]),
     "hinm_importance_noalloc": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp]),
+    "hinm_selftest_wait_timeout": (_i32, [ctypes.c_ulonglong, _vp]),
     "hinm_counts_from_vs": (_i32, [_i32, _f64, _f64, ctypes.POINTER(ctypes.c_int32)]),
     "hinm_search_num_candidates": (_i32, [_i32, _f64, _f64, ctypes.POINTER(ctypes.c_int32)]),
     "hinm_search_workspace_size": (_i32, [_i32, _i32, _i32, _f64, _f64, _szp]),
@@ -138,6 +139,13 @@ def hinm_importance(W, X, I_out=None, workspace=None, stream=None):
     _check(_lib.hinm_importance(_ptr(W), _ptr(X), M, K, N, _ptr(I_out), _ptr(workspace),
                                 workspace.numel(), _stream(stream)), "hinm_importance")
     return I_out
+
+
+def hinm_selftest_wait_timeout(limit_ns: int, stream=None):
+    """Launches the bounded-wait self test (see hinm.h); read the outcome with
+    hinm_device_status()."""
+    _check(_lib.hinm_selftest_wait_timeout(int(limit_ns), _stream(stream)),
+           "hinm_selftest_wait_timeout")
 
 
 def hinm_importance_noalloc(W, X, I_out, stream=None):

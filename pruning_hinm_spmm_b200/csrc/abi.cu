@@ -441,6 +441,17 @@ hinm_status hinm_spmm(const hinm_layout* layout, const void* X, int N, float* Y_
   return ok();
 }
 
+hinm_status hinm_selftest_wait_timeout(unsigned long long limit_ns, void* stream) {
+  if (limit_ns == 0 || limit_ns > 2000000000ull)
+    return fail(HINM_ERR_INVALID_ARG, "limit_ns=%llu: need 0 < limit_ns <= 2e9", limit_ns);
+  int* status = hinm::device_status_ptr();
+  if (!status) return fail(HINM_ERR_CUDA, "no device status word");
+  cudaError_t e =
+      hinm::launch_wait_timeout_selftest(limit_ns, status, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "hinm_selftest_wait_timeout launch");
+  return ok();
+}
+
 hinm_status hinm_device_status(void* stream, int32_t* status_host) {
   if (!status_host) return fail(HINM_ERR_INVALID_ARG, "status_host is NULL");
   int* p = hinm::device_status_ptr();

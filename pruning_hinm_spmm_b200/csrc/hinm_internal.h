@@ -78,6 +78,9 @@ cudaError_t launch_compress(const uint16_t* W, const uint32_t* bitmask, const in
                             const int32_t* perm, const int32_t* counts, int M, int K, int T,
                             const hinm_layout& L, void* ws, int* status, cudaStream_t s);
 
+cudaError_t launch_wait_timeout_selftest(unsigned long long limit_ns, int* status,
+                                         cudaStream_t s);
+
 cudaError_t launch_spmm(const hinm_layout& L, const uint16_t* X, int N, float* Y,
                         int* status, cudaStream_t s);
 

@@ -67,20 +67,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait.  `abort` (shared memory, may be null) lets one role stop the others.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* status,
-                                          volatile int* abort) {
+// Bounded wait.  `abort` (shared memory, may be null) lets one role stop the others; past
+// `limit_ns` the wait records HINM_ERR_DEVICE_TIMEOUT, raises `abort` and returns false.
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, int* status,
+                                              volatile int* abort, unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (abort && *abort) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       record_status(status, HINM_ERR_DEVICE_TIMEOUT);
       if (abort) *abort = 1;
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* status,
+                                          volatile int* abort) {
+  return mbar_wait_for(bar, parity, status, abort, kWaitLimitNs);
 }
 
 // ---------------------------------------------------------------- bulk copies

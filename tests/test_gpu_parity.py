@@ -329,3 +329,23 @@ def test_invalid_permutation_reported(H):
         torch.cuda.synchronize()
         assert H.hinm_device_status() == H.HINM_ERR_INVALID_ARG
         assert H.hinm_device_status() == 0  # cleared by the read
+
+
+def test_bounded_wait_times_out_and_context_survives(H):
+    """A wait that nothing completes gives up after its limit with HINM_ERR_DEVICE_TIMEOUT
+    (the same bounded wait every pipelined kernel uses); the abort flag releases the other
+    waiter, and the context keeps working afterwards."""
+    import time
+    torch.cuda.synchronize()
+    assert H.hinm_device_status() == 0
+    t0 = time.perf_counter()
+    H.hinm_selftest_wait_timeout(20_000_000)  # 20 ms
+    torch.cuda.synchronize()
+    elapsed = time.perf_counter() - t0
+    assert H.hinm_device_status() == H.HINM_ERR_DEVICE_TIMEOUT
+    assert 0.015 < elapsed < 1.0  # gave up after about the limit, not the 2 s default
+    assert H.hinm_device_status() == 0
+    w = hi.tiny_hinm()
+    g = run_path(H, w, None)  # the context is still usable
+    assert H.hinm_device_status() == 0
+    assert g["counts"].shape[0] == w.M // w.T
