@@ -227,12 +227,12 @@ __global__ void __launch_bounds__(kMaskThreads) bitmask_kernel(
   }
 }
 
-// Rows per bitmask CTA: the largest power of two <= 8 whose rows fit in 64 KB of shared
-// memory (T is a multiple of it).
+// Rows per bitmask CTA: the largest power of two <= 8 whose rows fit in 96 KB of shared
+// memory (T is a multiple of it), so that wide rows (K ~ 11008) still get two per CTA.
 static int mask_rows(int K) {
   const size_t K8 = ((size_t)K + 7) & ~size_t(7);
   int rb = 8;
-  while (rb > 1 && (size_t)rb * K8 * sizeof(float) > 64u * 1024u) rb >>= 1;
+  while (rb > 1 && (size_t)rb * K8 * sizeof(float) > 96u * 1024u) rb >>= 1;
   return rb;
 }
 
@@ -270,7 +270,7 @@ cudaError_t launch_mask(const float* I, const int32_t* perm, const int32_t* coun
   const size_t smem = (size_t)RB * (((size_t)K + 7) & ~size_t(7)) * sizeof(float) + (size_t)K;
   for (const void* fn : {(const void*)bitmask_kernel<1>, (const void*)bitmask_kernel<2>,
                          (const void*)bitmask_kernel<4>, (const void*)bitmask_kernel<8>}) {
-    e = set_max_dynamic_smem(fn, 64 * 1024 + kMaxK);
+    e = set_max_dynamic_smem(fn, 96 * 1024 + kMaxK);
     if (e != cudaSuccess) return e;
   }
   const dim3 g(T / RB, nt);
