@@ -2,7 +2,7 @@
 // I[i,c] = fl32(fl32(w_ic^2) * s_c)  (FlexHiNM-GP notes, 关键设计 1/2: second-order
 // importance, importance matrix D; diagonal proxy w^2 ||x_c||^2).
 //
-// Both kernels are HBM streams.  channel_energy reads X once (one thread per channel,
+// Both kernels are HBM streams.  channel_energy reads X once (one warp per channel,
 // 16-byte loads along its row); importance reads W once and writes I once, 4 elements
 // per thread with 8-byte loads and 16-byte stores, grid-stride over the matrix.
 #include <cuda_bf16.h>
@@ -18,73 +18,52 @@ __device__ __forceinline__ double bf16_to_f64(uint32_t bits16) {
   return static_cast<double>(__uint_as_float(bits16 << 16));
 }
 
-// One CTA per 32 channels.  The order of the sum is fixed (n ascending, one fp64 chain per
-// channel), so the sum itself cannot be split; what is parallel is the loading.  All 128
-// threads stage [32 channels x 256 values] chunks of X into shared memory with 16-byte
-// cp.async, double-buffered, while warp 0 runs the 32 chains over the previous chunk
-// (lane = channel; rows padded by 16 bytes so the 16-byte reads are conflict-free).
-constexpr int kEnergyChannels = 32;
-constexpr int kEnergyChunk = 256;                      // values per channel per chunk
-constexpr int kEnergyRowBytes = kEnergyChunk * 2 + 16;  // padded row
-constexpr int kEnergyThreads = 128;
+// One warp per channel.  s_c is fl32 of the sequential fp64 sum of x_cn^2 over n ascending.
+// The warp adds the squares in its own order instead (per lane, then a shuffle tree).  The
+// squares of bf16 values are exact in fp64, and for N non-negative terms every order of fp64
+// additions, the sequential one included, ends within gamma = (N-1) 2^-53 / (1 - (N-1) 2^-53)
+// (relative) of the exact sum; so the sequential result lies in [p (1 - d), p (1 + d)] with
+// d = 4 N 2^-53 > 2.01 gamma, p the warp's sum.  When both ends of that interval round to the
+// same fp32 value, that value is fl32 of the sequential sum (rounding is monotone).  Otherwise
+// (p within about N 2^-51 of an fp32 rounding boundary, or not finite: rare) lane 0 runs the
+// sequential chain itself.
+constexpr int kEnergyWarps = 8;
 
-__device__ __forceinline__ void energy_cp16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-
-__global__ void __launch_bounds__(kEnergyThreads) channel_energy_kernel(
+__global__ void __launch_bounds__(kEnergyWarps * 32) channel_energy_kernel(
     const uint16_t* __restrict__ X, int K, int N, float* __restrict__ s) {
-  __shared__ __align__(16) uint8_t buf[2][kEnergyChannels * kEnergyRowBytes];
-  const int c0 = blockIdx.x * kEnergyChannels;
-  const int nch = min(kEnergyChannels, K - c0);
-  const int nchunks = (N + kEnergyChunk - 1) / kEnergyChunk;
-  constexpr int kPieces = kEnergyChunk / 8;  // 16-byte pieces per channel per chunk
-
-  auto stage = [&](int chunk, int b) {
-    const int n0 = chunk * kEnergyChunk;
-    const int pieces = min(kPieces, (N - n0) / 8);
-    const uint32_t base = (uint32_t)__cvta_generic_to_shared(buf[b]);
-    for (int q = threadIdx.x; q < kEnergyChannels * kPieces; q += kEnergyThreads) {
-      const int ch = q / kPieces, p = q - ch * kPieces;
-      if (ch < nch && p < pieces)
-        energy_cp16(base + ch * kEnergyRowBytes + p * 16, X + (size_t)(c0 + ch) * N + n0 + p * 8);
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-  };
-
-  double acc = 0.0;
-  stage(0, 0);
-  for (int chunk = 0; chunk < nchunks; ++chunk) {
-    if (chunk + 1 < nchunks) {
-      stage(chunk + 1, (chunk + 1) & 1);
-      asm volatile("cp.async.wait_group 1;" ::: "memory");
-    } else {
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
-    }
-    __syncthreads();
-    if (threadIdx.x < nch) {
-      const int nv = min(kEnergyChunk, N - chunk * kEnergyChunk) / 8;
-      const uint4* row = reinterpret_cast<const uint4*>(buf[chunk & 1] + threadIdx.x * kEnergyRowBytes);
-      uint4 q = row[0];
-      for (int v = 0; v < nv; ++v) {
-        const uint4 cur = q;
-        if (v + 1 < nv) q = row[v + 1];  // next 8 values in flight during this chain
-        const uint32_t w[4] = {cur.x, cur.y, cur.z, cur.w};
-        double sq[8];  // x^2 of a bf16 is exact in fp64; computed off the chain
+  const int lane = threadIdx.x & 31;
+  const int c = blockIdx.x * kEnergyWarps + (threadIdx.x >> 5);
+  if (c >= K) return;  // warp-uniform
+  const uint16_t* row = X + (size_t)c * N;
+  double p = 0.0;
+#pragma unroll 4
+  for (int base = lane * 8; base < N; base += 32 * 8) {  // N % 8 == 0: whole 16-byte pieces
+    const uint4 q = __ldg(reinterpret_cast<const uint4*>(row + base));
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const double a = bf16_to_f64(w[h] & 0xFFFFu);
-          const double b = bf16_to_f64(w[h] >> 16);
-          sq[2 * h] = __dmul_rn(a, a);
-          sq[2 * h + 1] = __dmul_rn(b, b);
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc = __dadd_rn(acc, sq[e]);  // n ascending
-      }
+    for (int h = 0; h < 4; ++h) {
+      const double a = bf16_to_f64(w[h] & 0xFFFFu);
+      const double b = bf16_to_f64(w[h] >> 16);
+      p = __dadd_rn(p, __dadd_rn(__dmul_rn(a, a), __dmul_rn(b, b)));
     }
-    __syncthreads();  // buffer (chunk & 1) is refilled by the next iteration's stage()
   }
-  if (threadIdx.x < nch) s[c0 + threadIdx.x] = __double2float_rn(acc);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) p = __dadd_rn(p, __shfl_xor_sync(0xffffffffu, p, o));
+  if (lane == 0) {
+    const double d = __dmul_rn(p, __dmul_rn((double)N, 0x1p-51));
+    const float lo = __double2float_rn(__dsub_rn(p, d));
+    const float hi = __double2float_rn(__dadd_rn(p, d));
+    float r = lo;
+    if (!(lo == hi)) {
+      double acc = 0.0;  // the sequential chain, n ascending
+      for (int n = 0; n < N; ++n) {
+        const double v = bf16_to_f64(row[n]);
+        acc = __dadd_rn(acc, __dmul_rn(v, v));
+      }
+      r = __double2float_rn(acc);
+    }
+    s[c] = r;
+  }
 }
 
 // 4 consecutive elements of one row per quad (K % 4 == 0); each thread takes kQuads quads
@@ -169,7 +148,7 @@ size_t importance_workspace_bytes(int K) { return ((size_t)K * sizeof(float) + 2
 
 cudaError_t launch_importance(const uint16_t* W, const uint16_t* X, int M, int K, int N,
                               float* I, float* s_scratch, cudaStream_t st) {
-  channel_energy_kernel<<<(K + kEnergyChannels - 1) / kEnergyChannels, kEnergyThreads, 0, st>>>(
+  channel_energy_kernel<<<(K + kEnergyWarps - 1) / kEnergyWarps, kEnergyWarps * 32, 0, st>>>(
       X, K, N, s_scratch);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -161,6 +161,25 @@ def test_integer_product_bitwise(H, T, N, perm):
     assert np.array_equal(g["Y"], np.round(g["Y"]))
 
 
+def test_channel_energy_rounding_fallback(H):
+    """Channels whose fp64 sum sits on an fp32 rounding midpoint: the order matters there,
+    so the GPU must reproduce the sequential sum (1 first: 1.0; 1 last: 1 + 2^-23)."""
+    K, N, M = 64, 64, 8
+    rng = np.random.default_rng(11)
+    Xf = rng.normal(0.0, 1.0, (K, N)).astype(np.float32)
+    Xf[0] = [1.0, 2.0 ** -12] + [2.0 ** -27] * (N - 2)
+    Xf[1] = [2.0 ** -12] + [2.0 ** -27] * (N - 2) + [1.0]
+    Xf[2] = 2.0 ** -27                       # all tiny: exact in any order
+    Xf[3] = 0.0
+    X = hi.f32_to_bf16_bits(Xf)
+    W = hi.f32_to_bf16_bits(np.ones((M, K), dtype=np.float32))
+    I = H.hinm_importance(dev_bf16(W), dev_bf16(X)).cpu().numpy()
+    status_ok(H)
+    I_ref = O.importance(W, X)
+    assert I_ref[0, 0] == np.float32(1.0) and I_ref[0, 1] == np.float32(1.0 + 2.0 ** -23)
+    np.testing.assert_array_equal(I.view(np.uint32), I_ref.view(np.uint32))
+
+
 def test_hand_built_first_drop(H):
     """The hand-built tile where regrouping makes R drop at m = 2: the GPU scan stops at m=1."""
     K, N, T = 64, 8, 64

@@ -39,6 +39,24 @@ def test_energy_closed_form_ones():
                                                  dtype=np.float32) * N)
 
 
+def test_energy_is_the_sequential_fp64_sum():
+    # The reading fixes the order (n ascending, fp64).  Row [1, 2^-12, 62 x 2^-27]: the
+    # squares are 1, 2^-24 and 2^-54.  In order, 1 + 2^-24 is exact and each 2^-54 is a
+    # quarter of an fp64 ulp at 1, so it is lost: the sum is 1 + 2^-24, the midpoint between
+    # fp32 1 and 1 + 2^-23, which rounds to even (1).  The same squares with the 1 last add
+    # up exactly first (2^-24 + 62 * 2^-54), then 1 + 2^-24 + 31 * 2^-53 rounds to
+    # 1 + 2^-24 + 2^-48 in fp64, above the midpoint: 1 + 2^-23.  The exact sum rounds up too.
+    N = 64
+    a = [1.0, 2.0 ** -12] + [2.0 ** -27] * (N - 2)
+    b = [2.0 ** -12] + [2.0 ** -27] * (N - 2) + [1.0]
+    X = bf([a, b])
+    s = O.channel_energy(X)
+    assert s[0] == np.float32(1.0)
+    assert s[1] == np.float32(1.0 + 2.0 ** -23)
+    exact = sum(Fraction(v) ** 2 for v in a)
+    assert exact > 1 + Fraction(1, 2 ** 24)          # so fl32(exact sum) would be 1 + 2^-23
+
+
 def test_importance_hand_example_not_transposed():
     # W = [[1, 2], [3, 0.5]], X = [[1, 1, 1], [2, 0, 0]]  ->  s = [3, 4]
     # I = [[1*3, 4*4], [9*3, 0.25*4]] = [[3, 16], [27, 1]]
