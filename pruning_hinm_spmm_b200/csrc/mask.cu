@@ -13,6 +13,7 @@
 
 #include "hinm_internal.h"
 #include "ptx.cuh"
+#include "stage_rows.cuh"
 
 namespace hinm {
 
@@ -107,13 +108,6 @@ __global__ void __launch_bounds__(1024) classify_kernel(const int32_t* __restric
 // warp ballots, 32 words per warp and row, and stored coalesced.
 constexpr int kMaskThreads = 512;
 
-// Slot of channel c in the channel-major shared rows (rows padded to a multiple of 8
-// channels): within each aligned group of 8 channels the 16-byte bank slot is permuted by
-// higher bits of c, so that strided channels of consecutive groups use different banks.
-__device__ __forceinline__ int mask_chan_slot(int c) {
-  return (c & ~7) | ((c ^ (c >> 3) ^ (c >> 6)) & 7);
-}
-
 template <int RB>
 __device__ __forceinline__ void mask_load_rows(const float* p, float (&v)[RB]) {
   if constexpr (RB == 8) {
@@ -138,7 +132,7 @@ __global__ void __launch_bounds__(kMaskThreads) bitmask_kernel(
     const int32_t* __restrict__ member, int K, int T, uint32_t* __restrict__ bitmask) {
   extern __shared__ __align__(16) uint8_t mask_smem[];
   const int K8 = (K + 7) & ~7;
-  float* rows_s = reinterpret_cast<float*>(mask_smem);  // [K8][RB], mask_chan_slot order
+  float* rows_s = reinterpret_cast<float*>(mask_smem);  // [K8][RB], stage_slot order
   uint8_t* keep = mask_smem + (size_t)K8 * RB * sizeof(float);
   const int words = (K + 31) >> 5;
   const int t = blockIdx.y;
@@ -148,22 +142,15 @@ __global__ void __launch_bounds__(kMaskThreads) bitmask_kernel(
   const int8_t* reg = region + (size_t)t * K;
   const float* src = I + ((size_t)t * T + r0) * K;
   constexpr uint8_t kAll = (uint8_t)((1u << RB) - 1u);
-  for (int c = threadIdx.x; c < K; c += kMaskThreads) {
-    float v[RB];
-#pragma unroll
-    for (int r = 0; r < RB; ++r) v[r] = __ldg(src + (size_t)r * K + c);
-    float* d = rows_s + (size_t)mask_chan_slot(c) * RB;
-    if constexpr (RB == 8) {
-      reinterpret_cast<float4*>(d)[0] = make_float4(v[0], v[1], v[2], v[3]);
-      reinterpret_cast<float4*>(d)[1] = make_float4(v[4], v[5], v[6], v[7]);
-    } else if constexpr (RB == 4) {
-      *reinterpret_cast<float4*>(d) = make_float4(v[0], v[1], v[2], v[3]);
-    } else if constexpr (RB == 2) {
-      *reinterpret_cast<float2*>(d) = make_float2(v[0], v[1]);
-    } else {
-      d[0] = v[0];
-    }
-    keep[c] = __ldg(reg + c) == HINM_REGION_DENSE ? kAll : (uint8_t)0;
+  stage_rows<RB, kMaskThreads>(src, K, rows_s);
+  // dense channels keep every row; 4 channels per thread (K % 4 == 0)
+  for (int q = threadIdx.x; q < (K >> 2); q += kMaskThreads) {
+    const char4 rq = __ldg(reinterpret_cast<const char4*>(reg) + q);
+    const uint32_t k4 = (rq.x == HINM_REGION_DENSE ? (uint32_t)kAll : 0u) |
+                        (rq.y == HINM_REGION_DENSE ? (uint32_t)kAll << 8 : 0u) |
+                        (rq.z == HINM_REGION_DENSE ? (uint32_t)kAll << 16 : 0u) |
+                        (rq.w == HINM_REGION_DENSE ? (uint32_t)kAll << 24 : 0u);
+    reinterpret_cast<uint32_t*>(keep)[q] = k4;
   }
   __syncthreads();
 
@@ -181,7 +168,7 @@ __global__ void __launch_bounds__(kMaskThreads) bitmask_kernel(
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       c[k] = ((unsigned)cc[k] < (unsigned)K) ? cc[k] : 0;  // never index outside I
-      mask_load_rows<RB>(rows_s + (size_t)mask_chan_slot(c[k]) * RB, v[k]);
+      mask_load_rows<RB>(rows_s + (size_t)stage_slot(c[k]) * RB, v[k]);
     }
     // g_kl bit r: member l beats member k (k < l) in row r, i.e. v_l > v_k (equal values:
     // the lower position k wins).  Member k is kept iff at most one member beats it: the

@@ -23,6 +23,7 @@
 
 #include "hinm_internal.h"
 #include "ptx.cuh"
+#include "stage_rows.cuh"
 
 namespace hinm {
 
@@ -468,15 +469,8 @@ struct CandidateList {
   Candidate c[kMaxCandidates];
 };
 
-// Slot of channel c in the channel-major shared rows: within each aligned group of 8
-// channels, the 16-byte bank slot is permuted by higher bits of c, so that the strided
-// channels of consecutive groups (4, 8, 16, 32 or 64 apart) fall into different banks.
-__device__ __forceinline__ int chan_slot(int c) {
-  return (c & ~7) | ((c ^ (c >> 3) ^ (c >> 6)) & 7);
-}
-
 // Per (candidate m, tile), 512 threads: the channels of the 2:4 band in ascending working
-// position (block-wide prefix count), stored as their shared-memory slots chan_slot(c) in
+// position (block-wide prefix count), stored as their shared-memory slots stage_slot(c) in
 // band_sum's staged rows -> band[t][m][q], and the exact sum of the dense
 // vectors' column sums -> rdense[t][m] (values below the tile's scale go to the buckets).
 template <int kPerMax>
@@ -553,7 +547,7 @@ __global__ void __launch_bounds__(512, 2) candidate_lists_kernel(
           }
         }
       } else if (r < n4 + n24) {
-        out[pos++] = (unsigned short)chan_slot(c[q]);
+        out[pos++] = (unsigned short)stage_slot(c[q]);
       }
     }
   }
@@ -593,20 +587,6 @@ __device__ __forceinline__ void load_rows(const float* p, float (&v)[RB]) {
   }
 }
 
-template <int RB>
-__device__ __forceinline__ void store_rows(float* p, const float (&v)[RB]) {
-  if constexpr (RB == 8) {
-    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
-    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
-  } else if constexpr (RB == 4) {
-    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
-  } else if constexpr (RB == 2) {
-    *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
-  } else {
-    *p = v[0];
-  }
-}
-
 // Exact sum of a value that missed the fast path (p < eb): to the tile-scale 128-bit sum
 // `ex` when p >= lsb, else to the exponent buckets.
 __device__ __forceinline__ void band_slow(float v, U128& ex, int lsb, unsigned long long* bkt,
@@ -624,7 +604,7 @@ __device__ __forceinline__ void band_slow(float v, U128& ex, int lsb, unsigned l
 }
 
 // Per (tile, chunk of RB rows), 512 threads.  The chunk's rows of I are staged in shared
-// memory channel-major (the RB values of channel c contiguous at slot chan_slot(c), one
+// memory channel-major (the RB values of channel c contiguous at slot stage_slot(c), one
 // vector load each).  Then, candidate by candidate, the candidate's 2:4 groups are dealt to
 // the warps in chunks (the starting warp rotates, so the work stays even over the scan)
 // and, for every row, the top 2 of the group's 4 values are summed.
@@ -641,7 +621,7 @@ __global__ void __launch_bounds__(kThreads) band_sum_kernel(
     const int* __restrict__ tile_pmax, int K, int T, CandidateList cl, int ncand,
     U128* __restrict__ part, unsigned long long* __restrict__ bucket,
     int* __restrict__ bucket_used) {
-  extern __shared__ __align__(16) float rows_s[];  // [K rounded up to 8][RB], chan_slot order
+  extern __shared__ __align__(16) float rows_s[];  // [K rounded up to 8][RB], stage_slot order
   __shared__ unsigned long long fast_sum[kMaxCandidates];   // units of 2^(eb - 149)
   __shared__ unsigned long long digits[kMaxCandidates][4];  // slow path, units of 2^(lsb - 149)
   const int chunk = blockIdx.x, t = blockIdx.y;
@@ -655,13 +635,7 @@ __global__ void __launch_bounds__(kThreads) band_sum_kernel(
   const double unit_scale = pow2(149 - eb);                      // fp64 sum -> integer units
   for (int x = threadIdx.x; x < kMaxCandidates; x += kThreads) fast_sum[x] = 0ull;
   for (int x = threadIdx.x; x < kMaxCandidates * 4; x += kThreads) (&digits[0][0])[x] = 0ull;
-  const float* src = I + ((size_t)t * T + (size_t)chunk * RB) * K;
-  for (int c = threadIdx.x; c < K; c += kThreads) {
-    float v[RB];
-#pragma unroll
-    for (int r = 0; r < RB; ++r) v[r] = __ldg(src + (size_t)r * K + c);
-    store_rows<RB>(rows_s + (size_t)chan_slot(c) * RB, v);
-  }
+  stage_rows<RB, kThreads>(I + ((size_t)t * T + (size_t)chunk * RB) * K, K, rows_s);
   __syncthreads();
 
   const unsigned short* band_t = band + (size_t)t * ncand * K;
@@ -693,7 +667,7 @@ __global__ void __launch_bounds__(kThreads) band_sum_kernel(
 #pragma unroll
       for (int j = 0; j < kG; ++j) {
         if (gb + 32 * j >= ng) break;
-        // the lists hold shared-memory slots (chan_slot of the channel), below K rounded up to 8
+        // the lists hold shared-memory slots (stage_slot of the channel), below K rounded up to 8
         float v0[RB], v1[RB], v2[RB], v3[RB];
         load_rows<RB>(rows_s + min((int)cq[j].x, K8 - 1) * RB, v0);
         load_rows<RB>(rows_s + min((int)cq[j].y, K8 - 1) * RB, v1);
@@ -828,7 +802,7 @@ struct BandCfg {
   int rows, threads;
 };
 static BandCfg band_config(int K) {
-  const size_t K8 = ((size_t)K + 7) & ~size_t(7);  // chan_slot stays below K rounded up to 8
+  const size_t K8 = ((size_t)K + 7) & ~size_t(7);  // stage_slot stays below K rounded up to 8
   int rb = 4;
   while (rb > 1 && (size_t)rb * K8 * sizeof(float) > 96u * 1024u) rb >>= 1;
   return {rb, 512};
