@@ -180,6 +180,28 @@ def test_channel_energy_rounding_fallback(H):
     np.testing.assert_array_equal(I.view(np.uint32), I_ref.view(np.uint32))
 
 
+@pytest.mark.parametrize("name,make,v_s", CASES, ids=[c[0] for c in CASES])
+def test_search_decision_without_retained_matches_full_scan(H, name, make, v_s):
+    """With no R requested the scan may stop evaluating candidates after a tile's decision;
+    the counts and v_s must still equal the full scan's and the oracle's."""
+    w = make()
+    M, K, T = w.M, w.K, w.T
+    I = H.hinm_importance(dev_bf16(w.W_bits), dev_bf16(w.X_bits))
+    perm = dev_i32(w.perm)
+    c_e, vs_e, _ = H.hinm_boundary_search(I, perm, T, w.t_s, w.alpha, want_rank=False)
+    nc = H.hinm_search_num_candidates(K, w.t_s, w.alpha)
+    R = torch.empty((M // T, nc), dtype=torch.float64, device="cuda")
+    c_f, vs_f, _ = H.hinm_boundary_search(I, perm, T, w.t_s, w.alpha, want_rank=False,
+                                          retained_out=R)
+    torch.cuda.synchronize()
+    status_ok(H)
+    sr = O.boundary_search(I.cpu().numpy(), w.perm, T, w.t_s, w.alpha)
+    np.testing.assert_array_equal(c_e.cpu().numpy(), sr.counts)
+    np.testing.assert_array_equal(vs_e.cpu().numpy(), np.asarray(sr.v_s))
+    np.testing.assert_array_equal(c_f.cpu().numpy(), sr.counts)
+    np.testing.assert_array_equal(vs_f.cpu().numpy(), np.asarray(sr.v_s))
+
+
 def test_hand_built_first_drop(H):
     """The hand-built tile where regrouping makes R drop at m = 2: the GPU scan stops at m=1."""
     K, N, T = 64, 8, 64
