@@ -177,20 +177,14 @@ __device__ __forceinline__ bool mask_bit(const uint32_t* bm, int words, int i, i
   return (__ldg(bm + (size_t)i * words + (c >> 5)) >> (c & 31)) & 1u;
 }
 
-// The stored pair of one 2:4 group from its 4 weights and kept bits: positions a < b and
-// their values.  The common case has exactly two kept positions.  A malformed group is
-// reported (HINM_ERR_BAD_MASK); its kept positions, lowest first, are completed from the
-// unkept ones with value 0, so the pair stays a legal (a < b) pattern.
-__device__ __forceinline__ void select_pair(const uint32_t (&w)[4], uint32_t kept, uint32_t& a,
-                                            uint32_t& bb, uint32_t& va, uint32_t& vb,
-                                            int* status) {
-  if (__popc(kept) == 2) {
-    a = (uint32_t)(__ffs(kept) - 1);
-    bb = (uint32_t)(31 - __clz(kept));
-    va = a == 0 ? w[0] : (a == 1 ? w[1] : w[2]);   // a <= 2
-    vb = bb == 1 ? w[1] : (bb == 2 ? w[2] : w[3]);  // b >= 1
-    return;
-  }
+// A malformed group (not exactly two kept positions) is reported (HINM_ERR_BAD_MASK); its
+// kept positions, lowest first, are completed from the unkept ones with value 0, so the pair
+// stays a legal (a < b) pattern.  Out of line: it is rare, and inlined into every unrolled
+// item it would crowd the packing loops out of the instruction cache.
+__device__ __noinline__ void select_pair_malformed(uint32_t w0, uint32_t w1, uint32_t w2,
+                                                   uint32_t w3, uint32_t kept, uint32_t* out,
+                                                   int* status) {
+  const uint32_t w[4] = {w0, w1, w2, w3};
   ptx::record_status(status, HINM_ERR_BAD_MASK);
   int pos[2], np = 0;
 #pragma unroll
@@ -203,10 +197,30 @@ __device__ __forceinline__ void select_pair(const uint32_t (&w)[4], uint32_t kep
   const int pb = pos[1] < 0 ? -1 - pos[1] : pos[1];
   const bool ua = pos[0] >= 0, ub = pos[1] >= 0;
   if (pa < pb) {  // order the pair by position
-    a = pa; bb = pb; va = ua ? w[pa] : 0u; vb = ub ? w[pb] : 0u;
+    out[0] = pa; out[1] = pb; out[2] = ua ? w[pa] : 0u; out[3] = ub ? w[pb] : 0u;
   } else {
-    a = pb; bb = pa; va = ub ? w[pb] : 0u; vb = ua ? w[pa] : 0u;
+    out[0] = pb; out[1] = pa; out[2] = ub ? w[pb] : 0u; out[3] = ua ? w[pa] : 0u;
   }
+}
+
+// The stored pair of one 2:4 group from its 4 weights and kept bits: positions a < b and
+// their values.  The common case has exactly two kept positions.
+__device__ __forceinline__ void select_pair(const uint32_t (&w)[4], uint32_t kept, uint32_t& a,
+                                            uint32_t& bb, uint32_t& va, uint32_t& vb,
+                                            int* status) {
+  if (__popc(kept) == 2) {
+    a = (uint32_t)(__ffs(kept) - 1);
+    bb = (uint32_t)(31 - __clz(kept));
+    va = a == 0 ? w[0] : (a == 1 ? w[1] : w[2]);   // a <= 2
+    vb = bb == 1 ? w[1] : (bb == 2 ? w[2] : w[3]);  // b >= 1
+    return;
+  }
+  uint32_t out[4];
+  select_pair_malformed(w[0], w[1], w[2], w[3], kept, out, status);
+  a = out[0];
+  bb = out[1];
+  va = out[2];
+  vb = out[3];
 }
 
 __global__ void __launch_bounds__(256) pack_kernel(const uint16_t* __restrict__ W,
