@@ -422,40 +422,64 @@ def main():
     value = job_value(model["flops_eff"], world, t_step)
 
     # ---------------- end to end through the public API with host buffers
+    # Every step copies its inputs in from pinned host memory and its Y out.  Two device
+    # buffer sets (each with its own HotPath) let step k+1's upload and step k-1's download
+    # run on their own streams while step k computes; a set is reused only after its inputs
+    # were consumed and its Y was read back (events).
     W_h = torch.from_numpy(w.W_bits.view(np.int16)).pin_memory()
     X_h = torch.from_numpy(w.X_bits.view(np.int16)).pin_memory()
     P_h = torch.from_numpy(w.perm).pin_memory()
-    Y_h = torch.empty((M, N), dtype=torch.float32).pin_memory()
-    W_d = torch.empty_like(W)
-    X_d = torch.empty_like(X)
-    P_d = torch.empty_like(perm)
+    sets = []
+    for b in range(2):
+        hp_b = hp if b == 0 else H.HotPath(M, K, N, T, w.t_s, w.alpha, device=dev)
+        sets.append(dict(hp=hp_b, W=torch.empty_like(W), X=torch.empty_like(X),
+                         P=torch.empty_like(perm),
+                         Y=torch.empty((M, N), dtype=torch.float32).pin_memory(),
+                         consumed=torch.cuda.Event(), read=torch.cuda.Event(),
+                         loaded=torch.cuda.Event()))
+    s_up, s_comp, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    for st in sets:  # both sets start free
+        st["consumed"].record(s_comp)
+        st["read"].record(s_down)
 
-    def e2e_step():
-        W_d.view(torch.int16).copy_(W_h, non_blocking=True)
-        X_d.view(torch.int16).copy_(X_h, non_blocking=True)
-        P_d.copy_(P_h, non_blocking=True)
-        hp.run(W_d, X_d, P_d, fixed_counts=fixed)
-        Y_h.copy_(hp.Y, non_blocking=True)
+    def e2e_step(k):
+        st = sets[k % 2]
+        s_up.wait_event(st["consumed"])
+        with torch.cuda.stream(s_up):
+            st["W"].view(torch.int16).copy_(W_h, non_blocking=True)
+            st["X"].view(torch.int16).copy_(X_h, non_blocking=True)
+            st["P"].copy_(P_h, non_blocking=True)
+        st["loaded"].record(s_up)
+        s_comp.wait_event(st["loaded"])
+        s_comp.wait_event(st["read"])
+        with torch.cuda.stream(s_comp):
+            st["hp"].run(st["W"], st["X"], st["P"], fixed_counts=fixed, stream=s_comp)
+        st["consumed"].record(s_comp)
+        s_down.wait_event(st["consumed"])
+        with torch.cuda.stream(s_down):
+            st["Y"].copy_(st["hp"].Y, non_blocking=True)
+        st["read"].record(s_down)
 
-    for _ in range(2):
-        e2e_step()
+    for k in range(2):
+        e2e_step(k)
     torch.cuda.synchronize()
     e_start = torch.cuda.Event(enable_timing=True)
     e_end = torch.cuda.Event(enable_timing=True)
-    e2e_steps = max(3, min(args.steps, 10))
+    e2e_steps = max(4, min(args.steps, 10))
     if dist:
         dist.barrier()
-    e_start.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e_end.record(stream)
+    e_start.record(s_up)
+    for k in range(e2e_steps):
+        e2e_step(k)
+    e_end.record(s_down)
     torch.cuda.synchronize()
     t_e2e = e_start.elapsed_time(e_end) * 1e-3 / e2e_steps
     t_e2e = max_over_ranks(t_e2e, dist, dev)
     h2d = W_h.numel() * 2 + X_h.numel() * 2 + P_h.numel() * 4
-    d2h = Y_h.numel() * 4
-    # the e2e output must match the device-resident path
-    assert torch.equal(Y_h, hp.Y.cpu())
+    d2h = sets[0]["Y"].numel() * 4
+    # the e2e outputs must match the device-resident path
+    for st in sets:
+        assert torch.equal(st["Y"], hp.Y.cpu())
 
     if dist:
         dist.destroy_process_group()
@@ -520,7 +544,9 @@ def main():
         "cpu_baseline": cpu,
         "e2e": {"value": job_value(model["flops_eff"], world, t_e2e), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": t_e2e * 1e3},
+                "ms_per_step": t_e2e * 1e3,
+                "pipelining": "two buffer sets; upload, compute and download on their own "
+                              "streams"},
         "gpu_launches": kernels_per_step * args.steps,
         "gpu_launches_phase_pass": kernels_per_step * args.steps,
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
