@@ -390,3 +390,46 @@ def test_bounded_wait_times_out_and_context_survives(H):
     g = run_path(H, w, None)  # the context is still usable
     assert H.hinm_device_status() == 0
     assert g["counts"].shape[0] == w.M // w.T
+
+
+SWEEP_LINEARS = ["q", "k", "v", "o", "gate", "up", "down"]
+SWEEP_TS = [0.5, 0.625, 0.75]
+
+
+@pytest.mark.parametrize("layer", list(range(1, 32)))
+def test_llama_sweep_other_layers_sampled(H, layer):
+    """Layers 1..31 of the sweep (one linear and one t_s per layer, rotating; N = 16): the
+    search's counts, v_s and ranking, the mask, region and layout bytes of one sampled tile
+    bit for bit, and that tile's Y within tolerance."""
+    linear = SWEEP_LINEARS[layer % 7]
+    t_s = SWEEP_TS[layer % 3]
+    N = 16
+    w = hi.llama_sweep_layer(layer, linear, N, t_s)
+    M, K, T = w.M, w.K, w.T
+    nt = M // T
+    W, X, perm = dev_bf16(w.W_bits), dev_bf16(w.X_bits), dev_i32(w.perm)
+    hp = H.HotPath(M, K, N, T, w.t_s, w.alpha)
+    Y = hp.run(W, X, perm)  # counts from the search
+    torch.cuda.synchronize()
+    status_ok(H)
+    tiles = [layer % nt]
+    rows = np.concatenate([np.arange(t * T, (t + 1) * T) for t in tiles])
+    s = O.channel_energy(w.X_bits)
+    Wf = hi.bf16_bits_to_f32(w.W_bits[rows])
+    I_rows = ((Wf * Wf).astype(np.float32) * s[None, :]).astype(np.float32)
+    np.testing.assert_array_equal(hp.I[rows].cpu().numpy().view(np.uint32), I_rows.view(np.uint32))
+    I_full_rows = np.zeros((M, K), dtype=np.float32)
+    I_full_rows[rows] = I_rows
+    sr = O.boundary_search(I_full_rows, w.perm, T, t_s, w.alpha, tiles=tiles)
+    counts = hp.counts.cpu().numpy()
+    np.testing.assert_array_equal(counts[tiles], sr.counts[tiles])
+    np.testing.assert_array_equal(hp.vs.cpu().numpy()[tiles], np.asarray(sr.v_s)[tiles])
+    np.testing.assert_array_equal(hp.rank.cpu().numpy()[tiles], sr.rank[tiles])
+    bm_ref, reg_ref = O.mask(I_full_rows, w.perm, T, counts, tiles=tiles)
+    bm = hp.bitmask.cpu().numpy().view(np.uint32)
+    np.testing.assert_array_equal(bm[rows], bm_ref[rows])
+    np.testing.assert_array_equal(hp.region.cpu().numpy()[tiles], reg_ref[tiles])
+    L_ref = O.compress(w.W_bits, bm_ref, reg_ref, w.perm, counts, T, tiles=tiles)
+    layout_equal(hp.layout, L_ref, tiles=tiles)
+    y_ref, bound = O.spmm_reference(w.W_bits, bm_ref, w.X_bits, rows=rows)
+    check_y(Y.cpu().numpy(), y_ref, bound, rows=rows)
