@@ -202,6 +202,44 @@ def test_search_decision_without_retained_matches_full_scan(H, name, make, v_s):
     np.testing.assert_array_equal(vs_f.cpu().numpy(), np.asarray(sr.v_s))
 
 
+def test_gpu_permutation_invariance(H):
+    """Reordering input channels consistently leaves the GPU result unchanged (FlexHiNM-GP
+    notes, 关键设计 2): run(W, X, pi) and run(W[:, pi], X[pi, :], identity) give the same
+    counts, the same mask after remapping, the same value and metadata bytes, indices related
+    by pi, and bitwise the same Y."""
+    w = hi.custom(256, 640, 72, 128, seed=31, t_s=0.625, v_s=None, random_perm=True)
+    M, K, N, T = w.M, w.K, w.N, w.T
+    Wp = np.ascontiguousarray(w.W_bits[:, w.perm])
+    Xp = np.ascontiguousarray(w.X_bits[w.perm, :])
+    ident = np.arange(K, dtype=np.int32)
+    out = []
+    for Wb, Xb, pm in ((w.W_bits, w.X_bits, w.perm), (Wp, Xp, ident)):
+        hp = H.HotPath(M, K, N, T, w.t_s, w.alpha)
+        Y = hp.run(dev_bf16(Wb), dev_bf16(Xb), dev_i32(pm))
+        torch.cuda.synchronize()
+        status_ok(H)
+        L = hp.layout
+        out.append(dict(counts=hp.counts.cpu().numpy(), Y=Y.cpu().numpy(),
+                        bits=O.unpack_bits(hp.bitmask.cpu().numpy().view(np.uint32), K),
+                        vd=L.vals_dense.cpu().numpy(), vsp=L.vals_sparse.cpu().numpy(),
+                        meta=L.meta.cpu().numpy(), info=L.tile_info.cpu().numpy(),
+                        idd=L.idx_dense.cpu().numpy(), ids=L.idx_sparse.cpu().numpy()))
+    a, b = out
+    np.testing.assert_array_equal(a["counts"], b["counts"])
+    np.testing.assert_array_equal(a["bits"][:, w.perm], b["bits"])
+    np.testing.assert_array_equal(a["info"], b["info"])
+    # the blocks each tile uses (buffers are allocated to capacity)
+    dense = np.concatenate([np.arange(d0, d0 + nd) for nd, ns, d0, s0 in a["info"]])
+    sparse = np.concatenate([np.arange(s0, s0 + ns) for nd, ns, d0, s0 in a["info"]])
+    np.testing.assert_array_equal(a["vd"][dense], b["vd"][dense])
+    np.testing.assert_array_equal(a["vsp"][sparse], b["vsp"][sparse])
+    np.testing.assert_array_equal(a["meta"][sparse], b["meta"][sparse])
+    for ia, ib in ((a["idd"][dense], b["idd"][dense]), (a["ids"][sparse], b["ids"][sparse])):
+        real = ~((ia == 0) & (ib == 0))  # padding entries are 0 on both sides
+        np.testing.assert_array_equal(ia[real], w.perm[ib[real]])
+    np.testing.assert_array_equal(a["Y"].view(np.uint32), b["Y"].view(np.uint32))
+
+
 def test_hand_built_first_drop(H):
     """The hand-built tile where regrouping makes R drop at m = 2: the GPU scan stops at m=1."""
     K, N, T = 64, 8, 64
