@@ -202,6 +202,26 @@ def test_search_decision_without_retained_matches_full_scan(H, name, make, v_s):
     np.testing.assert_array_equal(vs_f.cpu().numpy(), np.asarray(sr.v_s))
 
 
+@pytest.mark.parametrize("M,K,N,perm", [(256, 512, 128, False), (384, 640, 264, True),
+                                         (128, 4096, 16, True)])
+def test_dense_ts0_matches_torch_matmul(H, M, K, N, perm):
+    """t_s = 0 keeps every weight: the SpMM is a dense GEMM, so torch.matmul (fp32 of the bf16
+    inputs) is an independent third opinion next to the oracle."""
+    w = hi.custom(M, K, N, 128, seed=41, t_s=0.0, v_s=None, random_perm=perm)
+    W, X = dev_bf16(w.W_bits), dev_bf16(w.X_bits)
+    hp = H.HotPath(M, K, N, 128, 0.0, w.alpha)
+    Y = hp.run(W, X, dev_i32(w.perm))
+    torch.cuda.synchronize()
+    status_ok(H)
+    assert int(hp.counts[:, 2].min()) == K  # every vector dense
+    Wf, Xf = W.float(), X.float()
+    ref = (Wf.double() @ Xf.double()).cpu().numpy()
+    bound = (Wf.abs().double() @ Xf.abs().double()).cpu().numpy()
+    check_y(Y.cpu().numpy(), ref, bound)
+    mm = torch.matmul(Wf, Xf).cpu().numpy()
+    check_y(Y.cpu().numpy(), mm.astype(np.float64), bound)
+
+
 def test_gpu_permutation_invariance(H):
     """Reordering input channels consistently leaves the GPU result unchanged (FlexHiNM-GP
     notes, 关键设计 2): run(W, X, pi) and run(W[:, pi], X[pi, :], identity) give the same
