@@ -65,6 +65,9 @@ struct SpmmCfg {
                                    : kTmemNeed <= 256 ? 256 : 512;
   static constexpr size_t kSmemBytes = (size_t)kStages * (kStageBytes + kIdxBytes) +
                                        1024 /*align*/ + 512 /*barriers*/ + kRedBytes;
+  // wide N: the second 64 K-rows of a 2:4 block's B land on a barrier of their own, so the
+  // MMAs on the first 64 rows start before the second half arrives
+  static constexpr bool kSplitB = BN >= 128;
   static constexpr int kProducers = 128;
   static constexpr int kMmaWarp = 4;
   static constexpr int kBulkWarp = 9;
@@ -116,10 +119,13 @@ struct Gather {
 #pragma unroll
     for (int i = 0; i < kPer; ++i) xr[i] = idx_s[(ptid + C::kProducers * i) / C::kChunksPerRow];
   }
+  // items [I0, I1): item i covers row (ptid + kProducers i) / kChunksPerRow, so for 128 rows
+  // the first kPer / 2 items are rows 0..63 and the rest rows 64..127
+  template <int I0 = 0, int I1 = kPer>
   __device__ __forceinline__ void copy(uint32_t B_s, const uint16_t* __restrict__ X, int N,
                                        int n0, int ptid) const {
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
+    for (int i = I0; i < I1; ++i) {
       const int q = ptid + C::kProducers * i;
       const int r = q / C::kChunksPerRow, cc = q - r * C::kChunksPerRow;
       const int at = cc / C::kChunksPerAtom, c = cc - at * C::kChunksPerAtom;
@@ -144,9 +150,9 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* idx_region = smem + C::kStages * C::kStageBytes;  // [S][kIdxBytes]
   uint64_t* bars = reinterpret_cast<uint64_t*>(idx_region + C::kStages * C::kIdxBytes);
   // [0,S) full, [S,2S) empty, 2S+{0,1} accumulator full, 2S+{2,3} accumulator empty,
-  // 2S+4 drain, [2S+5, 3S+5) index ready; then the TMEM address, the abort flag and one run
-  // flag per stage (at most 272 bytes of the 512 reserved)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * C::kStages + 5);
+  // 2S+4 drain, [2S+5, 3S+5) index ready, [3S+5, 4S+5) second-half full; then the TMEM
+  // address, the abort flag and one run flag per stage (at most 336 bytes of the 512 reserved)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 * C::kStages + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* run_s = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
@@ -157,12 +163,14 @@ __global__ void __launch_bounds__(320, 1)
   auto acce_bar = [&](int b) { return ptx::smem_u32(bars + 2 * C::kStages + 2 + b); };
   const uint32_t drain_bar = ptx::smem_u32(bars + 2 * C::kStages + 4);
   auto idx_bar = [&](int s) { return ptx::smem_u32(bars + 2 * C::kStages + 5 + s); };
+  auto full2_bar = [&](int s) { return ptx::smem_u32(bars + 3 * C::kStages + 5 + s); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       ptx::mbar_init(full_bar(s), 1 + C::kProducers);  // expect_tx arrival + one per producer
       ptx::mbar_init(empty_bar(s), 1);
       ptx::mbar_init(idx_bar(s), 1);
+      ptx::mbar_init(full2_bar(s), 1 + C::kProducers);  // used when kSplitB
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(accf_bar(b), 1);
@@ -202,7 +210,9 @@ __global__ void __launch_bounds__(320, 1)
     // then either gather the X rows the block's index selects (16-byte cp.async, arrival
     // when they land) or, for a contiguous run it moves by TMA, just arrive.  Every thread
     // arrives on the stage's full barrier once per block, after its last read of the
-    // stage's run flag and indices, so the stage cannot be recycled under it.
+    // stage's run flag and indices, so the stage cannot be recycled under it.  With
+    // kSplitB, rows 64..127 of a 2:4 block arrive on the stage's second-half barrier (every
+    // thread arrives there once per block too, after its first-half arrival).
     const int ptid = threadIdx.x;
     uint32_t it = 0;  // K-blocks handled by this CTA (stage ring position)
     bool stop = false;
@@ -226,17 +236,28 @@ __global__ void __launch_bounds__(320, 1)
         const int* idx_s = reinterpret_cast<const int*>(idx_region + s * C::kIdxBytes);
         if (run < 0) {
           if (sparse) {
-            Gather<C, kSparseBK> gs;
+            using G = Gather<C, kSparseBK>;
+            G gs;
             gs.load_index(idx_s, ptid);
-            gs.copy(B_s, a.X, a.N, n0, ptid);
+            if constexpr (C::kSplitB) {
+              gs.template copy<0, G::kPer / 2>(B_s, a.X, a.N, n0, ptid);
+              cp_async_arrive_noinc(full_bar(s));
+              gs.template copy<G::kPer / 2, G::kPer>(B_s, a.X, a.N, n0, ptid);
+              cp_async_arrive_noinc(full2_bar(s));
+            } else {
+              gs.copy(B_s, a.X, a.N, n0, ptid);
+              cp_async_arrive_noinc(full_bar(s));
+            }
           } else {
             Gather<C, kDenseBK> gd;
             gd.load_index(idx_s, ptid);
             gd.copy(B_s, a.X, a.N, n0, ptid);
+            cp_async_arrive_noinc(full_bar(s));
+            if constexpr (C::kSplitB) ptx::mbar_arrive(full2_bar(s));
           }
-          cp_async_arrive_noinc(full_bar(s));
         } else {
           ptx::mbar_arrive(full_bar(s));
+          if constexpr (C::kSplitB) ptx::mbar_arrive(full2_bar(s));
         }
       }
     }
@@ -279,9 +300,15 @@ __global__ void __launch_bounds__(320, 1)
           } else {
             ptx::mbar_arrive(idx_bar(s));
           }
+          // with kSplitB the full barrier takes A, metadata and the first 64 rows of X; the
+          // second-half barrier the rest of a run's rows (none for a dense block or a gather)
+          const int rows1 = C::kSplitB ? 64 : rows;
           const uint32_t bytes = C::kABytes + (sparse ? C::kEBytes : 0) +
-                                 (run >= 0 ? (uint32_t)rows * BN * 2u : 0u);
+                                 (run >= 0 ? (uint32_t)rows1 * BN * 2u : 0u);
           ptx::mbar_arrive_expect_tx(full_bar(s), bytes);
+          if constexpr (C::kSplitB)
+            ptx::mbar_arrive_expect_tx(full2_bar(s),
+                                       run >= 0 ? (uint32_t)(rows - rows1) * BN * 2u : 0u);
           ptx::bulk_g2s(A_s, (sparse ? a.vals_sparse : a.vals_dense) + blk * 8192, C::kABytes,
                         full_bar(s));
           if (sparse) ptx::bulk_g2s(E_s, a.meta + blk * kMetaWords, C::kEBytes, full_bar(s));
@@ -290,14 +317,15 @@ __global__ void __launch_bounds__(320, 1)
             // column atoms, or one 2-D box per atom
 #pragma unroll 1
             for (int h = 0; h < rows / 64; ++h) {
+              const uint32_t fb = (C::kSplitB && h == 1) ? full2_bar(s) : full_bar(s);
               if (a.x3d) {
                 ptx::tma_load_3d(B_s + h * C::kBHalfBytes, &tmX, 0, run + h * 64, n0 / C::kAtom,
-                                 full_bar(s));
+                                 fb);
               } else {
 #pragma unroll 1
                 for (int at = 0; at < BN / C::kAtom; ++at)
                   ptx::tma_load_2d(B_s + h * C::kBHalfBytes + at * C::kBAtomStride, &tmX,
-                                   n0 + at * C::kAtom, run + h * 64, full_bar(s));
+                                   n0 + at * C::kAtom, run + h * 64, fb);
               }
             }
           }
@@ -308,6 +336,8 @@ __global__ void __launch_bounds__(320, 1)
         for (uint32_t k = (it > (uint32_t)C::kStages ? it - C::kStages : 0u); k < it; ++k) {
           ptx::mbar_wait(idx_bar(k % C::kStages), (k / C::kStages) & 1, a.status, nullptr);
           ptx::mbar_wait(full_bar(k % C::kStages), (k / C::kStages) & 1, a.status, nullptr);
+          if constexpr (C::kSplitB)
+            ptx::mbar_wait(full2_bar(k % C::kStages), (k / C::kStages) & 1, a.status, nullptr);
         }
       }
     }
@@ -348,6 +378,14 @@ __global__ void __launch_bounds__(320, 1)
             ptx::tc_cp_128x128b(e_col, ptx::smem_desc(E_s, 2048, 128, 0));
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
+              if (C::kSplitB && k == 2) {  // rows 64..127 of B
+                if (!ptx::mbar_wait(full2_bar(s), ph, a.status, abort_flag)) {
+                  stop = true;
+                  break;
+                }
+                ptx::fence_proxy_async_smem();
+                ptx::tc_fence_after();
+              }
               const uint64_t ad = ptx::smem_desc(A_s + 32 * k, 16, 1024, 2);
               const uint64_t bd =
                   ptx::smem_desc(B_s + (k >> 1) * C::kBHalfBytes + 32 * (k & 1) * C::kAtomBytes,
@@ -355,6 +393,7 @@ __global__ void __launch_bounds__(320, 1)
               const uint32_t e = e_col + k;
               ptx::mma_sp_bf16(acc, ad, bd, e & ~1u, idesc_s | (e & 1u), (accum0 | k) ? 1u : 0u);
             }
+            if (stop) break;
           } else {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -362,6 +401,14 @@ __global__ void __launch_bounds__(320, 1)
               const uint64_t bd = ptx::smem_desc(B_s + 16 * k * C::kAtomBytes, C::kBAtomStride,
                                                  8 * C::kAtomBytes, C::kBLayout);
               ptx::mma_bf16(acc, ad, bd, idesc_d, (accum0 | k) ? 1u : 0u);
+            }
+            // a dense block has no second half: its barrier phase completes on the plain
+            // arrivals; waiting keeps every phase consumed before the stage is reused
+            if constexpr (C::kSplitB) {
+              if (!ptx::mbar_wait(full2_bar(s), ph, a.status, abort_flag)) {
+                stop = true;
+                break;
+              }
             }
           }
           ptx::tc_commit(empty_bar(s));
