@@ -6,9 +6,10 @@
 //   classify_kernel       one CTA per tile: region of every working position and the
 //                         2:4 members' input channels in ascending working position
 //                         (member[t][q])
-//   bitmask_kernel        one CTA per (tile, 16 rows): dense words by ballot over the
-//                         region, 2:4 groups top-2 of 4 per row, words assembled in shared
-//                         memory and written once, coalesced.
+//   bitmask_kernel        one CTA per (tile, RB <= 8 rows): the rows staged channel-major
+//                         in shared memory (16-byte quad loads), keep bytes (dense channels
+//                         all rows, 2:4 groups top-2 of 4 per row), then the bitmask words
+//                         assembled by warp ballots and written once, coalesced.
 #include <cuda_runtime.h>
 
 #include "hinm_internal.h"

@@ -4,20 +4,28 @@
 // The pages run two CUDA streams (mma and mma.sp) merged by atomicAdd.  Here a persistent
 // kernel (one CTA per SM) walks work units (tile, BN-column block); in each unit both kinds
 // of K-block accumulate into ONE tensor-memory accumulator, double-buffered so the
-// epilogue of a unit overlaps the main loop of the next.
+// epilogue of a unit overlaps the main loop of the next.  At narrow N, when the units fill
+// less than half of the SMs, a cluster of up to 8 CTAs shares each unit's K-blocks and the
+// leader adds the others' partial accumulators (received over DSMEM) in rank order.
 //
-//   warps 0-3  producers: per K-block, thread 0 bulk-copies the pre-swizzled 16 KB A block
-//              (and, for a 2:4 block, its 2 KB metadata); the X rows the block's index
-//              selects are copied by all 128 threads with 16-byte cp.async into the
-//              swizzled MN-major B tile (coalesced 2*BN-byte row segments), or, when the
-//              index is one contiguous run, by thread 0 as 2-D tiled TMA boxes.
+//   warps 0-3  gather producers: for a K-block whose index is not one contiguous run, the
+//              X rows it selects, 16-byte cp.async into the swizzled MN-major B tile
+//              (coalesced 2*BN-byte row segments); arrival on the stage's barrier when
+//              they land.
 //   warp 4     MMA: one thread; 2:4 block -> tcgen05.cp of the metadata into tensor memory,
 //              then 4 x tcgen05.mma.sp (K = 32 each); dense block -> 4 x tcgen05.mma
 //              (K = 16 each); tcgen05.commit frees the stage / publishes the accumulator.
-//   warps 5-8  epilogue: tcgen05.ld of the 128 x BN fp32 accumulator, stores to Y.
+//   warps 5-8  epilogue: tcgen05.ld of the 128 x BN fp32 accumulator, stores to Y (or, in
+//              a split-K cluster, to the leader's reduction buffer).
+//   warp 9     bulk copies: one thread runs ahead by up to a full ring; per K-block it
+//              publishes the block's run flag and index list and bulk-copies the
+//              pre-swizzled 16 KB A block, its 2 KB metadata and, for a contiguous run,
+//              the X rows as 3-D tiled TMA boxes (one per 64 K-rows).
 //
 // Shared memory holds STAGES stages of [A 16 KB | B 128 x BN bf16 | E 2 KB]; the stage ring
-// runs across work units.  Every wait is bounded (2 s), after which the CTA records
+// runs across work units.  At wide N the second 64 K-rows of a stage complete a barrier of
+// their own, so that the first two MMAs of a 2:4 block do not wait for them.  No load uses
+// cluster multicast.  Every wait is bounded (2 s), after which the CTA records
 // HINM_ERR_DEVICE_TIMEOUT, stops all roles, drains what it issued, frees tensor memory and
 // returns.
 #include <cuda.h>
