@@ -15,8 +15,10 @@
 //   warp 4     MMA: one thread; 2:4 block -> tcgen05.cp of the metadata into tensor memory,
 //              then 4 x tcgen05.mma.sp (K = 32 each); dense block -> 4 x tcgen05.mma
 //              (K = 16 each); tcgen05.commit frees the stage / publishes the accumulator.
-//   warps 5-8  epilogue: tcgen05.ld of the 128 x BN fp32 accumulator, stores to Y (or, in
-//              a split-K cluster, to the leader's reduction buffer).
+//   warps 5-8  epilogue: tcgen05.ld of the 128 x BN fp32 accumulator (a lane holds one
+//              row), 32 columns at a time transposed through a per-warp swizzled 4 KB
+//              shared tile so that each store instruction writes 128-byte row segments of
+//              four rows of Y (or, in a split-K cluster, to the leader's reduction buffer).
 //   warp 9     bulk copies: one thread runs ahead by up to a full ring; per K-block it
 //              publishes the block's run flag and index list and bulk-copies the
 //              pre-swizzled 16 KB A block, its 2 KB metadata and, for a contiguous run,
@@ -71,8 +73,11 @@ struct SpmmCfg {
   static constexpr int kTmemNeed = kAccBufs * kAccCols + 4 * kStages;
   static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                    : kTmemNeed <= 256 ? 256 : 512;
+  // persistent kernel with 32-column chunks: one 32 x 32 fp32 staging tile per epilogue
+  // warp, through which its lanes' accumulator rows become 128-byte row segments of Y
+  static constexpr int kEpiBytes = (SPLIT || BN < 32) ? 0 : 4 * 32 * 32 * 4;
   static constexpr size_t kSmemBytes = (size_t)kStages * (kStageBytes + kIdxBytes) +
-                                       1024 /*align*/ + 512 /*barriers*/ + kRedBytes;
+                                       1024 /*align*/ + 512 /*barriers*/ + kRedBytes + kEpiBytes;
   // wide N: the second 64 K-rows of a 2:4 block's B land on a barrier of their own, so the
   // MMAs on the first 64 rows start before the second half arrives
   static constexpr bool kSplitB = BN >= 128;
@@ -83,6 +88,7 @@ struct SpmmCfg {
   static_assert(BN == 16 || BN == 32 || (BN % 64 == 0 && BN <= 256), "BN");
   static_assert(kStages >= 2, "stages");
   static_assert(kTmemNeed <= 512, "tmem");
+  static_assert(kSmemBytes <= 232448, "shared memory");
   static_assert(!SPLIT || BN <= 32, "split-K is for narrow N");
 };
 
@@ -198,6 +204,8 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t meta_col0 = C::kAccBufs * C::kAccCols;
   float* red = reinterpret_cast<float*>(idx_region + C::kStages * C::kIdxBytes + 512);
+  // [4 warps][32 rows][8 x 16-byte pieces], piece p of row r at slot p ^ (r & 7)
+  uint8_t* epi_stage = reinterpret_cast<uint8_t*>(red) + C::kRedBytes;
   // Work: persistent CTAs stride over the units; split-K CTAs take one unit each and the
   // K-block range [kb0, kb1) of their cluster rank.
   const int u_first = SPLIT ? (int)blockIdx.x / a.split : (int)blockIdx.x;
@@ -474,6 +482,39 @@ __global__ void __launch_bounds__(320, 1)
                                  __uint_as_float(v[i + 1]), __uint_as_float(v[i + 2]),
                                  __uint_as_float(v[i + 3]));
           }
+        }
+      } else if constexpr (kChunk == 32) {
+        // Per 32-column chunk: lane l holds row q*32 + l of the accumulator; it writes the
+        // row into the warp's staging tile (16-byte pieces, slot = piece ^ (row & 7): no bank
+        // conflict either way), and reads back piece l % 8 of row 4 i + l / 8, so that each
+        // 16-byte store instruction writes 128 contiguous bytes of 4 rows of Y.
+        const uint32_t ep = ptx::smem_u32(epi_stage + (warp & 3) * 4096);
+        const int rr = lane >> 3, pc = lane & 7;
+        for (int col = 0; col < BN; col += 32) {
+          uint32_t v[32];
+          if (has) {
+            ptx::tmem_ld_32x32b_x32(
+                tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::kAccCols + col), v);
+            ptx::tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0u;
+          }
+#pragma unroll
+          for (int p = 0; p < 8; ++p)
+            ptx::st_shared_v4(ep + lane * 128 + ((p ^ (lane & 7)) << 4), v[4 * p], v[4 * p + 1],
+                              v[4 * p + 2], v[4 * p + 3]);
+          __syncwarp();
+          const int gc = n0 + col + 4 * pc;  // N % 8 == 0: a piece is wholly in or out
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = 4 * i + rr;  // row within the warp's quadrant
+            const uint4 o = ptx::ld_shared_v4(ep + r * 128 + ((pc ^ (r & 7)) << 4));
+            const int rw = q * 32 + r;
+            if (rw < a.T && gc < a.N)
+              *reinterpret_cast<uint4*>(a.Y + (size_t)(tile * a.T + rw) * a.N + gc) = o;
+          }
+          __syncwarp();  // the tile is rewritten by the next chunk
         }
       } else {
         const bool row_ok = row < a.T;

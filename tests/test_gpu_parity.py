@@ -222,6 +222,30 @@ def test_dense_ts0_matches_torch_matmul(H, M, K, N, perm):
     check_y(Y.cpu().numpy(), mm.astype(np.float64), bound)
 
 
+@pytest.mark.parametrize("M,K,N,T,v_s", [
+    (5120, 256, 2048, 128, 0.0),    # 320 units of 256 columns on at most 148 CTAs
+    (25600, 128, 16, 128, 0.25),    # 200 units of 16 columns, persistent (no split-K)
+    (20480, 128, 264, 64, 0.25),    # T = 64, 320 tiles x 2 column blocks, ragged N
+])
+def test_spmm_units_shared_across_ctas(H, M, K, N, T, v_s):
+    """More column blocks than SMs (several per persistent CTA, with a ragged last wave):
+    Y against the fp64 masked product (the GPU's mask, checked elsewhere), and bitwise the
+    same over two runs."""
+    w = hi.custom(M, K, N, T, seed=51, t_s=0.5, v_s=v_s, random_perm=True)
+    W, X, perm = dev_bf16(w.W_bits), dev_bf16(w.X_bits), dev_i32(w.perm)
+    nt = M // T
+    c = dev_i32(np.tile(np.array(H.hinm_counts_from_vs(K, 0.5, v_s), dtype=np.int32), (nt, 1)))
+    hp = H.HotPath(M, K, N, T, 0.5, w.alpha)
+    Y1 = hp.run(W, X, perm, fixed_counts=c).clone()
+    Y2 = hp.run(W, X, perm, fixed_counts=c).clone()
+    torch.cuda.synchronize()
+    status_ok(H)
+    np.testing.assert_array_equal(Y1.cpu().numpy().view(np.uint32), Y2.cpu().numpy().view(np.uint32))
+    bm = hp.bitmask.cpu().numpy().view(np.uint32)
+    y_ref, bound = O.spmm_reference(w.W_bits, bm, w.X_bits)
+    check_y(Y1.cpu().numpy(), y_ref, bound)
+
+
 def test_gpu_permutation_invariance(H):
     """Reordering input channels consistently leaves the GPU result unchanged (FlexHiNM-GP
     notes, 关键设计 2): run(W, X, pi) and run(W[:, pi], X[pi, :], identity) give the same
