@@ -214,6 +214,19 @@ hinm_status hinm_compress(const void* W, const uint32_t* bitmask, const int8_t* 
 hinm_status hinm_spmm(const hinm_layout* layout, const void* X, int N, float* Y_out,
                       void* stream);
 
+/* hinm_spmm with flags (0 = hinm_spmm).  Same arguments, layout, result and errors; an
+ * unknown flag bit returns HINM_ERR_INVALID_ARG.
+ *   HINM_SPMM_TILE_PAIRS: a performance hint from a caller that knows its tiles select the
+ *   same X rows, i.e. every tile has one region (all 2:4 or all dense) and the permutation
+ *   is ascending, so that every block of X is one run of rows.  With T == 128 and N >= 1024
+ *   the SpMM then takes tiles two at a time (2p, 2p+1) on 240-column blocks: where both
+ *   tiles' blocks are the same runs (checked on the device, pair by pair) one copy of each
+ *   X block feeds the tensor-core products of both.  A pair that differs runs tile by tile:
+ *   the result is the same, only slower.  Otherwise ignored. */
+#define HINM_SPMM_TILE_PAIRS 1
+hinm_status hinm_spmm_ex(const hinm_layout* layout, const void* X, int N, float* Y_out,
+                         int flags, void* stream);
+
 /* Diagnostic with no counterpart in the pages: launches one small kernel whose bounded
  * wait cannot complete (it waits on an mbarrier nothing arrives at), so that after about
  * limit_ns nanoseconds it records HINM_ERR_DEVICE_TIMEOUT and returns, exercising the

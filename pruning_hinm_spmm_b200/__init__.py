@@ -26,6 +26,7 @@ HINM_ERR_DEVICE_TIMEOUT = 6
 HINM_ERR_BAD_MASK = 7
 HINM_ERR_WORKSPACE = 8
 HINM_LAYOUT_VERSION = 2
+HINM_SPMM_TILE_PAIRS = 1   # hinm_spmm_ex flag
 
 REGION_PRUNED, REGION_24, REGION_DENSE = 0, 1, 2
 
@@ -75,6 +76,7 @@ _SIGS = {
     "hinm_compress": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
                              ctypes.POINTER(hinm_layout), _vp, _sz, _vp]),
     "hinm_spmm": (_i32, [ctypes.POINTER(hinm_layout), _vp, _i32, _vp, _vp]),
+    "hinm_spmm_ex": (_i32, [ctypes.POINTER(hinm_layout), _vp, _i32, _vp, _i32, _vp]),
     "hinm_device_status": (_i32, [_vp, ctypes.POINTER(ctypes.c_int32)]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -296,14 +298,21 @@ def hinm_compress(W, bitmask, region, perm, counts, T: int, layout: Optional[Hin
 
 
 # ----------------------------------------------------------------------------- a6
-def hinm_spmm(layout: HinmLayout, X, Y_out=None, stream=None, c_layout: Optional[hinm_layout] = None):
-    """Y (fp32 [M, N]) = W_HiNM . X (X bf16 [K, N])."""
+def hinm_spmm(layout: HinmLayout, X, Y_out=None, stream=None, c_layout: Optional[hinm_layout] = None,
+              tile_pairs: bool = False):
+    """Y (fp32 [M, N]) = W_HiNM . X (X bf16 [K, N]).  ``tile_pairs``: the caller knows every
+    tile selects the same X rows (HINM_SPMM_TILE_PAIRS; a hint, the result is the same)."""
     torch = _torch()
     N = X.shape[1]
     if Y_out is None:
         Y_out = torch.empty((layout.M, N), dtype=torch.float32, device=X.device)
     c = c_layout if c_layout is not None else layout.as_c()
-    _check(_lib.hinm_spmm(ctypes.byref(c), _ptr(X), N, _ptr(Y_out), _stream(stream)), "hinm_spmm")
+    if tile_pairs:
+        _check(_lib.hinm_spmm_ex(ctypes.byref(c), _ptr(X), N, _ptr(Y_out), HINM_SPMM_TILE_PAIRS,
+                                 _stream(stream)), "hinm_spmm_ex")
+    else:
+        _check(_lib.hinm_spmm(ctypes.byref(c), _ptr(X), N, _ptr(Y_out), _stream(stream)),
+               "hinm_spmm")
     return Y_out
 
 
@@ -311,6 +320,20 @@ def hinm_device_status(stream=None) -> int:
     out = ctypes.c_int32(0)
     _check(_lib.hinm_device_status(_stream(stream), ctypes.byref(out)), "hinm_device_status")
     return int(out.value)
+
+
+def tile_pairs_hint(counts, perm, K: int) -> bool:
+    """Whether hinm_spmm's ``tile_pairs`` hint holds for host-side counts (int32 [M/T, 3] or
+    one row for every tile) and permutation (int32 [K] or None = identity): every tile has
+    the same single region (all 2:4 or all dense) and the permutation is ascending, so every
+    block of X that a tile reads is the same run of rows in every tile."""
+    import numpy as np
+    c = np.asarray(counts, dtype=np.int64).reshape(-1, 3)
+    if not (c == c[0]).all():
+        return False
+    one_region = c[0, 1] == K or c[0, 2] == K
+    ascending = perm is None or bool(np.array_equal(np.asarray(perm), np.arange(K)))
+    return bool(one_region and ascending)
 
 
 # ----------------------------------------------------------------------------- whole path
@@ -337,9 +360,10 @@ class HotPath:
                  hinm_mask_workspace_size(M, K, T), hinm_compress_workspace_size(M, K, T))
         self.ws = _empty_bytes(ws, device)
 
-    def run(self, W, X, perm, fixed_counts=None, stream=None):
+    def run(self, W, X, perm, fixed_counts=None, stream=None, tile_pairs=False):
         """One pass of the path.  The search always runs (its ranking feeds the mask);
-        ``fixed_counts`` (int32 [M/T, 3]) replaces its counts when given."""
+        ``fixed_counts`` (int32 [M/T, 3]) replaces its counts when given; ``tile_pairs`` is
+        the SpMM hint (hinm_spmm)."""
         hinm_importance(W, X, self.I, self.ws, stream)
         hinm_boundary_search(self.I, perm, self.T, self.t_s, self.alpha, self.counts, self.vs,
                              self.rank, self.ws, stream=stream)
@@ -348,5 +372,5 @@ class HotPath:
                   stream)
         hinm_compress(W, self.bitmask, self.region, perm, counts, self.T, self.layout, self.ws,
                       stream)
-        hinm_spmm(self.layout, X, self.Y, stream, self.c_layout)
+        hinm_spmm(self.layout, X, self.Y, stream, self.c_layout, tile_pairs)
         return self.Y

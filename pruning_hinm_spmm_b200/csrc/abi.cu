@@ -429,6 +429,12 @@ hinm_status hinm_compress(const void* W, const uint32_t* bitmask, const int8_t* 
 
 hinm_status hinm_spmm(const hinm_layout* layout, const void* X, int N, float* Y_out,
                       void* stream) {
+  return hinm_spmm_ex(layout, X, N, Y_out, 0, stream);
+}
+
+hinm_status hinm_spmm_ex(const hinm_layout* layout, const void* X, int N, float* Y_out,
+                         int flags, void* stream) {
+  if (flags & ~HINM_SPMM_TILE_PAIRS) return fail(HINM_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   hinm_status st = check_layout(layout);
   if (st != HINM_OK) return st;
   REQUIRE_PTR(X);
@@ -436,6 +442,7 @@ hinm_status hinm_spmm(const hinm_layout* layout, const void* X, int N, float* Y_
   st = check_n(N);
   if (st != HINM_OK) return st;
   cudaError_t e = hinm::launch_spmm(*layout, static_cast<const uint16_t*>(X), N, Y_out,
+                                    (flags & HINM_SPMM_TILE_PAIRS) != 0,
                                     hinm::device_status_ptr(), static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "hinm_spmm launch");
   return ok();

@@ -81,8 +81,9 @@ cudaError_t launch_compress(const uint16_t* W, const uint32_t* bitmask, const in
 cudaError_t launch_wait_timeout_selftest(unsigned long long limit_ns, int* status,
                                          cudaStream_t s);
 
+// tile_pairs: the caller's hint that tiles select the same X rows (HINM_SPMM_TILE_PAIRS)
 cudaError_t launch_spmm(const hinm_layout& L, const uint16_t* X, int N, float* Y,
-                        int* status, cudaStream_t s);
+                        bool tile_pairs, int* status, cudaStream_t s);
 
 // Shared by the rank users (search and mask): V (fp64 column sums per tile) and the rank
 // of every working position.

@@ -24,6 +24,11 @@
 //              pre-swizzled 16 KB A block, its 2 KB metadata and, for a contiguous run,
 //              the X rows as 3-D tiled TMA boxes (one per 64 K-rows).
 //
+// spmm_pair_kernel (T = 128, wide N, on the caller's hint that tiles select the same X rows)
+// takes tile pairs x 240 columns with the same roles: where both tiles' blocks are the same
+// runs of X rows, one B stage feeds the MMAs of both tiles (two accumulators in tensor
+// memory), else the pair's tiles run one after the other.
+//
 // Shared memory holds STAGES stages of [A 16 KB | B 128 x BN bf16 | E 2 KB]; the stage ring
 // runs across work units.  At wide N the second 64 K-rows of a stage complete a barrier of
 // their own, so that the first two MMAs of a 2:4 block do not wait for them.  No load uses
@@ -614,6 +619,443 @@ __global__ void __launch_bounds__(320, 1)
   }
 }
 
+// ------------------------------------------------------------------ tile pairs
+// Wide N with T = 128: work units are (tile pair 2p, 2p+1; 240-column block).  When the two
+// tiles select the same X rows block by block (same block counts, and every block of both
+// is the same ascending run: no vector pruned, or every vector dense), one B stage feeds the
+// MMAs of both tiles, which halves the operand traffic that bounds the kernel.  Otherwise
+// the unit runs the two tiles one after the other.  Tile q of the pair always accumulates in
+// tensor-memory buffer q (2 x 240 columns + 16 metadata columns), so in a sequential unit the
+// epilogue of one tile overlaps the main loop of the next.  The B stage is 4 column atoms of
+// 64 (128-byte swizzle rows: full-width TMA rows, conflict-free gathers); a unit fills and
+// multiplies its first 240 columns.
+struct PairCfg {
+  static constexpr int BN = 240;
+  static constexpr int kAtom = 64;
+  static constexpr int kAtoms = 4;
+  static constexpr int kAtomBytes = 128;
+  static constexpr int kSwzBits = 3;
+  static constexpr int kChunksPerAtom = 8;
+  static constexpr int kChunksPerRow = BN / 8;  // the gather fills 240 columns
+  static constexpr int kBHalfBytes = 64 * kAtoms * kAtomBytes;
+  static constexpr int kBBytes = 2 * kBHalfBytes;
+  static constexpr int kBAtomStride = 64 * kAtomBytes;
+  static constexpr int kEBytes = 2048;
+  // stage: [A tile 0 | A tile 1 | B | E tile 0 | E tile 1]; a sequential unit uses the
+  // tile-0 slots for either tile
+  static constexpr int kAOff1 = kBlockBytes;
+  static constexpr int kBOff = 2 * kBlockBytes;
+  static constexpr int kEOff = kBOff + kBBytes;
+  static constexpr int kStageBytes = kEOff + 2 * kEBytes;
+  static constexpr int kIdxBytes = 512;
+  static constexpr int kStages = 2;
+  static constexpr uint32_t kBLayout = 2u;  // 128-byte swizzle
+  static constexpr int kAccCols = BN;
+  static constexpr int kMetaCol0 = 2 * BN;  // stage s, tile q: columns kMetaCol0 + 8 s + 4 q
+  static constexpr int kTmemCols = 512;
+  static constexpr int kEpiBytes = 4 * 32 * 32 * 4;
+  static constexpr size_t kSmemBytes =
+      (size_t)kStages * (kStageBytes + kIdxBytes) + 1024 /*align*/ + 512 /*barriers*/ + kEpiBytes;
+  static constexpr bool kSplitB = true;
+  static constexpr int kProducers = 128;
+  static constexpr int kMmaWarp = 4;
+  static constexpr int kBulkWarp = 9;
+  static constexpr int kThreads = 320;
+  static_assert(kStageBytes % 1024 == 0, "stage alignment");
+  static_assert(kMetaCol0 + 8 * kStages <= kTmemCols, "tmem");
+  static_assert(kSmemBytes <= 232448, "shared memory");
+};
+
+// Warp-collective (every lane calls it with the same p): whether tiles 2p and 2p+1 read the
+// same X rows block by block.  Gathered blocks (run -1) never count as shared.
+__device__ __forceinline__ bool pair_shares_b(const SpmmArgs& a, int p, int lane) {
+  const int t0 = 2 * p;
+  if (t0 + 1 >= a.num_tiles) return false;
+  const int4 i0 = __ldg(reinterpret_cast<const int4*>(a.tile_info) + t0);
+  const int4 i1 = __ldg(reinterpret_cast<const int4*>(a.tile_info) + t0 + 1);
+  if (i0.x != i1.x || i0.y != i1.y) return false;
+  bool ok = true;
+  for (int kb = lane; kb < i0.x + i0.y; kb += 32) {
+    const bool sp = kb >= i0.x;
+    const int r0 = sp ? __ldg(a.run_sparse + i0.w + kb - i0.x) : __ldg(a.run_dense + i0.z + kb);
+    const int r1 = sp ? __ldg(a.run_sparse + i1.w + kb - i1.x) : __ldg(a.run_dense + i1.z + kb);
+    ok = ok && r0 >= 0 && r0 == r1;
+  }
+  return __all_sync(0xffffffffu, ok);
+}
+
+// tmX3: X as (column, row, atom) with the atom stride 128 bytes inside a row, so that one
+// box at column n0 covers columns n0 .. n0+255 of 64 rows (used while n0 + 256 <= N: every
+// address stays in its row); tmX2: X as (column, row) with boxes of 64 x 64 (columns past N
+// read as zeros), used for the last column block.
+__global__ void __launch_bounds__(320, 1)
+    spmm_pair_kernel(const __grid_constant__ CUtensorMap tmX3,
+                     const __grid_constant__ CUtensorMap tmX2, const SpmmArgs a) {
+  using C = PairCfg;
+  constexpr int BN = C::BN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* idx_region = smem + C::kStages * C::kStageBytes;  // [S][kIdxBytes]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(idx_region + C::kStages * C::kIdxBytes);
+  // [0,S) full, [S,2S) empty, 2S+{0,1} accumulator full, 2S+{2,3} accumulator empty,
+  // 2S+4 drain, [2S+5, 3S+5) index ready, [3S+5, 4S+5) second-half full; then the TMEM
+  // address, the abort flag and one run flag per stage
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 * C::kStages + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* run_s = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  uint8_t* epi_stage = reinterpret_cast<uint8_t*>(bars) + 512;  // [4 warps][4 KB]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto full_bar = [&](int s) { return ptx::smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return ptx::smem_u32(bars + C::kStages + s); };
+  auto accf_bar = [&](int b) { return ptx::smem_u32(bars + 2 * C::kStages + b); };
+  auto acce_bar = [&](int b) { return ptx::smem_u32(bars + 2 * C::kStages + 2 + b); };
+  const uint32_t drain_bar = ptx::smem_u32(bars + 2 * C::kStages + 4);
+  auto idx_bar = [&](int s) { return ptx::smem_u32(bars + 2 * C::kStages + 5 + s); };
+  auto full2_bar = [&](int s) { return ptx::smem_u32(bars + 3 * C::kStages + 5 + s); };
+  auto info_of = [&](int t) { return __ldg(reinterpret_cast<const int4*>(a.tile_info) + t); };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      ptx::mbar_init(full_bar(s), 1 + C::kProducers);
+      ptx::mbar_init(empty_bar(s), 1);
+      ptx::mbar_init(idx_bar(s), 1);
+      ptx::mbar_init(full2_bar(s), 1 + C::kProducers);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(accf_bar(b), 1);
+      ptx::mbar_init(acce_bar(b), 4);
+    }
+    ptx::mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == C::kMmaWarp) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), C::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int pairs_last = a.num_tiles - 1;  // tile 2p + 1 exists iff 2p + 1 <= pairs_last
+
+  if (warp < 4) {
+    // ------------------------------------------------------------ gather producers
+    // As in spmm_kernel; every stop is warp-uniform (vote after each wait), because the
+    // next unit starts with a warp-collective test.
+    const int ptid = threadIdx.x;
+    uint32_t it = 0;
+    bool stop = false;
+    for (int u = blockIdx.x; u < a.num_units && !stop; u += gridDim.x) {
+      const int p = u / a.nblk_n, n0 = (u - p * a.nblk_n) * BN;
+      const bool pm = pair_shares_b(a, p, lane);
+      const int nq = pm ? 1 : (2 * p + 1 <= pairs_last ? 2 : 1);
+      for (int q = 0; q < nq && !stop; ++q) {
+        const int4 info = info_of(2 * p + q);
+        const int nd = info.x, nblk = info.x + info.y;
+        for (int kb = 0; kb < nblk; ++kb, ++it) {
+          const bool sparse = kb >= nd;
+          const int s = it % C::kStages;
+          const uint32_t ph = (it / C::kStages) & 1;
+          const bool ok = ptx::mbar_wait(idx_bar(s), ph, a.status, abort_flag);
+          if (!__all_sync(0xffffffffu, ok)) {
+            stop = true;
+            break;
+          }
+          const int run = run_s[s];
+          const uint32_t B_s = ptx::smem_u32(smem + s * C::kStageBytes + C::kBOff);
+          const int* idx_s = reinterpret_cast<const int*>(idx_region + s * C::kIdxBytes);
+          if (run < 0) {
+            if (sparse) {
+              using G = Gather<C, kSparseBK>;
+              G gs;
+              gs.load_index(idx_s, ptid);
+              gs.template copy<0, G::kPer / 2>(B_s, a.X, a.N, n0, ptid);
+              cp_async_arrive_noinc(full_bar(s));
+              gs.template copy<G::kPer / 2, G::kPer>(B_s, a.X, a.N, n0, ptid);
+              cp_async_arrive_noinc(full2_bar(s));
+            } else {
+              Gather<C, kDenseBK> gd;
+              gd.load_index(idx_s, ptid);
+              gd.copy(B_s, a.X, a.N, n0, ptid);
+              cp_async_arrive_noinc(full_bar(s));
+              ptx::mbar_arrive(full2_bar(s));
+            }
+          } else {
+            ptx::mbar_arrive(full_bar(s));
+            ptx::mbar_arrive(full2_bar(s));
+          }
+        }
+      }
+    }
+    cp_async_wait_all();
+  } else if (warp == C::kBulkWarp) {
+    // ------------------------------------------------------------ bulk copies
+    uint32_t it = 0;
+    bool stop = false;
+    for (int u = blockIdx.x; u < a.num_units && !stop; u += gridDim.x) {
+      const int p = u / a.nblk_n, n0 = (u - p * a.nblk_n) * BN;
+      const bool pm = pair_shares_b(a, p, lane);
+      if (lane == 0) {
+        const int nq = pm ? 1 : (2 * p + 1 <= pairs_last ? 2 : 1);
+        for (int q = 0; q < nq && !stop; ++q) {
+          const int4 info = info_of(2 * p + q);
+          const int4 info1 = pm ? info_of(2 * p + 1) : info;
+          const int nd = info.x, nblk = info.x + info.y;
+          for (int kb = 0; kb < nblk; ++kb, ++it) {
+            const bool sparse = kb >= nd;
+            const size_t blk = sparse ? (size_t)(info.w + kb - nd) : (size_t)(info.z + kb);
+            const size_t blk1 = sparse ? (size_t)(info1.w + kb - nd) : (size_t)(info1.z + kb);
+            const int run = __ldg(sparse ? a.run_sparse + blk : a.run_dense + blk);
+            const int s = it % C::kStages;
+            const uint32_t ph = (it / C::kStages) & 1;
+            if (!ptx::mbar_wait(empty_bar(s), ph ^ 1, a.status, abort_flag)) {
+              stop = true;
+              break;
+            }
+            const uint32_t A_s = ptx::smem_u32(smem + s * C::kStageBytes);
+            const uint32_t B_s = A_s + C::kBOff;
+            const uint32_t E_s = A_s + C::kEOff;
+            const uint32_t I_s = ptx::smem_u32(idx_region + s * C::kIdxBytes);
+            const int rows = sparse ? kSparseBK : kDenseBK;
+            run_s[s] = run;  // published by the arrive below (release)
+            if (run < 0) {
+              ptx::mbar_arrive_expect_tx(idx_bar(s), (uint32_t)rows * 4u);
+              ptx::bulk_g2s(I_s,
+                            sparse ? a.idx_sparse + blk * kSparseBK : a.idx_dense + blk * kDenseBK,
+                            (uint32_t)rows * 4u, idx_bar(s));
+            } else {
+              ptx::mbar_arrive(idx_bar(s));
+            }
+            // the full barrier takes A (both tiles' in a shared unit), the metadata and the
+            // first 64 rows of a run; the second-half barrier the rest of the run
+            const uint32_t na = pm ? 2u : 1u;
+            const uint32_t bytes = na * (kBlockBytes + (sparse ? C::kEBytes : 0)) +
+                                   (run >= 0 ? (uint32_t)C::kBHalfBytes : 0u);
+            ptx::mbar_arrive_expect_tx(full_bar(s), bytes);
+            ptx::mbar_arrive_expect_tx(full2_bar(s),
+                                       run >= 0 && rows > 64 ? (uint32_t)C::kBHalfBytes : 0u);
+            const uint16_t* vals = sparse ? a.vals_sparse : a.vals_dense;
+            ptx::bulk_g2s(A_s, vals + blk * 8192, kBlockBytes, full_bar(s));
+            if (pm) ptx::bulk_g2s(A_s + C::kAOff1, vals + blk1 * 8192, kBlockBytes, full_bar(s));
+            if (sparse) {
+              ptx::bulk_g2s(E_s, a.meta + blk * kMetaWords, C::kEBytes, full_bar(s));
+              if (pm)
+                ptx::bulk_g2s(E_s + C::kEBytes, a.meta + blk1 * kMetaWords, C::kEBytes,
+                              full_bar(s));
+            }
+            if (run >= 0) {
+#pragma unroll 1
+              for (int h = 0; h < rows / 64; ++h) {
+                const uint32_t fb = h == 1 ? full2_bar(s) : full_bar(s);
+                if (a.x3d && n0 + C::kAtoms * C::kAtom <= a.N) {
+                  ptx::tma_load_3d(B_s + h * C::kBHalfBytes, &tmX3, n0, run + h * 64, 0, fb);
+                } else {
+#pragma unroll 1
+                  for (int at = 0; at < C::kAtoms; ++at)
+                    ptx::tma_load_2d(B_s + h * C::kBHalfBytes + at * C::kBAtomStride, &tmX2,
+                                     n0 + at * C::kAtom, run + h * 64, fb);
+                }
+              }
+            }
+          }
+        }
+      }
+      stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
+    }
+    if (lane == 0 && *abort_flag) {
+      // wait (bounded) for the bulk / tensor copies of the last stages
+      for (uint32_t k = (it > (uint32_t)C::kStages ? it - C::kStages : 0u); k < it; ++k) {
+        ptx::mbar_wait(idx_bar(k % C::kStages), (k / C::kStages) & 1, a.status, nullptr);
+        ptx::mbar_wait(full_bar(k % C::kStages), (k / C::kStages) & 1, a.status, nullptr);
+        ptx::mbar_wait(full2_bar(k % C::kStages), (k / C::kStages) & 1, a.status, nullptr);
+      }
+    }
+    __syncwarp();
+  } else if (warp == C::kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    uint32_t it = 0, lu0 = 0, lu1 = 0;
+    bool stop = false;
+    for (int u = blockIdx.x; u < a.num_units && !stop; u += gridDim.x) {
+      const int p = u / a.nblk_n, n0 = (u - p * a.nblk_n) * BN;
+      const bool pm = pair_shares_b(a, p, lane);
+      if (lane == 0) {
+        const int w = a.N - n0 < BN ? a.N - n0 : BN;
+        const int nmma = (w + 15) & ~15;  // MMA width: the unit's columns, rounded up to 16
+        const uint32_t idesc_d = ptx::idesc_bf16(nmma, 1, 0);
+        const uint32_t idesc_s = ptx::idesc_bf16(nmma, 1, 1);
+        const int nq = pm ? 1 : (2 * p + 1 <= pairs_last ? 2 : 1);
+        for (int q = 0; q < nq && !stop; ++q) {
+          // buffers this pass writes: both in a shared unit, else buffer q
+          if (pm || q == 0) {
+            if (!ptx::mbar_wait(acce_bar(0), (lu0 & 1) ^ 1, a.status, abort_flag)) {
+              stop = true;
+              break;
+            }
+          }
+          if (pm || q == 1) {
+            if (!ptx::mbar_wait(acce_bar(1), (lu1 & 1) ^ 1, a.status, abort_flag)) {
+              stop = true;
+              break;
+            }
+          }
+          ptx::tc_fence_after();
+          const uint32_t acc0 = tmem + (uint32_t)(q * C::kAccCols);  // this pass's tile
+          const uint32_t acc1 = tmem + (uint32_t)C::kAccCols;        // tile 1 of a shared unit
+          const int4 info = info_of(2 * p + q);
+          const int nd = info.x, nblk = info.x + info.y;
+          for (int kb = 0; kb < nblk; ++kb, ++it) {
+            const int s = it % C::kStages;
+            const uint32_t ph = (it / C::kStages) & 1;
+            const uint32_t accum0 = kb != 0 ? 1u : 0u;  // first K-block overwrites
+            if (!ptx::mbar_wait(full_bar(s), ph, a.status, abort_flag)) {
+              stop = true;
+              break;
+            }
+            ptx::fence_proxy_async_smem();  // cp.async (generic proxy) -> tensor-core reads
+            ptx::tc_fence_after();
+            const uint32_t A_s = ptx::smem_u32(smem + s * C::kStageBytes);
+            const uint32_t B_s = A_s + C::kBOff;
+            const uint32_t E_s = A_s + C::kEOff;
+            if (kb >= nd) {
+              const uint32_t e0 = tmem + (uint32_t)(C::kMetaCol0 + 8 * s);
+              const uint32_t e1 = e0 + 4;
+              ptx::tc_cp_128x128b(e0, ptx::smem_desc(E_s, 2048, 128, 0));
+              if (pm) ptx::tc_cp_128x128b(e1, ptx::smem_desc(E_s + C::kEBytes, 2048, 128, 0));
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                if (k == 2) {  // rows 64..127 of B
+                  if (!ptx::mbar_wait(full2_bar(s), ph, a.status, abort_flag)) {
+                    stop = true;
+                    break;
+                  }
+                  ptx::fence_proxy_async_smem();
+                  ptx::tc_fence_after();
+                }
+                const uint64_t bd =
+                    ptx::smem_desc(B_s + (k >> 1) * C::kBHalfBytes + 32 * (k & 1) * C::kAtomBytes,
+                                   C::kBAtomStride, 8 * C::kAtomBytes, C::kBLayout);
+                const uint32_t acc_on = (accum0 | k) ? 1u : 0u;
+                const uint32_t f0 = e0 + k;
+                ptx::mma_sp_bf16(acc0, ptx::smem_desc(A_s + 32 * k, 16, 1024, 2), bd, f0 & ~1u,
+                                 idesc_s | (f0 & 1u), acc_on);
+                if (pm) {
+                  const uint32_t f1 = e1 + k;
+                  ptx::mma_sp_bf16(acc1, ptx::smem_desc(A_s + C::kAOff1 + 32 * k, 16, 1024, 2),
+                                   bd, f1 & ~1u, idesc_s | (f1 & 1u), acc_on);
+                }
+              }
+              if (stop) break;
+            } else {
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const uint64_t bd = ptx::smem_desc(B_s + 16 * k * C::kAtomBytes, C::kBAtomStride,
+                                                   8 * C::kAtomBytes, C::kBLayout);
+                const uint32_t acc_on = (accum0 | k) ? 1u : 0u;
+                ptx::mma_bf16(acc0, ptx::smem_desc(A_s + 32 * k, 16, 1024, 2), bd, idesc_d,
+                              acc_on);
+                if (pm)
+                  ptx::mma_bf16(acc1, ptx::smem_desc(A_s + C::kAOff1 + 32 * k, 16, 1024, 2), bd,
+                                idesc_d, acc_on);
+              }
+              // a dense block has no second half: its barrier phase completes on the plain
+              // arrivals; waiting keeps every phase consumed before the stage is reused
+              if (!ptx::mbar_wait(full2_bar(s), ph, a.status, abort_flag)) {
+                stop = true;
+                break;
+              }
+            }
+            ptx::tc_commit(empty_bar(s));
+          }
+          if (stop) break;
+          // accumulator(s) ready (immediately if the tile has no K-blocks)
+          if (pm || q == 0) {
+            ptx::tc_commit(accf_bar(0));
+            ++lu0;
+          }
+          if (pm || q == 1) {
+            ptx::tc_commit(accf_bar(1));
+            ++lu1;
+          }
+        }
+      }
+      stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
+    }
+    if (lane == 0) {
+      // every tcgen05 operation issued above has completed once drain_bar flips
+      ptx::tc_commit(drain_bar);
+      ptx::mbar_wait(drain_bar, 0, a.status, nullptr);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 5..8)
+    // Tile q of each unit from buffer q; per 32-column chunk the lanes' accumulator rows go
+    // through the warp's swizzled shared tile and out as 128-byte row segments of Y.
+    const int qd = warp & 3;  // tensor-memory lane quadrant this warp may access
+    const uint32_t ep = ptx::smem_u32(epi_stage + qd * 4096);
+    const int rr = lane >> 3, pc = lane & 7;
+    uint32_t lu[2] = {0u, 0u};
+    bool stop = false;
+    for (int u = blockIdx.x; u < a.num_units && !stop; u += gridDim.x) {
+      const int p = u / a.nblk_n, n0 = (u - p * a.nblk_n) * BN;
+      const int w = a.N - n0 < BN ? a.N - n0 : BN;
+      const int nq = 2 * p + 1 <= pairs_last ? 2 : 1;
+      for (int q = 0; q < nq; ++q) {
+        const int tile = 2 * p + q;
+        const int4 info = info_of(tile);
+        const bool has = info.x + info.y > 0;  // else the accumulator was never written
+        const bool ok = ptx::mbar_wait(accf_bar(q), lu[q] & 1, a.status, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) {
+          stop = true;
+          break;
+        }
+        ++lu[q];
+        ptx::tc_fence_after();
+        for (int col = 0; col < w; col += 32) {
+          const int cw = w - col < 32 ? w - col : 32;  // a multiple of 8
+          uint32_t v[32];
+          if (has) {
+            const uint32_t taddr =
+                tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(q * C::kAccCols + col);
+            if (cw > 16) ptx::tmem_ld_32x32b_x32(taddr, v);
+            else ptx::tmem_ld_32x32b_x16(taddr, v);
+            ptx::tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0u;
+          }
+#pragma unroll
+          for (int pp = 0; pp < 8; ++pp)
+            ptx::st_shared_v4(ep + lane * 128 + ((pp ^ (lane & 7)) << 4), v[4 * pp],
+                              v[4 * pp + 1], v[4 * pp + 2], v[4 * pp + 3]);
+          __syncwarp();
+          const int gc = n0 + col + 4 * pc;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = 4 * i + rr;  // row within the warp's quadrant
+            const uint4 o = ptx::ld_shared_v4(ep + r * 128 + ((pc ^ (r & 7)) << 4));
+            const int rw = qd * 32 + r;
+            if (4 * pc < cw && rw < a.T)
+              *reinterpret_cast<uint4*>(a.Y + (size_t)(tile * a.T + rw) * a.N + gc) = o;
+          }
+          __syncwarp();  // the tile is rewritten by the next chunk
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(acce_bar(q));  // buffer q may be overwritten
+      }
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == C::kMmaWarp) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
 // ------------------------------------------------------------------ host side
 namespace {
 
@@ -631,11 +1073,27 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// X (K rows x N bf16, row-major) as a tensor map swizzled like the B operand (atom * 2
-// bytes per swizzle row).  With 64-column atoms and N a multiple of 64 it is 3-D
+// X (K rows x N bf16, row-major) as a 2-D tensor map swizzled like the B operand (atom * 2
+// bytes per swizzle row), box 64 rows x `atom` columns; columns past N read as zeros.
+bool make_x_map_2d(CUtensorMap* m, const uint16_t* X, int K, int N, int atom) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)K};
+  cuuint64_t strides[1] = {(cuuint64_t)N * 2};
+  cuuint32_t box[2] = {(cuuint32_t)atom, (cuuint32_t)(K < 64 ? K : 64)};
+  cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw = atom == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : atom == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                             : CU_TENSOR_MAP_SWIZZLE_32B;
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// The tensor map of spmm_kernel.  With 64-column atoms and N a multiple of 64 it is 3-D
 // (column within the atom, row, atom; the atom stride is 128 bytes) with a box of all the
-// unit's atoms for 64 rows, so one load fills a half of the B tile; else 2-D with a box of
-// 64 rows x `atom` columns.
+// unit's atoms for 64 rows, so one load fills a half of the B tile; else the 2-D map.
 bool make_x_map(CUtensorMap* m, const uint16_t* X, int K, int N, int atom, int atoms, bool* x3d) {
   auto fn = encode_fn();
   if (!fn) return false;
@@ -653,17 +1111,23 @@ bool make_x_map(CUtensorMap* m, const uint16_t* X, int K, int N, int atom, int a
       return true;
     }
   }
-  cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)K};
-  cuuint64_t strides[1] = {(cuuint64_t)N * 2};
-  cuuint32_t box[2] = {(cuuint32_t)atom, (cuuint32_t)(K < 64 ? K : 64)};
-  cuuint32_t estr[2] = {1, 1};
-  const CUtensorMapSwizzle sw = atom == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
-                                : atom == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                             : CU_TENSOR_MAP_SWIZZLE_32B;
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return make_x_map_2d(m, X, K, N, atom);
+}
+
+// X as (column, row, atom): dims {N, K, atoms}, the atom stride `atom` columns within the
+// row, so that a box of {atom, 64, atoms} at column n0 reads columns n0 .. n0 + atom*atoms - 1
+// of 64 rows.  Columns are bounds-checked only against N along the first dimension: the
+// caller uses it only for boxes with n0 + atom*atoms <= N.  false if the driver refuses it.
+bool make_x_row_atoms_map(CUtensorMap* m, const uint16_t* X, int K, int N, int atom, int atoms) {
+  auto fn = encode_fn();
+  if (!fn || K < 64 || N < atom * atoms) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)K, (cuuint64_t)atoms};
+  cuuint64_t strides[2] = {(cuuint64_t)N * 2, (cuuint64_t)atom * 2};
+  cuuint32_t box[3] = {(cuuint32_t)atom, 64, (cuuint32_t)atoms};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(X), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int num_sms() {
@@ -715,6 +1179,27 @@ cudaError_t run(const hinm_layout& L, const uint16_t* X, int N, float* Y, int sp
   }
 }
 
+// Tile pairs x 240-column blocks (T = 128, wide N).
+constexpr int kPairMinN = 1024;
+cudaError_t run_pair(const hinm_layout& L, const uint16_t* X, int N, float* Y, int* status,
+                     cudaStream_t s) {
+  using C = PairCfg;
+  cudaError_t attr_err = set_max_dynamic_smem((const void*)spmm_pair_kernel, (int)C::kSmemBytes);
+  if (attr_err != cudaSuccess) return attr_err;
+  CUtensorMap map3, map2;
+  if (!make_x_map_2d(&map2, X, L.K, N, C::kAtom)) return cudaErrorInvalidValue;
+  const bool x3d = make_x_row_atoms_map(&map3, X, L.K, N, C::kAtom, C::kAtoms);
+  if (!x3d) map3 = map2;
+  const int nblk_n = (N + C::BN - 1) / C::BN;
+  const int units = (L.num_tiles + 1) / 2 * nblk_n;
+  SpmmArgs a{L.tile_info, L.vals_dense, L.vals_sparse, L.meta,   L.idx_dense, L.idx_sparse,
+             L.run_dense, L.run_sparse, X,             Y,        N,           L.T,
+             L.num_tiles, nblk_n,       units,         1,        x3d ? 1 : 0, status};
+  const int grid = units < num_sms() ? units : num_sms();
+  spmm_pair_kernel<<<grid, C::kThreads, C::kSmemBytes, s>>>(map3, map2, a);
+  return cudaGetLastError();
+}
+
 // Split-K when the units (tile x column block) fill less than half of the SMs: each unit's
 // K-blocks are shared by a cluster of up to kMaxSplit CTAs.
 template <int BN>
@@ -731,12 +1216,13 @@ cudaError_t run_auto(const hinm_layout& L, const uint16_t* X, int N, float* Y, i
 
 }  // namespace
 
-cudaError_t launch_spmm(const hinm_layout& L, const uint16_t* X, int N, float* Y, int* status,
-                        cudaStream_t s) {
+cudaError_t launch_spmm(const hinm_layout& L, const uint16_t* X, int N, float* Y,
+                        bool tile_pairs, int* status, cudaStream_t s) {
   if (N <= 16) return run_auto<16>(L, X, N, Y, status, s);
   if (N <= 32) return run_auto<32>(L, X, N, Y, status, s);
   if (N <= 64) return run_auto<64>(L, X, N, Y, status, s);
   if (N < 256) return run_auto<128>(L, X, N, Y, status, s);
+  if (tile_pairs && L.T == 128 && N >= kPairMinN) return run_pair(L, X, N, Y, status, s);
   return run_auto<256>(L, X, N, Y, status, s);
 }
 

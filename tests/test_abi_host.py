@@ -113,7 +113,29 @@ def test_validation_rejects_before_launch(H):
     L = H.hinm_layout(H.HINM_LAYOUT_VERSION, 256, 256, 64, 4, 1, 1, fake, fake, fake, fake, fake, fake, fake, fake)
     assert lib.hinm_spmm(ctypes.byref(L), fake, 20, fake, None) == H.HINM_ERR_SHAPE
     assert lib.hinm_spmm(ctypes.byref(L), fake + 8, 16, fake, None) == H.HINM_ERR_ALIGNMENT
+    # hinm_spmm_ex: unknown flag bits are refused before anything else; the hint flag
+    # passes the same argument checks as hinm_spmm
+    assert lib.hinm_spmm_ex(ctypes.byref(L), fake, 16, fake, 2, None) == H.HINM_ERR_INVALID_ARG
+    assert lib.hinm_spmm_ex(ctypes.byref(L), fake, 20, fake, H.HINM_SPMM_TILE_PAIRS,
+                            None) == H.HINM_ERR_SHAPE
+    assert lib.hinm_spmm_ex(ctypes.byref(L), fake + 8, 16, fake, H.HINM_SPMM_TILE_PAIRS,
+                            None) == H.HINM_ERR_ALIGNMENT
     # compress size rejects inconsistent counts
     bad = (ctypes.c_int32 * 3)(10, 11, 235)
     out = H.hinm_layout_sizes()
     assert lib.hinm_compress_size(bad, 64, 256, 64, ctypes.byref(out)) == H.HINM_ERR_INVALID_ARG
+
+
+def test_tile_pairs_hint_rule():
+    """The host rule behind the SpMM's tile-pair hint: one shared single region (all 2:4 or
+    all dense) in every tile and an ascending permutation; anything else gives no hint."""
+    import numpy as np
+    import pruning_hinm_spmm_b200 as H
+    K = 256
+    assert H.tile_pairs_hint([0, K, 0], None, K)                       # all 2:4
+    assert H.tile_pairs_hint([[0, 0, K]] * 4, np.arange(K), K)         # all dense
+    assert not H.tile_pairs_hint([64, 128, 64], None, K)               # HiNM regions
+    assert not H.tile_pairs_hint([0, K, 0], np.arange(K)[::-1], K)     # permuted X rows
+    assert not H.tile_pairs_hint([[0, K, 0], [0, 0, K]], None, K)      # tiles differ
+    assert H.tile_pairs_hint(H.hinm_counts_from_vs(K, 0.5, 0.0), None, K)
+    assert not H.tile_pairs_hint(H.hinm_counts_from_vs(K, 0.5, 0.25), None, K)

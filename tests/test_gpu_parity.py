@@ -161,6 +161,41 @@ def test_integer_product_bitwise(H, T, N, perm):
     assert np.array_equal(g["Y"], np.round(g["Y"]))
 
 
+@pytest.mark.parametrize("ntiles,N", [(7, 1032), (9, 1040), (6, 2048)])
+def test_tile_pairs_mixed_modes_integer_bitwise(H, ntiles, N):
+    """Wide N, T = 128: the SpMM's work units are tile pairs.  Per-tile counts make some
+    pairs select the same X rows block by block (both all 2:4, or both all dense: one B
+    stage feeds both tiles) and others not (HiNM counts with gathered blocks, or different
+    counts: the tiles run in sequence), with an odd tile count (a lone last tile), N not a
+    multiple of 240 (a ragged last column block) and N % 16 == 8 (column boxes of 16).
+    Integer inputs: Y must equal the masked product exactly."""
+    T, K = 128, 384
+    w = hi.integer_workload(ntiles * T, K, N, T, seed=12, t_s=0.5, v_s=None)
+    all24 = list(H.hinm_counts_from_vs(K, 0.5, 0.0))
+    hinm = list(H.hinm_counts_from_vs(K, 0.5, 0.25))
+    dense = [K, 0, 0]
+    pattern = [all24, all24, dense, dense, hinm, hinm, all24, dense, all24]
+    counts = np.array([pattern[t % len(pattern)] for t in range(ntiles)], dtype=np.int32)
+    W, X, perm = dev_bf16(w.W_bits), dev_bf16(w.X_bits), dev_i32(w.perm)
+    I = H.hinm_importance(W, X)
+    _, _, rank = H.hinm_boundary_search(I, perm, T, w.t_s, w.alpha)
+    c = dev_i32(counts)
+    bm, region = H.hinm_mask(I, perm, c, T, rank)
+    L = H.hinm_compress(W, bm, region, perm, c, T)
+    Y = H.hinm_spmm(L, X, tile_pairs=True)   # pairs where they share, tile by tile elsewhere
+    Y0 = H.hinm_spmm(L, X)                   # no hint: one tile per work unit
+    torch.cuda.synchronize()
+    status_ok(H)
+    run_d, run_s = L.run_dense.cpu().numpy(), L.run_sparse.cpu().numpy()
+    info = L.tile_info.cpu().numpy()
+    assert (run_s[info[0, 3]:info[0, 3] + info[0, 1]] >= 0).all()  # pair 0 shares its B
+    assert (run_d[info[4, 2]:info[4, 2] + info[4, 0]] < 0).any()   # pair 2 gathers
+    Wm = O.masked_weight(w.W_bits, bm.cpu().numpy().view(np.uint32)).astype(np.int64)
+    Xi = hi.bf16_bits_to_f32(w.X_bits).astype(np.int64)
+    np.testing.assert_array_equal(Y.cpu().numpy().astype(np.int64), Wm @ Xi)
+    np.testing.assert_array_equal(Y0.cpu().numpy().astype(np.int64), Wm @ Xi)
+
+
 def test_channel_energy_rounding_fallback(H):
     """Channels whose fp64 sum sits on an fp32 rounding midpoint: the order matters there,
     so the GPU must reproduce the sequential sum (1 first: 1.0; 1 last: 1 + 2^-23)."""
@@ -222,22 +257,25 @@ def test_dense_ts0_matches_torch_matmul(H, M, K, N, perm):
     check_y(Y.cpu().numpy(), mm.astype(np.float64), bound)
 
 
-@pytest.mark.parametrize("M,K,N,T,v_s", [
-    (5120, 256, 2048, 128, 0.0),    # 320 units of 256 columns on at most 148 CTAs
-    (25600, 128, 16, 128, 0.25),    # 200 units of 16 columns, persistent (no split-K)
-    (20480, 128, 264, 64, 0.25),    # T = 64, 320 tiles x 2 column blocks, ragged N
+@pytest.mark.parametrize("M,K,N,T,v_s,rperm", [
+    (5120, 256, 2048, 128, 0.0, True),    # 20 tile pairs x 9 column blocks, gathered X rows
+    (5120, 256, 2048, 128, 0.0, False),   # the same with every pair sharing its B stages
+    (25600, 128, 16, 128, 0.25, True),    # 200 units of 16 columns, persistent (no split-K)
+    (20480, 128, 264, 64, 0.25, True),    # T = 64, 320 tiles x 2 column blocks, ragged N
 ])
-def test_spmm_units_shared_across_ctas(H, M, K, N, T, v_s):
-    """More column blocks than SMs (several per persistent CTA, with a ragged last wave):
+def test_spmm_units_shared_across_ctas(H, M, K, N, T, v_s, rperm):
+    """More work units than SMs (several per persistent CTA, with a ragged last wave):
     Y against the fp64 masked product (the GPU's mask, checked elsewhere), and bitwise the
     same over two runs."""
-    w = hi.custom(M, K, N, T, seed=51, t_s=0.5, v_s=v_s, random_perm=True)
+    w = hi.custom(M, K, N, T, seed=51, t_s=0.5, v_s=v_s, random_perm=rperm)
     W, X, perm = dev_bf16(w.W_bits), dev_bf16(w.X_bits), dev_i32(w.perm)
     nt = M // T
     c = dev_i32(np.tile(np.array(H.hinm_counts_from_vs(K, 0.5, v_s), dtype=np.int32), (nt, 1)))
     hp = H.HotPath(M, K, N, T, 0.5, w.alpha)
-    Y1 = hp.run(W, X, perm, fixed_counts=c).clone()
-    Y2 = hp.run(W, X, perm, fixed_counts=c).clone()
+    pairs = H.tile_pairs_hint(H.hinm_counts_from_vs(K, 0.5, v_s), w.perm, K)
+    assert pairs == (v_s == 0.0 and not rperm)
+    Y1 = hp.run(W, X, perm, fixed_counts=c, tile_pairs=pairs).clone()
+    Y2 = hp.run(W, X, perm, fixed_counts=c, tile_pairs=pairs).clone()
     torch.cuda.synchronize()
     status_ok(H)
     np.testing.assert_array_equal(Y1.cpu().numpy().view(np.uint32), Y2.cpu().numpy().view(np.uint32))
@@ -329,7 +367,7 @@ def test_full_size_sampled(H, name, make, v_s):
     hp = H.HotPath(M, K, N, T, w.t_s, w.alpha)
     c = np.array(H.hinm_counts_from_vs(K, w.t_s, v_s), dtype=np.int32)
     fixed = dev_i32(np.tile(c, (nt, 1)))
-    Y = hp.run(W, X, perm, fixed_counts=fixed)
+    Y = hp.run(W, X, perm, fixed_counts=fixed, tile_pairs=H.tile_pairs_hint(c, w.perm, K))
     torch.cuda.synchronize()
     status_ok(H)
     tiles = sorted({0, nt // 2, nt - 1})
