@@ -357,10 +357,11 @@ def main():
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        H.hinm_importance(W, X, hp.I, hp.ws)
+        H.hinm_importance_stats(W, X, T, hp.I, hp.stats, hp.ws)
         if ev is not None:
             ev[1].record(stream)
-        H.hinm_boundary_search(hp.I, perm, T, w.t_s, w.alpha, hp.counts, hp.vs, hp.rank, hp.ws)
+        H.hinm_boundary_search(hp.I, perm, T, w.t_s, w.alpha, hp.counts, hp.vs, hp.rank, hp.ws,
+                               stats=hp.stats)
         if ev is not None:
             ev[2].record(stream)
         H.hinm_mask(hp.I, perm, counts_used, T, hp.rank, hp.bitmask, hp.region, hp.ws)
@@ -522,11 +523,12 @@ def main():
                          "importance, search, mask, compress and fp64 masked product",
                "seconds": dt}
     clocks = sampler.summary()
-    # this library's kernels per step: importance 2 (channel energies, importance), search 7
-    # (vector scores, chunk sort, merge rank, column sums, candidate lists, band sums,
-    # finalize), mask 2 (classify with the permutation check, bitmask), compress 3 (tile
-    # offsets, lists, pack), SpMM 1; the memsets between them are not counted
-    kernels_per_step = 2 + 7 + 2 + 3 + 1
+    # this library's kernels per step: importance 2 (channel energies, importance with the
+    # tile statistics), search 6 (chunk sort, merge rank, column sums, candidate lists, band
+    # sums, finalize; V comes from the importance step), mask 2 (classify with the
+    # permutation check, bitmask), compress 3 (tile offsets, lists, pack), SpMM 1; the
+    # memsets between them are not counted
+    kernels_per_step = 2 + 6 + 2 + 3 + 1
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True,

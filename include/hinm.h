@@ -102,6 +102,20 @@ hinm_status hinm_importance(const void* W, const void* X, int M, int K, int N,
 hinm_status hinm_importance_noalloc(const void* W, const void* X, int M, int K, int N,
                                     float* I_out, void* stream);
 
+/* Importance with the boundary search's tile statistics made in the same pass.  The
+ * method's description has no counterpart: the statistics are the search's own first step
+ * (a2 below), computed here while I is written so that the search does not read I for them.
+ *   I_out: as hinm_importance (bit for bit).  stats_out (device, hinm_tile_stats_size()
+ *   bytes, caller-owned): V[t][c] = sum over the tile's rows (ascending, fp64) of I[row, c]
+ *   by input channel c, and each tile's largest importance; an opaque layout that only
+ *   hinm_boundary_search_stats reads.  T as for the search (64 or 128).
+ *   Errors: as hinm_importance, plus HINM_ERR_SHAPE for T, HINM_ERR_INVALID_ARG for a NULL
+ *   or too small stats_out. */
+hinm_status hinm_tile_stats_size(int M, int K, int T, size_t* bytes_host);
+hinm_status hinm_importance_stats(const void* W, const void* X, int M, int K, int N, int T,
+                                  float* I_out, void* stats_out, size_t stats_bytes,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---------------------------------------------------------------------------------
  * Region counts for a fixed boundary (host only).  ([P1] 关键设计 1, closed form)
  *   n_24 = 4 * floor(2 (t_s - v_s) K / 4 + 1/2), n_0 = t_s K - n_24 / 2,
@@ -135,6 +149,16 @@ hinm_status hinm_boundary_search(const float* I, const int32_t* perm, int M, int
                                  double t_s, double alpha, int32_t* counts_out,
                                  double* vs_out, int32_t* rank_out, double* retained_out,
                                  void* workspace, size_t workspace_bytes, void* stream);
+/* hinm_boundary_search with the tile statistics that hinm_importance_stats made with this
+ * I (same M, K, T): the same results, without the search's own pass over I for V.  stats
+ * from another I or T give meaningless results (nothing checks that they match).
+ * Errors: as hinm_boundary_search, plus HINM_ERR_INVALID_ARG for a NULL or too small
+ * stats. */
+hinm_status hinm_boundary_search_stats(const float* I, const void* stats, size_t stats_bytes,
+                                       const int32_t* perm, int M, int K, int T, double t_s,
+                                       double alpha, int32_t* counts_out, double* vs_out,
+                                       int32_t* rank_out, double* retained_out,
+                                       void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------
  * a4. Mask  ([P1] 亮点与洞察: high -> dense, middle -> 2:4, low -> pruned;

@@ -63,6 +63,11 @@ _SIGS = {
     "hinm_importance_workspace_size": (_i32, [_i32, _i32, _i32, _szp]),
     "hinm_importance": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _sz, _vp]),
     "hinm_importance_noalloc": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp]),
+    "hinm_tile_stats_size": (_i32, [_i32, _i32, _i32, _szp]),
+    "hinm_importance_stats": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _sz, _vp, _sz,
+                                     _vp]),
+    "hinm_boundary_search_stats": (_i32, [_vp, _vp, _sz, _vp, _i32, _i32, _i32, _f64, _f64, _vp,
+                                          _vp, _vp, _vp, _vp, _sz, _vp]),
     "hinm_selftest_wait_timeout": (_i32, [ctypes.c_ulonglong, _vp]),
     "hinm_counts_from_vs": (_i32, [_i32, _f64, _f64, ctypes.POINTER(ctypes.c_int32)]),
     "hinm_search_num_candidates": (_i32, [_i32, _f64, _f64, ctypes.POINTER(ctypes.c_int32)]),
@@ -143,6 +148,39 @@ def hinm_importance(W, X, I_out=None, workspace=None, stream=None):
     return I_out
 
 
+def hinm_tile_stats_size(M: int, K: int, T: int) -> int:
+    return _size(_lib.hinm_tile_stats_size, M, K, T)
+
+
+def hinm_importance_stats(W, X, T: int, I_out=None, stats_out=None, workspace=None, stream=None):
+    """hinm_importance that also writes the boundary search's tile statistics (V and the
+    tile maxima) in the same pass.  Returns (I, stats); stats is an opaque uint8 buffer for
+    hinm_boundary_search(..., stats=stats)."""
+    torch = _torch()
+    M, K = W.shape
+    N = X.shape[1]
+    if I_out is None:
+        I_out = torch.empty((M, K), dtype=torch.float32, device=W.device)
+    if stats_out is None:
+        stats_out = _empty_bytes(hinm_tile_stats_size(M, K, T), W.device)
+    if workspace is None:
+        workspace = _empty_bytes(_size(_lib.hinm_importance_workspace_size, M, K, N), W.device)
+    _check(_lib.hinm_importance_stats(_ptr(W), _ptr(X), M, K, N, T, _ptr(I_out), _ptr(stats_out),
+                                      stats_out.numel(), _ptr(workspace), workspace.numel(),
+                                      _stream(stream)), "hinm_importance_stats")
+    return I_out, stats_out
+
+
+def tile_stats_views(stats, M: int, K: int, T: int):
+    """(V fp64 [M/T, K], tile maxima int32 [M/T]) as views of a stats buffer (for tests)."""
+    torch = _torch()
+    nt = M // T
+    v_bytes = (nt * K * 8 + 255) & ~255
+    V = stats[:nt * K * 8].view(torch.float64).view(nt, K)
+    pmax = stats[v_bytes:v_bytes + nt * 4].view(torch.int32)
+    return V, pmax
+
+
 def hinm_selftest_wait_timeout(limit_ns: int, stream=None):
     """Launches the bounded-wait self test (see hinm.h); read the outcome with
     hinm_device_status()."""
@@ -181,9 +219,11 @@ def hinm_search_num_candidates(K: int, t_s: float, alpha: float = 1.0 / 32.0) ->
 
 def hinm_boundary_search(I, perm, T: int, t_s: float, alpha: float = 1.0 / 32.0,
                          counts_out=None, vs_out=None, rank_out=None, workspace=None,
-                         want_rank: bool = True, retained_out=None, stream=None):
+                         want_rank: bool = True, retained_out=None, stream=None, stats=None):
     """Per-tile first-drop scan of v_s.  Returns (counts int32 [M/T,3], v_s fp64 [M/T], rank).
-    ``retained_out`` (fp64 [M/T, n_cand]) optionally receives R(m) of every candidate."""
+    ``retained_out`` (fp64 [M/T, n_cand]) optionally receives R(m) of every candidate;
+    ``stats`` (from hinm_importance_stats for this I and T) spares the search its pass over
+    I for V."""
     torch = _torch()
     M, K = I.shape
     nt = M // T
@@ -196,10 +236,17 @@ def hinm_boundary_search(I, perm, T: int, t_s: float, alpha: float = 1.0 / 32.0,
         rank_out = torch.empty((nt, K), dtype=torch.int32, device=dev)
     if workspace is None:
         workspace = _empty_bytes(hinm_search_workspace_size(M, K, T, t_s, alpha), dev)
-    _check(_lib.hinm_boundary_search(_ptr(I), _ptr(perm), M, K, T, t_s, alpha, _ptr(counts_out),
-                                     _ptr(vs_out), _ptr(rank_out), _ptr(retained_out),
-                                     _ptr(workspace), workspace.numel(), _stream(stream)),
-           "hinm_boundary_search")
+    if stats is not None:
+        _check(_lib.hinm_boundary_search_stats(_ptr(I), _ptr(stats), stats.numel(), _ptr(perm), M,
+                                               K, T, t_s, alpha, _ptr(counts_out), _ptr(vs_out),
+                                               _ptr(rank_out), _ptr(retained_out),
+                                               _ptr(workspace), workspace.numel(),
+                                               _stream(stream)), "hinm_boundary_search_stats")
+    else:
+        _check(_lib.hinm_boundary_search(_ptr(I), _ptr(perm), M, K, T, t_s, alpha,
+                                         _ptr(counts_out), _ptr(vs_out), _ptr(rank_out),
+                                         _ptr(retained_out), _ptr(workspace), workspace.numel(),
+                                         _stream(stream)), "hinm_boundary_search")
     return counts_out, vs_out, rank_out
 
 
@@ -359,14 +406,15 @@ class HotPath:
                  hinm_search_workspace_size(M, K, T, t_s, alpha),
                  hinm_mask_workspace_size(M, K, T), hinm_compress_workspace_size(M, K, T))
         self.ws = _empty_bytes(ws, device)
+        self.stats = _empty_bytes(hinm_tile_stats_size(M, K, T), device)
 
     def run(self, W, X, perm, fixed_counts=None, stream=None, tile_pairs=False):
         """One pass of the path.  The search always runs (its ranking feeds the mask);
         ``fixed_counts`` (int32 [M/T, 3]) replaces its counts when given; ``tile_pairs`` is
         the SpMM hint (hinm_spmm)."""
-        hinm_importance(W, X, self.I, self.ws, stream)
+        hinm_importance_stats(W, X, self.T, self.I, self.stats, self.ws, stream)
         hinm_boundary_search(self.I, perm, self.T, self.t_s, self.alpha, self.counts, self.vs,
-                             self.rank, self.ws, stream=stream)
+                             self.rank, self.ws, stream=stream, stats=self.stats)
         counts = self.counts if fixed_counts is None else fixed_counts
         hinm_mask(self.I, perm, counts, self.T, self.rank, self.bitmask, self.region, self.ws,
                   stream)

@@ -223,6 +223,39 @@ hinm_status hinm_importance(const void* W, const void* X, int M, int K, int N, f
   return ok();
 }
 
+hinm_status hinm_tile_stats_size(int M, int K, int T, size_t* bytes_host) {
+  if (!bytes_host) return fail(HINM_ERR_INVALID_ARG, "bytes_host is NULL");
+  hinm_status st = check_mkt(M, K, T);
+  if (st != HINM_OK) return st;
+  *bytes_host = hinm::tile_stats_bytes(M, K, T);
+  return ok();
+}
+
+hinm_status hinm_importance_stats(const void* W, const void* X, int M, int K, int N, int T,
+                                  float* I_out, void* stats_out, size_t stats_bytes,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  REQUIRE_PTR(W);
+  REQUIRE_PTR(X);
+  REQUIRE_PTR(I_out);
+  REQUIRE_PTR(stats_out);
+  hinm_status st = check_mkt(M, K, T);
+  if (st != HINM_OK) return st;
+  st = check_n(N);
+  if (st != HINM_OK) return st;
+  if (stats_bytes < hinm::tile_stats_bytes(M, K, T))
+    return fail(HINM_ERR_INVALID_ARG, "stats %zu bytes, need %zu", stats_bytes,
+                hinm::tile_stats_bytes(M, K, T));
+  const size_t need = hinm::importance_workspace_bytes(K);
+  if (!workspace || workspace_bytes < need)
+    return fail(HINM_ERR_WORKSPACE, "workspace %zu bytes, need %zu", workspace_bytes, need);
+  REQUIRE_PTR(workspace);
+  cudaError_t e = hinm::launch_importance_stats(
+      static_cast<const uint16_t*>(W), static_cast<const uint16_t*>(X), M, K, N, T, I_out,
+      stats_out, static_cast<float*>(workspace), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "hinm_importance_stats launch");
+  return ok();
+}
+
 hinm_status hinm_importance_noalloc(const void* W, const void* X, int M, int K, int N,
                                     float* I_out, void* stream) {
   REQUIRE_PTR(W);
@@ -270,10 +303,14 @@ hinm_status hinm_search_workspace_size(int M, int K, int T, double t_s, double a
   return ok();
 }
 
-hinm_status hinm_boundary_search(const float* I, const int32_t* perm, int M, int K, int T,
-                                 double t_s, double alpha, int32_t* counts_out, double* vs_out,
-                                 int32_t* rank_out, double* retained_out, void* workspace,
-                                 size_t workspace_bytes, void* stream) {
+namespace {
+
+// hinm_boundary_search(_stats): stats (with its size) or nullptr
+hinm_status search_impl(const float* I, const void* stats, size_t stats_bytes,
+                        const int32_t* perm, int M, int K, int T, double t_s, double alpha,
+                        int32_t* counts_out, double* vs_out, int32_t* rank_out,
+                        double* retained_out, void* workspace, size_t workspace_bytes,
+                        void* stream) {
   REQUIRE_PTR(I);
   REQUIRE_ALIGNED_OR_NULL(perm);
   REQUIRE_PTR(counts_out);
@@ -284,6 +321,9 @@ hinm_status hinm_boundary_search(const float* I, const int32_t* perm, int M, int
   if (st != HINM_OK) return st;
   st = check_search_params(t_s, alpha);
   if (st != HINM_OK) return st;
+  if (stats && stats_bytes < hinm::tile_stats_bytes(M, K, T))
+    return fail(HINM_ERR_INVALID_ARG, "stats %zu bytes, need %zu", stats_bytes,
+                hinm::tile_stats_bytes(M, K, T));
   hinm::Candidate c[hinm::kMaxCandidates];
   const int n = hinm::search_candidates_host(K, t_s, alpha, c, hinm::kMaxCandidates);
   if (n < 0) return fail(HINM_ERR_INVALID_ARG, "t_s*K = %g is not a whole number", t_s * K);
@@ -295,12 +335,32 @@ hinm_status hinm_boundary_search(const float* I, const int32_t* perm, int M, int
   if (!workspace || workspace_bytes < need)
     return fail(HINM_ERR_WORKSPACE, "workspace %zu bytes, need %zu", workspace_bytes, need);
   REQUIRE_PTR(workspace);
-  cudaError_t e = hinm::launch_boundary_search(I, perm, M, K, T, t_s, alpha, c, n, counts_out,
-                                               vs_out, rank_out, retained_out, workspace,
-                                               hinm::device_status_ptr(),
+  cudaError_t e = hinm::launch_boundary_search(I, stats, perm, M, K, T, t_s, alpha, c, n,
+                                               counts_out, vs_out, rank_out, retained_out,
+                                               workspace, hinm::device_status_ptr(),
                                                static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "hinm_boundary_search launch");
   return ok();
+}
+
+}  // namespace
+
+hinm_status hinm_boundary_search(const float* I, const int32_t* perm, int M, int K, int T,
+                                 double t_s, double alpha, int32_t* counts_out, double* vs_out,
+                                 int32_t* rank_out, double* retained_out, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  return search_impl(I, nullptr, 0, perm, M, K, T, t_s, alpha, counts_out, vs_out, rank_out,
+                     retained_out, workspace, workspace_bytes, stream);
+}
+
+hinm_status hinm_boundary_search_stats(const float* I, const void* stats, size_t stats_bytes,
+                                       const int32_t* perm, int M, int K, int T, double t_s,
+                                       double alpha, int32_t* counts_out, double* vs_out,
+                                       int32_t* rank_out, double* retained_out,
+                                       void* workspace, size_t workspace_bytes, void* stream) {
+  REQUIRE_PTR(stats);
+  return search_impl(I, stats, stats_bytes, perm, M, K, T, t_s, alpha, counts_out, vs_out,
+                     rank_out, retained_out, workspace, workspace_bytes, stream);
 }
 
 hinm_status hinm_mask_workspace_size(int M, int K, int T, size_t* bytes_host) {

@@ -56,6 +56,13 @@ struct Carve {
 size_t importance_workspace_bytes(int K);
 cudaError_t launch_importance(const uint16_t* W, const uint16_t* X, int M, int K, int N,
                               float* I, float* s_scratch, cudaStream_t s);
+// Tile statistics of the boundary search made with I: V (fp64 [M/T][K], channel order) at
+// offset 0, then the tile maxima (int [M/T]) at tile_stats_v_bytes().
+size_t tile_stats_v_bytes(int M, int K, int T);
+size_t tile_stats_bytes(int M, int K, int T);
+cudaError_t launch_importance_stats(const uint16_t* W, const uint16_t* X, int M, int K, int N,
+                                    int T, float* I, void* stats, float* s_scratch,
+                                    cudaStream_t s);
 
 // Workspace-free variant: channel energies in a static per-device array of kNoAllocMaxK
 // floats (64 KiB).
@@ -63,10 +70,12 @@ constexpr int kNoAllocMaxK = 16384;
 cudaError_t noalloc_energy_scratch(float** out);
 
 size_t search_workspace_bytes(int M, int K, int T, int ncand);
-cudaError_t launch_boundary_search(const float* I, const int32_t* perm, int M, int K, int T,
-                                   double t_s, double alpha, const Candidate* cands, int ncand,
-                                   int32_t* counts_out, double* vs_out, int32_t* rank_out,
-                                   double* retained_out, void* ws, int* status, cudaStream_t s);
+// stats: from launch_importance_stats for this I and T, or nullptr (computed here from I)
+cudaError_t launch_boundary_search(const float* I, const void* stats, const int32_t* perm,
+                                   int M, int K, int T, double t_s, double alpha,
+                                   const Candidate* cands, int ncand, int32_t* counts_out,
+                                   double* vs_out, int32_t* rank_out, double* retained_out,
+                                   void* ws, int* status, cudaStream_t s);
 
 size_t mask_workspace_bytes(int M, int K, int T);
 cudaError_t launch_mask(const float* I, const int32_t* perm, const int32_t* counts,

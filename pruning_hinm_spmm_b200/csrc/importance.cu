@@ -103,6 +103,62 @@ __global__ void importance_kernel(const uint16_t* __restrict__ W, const float* _
   }
 }
 
+// I as importance_kernel computes it, and with it the boundary search's tile statistics:
+// V[t, c] = the fp64 sum of the tile's I[., c] over its rows in ascending order (the same
+// additions in the same order as the search's own vector scores), and tile_pmax[t] = the
+// exponent index p (value = m 2^(p-149)) of the tile's largest importance.  One thread per
+// (tile, 2 channels) walks the tile's rows; 16 rows' loads are in flight ahead of the
+// dependent fp64 chains.  tile_pmax must be 0 before the launch.
+constexpr int kStatRows = 16;  // T is a multiple of 16
+
+__global__ void importance_stats_kernel(const uint16_t* __restrict__ W,
+                                        const float* __restrict__ s, int K, int T,
+                                        float* __restrict__ I, double* __restrict__ V,
+                                        int* __restrict__ tile_pmax) {
+  const int cp = blockIdx.x * blockDim.x + threadIdx.x;  // channel pair
+  const int t = blockIdx.y;
+  uint32_t mb = 0;  // largest bit pattern = largest value (non-negative floats)
+  if (2 * cp < K) {
+    const int c0 = 2 * cp;
+    const float s0 = __ldg(s + c0), s1 = __ldg(s + c0 + 1);
+    const uint32_t* wp = reinterpret_cast<const uint32_t*>(W + (size_t)t * T * K + c0);
+    float2* ip = reinterpret_cast<float2*>(I + (size_t)t * T * K + c0);
+    const size_t step = (size_t)K / 2;  // one row, in channel pairs
+    double v0 = 0.0, v1 = 0.0;
+    uint32_t wv[kStatRows], nx[kStatRows];
+#pragma unroll
+    for (int k = 0; k < kStatRows; ++k) wv[k] = __ldg(wp + (size_t)k * step);
+    for (int r0 = 0; r0 < T; r0 += kStatRows) {
+      if (r0 + kStatRows < T) {  // the next rows' loads in flight during these rows
+#pragma unroll
+        for (int k = 0; k < kStatRows; ++k) nx[k] = __ldg(wp + (size_t)(r0 + kStatRows + k) * step);
+      }
+#pragma unroll
+      for (int k = 0; k < kStatRows; ++k) {  // rows ascending
+        const float w0 = __uint_as_float(wv[k] << 16), w1 = __uint_as_float(wv[k] & 0xFFFF0000u);
+        const float i0 = __fmul_rn(__fmul_rn(w0, w0), s0);
+        const float i1 = __fmul_rn(__fmul_rn(w1, w1), s1);
+        __stcs(ip + (size_t)(r0 + k) * step, make_float2(i0, i1));
+        v0 = __dadd_rn(v0, (double)i0);
+        v1 = __dadd_rn(v1, (double)i1);
+        mb = max(mb, max(__float_as_uint(i0), __float_as_uint(i1)));
+      }
+#pragma unroll
+      for (int k = 0; k < kStatRows; ++k) wv[k] = nx[k];
+    }
+    V[(size_t)t * K + c0] = v0;
+    V[(size_t)t * K + c0 + 1] = v1;
+  }
+  int pm = 0;
+  if (mb) {
+    const uint32_t e = mb >> 23;
+    pm = (e ? (int)e : 1) - 1;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) pm = max(pm, __shfl_xor_sync(0xffffffffu, pm, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(tile_pmax + t, pm);
+}
+
 int sm_count() {
   static int n = 0;
   if (n == 0) {
@@ -142,6 +198,30 @@ cudaError_t noalloc_energy_scratch(float** out) {
   }
   *out = g_noalloc_ptr[dev];
   return cudaSuccess;
+}
+
+size_t tile_stats_v_bytes(int M, int K, int T) {
+  return ((size_t)(M / T) * K * sizeof(double) + 255) & ~size_t(255);
+}
+size_t tile_stats_bytes(int M, int K, int T) {
+  return tile_stats_v_bytes(M, K, T) + (((size_t)(M / T) * sizeof(int) + 255) & ~size_t(255));
+}
+
+cudaError_t launch_importance_stats(const uint16_t* W, const uint16_t* X, int M, int K, int N,
+                                    int T, float* I, void* stats, float* s_scratch,
+                                    cudaStream_t st) {
+  const int nt = M / T;
+  double* V = static_cast<double*>(stats);
+  int* pmax = reinterpret_cast<int*>(static_cast<char*>(stats) + tile_stats_v_bytes(M, K, T));
+  cudaError_t e = cudaMemsetAsync(pmax, 0, (size_t)nt * sizeof(int), st);
+  if (e != cudaSuccess) return e;
+  channel_energy_kernel<<<(K + kEnergyWarps - 1) / kEnergyWarps, kEnergyWarps * 32, 0, st>>>(
+      X, K, N, s_scratch);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const dim3 g((K / 2 + 255) / 256, nt);
+  importance_stats_kernel<<<g, 256, 0, st>>>(W, s_scratch, K, T, I, V, pmax);
+  return cudaGetLastError();
 }
 
 size_t importance_workspace_bytes(int K) { return ((size_t)K * sizeof(float) + 255) & ~size_t(255); }

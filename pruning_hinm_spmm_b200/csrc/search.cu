@@ -827,24 +827,35 @@ size_t search_workspace_bytes(int M, int K, int T, int ncand) {
   return (c.off + 255) & ~size_t(255);
 }
 
-cudaError_t launch_boundary_search(const float* I, const int32_t* perm, int M, int K, int T,
-                                   double t_s, double alpha, const Candidate* cands, int ncand,
-                                   int32_t* counts_out, double* vs_out, int32_t* rank_out,
-                                   double* retained_out, void* ws, int* status, cudaStream_t s) {
+cudaError_t launch_boundary_search(const float* I, const void* stats, const int32_t* perm,
+                                   int M, int K, int T, double t_s, double alpha,
+                                   const Candidate* cands, int ncand, int32_t* counts_out,
+                                   double* vs_out, int32_t* rank_out, double* retained_out,
+                                   void* ws, int* status, cudaStream_t s) {
   (void)status;
   const int nt = M / T;
   Carve c{static_cast<char*>(ws), 0};
-  double* V = c.take<double>((size_t)nt * K);
+  double* V_ws = c.take<double>((size_t)nt * K);
   int32_t* rank_ws = c.take<int32_t>((size_t)nt * K);
   double* R_ws = c.take<double>((size_t)nt * ncand);
   double* R = retained_out ? retained_out : R_ws;
-  int* pmax = c.take<int>((size_t)nt);
+  int* pmax_ws = c.take<int>((size_t)nt);
   U128* colsum = c.take<U128>((size_t)nt * K);
   unsigned char* coltiny = c.take<unsigned char>((size_t)nt * K);
   char* rank_scratch = c.take<char>(rank_scratch_bytes(M, K, T));
   int32_t* rank = rank_out ? rank_out : rank_ws;
-  cudaError_t e = launch_vector_scores(I, M, K, T, V, pmax, s);
-  if (e != cudaSuccess) return e;
+  // V and the tile maxima: made with I by the importance step, or computed here
+  const double* V = V_ws;
+  const int* pmax = pmax_ws;
+  cudaError_t e = cudaSuccess;
+  if (stats) {
+    V = static_cast<const double*>(stats);
+    pmax = reinterpret_cast<const int*>(static_cast<const char*>(stats) +
+                                        tile_stats_v_bytes(M, K, T));
+  } else {
+    e = launch_vector_scores(I, M, K, T, V_ws, pmax_ws, s);
+    if (e != cudaSuccess) return e;
+  }
   {
     // the exact column sums (which need the tile maxima) run on the side stream while the
     // ranking (which needs V) runs on the caller's stream; joined before the candidates

@@ -113,6 +113,23 @@ def test_validation_rejects_before_launch(H):
     L = H.hinm_layout(H.HINM_LAYOUT_VERSION, 256, 256, 64, 4, 1, 1, fake, fake, fake, fake, fake, fake, fake, fake)
     assert lib.hinm_spmm(ctypes.byref(L), fake, 20, fake, None) == H.HINM_ERR_SHAPE
     assert lib.hinm_spmm(ctypes.byref(L), fake + 8, 16, fake, None) == H.HINM_ERR_ALIGNMENT
+    # the fused importance statistics: T checked, stats buffer required and large enough
+    sz = ctypes.c_size_t(0)
+    assert lib.hinm_tile_stats_size(256, 256, 96, ctypes.byref(sz)) == H.HINM_ERR_SHAPE
+    assert lib.hinm_tile_stats_size(256, 256, 128, ctypes.byref(sz)) == H.HINM_OK
+    assert sz.value >= 2 * 256 * 8 + 2 * 4
+    assert lib.hinm_importance_stats(fake, fake, 256, 256, 16, 128, fake, None, sz.value, fake,
+                                     1 << 20, None) == H.HINM_ERR_INVALID_ARG
+    assert lib.hinm_importance_stats(fake, fake, 256, 256, 16, 128, fake, fake, sz.value - 1,
+                                     fake, 1 << 20, None) == H.HINM_ERR_INVALID_ARG
+    assert lib.hinm_importance_stats(fake, fake, 256, 256, 16, 96, fake, fake, sz.value, fake,
+                                     1 << 20, None) == H.HINM_ERR_SHAPE
+    assert lib.hinm_boundary_search_stats(fake, None, sz.value, None, 256, 256, 128, 0.5,
+                                          1 / 32, fake, fake, None, None, fake, 1 << 30,
+                                          None) == H.HINM_ERR_INVALID_ARG
+    assert lib.hinm_boundary_search_stats(fake, fake, 8, None, 256, 256, 128, 0.5, 1 / 32, fake,
+                                          fake, None, None, fake, 1 << 30,
+                                          None) == H.HINM_ERR_INVALID_ARG
     # hinm_spmm_ex: unknown flag bits are refused before anything else; the hint flag
     # passes the same argument checks as hinm_spmm
     assert lib.hinm_spmm_ex(ctypes.byref(L), fake, 16, fake, 2, None) == H.HINM_ERR_INVALID_ARG

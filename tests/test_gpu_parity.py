@@ -216,6 +216,36 @@ def test_channel_energy_rounding_fallback(H):
 
 
 @pytest.mark.parametrize("name,make,v_s", CASES, ids=[c[0] for c in CASES])
+def test_importance_stats_and_search_with_stats(H, name, make, v_s):
+    """The importance step's fused tile statistics: I bit for bit as hinm_importance, V
+    equal to the oracle's vector scores (by channel), the tile maxima equal to the largest
+    exponent of the tile's importances, and the search given them returns exactly what the
+    search computing them itself returns (counts, v_s, rank, every R(m))."""
+    w = make()
+    M, K, T = w.M, w.K, w.T
+    nt = M // T
+    W, X, perm = dev_bf16(w.W_bits), dev_bf16(w.X_bits), dev_i32(w.perm)
+    I0 = H.hinm_importance(W, X)
+    I1, stats = H.hinm_importance_stats(W, X, T)
+    nc = H.hinm_search_num_candidates(K, w.t_s, w.alpha)
+    R0 = torch.empty((nt, nc), dtype=torch.float64, device="cuda")
+    R1 = torch.empty((nt, nc), dtype=torch.float64, device="cuda")
+    c0, v0, r0 = H.hinm_boundary_search(I0, perm, T, w.t_s, w.alpha, retained_out=R0)
+    c1, v1, r1 = H.hinm_boundary_search(I1, perm, T, w.t_s, w.alpha, retained_out=R1, stats=stats)
+    torch.cuda.synchronize()
+    status_ok(H)
+    I_np = I0.cpu().numpy()
+    np.testing.assert_array_equal(I1.cpu().numpy().view(np.uint32), I_np.view(np.uint32))
+    V, pmax = H.tile_stats_views(stats, M, K, T)
+    np.testing.assert_array_equal(V.cpu().numpy()[:, w.perm], O.vector_scores(I_np, w.perm, T))
+    top = I_np.view(np.uint32).reshape(nt, T * K).max(axis=1).astype(np.int64)
+    p_ref = np.where(top > 0, np.maximum(top >> 23, 1) - 1, 0)
+    np.testing.assert_array_equal(pmax.cpu().numpy(), p_ref)
+    for a, b in ((c0, c1), (v0, v1), (r0, r1), (R0, R1)):
+        np.testing.assert_array_equal(a.cpu().numpy(), b.cpu().numpy())
+
+
+@pytest.mark.parametrize("name,make,v_s", CASES, ids=[c[0] for c in CASES])
 def test_search_decision_without_retained_matches_full_scan(H, name, make, v_s):
     """With no R requested the scan may stop evaluating candidates after a tile's decision;
     the counts and v_s must still equal the full scan's and the oracle's."""
