@@ -107,9 +107,9 @@ __global__ void importance_kernel(const uint16_t* __restrict__ W, const float* _
 // V[t, c] = the fp64 sum of the tile's I[., c] over its rows in ascending order (the same
 // additions in the same order as the search's own vector scores), and tile_pmax[t] = the
 // exponent index p (value = m 2^(p-149)) of the tile's largest importance.  One thread per
-// (tile, 2 channels) walks the tile's rows; 16 rows' loads are in flight ahead of the
+// (tile, 2 channels) walks the tile's rows; 32 rows' loads are in flight ahead of the
 // dependent fp64 chains.  tile_pmax must be 0 before the launch.
-constexpr int kStatRows = 16;  // T is a multiple of 16
+constexpr int kStatRows = 32;  // T is a multiple of 32 (64 or 128)
 
 __global__ void importance_stats_kernel(const uint16_t* __restrict__ W,
                                         const float* __restrict__ s, int K, int T,
