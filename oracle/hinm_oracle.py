@@ -500,6 +500,26 @@ def contiguous_runs(idx: np.ndarray) -> np.ndarray:
     return out
 
 
+def translate_index(L: Layout, row_of_channel: np.ndarray) -> Layout:
+    """Cross-layer index translation: the layout for an X whose rows arrive reordered.
+
+    [P1] 关键设计 2: reordering channels leaves the result unchanged, and the translation
+    between layers is folded into the HiNM index, done while the data is moved, with no
+    extra runtime step.  [reading] When X arrives with row r holding input channel
+    sigma[r] (the previous layer's output in its permuted row order), every index entry
+    c becomes row_of_channel[c] = sigma^-1[c], and each block's run flag is recomputed by
+    the same rule as ``compress`` (``contiguous_runs``).  Values, metadata and tile_info
+    are unchanged, so the product with the reordered X equals the original product.
+    """
+    roc = np.asarray(row_of_channel, dtype=np.int64)
+    idx_d = roc[L.idx_dense].astype(np.int32) if L.idx_dense.size else L.idx_dense.copy()
+    idx_s = roc[L.idx_sparse].astype(np.int32) if L.idx_sparse.size else L.idx_sparse.copy()
+    return Layout(M=L.M, K=L.K, T=L.T, tile_info=L.tile_info.copy(),
+                  vals_dense=L.vals_dense.copy(), vals_sparse=L.vals_sparse.copy(),
+                  meta=L.meta.copy(), idx_dense=idx_d, idx_sparse=idx_s,
+                  run_dense=contiguous_runs(idx_d), run_sparse=contiguous_runs(idx_s))
+
+
 def decompress(L: Layout) -> np.ndarray:
     """Rebuild W ⊙ M (fp32, M x K) from a layout; the inverse of ``compress``."""
     out = np.zeros((L.M, L.K), dtype=np.float32)

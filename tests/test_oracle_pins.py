@@ -430,6 +430,46 @@ def test_contiguous_runs_identity_pure24():
     np.testing.assert_array_equal(L.run_sparse, [0, 128])
 
 
+# ----------------------------------------------------------------------------- index translation
+def _layout_fields_equal(A, B):
+    for f in ("tile_info", "vals_dense", "vals_sparse", "meta", "idx_dense", "idx_sparse",
+              "run_dense", "run_sparse"):
+        np.testing.assert_array_equal(getattr(A, f), getattr(B, f), err_msg=f)
+
+
+@pytest.mark.parametrize("v_s,perm", [(0.25, True), (0.0, False), (0.5, False)])
+def test_translate_index_pins(v_s, perm):
+    """The cross-layer index translation ([P1] 关键设计 2): (i) the identity row map leaves
+    the layout unchanged (its run flags included: the recomputation is compress's rule);
+    (ii) translations compose, translate(translate(L, a), b) == translate(L, b[a]); (iii)
+    the translated layout times X with its rows reordered equals the original product
+    exactly (integer data, so the fp64 sums are exact), through decompress, itself pinned
+    by the round trip above."""
+    T, K = 64, 256
+    w = hi.integer_workload(2 * T, K, 8, T, seed=7, t_s=0.5, v_s=v_s, random_perm=perm)
+    I = O.importance(w.W_bits, w.X_bits)
+    counts = np.tile(np.array(O.counts_from_vs(K, 0.5, v_s)), (2, 1))
+    bm, region = O.mask(I, w.perm, T, counts)
+    L = O.compress(w.W_bits, bm, region, w.perm, counts, T)
+    _layout_fields_equal(O.translate_index(L, np.arange(K)), L)
+    rng = np.random.default_rng(11)
+    a, b = rng.permutation(K), rng.permutation(K)
+    _layout_fields_equal(O.translate_index(O.translate_index(L, a), b), O.translate_index(L, b[a]))
+    sigma = rng.permutation(K)                 # delivered row r holds channel sigma[r]
+    row_of_channel = np.argsort(sigma)         # sigma^-1
+    Lt = O.translate_index(L, row_of_channel)
+    X = f32(w.X_bits).astype(np.float64)
+    X_del = X[sigma]
+    y = O.decompress(L).astype(np.float64) @ X
+    y_t = O.decompress(Lt).astype(np.float64) @ X_del
+    np.testing.assert_array_equal(y_t, y)
+    # a reordered X generally breaks the runs: only blocks that stay ascending keep a flag
+    for idx, run in ((Lt.idx_dense, Lt.run_dense), (Lt.idx_sparse, Lt.run_sparse)):
+        for k in range(idx.shape[0]):
+            ok = all(int(idx[k, v]) == int(idx[k, 0]) + v for v in range(idx.shape[1]))
+            assert run[k] == (idx[k, 0] if ok else -1)
+
+
 # ----------------------------------------------------------------------------- spmm reference
 def test_spmm_identity_x_gives_masked_weight():
     w = hi.custom(128, 64, 64, 64, seed=2, t_s=0.5, v_s=0.25)
