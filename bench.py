@@ -299,6 +299,34 @@ def run_sweep(args):
 
 
 # ------------------------------------------------------------------ GPU arm
+def time_index_translate(H, hp, K, stream, reps=20):
+    """The cross-layer index translation on this workload's layout, with the identity map
+    (every index rewritten to itself, every run flag recomputed): CUDA events over `reps`
+    back-to-back calls after 3 untimed ones.  Bytes: 4 B read + 4 B written per index entry,
+    4 B read from the map per entry, 4 B written per block."""
+    import torch
+    ident = torch.arange(K, dtype=torch.int32, device=hp.I.device)
+    info = hp.layout.tile_info.cpu().numpy()
+    nd, ns = int(info[:, 0].sum()), int(info[:, 1].sum())
+    entries = nd * 64 + ns * 128
+    for _ in range(3):
+        H.hinm_translate_index(hp.layout, ident, None, hp.c_layout)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        H.hinm_translate_index(hp.layout, ident, None, hp.c_layout)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    st = H.hinm_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after the index translation")
+    t = e0.elapsed_time(e1) / 1e3 / reps
+    nbytes = entries * 12 + (nd + ns) * 4
+    return {"us_per_call": t * 1e6, "index_entries": entries, "blocks": nd + ns,
+            "gbs": nbytes / t / 1e9, "kernel": "translate_index_kernel", "launches": 1,
+            "note": "identity map on the step's layout; back-to-back calls (L2-warm)"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -523,6 +551,7 @@ def main():
                          "importance, search, mask, compress and fp64 masked product",
                "seconds": dt}
     clocks = sampler.summary()
+    next_rows = {"index_translate": time_index_translate(H, hp, K, stream)}
     # this library's kernels per step: importance 2 (channel energies, importance with the
     # tile statistics), search 6 (chunk sort, merge rank, column sums, candidate lists, band
     # sums, finalize; V comes from the importance step), mask 2 (classify with the
@@ -555,6 +584,7 @@ def main():
                               "streams"},
         "gpu_launches": kernels_per_step * args.steps,
         "gpu_launches_phase_pass": kernels_per_step * args.steps,
+        "next_rows": next_rows,
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                    "reasons": clocks["reasons"], "samples": clocks["samples"]},
     }

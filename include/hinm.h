@@ -228,6 +228,19 @@ hinm_status hinm_compress(const void* W, const uint32_t* bitmask, const int8_t* 
                           const hinm_layout* layout, void* workspace,
                           size_t workspace_bytes, void* stream);
 
+/* Cross-layer index translation  ([P1] 关键设计 2: channel reordering leaves the result
+ * unchanged, and the translation between layers is folded into the HiNM index).
+ * For an X whose rows arrive reordered -- row r holds input channel sigma[r], e.g. the
+ * previous layer's output in its own permuted row order -- rewrites the layout in place:
+ * every vector index c becomes row_of_channel[c] (= sigma^-1[c]) and every block's run flag
+ * is recomputed.  hinm_spmm(translated layout, reordered X) then equals hinm_spmm(layout,
+ * X) bit for bit, with no reordering of X at run time.
+ * row_of_channel: device int32 [K], a permutation of 0..K-1 (an entry outside [0, K) sets
+ * HINM_ERR_INVALID_ARG in the device status word and maps to row 0; a repeated entry is not
+ * detected and gives a different product).  Values, metadata and tile_info are untouched. */
+hinm_status hinm_translate_index(const hinm_layout* layout, const int32_t* row_of_channel,
+                                 void* stream);
+
 /* ---------------------------------------------------------------------------------
  * a6. SpMM  ([P1] 关键设计 4: Y = dense part + 2:4 part, one output)
  *   Y[t*T + r, n] = sum over dense vectors v of Wd[r, v] * X[idx_d(v), n]

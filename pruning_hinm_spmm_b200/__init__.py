@@ -80,6 +80,7 @@ _SIGS = {
     "hinm_compress_workspace_size": (_i32, [_i32, _i32, _i32, _szp]),
     "hinm_compress": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
                              ctypes.POINTER(hinm_layout), _vp, _sz, _vp]),
+    "hinm_translate_index": (_i32, [ctypes.POINTER(hinm_layout), _vp, _vp]),
     "hinm_spmm": (_i32, [ctypes.POINTER(hinm_layout), _vp, _i32, _vp, _vp]),
     "hinm_spmm_ex": (_i32, [ctypes.POINTER(hinm_layout), _vp, _i32, _vp, _i32, _vp]),
     "hinm_device_status": (_i32, [_vp, ctypes.POINTER(ctypes.c_int32)]),
@@ -361,6 +362,16 @@ def hinm_spmm(layout: HinmLayout, X, Y_out=None, stream=None, c_layout: Optional
         _check(_lib.hinm_spmm(ctypes.byref(c), _ptr(X), N, _ptr(Y_out), _stream(stream)),
                "hinm_spmm")
     return Y_out
+
+
+def hinm_translate_index(layout: HinmLayout, row_of_channel, stream=None,
+                         c_layout: Optional[hinm_layout] = None):
+    """Rewrites the layout's indices in place for an X whose row r holds channel sigma[r]:
+    row_of_channel = sigma^-1 (device int32 [K])."""
+    c = c_layout if c_layout is not None else layout.as_c()
+    _check(_lib.hinm_translate_index(ctypes.byref(c), _ptr(row_of_channel), _stream(stream)),
+           "hinm_translate_index")
+    return layout
 
 
 def hinm_device_status(stream=None) -> int:

@@ -487,6 +487,17 @@ hinm_status hinm_compress(const void* W, const uint32_t* bitmask, const int8_t* 
   return ok();
 }
 
+hinm_status hinm_translate_index(const hinm_layout* layout, const int32_t* row_of_channel,
+                                void* stream) {
+  hinm_status st = check_layout(layout);
+  if (st != HINM_OK) return st;
+  REQUIRE_PTR(row_of_channel);
+  cudaError_t e = hinm::launch_translate_index(*layout, row_of_channel, hinm::device_status_ptr(),
+                                               static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "hinm_translate_index launch");
+  return ok();
+}
+
 hinm_status hinm_spmm(const hinm_layout* layout, const void* X, int N, float* Y_out,
                       void* stream) {
   return hinm_spmm_ex(layout, X, N, Y_out, 0, stream);

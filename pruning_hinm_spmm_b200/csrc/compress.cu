@@ -383,6 +383,49 @@ size_t compress_workspace_bytes(int M, int K, int T) {
   return (((size_t)nt * K * sizeof(int32_t)) + 255) & ~size_t(255);
 }
 
+// Cross-layer index translation, one CTA per (block, tile) as pack_kernel: every index
+// entry c of the block becomes row_of_channel[c], then the block's run flag is recomputed
+// (first index when the entries are one ascending run, else -1).  An entry or map value
+// outside [0, K) is reported as HINM_ERR_INVALID_ARG and written as 0.
+__global__ void __launch_bounds__(kSparseBK) translate_index_kernel(
+    const int32_t* __restrict__ row_of_channel, int K, hinm_layout L, int* status) {
+  __shared__ int first;
+  const int t = blockIdx.y, b = blockIdx.x;
+  const int nd = L.tile_info[4 * t + 0], ns = L.tile_info[4 * t + 1];
+  if (b >= nd + ns) return;
+  const bool sparse = b >= nd;
+  const int nvec = sparse ? kSparseBK : kDenseBK;
+  int32_t* idx = sparse ? L.idx_sparse + (size_t)(L.tile_info[4 * t + 3] + b - nd) * kSparseBK
+                        : L.idx_dense + (size_t)(L.tile_info[4 * t + 2] + b) * kDenseBK;
+  int v = 0;
+  if ((int)threadIdx.x < nvec) {
+    const int c = idx[threadIdx.x];
+    if (c >= 0 && c < K) v = __ldg(row_of_channel + c);
+    if (c < 0 || c >= K || v < 0 || v >= K) {
+      ptx::record_status(status, HINM_ERR_INVALID_ARG);
+      v = 0;
+    }
+    idx[threadIdx.x] = v;
+  }
+  if (threadIdx.x == 0) first = v;
+  __syncthreads();
+  const bool step_ok = (int)threadIdx.x >= nvec || v == first + (int)threadIdx.x;
+  const bool run = __syncthreads_and(step_ok);
+  if (threadIdx.x == 0) {
+    if (sparse) L.run_sparse[L.tile_info[4 * t + 3] + b - nd] = run ? first : -1;
+    else L.run_dense[L.tile_info[4 * t + 2] + b] = run ? first : -1;
+  }
+}
+
+cudaError_t launch_translate_index(const hinm_layout& L, const int32_t* row_of_channel,
+                                   int* status, cudaStream_t s) {
+  const int nt = L.num_tiles, K = L.K;
+  if (nt <= 0) return cudaSuccess;
+  const int max_blocks = (K + kDenseBK - 1) / kDenseBK + (K + kSparseBK - 1) / kSparseBK;
+  translate_index_kernel<<<dim3(max_blocks, nt), kSparseBK, 0, s>>>(row_of_channel, K, L, status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_compress(const uint16_t* W, const uint32_t* bitmask, const int8_t* region,
                             const int32_t* perm, const int32_t* counts, int M, int K, int T,
                             const hinm_layout& L, void* ws, int* status, cudaStream_t s) {

@@ -130,6 +130,11 @@ def test_validation_rejects_before_launch(H):
     assert lib.hinm_boundary_search_stats(fake, fake, 8, None, 256, 256, 128, 0.5, 1 / 32, fake,
                                           fake, None, None, fake, 1 << 30,
                                           None) == H.HINM_ERR_INVALID_ARG
+    # index translation: a NULL map is refused, and so is a layout of another version
+    assert lib.hinm_translate_index(ctypes.byref(L), None, None) == H.HINM_ERR_INVALID_ARG
+    Lbad = H.hinm_layout(H.HINM_LAYOUT_VERSION + 1, 256, 256, 64, 4, 1, 1, fake, fake, fake, fake,
+                         fake, fake, fake, fake)
+    assert lib.hinm_translate_index(ctypes.byref(Lbad), fake, None) == H.HINM_ERR_INVALID_ARG
     # hinm_spmm_ex: unknown flag bits are refused before anything else; the hint flag
     # passes the same argument checks as hinm_spmm
     assert lib.hinm_spmm_ex(ctypes.byref(L), fake, 16, fake, 2, None) == H.HINM_ERR_INVALID_ARG

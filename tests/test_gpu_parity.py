@@ -196,6 +196,50 @@ def test_tile_pairs_mixed_modes_integer_bitwise(H, ntiles, N):
     np.testing.assert_array_equal(Y0.cpu().numpy().astype(np.int64), Wm @ Xi)
 
 
+@pytest.mark.parametrize("T,N,pairs", [(128, 264, False), (64, 40, False), (128, 1040, True)])
+def test_translate_index_layout_and_product(H, T, N, pairs):
+    """Cross-layer index translation on the GPU: the translated layout equals the oracle's
+    translation of the oracle's layout byte for byte, an identity map changes nothing, and
+    the product with the reordered X is bitwise the original product (integer inputs, also
+    equal to the exact masked product), with and without the tile-pair hint."""
+    K = 384
+    w = hi.integer_workload(3 * T, K, N, T, seed=21, t_s=0.625, v_s=None, random_perm=True)
+    g = run_path(H, w, v_s=0.375)
+    L = g["layout"]
+    X = dev_bf16(w.X_bits)
+    Y0 = H.hinm_spmm(L, X, tile_pairs=pairs).cpu().numpy()
+    H.hinm_translate_index(L, dev_i32(np.arange(K)))
+    torch.cuda.synchronize()
+    status_ok(H)
+    L_ref = O.compress(w.W_bits, g["bitmask"], g["region"], w.perm, g["counts_used"], T)
+    layout_equal(L, L_ref)
+    rng = np.random.default_rng(5)
+    sigma = rng.permutation(K).astype(np.int32)      # delivered row r holds channel sigma[r]
+    roc = np.argsort(sigma).astype(np.int32)
+    H.hinm_translate_index(L, dev_i32(roc))
+    X_del = dev_bf16(w.X_bits[sigma])
+    Y1 = H.hinm_spmm(L, X_del, tile_pairs=pairs).cpu().numpy()
+    torch.cuda.synchronize()
+    status_ok(H)
+    layout_equal(L, O.translate_index(L_ref, roc))
+    np.testing.assert_array_equal(Y1.view(np.uint32), Y0.view(np.uint32))
+    Wm = O.masked_weight(w.W_bits, g["bitmask"]).astype(np.int64)
+    np.testing.assert_array_equal(Y1.astype(np.int64), Wm @ hi.bf16_bits_to_f32(w.X_bits).astype(np.int64))
+
+
+def test_translate_index_bad_map_reported(H):
+    """A map entry outside [0, K) is reported as HINM_ERR_INVALID_ARG (and mapped to row 0),
+    not a fault; the context stays usable."""
+    w = hi.custom(128, 128, 16, 128, seed=4, t_s=0.5, v_s=None)
+    g = run_path(H, w, v_s=0.25)
+    bad = np.arange(128, dtype=np.int32)
+    bad[3] = 1 << 20
+    H.hinm_translate_index(g["layout"], dev_i32(bad))
+    torch.cuda.synchronize()
+    assert H.hinm_device_status() == H.HINM_ERR_INVALID_ARG
+    assert H.hinm_device_status() == 0
+
+
 def test_channel_energy_rounding_fallback(H):
     """Channels whose fp64 sum sits on an fp32 rounding midpoint: the order matters there,
     so the GPU must reproduce the sequential sum (1 first: 1.0; 1 last: 1 + 2^-23)."""
