@@ -591,3 +591,32 @@ def hot_path(W_bits: np.ndarray, X_bits: np.ndarray, perm: np.ndarray, T: int, t
     y, bound = spmm_reference(W_bits, bitmask, X_bits)
     return dict(I=I, search=sr, counts=counts, bitmask=bitmask, region=region,
                 layout=lay, y=y, bound=bound)
+
+
+# ---------------------------------------------------------------------------------------
+# Hard-Concrete soft 2:4 mask, forward
+# ---------------------------------------------------------------------------------------
+HC_LOW, HC_HIGH = -0.1, 1.1   # the stretch interval (-0.1, 1.1) of [P1] 关键设计 3
+
+
+def hard_concrete(log_alpha: np.ndarray, eps: np.ndarray, tau: float):
+    """Hard-Concrete forward over groups of 4 consecutive elements, in fp64.
+
+    [P1] 关键设计 3: with noise eps ~ U(0, 1) (an input here), the soft mask is
+    s = sigmoid((log eps - log(1 - eps) + log alpha) / tau), stretched to (-0.1, 1.1) and
+    clipped to [0, 1]: z = min(1, max(0, s * (1.1 - (-0.1)) + (-0.1))).  The two
+    regularisers are mean(z) (overall sparsity) and the mean over groups of |sum of the
+    group's 4 z - 2| (exactly two kept per group); the hardened mask thresholds z at 0.5.
+    [reading] "at 0.5" keeps z > 0.5; the regularisers are returned as sums (before their
+    means and weights): (sum z, sum over groups |sum z - 2|).
+    """
+    la = np.asarray(log_alpha, dtype=np.float64).ravel()
+    e = np.asarray(eps, dtype=np.float64).ravel()
+    if la.size % 4:
+        raise ValueError("elements come in groups of 4")
+    x = (np.log(e) - np.log1p(-e) + la) / float(tau)
+    s = 1.0 / (1.0 + np.exp(-x))
+    z = np.minimum(1.0, np.maximum(0.0, s * (HC_HIGH - HC_LOW) + HC_LOW))
+    hard = (z > 0.5).astype(np.uint8)
+    sums = np.array([z.sum(), np.abs(z.reshape(-1, 4).sum(axis=1) - 2.0).sum()])
+    return z, hard, sums

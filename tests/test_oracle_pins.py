@@ -503,3 +503,56 @@ def test_spmm_integer_exact():
     Wm = O.masked_weight(w.W_bits, r["bitmask"]).astype(np.int64)
     Xi = f32(w.X_bits).astype(np.int64)
     assert np.array_equal(r["y"].astype(np.int64), Wm @ Xi)
+
+
+# ----------------------------------------------------------------------------- Hard-Concrete
+def test_hard_concrete_closed_forms():
+    """eps = 1/2 and log alpha = 0 give s = 1/2, z = 1/2; s = 1/12 and s = 11/12 sit exactly on
+    the clip edges (z = 0, z = 1); large |log alpha| saturates to 0 / 1; the regularisers of
+    a binary mask with two ones per group are (n/2, 0)."""
+    tau = 2.0 / 3.0
+    logit = lambda p: math.log(p / (1.0 - p))
+    la = np.array([0.0, tau * logit(1 / 12), tau * logit(11 / 12), 60.0], dtype=np.float64)
+    z, hard, sums = O.hard_concrete(la, np.full(4, 0.5), tau)
+    # z[0] is 1/2 up to the fp64 rounding of the stretch (1.1 - (-0.1) is not exact), so its
+    # hardening is a tie and is not asserted
+    assert abs(z[0] - 0.5) < 1e-15
+    assert abs(z[1]) < 1e-15 and abs(z[2] - 1.0) < 1e-15 and z[3] == 1.0
+    np.testing.assert_array_equal(hard[1:], [0, 1, 1])
+    z2, _, s2 = O.hard_concrete(np.array([50.0, -50.0, 50.0, -50.0] * 3), np.full(12, 0.5), tau)
+    np.testing.assert_array_equal(z2, [1.0, 0.0] * 6)
+    np.testing.assert_array_equal(s2, [6.0, 0.0])
+
+
+def test_hard_concrete_mirror_and_regularisers():
+    """Flipping both the noise and the logit mirrors the mask: z(eps, a) + z(1 - eps, -a) = 1
+    (the logit changes sign, the stretch and the clip are symmetric about 1/2); the
+    regularisers equal their loops written out."""
+    rng = np.random.default_rng(3)
+    la = rng.normal(0, 2, 4096)
+    eps = rng.uniform(1e-6, 1 - 1e-6, 4096)
+    z, hard, sums = O.hard_concrete(la, eps, 0.5)
+    zm, _, _ = O.hard_concrete(-la, 1.0 - eps, 0.5)
+    assert np.abs(z + zm - 1.0).max() < 1e-12
+    want0 = math.fsum(z.tolist())
+    want1 = math.fsum(abs(math.fsum(z[4 * g:4 * g + 4].tolist()) - 2.0) for g in range(1024))
+    assert abs(sums[0] - want0) <= 1e-9 and abs(sums[1] - want1) <= 1e-9
+    np.testing.assert_array_equal(hard, (z > 0.5).astype(np.uint8))
+
+
+def test_hard_concrete_clip_mass_matches_the_logistic_law():
+    """With eps uniform, log(eps) - log(1 - eps) is logistic (CDF sigmoid), so
+    P(z = 0) = sigmoid(tau logit(1/12) - log alpha) and P(z = 1) = sigmoid(-tau logit(11/12)
+    + log alpha).  On 2^20 seeded draws the empirical masses match within 5 standard
+    deviations: this pins the sign of the noise and of log alpha and the stretch interval."""
+    n, tau, la0 = 1 << 20, 2.0 / 3.0, 0.7
+    rng = np.random.default_rng(9)
+    eps = rng.uniform(0.0, 1.0, n)
+    eps = np.clip(eps, 1e-12, 1 - 1e-12)
+    z, _, _ = O.hard_concrete(np.full(n, la0), eps, tau)
+    logit = lambda p: math.log(p / (1.0 - p))
+    sig = lambda x: 1.0 / (1.0 + math.exp(-x))
+    p0 = sig(tau * logit(1 / 12) - la0)
+    p1 = sig(-tau * logit(11 / 12) + la0)
+    for got, p in (((z == 0.0).mean(), p0), ((z == 1.0).mean(), p1)):
+        assert abs(got - p) < 5 * math.sqrt(p * (1 - p) / n), (got, p)
