@@ -327,6 +327,35 @@ def time_index_translate(H, hp, K, stream, reps=20):
             "note": "identity map on the step's layout; back-to-back calls (L2-warm)"}
 
 
+def time_hard_concrete(H, n, peaks, stream, reps=10):
+    """The Hard-Concrete forward over n = M*K elements (logits N(0, 2), noise U(0, 1), drawn
+    on the device from a fixed seed; tau = 2/3): CUDA events over `reps` back-to-back calls
+    after 3 untimed ones.  Algorithmic bytes: 4 (log alpha) + 4 (eps) in, 4 (z) + 1 (hard)
+    out per element; the arrays (13 B x n) exceed L2 at the benchmark sizes."""
+    import torch
+    g = torch.Generator(device="cuda").manual_seed(1234)
+    la = torch.randn(n, generator=g, device="cuda") * 2.0
+    eps = torch.rand(n, generator=g, device="cuda")
+    z = torch.empty(n, dtype=torch.float32, device="cuda")
+    hard = torch.empty(n, dtype=torch.uint8, device="cuda")
+    sums = torch.empty(2, dtype=torch.float64, device="cuda")
+    for _ in range(3):
+        H.hinm_hard_concrete_forward(la, eps, 2.0 / 3.0, z, hard, sums)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        H.hinm_hard_concrete_forward(la, eps, 2.0 / 3.0, z, hard, sums)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / 1e3 / reps
+    gbs = 13.0 * n / t / 1e9
+    peak = peaks.get("hbm_gbs") if peaks else None
+    return {"us_per_call": t * 1e6, "elements": n, "gbs": gbs, "bound": "hbm",
+            "peak_gbs": peak, "frac": (gbs / peak) if peak else None,
+            "kernel": "hard_concrete_kernel", "launches": 1,
+            "note": "back-to-back calls; 13 B per element, arrays larger than L2"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -551,7 +580,8 @@ def main():
                          "importance, search, mask, compress and fp64 masked product",
                "seconds": dt}
     clocks = sampler.summary()
-    next_rows = {"index_translate": time_index_translate(H, hp, K, stream)}
+    next_rows = {"index_translate": time_index_translate(H, hp, K, stream),
+                 "hard_concrete": time_hard_concrete(H, M * K, peaks, stream)}
     # this library's kernels per step: importance 2 (channel energies, importance with the
     # tile statistics), search 6 (chunk sort, merge rank, column sums, candidate lists, band
     # sums, finalize; V comes from the importance step), mask 2 (classify with the

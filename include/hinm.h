@@ -228,6 +228,23 @@ hinm_status hinm_compress(const void* W, const uint32_t* bitmask, const int8_t* 
                           const hinm_layout* layout, void* workspace,
                           size_t workspace_bytes, void* stream);
 
+/* Hard-Concrete soft 2:4 mask, forward  ([P1] 关键设计 3: each group of 4 has learnable
+ * logits log alpha; with noise eps ~ U(0, 1) the soft mask is
+ *   s = sigmoid((log eps - log(1 - eps) + log alpha) / tau),
+ * stretched to (-0.1, 1.1) and clipped to [0, 1]; the regularisers are mean(z) and the mean
+ * over groups of |sum of the group's z - 2|; the hardened mask thresholds z at 0.5).
+ *   z_i = min(1, max(0, 1.2 s_i - 0.1)) (fp32, with CUDA's logf / log1pf / expf)
+ * log_alpha, eps: device fp32 [n], n % 4 == 0, groups = 4 consecutive elements; eps is the
+ * caller's noise (eps = 1/2 everywhere gives the deterministic mask; eps = 0 or 1 give
+ * z = 0 or 1; NaN in, NaN out).  tau > 0.
+ * z_out: fp32 [n].  hard_out (NULL allowed): uint8 [n], 1 where z > 0.5.
+ * sums_out (NULL allowed): fp64 [2] = { sum z, sum over groups |sum z - 2| } (zeroed by the
+ * call, then added to in an unspecified order: the last bits may differ between calls).
+ * Errors: HINM_ERR_SHAPE (n), HINM_ERR_INVALID_ARG (tau, NULL), HINM_ERR_ALIGNMENT. */
+hinm_status hinm_hard_concrete_forward(const float* log_alpha, const float* eps, long long n,
+                                       float tau, float* z_out, uint8_t* hard_out,
+                                       double* sums_out, void* stream);
+
 /* Cross-layer index translation  ([P1] 关键设计 2: channel reordering leaves the result
  * unchanged, and the translation between layers is folded into the HiNM index).
  * For an X whose rows arrive reordered -- row r holds input channel sigma[r], e.g. the

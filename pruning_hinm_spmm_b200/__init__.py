@@ -81,6 +81,8 @@ _SIGS = {
     "hinm_compress": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
                              ctypes.POINTER(hinm_layout), _vp, _sz, _vp]),
     "hinm_translate_index": (_i32, [ctypes.POINTER(hinm_layout), _vp, _vp]),
+    "hinm_hard_concrete_forward": (_i32, [_vp, _vp, ctypes.c_longlong, ctypes.c_float, _vp, _vp,
+                                          _vp, _vp]),
     "hinm_spmm": (_i32, [ctypes.POINTER(hinm_layout), _vp, _i32, _vp, _vp]),
     "hinm_spmm_ex": (_i32, [ctypes.POINTER(hinm_layout), _vp, _i32, _vp, _i32, _vp]),
     "hinm_device_status": (_i32, [_vp, ctypes.POINTER(ctypes.c_int32)]),
@@ -372,6 +374,25 @@ def hinm_translate_index(layout: HinmLayout, row_of_channel, stream=None,
     _check(_lib.hinm_translate_index(ctypes.byref(c), _ptr(row_of_channel), _stream(stream)),
            "hinm_translate_index")
     return layout
+
+
+def hinm_hard_concrete_forward(log_alpha, eps, tau: float, z_out=None, hard_out=None,
+                               sums_out=None, stream=None):
+    """Hard-Concrete soft 2:4 mask (fp32 [n], groups of 4): returns (z, hard uint8 [n],
+    sums fp64 [2] = (sum z, sum over groups |sum z - 2|))."""
+    torch = _torch()
+    n = log_alpha.numel()
+    dev = log_alpha.device
+    if z_out is None:
+        z_out = torch.empty(n, dtype=torch.float32, device=dev)
+    if hard_out is None:
+        hard_out = torch.empty(n, dtype=torch.uint8, device=dev)
+    if sums_out is None:
+        sums_out = torch.empty(2, dtype=torch.float64, device=dev)
+    _check(_lib.hinm_hard_concrete_forward(_ptr(log_alpha), _ptr(eps), n, float(tau), _ptr(z_out),
+                                           _ptr(hard_out), _ptr(sums_out), _stream(stream)),
+           "hinm_hard_concrete_forward")
+    return z_out, hard_out, sums_out
 
 
 def hinm_device_status(stream=None) -> int:

@@ -487,6 +487,24 @@ hinm_status hinm_compress(const void* W, const uint32_t* bitmask, const int8_t* 
   return ok();
 }
 
+hinm_status hinm_hard_concrete_forward(const float* log_alpha, const float* eps, long long n,
+                                      float tau, float* z_out, uint8_t* hard_out,
+                                      double* sums_out, void* stream) {
+  REQUIRE_PTR(log_alpha);
+  REQUIRE_PTR(eps);
+  REQUIRE_PTR(z_out);
+  REQUIRE_ALIGNED_OR_NULL(hard_out);
+  REQUIRE_ALIGNED_OR_NULL(sums_out);
+  if (n <= 0 || n % 4 != 0)
+    return fail(HINM_ERR_SHAPE, "n=%lld must be a positive multiple of 4", n);
+  if (!(tau > 0.0f) || !std::isfinite(tau))
+    return fail(HINM_ERR_INVALID_ARG, "tau=%g must be positive and finite", (double)tau);
+  cudaError_t e = hinm::launch_hard_concrete(log_alpha, eps, n, tau, z_out, hard_out, sums_out,
+                                             static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "hinm_hard_concrete_forward launch");
+  return ok();
+}
+
 hinm_status hinm_translate_index(const hinm_layout* layout, const int32_t* row_of_channel,
                                 void* stream) {
   hinm_status st = check_layout(layout);

@@ -91,6 +91,9 @@ cudaError_t launch_wait_timeout_selftest(unsigned long long limit_ns, int* statu
                                          cudaStream_t s);
 
 // tile_pairs: the caller's hint that tiles select the same X rows (HINM_SPMM_TILE_PAIRS)
+cudaError_t launch_hard_concrete(const float* log_alpha, const float* eps, long long n, float tau,
+                                 float* z, uint8_t* hard, double* sums, cudaStream_t s);
+
 cudaError_t launch_translate_index(const hinm_layout& L, const int32_t* row_of_channel,
                                    int* status, cudaStream_t s);
 

@@ -130,6 +130,16 @@ def test_validation_rejects_before_launch(H):
     assert lib.hinm_boundary_search_stats(fake, fake, 8, None, 256, 256, 128, 0.5, 1 / 32, fake,
                                           fake, None, None, fake, 1 << 30,
                                           None) == H.HINM_ERR_INVALID_ARG
+    # Hard-Concrete: n a positive multiple of 4, tau positive and finite, pointers aligned
+    assert lib.hinm_hard_concrete_forward(fake, fake, ctypes.c_longlong(6), ctypes.c_float(0.5),
+                                          fake, None, None, None) == H.HINM_ERR_SHAPE
+    assert lib.hinm_hard_concrete_forward(fake, fake, ctypes.c_longlong(8), ctypes.c_float(0.0),
+                                          fake, None, None, None) == H.HINM_ERR_INVALID_ARG
+    assert lib.hinm_hard_concrete_forward(fake, fake, ctypes.c_longlong(8),
+                                          ctypes.c_float(float("inf")), fake, None, None,
+                                          None) == H.HINM_ERR_INVALID_ARG
+    assert lib.hinm_hard_concrete_forward(fake + 4, fake, ctypes.c_longlong(8), ctypes.c_float(0.5),
+                                          fake, None, None, None) == H.HINM_ERR_ALIGNMENT
     # index translation: a NULL map is refused, and so is a layout of another version
     assert lib.hinm_translate_index(ctypes.byref(L), None, None) == H.HINM_ERR_INVALID_ARG
     Lbad = H.hinm_layout(H.HINM_LAYOUT_VERSION + 1, 256, 256, 64, 4, 1, 1, fake, fake, fake, fake,

@@ -240,6 +240,67 @@ def test_translate_index_bad_map_reported(H):
     assert H.hinm_device_status() == 0
 
 
+def _hc_bound(la, eps, tau):
+    """Per-element bound on |z_fp32 - z_fp64| from the fp32 operation order of the kernel:
+    logf and log1pf within 1 ulp, expf within 2 ulp (CUDA's documented maxima), each fp32
+    add / multiply / divide within half an ulp, carried through the sigmoid's slope s(1 - s)
+    and the stretch by 1.2; plus the fp32 stretch constants' offset from the fp64 ones."""
+    d = 2.0 ** -24
+    la = la.astype(np.float64)
+    e = eps.astype(np.float64)
+    l1, l2 = np.abs(np.log(e)), np.abs(np.log1p(-e))
+    logit = np.log(e) - np.log1p(-e)
+    err_logit = (l1 + l2) * 2 * d + np.abs(logit) * d
+    x = (logit + la) / tau
+    err_x = (err_logit + np.abs(logit + la) * d) / tau + np.abs(x) * d
+    s = 1.0 / (1.0 + np.exp(-x))
+    err_s = s * (1 - s) * err_x + 8 * d * s
+    return 2.0 * (1.2 * err_s + 1.2 * s * 1e-7 + 4 * d + 4e-9)
+
+
+@pytest.mark.parametrize("n,tau", [(4 * 10007, 2.0 / 3.0), (4 * 262147, 0.1), (1 << 22, 1.0)])
+def test_hard_concrete_forward_matches_oracle(H, n, tau):
+    """The Hard-Concrete forward on the GPU against the fp64 oracle: z within the fp32
+    bound per element, the hardened bits exactly (z > 0.5) of the GPU's own z, and both
+    regularisers within the summed bound; noise at the ends (eps = 0, 1) gives z = 0, 1."""
+    rng = np.random.default_rng(n)
+    la = rng.normal(0.0, 2.0, n).astype(np.float32)
+    eps = rng.uniform(0.0, 1.0, n).astype(np.float32)
+    eps[:4] = (0.0, 1.0, 0.5, 0.5)
+    la[2:4] = (0.0, 40.0)
+    z, hard, sums = H.hinm_hard_concrete_forward(torch.from_numpy(la).cuda(),
+                                                 torch.from_numpy(eps).cuda(), tau)
+    torch.cuda.synchronize()
+    z, hard, sums = z.cpu().numpy(), hard.cpu().numpy(), sums.cpu().numpy()
+    assert tuple(z[:4]) == (0.0, 1.0, z[2], 1.0) and abs(z[2] - 0.5) < 1e-6
+    inner = slice(4, None)
+    z_ref, _, _ = O.hard_concrete(la[inner], eps[inner], tau)
+    bound = _hc_bound(la[inner], eps[inner], tau)
+    err = np.abs(z[inner].astype(np.float64) - z_ref)
+    assert (err <= bound).all(), f"worst excess {(err - bound).max():.3e}"
+    np.testing.assert_array_equal(hard, (z > 0.5).astype(np.uint8))
+    # the first group's reference from the GPU's own values (the ends of the noise range)
+    s0 = float(z[:4].astype(np.float64).sum())
+    want_z = s0 + float(z_ref.sum())
+    want_h = abs(s0 - 2.0) + float(np.abs(z_ref.reshape(-1, 4).sum(axis=1) - 2.0).sum())
+    tol = float(bound.sum()) * 4 + 1e-9 * n
+    assert abs(sums[0] - want_z) <= tol and abs(sums[1] - want_h) <= tol
+
+
+def test_hard_concrete_deterministic_mode(H):
+    """eps = 1/2 removes the noise: z = clip(1.2 sigmoid(log alpha / tau) - 0.1) exactly as
+    the oracle's deterministic mask, with the hardened mask at 0.5."""
+    n, tau = 4096, 0.5
+    la = np.linspace(-3.0, 3.0, n).astype(np.float32)
+    eps = np.full(n, 0.5, dtype=np.float32)
+    z, hard, _ = H.hinm_hard_concrete_forward(torch.from_numpy(la).cuda(),
+                                              torch.from_numpy(eps).cuda(), tau)
+    z = z.cpu().numpy()
+    z_ref, _, _ = O.hard_concrete(la, eps, tau)
+    assert (np.abs(z - z_ref) <= _hc_bound(la, eps, tau)).all()
+    assert (z[la < -1.0] < 0.5).all() and (z[la > 1.0] > 0.5).all()
+
+
 def test_channel_energy_rounding_fallback(H):
     """Channels whose fp64 sum sits on an fp32 rounding midpoint: the order matters there,
     so the GPU must reproduce the sequential sum (1 first: 1.0; 1 last: 1 + 2^-23)."""
