@@ -26,10 +26,11 @@ int hc_sm_count() {
   return n > 0 ? n : 148;
 }
 
-__device__ __forceinline__ float hc_z(float la, float e, float tau) {
+// inv_tau = fl32(1 / tau); the reciprocal of 1 + exp(-x) is the correctly rounded one
+__device__ __forceinline__ float hc_z(float la, float e, float inv_tau) {
   const float logit = __fsub_rn(logf(e), log1pf(-e));   // log eps - log(1 - eps)
-  const float x = __fdiv_rn(__fadd_rn(logit, la), tau);
-  const float s = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-x)));
+  const float x = __fmul_rn(__fadd_rn(logit, la), inv_tau);
+  const float s = __frcp_rn(__fadd_rn(1.0f, expf(-x)));
   const float sb = __fadd_rn(__fmul_rn(s, __fsub_rn(kHcHigh, kHcLow)), kHcLow);
   return fminf(1.0f, fmaxf(0.0f, sb));
 }
@@ -39,6 +40,7 @@ __global__ void __launch_bounds__(kHcThreads) hard_concrete_kernel(
     float tau, float4* __restrict__ z, uchar4* __restrict__ hard, double* __restrict__ sums) {
   __shared__ double red[2][kHcThreads / 32];
   double acc_z = 0.0, acc_h = 0.0;
+  const float inv_tau = __frcp_rn(tau);
   const long long stride = (long long)gridDim.x * blockDim.x;
   for (long long g0 = blockIdx.x * (long long)blockDim.x + threadIdx.x; g0 < ngroups;
        g0 += stride * kHcUnroll) {
@@ -56,10 +58,10 @@ __global__ void __launch_bounds__(kHcThreads) hard_concrete_kernel(
       const long long g = g0 + u * stride;
       if (g >= ngroups) break;
       float4 o;
-      o.x = hc_z(a[u].x, e[u].x, tau);
-      o.y = hc_z(a[u].y, e[u].y, tau);
-      o.z = hc_z(a[u].z, e[u].z, tau);
-      o.w = hc_z(a[u].w, e[u].w, tau);
+      o.x = hc_z(a[u].x, e[u].x, inv_tau);
+      o.y = hc_z(a[u].y, e[u].y, inv_tau);
+      o.z = hc_z(a[u].z, e[u].z, inv_tau);
+      o.w = hc_z(a[u].w, e[u].w, inv_tau);
       __stcs(z + g, o);
       if (hard)
         hard[g] = make_uchar4(o.x > 0.5f, o.y > 0.5f, o.z > 0.5f, o.w > 0.5f);

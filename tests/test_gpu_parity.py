@@ -243,8 +243,9 @@ def test_translate_index_bad_map_reported(H):
 def _hc_bound(la, eps, tau):
     """Per-element bound on |z_fp32 - z_fp64| from the fp32 operation order of the kernel:
     logf and log1pf within 1 ulp, expf within 2 ulp (CUDA's documented maxima), each fp32
-    add / multiply / divide within half an ulp, carried through the sigmoid's slope s(1 - s)
-    and the stretch by 1.2; plus the fp32 stretch constants' offset from the fp64 ones."""
+    add / multiply / reciprocal within half an ulp (the scale by 1/tau: the reciprocal's and
+    the product's roundings), carried through the sigmoid's slope s(1 - s) and the stretch by
+    1.2; plus the fp32 stretch constants' offset from the fp64 ones."""
     d = 2.0 ** -24
     la = la.astype(np.float64)
     e = eps.astype(np.float64)
@@ -252,7 +253,7 @@ def _hc_bound(la, eps, tau):
     logit = np.log(e) - np.log1p(-e)
     err_logit = (l1 + l2) * 2 * d + np.abs(logit) * d
     x = (logit + la) / tau
-    err_x = (err_logit + np.abs(logit + la) * d) / tau + np.abs(x) * d
+    err_x = (err_logit + np.abs(logit + la) * d) / tau + np.abs(x) * 3 * d
     s = 1.0 / (1.0 + np.exp(-x))
     err_s = s * (1 - s) * err_x + 8 * d * s
     return 2.0 * (1.2 * err_s + 1.2 * s * 1e-7 + 4 * d + 4e-9)
