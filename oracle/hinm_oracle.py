@@ -620,3 +620,36 @@ def hard_concrete(log_alpha: np.ndarray, eps: np.ndarray, tau: float):
     hard = (z > 0.5).astype(np.uint8)
     sums = np.array([z.sum(), np.abs(z.reshape(-1, 4).sum(axis=1) - 2.0).sum()])
     return z, hard, sums
+
+
+# ---------------------------------------------------------------------------------------
+# SpMM epilogue: bias, activation, bf16 output
+# ---------------------------------------------------------------------------------------
+ACT_NONE, ACT_RELU, ACT_SILU, ACT_GELU = 0, 1, 2, 3
+
+
+def activation(x: np.ndarray, act: int) -> np.ndarray:
+    """The epilogue's activations in fp64.  [reading] The pages name none; these are the
+    common ones of the linears the method prunes: ReLU max(x, 0), SiLU x sigmoid(x), GELU
+    x Phi(x) = x (1 + erf(x / sqrt 2)) / 2 (the erf form)."""
+    x = np.asarray(x, dtype=np.float64)
+    if act == ACT_NONE:
+        return x.copy()
+    if act == ACT_RELU:
+        return np.maximum(x, 0.0)
+    if act == ACT_SILU:
+        return x / (1.0 + np.exp(-x))
+    if act == ACT_GELU:
+        erf = np.vectorize(math.erf)
+        return 0.5 * x * (1.0 + erf(x / math.sqrt(2.0)))
+    raise ValueError(f"activation {act}")
+
+
+def spmm_epilogue_reference(y: np.ndarray, bias: Optional[np.ndarray], act: int) -> np.ndarray:
+    """act(y + bias[row]) in fp64 on the SpMM's fp64 reference product ([P1] 关键设计 4:
+    the one output of the dense and 2:4 parts; [reading] the bias is per output row of Y,
+    i.e. per output channel of the layer)."""
+    z = np.asarray(y, dtype=np.float64)
+    if bias is not None:
+        z = z + np.asarray(bias, dtype=np.float64)[:, None]
+    return activation(z, act)

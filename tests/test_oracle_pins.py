@@ -556,3 +556,28 @@ def test_hard_concrete_clip_mass_matches_the_logistic_law():
     p1 = sig(-tau * logit(11 / 12) + la0)
     for got, p in (((z == 0.0).mean(), p0), ((z == 1.0).mean(), p1)):
         assert abs(got - p) < 5 * math.sqrt(p * (1 - p) / n), (got, p)
+
+
+# ----------------------------------------------------------------------------- SpMM epilogue
+def test_activation_closed_forms_and_identities():
+    """ReLU, SiLU, GELU: values at 0 and at known points, SiLU(x) - SiLU(-x) = x and
+    GELU(x) - GELU(-x) = x (sigmoid(x) + sigmoid(-x) = 1, Phi(x) + Phi(-x) = 1), GELU(1) =
+    Phi(1) = 0.8413447460685429..., SiLU(1) = 1 / (1 + e^-1)."""
+    x = np.linspace(-6.0, 6.0, 241)
+    np.testing.assert_array_equal(O.activation(x, O.ACT_NONE), x)
+    np.testing.assert_array_equal(O.activation(x, O.ACT_RELU), np.where(x > 0, x, 0.0))
+    for act in (O.ACT_SILU, O.ACT_GELU):
+        d = O.activation(x, act) - O.activation(-x, act)
+        assert np.abs(d - x).max() < 1e-14
+        assert O.activation(np.array([0.0]), act)[0] == 0.0
+    assert abs(O.activation(np.array([1.0]), O.ACT_GELU)[0] - 0.8413447460685429) < 1e-15
+    assert abs(O.activation(np.array([1.0]), O.ACT_SILU)[0] - 1.0 / (1.0 + math.exp(-1.0))) < 1e-15
+
+
+def test_epilogue_reference_bias_per_row():
+    """The bias is added per output row (output channel) before the activation."""
+    y = np.arange(12, dtype=np.float64).reshape(3, 4) - 5.0
+    b = np.array([1.0, -2.0, 0.5])
+    got = O.spmm_epilogue_reference(y, b, O.ACT_RELU)
+    np.testing.assert_array_equal(got, np.maximum(y + b[:, None], 0.0))
+    np.testing.assert_array_equal(O.spmm_epilogue_reference(y, None, O.ACT_NONE), y)
