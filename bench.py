@@ -327,6 +327,39 @@ def time_index_translate(H, hp, K, stream, reps=20):
             "note": "identity map on the step's layout; back-to-back calls (L2-warm)"}
 
 
+def time_epilogue(H, hp, X, M, N, tile_pairs, flush, stream, reps=10):
+    """The SpMM with the fused epilogue (per-row bias, GELU, bf16 Y) against the plain fp32
+    SpMM on this step's layout: each call timed alone by CUDA events after the 256 MB L2
+    flush, the median of `reps`; Y bytes halve (4 -> 2 per output)."""
+    import torch
+    bias = torch.linspace(-0.1, 0.1, M, device=X.device, dtype=torch.float32)
+    yb = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+
+    def timed(fn):
+        ts = []
+        for i in range(reps + 2):
+            flush.fill_(i & 0xFF)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if i >= 2:
+                ts.append(e0.elapsed_time(e1) * 1e3)
+        return float(np.median(ts))
+
+    t_plain = timed(lambda: H.hinm_spmm(hp.layout, X, hp.Y, None, hp.c_layout, tile_pairs))
+    t_epi = timed(lambda: H.hinm_spmm_epilogue(hp.layout, X, bias, H.HINM_ACT_GELU, True, yb,
+                                               None, hp.c_layout, tile_pairs))
+    st = H.hinm_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after the epilogue timing")
+    return {"us_plain_fp32": t_plain, "us_bias_gelu_bf16": t_epi,
+            "y_bytes_fp32": 4 * M * N, "y_bytes_bf16": 2 * M * N,
+            "kernel": "same SpMM kernel, epilogue fused", "launches": 1,
+            "note": "one call per timing after the L2 flush; median of %d" % reps}
+
+
 def time_hard_concrete(H, n, peaks, stream, reps=10):
     """The Hard-Concrete forward over n = M*K elements (logits N(0, 2), noise U(0, 1), drawn
     on the device from a fixed seed; tau = 2/3): CUDA events over `reps` back-to-back calls
@@ -581,7 +614,8 @@ def main():
                "seconds": dt}
     clocks = sampler.summary()
     next_rows = {"index_translate": time_index_translate(H, hp, K, stream),
-                 "hard_concrete": time_hard_concrete(H, M * K, peaks, stream)}
+                 "hard_concrete": time_hard_concrete(H, M * K, peaks, stream),
+                 "epilogue_bf16": time_epilogue(H, hp, X, M, N, tile_pairs, flush, stream)}
     # this library's kernels per step: importance 2 (channel energies, importance with the
     # tile statistics), search 6 (chunk sort, merge rank, column sums, candidate lists, band
     # sums, finalize; V comes from the importance step), mask 2 (classify with the

@@ -281,6 +281,23 @@ hinm_status hinm_spmm(const hinm_layout* layout, const void* X, int N, float* Y_
 hinm_status hinm_spmm_ex(const hinm_layout* layout, const void* X, int N, float* Y_out,
                          int flags, void* stream);
 
+/* hinm_spmm_ex with a fused epilogue (an extension of a6: the pages merge the two
+ * parts into one output and name no epilogue; [reading] per output row bias, an activation
+ * and a bf16 output, applied to the fp32 accumulator before the one store of Y):
+ *   y[i, n] = act(acc[i, n] + bias[i])   (bias NULL: 0; act HINM_ACT_*)
+ * stored as fp32 to Y_out (fp32 [M][N]) or, with out_bf16 != 0, as bf16 (round to nearest
+ * even) to Y_out (bf16 [M][N]), which halves the bytes of Y.  ReLU max(x, 0); SiLU
+ * x / (1 + exp(-x)); GELU x (1 + erf(x / sqrt 2)) / 2 -- with CUDA's expf and erff.
+ * bias: device fp32 [M] or NULL.  Errors: as hinm_spmm_ex, plus HINM_ERR_INVALID_ARG for an
+ * unknown activation. */
+#define HINM_ACT_NONE 0
+#define HINM_ACT_RELU 1
+#define HINM_ACT_SILU 2
+#define HINM_ACT_GELU 3
+hinm_status hinm_spmm_epilogue(const hinm_layout* layout, const void* X, int N, void* Y_out,
+                               const float* bias, int activation, int out_bf16, int flags,
+                               void* stream);
+
 /* Diagnostic with no counterpart in the pages: launches one small kernel whose bounded
  * wait cannot complete (it waits on an mbarrier nothing arrives at), so that after about
  * limit_ns nanoseconds it records HINM_ERR_DEVICE_TIMEOUT and returns, exercising the

@@ -26,7 +26,7 @@ the pages leave the precision open.  Sources (page title, section):
   the mask is chosen on the permuted importance S·P, i.e. in working order.
 * [P5] "非结构化剪枝与结构化剪枝" (apxml.com), 结构化剪枝: removing a whole column.
 
-Readings where the pages are silent are marked [reading] and are listed in the design doc.
+Readings where the pages are silent are marked [reading] at the step that takes them.
 
 Parity pins: every function here is pinned by ``tests/test_oracle_pins.py`` against
 closed forms, brute force on tiny inputs, exact rational arithmetic, invariants and the
@@ -354,7 +354,7 @@ def unpack_bits(bitmask: np.ndarray, K: int) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------------------
-# a5. compress -- the HiNM layout (documented byte for byte in the design doc)
+# a5. compress -- the HiNM layout (byte for byte as include/hinm.h documents it)
 # ---------------------------------------------------------------------------------------
 def swizzled_offset(r: int, k: int) -> int:
     """Byte offset of bf16 element (row r, column k) in a 128-row x 64-column block.

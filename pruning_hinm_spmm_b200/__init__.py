@@ -27,6 +27,7 @@ HINM_ERR_BAD_MASK = 7
 HINM_ERR_WORKSPACE = 8
 HINM_LAYOUT_VERSION = 2
 HINM_SPMM_TILE_PAIRS = 1   # hinm_spmm_ex flag
+HINM_ACT_NONE, HINM_ACT_RELU, HINM_ACT_SILU, HINM_ACT_GELU = 0, 1, 2, 3
 
 REGION_PRUNED, REGION_24, REGION_DENSE = 0, 1, 2
 
@@ -85,6 +86,8 @@ _SIGS = {
                                           _vp, _vp]),
     "hinm_spmm": (_i32, [ctypes.POINTER(hinm_layout), _vp, _i32, _vp, _vp]),
     "hinm_spmm_ex": (_i32, [ctypes.POINTER(hinm_layout), _vp, _i32, _vp, _i32, _vp]),
+    "hinm_spmm_epilogue": (_i32, [ctypes.POINTER(hinm_layout), _vp, _i32, _vp, _vp, _i32, _i32,
+                                  _i32, _vp]),
     "hinm_device_status": (_i32, [_vp, ctypes.POINTER(ctypes.c_int32)]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -363,6 +366,23 @@ def hinm_spmm(layout: HinmLayout, X, Y_out=None, stream=None, c_layout: Optional
     else:
         _check(_lib.hinm_spmm(ctypes.byref(c), _ptr(X), N, _ptr(Y_out), _stream(stream)),
                "hinm_spmm")
+    return Y_out
+
+
+def hinm_spmm_epilogue(layout: HinmLayout, X, bias=None, activation: int = HINM_ACT_NONE,
+                       out_bf16: bool = False, Y_out=None, stream=None,
+                       c_layout: Optional[hinm_layout] = None, tile_pairs: bool = False):
+    """Y = act(W_HiNM . X + bias[row]) as fp32 or bf16 [M, N] (bias fp32 [M] or None)."""
+    torch = _torch()
+    N = X.shape[1]
+    if Y_out is None:
+        Y_out = torch.empty((layout.M, N), dtype=torch.bfloat16 if out_bf16 else torch.float32,
+                            device=X.device)
+    c = c_layout if c_layout is not None else layout.as_c()
+    _check(_lib.hinm_spmm_epilogue(ctypes.byref(c), _ptr(X), N, _ptr(Y_out), _ptr(bias),
+                                   int(activation), 1 if out_bf16 else 0,
+                                   HINM_SPMM_TILE_PAIRS if tile_pairs else 0, _stream(stream)),
+           "hinm_spmm_epilogue")
     return Y_out
 
 

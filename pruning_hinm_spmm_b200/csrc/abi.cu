@@ -523,14 +523,25 @@ hinm_status hinm_spmm(const hinm_layout* layout, const void* X, int N, float* Y_
 
 hinm_status hinm_spmm_ex(const hinm_layout* layout, const void* X, int N, float* Y_out,
                          int flags, void* stream) {
+  return hinm_spmm_epilogue(layout, X, N, Y_out, nullptr, HINM_ACT_NONE, 0, flags, stream);
+}
+
+hinm_status hinm_spmm_epilogue(const hinm_layout* layout, const void* X, int N, void* Y_out,
+                               const float* bias, int activation, int out_bf16, int flags,
+                               void* stream) {
   if (flags & ~HINM_SPMM_TILE_PAIRS) return fail(HINM_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (activation < HINM_ACT_NONE || activation > HINM_ACT_GELU)
+    return fail(HINM_ERR_INVALID_ARG, "unknown activation %d", activation);
+  REQUIRE_ALIGNED_OR_NULL(bias);
   hinm_status st = check_layout(layout);
   if (st != HINM_OK) return st;
   REQUIRE_PTR(X);
   REQUIRE_PTR(Y_out);
   st = check_n(N);
   if (st != HINM_OK) return st;
-  cudaError_t e = hinm::launch_spmm(*layout, static_cast<const uint16_t*>(X), N, Y_out,
+  hinm::SpmmOut out{out_bf16 ? nullptr : static_cast<float*>(Y_out),
+                     out_bf16 ? static_cast<uint16_t*>(Y_out) : nullptr, bias, activation};
+  cudaError_t e = hinm::launch_spmm(*layout, static_cast<const uint16_t*>(X), N, out,
                                     (flags & HINM_SPMM_TILE_PAIRS) != 0,
                                     hinm::device_status_ptr(), static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "hinm_spmm launch");

@@ -97,7 +97,16 @@ cudaError_t launch_hard_concrete(const float* log_alpha, const float* eps, long 
 cudaError_t launch_translate_index(const hinm_layout& L, const int32_t* row_of_channel,
                                    int* status, cudaStream_t s);
 
-cudaError_t launch_spmm(const hinm_layout& L, const uint16_t* X, int N, float* Y,
+// The SpMM's output: y = act(acc + bias[row]) stored as fp32 to Y, or as bf16 to Yb when Yb
+// is set (then Y is unused); bias per output row or nullptr; act one of HINM_ACT_*.
+// tile_pairs: the caller's hint that tiles select the same X rows (HINM_SPMM_TILE_PAIRS).
+struct SpmmOut {
+  float* Y;
+  uint16_t* Yb;
+  const float* bias;
+  int act;
+};
+cudaError_t launch_spmm(const hinm_layout& L, const uint16_t* X, int N, const SpmmOut& o,
                         bool tile_pairs, int* status, cudaStream_t s);
 
 // Shared by the rank users (search and mask): V (fp64 column sums per tile) and the rank

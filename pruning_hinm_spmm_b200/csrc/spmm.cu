@@ -36,6 +36,7 @@
 // HINM_ERR_DEVICE_TIMEOUT, stops all roles, drains what it issued, frees tensor memory and
 // returns.
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
@@ -113,7 +114,30 @@ struct SpmmArgs {
   int split;  // CTAs (one cluster) per unit; 1 = persistent, no split
   int x3d;    // the X tensor map is 3-D (columns within an atom, rows, atoms)
   int* status;
+  // epilogue: y = act(acc + bias[row]), stored as fp32 to Y or, when Yb is set, as bf16 to Yb
+  const float* bias;  // per output row, or nullptr
+  int act;            // HINM_ACT_*
+  uint16_t* Yb;
 };
+
+__device__ __forceinline__ float epi_act(float x, int act) {
+  if (act == HINM_ACT_RELU) return fmaxf(x, 0.0f);
+  if (act == HINM_ACT_SILU) return __fdiv_rn(x, __fadd_rn(1.0f, expf(-x)));
+  if (act == HINM_ACT_GELU)
+    return __fmul_rn(__fmul_rn(0.5f, x), __fadd_rn(1.0f, erff(__fmul_rn(x, 0.70710678118654752f))));
+  return x;
+}
+// v[0..n): fp32 bits of one row's accumulator columns -> act(v + b)
+template <int NV>
+__device__ __forceinline__ void epi_apply(uint32_t (&v)[32], float b, int act) {
+#pragma unroll
+  for (int i = 0; i < NV; ++i) v[i] = __float_as_uint(epi_act(__fadd_rn(__uint_as_float(v[i]), b), act));
+}
+// bf16 (round to nearest even) of two fp32 bit patterns, packed low | high << 16
+__device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo, uint32_t hi) {
+  const __nv_bfloat162 h = __float22bfloat162_rn(make_float2(__uint_as_float(lo), __uint_as_float(hi)));
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
 
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
@@ -158,6 +182,75 @@ struct Gather {
     }
   }
 };
+
+// One warp's 32 rows x cw (<= 32, a multiple of 8) columns of Y: lane l holds row r0 + l's
+// values v.  They go through the warp's swizzled 4 KB shared tile (16-byte pieces, piece
+// slot XOR row mod 8) and out as row segments: 128 bytes of 4 rows per fp32 store
+// instruction, 64 bytes of 8 rows per bf16 one.  rows are tile rows (rows >= T not stored).
+__device__ __forceinline__ void store_chunk32(const SpmmArgs& a, uint32_t ep, uint32_t (&v)[32],
+                                              int lane, int r0, int tile, int gc0, int cw) {
+  if (a.Yb) {
+    uint32_t h[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) h[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+      ptx::st_shared_v4(ep + lane * 128 + ((p ^ (lane & 7)) << 4), h[4 * p], h[4 * p + 1],
+                        h[4 * p + 2], h[4 * p + 3]);
+    __syncwarp();
+    const int rr = lane >> 2, pc = lane & 3;
+    const int gc = gc0 + 8 * pc;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = 8 * i + rr;
+      const uint4 o = ptx::ld_shared_v4(ep + r * 128 + ((pc ^ (r & 7)) << 4));
+      const int rw = r0 + r;
+      if (8 * pc < cw && rw < a.T)
+        *reinterpret_cast<uint4*>(a.Yb + (size_t)(tile * a.T + rw) * a.N + gc) = o;
+    }
+  } else {
+#pragma unroll
+    for (int p = 0; p < 8; ++p)
+      ptx::st_shared_v4(ep + lane * 128 + ((p ^ (lane & 7)) << 4), v[4 * p], v[4 * p + 1],
+                        v[4 * p + 2], v[4 * p + 3]);
+    __syncwarp();
+    const int rr = lane >> 3, pc = lane & 7;
+    const int gc = gc0 + 4 * pc;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = 4 * i + rr;
+      const uint4 o = ptx::ld_shared_v4(ep + r * 128 + ((pc ^ (r & 7)) << 4));
+      const int rw = r0 + r;
+      if (4 * pc < cw && rw < a.T)
+        *reinterpret_cast<uint4*>(a.Y + (size_t)(tile * a.T + rw) * a.N + gc) = o;
+    }
+  }
+  __syncwarp();  // the tile is rewritten by the next chunk
+}
+
+// One row's n (16 or 32) columns from column gc: fp32 or bf16, 16-byte stores while the row
+// has room for them (N % 8 == 0), else element by element.
+__device__ __forceinline__ void store_row(const SpmmArgs& a, const uint32_t (&v)[32], int n,
+                                          int grow, int gc) {
+  if (a.Yb) {
+    uint16_t* yr = a.Yb + (size_t)grow * a.N;
+    for (int i = 0; i < n; i += 8) {
+      if (gc + i + 8 <= a.N) {
+        *reinterpret_cast<uint4*>(yr + gc + i) =
+            make_uint4(pack_bf16x2(v[i], v[i + 1]), pack_bf16x2(v[i + 2], v[i + 3]),
+                       pack_bf16x2(v[i + 4], v[i + 5]), pack_bf16x2(v[i + 6], v[i + 7]));
+      }
+    }
+  } else {
+    float* yr = a.Y + (size_t)grow * a.N;
+    for (int i = 0; i < n; i += 4) {
+      if (gc + i + 4 <= a.N)
+        *reinterpret_cast<float4*>(yr + gc + i) =
+            make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                        __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+    }
+  }
+}
 
 template <int BN, bool SPLIT>
 __global__ void __launch_bounds__(320, 1)
@@ -494,7 +587,8 @@ __global__ void __launch_bounds__(320, 1)
         // conflict either way), and reads back piece l % 8 of row 4 i + l / 8, so that each
         // 16-byte store instruction writes 128 contiguous bytes of 4 rows of Y.
         const uint32_t ep = ptx::smem_u32(epi_stage + (warp & 3) * 4096);
-        const int rr = lane >> 3, pc = lane & 7;
+        const bool epi = a.bias != nullptr || a.act != HINM_ACT_NONE;
+        const float brow = (a.bias && row < a.T) ? __ldg(a.bias + tile * a.T + row) : 0.0f;
         for (int col = 0; col < BN; col += 32) {
           uint32_t v[32];
           if (has) {
@@ -505,25 +599,13 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = 0u;
           }
-#pragma unroll
-          for (int p = 0; p < 8; ++p)
-            ptx::st_shared_v4(ep + lane * 128 + ((p ^ (lane & 7)) << 4), v[4 * p], v[4 * p + 1],
-                              v[4 * p + 2], v[4 * p + 3]);
-          __syncwarp();
-          const int gc = n0 + col + 4 * pc;  // N % 8 == 0: a piece is wholly in or out
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int r = 4 * i + rr;  // row within the warp's quadrant
-            const uint4 o = ptx::ld_shared_v4(ep + r * 128 + ((pc ^ (r & 7)) << 4));
-            const int rw = q * 32 + r;
-            if (rw < a.T && gc < a.N)
-              *reinterpret_cast<uint4*>(a.Y + (size_t)(tile * a.T + rw) * a.N + gc) = o;
-          }
-          __syncwarp();  // the tile is rewritten by the next chunk
+          if (epi) epi_apply<32>(v, brow, a.act);
+          // columns of this chunk inside Y (a multiple of 8; <= 0 past N: nothing stored)
+          const int cw = a.N - (n0 + col) < 32 ? a.N - (n0 + col) : 32;
+          store_chunk32(a, ep, v, lane, q * 32, tile, n0 + col, cw);
         }
       } else {
         const bool row_ok = row < a.T;
-        float* yrow = a.Y + (size_t)(tile * a.T + row) * a.N;
         for (int col = 0; col < BN; col += kChunk) {
           uint32_t v[32];
           if (has) {
@@ -539,20 +621,10 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = 0u;
           }
-          if (row_ok) {
-            const int gc = n0 + col;
-            if (gc + kChunk <= a.N) {
-#pragma unroll
-              for (int i = 0; i < kChunk; i += 4) {
-                float4 o = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
-                                       __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
-                *reinterpret_cast<float4*>(yrow + gc + i) = o;
-              }
-            } else {
-              for (int i = 0; i < kChunk; ++i)
-                if (gc + i < a.N) yrow[gc + i] = __uint_as_float(v[i]);
-            }
-          }
+          if (a.bias != nullptr || a.act != HINM_ACT_NONE)
+            epi_apply<kChunk>(v, (a.bias && row_ok) ? __ldg(a.bias + tile * a.T + row) : 0.0f,
+                              a.act);
+          if (row_ok) store_row(a, v, kChunk, tile * a.T + row, n0 + col);
         }
       }
       ptx::tc_fence_before();
@@ -570,7 +642,6 @@ __global__ void __launch_bounds__(320, 1)
       const int row = q * 32 + lane;
       constexpr int kChunk = BN >= 32 ? 32 : 16;
       const bool row_ok = row < a.T;
-      float* yrow = a.Y + (size_t)(split_tile * a.T + row) * a.N;
       for (int col = 0; col < BN; col += kChunk) {
         uint32_t v[32];
         if (split_has) {
@@ -597,17 +668,13 @@ __global__ void __launch_bounds__(320, 1)
             o[i + 3] = __fadd_rn(o[i + 3], pv.w);
           }
         }
-        if (row_ok) {
-          const int gc = split_n0 + col;
-          if (gc + kChunk <= a.N) {
+        uint32_t ob[32];
 #pragma unroll
-            for (int i = 0; i < kChunk; i += 4)
-              *reinterpret_cast<float4*>(yrow + gc + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
-          } else {
-            for (int i = 0; i < kChunk; ++i)
-              if (gc + i < a.N) yrow[gc + i] = o[i];
-          }
-        }
+        for (int i = 0; i < 32; ++i) ob[i] = i < kChunk ? __float_as_uint(o[i]) : 0u;
+        if (a.bias != nullptr || a.act != HINM_ACT_NONE)
+          epi_apply<kChunk>(ob, (a.bias && row_ok) ? __ldg(a.bias + split_tile * a.T + row) : 0.0f,
+                            a.act);
+        if (row_ok) store_row(a, ob, kChunk, split_tile * a.T + row, split_n0 + col);
       }
     }
   }
@@ -995,7 +1062,7 @@ __global__ void __launch_bounds__(320, 1)
     // through the warp's swizzled shared tile and out as 128-byte row segments of Y.
     const int qd = warp & 3;  // tensor-memory lane quadrant this warp may access
     const uint32_t ep = ptx::smem_u32(epi_stage + qd * 4096);
-    const int rr = lane >> 3, pc = lane & 7;
+    const bool epi = a.bias != nullptr || a.act != HINM_ACT_NONE;
     uint32_t lu[2] = {0u, 0u};
     bool stop = false;
     for (int u = blockIdx.x; u < a.num_units && !stop; u += gridDim.x) {
@@ -1013,6 +1080,7 @@ __global__ void __launch_bounds__(320, 1)
         }
         ++lu[q];
         ptx::tc_fence_after();
+        const float brow = a.bias ? __ldg(a.bias + tile * a.T + qd * 32 + lane) : 0.0f;
         for (int col = 0; col < w; col += 32) {
           const int cw = w - col < 32 ? w - col : 32;  // a multiple of 8
           uint32_t v[32];
@@ -1026,21 +1094,8 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = 0u;
           }
-#pragma unroll
-          for (int pp = 0; pp < 8; ++pp)
-            ptx::st_shared_v4(ep + lane * 128 + ((pp ^ (lane & 7)) << 4), v[4 * pp],
-                              v[4 * pp + 1], v[4 * pp + 2], v[4 * pp + 3]);
-          __syncwarp();
-          const int gc = n0 + col + 4 * pc;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int r = 4 * i + rr;  // row within the warp's quadrant
-            const uint4 o = ptx::ld_shared_v4(ep + r * 128 + ((pc ^ (r & 7)) << 4));
-            const int rw = qd * 32 + r;
-            if (4 * pc < cw && rw < a.T)
-              *reinterpret_cast<uint4*>(a.Y + (size_t)(tile * a.T + rw) * a.N + gc) = o;
-          }
-          __syncwarp();  // the tile is rewritten by the next chunk
+          if (epi) epi_apply<32>(v, brow, a.act);
+          store_chunk32(a, ep, v, lane, qd * 32, tile, n0 + col, cw);
         }
         ptx::tc_fence_before();
         __syncwarp();
@@ -1142,7 +1197,7 @@ int num_sms() {
 }
 
 template <int BN, bool SPLIT>
-cudaError_t run(const hinm_layout& L, const uint16_t* X, int N, float* Y, int split, int* status,
+cudaError_t run(const hinm_layout& L, const uint16_t* X, int N, const SpmmOut& o, int split, int* status,
                 cudaStream_t s) {
   using C = SpmmCfg<BN, SPLIT>;
   cudaError_t attr_err =
@@ -1154,9 +1209,9 @@ cudaError_t run(const hinm_layout& L, const uint16_t* X, int N, float* Y, int sp
   const int nblk_n = (N + BN - 1) / BN;
   const int units = L.num_tiles * nblk_n;
   SpmmArgs a{L.tile_info, L.vals_dense, L.vals_sparse, L.meta,   L.idx_dense, L.idx_sparse,
-             L.run_dense, L.run_sparse, X,             Y,        N,           L.T,
+             L.run_dense, L.run_sparse, X,             o.Y,      N,           L.T,
              L.num_tiles, nblk_n,       units,         SPLIT ? split : 1,       x3d ? 1 : 0,
-             status};
+             status,      o.bias,       o.act,         o.Yb};
   if constexpr (!SPLIT) {
     const int grid = units < num_sms() ? units : num_sms();
     spmm_kernel<BN, false><<<grid, C::kThreads, C::kSmemBytes, s>>>(map, a);
@@ -1181,7 +1236,7 @@ cudaError_t run(const hinm_layout& L, const uint16_t* X, int N, float* Y, int sp
 
 // Tile pairs x 240-column blocks (T = 128, wide N).
 constexpr int kPairMinN = 1024;
-cudaError_t run_pair(const hinm_layout& L, const uint16_t* X, int N, float* Y, int* status,
+cudaError_t run_pair(const hinm_layout& L, const uint16_t* X, int N, const SpmmOut& o, int* status,
                      cudaStream_t s) {
   using C = PairCfg;
   cudaError_t attr_err = set_max_dynamic_smem((const void*)spmm_pair_kernel, (int)C::kSmemBytes);
@@ -1193,8 +1248,9 @@ cudaError_t run_pair(const hinm_layout& L, const uint16_t* X, int N, float* Y, i
   const int nblk_n = (N + C::BN - 1) / C::BN;
   const int units = (L.num_tiles + 1) / 2 * nblk_n;
   SpmmArgs a{L.tile_info, L.vals_dense, L.vals_sparse, L.meta,   L.idx_dense, L.idx_sparse,
-             L.run_dense, L.run_sparse, X,             Y,        N,           L.T,
-             L.num_tiles, nblk_n,       units,         1,        x3d ? 1 : 0, status};
+             L.run_dense, L.run_sparse, X,             o.Y,      N,           L.T,
+             L.num_tiles, nblk_n,       units,         1,        x3d ? 1 : 0, status,
+             o.bias,      o.act,        o.Yb};
   const int grid = units < num_sms() ? units : num_sms();
   spmm_pair_kernel<<<grid, C::kThreads, C::kSmemBytes, s>>>(map3, map2, a);
   return cudaGetLastError();
@@ -1203,27 +1259,27 @@ cudaError_t run_pair(const hinm_layout& L, const uint16_t* X, int N, float* Y, i
 // Split-K when the units (tile x column block) fill less than half of the SMs: each unit's
 // K-blocks are shared by a cluster of up to kMaxSplit CTAs.
 template <int BN>
-cudaError_t run_auto(const hinm_layout& L, const uint16_t* X, int N, float* Y, int* status,
+cudaError_t run_auto(const hinm_layout& L, const uint16_t* X, int N, const SpmmOut& o, int* status,
                      cudaStream_t s) {
   const int units = L.num_tiles * ((N + BN - 1) / BN);
   if constexpr (BN <= 32) {
     int split = units > 0 ? num_sms() / units : 1;
     if (split > SpmmCfg<BN, true>::kMaxSplit) split = SpmmCfg<BN, true>::kMaxSplit;
-    if (split >= 2) return run<BN, true>(L, X, N, Y, split, status, s);
+    if (split >= 2) return run<BN, true>(L, X, N, o, split, status, s);
   }
-  return run<BN, false>(L, X, N, Y, 1, status, s);
+  return run<BN, false>(L, X, N, o, 1, status, s);
 }
 
 }  // namespace
 
-cudaError_t launch_spmm(const hinm_layout& L, const uint16_t* X, int N, float* Y,
+cudaError_t launch_spmm(const hinm_layout& L, const uint16_t* X, int N, const SpmmOut& o,
                         bool tile_pairs, int* status, cudaStream_t s) {
-  if (N <= 16) return run_auto<16>(L, X, N, Y, status, s);
-  if (N <= 32) return run_auto<32>(L, X, N, Y, status, s);
-  if (N <= 64) return run_auto<64>(L, X, N, Y, status, s);
-  if (N < 256) return run_auto<128>(L, X, N, Y, status, s);
-  if (tile_pairs && L.T == 128 && N >= kPairMinN) return run_pair(L, X, N, Y, status, s);
-  return run_auto<256>(L, X, N, Y, status, s);
+  if (N <= 16) return run_auto<16>(L, X, N, o, status, s);
+  if (N <= 32) return run_auto<32>(L, X, N, o, status, s);
+  if (N <= 64) return run_auto<64>(L, X, N, o, status, s);
+  if (N < 256) return run_auto<128>(L, X, N, o, status, s);
+  if (tile_pairs && L.T == 128 && N >= kPairMinN) return run_pair(L, X, N, o, status, s);
+  return run_auto<256>(L, X, N, o, status, s);
 }
 
 }  // namespace hinm

@@ -130,6 +130,13 @@ def test_validation_rejects_before_launch(H):
     assert lib.hinm_boundary_search_stats(fake, fake, 8, None, 256, 256, 128, 0.5, 1 / 32, fake,
                                           fake, None, None, fake, 1 << 30,
                                           None) == H.HINM_ERR_INVALID_ARG
+    # the fused epilogue: an unknown activation is refused; the flags are checked first
+    assert lib.hinm_spmm_epilogue(ctypes.byref(L), fake, 16, fake, None, 4, 0, 0,
+                                  None) == H.HINM_ERR_INVALID_ARG
+    assert lib.hinm_spmm_epilogue(ctypes.byref(L), fake, 16, fake, None, 1, 1, 8,
+                                  None) == H.HINM_ERR_INVALID_ARG
+    assert lib.hinm_spmm_epilogue(ctypes.byref(L), fake, 16, fake, fake + 4, 1, 0, 0,
+                                  None) == H.HINM_ERR_ALIGNMENT
     # Hard-Concrete: n a positive multiple of 4, tau positive and finite, pointers aligned
     assert lib.hinm_hard_concrete_forward(fake, fake, ctypes.c_longlong(6), ctypes.c_float(0.5),
                                           fake, None, None, None) == H.HINM_ERR_SHAPE

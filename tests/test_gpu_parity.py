@@ -240,6 +240,60 @@ def test_translate_index_bad_map_reported(H):
     assert H.hinm_device_status() == 0
 
 
+# one case per epilogue store site: the 256-column kernel (ragged N), the 16-column persistent
+# path (more units than half the SMs), the split-K leader (decode shape), the pair kernel
+EPI_CASES = [
+    ("bn256_ragged", dict(M=384, K=384, N=264, T=128, v_s=None, perm=True, pairs=False)),
+    ("bn16_persistent", dict(M=25600, K=128, N=16, T=128, v_s=None, perm=True, pairs=False)),
+    ("splitk_leader", dict(M=256, K=1024, N=16, T=128, v_s=None, perm=True, pairs=False)),
+    ("pair_kernel", dict(M=640, K=256, N=1040, T=128, v_s=0.0, perm=False, pairs=True)),
+]
+
+
+@pytest.mark.parametrize("name,cfg", EPI_CASES, ids=[c[0] for c in EPI_CASES])
+def test_spmm_epilogue_matches_oracle(H, name, cfg):
+    """The fused epilogue (per-row bias, ReLU / SiLU / GELU, fp32 or bf16 Y) at every store
+    site.  Exact: no epilogue = hinm_spmm bit for bit, and the bf16 Y of the plain product is
+    the round-to-nearest-even of the GPU's own fp32 Y.  Against the oracle: act(y + bias)
+    within the product's bound times the activations' slope (<= 1.2), plus their fp32
+    evaluation and, for bf16, half a bf16 ulp."""
+    M, K, N, T = cfg["M"], cfg["K"], cfg["N"], cfg["T"]
+    w = hi.custom(M, K, N, T, seed=31, t_s=0.5, v_s=cfg["v_s"], random_perm=cfg["perm"])
+    W, X, perm = dev_bf16(w.W_bits), dev_bf16(w.X_bits), dev_i32(w.perm)
+    hp = H.HotPath(M, K, N, T, 0.5, w.alpha)
+    fixed = None
+    if cfg["v_s"] is not None:
+        fixed = dev_i32(np.tile(np.array(H.hinm_counts_from_vs(K, 0.5, cfg["v_s"]), dtype=np.int32),
+                                (M // T, 1)))
+    pairs = cfg["pairs"]
+    Y = hp.run(W, X, perm, fixed_counts=fixed, tile_pairs=pairs).clone()
+    L = hp.layout
+    Y_plain = H.hinm_spmm_epilogue(L, X, tile_pairs=pairs)
+    Y_b16 = H.hinm_spmm_epilogue(L, X, out_bf16=True, tile_pairs=pairs)
+    torch.cuda.synchronize()
+    status_ok(H)
+    np.testing.assert_array_equal(Y_plain.cpu().numpy().view(np.uint32), Y.cpu().numpy().view(np.uint32))
+    np.testing.assert_array_equal(Y_b16.view(torch.int16).cpu().numpy(),
+                                  Y.to(torch.bfloat16).view(torch.int16).cpu().numpy())
+    bm = hp.bitmask.cpu().numpy().view(np.uint32)
+    y_ref, bound = O.spmm_reference(w.W_bits, bm, w.X_bits)
+    rng = np.random.default_rng(3)
+    bias = rng.normal(0.0, 0.05, M).astype(np.float32)
+    bias_d = torch.from_numpy(bias).cuda()
+    for act in (H.HINM_ACT_RELU, H.HINM_ACT_SILU, H.HINM_ACT_GELU):
+        ref = O.spmm_epilogue_reference(y_ref, bias, act)
+        base = 1.2 * (TOL_REL * bound + TOL_ABS) + 1e-6 * (np.abs(ref) + 1.0)
+        for b16 in (False, True):
+            got = H.hinm_spmm_epilogue(L, X, bias=bias_d, activation=act, out_bf16=b16,
+                                       tile_pairs=pairs)
+            torch.cuda.synchronize()
+            g = got.float().cpu().numpy().astype(np.float64)
+            tol = base + (2.0 ** -8) * (np.abs(ref) + base) if b16 else base
+            err = np.abs(g - ref)
+            assert (err <= tol).all(), f"act {act} bf16 {b16}: worst excess {(err - tol).max():.3e}"
+    status_ok(H)
+
+
 def _hc_bound(la, eps, tau):
     """Per-element bound on |z_fp32 - z_fp64| from the fp32 operation order of the kernel:
     logf and log1pf within 1 ulp, expf within 2 ulp (CUDA's documented maxima), each fp32
