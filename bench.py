@@ -396,6 +396,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="hinm", choices=["hinm", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next-rows", action="store_true",
+                    help="skip the extra timings of the index translation, the fused epilogue "
+                         "and the Hard-Concrete forward (for a launch list of the step alone)")
     ap.add_argument("--workload", default="pure24", choices=sorted(WORKLOADS) + ["sweep"],
                     help="synthetic workload (default: the pure 2:4 4096x4096x2048 benchmark); "
                          "'sweep' times the LLaMA-2-7B-shaped layer sweep")
@@ -613,9 +616,11 @@ def main():
                          "importance, search, mask, compress and fp64 masked product",
                "seconds": dt}
     clocks = sampler.summary()
-    next_rows = {"index_translate": time_index_translate(H, hp, K, stream),
-                 "hard_concrete": time_hard_concrete(H, M * K, peaks, stream),
-                 "epilogue_bf16": time_epilogue(H, hp, X, M, N, tile_pairs, flush, stream)}
+    next_rows = None
+    if not args.no_next_rows:
+        next_rows = {"index_translate": time_index_translate(H, hp, K, stream),
+                     "hard_concrete": time_hard_concrete(H, M * K, peaks, stream),
+                     "epilogue_bf16": time_epilogue(H, hp, X, M, N, tile_pairs, flush, stream)}
     # this library's kernels per step: importance 2 (channel energies, importance with the
     # tile statistics), search 6 (chunk sort, merge rank, column sums, candidate lists, band
     # sums, finalize; V comes from the importance step), mask 2 (classify with the
