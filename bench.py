@@ -360,6 +360,28 @@ def time_epilogue(H, hp, X, M, N, tile_pairs, flush, stream, reps=10):
             "note": "one call per timing after the L2 flush; median of %d" % reps}
 
 
+def time_dense_context(M, K, N, flush, stream, reps=10):
+    """Context, not a target: a dense bf16 GEMM of the same shape (torch.matmul, cuBLAS, fp32
+    accumulation, bf16 output) on random operands, one call per timing after the L2 flush,
+    the median of `reps`."""
+    import torch
+    A = torch.randn(M, K, device="cuda").to(torch.bfloat16)
+    B = torch.randn(K, N, device="cuda").to(torch.bfloat16)
+    ts = []
+    for i in range(reps + 2):
+        flush.fill_(i & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        torch.matmul(A, B)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= 2:
+            ts.append(e0.elapsed_time(e1) * 1e3)
+    t = float(np.median(ts))
+    return {"torch_matmul_dense_bf16_us": t, "tflops": 2.0 * M * K * N / (t * 1e-6) / 1e12,
+            "note": "dense W (no pruning) through cuBLAS, same M, K, N; context only"}
+
+
 def time_hard_concrete(H, n, peaks, stream, reps=10):
     """The Hard-Concrete forward over n = M*K elements (logits N(0, 2), noise U(0, 1), drawn
     on the device from a fixed seed; tau = 2/3): CUDA events over `reps` back-to-back calls
@@ -616,8 +638,9 @@ def main():
                          "importance, search, mask, compress and fp64 masked product",
                "seconds": dt}
     clocks = sampler.summary()
-    next_rows = None
+    next_rows = context = None
     if not args.no_next_rows:
+        context = time_dense_context(M, K, N, flush, stream)
         next_rows = {"index_translate": time_index_translate(H, hp, K, stream),
                      "hard_concrete": time_hard_concrete(H, M * K, peaks, stream),
                      "epilogue_bf16": time_epilogue(H, hp, X, M, N, tile_pairs, flush, stream)}
@@ -654,6 +677,7 @@ def main():
         "gpu_launches": kernels_per_step * args.steps,
         "gpu_launches_phase_pass": kernels_per_step * args.steps,
         "next_rows": next_rows,
+        "context": context,
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                    "reasons": clocks["reasons"], "samples": clocks["samples"]},
     }
