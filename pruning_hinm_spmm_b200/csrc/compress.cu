@@ -395,8 +395,13 @@ __global__ void __launch_bounds__(kSparseBK) translate_index_kernel(
   if (b >= nd + ns) return;
   const bool sparse = b >= nd;
   const int nvec = sparse ? kSparseBK : kDenseBK;
-  int32_t* idx = sparse ? L.idx_sparse + (size_t)(L.tile_info[4 * t + 3] + b - nd) * kSparseBK
-                        : L.idx_dense + (size_t)(L.tile_info[4 * t + 2] + b) * kDenseBK;
+  const int blk = sparse ? L.tile_info[4 * t + 3] + b - nd : L.tile_info[4 * t + 2] + b;
+  if (blk < 0 || blk >= (sparse ? L.max_sparse_blocks : L.max_dense_blocks)) {
+    // tile_info not from hinm_compress for this layout: report, touch nothing
+    if (threadIdx.x == 0) ptx::record_status(status, HINM_ERR_INVALID_ARG);
+    return;
+  }
+  int32_t* idx = sparse ? L.idx_sparse + (size_t)blk * kSparseBK : L.idx_dense + (size_t)blk * kDenseBK;
   int v = 0;
   if ((int)threadIdx.x < nvec) {
     const int c = idx[threadIdx.x];
@@ -411,10 +416,7 @@ __global__ void __launch_bounds__(kSparseBK) translate_index_kernel(
   __syncthreads();
   const bool step_ok = (int)threadIdx.x >= nvec || v == first + (int)threadIdx.x;
   const bool run = __syncthreads_and(step_ok);
-  if (threadIdx.x == 0) {
-    if (sparse) L.run_sparse[L.tile_info[4 * t + 3] + b - nd] = run ? first : -1;
-    else L.run_dense[L.tile_info[4 * t + 2] + b] = run ? first : -1;
-  }
+  if (threadIdx.x == 0) (sparse ? L.run_sparse : L.run_dense)[blk] = run ? first : -1;
 }
 
 cudaError_t launch_translate_index(const hinm_layout& L, const int32_t* row_of_channel,

@@ -806,7 +806,7 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int pairs_last = a.num_tiles - 1;  // tile 2p + 1 exists iff 2p + 1 <= pairs_last
+  const int last_tile = a.num_tiles - 1;  // tile 2p + 1 exists iff 2p + 1 <= last_tile
 
   if (warp < 4) {
     // ------------------------------------------------------------ gather producers
@@ -818,7 +818,7 @@ __global__ void __launch_bounds__(320, 1)
     for (int u = blockIdx.x; u < a.num_units && !stop; u += gridDim.x) {
       const int p = u / a.nblk_n, n0 = (u - p * a.nblk_n) * BN;
       const bool pm = pair_shares_b(a, p, lane);
-      const int nq = pm ? 1 : (2 * p + 1 <= pairs_last ? 2 : 1);
+      const int nq = pm ? 1 : (2 * p + 1 <= last_tile ? 2 : 1);
       for (int q = 0; q < nq && !stop; ++q) {
         const int4 info = info_of(2 * p + q);
         const int nd = info.x, nblk = info.x + info.y;
@@ -866,7 +866,7 @@ __global__ void __launch_bounds__(320, 1)
       const int p = u / a.nblk_n, n0 = (u - p * a.nblk_n) * BN;
       const bool pm = pair_shares_b(a, p, lane);
       if (lane == 0) {
-        const int nq = pm ? 1 : (2 * p + 1 <= pairs_last ? 2 : 1);
+        const int nq = pm ? 1 : (2 * p + 1 <= last_tile ? 2 : 1);
         for (int q = 0; q < nq && !stop; ++q) {
           const int4 info = info_of(2 * p + q);
           const int4 info1 = pm ? info_of(2 * p + 1) : info;
@@ -953,7 +953,7 @@ __global__ void __launch_bounds__(320, 1)
         const int nmma = (w + 15) & ~15;  // MMA width: the unit's columns, rounded up to 16
         const uint32_t idesc_d = ptx::idesc_bf16(nmma, 1, 0);
         const uint32_t idesc_s = ptx::idesc_bf16(nmma, 1, 1);
-        const int nq = pm ? 1 : (2 * p + 1 <= pairs_last ? 2 : 1);
+        const int nq = pm ? 1 : (2 * p + 1 <= last_tile ? 2 : 1);
         for (int q = 0; q < nq && !stop; ++q) {
           // buffers this pass writes: both in a shared unit, else buffer q
           if (pm || q == 0) {
@@ -1068,7 +1068,7 @@ __global__ void __launch_bounds__(320, 1)
     for (int u = blockIdx.x; u < a.num_units && !stop; u += gridDim.x) {
       const int p = u / a.nblk_n, n0 = (u - p * a.nblk_n) * BN;
       const int w = a.N - n0 < BN ? a.N - n0 : BN;
-      const int nq = 2 * p + 1 <= pairs_last ? 2 : 1;
+      const int nq = 2 * p + 1 <= last_tile ? 2 : 1;
       for (int q = 0; q < nq; ++q) {
         const int tile = 2 * p + q;
         const int4 info = info_of(tile);
