@@ -233,7 +233,8 @@ hinm_status hinm_compress(const void* W, const uint32_t* bitmask, const int8_t* 
  *   s = sigmoid((log eps - log(1 - eps) + log alpha) / tau),
  * stretched to (-0.1, 1.1) and clipped to [0, 1]; the regularisers are mean(z) and the mean
  * over groups of |sum of the group's z - 2|; the hardened mask thresholds z at 0.5).
- *   z_i = min(1, max(0, 1.2 s_i - 0.1)) (fp32, with CUDA's logf / log1pf / expf)
+ *   z_i = min(1, max(0, 1.2 s_i - 0.1)) (fp32, with CUDA's logf and expf; the noise logit
+ *   as logf of eps / (1 - eps))
  * log_alpha, eps: device fp32 [n], n % 4 == 0, groups = 4 consecutive elements; eps is the
  * caller's noise (eps = 1/2 everywhere gives the deterministic mask; eps = 0 or 1 give
  * z = 0 or 1; NaN in, NaN out).  tau > 0.

@@ -7,7 +7,7 @@
 // One HBM stream: a thread per group of 4 (16-byte loads of log alpha and eps, a 16-byte
 // store of z and a 4-byte store of the hardened bits), kHcUnroll groups in flight per thread,
 // grid-stride; the two regulariser sums in fp64, block-reduced, one atomic add per block.
-// The fp32 arithmetic calls CUDA's logf, log1pf and expf.
+// The fp32 arithmetic calls CUDA's logf and expf.
 #include <cuda_runtime.h>
 
 #include "hinm_internal.h"
@@ -26,9 +26,11 @@ int hc_sm_count() {
   return n > 0 ? n : 148;
 }
 
-// inv_tau = fl32(1 / tau); the reciprocal of 1 + exp(-x) is the correctly rounded one
+// inv_tau = fl32(1 / tau); the reciprocals are the correctly rounded ones.  The noise logit
+// log(eps / (1 - eps)) takes one logf of the ratio (three fp32 roundings: 1 - eps, its
+// reciprocal, the product; eps = 0 or 1 still give -inf / +inf).
 __device__ __forceinline__ float hc_z(float la, float e, float inv_tau) {
-  const float logit = __fsub_rn(logf(e), log1pf(-e));   // log eps - log(1 - eps)
+  const float logit = logf(__fmul_rn(e, __frcp_rn(__fsub_rn(1.0f, e))));
   const float x = __fmul_rn(__fadd_rn(logit, la), inv_tau);
   const float s = __frcp_rn(__fadd_rn(1.0f, expf(-x)));
   const float sb = __fadd_rn(__fmul_rn(s, __fsub_rn(kHcHigh, kHcLow)), kHcLow);

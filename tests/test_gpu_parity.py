@@ -296,16 +296,18 @@ def test_spmm_epilogue_matches_oracle(H, name, cfg):
 
 def _hc_bound(la, eps, tau):
     """Per-element bound on |z_fp32 - z_fp64| from the fp32 operation order of the kernel:
-    logf and log1pf within 1 ulp, expf within 2 ulp (CUDA's documented maxima), each fp32
-    add / multiply / reciprocal within half an ulp (the scale by 1/tau: the reciprocal's and
-    the product's roundings), carried through the sigmoid's slope s(1 - s) and the stretch by
-    1.2; plus the fp32 stretch constants' offset from the fp64 ones."""
+    the noise logit as logf of eps / (1 - eps) (three roundings of the ratio: 3 half-ulps of
+    relative error, so 3 * 2^-24 absolute after the log) with logf within 1 ulp, expf within
+    2 ulp (CUDA's documented maxima), each fp32 add / multiply / reciprocal within half an
+    ulp (the scale by 1/tau: the reciprocal's and the product's roundings), carried through
+    the sigmoid's slope s(1 - s) and the stretch by 1.2; plus the fp32 stretch constants'
+    offset from the fp64 ones."""
     d = 2.0 ** -24
     la = la.astype(np.float64)
     e = eps.astype(np.float64)
     l1, l2 = np.abs(np.log(e)), np.abs(np.log1p(-e))
     logit = np.log(e) - np.log1p(-e)
-    err_logit = (l1 + l2) * 2 * d + np.abs(logit) * d
+    err_logit = 4 * d + np.abs(logit) * 2 * d + (l1 + l2) * 2 * d
     x = (logit + la) / tau
     err_x = (err_logit + np.abs(logit + la) * d) / tau + np.abs(x) * 3 * d
     s = 1.0 / (1.0 + np.exp(-x))
