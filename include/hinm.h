@@ -58,7 +58,7 @@ typedef enum {
   HINM_ERR_INVALID_ARG = 1,      /* null pointer, NaN parameter, bad enum */
   HINM_ERR_SHAPE = 2,            /* sizes violate the supported-size rules above */
   HINM_ERR_ALIGNMENT = 3,        /* a device pointer is not 16-byte aligned */
-  HINM_ERR_UNSUPPORTED = 4,      /* a valid request this build does not implement */
+  HINM_ERR_UNSUPPORTED = 4,      /* a valid request this library does not implement */
   HINM_ERR_CUDA = 5,             /* a CUDA runtime call failed (launch, memcpy, ...) */
   HINM_ERR_DEVICE_TIMEOUT = 6,   /* device status: a bounded wait gave up */
   HINM_ERR_BAD_MASK = 7,         /* device status: a 2:4 group without exactly 2 kept */
