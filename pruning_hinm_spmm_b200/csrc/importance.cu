@@ -29,8 +29,14 @@ __device__ __forceinline__ double bf16_to_f64(uint32_t bits16) {
 // sequential chain itself.
 constexpr int kEnergyWarps = 8;
 
+// zero_int (nullptr allowed): n_zero ints of a later kernel cleared by the grid on the way
+// (the tile maxima that importance_stats_kernel raises with atomicMax)
 __global__ void __launch_bounds__(kEnergyWarps * 32) channel_energy_kernel(
-    const uint16_t* __restrict__ X, int K, int N, float* __restrict__ s) {
+    const uint16_t* __restrict__ X, int K, int N, float* __restrict__ s,
+    int* __restrict__ zero_int = nullptr, int n_zero = 0) {
+  if (zero_int)
+    for (int x = blockIdx.x * blockDim.x + threadIdx.x; x < n_zero; x += gridDim.x * blockDim.x)
+      zero_int[x] = 0;
   const int lane = threadIdx.x & 31;
   const int c = blockIdx.x * kEnergyWarps + (threadIdx.x >> 5);
   if (c >= K) return;  // warp-uniform
@@ -213,11 +219,10 @@ cudaError_t launch_importance_stats(const uint16_t* W, const uint16_t* X, int M,
   const int nt = M / T;
   double* V = static_cast<double*>(stats);
   int* pmax = reinterpret_cast<int*>(static_cast<char*>(stats) + tile_stats_v_bytes(M, K, T));
-  cudaError_t e = cudaMemsetAsync(pmax, 0, (size_t)nt * sizeof(int), st);
-  if (e != cudaSuccess) return e;
+  // the energies' grid also clears the tile maxima (raised by importance_stats_kernel next)
   channel_energy_kernel<<<(K + kEnergyWarps - 1) / kEnergyWarps, kEnergyWarps * 32, 0, st>>>(
-      X, K, N, s_scratch);
-  e = cudaGetLastError();
+      X, K, N, s_scratch, pmax, nt);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const dim3 g((K / 2 + 255) / 256, nt);
   importance_stats_kernel<<<g, 256, 0, st>>>(W, s_scratch, K, T, I, V, pmax);

@@ -233,11 +233,22 @@ __device__ __forceinline__ bool pair_less(unsigned long long ka, unsigned ia,
 // Sorts one chunk of kRankChunk working positions of one tile by (key, index) ascending:
 // a bitonic network with one element per thread; compare-exchange stages with partner
 // distance < 32 run on warp shuffles, the wider ones through shared memory.
+// zero64 / zero32 (nullptr allowed): buffers of a later kernel of the search, cleared here by
+// the whole grid (grid-stride) instead of by separate memsets.
 __global__ void __launch_bounds__(kRankChunk) chunk_sort_kernel(
     const double* __restrict__ Vc, const int32_t* __restrict__ perm, int K, int Kp,
-    unsigned long long* __restrict__ skey, unsigned short* __restrict__ sidx) {
+    unsigned long long* __restrict__ skey, unsigned short* __restrict__ sidx,
+    unsigned long long* __restrict__ zero64, size_t n64, int* __restrict__ zero32, size_t n32) {
   __shared__ unsigned long long key_s[kRankChunk];
   __shared__ unsigned short idx_s[kRankChunk];
+  {
+    const size_t gt = ((size_t)blockIdx.y * gridDim.x + blockIdx.x) * kRankChunk + threadIdx.x;
+    const size_t gs = (size_t)gridDim.x * gridDim.y * kRankChunk;
+    if (zero64)
+      for (size_t x = gt; x < n64; x += gs) zero64[x] = 0ull;
+    if (zero32)
+      for (size_t x = gt; x < n32; x += gs) zero32[x] = 0;
+  }
   const int t = blockIdx.y, base = blockIdx.x * kRankChunk;
   const int i = threadIdx.x;
   const int j = base + i;
@@ -331,7 +342,9 @@ cudaError_t launch_vector_scores(const float* I, int M, int K, int T, double* V,
 
 // The ranking from V: chunk sort, then merge.
 cudaError_t launch_rank_sort(const double* V, const int32_t* perm, int M, int K, int T,
-                             int32_t* rank, void* scratch, cudaStream_t s) {
+                             int32_t* rank, void* scratch, cudaStream_t s,
+                             unsigned long long* zero64 = nullptr, size_t n64 = 0,
+                             int* zero32 = nullptr, size_t n32 = 0) {
   const int nt = M / T;
   cudaError_t e;
   const int nchunk = (K + kRankChunk - 1) / kRankChunk;
@@ -339,7 +352,8 @@ cudaError_t launch_rank_sort(const double* V, const int32_t* perm, int M, int K,
   Carve c{static_cast<char*>(scratch), 0};
   unsigned long long* skey = c.take<unsigned long long>((size_t)nt * Kp);
   unsigned short* sidx = c.take<unsigned short>((size_t)nt * Kp);
-  chunk_sort_kernel<<<dim3(nchunk, nt), kRankChunk, 0, s>>>(V, perm, K, Kp, skey, sidx);
+  chunk_sort_kernel<<<dim3(nchunk, nt), kRankChunk, 0, s>>>(V, perm, K, Kp, skey, sidx, zero64,
+                                                            n64, zero32, n32);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   merge_rank_kernel<<<dim3(nchunk, nt), kRankChunk, 0, s>>>(skey, sidx, K, Kp, rank);
@@ -844,6 +858,15 @@ cudaError_t launch_boundary_search(const float* I, const void* stats, const int3
   unsigned char* coltiny = c.take<unsigned char>((size_t)nt * K);
   char* rank_scratch = c.take<char>(rank_scratch_bytes(M, K, T));
   int32_t* rank = rank_out ? rank_out : rank_ws;
+  // the candidates' buffers (same carving order as search_workspace_bytes)
+  const BandCfg bc = band_config(K);
+  const int RB = bc.rows;
+  const int nchunks = T / RB;
+  unsigned short* band = c.take<unsigned short>((size_t)nt * ncand * K);
+  U128* rdense = c.take<U128>((size_t)nt * ncand);
+  U128* part = c.take<U128>((size_t)nt * ncand * nchunks);
+  unsigned long long* bucket = c.take<unsigned long long>((size_t)nt * ncand * 256);
+  int* bucket_used = c.take<int>((size_t)nt * ncand);
   // V and the tile maxima: made with I by the importance step, or computed here
   const double* V = V_ws;
   const int* pmax = pmax_ws;
@@ -873,25 +896,15 @@ cudaError_t launch_boundary_search(const float* I, const void* stats, const int3
     if (e != cudaSuccess) return e;
     e = cudaEventRecord(ss->join, ss->stream);
     if (e != cudaSuccess) return e;
-    e = launch_rank_sort(V, perm, M, K, T, rank, rank_scratch, s);
+    // the sort also clears the exponent buckets and their flags (used from candidate_lists on)
+    e = launch_rank_sort(V, perm, M, K, T, rank, rank_scratch, s, bucket,
+                         (size_t)nt * ncand * 256, bucket_used, (size_t)nt * ncand);
     if (e != cudaSuccess) return e;
     e = cudaStreamWaitEvent(s, ss->join, 0);
     if (e != cudaSuccess) return e;
   }
   CandidateList cl;
   for (int i = 0; i < kMaxCandidates; ++i) cl.c[i] = i < ncand ? cands[i] : Candidate{0, 0, 0};
-  const BandCfg bc = band_config(K);
-  const int RB = bc.rows;
-  const int nchunks = T / RB;
-  unsigned short* band = c.take<unsigned short>((size_t)nt * ncand * K);
-  U128* rdense = c.take<U128>((size_t)nt * ncand);
-  U128* part = c.take<U128>((size_t)nt * ncand * nchunks);
-  unsigned long long* bucket = c.take<unsigned long long>((size_t)nt * ncand * 256);
-  int* bucket_used = c.take<int>((size_t)nt * ncand);
-  e = cudaMemsetAsync(bucket, 0, (size_t)nt * ncand * 256 * sizeof(unsigned long long), s);
-  if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(bucket_used, 0, (size_t)nt * ncand * sizeof(int), s);
-  if (e != cudaSuccess) return e;
   {
     const dim3 gl(ncand, nt);
     const int per = (K + 511) / 512;
