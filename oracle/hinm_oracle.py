@@ -653,3 +653,58 @@ def spmm_epilogue_reference(y: np.ndarray, bias: Optional[np.ndarray], act: int)
     if bias is not None:
         z = z + np.asarray(bias, dtype=np.float64)[:, None]
     return activation(z, act)
+
+
+# ---------------------------------------------------------------------------------------
+# Gyro-style refinement of a tile's 2:4 grouping (offline; produces the working order)
+# ---------------------------------------------------------------------------------------
+def group_retained(I_tile: np.ndarray, members: List[int]) -> float:
+    """Retained 2:4 importance of one group: over the tile's rows (ascending, fp64 sum),
+    the two largest of the group's four values, each added as fp64 ([P1] 关键设计 1: the
+    retained second-order importance of a 2:4 group)."""
+    acc = 0.0
+    for r in range(I_tile.shape[0]):
+        v = sorted((float(I_tile[r, c]) for c in members), reverse=True)
+        acc += v[0] + v[1]
+    return acc
+
+
+def gyro_refine(I_tile: np.ndarray, band: np.ndarray, schedule: np.ndarray):
+    """Refine the grouping of a tile's 2:4 band (channels in working order, groups of 4
+    consecutive entries) by sampled re-assignment ([P1] 关键设计 2, gyro-permutation: sample
+    vectors per tile, cluster them into balanced clusters, and assign by the Hungarian
+    algorithm on the pruning-cost matrix; the permutation leaves the product unchanged).
+
+    [reading] Iteration i takes the schedule's S (group, slot) pairs (distinct groups; the
+    caller's random draws): the S sampled vectors leave their slots, and the balanced
+    clustering of S vectors into the S freed slots (capacity 1 each) is the assignment that
+    maximises the sum over groups of the retained importance of each group with the vector
+    placed in its freed slot -- the Hungarian algorithm on that cost matrix (here
+    scipy.optimize.linear_sum_assignment as the assignment step).  Keeping every vector in
+    place is one assignment, so the retained importance never decreases.
+    Returns (refined band, retained importance of the band before and after each iteration).
+    """
+    from scipy.optimize import linear_sum_assignment
+
+    band = np.array(band, dtype=np.int64).copy()
+    ng = band.size // 4
+
+    def total(b):
+        return sum(group_retained(I_tile, [int(x) for x in b[4 * g:4 * g + 4]]) for g in range(ng))
+
+    hist = [total(band)]
+    for it in range(schedule.shape[0]):
+        groups = [int(g) for g in schedule[it, :, 0]]
+        slots = [int(k) for k in schedule[it, :, 1]]
+        vecs = [int(band[4 * g + k]) for g, k in zip(groups, slots)]
+        S = len(groups)
+        C = np.zeros((S, S))
+        for b, (g, k) in enumerate(zip(groups, slots)):
+            rest = [int(band[4 * g + j]) for j in range(4) if j != k]
+            for a in range(S):
+                C[a, b] = group_retained(I_tile, rest + [vecs[a]])
+        rows, cols = linear_sum_assignment(C, maximize=True)
+        for a, b in zip(rows, cols):
+            band[4 * groups[b] + slots[b]] = vecs[a]
+        hist.append(total(band))
+    return band, np.array(hist)

@@ -581,3 +581,46 @@ def test_epilogue_reference_bias_per_row():
     got = O.spmm_epilogue_reference(y, b, O.ACT_RELU)
     np.testing.assert_array_equal(got, np.maximum(y + b[:, None], 0.0))
     np.testing.assert_array_equal(O.spmm_epilogue_reference(y, None, O.ACT_NONE), y)
+
+
+# ----------------------------------------------------------------------------- gyro refinement
+def test_gyro_refine_hand_example():
+    """One row, two groups [9, 8, 7, 1] and [6, 5, 4, 3]: retained 17 + 11 = 28.  Sampling the
+    7 (group 0, slot 2) and the 3 (group 1, slot 3) and swapping them gives [9, 8, 3, 1] and
+    [6, 5, 4, 7]: 17 + 13 = 30, the better of the two assignments."""
+    I_tile = np.array([[9, 8, 7, 1, 6, 5, 4, 3]], dtype=np.float32)
+    band = np.arange(8)
+    sched = np.array([[[0, 2], [1, 3]]])
+    out, hist = O.gyro_refine(I_tile, band, sched)
+    np.testing.assert_array_equal(hist, [28.0, 30.0])
+    np.testing.assert_array_equal(out, [0, 1, 7, 3, 4, 5, 6, 2])
+
+
+def test_gyro_refine_brute_force_and_invariants():
+    """S = 4 sampled groups: the chosen assignment's total equals the best of all 24
+    (brute force); over several iterations the retained importance never falls, the band
+    stays a permutation of its channels and the groups not sampled keep their members."""
+    import itertools
+    rng = np.random.default_rng(17)
+    T, K = 16, 64
+    I_tile = rng.exponential(1.0, (T, K)).astype(np.float32)
+    band = rng.permutation(K)[:48]                  # 12 groups of a 2:4 band
+    sched = np.array([[[1, 0], [4, 3], [7, 1], [10, 2]]])
+    out, hist = O.gyro_refine(I_tile, band, sched)
+    groups, slots = [1, 4, 7, 10], [0, 3, 1, 2]
+    vecs = [int(band[4 * g + k]) for g, k in zip(groups, slots)]
+    best = -1.0
+    for p in itertools.permutations(range(4)):
+        b2 = band.copy()
+        for a, b in enumerate(p):
+            b2[4 * groups[b] + slots[b]] = vecs[a]
+        best = max(best, sum(O.group_retained(I_tile, list(b2[4 * g:4 * g + 4])) for g in range(12)))
+    assert abs(hist[1] - best) <= 1e-9 * best
+    sched4 = np.array([[[g, (g * 7 + it) % 4] for g in rng.choice(12, 6, replace=False)]
+                       for it in range(5)])
+    out4, hist4 = O.gyro_refine(I_tile, band, sched4)
+    assert (np.diff(hist4) >= -1e-12 * hist4[0]).all()
+    assert sorted(out4.tolist()) == sorted(band.tolist())
+    touched = set(int(g) for g in sched4[:, :, 0].ravel())
+    for g in set(range(12)) - touched:
+        np.testing.assert_array_equal(out4[4 * g:4 * g + 4], band[4 * g:4 * g + 4])
