@@ -382,6 +382,29 @@ def time_dense_context(M, K, N, flush, stream, reps=10):
             "note": "dense W (no pruning) through cuBLAS, same M, K, N; context only"}
 
 
+def time_gyro(H, hp, perm, T, K, S=64, iters=4):
+    """The host gyro-style refinement on tile 0 of this step: its importance rows, its 2:4
+    band in working order (from the step's regions), a seeded schedule of S (group, slot)
+    samples per iteration; wall-clock time on one host core."""
+    import time
+    I_tile = hp.I[:T].cpu().numpy()
+    region0 = hp.region[0].cpu().numpy()
+    band = np.array([c for c in perm if region0[c] == 1], dtype=np.int32)
+    ng = band.size // 4
+    if ng == 0:
+        return {"note": "tile 0 has no 2:4 band"}
+    S = min(S, ng)
+    rng = np.random.default_rng(7)
+    sched = np.stack([np.stack([rng.choice(ng, S, replace=False), rng.integers(0, 4, S)], axis=1)
+                      for _ in range(iters)]).astype(np.int32)
+    t0 = time.perf_counter()
+    _, hist = H.hinm_gyro_refine_host(I_tile, band, sched)
+    dt = time.perf_counter() - t0
+    return {"ms_per_iteration": dt / iters * 1e3, "groups": ng, "samples_per_iteration": S,
+            "iterations": iters, "retained_gain": float(hist[-1] / hist[0] - 1.0),
+            "where": "host (offline, once per layer)", "cores": 1}
+
+
 def time_hard_concrete(H, n, peaks, stream, reps=10):
     """The Hard-Concrete forward over n = M*K elements (logits N(0, 2), noise U(0, 1), drawn
     on the device from a fixed seed; tau = 2/3): CUDA events over `reps` back-to-back calls
@@ -643,7 +666,8 @@ def main():
         context = time_dense_context(M, K, N, flush, stream)
         next_rows = {"index_translate": time_index_translate(H, hp, K, stream),
                      "hard_concrete": time_hard_concrete(H, M * K, peaks, stream),
-                     "epilogue_bf16": time_epilogue(H, hp, X, M, N, tile_pairs, flush, stream)}
+                     "epilogue_bf16": time_epilogue(H, hp, X, M, N, tile_pairs, flush, stream),
+                     "gyro_refine_host": time_gyro(H, hp, w.perm, T, K)}
     # this library's kernels per step: importance 2 (channel energies, importance with the
     # tile statistics), search 6 (chunk sort, merge rank, column sums, candidate lists, band
     # sums, finalize; V comes from the importance step), mask 2 (classify with the

@@ -228,6 +228,27 @@ hinm_status hinm_compress(const void* W, const uint32_t* bitmask, const int8_t* 
                           const hinm_layout* layout, void* workspace,
                           size_t workspace_bytes, void* stream);
 
+/* Gyro-style refinement of one tile's 2:4 grouping, on the host  ([P1] 关键设计 2: the
+ * channel permutation reorders channels without changing the product so that important
+ * weights land where they are kept; per tile, sampled vectors are re-assigned by the
+ * Hungarian algorithm on the pruning-cost matrix, iterated to refine).  An offline,
+ * once-per-layer step: its output is the working order the hot path takes as `perm`.
+ *   The band is the tile's 2:4 channels in working order, groups = 4 consecutive entries;
+ *   a group's retained importance = sum over the tile's rows (ascending, fp64) of its two
+ *   largest values.  Iteration i takes schedule[i][0..S) = (group, slot) pairs (distinct
+ *   groups; the caller's random draws): the S sampled channels leave their slots and go
+ *   back by the assignment that maximises the sampled groups' total retained importance
+ *   (reading: the balanced clustering of S vectors into the S freed slots, capacity 1 each,
+ *   is that assignment).  The retained importance never decreases.
+ * I_tile: host fp32 [T][K] (the tile's importance rows, by channel); band: host int32 [n],
+ * n % 4 == 0, n <= K, entries in [0, K), refined in place; schedule: host int32
+ * [iters][S][2]; retained_out (NULL allowed): host fp64 [iters + 1], the band's retained
+ * importance before and after each iteration.
+ * Errors (checked before any work): HINM_ERR_SHAPE, HINM_ERR_INVALID_ARG. */
+hinm_status hinm_gyro_refine_host(const float* I_tile, int T, int K, int32_t* band, int n,
+                                  const int32_t* schedule, int iters, int S,
+                                  double* retained_out);
+
 /* Hard-Concrete soft 2:4 mask, forward  ([P1] 关键设计 3: each group of 4 has learnable
  * logits log alpha; with noise eps ~ U(0, 1) the soft mask is
  *   s = sigmoid((log eps - log(1 - eps) + log alpha) / tau),

@@ -82,6 +82,7 @@ _SIGS = {
     "hinm_compress": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
                              ctypes.POINTER(hinm_layout), _vp, _sz, _vp]),
     "hinm_translate_index": (_i32, [ctypes.POINTER(hinm_layout), _vp, _vp]),
+    "hinm_gyro_refine_host": (_i32, [_vp, _i32, _i32, _vp, _i32, _vp, _i32, _i32, _vp]),
     "hinm_hard_concrete_forward": (_i32, [_vp, _vp, ctypes.c_longlong, ctypes.c_float, _vp, _vp,
                                           _vp, _vp]),
     "hinm_spmm": (_i32, [ctypes.POINTER(hinm_layout), _vp, _i32, _vp, _vp]),
@@ -413,6 +414,23 @@ def hinm_hard_concrete_forward(log_alpha, eps, tau: float, z_out=None, hard_out=
                                            _ptr(hard_out), _ptr(sums_out), _stream(stream)),
            "hinm_hard_concrete_forward")
     return z_out, hard_out, sums_out
+
+
+def hinm_gyro_refine_host(I_tile, band, schedule):
+    """Host refinement of a tile's 2:4 grouping (numpy in, numpy out): I_tile fp32 [T, K],
+    band int32 [n] (working order of the 2:4 channels), schedule int32 [iters, S, 2] of
+    (group, slot).  Returns (refined band, retained importance before / after each iteration)."""
+    import numpy as np
+    I_tile = np.ascontiguousarray(I_tile, dtype=np.float32)
+    band = np.ascontiguousarray(band, dtype=np.int32).copy()
+    schedule = np.ascontiguousarray(schedule, dtype=np.int32)
+    T, K = I_tile.shape
+    iters, S = schedule.shape[0], schedule.shape[1]
+    retained = np.zeros(iters + 1, dtype=np.float64)
+    _check(_lib.hinm_gyro_refine_host(I_tile.ctypes.data, T, K, band.ctypes.data, band.size,
+                                      schedule.ctypes.data, iters, S, retained.ctypes.data),
+           "hinm_gyro_refine_host")
+    return band, retained
 
 
 def hinm_device_status(stream=None) -> int:

@@ -15,7 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 SOURCES = ["abi.cu", "importance.cu", "search.cu", "mask.cu", "compress.cu", "spmm.cu",
-           "selftest.cu", "hard_concrete.cu"]
+           "selftest.cu", "hard_concrete.cu", "gyro.cu"]
 LIB = os.path.join(HERE, "libhinm.so")
 BUILD_DIR = os.path.join(HERE, "_build")
 

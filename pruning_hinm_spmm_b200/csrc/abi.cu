@@ -8,6 +8,8 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <vector>
+#include <algorithm>
 
 #include "../../include/hinm.h"
 #include "hinm_internal.h"
@@ -484,6 +486,32 @@ hinm_status hinm_compress(const void* W, const uint32_t* bitmask, const int8_t* 
                                         hinm::device_status_ptr(),
                                         static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "hinm_compress launch");
+  return ok();
+}
+
+hinm_status hinm_gyro_refine_host(const float* I_tile, int T, int K, int32_t* band, int n,
+                                  const int32_t* schedule, int iters, int S,
+                                  double* retained_out) {
+  if (!I_tile || !band) return fail(HINM_ERR_INVALID_ARG, "I_tile and band must not be NULL");
+  if (T <= 0 || K < 4 || n <= 0 || n % 4 != 0 || n > K)
+    return fail(HINM_ERR_SHAPE, "T=%d, K=%d, n=%d: need T > 0, n a positive multiple of 4, n <= K",
+                T, K, n);
+  if (iters < 0 || S < 1 || S > n / 4 || (iters > 0 && !schedule))
+    return fail(HINM_ERR_INVALID_ARG, "iters=%d, S=%d: need iters >= 0, 1 <= S <= n/4", iters, S);
+  for (int i = 0; i < n; ++i)
+    if (band[i] < 0 || band[i] >= K) return fail(HINM_ERR_INVALID_ARG, "band[%d]=%d outside [0, K)", i, band[i]);
+  std::vector<char> seen(n / 4);
+  for (int it = 0; it < iters; ++it) {
+    std::fill(seen.begin(), seen.end(), 0);
+    for (int a = 0; a < S; ++a) {
+      const int g = schedule[((size_t)it * S + a) * 2], k = schedule[((size_t)it * S + a) * 2 + 1];
+      if (g < 0 || g >= n / 4 || k < 0 || k > 3 || seen[g])
+        return fail(HINM_ERR_INVALID_ARG, "schedule[%d][%d] = (%d, %d): need distinct groups in "
+                    "[0, n/4) and slots in [0, 4)", it, a, g, k);
+      seen[g] = 1;
+    }
+  }
+  hinm::gyro_refine(I_tile, T, K, band, n, schedule, iters, S, retained_out);
   return ok();
 }
 

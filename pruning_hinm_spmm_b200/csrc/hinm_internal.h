@@ -91,6 +91,11 @@ cudaError_t launch_wait_timeout_selftest(unsigned long long limit_ns, int* statu
                                          cudaStream_t s);
 
 // tile_pairs: the caller's hint that tiles select the same X rows (HINM_SPMM_TILE_PAIRS)
+// Host: gyro-style refinement of a tile's 2:4 grouping (arguments checked by the caller).
+double gyro_band_retained(const float* I, int T, int K, const int32_t* band, int n);
+void gyro_refine(const float* I, int T, int K, int32_t* band, int n, const int32_t* schedule,
+                 int iters, int S, double* retained);
+
 cudaError_t launch_hard_concrete(const float* log_alpha, const float* eps, long long n, float tau,
                                  float* z, uint8_t* hard, double* sums, cudaStream_t s);
 

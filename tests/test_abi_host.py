@@ -178,3 +178,38 @@ def test_tile_pairs_hint_rule():
     assert not H.tile_pairs_hint([[0, K, 0], [0, 0, K]], None, K)      # tiles differ
     assert H.tile_pairs_hint(H.hinm_counts_from_vs(K, 0.5, 0.0), None, K)
     assert not H.tile_pairs_hint(H.hinm_counts_from_vs(K, 0.5, 0.25), None, K)
+
+
+@pytest.mark.parametrize("T,K,n,S,iters,seed", [(8, 32, 32, 4, 2, 1), (32, 128, 96, 8, 3, 2),
+                                                 (16, 256, 256, 32, 5, 3)])
+def test_gyro_refine_host_matches_oracle(T, K, n, S, iters, seed):
+    """The native gyro-style refinement (host code of the library) against the oracle's
+    (scipy's assignment as its step): the same refined band and the same retained-importance
+    history bit for bit (the same fp64 additions in the same order); the history never falls."""
+    import pruning_hinm_spmm_b200 as H
+    rng = np.random.default_rng(seed)
+    I_tile = rng.exponential(1.0, (T, K)).astype(np.float32)
+    band = rng.permutation(K)[:n].astype(np.int32)
+    sched = np.stack([np.stack([rng.choice(n // 4, S, replace=False), rng.integers(0, 4, S)], axis=1)
+                      for _ in range(iters)]).astype(np.int32)
+    got_band, got_hist = H.hinm_gyro_refine_host(I_tile, band, sched)
+    want_band, want_hist = O.gyro_refine(I_tile, band, sched)
+    np.testing.assert_array_equal(got_band, want_band)
+    np.testing.assert_array_equal(got_hist, want_hist)
+    assert (np.diff(got_hist) >= 0).all()
+
+
+def test_gyro_refine_host_validation():
+    import pruning_hinm_spmm_b200 as H
+    I_tile = np.ones((4, 16), dtype=np.float32)
+    band = np.arange(8, dtype=np.int32)
+    with pytest.raises(H.HinmError):
+        H.hinm_gyro_refine_host(I_tile, band[:6], np.zeros((1, 1, 2), dtype=np.int32))
+    with pytest.raises(H.HinmError):   # the same group twice in one iteration
+        H.hinm_gyro_refine_host(I_tile, band, np.array([[[0, 1], [0, 2]]], dtype=np.int32))
+    with pytest.raises(H.HinmError):   # slot outside 0..3
+        H.hinm_gyro_refine_host(I_tile, band, np.array([[[1, 4]]], dtype=np.int32))
+    bad = band.copy()
+    bad[3] = 99
+    with pytest.raises(H.HinmError):   # channel outside [0, K)
+        H.hinm_gyro_refine_host(I_tile, bad, np.array([[[1, 0]]], dtype=np.int32))
