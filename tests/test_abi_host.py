@@ -40,6 +40,21 @@ def test_exports_every_declared_symbol(H):
         assert hasattr(lib, n), f"{n} declared in include/ but not exported"
 
 
+def test_every_export_is_declared(H):
+    """The other direction: every hinm_ function the library exports is declared (and so
+    documented) in include/ -- no undocumented entry points."""
+    import shutil
+    import subprocess
+    if not shutil.which("nm"):
+        pytest.skip("nm not available")
+    out = subprocess.run(["nm", "-D", "--defined-only", H.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines()
+                if len(ln.split()) >= 3 and ln.split()[1] == "T" and ln.split()[-1].startswith("hinm_")}
+    assert exported, "no hinm_ exports found"
+    assert exported <= declared_functions(), sorted(exported - declared_functions())
+
+
 def test_versions_and_strings(H):
     lib = H.lib()
     assert lib.hinm_abi_version() == 1
