@@ -115,19 +115,45 @@ void gyro_refine(const float* I, int T, int K, int32_t* band, int n, const int32
   if (retained) retained[0] = gyro_band_retained(I, T, K, band, n);
   std::vector<double> cost((size_t)S * S);
   std::vector<int32_t> vec(S);
+  std::vector<float> top2((size_t)S * T * 2);  // per sampled group and row: the two largest
+  std::vector<float> xv((size_t)S * T);        // of its three remaining values; the vectors
   for (int it = 0; it < iters; ++it) {
     const int32_t* sc = schedule + (size_t)it * S * 2;
-    for (int a = 0; a < S; ++a) vec[a] = band[4 * sc[2 * a] + sc[2 * a + 1]];
+    for (int a = 0; a < S; ++a) {
+      vec[a] = band[4 * sc[2 * a] + sc[2 * a + 1]];
+      for (int r = 0; r < T; ++r) xv[(size_t)a * T + r] = I[(size_t)r * K + vec[a]];
+    }
     for (int b = 0; b < S; ++b) {
       const int g = sc[2 * b], k = sc[2 * b + 1];
-      int32_t m[4];
+      int32_t m[3];
       int q = 0;
       for (int j = 0; j < 4; ++j)
         if (j != k) m[q++] = band[4 * g + j];
-      for (int a = 0; a < S; ++a) {
-        m[3] = vec[a];
-        // maximise the retained importance: minimise its negative
-        cost[(size_t)a * S + b] = -group_retained(I, T, K, {m[0], m[1], m[2], m[3]});
+      for (int r = 0; r < T; ++r) {
+        const float* row = I + (size_t)r * K;
+        float v0 = row[m[0]], v1 = row[m[1]], v2 = row[m[2]];
+        if (v1 > v0) std::swap(v0, v1);
+        if (v2 > v1) std::swap(v1, v2);
+        if (v1 > v0) std::swap(v0, v1);
+        top2[((size_t)b * T + r) * 2] = v0;
+        top2[((size_t)b * T + r) * 2 + 1] = v1;
+      }
+    }
+    // cost[a][b] = -(retained importance of group b with vector a in its freed slot): per row
+    // the two largest of {x, s1, s2, s3} are {x, s1} (x >= s1), {s1, x} (s2 <= x < s1) or
+    // {s1, s2}, added as fp64 and summed over the rows in ascending order (the values and
+    // the order of group_retained, so the sums are the same)
+    for (int a = 0; a < S; ++a) {
+      const float* x = xv.data() + (size_t)a * T;
+      for (int b = 0; b < S; ++b) {
+        const float* t2 = top2.data() + (size_t)b * T * 2;
+        double acc = 0.0;
+        for (int r = 0; r < T; ++r) {
+          const float s1 = t2[2 * r], s2 = t2[2 * r + 1], xr = x[r];
+          acc += xr >= s1 ? (double)xr + (double)s1
+                          : (xr >= s2 ? (double)s1 + (double)xr : (double)s1 + (double)s2);
+        }
+        cost[(size_t)a * S + b] = -acc;  // maximise the retained importance
       }
     }
     const std::vector<int> to = min_cost_assignment(cost, S);
