@@ -84,7 +84,7 @@ def channel_energy(X_bits: np.ndarray) -> np.ndarray:
 def importance(W_bits: np.ndarray, X_bits: np.ndarray) -> np.ndarray:
     """I[i, c] = fl32( fl32(w_ic^2) * s_c ), an M x K fp32 matrix indexed by original channel.
 
-    [P1] 关键设计 1 ("保留权重的二阶重要度"), 关键设计 2 (importance matrix D).
+    [P1] 关键设计 1 (second-order importance of the weights), 关键设计 2 (importance matrix D).
     w^2 of a bf16 w is exact in fp32 (barring underflow); the product with s_c is one
     fp32 rounding.
     """
@@ -248,7 +248,8 @@ def tile_mask_working(I_tile_w: np.ndarray, region_w: np.ndarray) -> np.ndarray:
 def retained_importance(I_tile_w: np.ndarray, keep: np.ndarray) -> float:
     """R = sum of the importance of every kept element of a tile.
 
-    [P1] 关键设计 1: R_total = R_dense + R_24 ("保留权重的二阶重要度之和").  [reading] The
+    [P1] 关键设计 1: R_total = R_dense + R_24, the second-order importance summed over the
+    retained weights.  [reading] The
     sum is taken exactly and rounded once to fp64 (math.fsum is exactly rounded), so the
     comparison between candidates does not depend on a summation order.
     """
