@@ -76,7 +76,8 @@ const char* hinm_last_error(void);          /* detail of the last error on this 
 int hinm_abi_version(void);
 
 /* ---------------------------------------------------------------------------------
- * a1. Importance  ([P1] 关键设计 1 "二阶重要度", 关键设计 2 "D 是重要度矩阵")
+ * a1. Importance  ([P1] 关键设计 1: second-order importance; 关键设计 2: the importance
+ * matrix D)
  *   s_c    = sum_{n=0..N-1} x_cn^2, accumulated in fp64 with n ascending, rounded to fp32
  *   I[i,c] = fl32( fl32(w_ic^2) * s_c )
  * W: bf16 [M][K]; X: bf16 [K][N]; I_out: fp32 [M][K] (written in full).
