@@ -97,7 +97,9 @@ hinm_status hinm_importance(const void* W, const void* X, int M, int K, int N,
  *   to start at zero: every s_c is written before it is read, in stream order.
  *   Calls that overlap on one device (other streams or host threads) share the scratch
  *   and race: order them.  The first call on each device resolves the scratch address
- *   (cudaGetSymbolAddress, device current); make that call before any stream capture.
+ *   (cudaGetSymbolAddress, device current) and caches it for that device's current
+ *   context; a call from a new context (e.g. after cudaDeviceReset) resolves it again.
+ *   Make the first call in a context before any stream capture.
  *   Errors: as hinm_importance, plus HINM_ERR_CUDA if the address cannot be resolved.
  */
 hinm_status hinm_importance_noalloc(const void* W, const void* X, int M, int K, int N,

@@ -76,13 +76,64 @@ hinm_status check_search_params(double t_s, double alpha) {
   return HINM_OK;
 }
 
-// One status word per device, resolved with cudaGetSymbolAddress on first use.
+// One status word per device, its address resolved with cudaGetSymbolAddress on first use
+// in each context.
 __device__ int g_device_status;
-constexpr int kMaxDevices = 64;
-int* g_status_ptr[kMaxDevices];
-std::mutex g_status_mu;
+hinm::SymbolCache g_status_cache;
+
+// cuCtxGetCurrent, resolved through the runtime (the library does not link the driver).
+typedef int (*CtxGetCurrentFn)(void**);
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+void* current_context() {
+  void* ctx = nullptr;
+  CtxGetCurrentFn fn = ctx_get_current_fn();
+  if (!fn || fn(&ctx) != 0) return nullptr;
+  return ctx;
+}
 
 }  // namespace
+
+namespace hinm {
+
+// The address of a __device__ symbol belongs to the module loaded in one context: after
+// cudaDeviceReset (or any re-creation of the primary context) the module is loaded again
+// and the symbol can move.  The cache keeps, per device, the context the address was
+// resolved in and resolves it again when the current context differs.
+cudaError_t resolve_symbol(SymbolCache& c, const void* symbol, void** out) {
+  *out = nullptr;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= SymbolCache::kDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(c.mu);
+  void* ctx = current_context();
+  if (c.ptr[dev] && ctx && ctx == c.ctx[dev]) {
+    *out = c.ptr[dev];
+    return cudaSuccess;
+  }
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, symbol);  // makes the device's primary context current if none is
+  if (e != cudaSuccess) return e;
+  c.ptr[dev] = p;
+  c.ctx[dev] = ctx ? ctx : current_context();
+  *out = p;
+  return cudaSuccess;
+}
+
+}  // namespace hinm
 
 namespace hinm {
 
@@ -122,15 +173,9 @@ int search_candidates_host(int K, double t_s, double alpha, Candidate* out, int 
 }
 
 int* device_status_ptr() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lk(g_status_mu);
-  if (!g_status_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
-    g_status_ptr[dev] = static_cast<int*>(p);
-  }
-  return g_status_ptr[dev];
+  void* p = nullptr;
+  if (resolve_symbol(g_status_cache, &g_device_status, &p) != cudaSuccess) return nullptr;
+  return static_cast<int*>(p);
 }
 
 namespace {
@@ -500,6 +545,11 @@ hinm_status hinm_gyro_refine_host(const float* I_tile, int T, int K, int32_t* ba
     return fail(HINM_ERR_INVALID_ARG, "iters=%d, S=%d: need iters >= 0, 1 <= S <= n/4", iters, S);
   for (int i = 0; i < n; ++i)
     if (band[i] < 0 || band[i] >= K) return fail(HINM_ERR_INVALID_ARG, "band[%d]=%d outside [0, K)", i, band[i]);
+  // the assignment's potentials need finite costs: every importance the band reads is finite
+  for (int r = 0; r < T; ++r)
+    for (int i = 0; i < n; ++i)
+      if (!std::isfinite(I_tile[(size_t)r * K + band[i]]))
+        return fail(HINM_ERR_INVALID_ARG, "I_tile[%d][%d] is not finite", r, band[i]);
   std::vector<char> seen(n / 4);
   for (int it = 0; it < iters; ++it) {
     std::fill(seen.begin(), seen.end(), 0);

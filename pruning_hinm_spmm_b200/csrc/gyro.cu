@@ -64,6 +64,7 @@ std::vector<int> min_cost_assignment(const std::vector<double>& c, int n) {
           dm = d[j];
           jm = j;
         }
+      if (jm < 0) return {};  // no finite reduced cost left (the callers pass finite costs)
       settled[jm] = 1;
       if (row_of[jm] < 0) {
         jfree = jm;
@@ -157,6 +158,7 @@ void gyro_refine(const float* I, int T, int K, int32_t* band, int n, const int32
       }
     }
     const std::vector<int> to = min_cost_assignment(cost, S);
+    if ((int)to.size() != S) return;
     for (int a = 0; a < S; ++a) band[4 * sc[2 * to[a]] + sc[2 * to[a] + 1]] = vec[a];
     if (retained) retained[it + 1] = gyro_band_retained(I, T, K, band, n);
   }

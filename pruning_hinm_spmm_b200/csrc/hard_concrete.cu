@@ -34,7 +34,9 @@ __device__ __forceinline__ float hc_z(float la, float e, float inv_tau) {
   const float x = __fmul_rn(__fadd_rn(logit, la), inv_tau);
   const float s = __frcp_rn(__fadd_rn(1.0f, expf(-x)));
   const float sb = __fadd_rn(__fmul_rn(s, __fsub_rn(kHcHigh, kHcLow)), kHcLow);
-  return fminf(1.0f, fmaxf(0.0f, sb));
+  // clip to [0, 1] by comparisons, so that a NaN (a NaN input, or -inf + inf in the logit)
+  // passes through as NaN; fminf / fmaxf would return the non-NaN operand
+  return sb < 0.0f ? 0.0f : (sb > 1.0f ? 1.0f : sb);
 }
 
 __global__ void __launch_bounds__(kHcThreads) hard_concrete_kernel(

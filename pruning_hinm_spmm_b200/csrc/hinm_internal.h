@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/hinm.h"
 
 namespace hinm {
@@ -31,7 +33,17 @@ bool counts_from_vs_host(int K, double t_s, double v_s, int out[3]);
 // -1 when the start boundary itself is invalid.
 int search_candidates_host(int K, double t_s, double alpha, Candidate* out, int cap);
 
-// Per-device address of the library's status word (resolved once per device).
+// Device address of a __device__ symbol of this library in the current context: resolved
+// with cudaGetSymbolAddress once per (device, context) and cached.
+struct SymbolCache {
+  static constexpr int kDevices = 64;
+  std::mutex mu;
+  void* ctx[kDevices] = {};
+  void* ptr[kDevices] = {};
+};
+cudaError_t resolve_symbol(SymbolCache& c, const void* symbol, void** out);
+
+// Address of the library's status word on the current device (resolve_symbol).
 int* device_status_ptr();
 
 // Sets kernel `fn`'s maximum dynamic shared memory to `bytes` on the current device, once per

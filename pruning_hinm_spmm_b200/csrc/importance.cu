@@ -181,29 +181,17 @@ int sm_count() {
 // c < K before importance_kernel reads it, in stream order).
 static __device__ __align__(256) float g_noalloc_energy[kNoAllocMaxK];
 
-constexpr int kMaxNoAllocDevices = 64;
-std::mutex g_noalloc_mu;
-float* g_noalloc_ptr[kMaxNoAllocDevices] = {};
+SymbolCache g_noalloc_cache;
 
 }  // namespace
 
-// Address of this device's static scratch, resolved once per device (the caller's current
-// device is the one the call runs on).
+// Address of the static scratch on the current device (the caller's current device is the
+// one the call runs on), resolved with cudaGetSymbolAddress once per device and context.
 cudaError_t noalloc_energy_scratch(float** out) {
-  *out = nullptr;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxNoAllocDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_energy);
-    if (e != cudaSuccess) return e;
-    g_noalloc_ptr[dev] = static_cast<float*>(p);
-  }
-  *out = g_noalloc_ptr[dev];
-  return cudaSuccess;
+  void* p = nullptr;
+  cudaError_t e = resolve_symbol(g_noalloc_cache, &g_noalloc_energy, &p);
+  *out = static_cast<float*>(p);
+  return e;
 }
 
 size_t tile_stats_v_bytes(int M, int K, int T) {
