@@ -57,6 +57,21 @@ def job_value(flops_per_rank: float, world: int, t_max: float) -> float:
     return flops_per_rank * world / t_max / 1e12
 
 
+def gather_rows(Y_shard, M: int, T: int, world: int, dist, shard_tiles):
+    """The optional collective of the tile-sharded run: every rank's row block of Y, padded
+    to the largest shard, all-gathered (NCCL on GPUs, gloo on CPU) and cut back into the full
+    M x N matrix in rank order.  Every rank calls it at the same point."""
+    import torch
+    rows = [shard_tiles(M, T, world, r) for r in range(world)]
+    most = max(r1 - r0 for r0, r1 in rows)
+    N = Y_shard.shape[1]
+    pad = torch.zeros((most, N), dtype=Y_shard.dtype, device=Y_shard.device)
+    pad[:Y_shard.shape[0]] = Y_shard
+    parts = [torch.empty_like(pad) for _ in range(world)]
+    dist.all_gather(parts, pad)
+    return torch.cat([parts[r][:r1 - r0] for r, (r0, r1) in enumerate(rows)], dim=0)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -173,13 +188,14 @@ def cpu_oracle_sample(w, tiles_n: int):
     tiles = list(range(tiles_n))
     rows = np.arange(0, tiles_n * T)
     t0 = time.perf_counter()
-    s = O.channel_energy(w.X_bits)
-    Wf = hi.bf16_bits_to_f32(w.W_bits[rows])
     I = np.zeros((M, K), dtype=np.float32)
-    I[rows] = ((Wf * Wf).astype(np.float32) * s[None, :]).astype(np.float32)
+    I[rows] = O.importance_rows(w.W_bits, w.X_bits, rows)
     sr = O.boundary_search(I, w.perm, T, w.t_s, w.alpha, tiles=tiles)
-    bm, reg = O.mask(I, w.perm, T, sr.counts, tiles=tiles)
-    O.compress(w.W_bits, bm, reg, w.perm, sr.counts, T, tiles=tiles)
+    counts = sr.counts  # the GPU arm's rule: a fixed boundary's counts where the workload has one
+    if w.v_s is not None:
+        counts = np.tile(np.array(O.counts_from_vs(K, w.t_s, w.v_s), dtype=np.int32), (M // T, 1))
+    bm, reg = O.mask(I, w.perm, T, counts, tiles=tiles)
+    O.compress(w.W_bits, bm, reg, w.perm, counts, T, tiles=tiles)
     O.spmm_reference(w.W_bits, bm, w.X_bits, rows=rows)
     dt = time.perf_counter() - t0
     return dt, 2.0 * len(rows) * K * N

@@ -88,7 +88,14 @@ def importance(W_bits: np.ndarray, X_bits: np.ndarray) -> np.ndarray:
     w^2 of a bf16 w is exact in fp32 (barring underflow); the product with s_c is one
     fp32 rounding.
     """
-    W = _bf16_to_f32(W_bits)
+    return importance_rows(W_bits, X_bits, None)
+
+
+def importance_rows(W_bits: np.ndarray, X_bits: np.ndarray,
+                    rows: Optional[np.ndarray]) -> np.ndarray:
+    """The rows ``rows`` of ``importance(W, X)`` (every row when rows is None), with the
+    channel energies s_c still taken over all of X: I[i, c] = fl32(fl32(w_ic^2) * s_c)."""
+    W = _bf16_to_f32(W_bits if rows is None else np.asarray(W_bits)[rows])
     s = channel_energy(X_bits)
     w2 = (W * W).astype(np.float32)
     return (w2 * s[None, :]).astype(np.float32)

@@ -66,6 +66,17 @@ def test_importance_hand_example_not_transposed():
     np.testing.assert_array_equal(O.importance(W, X), np.array([[3, 16], [27, 1]], dtype=np.float32))
 
 
+def test_importance_rows_hand_example():
+    # the hand example above: row 1 alone is [27, 1], row 0 alone [3, 16]; the energies are
+    # still taken over all of X
+    W = bf([[1.0, 2.0], [3.0, 0.5]])
+    X = bf([[1.0, 1.0, 1.0], [2.0, 0.0, 0.0]])
+    np.testing.assert_array_equal(O.importance_rows(W, X, np.array([1])),
+                                  np.array([[27, 1]], dtype=np.float32))
+    np.testing.assert_array_equal(O.importance_rows(W, X, np.array([1, 0])),
+                                  np.array([[27, 1], [3, 16]], dtype=np.float32))
+
+
 def test_importance_exact_rational():
     rng = np.random.default_rng(3)
     M, K, N = 5, 6, 9
