@@ -453,6 +453,23 @@ def tile_pairs_hint(counts, perm, K: int) -> bool:
     return bool(one_region and ascending)
 
 
+# ----------------------------------------------------------------------------- multi-GPU
+def shard_tiles(M: int, T: int, world: int, rank: int) -> Tuple[int, int]:
+    """Output rows [row0, row1) of W (and of Y) that rank ``rank`` of ``world`` takes when the
+    tiles of one W are split across GPUs: every tile of T rows is computed independently
+    (importance rows, boundary search, mask, compress and product need only the tile's rows
+    of W and all of X), so rank r takes a contiguous run of whole tiles, the first
+    (M/T) mod world ranks one tile more than the rest.  The ranges cover [0, M) exactly and
+    in rank order; a rank may get none when there are fewer tiles than ranks."""
+    if T <= 0 or M % T or world <= 0 or not 0 <= rank < world:
+        raise ValueError(f"shard_tiles: M={M}, T={T}, world={world}, rank={rank}")
+    nt = M // T
+    base, extra = divmod(nt, world)
+    t0 = rank * base + min(rank, extra)
+    t1 = t0 + base + (1 if rank < extra else 0)
+    return t0 * T, t1 * T
+
+
 # ----------------------------------------------------------------------------- whole path
 class HotPath:
     """Preallocated buffers for importance -> search -> mask -> compress -> spmm on one

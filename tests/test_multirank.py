@@ -76,3 +76,100 @@ def test_two_gloo_ranks_shards_max_timing_and_reference_arm():
     line = json.loads(r0[6].strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["cpu_baseline"]["kind"] == "oracle"
     assert r1[6].strip() == ""                               # rank 1 prints nothing
+
+
+# ---------------------------------------------------------------- tile-sharded split
+def test_shard_tiles_cover_rows_exactly():
+    """Contiguous runs of whole tiles, in rank order, covering [0, M) exactly; sizes differ by
+    at most one tile; ranks beyond the tile count get empty ranges."""
+    import pruning_hinm_spmm_b200 as H
+    for M, T in ((11008, 128), (4096, 128), (256, 64), (640, 64), (128, 128)):
+        nt = M // T
+        for world in (1, 2, 3, 4, 7, 8, 16):
+            rng = [H.shard_tiles(M, T, world, r) for r in range(world)]
+            assert rng[0][0] == 0 and rng[-1][1] == M
+            for (a0, a1), (b0, b1) in zip(rng, rng[1:]):
+                assert a1 == b0
+            sizes = [(r1 - r0) // T for r0, r1 in rng]
+            assert all((r1 - r0) % T == 0 and r1 >= r0 for r0, r1 in rng)
+            assert max(sizes) - min(sizes) <= 1 and sum(sizes) == nt
+    with pytest.raises(ValueError):
+        H.shard_tiles(200, 64, 2, 0)
+
+
+def _shard_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import torch.distributed as dist
+    import bench
+    import hinm_inputs as hi
+    import pruning_hinm_spmm_b200 as H
+    from oracle import hinm_oracle as O
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    # 10 tiles of 64 rows over the ranks; X (and the permutation) replicated
+    w = hi.custom(640, 256, 24, 64, seed=11, t_s=0.625, v_s=None, random_perm=True)
+    r0, r1 = H.shard_tiles(w.M, w.T, world, rank)
+    part = O.hot_path(w.W_bits[r0:r1], w.X_bits, w.perm, w.T, w.t_s, w.alpha)
+    L = part["layout"]
+    blocks = []
+    for t in range(L.tile_info.shape[0]):
+        nd, ns, d0, s0 = (int(x) for x in L.tile_info[t])
+        blocks.append((L.vals_dense[d0:d0 + nd].tobytes(), L.vals_sparse[s0:s0 + ns].tobytes(),
+                       L.meta[s0:s0 + ns].tobytes(), L.idx_dense[d0:d0 + nd].tobytes(),
+                       L.idx_sparse[s0:s0 + ns].tobytes()))
+    Y = bench.gather_rows(torch.from_numpy(part["y"]), w.M, w.T, world, dist, H.shard_tiles)
+    gathered = [None] * world
+    dist.all_gather_object(gathered, dict(rows=(r0, r1), counts=part["counts"],
+                                          bitmask=part["bitmask"], region=part["region"],
+                                          blocks=blocks))
+    dist.barrier()
+    dist.destroy_process_group()
+    q.put((rank, Y.numpy(), gathered))
+
+
+def test_tile_sharded_run_equals_unsharded():
+    """Two gloo ranks each run the oracle's whole path on their tile shard of one W (X
+    replicated); concatenated in rank order, their counts, masks, regions, per-tile layout
+    bytes and Y rows (the Y rows through the same all-gather the benchmark uses) equal the
+    unsharded run's."""
+    import numpy as np
+    import hinm_inputs as hi
+    from oracle import hinm_oracle as O
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    world = 2
+    procs = [ctx.Process(target=_shard_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = {}
+    try:
+        for _ in range(world):
+            r = q.get(timeout=300)
+            res[r[0]] = r
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+            if p.is_alive():
+                p.kill()
+    assert all(p.exitcode == 0 for p in procs)
+    w = hi.custom(640, 256, 24, 64, seed=11, t_s=0.625, v_s=None, random_perm=True)
+    full = O.hot_path(w.W_bits, w.X_bits, w.perm, w.T, w.t_s, w.alpha)
+    parts = res[0][2]
+    assert [p["rows"] for p in parts] == [(0, 320), (320, 640)]
+    np.testing.assert_array_equal(np.concatenate([p["counts"] for p in parts]), full["counts"])
+    np.testing.assert_array_equal(np.concatenate([p["bitmask"] for p in parts]), full["bitmask"])
+    np.testing.assert_array_equal(np.concatenate([p["region"] for p in parts]), full["region"])
+    L = full["layout"]
+    blocks = [b for p in parts for b in p["blocks"]]
+    for t in range(L.tile_info.shape[0]):
+        nd, ns, d0, s0 = (int(x) for x in L.tile_info[t])
+        want = (L.vals_dense[d0:d0 + nd].tobytes(), L.vals_sparse[s0:s0 + ns].tobytes(),
+                L.meta[s0:s0 + ns].tobytes(), L.idx_dense[d0:d0 + nd].tobytes(),
+                L.idx_sparse[s0:s0 + ns].tobytes())
+        assert blocks[t] == want, f"tile {t}"
+    for r in range(world):  # the gathered Y on every rank: the unsharded rows
+        np.testing.assert_allclose(res[r][1], full["y"], rtol=1e-13, atol=1e-13)
