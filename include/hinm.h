@@ -231,26 +231,99 @@ hinm_status hinm_compress(const void* W, const uint32_t* bitmask, const int8_t* 
                           const hinm_layout* layout, void* workspace,
                           size_t workspace_bytes, void* stream);
 
-/* Gyro-style refinement of one tile's 2:4 grouping, on the host  ([P1] 关键设计 2: the
- * channel permutation reorders channels without changing the product so that important
- * weights land where they are kept; per tile, sampled vectors are re-assigned by the
- * Hungarian algorithm on the pruning-cost matrix, iterated to refine).  An offline,
- * once-per-layer step: its output is the working order the hot path takes as `perm`.
- *   The band is the tile's 2:4 channels in working order, groups = 4 consecutive entries;
- *   a group's retained importance = sum over the tile's rows (ascending, fp64) of its two
- *   largest values.  Iteration i takes schedule[i][0..S) = (group, slot) pairs (distinct
- *   groups; the caller's random draws): the S sampled channels leave their slots and go
- *   back by the assignment that maximises the sampled groups' total retained importance
- *   (reading: the balanced clustering of S vectors into the S freed slots, capacity 1 each,
- *   is that assignment).  The retained importance never decreases.
- * I_tile: host fp32 [T][K] (the tile's importance rows, by channel); band: host int32 [n],
- * n % 4 == 0, n <= K, entries in [0, K), refined in place; schedule: host int32
- * [iters][S][2]; retained_out (NULL allowed): host fp64 [iters + 1], the band's retained
- * importance before and after each iteration.
- * Errors (checked before any work): HINM_ERR_SHAPE, HINM_ERR_INVALID_ARG. */
-hinm_status hinm_gyro_refine_host(const float* I_tile, int T, int K, int32_t* band, int n,
-                                  const int32_t* schedule, int iters, int S,
-                                  double* retained_out);
+/* Per-tile working orders  ([P1] 关键设计 2: the input-channel permutation is found inside
+ * each tile, and it is folded into the tile's HiNM index).  The _ex forms of the search,
+ * the mask and compress take perm_per_tile: 0 = perm is one order int32 [K] for every tile
+ * (the calls above), 1 = perm is int32 [M/T][K], row t the working order of tile t (each
+ * row a permutation of 0..K-1; a bad row sets HINM_ERR_INVALID_ARG in the device status
+ * word, as for the shared order).  Working position j of tile t holds channel perm[t][j]:
+ * the tile's 2:4 groups are 4 consecutive 2:4 channels in that order, and compress folds
+ * perm[t] into tile t's index, so the SpMM needs nothing else.  The same perm and flag must
+ * be given to the three calls.  Other arguments, results and errors as the calls above;
+ * hinm_boundary_search_ex covers both search forms (stats may be NULL). */
+hinm_status hinm_boundary_search_ex(const float* I, const void* stats, size_t stats_bytes,
+                                    const int32_t* perm, int perm_per_tile, int M, int K, int T,
+                                    double t_s, double alpha, int32_t* counts_out, double* vs_out,
+                                    int32_t* rank_out, double* retained_out, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+hinm_status hinm_mask_ex(const float* I, const int32_t* perm, int perm_per_tile,
+                         const int32_t* counts, const int32_t* rank, int M, int K, int T,
+                         uint32_t* bitmask_out, int8_t* region_out, void* workspace,
+                         size_t workspace_bytes, void* stream);
+hinm_status hinm_compress_ex(const void* W, const uint32_t* bitmask, const int8_t* region,
+                             const int32_t* perm, int perm_per_tile, const int32_t* counts,
+                             int M, int K, int T, const hinm_layout* layout, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/* Gyro-permutation  ([P1] 关键设计 2: channel permutation reorders input and output
+ * channels without changing the product, so that important weights land where they are
+ * kept; the pipeline is output-channel permutation -> column-vector pruning -> in-tile
+ * input-channel permutation, and each round samples vectors per tile, clusters them with a
+ * balanced K-means and assigns the clusters by the Hungarian algorithm on the pruning-cost
+ * matrix, smaller cost better; iterated to refine).  Offline, once per layer; its outputs
+ * are the permutations the hot path takes: a per-tile working order (perm_per_tile of
+ * hinm_boundary_search_ex / hinm_mask_ex / hinm_compress_ex) and an output-row order.
+ * All costs are row-ascending fp64 sums of fp32 importances, so the host calls, the device
+ * call and an fp64 reference agree bit for bit.
+ *
+ * In-tile input-channel round.  band: the tile's 2:4-region channels in working order
+ * (groups = 4 consecutive entries), host int32 [n], n % 4 == 0, 4 <= n <= K, distinct
+ * entries in [0, K), refined in place.  The caller's random draws choose G distinct groups
+ * (groups: host int32 [G], in [0, n/4)) and k distinct slots in each (slots: host int32
+ * [G][k], in [0, 4), 1 <= k <= 4); the S = G k sampled vectors (sample i k + j = the vector
+ * in slot slots[i][j] of group groups[i]) leave their slots.  Reading of the pages: their
+ * features are their importance columns over the tile's rows; a balanced K-means (seeded
+ * by source group; Lloyd steps whose assignment is the min-cost assignment of the samples
+ * to G clusters x k seats under the squared distance; at most kmeans_iters steps, stopping
+ * when the partition repeats) groups them into G clusters of k; cost[c][i] = the pruning
+ * cost of group groups[i] (per row the two smallest of its four values) with its sampled
+ * slots, ascending, holding cluster c's vectors in ascending sample order; the min-cost
+ * assignment places the clusters, and the result is kept only if the sampled groups' total
+ * cost does not rise.  cost_out (NULL allowed): host fp64 [2] = {before, after}.
+ * I_tile: host fp32 [T][K], the tile's importance rows by channel; every value the round
+ * reads must be finite.  Errors (before any work): HINM_ERR_SHAPE, HINM_ERR_INVALID_ARG. */
+hinm_status hinm_gyro_input_round_host(const float* I_tile, int T, int K, int32_t* band, int n,
+                                       const int32_t* groups, const int32_t* slots, int G, int k,
+                                       int kmeans_iters, double* cost_out);
+
+/* Pruning cost of a whole band (fp64 sum over its groups, ascending): host. */
+hinm_status hinm_gyro_band_cost_host(const float* I_tile, int T, int K, const int32_t* band,
+                                     int n, double* cost_host);
+
+/* The input rounds' cost matrices of every tile of a layer on the GPU (the G x G x T part):
+ *   cost_out[t][c][i] = pruning cost of tile t's group groups[t][i] with its slots
+ *   slots[t][i][0..k) (ascending) holding the vectors of cluster c, clusters[t][c][0..k)
+ *   (ascending sample indices p in [0, G k), sample p = slot slots[t][p/k][p%k] of group
+ *   groups[t][p/k]).
+ * I: device fp32 [M][K] (tile t = rows t T .. t T + T - 1); bands: device int32
+ * [M/T][band_len]; groups [M/T][G], slots [M/T][G][k], clusters [M/T][G][k]: device int32;
+ * cost_out: device fp64 [M/T][G][G].  1 <= k <= 4, 1 <= G <= band_len / 4.  A channel
+ * outside [0, K) is read as channel 0 and reported as HINM_ERR_INVALID_ARG in the device
+ * status word; the other indices must be valid (they are not checked on the device). */
+hinm_status hinm_gyro_cost_matrix(const float* I, int M, int K, int T, const int32_t* bands,
+                                  int band_len, const int32_t* groups, const int32_t* slots,
+                                  const int32_t* clusters, int G, int k, double* cost_out,
+                                  void* stream);
+
+/* Output-channel round over a layer's tiles, on the host.  row_order: host int32 [M], a
+ * permutation of 0..M-1 listing the output channels in their current order (tile t holds
+ * row_order[t T .. t T + T - 1]), refined in place.  The caller's draws choose G distinct
+ * tiles (tiles: host int32 [G]) and k distinct positions in each (rows: host int32 [G][k],
+ * in [0, T)).  Reading: the S = G k output channels leave their positions; their features
+ * are their importance rows; the balanced K-means (as above) groups them into G clusters of
+ * k; cost[c][i] = the column-vector pruning cost of tile tiles[i] with its sampled
+ * positions, ascending, holding cluster c's channels: the sum of the tile's n0[tile]
+ * smallest vector scores (column sums over the tile's rows in their order, fp64; ties by
+ * channel), summed ascending; the min-cost assignment places the clusters, kept only if the
+ * sampled tiles' total cost does not rise.  The layer then computes W[row_order] and yields
+ * Y[row_order]; hinm_translate_index with the inverse order lets the next layer read it.
+ * I: host fp32 [M][K] (rows = output channels, by channel); n0: host int32 [M/T], in
+ * [0, K].  cost_out (NULL allowed): host fp64 [2] = {before, after}.
+ * Errors (before any work): HINM_ERR_SHAPE, HINM_ERR_INVALID_ARG. */
+hinm_status hinm_gyro_output_round_host(const float* I, int M, int K, int T, const int32_t* n0,
+                                        int32_t* row_order, const int32_t* tiles,
+                                        const int32_t* rows, int G, int k, int kmeans_iters,
+                                        double* cost_out);
 
 /* Hard-Concrete soft 2:4 mask, forward  ([P1] 关键设计 3: each group of 4 has learnable
  * logits log alpha; with noise eps ~ U(0, 1) the soft mask is

@@ -104,8 +104,15 @@ def importance_rows(W_bits: np.ndarray, X_bits: np.ndarray,
 # ---------------------------------------------------------------------------------------
 # a2. vector scores
 # ---------------------------------------------------------------------------------------
+def tile_perm(perm: np.ndarray, t: int) -> np.ndarray:
+    """Working order of tile t: ``perm`` is one order [K] for every tile or one per tile
+    [M/T, K] ([P1] 关键设计 2: the input-channel permutation is found inside each tile)."""
+    perm = np.asarray(perm)
+    return perm if perm.ndim == 1 else perm[t]
+
+
 def vector_scores(I: np.ndarray, perm: np.ndarray, T: int) -> np.ndarray:
-    """V[t, j] = sum over the tile's rows (ascending) of I[row, perm[j]], in fp64.
+    """V[t, j] = sum over the tile's rows (ascending) of I[row, perm_t[j]], in fp64.
 
     [P1] 整体框架 (W is cut into tiles of output rows), 研究背景 (vectors are ranked by
     importance), 亮点与洞察 (vector-level regions).  [reading] A vector is one input
@@ -114,7 +121,10 @@ def vector_scores(I: np.ndarray, perm: np.ndarray, T: int) -> np.ndarray:
     """
     M, K = I.shape
     nt = M // T
-    Iw = I[:, perm].reshape(nt, T, K)
+    if np.asarray(perm).ndim == 1:
+        Iw = I[:, perm].reshape(nt, T, K)
+    else:
+        Iw = np.stack([I[t * T:(t + 1) * T][:, tile_perm(perm, t)] for t in range(nt)])
     V = np.zeros((nt, K), dtype=np.float64)
     for i in range(T):                      # fixed order: rows ascending
         V += Iw[:, i, :].astype(np.float64)
@@ -294,8 +304,9 @@ def boundary_search(I: np.ndarray, perm: np.ndarray, T: int, t_s: float, alpha: 
     rank = np.zeros((nt, K), dtype=np.int32)
     Rs: List[List[float]] = [[] for _ in range(nt)]
     for t in (range(nt) if tiles is None else tiles):
-        I_tile_w = I[t * T:(t + 1) * T][:, perm]
-        V_t = V[t] if V is not None else vector_scores(I[t * T:(t + 1) * T], perm, T)[0]
+        I_tile_w = I[t * T:(t + 1) * T][:, tile_perm(perm, t)]
+        V_t = V[t] if V is not None else vector_scores(I[t * T:(t + 1) * T], tile_perm(perm, t),
+                                                       T)[0]
         order = vector_order(V_t)
         rank[t, order] = np.arange(K, dtype=np.int32)
         R = []
@@ -331,16 +342,17 @@ def mask(I: np.ndarray, perm: np.ndarray, T: int, counts: np.ndarray,
     bitmask = np.zeros((M, words), dtype=np.uint32)
     region = np.zeros((nt, K), dtype=np.int8)
     for t in (range(nt) if tiles is None else tiles):
-        I_tile_w = I[t * T:(t + 1) * T][:, perm]
-        V_t = vector_scores(I[t * T:(t + 1) * T], perm, T)[0]
+        pt = tile_perm(perm, t)
+        I_tile_w = I[t * T:(t + 1) * T][:, pt]
+        V_t = vector_scores(I[t * T:(t + 1) * T], pt, T)[0]
         order = vector_order(V_t)
         rank_t = np.empty(K, dtype=np.int32)
         rank_t[order] = np.arange(K, dtype=np.int32)
         reg_w = regions_from_rank(rank_t, tuple(int(x) for x in counts[t]))
         keep_w = tile_mask_working(I_tile_w, reg_w)
         keep_c = np.zeros((T, K), dtype=bool)
-        keep_c[:, perm] = keep_w
-        region[t, perm] = reg_w
+        keep_c[:, pt] = keep_w
+        region[t, pt] = reg_w
         bitmask[t * T:(t + 1) * T] = pack_bits(keep_c)
     return bitmask, region
 
@@ -444,7 +456,8 @@ def compress(W_bits: np.ndarray, bitmask: np.ndarray, region: np.ndarray, perm: 
     Wb = np.asarray(W_bits, dtype=np.uint16)
     for t in (range(nt) if tiles is None else tiles):
         nd, ns, d0, s0 = (int(x) for x in info[t])
-        reg_w = region[t][perm]
+        pt = tile_perm(perm, t)
+        reg_w = region[t][pt]
         dense_j = np.nonzero(reg_w == REGION_DENSE)[0]
         sp_j = np.nonzero(reg_w == REGION_24)[0]
         rows = range(t * T, (t + 1) * T)
@@ -455,7 +468,7 @@ def compress(W_bits: np.ndarray, bitmask: np.ndarray, region: np.ndarray, perm: 
                 p = b * DENSE_BK + k
                 if p >= dense_j.size:
                     continue
-                c = int(perm[dense_j[p]])
+                c = int(pt[dense_j[p]])
                 idx_dense[d0 + b, k] = c
                 for r, i in enumerate(rows):
                     v = int(Wb[i, c]) if keep_c[i, c] else 0
@@ -469,7 +482,7 @@ def compress(W_bits: np.ndarray, bitmask: np.ndarray, region: np.ndarray, perm: 
             mw = np.zeros(META_WORDS, dtype=np.uint64)
             for g in range(SPARSE_BK // 4):
                 base = b * SPARSE_BK + 4 * g
-                members = [int(perm[sp_j[base + k]]) if base + k < sp_j.size else None
+                members = [int(pt[sp_j[base + k]]) if base + k < sp_j.size else None
                            for k in range(4)]
                 for k in range(4):
                     if members[k] is not None:
@@ -664,7 +677,7 @@ def spmm_epilogue_reference(y: np.ndarray, bias: Optional[np.ndarray], act: int)
 
 
 # ---------------------------------------------------------------------------------------
-# Gyro-style refinement of a tile's 2:4 grouping (offline; produces the working order)
+# Gyro-permutation (offline; produces the per-tile working order and the row order)
 # ---------------------------------------------------------------------------------------
 def group_retained(I_tile: np.ndarray, members: List[int]) -> float:
     """Retained 2:4 importance of one group: over the tile's rows (ascending, fp64 sum),
@@ -677,42 +690,222 @@ def group_retained(I_tile: np.ndarray, members: List[int]) -> float:
     return acc
 
 
-def gyro_refine(I_tile: np.ndarray, band: np.ndarray, schedule: np.ndarray):
-    """Refine the grouping of a tile's 2:4 band (channels in working order, groups of 4
-    consecutive entries) by sampled re-assignment ([P1] 关键设计 2, gyro-permutation: sample
-    vectors per tile, cluster them into balanced clusters, and assign by the Hungarian
-    algorithm on the pruning-cost matrix; the permutation leaves the product unchanged).
+def group_pruning_cost(I_tile: np.ndarray, members: List[int]) -> float:
+    """Pruning cost of one 2:4 group: over the tile's rows (ascending, fp64 sum), the two
+    smallest of the group's four values -- the importance the 2:4 selection removes
+    ([P1] 关键设计 2: the assignment minimises the pruning cost).  Per row the larger of the
+    two is added first: acc += (double)third + (double)fourth."""
+    acc = 0.0
+    for r in range(I_tile.shape[0]):
+        v = sorted((float(I_tile[r, c]) for c in members), reverse=True)
+        acc += v[2] + v[3]
+    return acc
 
-    [reading] Iteration i takes the schedule's S (group, slot) pairs (distinct groups; the
-    caller's random draws): the S sampled vectors leave their slots, and the balanced
-    clustering of S vectors into the S freed slots (capacity 1 each) is the assignment that
-    maximises the sum over groups of the retained importance of each group with the vector
-    placed in its freed slot -- the Hungarian algorithm on that cost matrix (here
-    scipy.optimize.linear_sum_assignment as the assignment step).  Keeping every vector in
-    place is one assignment, so the retained importance never decreases.
-    Returns (refined band, retained importance of the band before and after each iteration).
+
+def balanced_kmeans(F: np.ndarray, k: int, iters: int) -> List[List[int]]:
+    """Balanced K-means of S = G k points (rows of F, fp64) into G clusters of exactly k.
+
+    [P1] 关键设计 2 names a balanced K-means over the sampled vectors.  [reading] Lloyd
+    iterations from the initial partition "points G_i k .. G_i k + k - 1 form cluster i" (the
+    vectors sampled from the same group); each iteration takes every cluster's centroid (the
+    mean of its members, summed in ascending point order, divided by k) and reassigns the
+    points by the min-cost assignment of the S points to the G k seats (cluster c's k seats)
+    under the squared Euclidean distance (summed over ascending coordinates) -- which keeps
+    every cluster at exactly k -- until the partition repeats or after ``iters`` iterations.
+    The assignment step is a library routine (scipy's linear_sum_assignment).  Returns the
+    clusters as ascending lists of point indices, cluster i's seed being group i.
+    """
+    from scipy.optimize import linear_sum_assignment
+
+    S, d = F.shape
+    G = S // k
+    clusters = [list(range(i * k, (i + 1) * k)) for i in range(G)]
+    for _ in range(iters):
+        C = np.zeros((G, d))
+        for c in range(G):
+            acc = np.zeros(d)
+            for p in clusters[c]:
+                acc = acc + F[p]
+            C[c] = acc / k
+        cost = np.zeros((S, S))
+        for p in range(S):
+            for c in range(G):
+                diff = F[p] - C[c]
+                dist = 0.0
+                for x in diff:                      # ascending coordinates
+                    dist += x * x
+                cost[p, c * k:(c + 1) * k] = dist
+        rows, cols = linear_sum_assignment(cost)
+        new = [sorted(int(p) for p, seat in zip(rows, cols) if seat // k == c) for c in range(G)]
+        if new == clusters:
+            break
+        clusters = new
+    return clusters
+
+
+def gyro_input_round(I_tile: np.ndarray, band: np.ndarray, groups: np.ndarray,
+                     slots: np.ndarray, kmeans_iters: int = 8):
+    """One round of the in-tile input-channel gyro-permutation on a tile's 2:4 band.
+
+    [P1] 关键设计 2: per tile, sample vectors, cluster them with a balanced K-means, then
+    assign the clusters by the Hungarian algorithm on the pruning-cost matrix (smaller is
+    better); the permutation leaves the product unchanged and is folded into the index.
+    [reading] ``band`` is the tile's 2:4-region channels in working order (groups of 4
+    consecutive entries).  The caller's random draws choose G distinct groups and, in each,
+    k slots (``groups`` [G], ``slots`` [G, k]); the S = G k vectors in those slots leave them
+    (sample order: group by group, slots as given).  Their features are their importance
+    columns over the tile's rows; the balanced K-means groups them into G clusters of k,
+    seeded by their source groups; cost[c][i] is the pruning cost of group groups[i] with its
+    sampled slots, in ascending slot order, holding cluster c's vectors in ascending sample
+    order.  The minimum-cost assignment (scipy's linear_sum_assignment) places the clusters;
+    the new arrangement is kept only if the sampled groups' total pruning cost (fp64, in the
+    order of ``groups``) does not rise ("iterated to refine": a round never makes it worse).
+    Returns (band, (cost before, cost after)).
     """
     from scipy.optimize import linear_sum_assignment
 
     band = np.array(band, dtype=np.int64).copy()
-    ng = band.size // 4
+    groups = [int(g) for g in np.asarray(groups).ravel()]
+    slots = np.asarray(slots, dtype=np.int64)
+    G, k = slots.shape
+    vecs = [int(band[4 * g + int(s)]) for g, ss in zip(groups, slots) for s in ss]
+    F = np.asarray(I_tile, dtype=np.float64)[:, vecs].T.copy()      # S x T
+    clusters = balanced_kmeans(F, k, kmeans_iters)
 
-    def total(b):
-        return sum(group_retained(I_tile, [int(x) for x in b[4 * g:4 * g + 4]]) for g in range(ng))
+    def members_with(i, cl):
+        g = groups[i]
+        m = [int(x) for x in band[4 * g:4 * g + 4]]
+        for s, p in zip(sorted(int(x) for x in slots[i]), cl):
+            m[s] = vecs[p]
+        return m
 
-    hist = [total(band)]
-    for it in range(schedule.shape[0]):
-        groups = [int(g) for g in schedule[it, :, 0]]
-        slots = [int(k) for k in schedule[it, :, 1]]
-        vecs = [int(band[4 * g + k]) for g, k in zip(groups, slots)]
-        S = len(groups)
-        C = np.zeros((S, S))
-        for b, (g, k) in enumerate(zip(groups, slots)):
-            rest = [int(band[4 * g + j]) for j in range(4) if j != k]
-            for a in range(S):
-                C[a, b] = group_retained(I_tile, rest + [vecs[a]])
-        rows, cols = linear_sum_assignment(C, maximize=True)
-        for a, b in zip(rows, cols):
-            band[4 * groups[b] + slots[b]] = vecs[a]
-        hist.append(total(band))
-    return band, np.array(hist)
+    cost = gyro_input_cost_matrix(I_tile, band, groups, slots, clusters)
+    rows, cols = linear_sum_assignment(cost)
+    before = 0.0
+    for i in range(G):
+        g = groups[i]
+        before += group_pruning_cost(I_tile, [int(x) for x in band[4 * g:4 * g + 4]])
+    assign = {int(i): int(c) for c, i in zip(rows, cols)}
+    after = 0.0
+    for i in range(G):
+        after += cost[assign[i], i]
+    if after <= before:
+        new = band.copy()
+        for i in range(G):
+            m = members_with(i, clusters[assign[i]])
+            new[4 * groups[i]:4 * groups[i] + 4] = m
+        return new, (before, after)
+    return band, (before, before)
+
+
+def gyro_input_cost_matrix(I_tile: np.ndarray, band: np.ndarray, groups, slots,
+                           clusters: List[List[int]]) -> np.ndarray:
+    """cost[c][i] of ``gyro_input_round``: the pruning cost of group groups[i] with its sampled
+    slots (ascending) holding the vectors of cluster c (ascending sample order; a sample's
+    vector is band[4 groups[g] + slots[g][j]] for sample g k + j)."""
+    band = np.asarray(band, dtype=np.int64)
+    groups = [int(g) for g in np.asarray(groups).ravel()]
+    slots = np.asarray(slots, dtype=np.int64)
+    G, k = slots.shape
+    vecs = [int(band[4 * g + int(s)]) for g, ss in zip(groups, slots) for s in ss]
+    cost = np.zeros((len(clusters), G))
+    for c, cl in enumerate(clusters):
+        for i in range(G):
+            g = groups[i]
+            m = [int(x) for x in band[4 * g:4 * g + 4]]
+            for s, p in zip(sorted(int(x) for x in slots[i]), cl):
+                m[s] = vecs[p]
+            cost[c, i] = group_pruning_cost(I_tile, m)
+    return cost
+
+
+def band_pruning_cost(I_tile: np.ndarray, band: np.ndarray) -> float:
+    """Pruning cost of a whole band: fp64 sum over its groups (ascending) of their costs."""
+    acc = 0.0
+    for g in range(len(band) // 4):
+        acc += group_pruning_cost(I_tile, [int(x) for x in band[4 * g:4 * g + 4]])
+    return acc
+
+
+def tile_perm_with_band(perm_t: np.ndarray, region_t: np.ndarray, band: np.ndarray) -> np.ndarray:
+    """A tile's working order with its 2:4 band rearranged: the working positions that hold
+    2:4-region channels (region by channel, ascending position) take the band's channels in
+    order; every other position keeps its channel.  Running the path with this order and the
+    same counts groups the band as given (regions depend on the channels' scores, not on
+    their positions, except for the position tie-break of equal scores)."""
+    perm_t = np.asarray(perm_t, dtype=np.int64)
+    pos = [j for j in range(perm_t.size) if region_t[perm_t[j]] == REGION_24]
+    out = perm_t.copy()
+    out[pos] = np.asarray(band, dtype=np.int64)
+    return out.astype(np.int32)
+
+
+def column_pruning_cost(I_rows: np.ndarray, n0: int) -> float:
+    """The importance that column-vector pruning removes from a tile with these rows: the
+    sum of its n0 smallest vector scores (a vector's score = its column sum over the rows,
+    fp64 in ascending row order), the n0 smallest summed in ascending order of score
+    (equal scores: lower channel first).  [P1] 关键设计 2 runs output-channel permutation
+    before the column-vector pruning; this is that step's cost."""
+    V = np.zeros(I_rows.shape[1])
+    for r in range(I_rows.shape[0]):
+        V = V + np.asarray(I_rows[r], dtype=np.float64)
+    order = np.lexsort((np.arange(V.size), V))
+    acc = 0.0
+    for j in order[:n0]:
+        acc += float(V[j])
+    return acc
+
+
+def gyro_output_round(I: np.ndarray, T: int, n0: np.ndarray, row_order: np.ndarray,
+                      tiles: np.ndarray, rows: np.ndarray, kmeans_iters: int = 8):
+    """One round of the output-channel gyro-permutation over a layer's tiles.
+
+    [P1] 关键设计 2: output channels are permuted before the column-vector pruning, by the
+    same sample / balanced K-means / Hungarian round.  [reading] ``row_order`` [M] lists the
+    output channels in their current order (tile t holds row_order[tT .. tT+T-1]); the
+    caller's draws pick G distinct tiles and k positions in each (``tiles`` [G],
+    ``rows`` [G, k]); those S = G k output channels leave their positions; their features
+    are their importance rows (fp64); the balanced K-means groups them into G clusters of k;
+    cost[c][i] is the column-pruning cost (``column_pruning_cost`` with the tile's n0) of
+    tile tiles[i] with its sampled positions, ascending, holding cluster c's channels in
+    ascending sample order.  The minimum-cost assignment places the clusters; kept only if
+    the sampled tiles' total cost does not rise.  Returns (row_order, (before, after)).
+    The layer then computes W[row_order] and produces Y[row_order]; the next layer's index
+    is translated by the inverse order (hinm_translate_index)."""
+    from scipy.optimize import linear_sum_assignment
+
+    order = np.array(row_order, dtype=np.int64).copy()
+    tiles = [int(t) for t in np.asarray(tiles).ravel()]
+    rows = np.asarray(rows, dtype=np.int64)
+    G, k = rows.shape
+    chans = [int(order[t * T + int(r)]) for t, rr in zip(tiles, rows) for r in rr]
+    F = np.asarray(I, dtype=np.float64)[chans]                       # S x K
+    clusters = balanced_kmeans(F, k, kmeans_iters)
+
+    def tile_rows_with(i, cl):
+        t = tiles[i]
+        ch = [int(x) for x in order[t * T:(t + 1) * T]]
+        for r, p in zip(sorted(int(x) for x in rows[i]), cl):
+            ch[r] = chans[p]
+        return ch
+
+    cost = np.zeros((G, G))
+    for c in range(G):
+        for i in range(G):
+            cost[c, i] = column_pruning_cost(I[tile_rows_with(i, clusters[c])], int(n0[tiles[i]]))
+    ra, ca = linear_sum_assignment(cost)
+    before = 0.0
+    for i in range(G):
+        t = tiles[i]
+        before += column_pruning_cost(I[order[t * T:(t + 1) * T]], int(n0[t]))
+    assign = {int(i): int(c) for c, i in zip(ra, ca)}
+    after = 0.0
+    for i in range(G):
+        after += cost[assign[i], i]
+    if after <= before:
+        new = order.copy()
+        for i in range(G):
+            t = tiles[i]
+            new[t * T:(t + 1) * T] = tile_rows_with(i, clusters[assign[i]])
+        return new, (before, after)
+    return order, (before, before)

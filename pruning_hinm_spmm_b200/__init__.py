@@ -75,6 +75,11 @@ _SIGS = {
     "hinm_search_workspace_size": (_i32, [_i32, _i32, _i32, _f64, _f64, _szp]),
     "hinm_boundary_search": (_i32, [_vp, _vp, _i32, _i32, _i32, _f64, _f64, _vp, _vp, _vp, _vp,
                                     _vp, _sz, _vp]),
+    "hinm_boundary_search_ex": (_i32, [_vp, _vp, _sz, _vp, _i32, _i32, _i32, _i32, _f64, _f64, _vp,
+                                       _vp, _vp, _vp, _vp, _sz, _vp]),
+    "hinm_mask_ex": (_i32, [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "hinm_compress_ex": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32,
+                                ctypes.POINTER(hinm_layout), _vp, _sz, _vp]),
     "hinm_mask_workspace_size": (_i32, [_i32, _i32, _i32, _szp]),
     "hinm_mask": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
     "hinm_compress_size": (_i32, [_vp, _i32, _i32, _i32, ctypes.POINTER(hinm_layout_sizes)]),
@@ -82,7 +87,13 @@ _SIGS = {
     "hinm_compress": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
                              ctypes.POINTER(hinm_layout), _vp, _sz, _vp]),
     "hinm_translate_index": (_i32, [ctypes.POINTER(hinm_layout), _vp, _vp]),
-    "hinm_gyro_refine_host": (_i32, [_vp, _i32, _i32, _vp, _i32, _vp, _i32, _i32, _vp]),
+    "hinm_gyro_input_round_host": (_i32, [_vp, _i32, _i32, _vp, _i32, _vp, _vp, _i32, _i32,
+                                           _i32, _vp]),
+    "hinm_gyro_band_cost_host": (_i32, [_vp, _i32, _i32, _vp, _i32, _vp]),
+    "hinm_gyro_cost_matrix": (_i32, [_vp, _i32, _i32, _i32, _vp, _i32, _vp, _vp, _vp, _i32, _i32,
+                                      _vp, _vp]),
+    "hinm_gyro_output_round_host": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _i32,
+                                            _i32, _vp]),
     "hinm_hard_concrete_forward": (_i32, [_vp, _vp, ctypes.c_longlong, ctypes.c_float, _vp, _vp,
                                           _vp, _vp]),
     "hinm_spmm": (_i32, [ctypes.POINTER(hinm_layout), _vp, _i32, _vp, _vp]),
@@ -133,6 +144,11 @@ def _size(fn, *args) -> int:
     out = ctypes.c_size_t(0)
     _check(fn(*args, ctypes.byref(out)), fn.__name__)
     return int(out.value)
+
+
+def _per_tile(perm) -> int:
+    """1 when perm holds one working order per tile ([M/T, K]), 0 for one shared order [K]."""
+    return 1 if perm is not None and perm.dim() == 2 else 0
 
 
 def _empty_bytes(nbytes: int, device):
@@ -230,7 +246,8 @@ def hinm_boundary_search(I, perm, T: int, t_s: float, alpha: float = 1.0 / 32.0,
     """Per-tile first-drop scan of v_s.  Returns (counts int32 [M/T,3], v_s fp64 [M/T], rank).
     ``retained_out`` (fp64 [M/T, n_cand]) optionally receives R(m) of every candidate;
     ``stats`` (from hinm_importance_stats for this I and T) spares the search its pass over
-    I for V."""
+    I for V.  ``perm``: int32 [K] (every tile) or [M/T, K] (one working order per tile), or
+    None (identity)."""
     torch = _torch()
     M, K = I.shape
     nt = M // T
@@ -243,17 +260,11 @@ def hinm_boundary_search(I, perm, T: int, t_s: float, alpha: float = 1.0 / 32.0,
         rank_out = torch.empty((nt, K), dtype=torch.int32, device=dev)
     if workspace is None:
         workspace = _empty_bytes(hinm_search_workspace_size(M, K, T, t_s, alpha), dev)
-    if stats is not None:
-        _check(_lib.hinm_boundary_search_stats(_ptr(I), _ptr(stats), stats.numel(), _ptr(perm), M,
-                                               K, T, t_s, alpha, _ptr(counts_out), _ptr(vs_out),
-                                               _ptr(rank_out), _ptr(retained_out),
-                                               _ptr(workspace), workspace.numel(),
-                                               _stream(stream)), "hinm_boundary_search_stats")
-    else:
-        _check(_lib.hinm_boundary_search(_ptr(I), _ptr(perm), M, K, T, t_s, alpha,
-                                         _ptr(counts_out), _ptr(vs_out), _ptr(rank_out),
-                                         _ptr(retained_out), _ptr(workspace), workspace.numel(),
-                                         _stream(stream)), "hinm_boundary_search")
+    _check(_lib.hinm_boundary_search_ex(_ptr(I), _ptr(stats), 0 if stats is None else stats.numel(),
+                                        _ptr(perm), _per_tile(perm), M, K, T, t_s, alpha,
+                                        _ptr(counts_out), _ptr(vs_out), _ptr(rank_out),
+                                        _ptr(retained_out), _ptr(workspace), workspace.numel(),
+                                        _stream(stream)), "hinm_boundary_search_ex")
     return counts_out, vs_out, rank_out
 
 
@@ -275,9 +286,9 @@ def hinm_mask(I, perm, counts, T: int, rank=None, bitmask_out=None, region_out=N
         region_out = torch.empty((M // T, K), dtype=torch.int8, device=dev)
     if workspace is None:
         workspace = _empty_bytes(hinm_mask_workspace_size(M, K, T), dev)
-    _check(_lib.hinm_mask(_ptr(I), _ptr(perm), _ptr(counts), _ptr(rank), M, K, T,
-                          _ptr(bitmask_out), _ptr(region_out), _ptr(workspace), workspace.numel(),
-                          _stream(stream)), "hinm_mask")
+    _check(_lib.hinm_mask_ex(_ptr(I), _ptr(perm), _per_tile(perm), _ptr(counts), _ptr(rank), M,
+                             K, T, _ptr(bitmask_out), _ptr(region_out), _ptr(workspace),
+                             workspace.numel(), _stream(stream)), "hinm_mask_ex")
     return bitmask_out, region_out
 
 
@@ -345,9 +356,10 @@ def hinm_compress(W, bitmask, region, perm, counts, T: int, layout: Optional[Hin
     if workspace is None:
         workspace = _empty_bytes(hinm_compress_workspace_size(M, K, T), W.device)
     c = layout.as_c()
-    _check(_lib.hinm_compress(_ptr(W), _ptr(bitmask), _ptr(region), _ptr(perm), _ptr(counts),
-                              M, K, T, ctypes.byref(c), _ptr(workspace), workspace.numel(),
-                              _stream(stream)), "hinm_compress")
+    _check(_lib.hinm_compress_ex(_ptr(W), _ptr(bitmask), _ptr(region), _ptr(perm),
+                                 _per_tile(perm), _ptr(counts), M, K, T, ctypes.byref(c),
+                                 _ptr(workspace), workspace.numel(), _stream(stream)),
+           "hinm_compress_ex")
     return layout
 
 
@@ -416,21 +428,92 @@ def hinm_hard_concrete_forward(log_alpha, eps, tau: float, z_out=None, hard_out=
     return z_out, hard_out, sums_out
 
 
-def hinm_gyro_refine_host(I_tile, band, schedule):
-    """Host refinement of a tile's 2:4 grouping (numpy in, numpy out): I_tile fp32 [T, K],
-    band int32 [n] (working order of the 2:4 channels), schedule int32 [iters, S, 2] of
-    (group, slot).  Returns (refined band, retained importance before / after each iteration)."""
+def _host_i32(a):
+    import numpy as np
+    return np.ascontiguousarray(a, dtype=np.int32)
+
+
+def hinm_gyro_input_round_host(I_tile, band, groups, slots, kmeans_iters: int = 8):
+    """One in-tile input-channel gyro round on the host (numpy in, numpy out): I_tile fp32
+    [T, K], band int32 [n] (the tile's 2:4 channels in working order), groups int32 [G],
+    slots int32 [G, k].  Returns (refined band, (cost before, cost after))."""
     import numpy as np
     I_tile = np.ascontiguousarray(I_tile, dtype=np.float32)
-    band = np.ascontiguousarray(band, dtype=np.int32).copy()
-    schedule = np.ascontiguousarray(schedule, dtype=np.int32)
+    band = _host_i32(band).copy()
+    groups = _host_i32(groups).ravel()
+    slots = _host_i32(slots)
     T, K = I_tile.shape
-    iters, S = schedule.shape[0], schedule.shape[1]
-    retained = np.zeros(iters + 1, dtype=np.float64)
-    _check(_lib.hinm_gyro_refine_host(I_tile.ctypes.data, T, K, band.ctypes.data, band.size,
-                                      schedule.ctypes.data, iters, S, retained.ctypes.data),
-           "hinm_gyro_refine_host")
-    return band, retained
+    G, k = slots.shape
+    cost = np.zeros(2, dtype=np.float64)
+    _check(_lib.hinm_gyro_input_round_host(I_tile.ctypes.data, T, K, band.ctypes.data, band.size,
+                                           groups.ctypes.data, slots.ctypes.data, G, k,
+                                           int(kmeans_iters), cost.ctypes.data),
+           "hinm_gyro_input_round_host")
+    return band, (float(cost[0]), float(cost[1]))
+
+
+def hinm_gyro_band_cost_host(I_tile, band) -> float:
+    import numpy as np
+    I_tile = np.ascontiguousarray(I_tile, dtype=np.float32)
+    band = _host_i32(band)
+    out = ctypes.c_double(0.0)
+    _check(_lib.hinm_gyro_band_cost_host(I_tile.ctypes.data, I_tile.shape[0], I_tile.shape[1],
+                                         band.ctypes.data, band.size, ctypes.byref(out)),
+           "hinm_gyro_band_cost_host")
+    return float(out.value)
+
+
+def hinm_gyro_cost_matrix(I, T: int, bands, groups, slots, clusters, cost_out=None, stream=None):
+    """The input rounds' cost matrices of every tile on the GPU: I fp32 [M, K], bands int32
+    [M/T, band_len], groups [M/T, G], slots / clusters [M/T, G, k] (device tensors).
+    Returns cost fp64 [M/T, G, G]."""
+    torch = _torch()
+    M, K = I.shape
+    G, k = slots.shape[1], slots.shape[2]
+    if cost_out is None:
+        cost_out = torch.empty((M // T, G, G), dtype=torch.float64, device=I.device)
+    _check(_lib.hinm_gyro_cost_matrix(_ptr(I), M, K, T, _ptr(bands), bands.shape[1],
+                                      _ptr(groups), _ptr(slots), _ptr(clusters), G, k,
+                                      _ptr(cost_out), _stream(stream)), "hinm_gyro_cost_matrix")
+    return cost_out
+
+
+def tile_orders_with_bands(perm, region, bands):
+    """Per-tile working orders int32 [M/T, K] for the hot path's perm after the in-tile gyro
+    rounds: in tile t the working positions that hold 2:4-region channels (region by channel,
+    ascending position) take the refined band bands[t] in order; the other positions keep
+    their channels.  perm: int32 [K] or [M/T, K]; region: int8 [M/T, K]; bands: a list of
+    int32 arrays (host numpy)."""
+    import numpy as np
+    region = np.asarray(region)
+    nt, K = region.shape
+    perm = np.asarray(perm, dtype=np.int32)
+    out = np.empty((nt, K), dtype=np.int32)
+    for t in range(nt):
+        pt = perm if perm.ndim == 1 else perm[t]
+        pos = np.nonzero(region[t][pt] == REGION_24)[0]
+        out[t] = pt
+        out[t, pos] = np.asarray(bands[t], dtype=np.int32)
+    return out
+
+
+def hinm_gyro_output_round_host(I, T: int, n0, row_order, tiles, rows, kmeans_iters: int = 8):
+    """One output-channel gyro round on the host: I fp32 [M, K], n0 int32 [M/T], row_order
+    int32 [M], tiles int32 [G], rows int32 [G, k].  Returns (row order, (before, after))."""
+    import numpy as np
+    I = np.ascontiguousarray(I, dtype=np.float32)
+    M, K = I.shape
+    n0 = _host_i32(n0)
+    order = _host_i32(row_order).copy()
+    tiles = _host_i32(tiles).ravel()
+    rows = _host_i32(rows)
+    G, k = rows.shape
+    cost = np.zeros(2, dtype=np.float64)
+    _check(_lib.hinm_gyro_output_round_host(I.ctypes.data, M, K, T, n0.ctypes.data,
+                                            order.ctypes.data, tiles.ctypes.data, rows.ctypes.data,
+                                            G, k, int(kmeans_iters), cost.ctypes.data),
+           "hinm_gyro_output_round_host")
+    return order, (float(cost[0]), float(cost[1]))
 
 
 def hinm_device_status(stream=None) -> int:

@@ -354,7 +354,8 @@ namespace {
 
 // hinm_boundary_search(_stats): stats (with its size) or nullptr
 hinm_status search_impl(const float* I, const void* stats, size_t stats_bytes,
-                        const int32_t* perm, int M, int K, int T, double t_s, double alpha,
+                        const int32_t* perm, int perm_per_tile, int M, int K, int T, double t_s,
+                        double alpha,
                         int32_t* counts_out, double* vs_out, int32_t* rank_out,
                         double* retained_out, void* workspace, size_t workspace_bytes,
                         void* stream) {
@@ -382,7 +383,10 @@ hinm_status search_impl(const float* I, const void* stats, size_t stats_bytes,
   if (!workspace || workspace_bytes < need)
     return fail(HINM_ERR_WORKSPACE, "workspace %zu bytes, need %zu", workspace_bytes, need);
   REQUIRE_PTR(workspace);
-  cudaError_t e = hinm::launch_boundary_search(I, stats, perm, M, K, T, t_s, alpha, c, n,
+  if (perm_per_tile != 0 && perm_per_tile != 1)
+    return fail(HINM_ERR_INVALID_ARG, "perm_per_tile=%d must be 0 or 1", perm_per_tile);
+  cudaError_t e = hinm::launch_boundary_search(I, stats, perm, perm_per_tile ? (long long)K : 0ll,
+                                               M, K, T, t_s, alpha, c, n,
                                                counts_out, vs_out, rank_out, retained_out,
                                                workspace, hinm::device_status_ptr(),
                                                static_cast<cudaStream_t>(stream));
@@ -396,7 +400,7 @@ hinm_status hinm_boundary_search(const float* I, const int32_t* perm, int M, int
                                  double t_s, double alpha, int32_t* counts_out, double* vs_out,
                                  int32_t* rank_out, double* retained_out, void* workspace,
                                  size_t workspace_bytes, void* stream) {
-  return search_impl(I, nullptr, 0, perm, M, K, T, t_s, alpha, counts_out, vs_out, rank_out,
+  return search_impl(I, nullptr, 0, perm, 0, M, K, T, t_s, alpha, counts_out, vs_out, rank_out,
                      retained_out, workspace, workspace_bytes, stream);
 }
 
@@ -406,8 +410,18 @@ hinm_status hinm_boundary_search_stats(const float* I, const void* stats, size_t
                                        int32_t* rank_out, double* retained_out,
                                        void* workspace, size_t workspace_bytes, void* stream) {
   REQUIRE_PTR(stats);
-  return search_impl(I, stats, stats_bytes, perm, M, K, T, t_s, alpha, counts_out, vs_out,
+  return search_impl(I, stats, stats_bytes, perm, 0, M, K, T, t_s, alpha, counts_out, vs_out,
                      rank_out, retained_out, workspace, workspace_bytes, stream);
+}
+
+hinm_status hinm_boundary_search_ex(const float* I, const void* stats, size_t stats_bytes,
+                                    const int32_t* perm, int perm_per_tile, int M, int K, int T,
+                                    double t_s, double alpha, int32_t* counts_out, double* vs_out,
+                                    int32_t* rank_out, double* retained_out, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  return search_impl(I, stats, stats ? stats_bytes : 0, perm, perm_per_tile, M, K, T, t_s, alpha,
+                     counts_out, vs_out, rank_out, retained_out, workspace, workspace_bytes,
+                     stream);
 }
 
 hinm_status hinm_mask_workspace_size(int M, int K, int T, size_t* bytes_host) {
@@ -422,7 +436,17 @@ hinm_status hinm_mask(const float* I, const int32_t* perm, const int32_t* counts
                       const int32_t* rank, int M, int K, int T, uint32_t* bitmask_out,
                       int8_t* region_out, void* workspace, size_t workspace_bytes,
                       void* stream) {
+  return hinm_mask_ex(I, perm, 0, counts, rank, M, K, T, bitmask_out, region_out, workspace,
+                      workspace_bytes, stream);
+}
+
+hinm_status hinm_mask_ex(const float* I, const int32_t* perm, int perm_per_tile,
+                         const int32_t* counts, const int32_t* rank, int M, int K, int T,
+                         uint32_t* bitmask_out, int8_t* region_out, void* workspace,
+                         size_t workspace_bytes, void* stream) {
   REQUIRE_PTR(I);
+  if (perm_per_tile != 0 && perm_per_tile != 1)
+    return fail(HINM_ERR_INVALID_ARG, "perm_per_tile=%d must be 0 or 1", perm_per_tile);
   REQUIRE_ALIGNED_OR_NULL(perm);
   REQUIRE_PTR(counts);
   REQUIRE_ALIGNED_OR_NULL(rank);
@@ -434,7 +458,8 @@ hinm_status hinm_mask(const float* I, const int32_t* perm, const int32_t* counts
   if (!workspace || workspace_bytes < need)
     return fail(HINM_ERR_WORKSPACE, "workspace %zu bytes, need %zu", workspace_bytes, need);
   REQUIRE_PTR(workspace);
-  cudaError_t e = hinm::launch_mask(I, perm, counts, rank, M, K, T, bitmask_out, region_out,
+  cudaError_t e = hinm::launch_mask(I, perm, perm_per_tile ? (long long)K : 0ll, counts, rank, M,
+                                    K, T, bitmask_out, region_out,
                                     workspace, hinm::device_status_ptr(),
                                     static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "hinm_mask launch");
@@ -510,7 +535,17 @@ hinm_status hinm_compress(const void* W, const uint32_t* bitmask, const int8_t* 
                           const int32_t* perm, const int32_t* counts, int M, int K, int T,
                           const hinm_layout* layout, void* workspace, size_t workspace_bytes,
                           void* stream) {
+  return hinm_compress_ex(W, bitmask, region, perm, 0, counts, M, K, T, layout, workspace,
+                          workspace_bytes, stream);
+}
+
+hinm_status hinm_compress_ex(const void* W, const uint32_t* bitmask, const int8_t* region,
+                             const int32_t* perm, int perm_per_tile, const int32_t* counts,
+                             int M, int K, int T, const hinm_layout* layout, void* workspace,
+                             size_t workspace_bytes, void* stream) {
   REQUIRE_PTR(W);
+  if (perm_per_tile != 0 && perm_per_tile != 1)
+    return fail(HINM_ERR_INVALID_ARG, "perm_per_tile=%d must be 0 or 1", perm_per_tile);
   REQUIRE_PTR(bitmask);
   REQUIRE_PTR(region);
   REQUIRE_ALIGNED_OR_NULL(perm);
@@ -527,41 +562,140 @@ hinm_status hinm_compress(const void* W, const uint32_t* bitmask, const int8_t* 
     return fail(HINM_ERR_WORKSPACE, "workspace %zu bytes, need %zu", workspace_bytes, need);
   REQUIRE_PTR(workspace);
   cudaError_t e = hinm::launch_compress(static_cast<const uint16_t*>(W), bitmask, region, perm,
-                                        counts, M, K, T, *layout, workspace,
+                                        perm_per_tile ? (long long)K : 0ll, counts, M, K, T, *layout, workspace,
                                         hinm::device_status_ptr(),
                                         static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "hinm_compress launch");
   return ok();
 }
 
-hinm_status hinm_gyro_refine_host(const float* I_tile, int T, int K, int32_t* band, int n,
-                                  const int32_t* schedule, int iters, int S,
-                                  double* retained_out) {
-  if (!I_tile || !band) return fail(HINM_ERR_INVALID_ARG, "I_tile and band must not be NULL");
-  if (T <= 0 || K < 4 || n <= 0 || n % 4 != 0 || n > K)
+namespace {
+// The band of a gyro input round: n % 4 == 0, 4 <= n <= K, distinct entries in [0, K).
+hinm_status check_band(int T, int K, const int32_t* band, int n) {
+  if (T <= 0 || K < 4 || n < 4 || n % 4 != 0 || n > K)
     return fail(HINM_ERR_SHAPE, "T=%d, K=%d, n=%d: need T > 0, n a positive multiple of 4, n <= K",
                 T, K, n);
-  if (iters < 0 || S < 1 || S > n / 4 || (iters > 0 && !schedule))
-    return fail(HINM_ERR_INVALID_ARG, "iters=%d, S=%d: need iters >= 0, 1 <= S <= n/4", iters, S);
-  for (int i = 0; i < n; ++i)
-    if (band[i] < 0 || band[i] >= K) return fail(HINM_ERR_INVALID_ARG, "band[%d]=%d outside [0, K)", i, band[i]);
-  // the assignment's potentials need finite costs: every importance the band reads is finite
+  std::vector<char> seen(K, 0);
+  for (int i = 0; i < n; ++i) {
+    if (band[i] < 0 || band[i] >= K)
+      return fail(HINM_ERR_INVALID_ARG, "band[%d]=%d outside [0, K)", i, band[i]);
+    if (seen[band[i]]) return fail(HINM_ERR_INVALID_ARG, "band[%d]=%d repeated", i, band[i]);
+    seen[band[i]] = 1;
+  }
+  return HINM_OK;
+}
+// G distinct items in [0, count) and, for each, k distinct sub-items in [0, sub).
+hinm_status check_samples(const int32_t* items, int count, const int32_t* sub, int subcount,
+                          int G, int k, const char* what) {
+  if (G < 1 || G > count || k < 1 || k > subcount)
+    return fail(HINM_ERR_INVALID_ARG, "%s: G=%d, k=%d: need 1 <= G <= %d, 1 <= k <= %d", what, G,
+                k, count, subcount);
+  std::vector<char> seen(count, 0);
+  for (int i = 0; i < G; ++i) {
+    if (items[i] < 0 || items[i] >= count || seen[items[i]])
+      return fail(HINM_ERR_INVALID_ARG, "%s[%d]=%d: need distinct values in [0, %d)", what, i,
+                  items[i], count);
+    seen[items[i]] = 1;
+    for (int j = 0; j < k; ++j) {
+      const int v = sub[(size_t)i * k + j];
+      if (v < 0 || v >= subcount)
+        return fail(HINM_ERR_INVALID_ARG, "%s sample [%d][%d]=%d outside [0, %d)", what, i, j, v,
+                    subcount);
+      for (int q = 0; q < j; ++q)
+        if (sub[(size_t)i * k + q] == v)
+          return fail(HINM_ERR_INVALID_ARG, "%s sample [%d] repeats %d", what, i, v);
+    }
+  }
+  return HINM_OK;
+}
+}  // namespace
+
+hinm_status hinm_gyro_input_round_host(const float* I_tile, int T, int K, int32_t* band, int n,
+                                       const int32_t* groups, const int32_t* slots, int G, int k,
+                                       int kmeans_iters, double* cost_out) {
+  if (!I_tile || !band || !groups || !slots)
+    return fail(HINM_ERR_INVALID_ARG, "I_tile, band, groups and slots must not be NULL");
+  hinm_status st = check_band(T, K, band, n);
+  if (st != HINM_OK) return st;
+  st = check_samples(groups, n / 4, slots, 4, G, k, "groups");
+  if (st != HINM_OK) return st;
+  if (kmeans_iters < 0) return fail(HINM_ERR_INVALID_ARG, "kmeans_iters=%d < 0", kmeans_iters);
+  // the costs and the K-means need finite values: every importance the round reads
   for (int r = 0; r < T; ++r)
     for (int i = 0; i < n; ++i)
       if (!std::isfinite(I_tile[(size_t)r * K + band[i]]))
         return fail(HINM_ERR_INVALID_ARG, "I_tile[%d][%d] is not finite", r, band[i]);
-  std::vector<char> seen(n / 4);
-  for (int it = 0; it < iters; ++it) {
-    std::fill(seen.begin(), seen.end(), 0);
-    for (int a = 0; a < S; ++a) {
-      const int g = schedule[((size_t)it * S + a) * 2], k = schedule[((size_t)it * S + a) * 2 + 1];
-      if (g < 0 || g >= n / 4 || k < 0 || k > 3 || seen[g])
-        return fail(HINM_ERR_INVALID_ARG, "schedule[%d][%d] = (%d, %d): need distinct groups in "
-                    "[0, n/4) and slots in [0, 4)", it, a, g, k);
-      seen[g] = 1;
-    }
+  if (!hinm::gyro_input_round(I_tile, T, K, band, groups, slots, G, k, kmeans_iters, cost_out))
+    return fail(HINM_ERR_INVALID_ARG, "the assignment could not be formed");
+  return ok();
+}
+
+hinm_status hinm_gyro_band_cost_host(const float* I_tile, int T, int K, const int32_t* band,
+                                     int n, double* cost_host) {
+  if (!I_tile || !band || !cost_host)
+    return fail(HINM_ERR_INVALID_ARG, "I_tile, band and cost_host must not be NULL");
+  hinm_status st = check_band(T, K, band, n);
+  if (st != HINM_OK) return st;
+  *cost_host = hinm::gyro_band_cost(I_tile, T, K, band, n);
+  return ok();
+}
+
+hinm_status hinm_gyro_cost_matrix(const float* I, int M, int K, int T, const int32_t* bands,
+                                  int band_len, const int32_t* groups, const int32_t* slots,
+                                  const int32_t* clusters, int G, int k, double* cost_out,
+                                  void* stream) {
+  REQUIRE_PTR(I);
+  REQUIRE_PTR(bands);
+  REQUIRE_PTR(groups);
+  REQUIRE_PTR(slots);
+  REQUIRE_PTR(clusters);
+  REQUIRE_PTR(cost_out);
+  if (T <= 0 || M <= 0 || M % T != 0 || K < 4)
+    return fail(HINM_ERR_SHAPE, "M=%d, K=%d, T=%d: need M a positive multiple of T, K >= 4", M,
+                K, T);
+  if (band_len < 4 || band_len % 4 != 0 || band_len > K)
+    return fail(HINM_ERR_SHAPE, "band_len=%d: need a multiple of 4 in [4, K]", band_len);
+  if (k < 1 || k > 4 || G < 1 || G > band_len / 4)
+    return fail(HINM_ERR_INVALID_ARG, "G=%d, k=%d: need 1 <= k <= 4, 1 <= G <= band_len/4", G, k);
+  cudaError_t e = hinm::launch_gyro_cost(I, K, T, M / T, bands, band_len, groups, slots, clusters,
+                                         G, k, cost_out, hinm::device_status_ptr(),
+                                         static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "hinm_gyro_cost_matrix launch");
+  return ok();
+}
+
+hinm_status hinm_gyro_output_round_host(const float* I, int M, int K, int T, const int32_t* n0,
+                                        int32_t* row_order, const int32_t* tiles,
+                                        const int32_t* rows, int G, int k, int kmeans_iters,
+                                        double* cost_out) {
+  if (!I || !n0 || !row_order || !tiles || !rows)
+    return fail(HINM_ERR_INVALID_ARG, "I, n0, row_order, tiles and rows must not be NULL");
+  if (T <= 0 || M <= 0 || M % T != 0 || K <= 0)
+    return fail(HINM_ERR_SHAPE, "M=%d, K=%d, T=%d: need M a positive multiple of T", M, K, T);
+  const int nt = M / T;
+  std::vector<char> seen(M, 0);
+  for (int i = 0; i < M; ++i) {
+    if (row_order[i] < 0 || row_order[i] >= M || seen[row_order[i]])
+      return fail(HINM_ERR_INVALID_ARG, "row_order[%d]=%d: need a permutation of 0..M-1", i,
+                  row_order[i]);
+    seen[row_order[i]] = 1;
   }
-  hinm::gyro_refine(I_tile, T, K, band, n, schedule, iters, S, retained_out);
+  for (int t = 0; t < nt; ++t)
+    if (n0[t] < 0 || n0[t] > K) return fail(HINM_ERR_INVALID_ARG, "n0[%d]=%d outside [0, K]", t, n0[t]);
+  hinm_status st = check_samples(tiles, nt, rows, T, G, k, "tiles");
+  if (st != HINM_OK) return st;
+  if (kmeans_iters < 0) return fail(HINM_ERR_INVALID_ARG, "kmeans_iters=%d < 0", kmeans_iters);
+  for (int i = 0; i < G; ++i)
+    for (int r = 0; r < T; ++r) {
+      const float* row = I + (size_t)row_order[(size_t)tiles[i] * T + r] * K;
+      for (int c = 0; c < K; ++c)
+        if (!std::isfinite(row[c]))
+          return fail(HINM_ERR_INVALID_ARG, "I[%d][%d] is not finite",
+                      row_order[(size_t)tiles[i] * T + r], c);
+    }
+  if (!hinm::gyro_output_round(I, M, K, T, n0, row_order, tiles, rows, G, k, kmeans_iters,
+                               cost_out))
+    return fail(HINM_ERR_INVALID_ARG, "the assignment could not be formed");
   return ok();
 }
 

@@ -114,11 +114,13 @@ __global__ void __launch_bounds__(kTileInfoThreads) tile_info_kernel(
 
 // lists[t][0 .. n_dense) = dense working positions, lists[t][n_dense .. ) = 2:4 ones.
 __global__ void __launch_bounds__(1024) lists_kernel(const int8_t* __restrict__ region,
-                                                     const int32_t* __restrict__ perm,
+                                                     const int32_t* __restrict__ perm_all,
+                                                     long long perm_stride,
                                                      const int32_t* __restrict__ counts, int K,
                                                      int32_t* __restrict__ lists, int* status) {
   __shared__ int warp_tot[2][32];
   const int t = blockIdx.x;
+  const int32_t* perm = perm_all ? perm_all + t * perm_stride : perm_all;  // this tile's order
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const int8_t* reg = region + (size_t)t * K;
   const int per = (K + blockDim.x - 1) / blockDim.x;
@@ -225,7 +227,8 @@ __device__ __forceinline__ void select_pair(const uint32_t (&w)[4], uint32_t kep
 
 __global__ void __launch_bounds__(256) pack_kernel(const uint16_t* __restrict__ W,
                                                    const uint32_t* __restrict__ bitmask,
-                                                   const int32_t* __restrict__ perm,
+                                                   const int32_t* __restrict__ perm_all,
+                                                   long long perm_stride,
                                                    const int32_t* __restrict__ counts,
                                                    const int32_t* __restrict__ lists, int K, int T,
                                                    hinm_layout L, int* status) {
@@ -233,6 +236,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint16_t* __restrict__ 
   __shared__ int chan[kSparseBK];  // input channel of every vector of the block, -1 = padding
   const int t = blockIdx.y;
   const int b = blockIdx.x;
+  const int32_t* perm = perm_all ? perm_all + t * perm_stride : perm_all;  // this tile's order
   const int nd = L.tile_info[4 * t + 0], ns = L.tile_info[4 * t + 1];
   const int d0 = L.tile_info[4 * t + 2], s0 = L.tile_info[4 * t + 3];
   if (b >= nd + ns) return;
@@ -429,7 +433,8 @@ cudaError_t launch_translate_index(const hinm_layout& L, const int32_t* row_of_c
 }
 
 cudaError_t launch_compress(const uint16_t* W, const uint32_t* bitmask, const int8_t* region,
-                            const int32_t* perm, const int32_t* counts, int M, int K, int T,
+                            const int32_t* perm, long long perm_stride, const int32_t* counts,
+                            int M, int K, int T,
                             const hinm_layout& L, void* ws, int* status, cudaStream_t s) {
   const int nt = M / T;
   int32_t* lists = static_cast<int32_t*>(ws);
@@ -438,12 +443,12 @@ cudaError_t launch_compress(const uint16_t* W, const uint32_t* bitmask, const in
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // lists are read only at positions below the counts, so no clearing is needed
-  lists_kernel<<<nt, 1024, 0, s>>>(region, perm, counts, K, lists, status);
+  lists_kernel<<<nt, 1024, 0, s>>>(region, perm, perm_stride, counts, K, lists, status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int max_blocks = (K + kDenseBK - 1) / kDenseBK + (K + kSparseBK - 1) / kSparseBK;
   dim3 g(max_blocks, nt);
-  pack_kernel<<<g, 256, 0, s>>>(W, bitmask, perm, counts, lists, K, T, L, status);
+  pack_kernel<<<g, 256, 0, s>>>(W, bitmask, perm, perm_stride, counts, lists, K, T, L, status);
   return cudaGetLastError();
 }
 

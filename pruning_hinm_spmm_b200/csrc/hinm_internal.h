@@ -82,31 +82,42 @@ constexpr int kNoAllocMaxK = 16384;
 cudaError_t noalloc_energy_scratch(float** out);
 
 size_t search_workspace_bytes(int M, int K, int T, int ncand);
+// perm: the working order, [K] shared by every tile (perm_stride 0) or [M/T][K] one per tile
+// (perm_stride K), or nullptr (identity).
 // stats: from launch_importance_stats for this I and T, or nullptr (computed here from I)
 cudaError_t launch_boundary_search(const float* I, const void* stats, const int32_t* perm,
-                                   int M, int K, int T, double t_s, double alpha,
+                                   long long perm_stride, int M, int K, int T, double t_s, double alpha,
                                    const Candidate* cands, int ncand, int32_t* counts_out,
                                    double* vs_out, int32_t* rank_out, double* retained_out,
                                    void* ws, int* status, cudaStream_t s);
 
 size_t mask_workspace_bytes(int M, int K, int T);
-cudaError_t launch_mask(const float* I, const int32_t* perm, const int32_t* counts,
+cudaError_t launch_mask(const float* I, const int32_t* perm, long long perm_stride,
+                        const int32_t* counts,
                         const int32_t* rank, int M, int K, int T, uint32_t* bitmask,
                         int8_t* region, void* ws, int* status, cudaStream_t s);
 
 size_t compress_workspace_bytes(int M, int K, int T);
 cudaError_t launch_compress(const uint16_t* W, const uint32_t* bitmask, const int8_t* region,
-                            const int32_t* perm, const int32_t* counts, int M, int K, int T,
+                            const int32_t* perm, long long perm_stride, const int32_t* counts, int M, int K, int T,
                             const hinm_layout& L, void* ws, int* status, cudaStream_t s);
 
 cudaError_t launch_wait_timeout_selftest(unsigned long long limit_ns, int* status,
                                          cudaStream_t s);
 
 // tile_pairs: the caller's hint that tiles select the same X rows (HINM_SPMM_TILE_PAIRS)
-// Host: gyro-style refinement of a tile's 2:4 grouping (arguments checked by the caller).
-double gyro_band_retained(const float* I, int T, int K, const int32_t* band, int n);
-void gyro_refine(const float* I, int T, int K, int32_t* band, int n, const int32_t* schedule,
-                 int iters, int S, double* retained);
+// Gyro-permutation rounds (host; arguments checked by the caller) and the device cost
+// matrices of the input rounds.
+double gyro_band_cost(const float* I, int T, int K, const int32_t* band, int n);
+bool gyro_input_round(const float* I, int T, int K, int32_t* band, const int32_t* groups,
+                      const int32_t* slots, int G, int k, int kmeans_iters, double* cost_out);
+bool gyro_output_round(const float* I, int M, int K, int T, const int32_t* n0, int32_t* order,
+                       const int32_t* tiles, const int32_t* rows, int G, int k, int kmeans_iters,
+                       double* cost_out);
+cudaError_t launch_gyro_cost(const float* I, int K, int T, int nt, const int32_t* bands, int nb,
+                             const int32_t* groups, const int32_t* slots,
+                             const int32_t* clusters, int G, int k, double* cost, int* status,
+                             cudaStream_t s);
 
 cudaError_t launch_hard_concrete(const float* log_alpha, const float* eps, long long n, float tau,
                                  float* z, uint8_t* hard, double* sums, cudaStream_t s);
@@ -131,7 +142,8 @@ cudaError_t launch_spmm(const hinm_layout& L, const uint16_t* X, int N, const Sp
 // tile_pmax (int [M/T]) receives each tile's largest fp32 exponent; scratch holds
 // rank_scratch_bytes() bytes.
 size_t rank_scratch_bytes(int M, int K, int T);
-cudaError_t launch_vector_rank(const float* I, const int32_t* perm, int M, int K, int T,
+cudaError_t launch_vector_rank(const float* I, const int32_t* perm, long long perm_stride, int M,
+                               int K, int T,
                                double* V, int32_t* rank, int* tile_pmax, void* scratch,
                                cudaStream_t s);
 

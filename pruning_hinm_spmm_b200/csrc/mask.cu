@@ -46,16 +46,18 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* t
 }
 
 __global__ void __launch_bounds__(1024) classify_kernel(const int32_t* __restrict__ rank,
-                                                        const int32_t* __restrict__ perm,
+                                                        const int32_t* __restrict__ perm_all,
+                                                        long long perm_stride,
                                                         const int32_t* __restrict__ counts, int K,
                                                         int8_t* __restrict__ region,
                                                         int32_t* __restrict__ member,
                                                         int* status) {
   __shared__ int warp_tot[32];
   __shared__ int total;
-  __shared__ uint32_t seen[kMaxK / 32];  // tile 0: which channels perm has named
+  __shared__ uint32_t seen[kMaxK / 32];  // which channels this tile's order has named
   const int t = blockIdx.x;
-  if (t == 0 && perm) {
+  const int32_t* perm = perm_all ? perm_all + t * perm_stride : perm_all;  // this tile's order
+  if ((t == 0 || perm_stride != 0) && perm) {
     // the permutation must name every channel 0..K-1 once: a repeated or out-of-range
     // entry is reported as HINM_ERR_INVALID_ARG (perm_at keeps every access in range)
     for (int w = threadIdx.x; w < kMaxK / 32; w += blockDim.x) seen[w] = 0u;
@@ -235,7 +237,8 @@ size_t mask_workspace_bytes(int M, int K, int T) {
   return (c.off + 255) & ~size_t(255);
 }
 
-cudaError_t launch_mask(const float* I, const int32_t* perm, const int32_t* counts,
+cudaError_t launch_mask(const float* I, const int32_t* perm, long long perm_stride,
+                        const int32_t* counts,
                         const int32_t* rank, int M, int K, int T, uint32_t* bitmask,
                         int8_t* region, void* ws, int* status, cudaStream_t s) {
   const int nt = M / T;
@@ -247,11 +250,12 @@ cudaError_t launch_mask(const float* I, const int32_t* perm, const int32_t* coun
   char* rank_scratch = cv.take<char>(rank_scratch_bytes(M, K, T));
   cudaError_t e;
   if (!rank) {
-    e = launch_vector_rank(I, perm, M, K, T, V, rank_ws, pmax, rank_scratch, s);
+    e = launch_vector_rank(I, perm, perm_stride, M, K, T, V, rank_ws, pmax, rank_scratch, s);
     if (e != cudaSuccess) return e;
     rank = rank_ws;
   }
-  classify_kernel<<<nt, 1024, 0, s>>>(rank, perm, counts, K, region, member, status);
+  classify_kernel<<<nt, 1024, 0, s>>>(rank, perm, perm_stride, counts, K, region, member,
+                                      status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int RB = mask_rows(K);

@@ -236,7 +236,8 @@ __device__ __forceinline__ bool pair_less(unsigned long long ka, unsigned ia,
 // zero64 / zero32 (nullptr allowed): buffers of a later kernel of the search, cleared here by
 // the whole grid (grid-stride) instead of by separate memsets.
 __global__ void __launch_bounds__(kRankChunk) chunk_sort_kernel(
-    const double* __restrict__ Vc, const int32_t* __restrict__ perm, int K, int Kp,
+    const double* __restrict__ Vc, const int32_t* __restrict__ perm, long long perm_stride,
+    int K, int Kp,
     unsigned long long* __restrict__ skey, unsigned short* __restrict__ sidx,
     unsigned long long* __restrict__ zero64, size_t n64, int* __restrict__ zero32, size_t n32) {
   __shared__ unsigned long long key_s[kRankChunk];
@@ -256,7 +257,8 @@ __global__ void __launch_bounds__(kRankChunk) chunk_sort_kernel(
   unsigned idx = 0xFFFFu;
   if (j < K) {
     key = ~static_cast<unsigned long long>(
-        __double_as_longlong(__ldg(Vc + (size_t)t * K + ptx::perm_at(perm, j, K))));
+        __double_as_longlong(__ldg(Vc + (size_t)t * K +
+                                   ptx::perm_at(perm ? perm + t * perm_stride : perm, j, K))));
     idx = (unsigned)j;
   }
   for (int k = 2; k <= kRankChunk; k <<= 1) {
@@ -341,7 +343,8 @@ cudaError_t launch_vector_scores(const float* I, int M, int K, int T, double* V,
 }
 
 // The ranking from V: chunk sort, then merge.
-cudaError_t launch_rank_sort(const double* V, const int32_t* perm, int M, int K, int T,
+cudaError_t launch_rank_sort(const double* V, const int32_t* perm, long long perm_stride, int M,
+                             int K, int T,
                              int32_t* rank, void* scratch, cudaStream_t s,
                              unsigned long long* zero64 = nullptr, size_t n64 = 0,
                              int* zero32 = nullptr, size_t n32 = 0) {
@@ -352,7 +355,8 @@ cudaError_t launch_rank_sort(const double* V, const int32_t* perm, int M, int K,
   Carve c{static_cast<char*>(scratch), 0};
   unsigned long long* skey = c.take<unsigned long long>((size_t)nt * Kp);
   unsigned short* sidx = c.take<unsigned short>((size_t)nt * Kp);
-  chunk_sort_kernel<<<dim3(nchunk, nt), kRankChunk, 0, s>>>(V, perm, K, Kp, skey, sidx, zero64,
+  chunk_sort_kernel<<<dim3(nchunk, nt), kRankChunk, 0, s>>>(V, perm, perm_stride, K, Kp, skey,
+                                                             sidx, zero64,
                                                             n64, zero32, n32);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -390,12 +394,13 @@ cudaError_t side_stream(SideStream** out) {
 
 }  // namespace
 
-cudaError_t launch_vector_rank(const float* I, const int32_t* perm, int M, int K, int T,
+cudaError_t launch_vector_rank(const float* I, const int32_t* perm, long long perm_stride, int M,
+                               int K, int T,
                                double* V, int32_t* rank, int* tile_pmax, void* scratch,
                                cudaStream_t s) {
   cudaError_t e = launch_vector_scores(I, M, K, T, V, tile_pmax, s);
   if (e != cudaSuccess) return e;
-  return launch_rank_sort(V, perm, M, K, T, rank, scratch, s);
+  return launch_rank_sort(V, perm, perm_stride, M, K, T, rank, scratch, s);
 }
 
 // Adds v * 2^sh (v < 2^64) into the little-endian multi-limb integer z[0..5].
@@ -489,7 +494,8 @@ struct CandidateList {
 // vectors' column sums -> rdense[t][m] (values below the tile's scale go to the buckets).
 template <int kPerMax>
 __global__ void __launch_bounds__(512, 2) candidate_lists_kernel(
-    const float* __restrict__ I, const int32_t* __restrict__ perm, const int32_t* __restrict__ rank,
+    const float* __restrict__ I, const int32_t* __restrict__ perm_all, long long perm_stride,
+    const int32_t* __restrict__ rank,
     const int* __restrict__ tile_pmax, const U128* __restrict__ colsum,
     const unsigned char* __restrict__ coltiny, int K, int T, CandidateList cl, int ncand,
     unsigned short* __restrict__ band, U128* __restrict__ rdense,
@@ -497,6 +503,7 @@ __global__ void __launch_bounds__(512, 2) candidate_lists_kernel(
   __shared__ int warp_tot[16];
   __shared__ U128 warp_acc[16];
   const int m = blockIdx.x, t = blockIdx.y;
+  const int32_t* perm = perm_all ? perm_all + t * perm_stride : perm_all;  // this tile's order
   const Candidate cand = cl.c[m];
   const int n4 = cand.n4, n24 = cand.n24;
   const int32_t* rk = rank + (size_t)t * K;
@@ -842,6 +849,7 @@ size_t search_workspace_bytes(int M, int K, int T, int ncand) {
 }
 
 cudaError_t launch_boundary_search(const float* I, const void* stats, const int32_t* perm,
+                                   long long perm_stride,
                                    int M, int K, int T, double t_s, double alpha,
                                    const Candidate* cands, int ncand, int32_t* counts_out,
                                    double* vs_out, int32_t* rank_out, double* retained_out,
@@ -897,7 +905,7 @@ cudaError_t launch_boundary_search(const float* I, const void* stats, const int3
     e = cudaEventRecord(ss->join, ss->stream);
     if (e != cudaSuccess) return e;
     // the sort also clears the exponent buckets and their flags (used from candidate_lists on)
-    e = launch_rank_sort(V, perm, M, K, T, rank, rank_scratch, s, bucket,
+    e = launch_rank_sort(V, perm, perm_stride, M, K, T, rank, rank_scratch, s, bucket,
                          (size_t)nt * ncand * 256, bucket_used, (size_t)nt * ncand);
     if (e != cudaSuccess) return e;
     e = cudaStreamWaitEvent(s, ss->join, 0);
@@ -909,13 +917,13 @@ cudaError_t launch_boundary_search(const float* I, const void* stats, const int3
     const dim3 gl(ncand, nt);
     const int per = (K + 511) / 512;
     if (per <= 8)
-      candidate_lists_kernel<8><<<gl, 512, 0, s>>>(I, perm, rank, pmax, colsum, coltiny, K, T, cl,
+      candidate_lists_kernel<8><<<gl, 512, 0, s>>>(I, perm, perm_stride, rank, pmax, colsum, coltiny, K, T, cl,
                                                    ncand, band, rdense, bucket, bucket_used);
     else if (per <= 16)
-      candidate_lists_kernel<16><<<gl, 512, 0, s>>>(I, perm, rank, pmax, colsum, coltiny, K, T, cl,
+      candidate_lists_kernel<16><<<gl, 512, 0, s>>>(I, perm, perm_stride, rank, pmax, colsum, coltiny, K, T, cl,
                                                     ncand, band, rdense, bucket, bucket_used);
     else
-      candidate_lists_kernel<32><<<gl, 512, 0, s>>>(I, perm, rank, pmax, colsum, coltiny, K, T, cl,
+      candidate_lists_kernel<32><<<gl, 512, 0, s>>>(I, perm, perm_stride, rank, pmax, colsum, coltiny, K, T, cl,
                                                     ncand, band, rdense, bucket, bucket_used);
   }
   e = cudaGetLastError();

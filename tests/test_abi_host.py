@@ -195,36 +195,80 @@ def test_tile_pairs_hint_rule():
     assert not H.tile_pairs_hint(H.hinm_counts_from_vs(K, 0.5, 0.25), None, K)
 
 
-@pytest.mark.parametrize("T,K,n,S,iters,seed", [(8, 32, 32, 4, 2, 1), (32, 128, 96, 8, 3, 2),
-                                                 (16, 256, 256, 32, 5, 3)])
-def test_gyro_refine_host_matches_oracle(T, K, n, S, iters, seed):
-    """The native gyro-style refinement (host code of the library) against the oracle's
-    (scipy's assignment as its step): the same refined band and the same retained-importance
-    history bit for bit (the same fp64 additions in the same order); the history never falls."""
+@pytest.mark.parametrize("T,K,n,G,k,seed", [(8, 64, 48, 4, 2, 1), (128, 1024, 512, 16, 2, 2),
+                                            (32, 256, 128, 8, 1, 3), (64, 512, 256, 12, 3, 4),
+                                            (16, 128, 96, 6, 4, 5)])
+def test_gyro_input_round_host_matches_oracle(T, K, n, G, k, seed):
+    """The native in-tile round (host code of the library) against the oracle, bit for bit:
+    the refined band and both costs, over three chained rounds with fresh draws."""
     import pruning_hinm_spmm_b200 as H
     rng = np.random.default_rng(seed)
     I_tile = rng.exponential(1.0, (T, K)).astype(np.float32)
     band = rng.permutation(K)[:n].astype(np.int32)
-    sched = np.stack([np.stack([rng.choice(n // 4, S, replace=False), rng.integers(0, 4, S)], axis=1)
-                      for _ in range(iters)]).astype(np.int32)
-    got_band, got_hist = H.hinm_gyro_refine_host(I_tile, band, sched)
-    want_band, want_hist = O.gyro_refine(I_tile, band, sched)
-    np.testing.assert_array_equal(got_band, want_band)
-    np.testing.assert_array_equal(got_hist, want_hist)
-    assert (np.diff(got_hist) >= 0).all()
+    got, want = band.copy(), band.copy()
+    for _ in range(3):
+        groups = rng.choice(n // 4, G, replace=False).astype(np.int32)
+        slots = np.stack([rng.choice(4, k, replace=False) for _ in range(G)]).astype(np.int32)
+        got, gc = H.hinm_gyro_input_round_host(I_tile, got, groups, slots)
+        want, wc = O.gyro_input_round(I_tile, want, groups, slots)
+        np.testing.assert_array_equal(got, want)
+        assert gc == wc
+    assert H.hinm_gyro_band_cost_host(I_tile, got) == O.band_pruning_cost(I_tile, got)
 
 
-def test_gyro_refine_host_validation():
+@pytest.mark.parametrize("T,K,nt,G,k,seed", [(4, 16, 5, 3, 1, 1), (16, 64, 6, 4, 2, 2),
+                                             (8, 256, 10, 5, 3, 3)])
+def test_gyro_output_round_host_matches_oracle(T, K, nt, G, k, seed):
+    """The native output-channel round against the oracle, bit for bit, over two rounds."""
+    import pruning_hinm_spmm_b200 as H
+    rng = np.random.default_rng(seed)
+    I = rng.exponential(1.0, (nt * T, K)).astype(np.float32)
+    n0 = rng.integers(0, K // 2, nt).astype(np.int32)
+    order = rng.permutation(nt * T).astype(np.int32)
+    got, want = order.copy(), order.copy()
+    for _ in range(2):
+        tiles = rng.choice(nt, G, replace=False).astype(np.int32)
+        rows = np.stack([rng.choice(T, k, replace=False) for _ in range(G)]).astype(np.int32)
+        got, gc = H.hinm_gyro_output_round_host(I, T, n0, got, tiles, rows)
+        want, wc = O.gyro_output_round(I, T, n0, want, tiles, rows)
+        np.testing.assert_array_equal(got, want)
+        assert gc == wc
+
+
+def test_gyro_host_validation():
     import pruning_hinm_spmm_b200 as H
     I_tile = np.ones((4, 16), dtype=np.float32)
     band = np.arange(8, dtype=np.int32)
-    with pytest.raises(H.HinmError):
-        H.hinm_gyro_refine_host(I_tile, band[:6], np.zeros((1, 1, 2), dtype=np.int32))
-    with pytest.raises(H.HinmError):   # the same group twice in one iteration
-        H.hinm_gyro_refine_host(I_tile, band, np.array([[[0, 1], [0, 2]]], dtype=np.int32))
-    with pytest.raises(H.HinmError):   # slot outside 0..3
-        H.hinm_gyro_refine_host(I_tile, band, np.array([[[1, 4]]], dtype=np.int32))
+    g1, s1 = np.array([0], dtype=np.int32), np.array([[1]], dtype=np.int32)
+    with pytest.raises(H.HinmError):      # band length not a multiple of 4
+        H.hinm_gyro_input_round_host(I_tile, band[:6], g1, s1)
+    with pytest.raises(H.HinmError):      # repeated group
+        H.hinm_gyro_input_round_host(I_tile, band, np.array([0, 0], dtype=np.int32),
+                                     np.array([[1], [2]], dtype=np.int32))
+    with pytest.raises(H.HinmError):      # slot outside [0, 4)
+        H.hinm_gyro_input_round_host(I_tile, band, g1, np.array([[4]], dtype=np.int32))
+    with pytest.raises(H.HinmError):      # repeated slot within a group
+        H.hinm_gyro_input_round_host(I_tile, band, g1, np.array([[1, 1]], dtype=np.int32))
     bad = band.copy()
-    bad[3] = 99
-    with pytest.raises(H.HinmError):   # channel outside [0, K)
-        H.hinm_gyro_refine_host(I_tile, bad, np.array([[[1, 0]]], dtype=np.int32))
+    bad[3] = 16
+    with pytest.raises(H.HinmError):      # channel outside [0, K)
+        H.hinm_gyro_input_round_host(I_tile, bad, g1, s1)
+    bad[3] = 0
+    with pytest.raises(H.HinmError):      # repeated channel
+        H.hinm_gyro_input_round_host(I_tile, bad, g1, s1)
+    inf = I_tile.copy()
+    inf[2, 5] = np.inf                    # a non-finite importance the round reads
+    with pytest.raises(H.HinmError):
+        H.hinm_gyro_input_round_host(inf, band, g1, s1)
+    nan = I_tile.copy()
+    nan[1, 0] = np.nan
+    with pytest.raises(H.HinmError):
+        H.hinm_gyro_input_round_host(nan, band, g1, s1)
+    I = np.ones((8, 16), dtype=np.float32)
+    with pytest.raises(H.HinmError):      # row order not a permutation
+        H.hinm_gyro_output_round_host(I, 4, [1, 1], [0, 1, 2, 3, 4, 5, 6, 6], [0], [[0]])
+    with pytest.raises(H.HinmError):      # n0 > K
+        H.hinm_gyro_output_round_host(I, 4, [1, 17], np.arange(8), [0], [[0]])
+    I[5, 3] = np.nan
+    with pytest.raises(H.HinmError):      # non-finite in a sampled tile
+        H.hinm_gyro_output_round_host(I, 4, [1, 1], np.arange(8), [1], [[0]])

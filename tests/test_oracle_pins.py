@@ -594,44 +594,168 @@ def test_epilogue_reference_bias_per_row():
     np.testing.assert_array_equal(O.spmm_epilogue_reference(y, None, O.ACT_NONE), y)
 
 
-# ----------------------------------------------------------------------------- gyro refinement
-def test_gyro_refine_hand_example():
-    """One row, two groups [9, 8, 7, 1] and [6, 5, 4, 3]: retained 17 + 11 = 28.  Sampling the
-    7 (group 0, slot 2) and the 3 (group 1, slot 3) and swapping them gives [9, 8, 3, 1] and
-    [6, 5, 4, 7]: 17 + 13 = 30, the better of the two assignments."""
+# ----------------------------------------------------------------------------- gyro-permutation
+def test_group_cost_and_retained_hand_example():
+    """Two rows whose top-2 differ: row 0 (9, 8, 7, 1) keeps 9 + 8 and prunes 7 + 1; row 1
+    (1, 2, 9, 8) keeps 9 + 8 and prunes 1 + 2.  Retained 17 + 17 = 34, pruned 8 + 3 = 11,
+    and together they are the group's whole importance (45)."""
+    I_tile = np.array([[9, 8, 7, 1], [1, 2, 9, 8]], dtype=np.float32)
+    assert O.group_retained(I_tile, [0, 1, 2, 3]) == 34.0
+    assert O.group_pruning_cost(I_tile, [0, 1, 2, 3]) == 11.0
+    # member order does not matter; a different grouping of the same channels changes both
+    assert O.group_pruning_cost(I_tile, [3, 1, 0, 2]) == 11.0
+    I2 = np.array([[9, 8, 7, 1, 6, 5, 4, 3], [1, 2, 9, 8, 3, 4, 5, 6]], dtype=np.float32)
+    assert O.group_pruning_cost(I2, [4, 5, 6, 7]) == 7.0 + 7.0   # (4 + 3), (3 + 4)
+    assert O.band_pruning_cost(I2, np.arange(8)) == 11.0 + 14.0
+
+
+def _brute_balanced_partitions(S, k):
+    """Every partition of range(S) into S/k unordered blocks of size k."""
+    def rec(rest):
+        if not rest:
+            yield []
+            return
+        first = rest[0]
+        import itertools
+        for comb in itertools.combinations(rest[1:], k - 1):
+            block = [first, *comb]
+            left = [x for x in rest if x not in block]
+            for tail in rec(left):
+                yield [block, *tail]
+    yield from rec(list(range(S)))
+
+
+def test_balanced_kmeans_regroups_planted_pairs():
+    """Points 0, 0.1 | 10, 5 | 5.1, 10.1 seeded as those three pairs: the seeds' centroids
+    are 0.05, 7.5 and 7.6; the best balanced assignment to them (worked out by hand:
+    {5, 5.1} -> 7.5 and {10, 10.1} -> 7.6 cost 24.02 against 25 for the seeds) regroups the
+    planted pairs {5, 5.1} and {10, 10.1}, which is then a fixed point; every cluster keeps
+    exactly k = 2 points."""
+    F = np.array([[0.0], [0.1], [10.0], [5.0], [5.1], [10.1]])
+    cl = O.balanced_kmeans(F, 2, 10)
+    assert cl == [[0, 1], [3, 4], [2, 5]]
+    assert O.balanced_kmeans(F, 2, 0) == [[0, 1], [2, 3], [4, 5]]   # no iteration: the seeds
+
+
+def test_balanced_kmeans_fixed_point_brute_force():
+    """The result is a fixed point of the balanced iteration: with the result's centroids,
+    no balanced partition (all 15 of 6 points into pairs, enumerated) has a smaller total
+    squared distance; and the within-cluster sum of squares does not rise from the seed
+    partition to the result."""
+    rng = np.random.default_rng(4)
+    for trial in range(20):
+        F = rng.normal(size=(6, 3))
+        cl = O.balanced_kmeans(F, 2, 20)
+        C = [F[c].mean(axis=0) for c in cl]
+
+        def assign_cost(part):
+            # best matching of the blocks to the centroids (3! ways), squared distances
+            import itertools
+            best = None
+            for p in itertools.permutations(range(3)):
+                v = sum(((F[b] - C[p[i]]) ** 2).sum() for i, blk in enumerate(part) for b in blk)
+                best = v if best is None else min(best, v)
+            return best
+        mine = sum(((F[b] - C[i]) ** 2).sum() for i, c in enumerate(cl) for b in c)
+        assert mine <= min(assign_cost(p) for p in _brute_balanced_partitions(6, 2)) + 1e-12
+        seed = [[0, 1], [2, 3], [4, 5]]
+        sse = lambda part: sum(((F[c] - F[c].mean(axis=0)) ** 2).sum() for c in part)
+        assert sse(cl) <= sse(seed) + 1e-12
+
+
+def test_gyro_input_round_k1_hand_example():
+    """k = 1 (every cluster one vector): tile row [9 8 7 1 | 6 5 4 3], sampling the 7 (group 0,
+    slot 2) and the 3 (group 1, slot 3): swapping them prunes 3 + 1 and 6 + 5 ... the
+    cheaper of the two assignments: cost 8 + 7 = 15 before, 4 + 9 = 13 after."""
     I_tile = np.array([[9, 8, 7, 1, 6, 5, 4, 3]], dtype=np.float32)
-    band = np.arange(8)
-    sched = np.array([[[0, 2], [1, 3]]])
-    out, hist = O.gyro_refine(I_tile, band, sched)
-    np.testing.assert_array_equal(hist, [28.0, 30.0])
+    out, (before, after) = O.gyro_input_round(I_tile, np.arange(8), [0, 1], [[2], [3]])
+    assert (before, after) == (15.0, 13.0)
     np.testing.assert_array_equal(out, [0, 1, 7, 3, 4, 5, 6, 2])
 
 
-def test_gyro_refine_brute_force_and_invariants():
-    """S = 4 sampled groups: the chosen assignment's total equals the best of all 24
-    (brute force); over several iterations the retained importance never falls, the band
-    stays a permutation of its channels and the groups not sampled keep their members."""
+def test_gyro_input_round_brute_force_and_invariants():
+    """k = 2, G = 3: the chosen placement of the clusters costs the least of all 3! (costs
+    recomputed here from sorted rows); the band stays a permutation of its channels, the
+    unsampled groups keep their members, and over rounds the band's pruning cost never rises."""
     import itertools
-    rng = np.random.default_rng(17)
-    T, K = 16, 64
+    rng = np.random.default_rng(21)
+    T, K = 12, 48
     I_tile = rng.exponential(1.0, (T, K)).astype(np.float32)
-    band = rng.permutation(K)[:48]                  # 12 groups of a 2:4 band
-    sched = np.array([[[1, 0], [4, 3], [7, 1], [10, 2]]])
-    out, hist = O.gyro_refine(I_tile, band, sched)
-    groups, slots = [1, 4, 7, 10], [0, 3, 1, 2]
-    vecs = [int(band[4 * g + k]) for g, k in zip(groups, slots)]
-    best = -1.0
-    for p in itertools.permutations(range(4)):
-        b2 = band.copy()
-        for a, b in enumerate(p):
-            b2[4 * groups[b] + slots[b]] = vecs[a]
-        best = max(best, sum(O.group_retained(I_tile, list(b2[4 * g:4 * g + 4])) for g in range(12)))
-    assert abs(hist[1] - best) <= 1e-9 * best
-    sched4 = np.array([[[g, (g * 7 + it) % 4] for g in rng.choice(12, 6, replace=False)]
-                       for it in range(5)])
-    out4, hist4 = O.gyro_refine(I_tile, band, sched4)
-    assert (np.diff(hist4) >= -1e-12 * hist4[0]).all()
-    assert sorted(out4.tolist()) == sorted(band.tolist())
-    touched = set(int(g) for g in sched4[:, :, 0].ravel())
-    for g in set(range(12)) - touched:
-        np.testing.assert_array_equal(out4[4 * g:4 * g + 4], band[4 * g:4 * g + 4])
+    band = rng.permutation(K)[:40]                      # 10 groups
+    groups, slots = [2, 5, 8], [[0, 3], [1, 2], [0, 1]]
+    out, (before, after) = O.gyro_input_round(I_tile, band, groups, slots)
+    vecs = [int(band[4 * g + s]) for g, ss in zip(groups, slots) for s in ss]
+    F = I_tile[:, vecs].T.astype(np.float64)
+    clusters = O.balanced_kmeans(F, 2, 8)
+
+    def cost(members):  # the two smallest per row, rows ascending
+        acc = 0.0
+        for r in range(T):
+            v = np.sort(I_tile[r, members].astype(np.float64))
+            acc += v[1] + v[0]
+        return acc
+
+    def members_with(i, cl):
+        m = [int(x) for x in band[4 * groups[i]:4 * groups[i] + 4]]
+        for s, p in zip(sorted(slots[i]), cl):
+            m[s] = vecs[p]
+        return m
+    best = min(sum(cost(members_with(i, clusters[p[i]])) for i in range(3))
+               for p in itertools.permutations(range(3)))
+    assert abs(min(after, before) - min(best, before)) <= 1e-9 * before
+    assert sorted(out.tolist()) == sorted(band.tolist())
+    for g in set(range(10)) - set(groups):
+        np.testing.assert_array_equal(out[4 * g:4 * g + 4], band[4 * g:4 * g + 4])
+    b = band.copy()
+    costs = [O.band_pruning_cost(I_tile, b)]
+    for it in range(4):
+        gs = rng.choice(10, 4, replace=False)
+        ss = [sorted(rng.choice(4, 2, replace=False)) for _ in gs]
+        b, _ = O.gyro_input_round(I_tile, b, gs, ss)
+        costs.append(O.band_pruning_cost(I_tile, b))
+    assert all(c1 <= c0 + 1e-9 * c0 for c0, c1 in zip(costs, costs[1:]))
+
+
+def test_tile_perm_with_band():
+    perm_t = np.array([5, 0, 3, 1, 4, 2])
+    region_t = np.array([1, 2, 0, 1, 1, 1], dtype=np.int8)   # by channel
+    # 2:4 channels in working order: 5, 0, 3, 4 at positions 0, 1, 2, 4 (1 dense, 2 pruned)
+    out = O.tile_perm_with_band(perm_t, region_t, [4, 3, 0, 5])
+    np.testing.assert_array_equal(out, [4, 3, 0, 1, 5, 2])
+
+
+def test_column_pruning_cost_hand_example():
+    """Rows [1 5 2 9], [2 1 2 0]: scores 3 6 4 9; the two smallest (3 + 4) = 7."""
+    I_rows = np.array([[1, 5, 2, 9], [2, 1, 2, 0]], dtype=np.float32)
+    assert O.column_pruning_cost(I_rows, 2) == 7.0
+    assert O.column_pruning_cost(I_rows, 0) == 0.0
+
+
+def test_gyro_output_round_brute_force_and_invariants():
+    """G = 3 tiles, k = 1 row each: the chosen placement costs the least of all 3!; the row
+    order stays a permutation; unsampled tiles keep their rows; rounds never raise the cost."""
+    import itertools
+    rng = np.random.default_rng(8)
+    T, K, nt = 4, 16, 5
+    I = rng.exponential(1.0, (nt * T, K)).astype(np.float32)
+    n0 = np.array([5, 6, 4, 7, 5])
+    order = rng.permutation(nt * T)
+    tiles, rows = [0, 2, 4], [[1], [3], [0]]
+    out, (before, after) = O.gyro_output_round(I, T, n0, order, tiles, rows)
+    chans = [int(order[t * T + r[0]]) for t, r in zip(tiles, rows)]
+
+    def cpc(rows_, n):  # independent: sort the column sums
+        V = np.sort(I[rows_].astype(np.float64).sum(axis=0))
+        return float(V[:n].sum())
+
+    def tile_with(i, ch):
+        t = tiles[i]
+        cur = [int(x) for x in order[t * T:(t + 1) * T]]
+        cur[rows[i][0]] = ch
+        return cur
+    best = min(sum(cpc(tile_with(i, chans[p[i]]), n0[tiles[i]]) for i in range(3))
+               for p in itertools.permutations(range(3)))
+    assert abs(min(after, before) - min(best, before)) <= 1e-9 * before
+    assert sorted(out.tolist()) == list(range(nt * T))
+    for t in (1, 3):
+        np.testing.assert_array_equal(out[t * T:(t + 1) * T], order[t * T:(t + 1) * T])
