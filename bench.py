@@ -1,17 +1,20 @@
 #!/usr/bin/env python
 """Benchmark of the HiNM hot path on B200: importance -> boundary search -> mask ->
-compress -> SpMM, one pass per step, on the pure 2:4 workload
-(W 4096x4096 bf16 ~N(0,0.02) with 1% x10 outliers, X 4096x2048 bf16 ~N(0,1), tile 128,
-t_s = 0.5, v_s from the search, alpha = 1/32).
+compress -> SpMM, one pass per step.  The headline workload is the HiNM up-projection
+(W 11008x4096 bf16 ~N(0,0.02), X 4096x4096 bf16 ~N(0,1), tile 128 rows, t_s = 0.75 with the
+fixed boundary v_s = 0.6, a seeded input-channel permutation folded into the index);
+the pure 2:4 (4096x4096x2048) and the decode down-projection (4096x11008x16) workloads are
+measured in the same run as extra keys.
 
 Prints ONE JSON line (rank 0).  `value` is the effective (dense-equivalent) TFLOP/s of the
-whole step, 2*M*K*N per step over all ranks / max-over-ranks step time; the per-kernel
-breakdown, the roofline of the dominant kernel, the end-to-end number through host
-buffers and the CPU oracle baseline are extra keys.
+whole step, 2*M*K*N of the whole problem / max-over-ranks step time; the per-kernel
+breakdown, the roofline of the SpMM, the end-to-end number through host buffers and the
+CPU oracle baseline are extra keys.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {hinm,reference}]
-Multi-GPU: launched with torch.distributed.run, one rank per GPU; every rank runs its own
-seeded shard of the same shape (weak scaling, no data-path collective).
+Multi-GPU: launched with torch.distributed.run, one rank per GPU; the tiles of the one W
+are split across the ranks (contiguous runs of whole tiles, X replicated, each rank writes
+its row block of Y; --gather-y adds the NCCL all-gather of Y to every step): strong scaling.
 """
 from __future__ import annotations
 
@@ -31,11 +34,11 @@ sys.path.insert(0, ROOT)
 import hinm_inputs as hi  # noqa: E402
 
 METRIC = "HiNM SpMM TFLOP/s (eff.) and HBM GB/s, % of 2:4-sparse/HBM roofline"
-WORKLOADS = {  # name -> seeded generator (rank r draws seed r)
-    "pure24": lambda r: hi.pure24(seed=r),
-    "tiny": lambda r: hi.tiny_hinm(seed=r),
-    "up": lambda r: hi.hinm_up_proj(seed=r),
-    "decode": lambda r: hi.decode_down_proj(seed=r),
+WORKLOADS = {  # name -> seeded generator (seed 0: every rank draws the same problem)
+    "pure24": lambda: hi.pure24(seed=0),
+    "tiny": lambda: hi.tiny_hinm(seed=0),
+    "up": lambda: hi.hinm_up_proj(seed=0),
+    "decode": lambda: hi.decode_down_proj(seed=0),
 }
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -52,9 +55,10 @@ def max_over_ranks(x: float, dist, device) -> float:
     return float(t.item())
 
 
-def job_value(flops_per_rank: float, world: int, t_max: float) -> float:
-    """Whole-job throughput in TFLOP/s: every rank's shard over the slowest rank's time."""
-    return flops_per_rank * world / t_max / 1e12
+def job_value(flops_total: float, t_max: float) -> float:
+    """Whole-job throughput in TFLOP/s: the whole problem's FLOPs over the slowest rank's
+    time (the ranks split one problem's tiles)."""
+    return flops_total / t_max / 1e12
 
 
 def gather_rows(Y_shard, M: int, T: int, world: int, dist, shard_tiles):
@@ -398,26 +402,30 @@ def time_dense_context(M, K, N, flush, stream, reps=10):
             "note": "dense W (no pruning) through cuBLAS, same M, K, N; context only"}
 
 
-def time_gyro(H, hp, perm, T, K, S=64, iters=4):
-    """The host gyro-style refinement on tile 0 of this step: its importance rows, its 2:4
-    band in working order (from the step's regions), a seeded schedule of S (group, slot)
-    samples per iteration; wall-clock time on one host core."""
+def time_gyro(H, hp, perm, T, K, G=16, k=2, rounds=4):
+    """The library's in-tile gyro rounds (host) on tile 0 of this step: its importance rows,
+    its 2:4 band in working order (from the step's regions), `rounds` rounds of G sampled
+    groups x k slots (seeded draws); wall-clock time on one host core, and the band's
+    pruning cost before and after."""
     import time
     I_tile = hp.I[:T].cpu().numpy()
     region0 = hp.region[0].cpu().numpy()
     band = np.array([c for c in perm if region0[c] == 1], dtype=np.int32)
     ng = band.size // 4
-    if ng == 0:
-        return {"note": "tile 0 has no 2:4 band"}
-    S = min(S, ng)
+    if ng < 2:
+        return {"note": "tile 0 has no 2:4 band to refine"}
+    G = min(G, ng)
     rng = np.random.default_rng(7)
-    sched = np.stack([np.stack([rng.choice(ng, S, replace=False), rng.integers(0, 4, S)], axis=1)
-                      for _ in range(iters)]).astype(np.int32)
+    c0 = H.hinm_gyro_band_cost_host(I_tile, band)
     t0 = time.perf_counter()
-    _, hist = H.hinm_gyro_refine_host(I_tile, band, sched)
+    for _ in range(rounds):
+        groups = rng.choice(ng, G, replace=False).astype(np.int32)
+        slots = np.stack([rng.choice(4, k, replace=False) for _ in range(G)]).astype(np.int32)
+        band, _ = H.hinm_gyro_input_round_host(I_tile, band, groups, slots)
     dt = time.perf_counter() - t0
-    return {"ms_per_iteration": dt / iters * 1e3, "groups": ng, "samples_per_iteration": S,
-            "iterations": iters, "retained_gain": float(hist[-1] / hist[0] - 1.0),
+    c1 = H.hinm_gyro_band_cost_host(I_tile, band)
+    return {"ms_per_round": dt / rounds * 1e3, "groups": ng, "sampled_groups": G,
+            "slots_per_group": k, "rounds": rounds, "pruning_cost_change": c1 / c0 - 1.0,
             "where": "host (offline, once per layer)", "cores": 1}
 
 
@@ -450,6 +458,220 @@ def time_hard_concrete(H, n, peaks, stream, reps=10):
             "note": "back-to-back calls; 13 B per element, arrays larger than L2"}
 
 
+# ------------------------------------------------------------------ SpMM operand ingest
+# The SpMM kernel's operand traffic from L2 into shared memory, per launch, by the kernel the
+# library picks for (N, T, hint): every tile's A blocks (16 KB, plus 2 KB of metadata for a
+# 2:4 block) once per column block of BN columns, and every tile's gathered X rows
+# (64 per dense block, 128 per 2:4 block) x the block's columns x 2 bytes; with the tile-pair
+# hint a pair whose blocks are the same runs reads each X block once for both tiles.
+def spmm_plan(N: int, T: int, tile_pairs: bool):
+    if N <= 16:
+        return "spmm_kernel<16>", 16
+    if N <= 32:
+        return "spmm_kernel<32>", 32
+    if N <= 64:
+        return "spmm_kernel<64>", 64
+    if N < 256:
+        return "spmm_kernel<128>", 128
+    if tile_pairs and T == 128 and N >= 1024:
+        return "spmm_pair_kernel", 240
+    return "spmm_kernel<256>", 256
+
+
+def l2_to_sm_bytes(M: int, N: int, T: int, counts, tile_pairs: bool) -> float:
+    c = np.asarray(counts, dtype=np.int64).reshape(-1, 3)
+    nd = -(-c[:, 2] // 64)
+    ns = -(-c[:, 1] // 128)
+    name, bn = spmm_plan(N, T, tile_pairs)
+    ncol = -(-N // bn)
+    a_bytes = float(((nd + ns) * 16384 + ns * 2048).sum()) * ncol
+    x_rows = (nd * 64 + ns * 128).astype(np.float64)
+    x_bytes = float(x_rows.sum()) * N * 2.0
+    if name == "spmm_pair_kernel":
+        # shared pairs (identical run lists: the hint's case) read each X block once
+        x_bytes = float(x_rows[::2].sum()) * N * 2.0
+    return a_bytes + x_bytes
+
+
+def count_graph_kernels(graph):
+    """(kernel launches one replay of the captured step issues, their function names),
+    counted on the captured cudaGraph_t through the CUDA runtime; (None, []) if the query is
+    not available."""
+    try:
+        import cuda.bindings.runtime as rt
+        g = rt.cudaGraph_t(init_value=graph.raw_cuda_graph())
+        err, _, n = rt.cudaGraphGetNodes(g, 0)
+        err, nodes, n = rt.cudaGraphGetNodes(g, n)
+        names, count = set(), 0
+        for node in nodes[:n]:
+            err, kind = rt.cudaGraphNodeGetType(node)
+            if kind != rt.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+                continue
+            count += 1
+            try:
+                err, prm = rt.cudaGraphKernelNodeGetParams(node)
+                err, nm = rt.cudaFuncGetName(prm.func)
+                names.add(nm.decode() if isinstance(nm, bytes) else str(nm))
+            except Exception:  # noqa: BLE001 - names are informative only
+                pass
+        return count, sorted(names)
+    except Exception:  # noqa: BLE001
+        return None, []
+
+
+# ------------------------------------------------------------------ one workload on the GPU
+def measure(H, w, args, dev, flush, stream, rows=None, dist=None, sampler=None):
+    """Time the five-call step of workload w on this rank's rows [r0, r1) of W (all rows on
+    one GPU): K CUDA-graph replays (L2 flushed between them) and K eager passes with events
+    between the phases.  Returns the measurements and the state the caller reuses."""
+    import torch
+    M, K, N, T = w.M, w.K, w.N, w.T
+    r0, r1 = rows if rows is not None else (0, M)
+    Ms = r1 - r0
+    have = Ms > 0
+    out = dict(rows=(r0, r1))
+    if have:
+        W = torch.from_numpy(np.ascontiguousarray(w.W_bits[r0:r1]).view(np.int16)).to(dev).view(torch.bfloat16)
+        X = torch.from_numpy(w.X_bits.view(np.int16)).to(dev).view(torch.bfloat16)
+        perm = torch.from_numpy(w.perm).to(dev)
+        hp = H.HotPath(Ms, K, N, T, w.t_s, w.alpha, device=dev)
+        # Workloads specified with a fixed boundary v_s use its closed-form counts; the search
+        # still runs every step (its ranking feeds the mask).  Otherwise the search's counts.
+        fixed = c = None
+        if w.v_s is not None:
+            c = H.hinm_counts_from_vs(K, w.t_s, w.v_s)
+            fixed = torch.tensor([c] * (Ms // T), dtype=torch.int32, device=dev)
+        counts_used = fixed if fixed is not None else hp.counts
+        # fixed counts known on the host: tell the SpMM when every tile reads the same X rows
+        tile_pairs = fixed is not None and H.tile_pairs_hint(c, w.perm, K)
+        Yfull = torch.empty((M, N), dtype=torch.float32, device=dev) if args.gather_y else None
+
+        def step(ev=None):
+            if ev is not None:
+                ev[0].record(stream)
+            H.hinm_importance_stats(W, X, T, hp.I, hp.stats, hp.ws)
+            if ev is not None:
+                ev[1].record(stream)
+            H.hinm_boundary_search(hp.I, perm, T, w.t_s, w.alpha, hp.counts, hp.vs, hp.rank,
+                                   hp.ws, stats=hp.stats)
+            if ev is not None:
+                ev[2].record(stream)
+            H.hinm_mask(hp.I, perm, counts_used, T, hp.rank, hp.bitmask, hp.region, hp.ws)
+            if ev is not None:
+                ev[3].record(stream)
+            H.hinm_compress(W, hp.bitmask, hp.region, perm, counts_used, T, hp.layout, hp.ws)
+            if ev is not None:
+                ev[4].record(stream)
+            H.hinm_spmm(hp.layout, X, hp.Y, None, hp.c_layout, tile_pairs)
+            if ev is not None:
+                ev[5].record(stream)
+
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        st = H.hinm_device_status()
+        if st != 0:
+            raise RuntimeError(f"device status {st} after warm-up")
+        counts = counts_used.cpu().numpy()
+        out.update(W=W, X=X, perm=perm, hp=hp, fixed=fixed, tile_pairs=tile_pairs, counts=counts,
+                   vs=hp.vs.cpu().numpy())
+        try:
+            graph = torch.cuda.CUDAGraph(keep_graph=True)
+        except TypeError:
+            graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        launches, kernel_names = count_graph_kernels(graph)
+        if hasattr(graph, "instantiate"):
+            try:
+                graph.instantiate()
+            except RuntimeError:
+                pass
+        torch.cuda.synchronize()
+    else:
+        graph = step = None
+        launches, kernel_names = 0, []
+    out.update(launches_per_step=launches, kernel_names=kernel_names)
+    gev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler is not None:
+        sampler.start()
+        time.sleep(0.4)
+    for k in range(args.steps):
+        flush.zero_()                     # evict L2 (256 MB > 126 MB) between timed steps
+        gev[k][0].record(stream)
+        if have:
+            graph.replay()
+        if args.gather_y and dist:
+            gathered = gather_rows(hp.Y if have else torch.zeros((0, N), device=dev), M, T,
+                                   dist.get_world_size(), dist, H.shard_tiles)
+            if have:
+                Yfull.copy_(gathered)
+        gev[k][1].record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    step_s = [gev[k][0].elapsed_time(gev[k][1]) * 1e-3 for k in range(args.steps)]
+    if have:
+        for k in range(args.steps):
+            flush.zero_()
+            step(evs[k])
+        torch.cuda.synchronize()
+        if H.hinm_device_status() != 0:
+            raise RuntimeError("device status after the timed passes")
+    if sampler is not None:
+        sampler.stop()
+    if dist:
+        dist.barrier()
+    phases = ["importance", "search", "mask", "compress", "spmm"]
+    if have:
+        out["per_phase"] = {p: statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) * 1e-3
+                                               for k in range(args.steps))
+                            for i, p in enumerate(phases)}
+        out["t_eager"] = statistics.mean(evs[k][0].elapsed_time(evs[k][5]) * 1e-3
+                                         for k in range(args.steps))
+    out["t_step"] = statistics.mean(step_s)
+    if graph is not None:
+        del graph
+    return out
+
+
+def spmm_roofline(M, K, N, T, counts, tile_pairs, t_spmm, peaks, peak_kind, traffic):
+    model = workload_model(M, K, N, T, counts)
+    bound, ach, pk, unit, frac = roofline_for("spmm", t_spmm, model, peaks, peak_kind)
+    name, bn = spmm_plan(N, T, tile_pairs)
+    ing = l2_to_sm_bytes(M, N, T, counts, tile_pairs)
+    return model, {
+        "bound": bound, "achieved": ach, "peak": pk, "unit": unit, "frac": frac,
+        "traffic": traffic, "kernel": name,
+        "peak_source": f"{peak_kind} (MEASURED_PEAKS.json burst; 2:4 = 2x dense bf16)",
+        "l2_to_sm": {"bytes_per_launch": ing, "achieved_tbs": ing / t_spmm / 1e12,
+                     "ceiling_tbs": L2_TO_SM_CEILING_TBS,
+                     "frac": ing / t_spmm / 1e12 / L2_TO_SM_CEILING_TBS,
+                     "ceiling_source": L2_TO_SM_CEILING_SOURCE,
+                     "basis": "A blocks (+metadata) once per BN-column block, gathered X rows "
+                              "x columns x 2 B per tile"}}
+
+
+# The L2 -> shared-memory ceiling the SpMM's operand stream is compared with: ncu's
+# peak-sustained rate of the L2 slices' output to the crossbar on this B200, derived from
+# the up-proj capture of spmm_kernel<256> (lts__lts2xbar_cycles_active 28.27 % of peak at
+# 6.48 TB/s of lts2xbar bytes).
+L2_TO_SM_CEILING_TBS = 22.9
+L2_TO_SM_CEILING_SOURCE = ("ncu peak-sustained lts2xbar rate on this B200 (28.27 % = 6.48 TB/s, "
+                           "up-proj spmm_kernel<256> capture)")
+
+
+def traffic_for(name, kernel):
+    tr_path = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tr_path):
+        return json.load(open(tr_path)).get(name, {}).get(kernel)
+    return None
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -458,10 +680,14 @@ def main():
     ap.add_argument("--impl", default="hinm", choices=["hinm", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-next-rows", action="store_true",
-                    help="skip the extra timings of the index translation, the fused epilogue "
-                         "and the Hard-Concrete forward (for a launch list of the step alone)")
-    ap.add_argument("--workload", default="pure24", choices=sorted(WORKLOADS) + ["sweep"],
-                    help="synthetic workload (default: the pure 2:4 4096x4096x2048 benchmark); "
+                    help="skip the extra timings of the index translation, the fused epilogue, "
+                         "the Hard-Concrete forward and the gyro refinement")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the pure 2:4 and decode workloads measured beside the headline")
+    ap.add_argument("--gather-y", action="store_true",
+                    help="multi-GPU: all-gather Y (NCCL) at the end of every timed step")
+    ap.add_argument("--workload", default="up", choices=sorted(WORKLOADS) + ["sweep"],
+                    help="synthetic workload (default: the HiNM up-proj 11008x4096x4096); "
                          "'sweep' times the LLaMA-2-7B-shaped layer sweep")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -474,7 +700,7 @@ def main():
         if world > 1 or args.impl == "reference":
             raise SystemExit("--workload sweep runs on one GPU with the CUDA arm only")
         return run_sweep(args)
-    w = WORKLOADS[args.workload](rank)
+    w = WORKLOADS[args.workload]()
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -490,154 +716,86 @@ def main():
 
     M, K, N, T = w.M, w.K, w.N, w.T
     dev = torch.device("cuda", local_rank)
-    W = torch.from_numpy(w.W_bits.view(np.int16)).to(dev).view(torch.bfloat16)
-    X = torch.from_numpy(w.X_bits.view(np.int16)).to(dev).view(torch.bfloat16)
-    perm = torch.from_numpy(w.perm).to(dev)
-    hp = H.HotPath(M, K, N, T, w.t_s, w.alpha, device=dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-
-    phases = ["importance", "search", "mask", "compress", "spmm"]
-    # Workloads specified with a fixed boundary v_s use its closed-form counts; the search
-    # still runs every step (its ranking feeds the mask).  Otherwise the search's counts.
-    fixed = None
-    if w.v_s is not None:
-        c = H.hinm_counts_from_vs(K, w.t_s, w.v_s)
-        fixed = torch.tensor([c] * (M // T), dtype=torch.int32, device=dev)
-    counts_used = fixed if fixed is not None else hp.counts
-    # fixed counts known on the host: tell the SpMM when every tile reads the same X rows
-    tile_pairs = fixed is not None and H.tile_pairs_hint(c, w.perm, K)
-
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        H.hinm_importance_stats(W, X, T, hp.I, hp.stats, hp.ws)
-        if ev is not None:
-            ev[1].record(stream)
-        H.hinm_boundary_search(hp.I, perm, T, w.t_s, w.alpha, hp.counts, hp.vs, hp.rank, hp.ws,
-                               stats=hp.stats)
-        if ev is not None:
-            ev[2].record(stream)
-        H.hinm_mask(hp.I, perm, counts_used, T, hp.rank, hp.bitmask, hp.region, hp.ws)
-        if ev is not None:
-            ev[3].record(stream)
-        H.hinm_compress(W, hp.bitmask, hp.region, perm, counts_used, T, hp.layout, hp.ws)
-        if ev is not None:
-            ev[4].record(stream)
-        H.hinm_spmm(hp.layout, X, hp.Y, None, hp.c_layout, tile_pairs)
-        if ev is not None:
-            ev[5].record(stream)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    st = H.hinm_device_status()
-    if st != 0:
-        raise RuntimeError(f"device status {st} after warm-up")
-    counts = counts_used.cpu().numpy()
-    vs = hp.vs.cpu().numpy()
-    model = workload_model(M, K, N, T, counts)
-
-    # The timed step replays a CUDA graph of the five calls, captured after the warm-up (which
-    # also did every one-time set-up); the per-phase times come from a second timed pass of
-    # the same step launched eagerly with events between the phases.
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        step()
-    torch.cuda.synchronize()
-    gev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    rows = H.shard_tiles(M, T, world, rank)
     sampler = ClockSampler(local_rank)
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    sampler.start()
-    time.sleep(0.4)
-    for k in range(args.steps):
-        flush.zero_()                     # evict L2 (256 MB > 126 MB) between timed steps
-        gev[k][0].record(stream)
-        graph.replay()
-        gev[k][1].record(stream)
-    torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    step_s = [gev[k][0].elapsed_time(gev[k][1]) * 1e-3 for k in range(args.steps)]
-    torch.cuda.synchronize()
-    for k in range(args.steps):
-        flush.zero_()
-        step(evs[k])
-    torch.cuda.synchronize()
-    sampler.stop()
-    if dist:
-        dist.barrier()
-    per_phase = {p: [evs[k][i].elapsed_time(evs[k][i + 1]) * 1e-3 for k in range(args.steps)]
-                 for i, p in enumerate(phases)}
-    t_step = statistics.mean(step_s)
-    t_eager = statistics.mean(evs[k][0].elapsed_time(evs[k][5]) * 1e-3 for k in range(args.steps))
-    del graph
-    t_step = max_over_ranks(t_step, dist, dev)
-    value = job_value(model["flops_eff"], world, t_step)
+    m = measure(H, w, args, dev, flush, stream, rows=rows, dist=dist, sampler=sampler)
+    have = rows[1] > rows[0]
+    t_step = max_over_ranks(m["t_step"], dist, dev)
+    value = job_value(2.0 * M * K * N, t_step)
 
     # ---------------- end to end through the public API with host buffers
-    # Every step copies its inputs in from pinned host memory and its Y out.  Two device
-    # buffer sets (each with its own HotPath) let step k+1's upload and step k-1's download
-    # run on their own streams while step k computes; a set is reused only after its inputs
-    # were consumed and its Y was read back (events).
-    W_h = torch.from_numpy(w.W_bits.view(np.int16)).pin_memory()
-    X_h = torch.from_numpy(w.X_bits.view(np.int16)).pin_memory()
-    P_h = torch.from_numpy(w.perm).pin_memory()
-    sets = []
-    for b in range(2):
-        hp_b = hp if b == 0 else H.HotPath(M, K, N, T, w.t_s, w.alpha, device=dev)
-        sets.append(dict(hp=hp_b, W=torch.empty_like(W), X=torch.empty_like(X),
-                         P=torch.empty_like(perm),
-                         Y=torch.empty((M, N), dtype=torch.float32).pin_memory(),
-                         consumed=torch.cuda.Event(), read=torch.cuda.Event(),
-                         loaded=torch.cuda.Event()))
-    s_up, s_comp, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    for st in sets:  # both sets start free
-        st["consumed"].record(s_comp)
-        st["read"].record(s_down)
-
-    def e2e_step(k):
-        st = sets[k % 2]
-        s_up.wait_event(st["consumed"])
-        with torch.cuda.stream(s_up):
-            st["W"].view(torch.int16).copy_(W_h, non_blocking=True)
-            st["X"].view(torch.int16).copy_(X_h, non_blocking=True)
-            st["P"].copy_(P_h, non_blocking=True)
-        st["loaded"].record(s_up)
-        s_comp.wait_event(st["loaded"])
-        s_comp.wait_event(st["read"])
-        with torch.cuda.stream(s_comp):
-            st["hp"].run(st["W"], st["X"], st["P"], fixed_counts=fixed, stream=s_comp,
-                         tile_pairs=tile_pairs)
-        st["consumed"].record(s_comp)
-        s_down.wait_event(st["consumed"])
-        with torch.cuda.stream(s_down):
-            st["Y"].copy_(st["hp"].Y, non_blocking=True)
-        st["read"].record(s_down)
-
-    for k in range(2):
-        e2e_step(k)
-    torch.cuda.synchronize()
-    e_start = torch.cuda.Event(enable_timing=True)
-    e_end = torch.cuda.Event(enable_timing=True)
+    # Every step copies this rank's inputs in from pinned host memory (its rows of W, all of
+    # X, the permutation) and its rows of Y out.  Two device buffer sets (each with its own
+    # HotPath) let step k+1's upload and step k-1's download run on their own streams while
+    # step k computes: the figure is the pipelined steady-state throughput, not the latency
+    # of one call.
+    r0, r1 = rows
+    Ms = r1 - r0
     e2e_steps = max(4, min(args.steps, 10))
-    if dist:
+    h2d = d2h = 0
+    t_e2e = 0.0
+    if have:
+        W_h = torch.from_numpy(np.ascontiguousarray(w.W_bits[r0:r1]).view(np.int16)).pin_memory()
+        X_h = torch.from_numpy(w.X_bits.view(np.int16)).pin_memory()
+        P_h = torch.from_numpy(w.perm).pin_memory()
+        hp0 = m["hp"]
+        sets = []
+        for b in range(2):
+            hp_b = hp0 if b == 0 else H.HotPath(Ms, K, N, T, w.t_s, w.alpha, device=dev)
+            sets.append(dict(hp=hp_b, W=torch.empty_like(m["W"]), X=torch.empty_like(m["X"]),
+                             P=torch.empty_like(m["perm"]),
+                             Y=torch.empty((Ms, N), dtype=torch.float32).pin_memory(),
+                             consumed=torch.cuda.Event(), read=torch.cuda.Event(),
+                             loaded=torch.cuda.Event()))
+        s_up, s_comp, s_down = (torch.cuda.Stream(dev), torch.cuda.Stream(dev),
+                                torch.cuda.Stream(dev))
+        for st in sets:  # both sets start free
+            st["consumed"].record(s_comp)
+            st["read"].record(s_down)
+
+        def e2e_step(k):
+            st = sets[k % 2]
+            s_up.wait_event(st["consumed"])
+            with torch.cuda.stream(s_up):
+                st["W"].view(torch.int16).copy_(W_h, non_blocking=True)
+                st["X"].view(torch.int16).copy_(X_h, non_blocking=True)
+                st["P"].copy_(P_h, non_blocking=True)
+            st["loaded"].record(s_up)
+            s_comp.wait_event(st["loaded"])
+            s_comp.wait_event(st["read"])
+            with torch.cuda.stream(s_comp):
+                st["hp"].run(st["W"], st["X"], st["P"], fixed_counts=m["fixed"], stream=s_comp,
+                             tile_pairs=m["tile_pairs"])
+            st["consumed"].record(s_comp)
+            s_down.wait_event(st["consumed"])
+            with torch.cuda.stream(s_down):
+                st["Y"].copy_(st["hp"].Y, non_blocking=True)
+            st["read"].record(s_down)
+
+        for k in range(2):
+            e2e_step(k)
+        torch.cuda.synchronize()
+        e_start = torch.cuda.Event(enable_timing=True)
+        e_end = torch.cuda.Event(enable_timing=True)
+        if dist:
+            dist.barrier()
+        e_start.record(s_up)
+        for k in range(e2e_steps):
+            e2e_step(k)
+        e_end.record(s_down)
+        torch.cuda.synchronize()
+        t_e2e = e_start.elapsed_time(e_end) * 1e-3 / e2e_steps
+        h2d = W_h.numel() * 2 + X_h.numel() * 2 + P_h.numel() * 4
+        d2h = sets[0]["Y"].numel() * 4
+        # the e2e outputs must match the device-resident path
+        for st in sets:
+            assert torch.equal(st["Y"], hp0.Y.cpu())
+    elif dist:
         dist.barrier()
-    e_start.record(s_up)
-    for k in range(e2e_steps):
-        e2e_step(k)
-    e_end.record(s_down)
-    torch.cuda.synchronize()
-    t_e2e = e_start.elapsed_time(e_end) * 1e-3 / e2e_steps
     t_e2e = max_over_ranks(t_e2e, dist, dev)
-    h2d = W_h.numel() * 2 + X_h.numel() * 2 + P_h.numel() * 4
-    d2h = sets[0]["Y"].numel() * 4
-    # the e2e outputs must match the device-resident path
-    for st in sets:
-        assert torch.equal(st["Y"], hp.Y.cpu())
+    launches = m["launches_per_step"]
 
     if dist:
         dist.destroy_process_group()
@@ -645,77 +803,93 @@ def main():
         return 0
 
     peaks, peak_kind = load_peaks()
-    mean_phase = {p: statistics.mean(v) for p, v in per_phase.items()}
+    counts = m["counts"]
+    Ms0 = rows[1] - rows[0]
+    model = workload_model(Ms0, K, N, T, counts)
     kernels = {}
-    for p in phases:
-        bound, ach, pk, unit, frac = roofline_for(p, mean_phase[p], model, peaks, peak_kind)
-        kernels[p] = {"ms": mean_phase[p] * 1e3, "bound": bound, "achieved": ach, "peak": pk,
+    for p, t in m["per_phase"].items():
+        bound, ach, pk, unit, frac = roofline_for(p, t, model, peaks, peak_kind)
+        kernels[p] = {"ms": t * 1e3, "bound": bound, "achieved": ach, "peak": pk,
                       "unit": unit, "frac": frac}
-    # The roofline line is the SpMM kernel's: the metric is its throughput, and it is one
-    # kernel launch per step (the other phases are several kernels each; they are listed
-    # in "kernels" with their own rooflines).
-    dom = "spmm"
-    spmm_name = "spmm_pair_kernel" if (tile_pairs and T == 128 and N >= 1024) else "spmm_kernel"
-    traffic = None  # per launch, from an ncu capture of this kernel on this workload
-    tr_path = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tr_path):
-        traffic = json.load(open(tr_path)).get(w.name, {}).get(spmm_name)
-    roof = {"bound": kernels[dom]["bound"], "achieved": kernels[dom]["achieved"],
-            "peak": kernels[dom]["peak"], "unit": kernels[dom]["unit"],
-            "frac": kernels[dom]["frac"], "traffic": traffic, "kernel": spmm_name,
-            "longest_phase": max(phases, key=lambda p: mean_phase[p]),
-            "peak_source": f"{peak_kind} (MEASURED_PEAKS.json burst; 2:4 = 2x dense bf16)"}
-    spmm_t = mean_phase["spmm"]
+    spmm_t = m["per_phase"]["spmm"]
+    name0, _ = spmm_plan(N, T, m["tile_pairs"])
+    _, roof = spmm_roofline(Ms0, K, N, T, counts, m["tile_pairs"], spmm_t, peaks, peak_kind,
+                            traffic_for(w.name, name0.split("<")[0]))
+    roof["longest_phase"] = max(m["per_phase"], key=lambda p: m["per_phase"][p])
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         from threadpoolctl import threadpool_limits
         cores = cpu_cores()
         with threadpool_limits(limits=cores):
-            dt, fl = cpu_oracle_sample(w, 8)
+            dt, fl = cpu_oracle_sample(w, 4)
         cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
-               "sample": f"8 of {M // T} tiles (1024 output rows) of {w.name}: channel energies, "
-                         "importance, search, mask, compress and fp64 masked product",
+               "sample": f"4 of {M // T} tiles ({4 * T} output rows) of {w.name}: channel "
+                         "energies, importance, search, mask, compress and fp64 masked product",
                "seconds": dt}
     clocks = sampler.summary()
-    next_rows = context = None
-    if not args.no_next_rows:
+    next_rows = context = others = None
+    if world == 1 and not args.no_next_rows:
+        hp = m["hp"]
         context = time_dense_context(M, K, N, flush, stream)
         next_rows = {"index_translate": time_index_translate(H, hp, K, stream),
                      "hard_concrete": time_hard_concrete(H, M * K, peaks, stream),
-                     "epilogue_bf16": time_epilogue(H, hp, X, M, N, tile_pairs, flush, stream),
+                     "epilogue_bf16": time_epilogue(H, hp, m["X"], M, N, m["tile_pairs"], flush,
+                                                    stream),
                      "gyro_refine_host": time_gyro(H, hp, w.perm, T, K)}
-    # this library's kernels per step: importance 2 (channel energies, importance with the
-    # tile statistics), search 6 (chunk sort, merge rank, column sums, candidate lists, band
-    # sums, finalize; V comes from the importance step), mask 2 (classify with the
-    # permutation check, bitmask), compress 3 (tile offsets, lists, pack), SpMM 1; the
-    # memsets between them are not counted
-    kernels_per_step = 2 + 6 + 2 + 3 + 1
+    if world == 1 and not args.no_other_configs:
+        others = {}
+        for oname in ("pure24", "decode"):
+            if oname == args.workload:
+                continue
+            wo = WORKLOADS[oname]()
+            mo = measure(H, wo, args, dev, flush, stream)
+            so = mo["per_phase"]["spmm"]
+            cn, _ = spmm_plan(wo.N, wo.T, mo["tile_pairs"])
+            _, ro = spmm_roofline(wo.M, wo.K, wo.N, wo.T, mo["counts"], mo["tile_pairs"], so,
+                                  peaks, peak_kind, traffic_for(wo.name, cn.split("<")[0]))
+            others[wo.name] = {
+                "ms_per_step": mo["t_step"] * 1e3,
+                "value": job_value(2.0 * wo.M * wo.K * wo.N, mo["t_step"]), "unit": UNIT,
+                "phases_ms": {p: t * 1e3 for p, t in mo["per_phase"].items()},
+                "spmm_ms": so * 1e3, "roofline": ro,
+                "launches_per_step": mo["launches_per_step"],
+                "config": {"M": wo.M, "K": wo.K, "N": wo.N, "T": wo.T, "t_s": wo.t_s,
+                           "v_s_used": wo.v_s, "counts_tile0": mo["counts"][0].tolist()}}
+            del mo
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True,
-        "ms_per_step_eager": t_eager * 1e3,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "ms_per_step_eager": m["t_eager"] * 1e3,
+        "scaling": "strong" if world > 1 else "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
         "config": {"workload": w.name, "M": M, "K": K, "N": N, "T": T, "t_s": w.t_s,
-                   "alpha": w.alpha, "v_s_searched": sorted(set(np.round(vs, 6).tolist())),
+                   "alpha": w.alpha, "v_s_searched": sorted(set(np.round(m["vs"], 6).tolist())),
                    "v_s_used": w.v_s if w.v_s is not None else "searched",
                    "counts_tile0": counts[0].tolist(),
                    "l2": "flushed between timed steps (256 MB write)",
                    "step": "importance+search+mask+compress+spmm",
                    "step_exec": "CUDA graph replay of the five calls (phase times: eager pass)",
-                   "parallelism": f"{world} independent shard(s), no collective"},
+                   "parallelism": (f"tiles sharded over {world} GPUs, X replicated"
+                                   + (", Y all-gathered (NCCL) every step" if args.gather_y
+                                      else ", each rank keeps its rows of Y"))
+                   if world > 1 else "1 GPU",
+                   "rank0_rows": list(rows)},
         "spmm_only": {"ms": spmm_t * 1e3, "tflops_eff": model["flops_eff"] / spmm_t / 1e12,
                       "tflops_actual": model["flops_actual"] / spmm_t / 1e12,
                       "gbs": model["bytes"]["spmm"] / spmm_t / 1e9},
         "kernels": kernels,
         "roofline": roof,
         "cpu_baseline": cpu,
-        "e2e": {"value": job_value(model["flops_eff"], world, t_e2e), "unit": UNIT,
+        "e2e": {"value": job_value(2.0 * M * K * N, t_e2e), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": t_e2e * 1e3,
-                "pipelining": "two buffer sets; upload, compute and download on their own "
-                              "streams"},
-        "gpu_launches": kernels_per_step * args.steps,
-        "gpu_launches_phase_pass": kernels_per_step * args.steps,
+                "kind": "pipelined steady-state throughput through the public API (two buffer "
+                        "sets; upload, compute and download on their own streams)"},
+        "gpu_launches": (launches * args.steps) if launches is not None else None,
+        "gpu_launches_counted": "kernel nodes of the captured step graph (CUDA runtime) x "
+                                "timed replays, rank 0",
+        "kernels_in_step": m["kernel_names"],
+        "other_configs": others,
         "next_rows": next_rows,
         "context": context,
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],

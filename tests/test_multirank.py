@@ -1,6 +1,7 @@
-"""The multi-rank plumbing of bench.py on CPU: two gloo ranks, each with its own seeded shard
-of the same shape (weak scaling, no data-path collective), the job time taken as the max over
-ranks, and the reference arm printing on rank 0 only."""
+"""The multi-rank plumbing of bench.py on CPU (gloo ranks): every rank draws the same problem
+and takes its tiles of it, the job time is the max over ranks and the job value the whole
+problem's FLOPs over it, the reference arm prints on rank 0 only; and the tile-sharded split
+itself (ranges, and the per-rank results against the unsharded run)."""
 import contextlib
 import datetime
 import hashlib
@@ -31,11 +32,11 @@ def _worker(rank, world, port, q):
     import bench
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=60))
-    w = bench.WORKLOADS["tiny"](rank)
+    w = bench.WORKLOADS["tiny"]()
     digest = hashlib.sha256(w.W_bits.tobytes() + w.X_bits.tobytes()).hexdigest()
     t_local = 0.001 * (rank + 1)
     t_max = bench.max_over_ranks(t_local, dist, torch.device("cpu"))
-    value = bench.job_value(2.0 * w.M * w.K * w.N, world, t_max)
+    value = bench.job_value(2.0 * w.M * w.K * w.N, t_max)
     dist.barrier()
     dist.destroy_process_group()
     # the reference arm: rank 0 prints one JSON line, the others exit 0 without work
@@ -46,7 +47,7 @@ def _worker(rank, world, port, q):
     q.put((rank, t_max, value, digest, (w.M, w.K, w.N, w.T), rc, out.getvalue()))
 
 
-def test_two_gloo_ranks_shards_max_timing_and_reference_arm():
+def test_two_gloo_ranks_same_problem_max_timing_and_reference_arm():
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
@@ -68,9 +69,8 @@ def test_two_gloo_ranks_shards_max_timing_and_reference_arm():
     assert r0[1] == r1[1] == pytest.approx(0.002)          # max over ranks, seen by both
     assert r0[2] == r1[2]                                    # same job value on every rank
     M, K, N, T = r0[4]
-    assert r0[2] == pytest.approx(2 * (2.0 * M * K * N) / 0.002 / 1e12)
-    assert r0[4] == r1[4]                                    # same shape (weak scaling) ...
-    assert r0[3] != r1[3]                                    # ... different seeded shard
+    assert r0[2] == pytest.approx((2.0 * M * K * N) / 0.002 / 1e12)  # whole problem / max time
+    assert r0[4] == r1[4] and r0[3] == r1[3]                 # one problem, split by tiles
     assert r0[5] == 0 and r1[5] == 0
     import json
     line = json.loads(r0[6].strip().splitlines()[-1])
