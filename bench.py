@@ -156,9 +156,12 @@ def workload_model(M, K, N, T, counts):
     return dict(
         flops_eff=flops_eff, flops_actual=2.0 * kept * N, flops_dense=flops_dense,
         flops_sparse_eq=flops_sparse_eq, kept=kept,
-        bytes=dict(importance=2.0 * M * K + 2.0 * K * N + 4.0 * M * K + 8.0 * K,
-                   search=4.0 * M * K + 4.0 * nt * K,
-                   mask=4.0 * M * K + M * ((K + 31) // 32) * 4.0 + nt * K,
+        # the step does not materialize I: the importance pass reads W and X and writes the
+        # tile statistics (V, tile maxima, s_c); the search and the mask read W (2 B per
+        # weight) and recompute the importance from it
+        bytes=dict(importance=2.0 * M * K + 2.0 * K * N + 8.0 * nt * K + 4.0 * nt + 4.0 * K,
+                   search=2.0 * M * K + 4.0 * nt * K,
+                   mask=2.0 * M * K + M * ((K + 31) // 32) * 4.0 + nt * K,
                    compress=2.0 * M * K + M * ((K + 31) // 32) * 4.0 + nt * K
                    + 2.0 * kept + T * n24 / 8.0 + 4.0 * (n4 + n24),
                    spmm=spmm_bytes))
@@ -325,7 +328,7 @@ def time_index_translate(H, hp, K, stream, reps=20):
     back-to-back calls after 3 untimed ones.  Bytes: 4 B read + 4 B written per index entry,
     4 B read from the map per entry, 4 B written per block."""
     import torch
-    ident = torch.arange(K, dtype=torch.int32, device=hp.I.device)
+    ident = torch.arange(K, dtype=torch.int32, device=hp.counts.device)
     info = hp.layout.tile_info.cpu().numpy()
     nd, ns = int(info[:, 0].sum()), int(info[:, 1].sum())
     entries = nd * 64 + ns * 128
@@ -402,13 +405,13 @@ def time_dense_context(M, K, N, flush, stream, reps=10):
             "note": "dense W (no pruning) through cuBLAS, same M, K, N; context only"}
 
 
-def time_gyro(H, hp, perm, T, K, G=16, k=2, rounds=4):
+def time_gyro(H, hp, W, X, perm, T, K, G=16, k=2, rounds=4):
     """The library's in-tile gyro rounds (host) on tile 0 of this step: its importance rows,
     its 2:4 band in working order (from the step's regions), `rounds` rounds of G sampled
     groups x k slots (seeded draws); wall-clock time on one host core, and the band's
     pruning cost before and after."""
     import time
-    I_tile = hp.I[:T].cpu().numpy()
+    I_tile = H.hinm_importance(W[:T], X).cpu().numpy()
     region0 = hp.region[0].cpu().numpy()
     band = np.array([c for c in perm if region0[c] == 1], dtype=np.int32)
     ng = band.size // 4
@@ -534,7 +537,8 @@ def measure(H, w, args, dev, flush, stream, rows=None, dist=None, sampler=None):
         W = torch.from_numpy(np.ascontiguousarray(w.W_bits[r0:r1]).view(np.int16)).to(dev).view(torch.bfloat16)
         X = torch.from_numpy(w.X_bits.view(np.int16)).to(dev).view(torch.bfloat16)
         perm = torch.from_numpy(w.perm).to(dev)
-        hp = H.HotPath(Ms, K, N, T, w.t_s, w.alpha, device=dev)
+        # the importance is not materialized: the search and the mask recompute it from W
+        hp = H.HotPath(Ms, K, N, T, w.t_s, w.alpha, device=dev, materialize_importance=False)
         # Workloads specified with a fixed boundary v_s use its closed-form counts; the search
         # still runs every step (its ranking feeds the mask).  Otherwise the search's counts.
         fixed = c = None
@@ -549,14 +553,15 @@ def measure(H, w, args, dev, flush, stream, rows=None, dist=None, sampler=None):
         def step(ev=None):
             if ev is not None:
                 ev[0].record(stream)
-            H.hinm_importance_stats(W, X, T, hp.I, hp.stats, hp.ws)
+            H.hinm_importance_stats(W, X, T, None, hp.stats, hp.ws, materialize=False)
             if ev is not None:
                 ev[1].record(stream)
-            H.hinm_boundary_search(hp.I, perm, T, w.t_s, w.alpha, hp.counts, hp.vs, hp.rank,
-                                   hp.ws, stats=hp.stats)
+            H.hinm_boundary_search(None, perm, T, w.t_s, w.alpha, hp.counts, hp.vs, hp.rank,
+                                   hp.ws, stats=hp.stats, W=W)
             if ev is not None:
                 ev[2].record(stream)
-            H.hinm_mask(hp.I, perm, counts_used, T, hp.rank, hp.bitmask, hp.region, hp.ws)
+            H.hinm_mask(None, perm, counts_used, T, hp.rank, hp.bitmask, hp.region, hp.ws,
+                        W=W, stats=hp.stats)
             if ev is not None:
                 ev[3].record(stream)
             H.hinm_compress(W, hp.bitmask, hp.region, perm, counts_used, T, hp.layout, hp.ws)
@@ -743,7 +748,8 @@ def main():
         hp0 = m["hp"]
         sets = []
         for b in range(2):
-            hp_b = hp0 if b == 0 else H.HotPath(Ms, K, N, T, w.t_s, w.alpha, device=dev)
+            hp_b = hp0 if b == 0 else H.HotPath(Ms, K, N, T, w.t_s, w.alpha, device=dev,
+                                                materialize_importance=False)
             sets.append(dict(hp=hp_b, W=torch.empty_like(m["W"]), X=torch.empty_like(m["X"]),
                              P=torch.empty_like(m["perm"]),
                              Y=torch.empty((Ms, N), dtype=torch.float32).pin_memory(),
@@ -835,7 +841,7 @@ def main():
                      "hard_concrete": time_hard_concrete(H, M * K, peaks, stream),
                      "epilogue_bf16": time_epilogue(H, hp, m["X"], M, N, m["tile_pairs"], flush,
                                                     stream),
-                     "gyro_refine_host": time_gyro(H, hp, w.perm, T, K)}
+                     "gyro_refine_host": time_gyro(H, hp, m["W"], m["X"], w.perm, T, K)}
     if world == 1 and not args.no_other_configs:
         others = {}
         for oname in ("pure24", "decode"):
@@ -868,6 +874,8 @@ def main():
                    "counts_tile0": counts[0].tolist(),
                    "l2": "flushed between timed steps (256 MB write)",
                    "step": "importance+search+mask+compress+spmm",
+                   "importance": "not materialized: the search and the mask recompute it from "
+                                 "W and the channel energies (the same bits)",
                    "step_exec": "CUDA graph replay of the five calls (phase times: eager pass)",
                    "parallelism": (f"tiles sharded over {world} GPUs, X replicated"
                                    + (", Y all-gathered (NCCL) every step" if args.gather_y

@@ -108,10 +108,12 @@ hinm_status hinm_importance_noalloc(const void* W, const void* X, int M, int K, 
 /* Importance with the boundary search's tile statistics made in the same pass.  The
  * method's description has no counterpart: the statistics are the search's own first step
  * (a2 below), computed here while I is written so that the search does not read I for them.
- *   I_out: as hinm_importance (bit for bit).  stats_out (device, hinm_tile_stats_size()
- *   bytes, caller-owned): V[t][c] = sum over the tile's rows (ascending, fp64) of I[row, c]
- *   by input channel c, and each tile's largest importance; an opaque layout that only
- *   hinm_boundary_search_stats reads.  T as for the search (64 or 128).
+ *   I_out: as hinm_importance (bit for bit), or NULL: I is then not written (the _ex search
+ *   and mask recompute it from W and these statistics).  stats_out (device,
+ *   hinm_tile_stats_size() bytes, caller-owned): V[t][c] = sum over the tile's rows
+ *   (ascending, fp64) of I[row, c] by input channel c, each tile's largest importance and
+ *   the channel energies s_c; an opaque layout that only the search and the mask read.
+ *   The workspace is not used (it may be NULL).  T as for the search (64 or 128).
  *   Errors: as hinm_importance, plus HINM_ERR_SHAPE for T, HINM_ERR_INVALID_ARG for a NULL
  *   or too small stats_out. */
 hinm_status hinm_tile_stats_size(int M, int K, int T, size_t* bytes_host);
@@ -240,16 +242,23 @@ hinm_status hinm_compress(const void* W, const uint32_t* bitmask, const int8_t* 
  * the tile's 2:4 groups are 4 consecutive 2:4 channels in that order, and compress folds
  * perm[t] into tile t's index, so the SpMM needs nothing else.  The same perm and flag must
  * be given to the three calls.  Other arguments, results and errors as the calls above;
- * hinm_boundary_search_ex covers both search forms (stats may be NULL). */
-hinm_status hinm_boundary_search_ex(const float* I, const void* stats, size_t stats_bytes,
-                                    const int32_t* perm, int perm_per_tile, int M, int K, int T,
-                                    double t_s, double alpha, int32_t* counts_out, double* vs_out,
-                                    int32_t* rank_out, double* retained_out, void* workspace,
+ * hinm_boundary_search_ex covers both search forms (stats may be NULL).
+ * The importance need not be materialized: with I NULL, the search and the mask recompute
+ * every value they read from W (device bf16 [M][K]) and the channel energies that
+ * hinm_importance_stats stored in `stats` (for this W, X and T), as fl32(fl32(w^2) s_c) --
+ * the same bits as I -- reading 2 bytes per weight instead of 4.  With I given, W may be
+ * NULL.  Errors: HINM_ERR_INVALID_ARG for I NULL without W and stats. */
+hinm_status hinm_boundary_search_ex(const float* I, const void* W, const void* stats,
+                                    size_t stats_bytes, const int32_t* perm, int perm_per_tile,
+                                    int M, int K, int T, double t_s, double alpha,
+                                    int32_t* counts_out, double* vs_out, int32_t* rank_out,
+                                    double* retained_out, void* workspace,
                                     size_t workspace_bytes, void* stream);
-hinm_status hinm_mask_ex(const float* I, const int32_t* perm, int perm_per_tile,
-                         const int32_t* counts, const int32_t* rank, int M, int K, int T,
-                         uint32_t* bitmask_out, int8_t* region_out, void* workspace,
-                         size_t workspace_bytes, void* stream);
+hinm_status hinm_mask_ex(const float* I, const void* W, const void* stats, size_t stats_bytes,
+                         const int32_t* perm, int perm_per_tile, const int32_t* counts,
+                         const int32_t* rank, int M, int K, int T, uint32_t* bitmask_out,
+                         int8_t* region_out, void* workspace, size_t workspace_bytes,
+                         void* stream);
 hinm_status hinm_compress_ex(const void* W, const uint32_t* bitmask, const int8_t* region,
                              const int32_t* perm, int perm_per_tile, const int32_t* counts,
                              int M, int K, int T, const hinm_layout* layout, void* workspace,

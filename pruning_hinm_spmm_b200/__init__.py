@@ -75,9 +75,10 @@ _SIGS = {
     "hinm_search_workspace_size": (_i32, [_i32, _i32, _i32, _f64, _f64, _szp]),
     "hinm_boundary_search": (_i32, [_vp, _vp, _i32, _i32, _i32, _f64, _f64, _vp, _vp, _vp, _vp,
                                     _vp, _sz, _vp]),
-    "hinm_boundary_search_ex": (_i32, [_vp, _vp, _sz, _vp, _i32, _i32, _i32, _i32, _f64, _f64, _vp,
-                                       _vp, _vp, _vp, _vp, _sz, _vp]),
-    "hinm_mask_ex": (_i32, [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "hinm_boundary_search_ex": (_i32, [_vp, _vp, _vp, _sz, _vp, _i32, _i32, _i32, _i32, _f64, _f64,
+                                       _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "hinm_mask_ex": (_i32, [_vp, _vp, _vp, _sz, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _vp, _vp,
+                            _vp, _sz, _vp]),
     "hinm_compress_ex": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32,
                                 ctypes.POINTER(hinm_layout), _vp, _sz, _vp]),
     "hinm_mask_workspace_size": (_i32, [_i32, _i32, _i32, _szp]),
@@ -175,14 +176,17 @@ def hinm_tile_stats_size(M: int, K: int, T: int) -> int:
     return _size(_lib.hinm_tile_stats_size, M, K, T)
 
 
-def hinm_importance_stats(W, X, T: int, I_out=None, stats_out=None, workspace=None, stream=None):
-    """hinm_importance that also writes the boundary search's tile statistics (V and the
-    tile maxima) in the same pass.  Returns (I, stats); stats is an opaque uint8 buffer for
-    hinm_boundary_search(..., stats=stats)."""
+def hinm_importance_stats(W, X, T: int, I_out=None, stats_out=None, workspace=None, stream=None,
+                          materialize: bool = True):
+    """hinm_importance that also writes the boundary search's tile statistics (V, the tile
+    maxima and the channel energies) in the same pass.  Returns (I, stats); stats is an
+    opaque uint8 buffer for hinm_boundary_search / hinm_mask (..., stats=stats).  With
+    materialize=False I is not written (returned as None): the search and the mask then
+    recompute it from W and stats."""
     torch = _torch()
     M, K = W.shape
     N = X.shape[1]
-    if I_out is None:
+    if I_out is None and materialize:
         I_out = torch.empty((M, K), dtype=torch.float32, device=W.device)
     if stats_out is None:
         stats_out = _empty_bytes(hinm_tile_stats_size(M, K, T), W.device)
@@ -242,16 +246,17 @@ def hinm_search_num_candidates(K: int, t_s: float, alpha: float = 1.0 / 32.0) ->
 
 def hinm_boundary_search(I, perm, T: int, t_s: float, alpha: float = 1.0 / 32.0,
                          counts_out=None, vs_out=None, rank_out=None, workspace=None,
-                         want_rank: bool = True, retained_out=None, stream=None, stats=None):
+                         want_rank: bool = True, retained_out=None, stream=None, stats=None,
+                         W=None):
     """Per-tile first-drop scan of v_s.  Returns (counts int32 [M/T,3], v_s fp64 [M/T], rank).
     ``retained_out`` (fp64 [M/T, n_cand]) optionally receives R(m) of every candidate;
     ``stats`` (from hinm_importance_stats for this I and T) spares the search its pass over
     I for V.  ``perm``: int32 [K] (every tile) or [M/T, K] (one working order per tile), or
-    None (identity)."""
+    None (identity).  I may be None when W and stats are given (I recomputed from them)."""
     torch = _torch()
-    M, K = I.shape
+    M, K = (I if I is not None else W).shape
     nt = M // T
-    dev = I.device
+    dev = (I if I is not None else W).device
     if counts_out is None:
         counts_out = torch.empty((nt, 3), dtype=torch.int32, device=dev)
     if vs_out is None:
@@ -260,7 +265,8 @@ def hinm_boundary_search(I, perm, T: int, t_s: float, alpha: float = 1.0 / 32.0,
         rank_out = torch.empty((nt, K), dtype=torch.int32, device=dev)
     if workspace is None:
         workspace = _empty_bytes(hinm_search_workspace_size(M, K, T, t_s, alpha), dev)
-    _check(_lib.hinm_boundary_search_ex(_ptr(I), _ptr(stats), 0 if stats is None else stats.numel(),
+    _check(_lib.hinm_boundary_search_ex(_ptr(I), _ptr(W), _ptr(stats),
+                                        0 if stats is None else stats.numel(),
                                         _ptr(perm), _per_tile(perm), M, K, T, t_s, alpha,
                                         _ptr(counts_out), _ptr(vs_out), _ptr(rank_out),
                                         _ptr(retained_out), _ptr(workspace), workspace.numel(),
@@ -274,11 +280,12 @@ def hinm_mask_workspace_size(M, K, T) -> int:
 
 
 def hinm_mask(I, perm, counts, T: int, rank=None, bitmask_out=None, region_out=None,
-              workspace=None, stream=None):
-    """Bit-packed mask uint32 [M, ceil(K/32)] (as int32) and region int8 [M/T, K]."""
+              workspace=None, stream=None, W=None, stats=None):
+    """Bit-packed mask uint32 [M, ceil(K/32)] (as int32) and region int8 [M/T, K].  I may be
+    None when W and stats (from hinm_importance_stats) are given."""
     torch = _torch()
-    M, K = I.shape
-    dev = I.device
+    M, K = (I if I is not None else W).shape
+    dev = (I if I is not None else W).device
     words = (K + 31) // 32
     if bitmask_out is None:
         bitmask_out = torch.empty((M, words), dtype=torch.int32, device=dev)
@@ -286,8 +293,9 @@ def hinm_mask(I, perm, counts, T: int, rank=None, bitmask_out=None, region_out=N
         region_out = torch.empty((M // T, K), dtype=torch.int8, device=dev)
     if workspace is None:
         workspace = _empty_bytes(hinm_mask_workspace_size(M, K, T), dev)
-    _check(_lib.hinm_mask_ex(_ptr(I), _ptr(perm), _per_tile(perm), _ptr(counts), _ptr(rank), M,
-                             K, T, _ptr(bitmask_out), _ptr(region_out), _ptr(workspace),
+    _check(_lib.hinm_mask_ex(_ptr(I), _ptr(W), _ptr(stats), 0 if stats is None else stats.numel(),
+                             _ptr(perm), _per_tile(perm), _ptr(counts), _ptr(rank), M, K, T,
+                             _ptr(bitmask_out), _ptr(region_out), _ptr(workspace),
                              workspace.numel(), _stream(stream)), "hinm_mask_ex")
     return bitmask_out, region_out
 
@@ -559,11 +567,14 @@ class HotPath:
     problem shape; run() enqueues the five steps on the current stream with no host sync."""
 
     def __init__(self, M: int, K: int, N: int, T: int, t_s: float, alpha: float = 1.0 / 32.0,
-                 device="cuda"):
+                 device="cuda", materialize_importance: bool = True):
         torch = _torch()
         self.M, self.K, self.N, self.T, self.t_s, self.alpha = M, K, N, T, t_s, alpha
         nt = M // T
-        self.I = torch.empty((M, K), dtype=torch.float32, device=device)
+        # materialize_importance=False: I is never written; the search and the mask recompute
+        # it from W and the tile statistics (half the bytes per weight)
+        self.I = (torch.empty((M, K), dtype=torch.float32, device=device)
+                  if materialize_importance else None)
         self.counts = torch.empty((nt, 3), dtype=torch.int32, device=device)
         self.vs = torch.empty((nt,), dtype=torch.float64, device=device)
         self.rank = torch.empty((nt, K), dtype=torch.int32, device=device)
@@ -582,12 +593,13 @@ class HotPath:
         """One pass of the path.  The search always runs (its ranking feeds the mask);
         ``fixed_counts`` (int32 [M/T, 3]) replaces its counts when given; ``tile_pairs`` is
         the SpMM hint (hinm_spmm)."""
-        hinm_importance_stats(W, X, self.T, self.I, self.stats, self.ws, stream)
+        hinm_importance_stats(W, X, self.T, self.I, self.stats, self.ws, stream,
+                              materialize=self.I is not None)
         hinm_boundary_search(self.I, perm, self.T, self.t_s, self.alpha, self.counts, self.vs,
-                             self.rank, self.ws, stream=stream, stats=self.stats)
+                             self.rank, self.ws, stream=stream, stats=self.stats, W=W)
         counts = self.counts if fixed_counts is None else fixed_counts
         hinm_mask(self.I, perm, counts, self.T, self.rank, self.bitmask, self.region, self.ws,
-                  stream)
+                  stream, W=W, stats=self.stats)
         hinm_compress(W, self.bitmask, self.region, perm, counts, self.T, self.layout, self.ws,
                       stream)
         hinm_spmm(self.layout, X, self.Y, stream, self.c_layout, tile_pairs)

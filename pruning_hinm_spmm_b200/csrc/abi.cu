@@ -182,6 +182,7 @@ namespace {
 struct SmemAttr {
   int dev;
   const void* fn;
+  int bytes;  // the largest limit set so far
 };
 std::mutex g_attr_mu;
 SmemAttr g_attr_done[1024];
@@ -193,12 +194,15 @@ cudaError_t set_max_dynamic_smem(const void* fn, int bytes) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lk(g_attr_mu);
+  int slot = -1;
   for (int i = 0; i < g_attr_count; ++i)
-    if (g_attr_done[i].dev == dev && g_attr_done[i].fn == fn) return cudaSuccess;
+    if (g_attr_done[i].dev == dev && g_attr_done[i].fn == fn) slot = i;
+  if (slot >= 0 && g_attr_done[slot].bytes >= bytes) return cudaSuccess;
   e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
-  if (g_attr_count < (int)(sizeof(g_attr_done) / sizeof(g_attr_done[0])))
-    g_attr_done[g_attr_count++] = SmemAttr{dev, fn};
+  if (slot >= 0) g_attr_done[slot].bytes = bytes;
+  else if (g_attr_count < (int)(sizeof(g_attr_done) / sizeof(g_attr_done[0])))
+    g_attr_done[g_attr_count++] = SmemAttr{dev, fn, bytes};
   return cudaSuccess;
 }
 
@@ -283,7 +287,7 @@ hinm_status hinm_importance_stats(const void* W, const void* X, int M, int K, in
                                   void* workspace, size_t workspace_bytes, void* stream) {
   REQUIRE_PTR(W);
   REQUIRE_PTR(X);
-  REQUIRE_PTR(I_out);
+  REQUIRE_ALIGNED_OR_NULL(I_out);
   REQUIRE_PTR(stats_out);
   hinm_status st = check_mkt(M, K, T);
   if (st != HINM_OK) return st;
@@ -292,13 +296,11 @@ hinm_status hinm_importance_stats(const void* W, const void* X, int M, int K, in
   if (stats_bytes < hinm::tile_stats_bytes(M, K, T))
     return fail(HINM_ERR_INVALID_ARG, "stats %zu bytes, need %zu", stats_bytes,
                 hinm::tile_stats_bytes(M, K, T));
-  const size_t need = hinm::importance_workspace_bytes(K);
-  if (!workspace || workspace_bytes < need)
-    return fail(HINM_ERR_WORKSPACE, "workspace %zu bytes, need %zu", workspace_bytes, need);
-  REQUIRE_PTR(workspace);
+  (void)workspace;  // the channel energies live in stats_out
+  (void)workspace_bytes;
   cudaError_t e = hinm::launch_importance_stats(
       static_cast<const uint16_t*>(W), static_cast<const uint16_t*>(X), M, K, N, T, I_out,
-      stats_out, static_cast<float*>(workspace), static_cast<cudaStream_t>(stream));
+      stats_out, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "hinm_importance_stats launch");
   return ok();
 }
@@ -353,13 +355,28 @@ hinm_status hinm_search_workspace_size(int M, int K, int T, double t_s, double a
 namespace {
 
 // hinm_boundary_search(_stats): stats (with its size) or nullptr
-hinm_status search_impl(const float* I, const void* stats, size_t stats_bytes,
+// The importance as the search and the mask read it: I, or W with the channel energies that
+// hinm_importance_stats stored in the statistics.
+hinm::ImpSrc imp_src(const float* I, const void* W, const void* stats, int M, int K, int T) {
+  hinm::ImpSrc q{I, nullptr, nullptr};
+  if (!I) {
+    q.W = static_cast<const uint16_t*>(W);
+    q.s = reinterpret_cast<const float*>(static_cast<const char*>(stats) +
+                                         hinm::tile_stats_s_offset(M, K, T));
+  }
+  return q;
+}
+
+hinm_status search_impl(const float* I, const void* W, const void* stats, size_t stats_bytes,
                         const int32_t* perm, int perm_per_tile, int M, int K, int T, double t_s,
                         double alpha,
                         int32_t* counts_out, double* vs_out, int32_t* rank_out,
                         double* retained_out, void* workspace, size_t workspace_bytes,
                         void* stream) {
-  REQUIRE_PTR(I);
+  REQUIRE_ALIGNED_OR_NULL(I);
+  REQUIRE_ALIGNED_OR_NULL(W);
+  if (!I && (!W || !stats))
+    return fail(HINM_ERR_INVALID_ARG, "I is NULL: W and stats are needed to recompute it");
   REQUIRE_ALIGNED_OR_NULL(perm);
   REQUIRE_PTR(counts_out);
   REQUIRE_PTR(vs_out);
@@ -385,7 +402,8 @@ hinm_status search_impl(const float* I, const void* stats, size_t stats_bytes,
   REQUIRE_PTR(workspace);
   if (perm_per_tile != 0 && perm_per_tile != 1)
     return fail(HINM_ERR_INVALID_ARG, "perm_per_tile=%d must be 0 or 1", perm_per_tile);
-  cudaError_t e = hinm::launch_boundary_search(I, stats, perm, perm_per_tile ? (long long)K : 0ll,
+  const hinm::ImpSrc src = imp_src(I, W, stats, M, K, T);
+  cudaError_t e = hinm::launch_boundary_search(src, stats, perm, perm_per_tile ? (long long)K : 0ll,
                                                M, K, T, t_s, alpha, c, n,
                                                counts_out, vs_out, rank_out, retained_out,
                                                workspace, hinm::device_status_ptr(),
@@ -400,8 +418,9 @@ hinm_status hinm_boundary_search(const float* I, const int32_t* perm, int M, int
                                  double t_s, double alpha, int32_t* counts_out, double* vs_out,
                                  int32_t* rank_out, double* retained_out, void* workspace,
                                  size_t workspace_bytes, void* stream) {
-  return search_impl(I, nullptr, 0, perm, 0, M, K, T, t_s, alpha, counts_out, vs_out, rank_out,
-                     retained_out, workspace, workspace_bytes, stream);
+  REQUIRE_PTR(I);
+  return search_impl(I, nullptr, nullptr, 0, perm, 0, M, K, T, t_s, alpha, counts_out, vs_out,
+                     rank_out, retained_out, workspace, workspace_bytes, stream);
 }
 
 hinm_status hinm_boundary_search_stats(const float* I, const void* stats, size_t stats_bytes,
@@ -409,19 +428,21 @@ hinm_status hinm_boundary_search_stats(const float* I, const void* stats, size_t
                                        double alpha, int32_t* counts_out, double* vs_out,
                                        int32_t* rank_out, double* retained_out,
                                        void* workspace, size_t workspace_bytes, void* stream) {
+  REQUIRE_PTR(I);
   REQUIRE_PTR(stats);
-  return search_impl(I, stats, stats_bytes, perm, 0, M, K, T, t_s, alpha, counts_out, vs_out,
-                     rank_out, retained_out, workspace, workspace_bytes, stream);
+  return search_impl(I, nullptr, stats, stats_bytes, perm, 0, M, K, T, t_s, alpha, counts_out,
+                     vs_out, rank_out, retained_out, workspace, workspace_bytes, stream);
 }
 
-hinm_status hinm_boundary_search_ex(const float* I, const void* stats, size_t stats_bytes,
-                                    const int32_t* perm, int perm_per_tile, int M, int K, int T,
-                                    double t_s, double alpha, int32_t* counts_out, double* vs_out,
-                                    int32_t* rank_out, double* retained_out, void* workspace,
+hinm_status hinm_boundary_search_ex(const float* I, const void* W, const void* stats,
+                                    size_t stats_bytes, const int32_t* perm, int perm_per_tile,
+                                    int M, int K, int T, double t_s, double alpha,
+                                    int32_t* counts_out, double* vs_out, int32_t* rank_out,
+                                    double* retained_out, void* workspace,
                                     size_t workspace_bytes, void* stream) {
-  return search_impl(I, stats, stats ? stats_bytes : 0, perm, perm_per_tile, M, K, T, t_s, alpha,
-                     counts_out, vs_out, rank_out, retained_out, workspace, workspace_bytes,
-                     stream);
+  return search_impl(I, W, stats, stats ? stats_bytes : 0, perm, perm_per_tile, M, K, T, t_s,
+                     alpha, counts_out, vs_out, rank_out, retained_out, workspace,
+                     workspace_bytes, stream);
 }
 
 hinm_status hinm_mask_workspace_size(int M, int K, int T, size_t* bytes_host) {
@@ -436,15 +457,20 @@ hinm_status hinm_mask(const float* I, const int32_t* perm, const int32_t* counts
                       const int32_t* rank, int M, int K, int T, uint32_t* bitmask_out,
                       int8_t* region_out, void* workspace, size_t workspace_bytes,
                       void* stream) {
-  return hinm_mask_ex(I, perm, 0, counts, rank, M, K, T, bitmask_out, region_out, workspace,
-                      workspace_bytes, stream);
+  REQUIRE_PTR(I);
+  return hinm_mask_ex(I, nullptr, nullptr, 0, perm, 0, counts, rank, M, K, T, bitmask_out,
+                      region_out, workspace, workspace_bytes, stream);
 }
 
-hinm_status hinm_mask_ex(const float* I, const int32_t* perm, int perm_per_tile,
-                         const int32_t* counts, const int32_t* rank, int M, int K, int T,
-                         uint32_t* bitmask_out, int8_t* region_out, void* workspace,
-                         size_t workspace_bytes, void* stream) {
-  REQUIRE_PTR(I);
+hinm_status hinm_mask_ex(const float* I, const void* W, const void* stats, size_t stats_bytes,
+                         const int32_t* perm, int perm_per_tile, const int32_t* counts,
+                         const int32_t* rank, int M, int K, int T, uint32_t* bitmask_out,
+                         int8_t* region_out, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  REQUIRE_ALIGNED_OR_NULL(I);
+  REQUIRE_ALIGNED_OR_NULL(W);
+  if (!I && (!W || !stats))
+    return fail(HINM_ERR_INVALID_ARG, "I is NULL: W and stats are needed to recompute it");
   if (perm_per_tile != 0 && perm_per_tile != 1)
     return fail(HINM_ERR_INVALID_ARG, "perm_per_tile=%d must be 0 or 1", perm_per_tile);
   REQUIRE_ALIGNED_OR_NULL(perm);
@@ -458,7 +484,11 @@ hinm_status hinm_mask_ex(const float* I, const int32_t* perm, int perm_per_tile,
   if (!workspace || workspace_bytes < need)
     return fail(HINM_ERR_WORKSPACE, "workspace %zu bytes, need %zu", workspace_bytes, need);
   REQUIRE_PTR(workspace);
-  cudaError_t e = hinm::launch_mask(I, perm, perm_per_tile ? (long long)K : 0ll, counts, rank, M,
+  if (!I && stats_bytes < hinm::tile_stats_bytes(M, K, T))
+    return fail(HINM_ERR_INVALID_ARG, "stats %zu bytes, need %zu", stats_bytes,
+                hinm::tile_stats_bytes(M, K, T));
+  const hinm::ImpSrc src = imp_src(I, W, stats, M, K, T);
+  cudaError_t e = hinm::launch_mask(src, perm, perm_per_tile ? (long long)K : 0ll, counts, rank, M,
                                     K, T, bitmask_out, region_out,
                                     workspace, hinm::device_status_ptr(),
                                     static_cast<cudaStream_t>(stream));

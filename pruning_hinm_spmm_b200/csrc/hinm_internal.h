@@ -11,6 +11,15 @@
 
 namespace hinm {
 
+// The importance matrix as the search and the mask read it: I itself, or (I null) W and
+// the channel energies s, from which each value is recomputed bit for bit as
+// fl32(fl32(w^2) s_c) (device helpers in stage_rows.cuh).
+struct ImpSrc {
+  const float* I;
+  const uint16_t* W;
+  const float* s;
+};
+
 // Device status word codes (a subset of hinm_status) written by kernels.
 constexpr int kStatusOk = 0;
 
@@ -46,9 +55,10 @@ cudaError_t resolve_symbol(SymbolCache& c, const void* symbol, void** out);
 // Address of the library's status word on the current device (resolve_symbol).
 int* device_status_ptr();
 
-// Sets kernel `fn`'s maximum dynamic shared memory to `bytes` on the current device, once per
-// (device, kernel): the attribute belongs to the device, and a process may drive several.
-// Thread-safe; call it before the first launch on each device (and before stream capture).
+// Raises kernel `fn`'s maximum dynamic shared memory on the current device to at least
+// `bytes`, calling the runtime only when the limit grows (the attribute belongs to the device,
+// and a process may drive several).  Thread-safe; call it before the first launch on each
+// device (and before stream capture).
 cudaError_t set_max_dynamic_smem(const void* fn, int bytes);
 
 // Workspace carving helper: 256-byte aligned sub-buffers.
@@ -69,12 +79,14 @@ size_t importance_workspace_bytes(int K);
 cudaError_t launch_importance(const uint16_t* W, const uint16_t* X, int M, int K, int N,
                               float* I, float* s_scratch, cudaStream_t s);
 // Tile statistics of the boundary search made with I: V (fp64 [M/T][K], channel order) at
-// offset 0, then the tile maxima (int [M/T]) at tile_stats_v_bytes().
+// offset 0, the tile maxima (int [M/T]) at tile_stats_v_bytes(), then the channel energies
+// s_c (fp32 [K]) at tile_stats_s_offset(), from which I can be recomputed.  I may be null
+// (the importance is then not materialized).
 size_t tile_stats_v_bytes(int M, int K, int T);
+size_t tile_stats_s_offset(int M, int K, int T);
 size_t tile_stats_bytes(int M, int K, int T);
 cudaError_t launch_importance_stats(const uint16_t* W, const uint16_t* X, int M, int K, int N,
-                                    int T, float* I, void* stats, float* s_scratch,
-                                    cudaStream_t s);
+                                    int T, float* I, void* stats, cudaStream_t s);
 
 // Workspace-free variant: channel energies in a static per-device array of kNoAllocMaxK
 // floats (64 KiB).
@@ -85,14 +97,14 @@ size_t search_workspace_bytes(int M, int K, int T, int ncand);
 // perm: the working order, [K] shared by every tile (perm_stride 0) or [M/T][K] one per tile
 // (perm_stride K), or nullptr (identity).
 // stats: from launch_importance_stats for this I and T, or nullptr (computed here from I)
-cudaError_t launch_boundary_search(const float* I, const void* stats, const int32_t* perm,
+cudaError_t launch_boundary_search(const ImpSrc& I, const void* stats, const int32_t* perm,
                                    long long perm_stride, int M, int K, int T, double t_s, double alpha,
                                    const Candidate* cands, int ncand, int32_t* counts_out,
                                    double* vs_out, int32_t* rank_out, double* retained_out,
                                    void* ws, int* status, cudaStream_t s);
 
 size_t mask_workspace_bytes(int M, int K, int T);
-cudaError_t launch_mask(const float* I, const int32_t* perm, long long perm_stride,
+cudaError_t launch_mask(const ImpSrc& I, const int32_t* perm, long long perm_stride,
                         const int32_t* counts,
                         const int32_t* rank, int M, int K, int T, uint32_t* bitmask,
                         int8_t* region, void* ws, int* status, cudaStream_t s);
@@ -142,7 +154,7 @@ cudaError_t launch_spmm(const hinm_layout& L, const uint16_t* X, int N, const Sp
 // tile_pmax (int [M/T]) receives each tile's largest fp32 exponent; scratch holds
 // rank_scratch_bytes() bytes.
 size_t rank_scratch_bytes(int M, int K, int T);
-cudaError_t launch_vector_rank(const float* I, const int32_t* perm, long long perm_stride, int M,
+cudaError_t launch_vector_rank(const ImpSrc& I, const int32_t* perm, long long perm_stride, int M,
                                int K, int T,
                                double* V, int32_t* rank, int* tile_pmax, void* scratch,
                                cudaStream_t s);

@@ -128,7 +128,7 @@ __global__ void importance_stats_kernel(const uint16_t* __restrict__ W,
     const int c0 = 2 * cp;
     const float s0 = __ldg(s + c0), s1 = __ldg(s + c0 + 1);
     const uint32_t* wp = reinterpret_cast<const uint32_t*>(W + (size_t)t * T * K + c0);
-    float2* ip = reinterpret_cast<float2*>(I + (size_t)t * T * K + c0);
+    float2* ip = I ? reinterpret_cast<float2*>(I + (size_t)t * T * K + c0) : nullptr;
     const size_t step = (size_t)K / 2;  // one row, in channel pairs
     double v0 = 0.0, v1 = 0.0;
     uint32_t wv[kStatRows], nx[kStatRows];
@@ -144,7 +144,7 @@ __global__ void importance_stats_kernel(const uint16_t* __restrict__ W,
         const float w0 = __uint_as_float(wv[k] << 16), w1 = __uint_as_float(wv[k] & 0xFFFF0000u);
         const float i0 = __fmul_rn(__fmul_rn(w0, w0), s0);
         const float i1 = __fmul_rn(__fmul_rn(w1, w1), s1);
-        __stcs(ip + (size_t)(r0 + k) * step, make_float2(i0, i1));
+        if (I) __stcs(ip + (size_t)(r0 + k) * step, make_float2(i0, i1));
         v0 = __dadd_rn(v0, (double)i0);
         v1 = __dadd_rn(v1, (double)i1);
         mb = max(mb, max(__float_as_uint(i0), __float_as_uint(i1)));
@@ -197,13 +197,18 @@ cudaError_t noalloc_energy_scratch(float** out) {
 size_t tile_stats_v_bytes(int M, int K, int T) {
   return ((size_t)(M / T) * K * sizeof(double) + 255) & ~size_t(255);
 }
-size_t tile_stats_bytes(int M, int K, int T) {
+size_t tile_stats_s_offset(int M, int K, int T) {
   return tile_stats_v_bytes(M, K, T) + (((size_t)(M / T) * sizeof(int) + 255) & ~size_t(255));
+}
+size_t tile_stats_bytes(int M, int K, int T) {
+  return tile_stats_s_offset(M, K, T) + (((size_t)K * sizeof(float) + 255) & ~size_t(255));
 }
 
 cudaError_t launch_importance_stats(const uint16_t* W, const uint16_t* X, int M, int K, int N,
-                                    int T, float* I, void* stats, float* s_scratch,
-                                    cudaStream_t st) {
+                                    int T, float* I, void* stats, cudaStream_t st) {
+  // the channel energies live in the statistics, so that I can be recomputed from W later
+  float* s_scratch = reinterpret_cast<float*>(static_cast<char*>(stats) +
+                                              tile_stats_s_offset(M, K, T));
   const int nt = M / T;
   double* V = static_cast<double*>(stats);
   int* pmax = reinterpret_cast<int*>(static_cast<char*>(stats) + tile_stats_v_bytes(M, K, T));

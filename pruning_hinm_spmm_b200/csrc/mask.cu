@@ -131,7 +131,7 @@ __device__ __forceinline__ void mask_load_rows(const float* p, float (&v)[RB]) {
 
 template <int RB>
 __global__ void __launch_bounds__(kMaskThreads) bitmask_kernel(
-    const float* __restrict__ I, const int8_t* __restrict__ region, const int32_t* __restrict__ counts,
+    const ImpSrc src, const int8_t* __restrict__ region, const int32_t* __restrict__ counts,
     const int32_t* __restrict__ member, int K, int T, uint32_t* __restrict__ bitmask) {
   extern __shared__ __align__(16) uint8_t mask_smem[];
   const int K8 = (K + 7) & ~7;
@@ -143,9 +143,8 @@ __global__ void __launch_bounds__(kMaskThreads) bitmask_kernel(
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   constexpr int nwarps = kMaskThreads / 32;
   const int8_t* reg = region + (size_t)t * K;
-  const float* src = I + ((size_t)t * T + r0) * K;
   constexpr uint8_t kAll = (uint8_t)((1u << RB) - 1u);
-  stage_rows<RB, kMaskThreads>(src, K, rows_s);
+  stage_rows_imp<RB, kMaskThreads>(src, (size_t)t * T + r0, K, rows_s);
   // dense channels keep every row; 4 channels per thread (K % 4 == 0)
   for (int q = threadIdx.x; q < (K >> 2); q += kMaskThreads) {
     const char4 rq = __ldg(reinterpret_cast<const char4*>(reg) + q);
@@ -237,7 +236,7 @@ size_t mask_workspace_bytes(int M, int K, int T) {
   return (c.off + 255) & ~size_t(255);
 }
 
-cudaError_t launch_mask(const float* I, const int32_t* perm, long long perm_stride,
+cudaError_t launch_mask(const ImpSrc& I, const int32_t* perm, long long perm_stride,
                         const int32_t* counts,
                         const int32_t* rank, int M, int K, int T, uint32_t* bitmask,
                         int8_t* region, void* ws, int* status, cudaStream_t s) {

@@ -120,24 +120,25 @@ __device__ __forceinline__ double pow2(int e) {
 
 // Pass 1, thread per (tile, channel): V[t, c] = sum over the tile's rows, ascending, of
 // I (fp64), and the tile's largest exponent P.
-__global__ void vector_score_kernel(const float* __restrict__ I, int K, int T,
+__global__ void vector_score_kernel(const ImpSrc src, int K, int T,
                                     double* __restrict__ Vc, int* __restrict__ tile_pmax) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   const int t = blockIdx.y;
   int pm = 0;
   if (c < K) {
-    const float* p = I + (size_t)t * T * K + c;
+    const size_t row0 = (size_t)t * T;
     double acc = 0.0;
     uint32_t mb = 0;  // largest bit pattern = largest value (non-negative floats)
     constexpr int kBatch = 16;  // T is a multiple of 16
     float v[kBatch], nx[kBatch];
+    const ImpColumn col = imp_column(src, K, c);
 #pragma unroll
-    for (int k = 0; k < kBatch; ++k) v[k] = __ldg(p + (size_t)k * K);
+    for (int k = 0; k < kBatch; ++k) v[k] = col.at(row0 + k);
     for (int i0 = 0; i0 < T; i0 += kBatch) {
       // the next batch's loads go out before this batch's dependent chain
       if (i0 + kBatch < T) {
 #pragma unroll
-        for (int k = 0; k < kBatch; ++k) nx[k] = __ldg(p + (size_t)(i0 + kBatch + k) * K);
+        for (int k = 0; k < kBatch; ++k) nx[k] = col.at(row0 + i0 + kBatch + k);
       }
 #pragma unroll
       for (int k = 0; k < kBatch; ++k) {  // rows ascending
@@ -157,65 +158,158 @@ __global__ void vector_score_kernel(const float* __restrict__ I, int K, int T,
   if ((threadIdx.x & 31) == 0) atomicMax(tile_pmax + t, pm);
 }
 
-// Pass 2, thread per (tile, channel): the column's exact sum at the tile's scale, and a
-// flag when some of its values fell below that scale (summed exactly elsewhere).
-// Two fp64 accumulators carry the common values exactly: level 1 takes p >= e1 =
-// max(P - 22, lsb), level 2 takes p in [e2, e1) with e2 = max(e1 - 22, lsb).  At each level
-// a value is an integer below 2^46 in units of 2^(level - 149), and a column has at most 128
-// values, so the fp64 sums stay integers below 2^53 and never round.  Smaller values take
-// the 128-bit path (p >= lsb) or set the flag.
-__global__ void column_sum_kernel(const float* __restrict__ I, int K, int T,
-                                  const int* __restrict__ tile_pmax, U128* __restrict__ colsum,
-                                  unsigned char* __restrict__ coltiny) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+// Pass 2: each column's exact sum at the tile's scale, and a flag when some of its values
+// fell below that scale (summed exactly elsewhere).  Two fp64 accumulators carry the common
+// values exactly: level 1 takes p >= e1 = max(P - 22, lsb), level 2 takes p in [e2, e1) with
+// e2 = max(e1 - 22, lsb).  At each level a value is an integer below 2^46 in units of
+// 2^(level - 149), and a column has at most 128 values, so the fp64 sums stay integers below
+// 2^53 and never round.  Smaller values (rare: 2^44 below the tile's largest) take a 128-bit
+// integer path (p >= lsb) or set the flag.
+//
+// CTA of 256 threads per (tile, 256 channels): a thread takes 4 adjacent channels (one 16-byte
+// load of I, or one 8-byte load of W, per row) over one of kSplit row ranges, with kBatch rows'
+// loads in flight.  The rare path and the final combination of the row ranges go through
+// shared memory (one 128-bit sum per (range, channel)), which keeps the registers to the fp64
+// sums and the loads.
+constexpr int kColThreads = 256;
+
+// The rare values of a column (below the second level): exactly into the column's 128-bit
+// sum in shared memory (p >= lsb, owner thread only), else the flag.  Out of line, so that
+// the common path stays short.
+__device__ __noinline__ void col_rare(float x, int lsb, U128* xs, unsigned char* tn) {
+  uint32_t m;
+  int e;
+  split_f32(x, m, e);
+  if (!m) return;
+  if (e >= lsb) {
+    U128 v = *xs;
+    add_shifted(v, m, e - lsb);
+    *xs = v;
+  } else {
+    *tn = 1;
+  }
+}
+
+// Channels c .. c + 3 (c a multiple of 4) of one row: the raw load (kW: 4 bf16 of W, else
+// 4 fp32 of I), and value j of it as the importance.
+template <bool kW>
+struct ImpQuad;
+template <>
+struct ImpQuad<false> {
+  using Raw = float4;
+  const float* I;
+  int K, c;
+  __device__ __forceinline__ Raw load(size_t row) const {
+    return __ldg(reinterpret_cast<const float4*>(I + row * K + c));
+  }
+  __device__ __forceinline__ float value(const Raw& r, int j) const {
+    return j == 0 ? r.x : (j == 1 ? r.y : (j == 2 ? r.z : r.w));
+  }
+};
+template <>
+struct ImpQuad<true> {
+  using Raw = uint2;
+  const uint16_t* W;
+  float s[4];
+  int K, c;
+  __device__ __forceinline__ Raw load(size_t row) const {
+    return __ldg(reinterpret_cast<const uint2*>(W + row * K + c));
+  }
+  __device__ __forceinline__ float value(const Raw& r, int j) const {
+    const uint32_t word = j < 2 ? r.x : r.y;
+    return imp_from_w((j & 1) ? (word >> 16) : (word & 0xFFFFu), s[j]);
+  }
+};
+
+// acc (units 2^(lsb - 149)) += a * 2^(e - lsb), a an fp64 integer below 2^53 in units
+// 2^(e - 149), e - lsb <= 61
+__device__ __forceinline__ void add_level(U128& acc, double a, int e, int lsb) {
+  const unsigned long long ai = __double2ull_rz(__dmul_rn(a, pow2(149 - e)));
+  const int sh = e - lsb;
+  U128 f{ai << sh, sh ? (ai >> (64 - sh)) : 0ull};
+  add128(acc, f);
+}
+
+template <int kBatch, int kSplit, bool kW>
+__global__ void __launch_bounds__(kColThreads, 3) column_sum_kernel(
+    const ImpSrc src, int K, int T, const int* __restrict__ tile_pmax,
+    U128* __restrict__ colsum, unsigned char* __restrict__ coltiny) {
+  constexpr int kQuads = kColThreads / kSplit;  // channel quads per CTA
+  __shared__ U128 xs[kSplit][kQuads * 4];
+  __shared__ unsigned char tn[kSplit][kQuads * 4];
+  const int q = threadIdx.x % kQuads, part = threadIdx.x / kQuads;
+  const int c = (blockIdx.x * kQuads + q) * 4;
   const int t = blockIdx.y;
-  if (c >= K) return;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    xs[part][4 * q + k] = U128{0ull, 0ull};
+    tn[part][4 * q + k] = 0;
+  }
   const int pmax = tile_pmax[t];
   const int lsb = tile_lsb(pmax);
   const int e1 = max(pmax - 22, lsb), e2 = max(e1 - 22, lsb);
   const float thr1 = __uint_as_float((uint32_t)(e1 + 1) << 23);  // smallest fp32 with p >= e1
   const float thr2 = __uint_as_float((uint32_t)(e2 + 1) << 23);
-  const float* p = I + (size_t)t * T * K + c;
-  double acc1 = 0.0, acc2 = 0.0;
-  U128 acc{0ull, 0ull};
-  unsigned char tiny = 0;
-  constexpr int kBatch = 16;
-  float v[kBatch], nx[kBatch];
-#pragma unroll
-  for (int k = 0; k < kBatch; ++k) v[k] = __ldg(p + (size_t)k * K);
-  for (int i0 = 0; i0 < T; i0 += kBatch) {
-    if (i0 + kBatch < T) {  // next batch in flight during this one
-#pragma unroll
-      for (int k = 0; k < kBatch; ++k) nx[k] = __ldg(p + (size_t)(i0 + kBatch + k) * K);
+  double a1[4] = {0.0, 0.0, 0.0, 0.0}, a2[4] = {0.0, 0.0, 0.0, 0.0};
+  if (c < K) {  // K is a multiple of 4
+    ImpQuad<kW> col;
+    if constexpr (kW) {
+      const float4 s4 = __ldg(reinterpret_cast<const float4*>(src.s + c));
+      col = ImpQuad<kW>{src.W, {s4.x, s4.y, s4.z, s4.w}, K, c};
+    } else {
+      col = ImpQuad<kW>{src.I, K, c};
     }
+    const int rows = T / kSplit;  // a multiple of kBatch
+    const size_t row0 = (size_t)t * T + (size_t)part * rows;
+    typename ImpQuad<kW>::Raw v[kBatch], nx[kBatch];
 #pragma unroll
-    for (int k = 0; k < kBatch; ++k) {
-      if (v[k] >= thr1) {
-        acc1 = __dadd_rn(acc1, (double)v[k]);
-      } else if (v[k] >= thr2) {
-        acc2 = __dadd_rn(acc2, (double)v[k]);
-      } else {
-        uint32_t m;
-        int e;
-        split_f32(v[k], m, e);
-        if (!m) continue;
-        if (e >= lsb) add_shifted(acc, m, e - lsb);
-        else tiny = 1;
+    for (int k = 0; k < kBatch; ++k) v[k] = col.load(row0 + k);
+    for (int i0 = 0; i0 < rows; i0 += kBatch) {
+      if (i0 + kBatch < rows) {  // next batch in flight during this one
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) nx[k] = col.load(row0 + i0 + kBatch + k);
       }
-    }
 #pragma unroll
-    for (int k = 0; k < kBatch; ++k) v[k] = nx[k];
+      for (int k = 0; k < kBatch; ++k) {  // rows ascending
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float x = col.value(v[k], j);
+          if (x >= thr1) {
+            a1[j] = __dadd_rn(a1[j], (double)x);
+          } else if (x >= thr2) {
+            a2[j] = __dadd_rn(a2[j], (double)x);
+          } else if (x != 0.0f) {
+            col_rare(x, lsb, &xs[part][4 * q + j], &tn[part][4 * q + j]);
+          }
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) v[k] = nx[k];
+    }
   }
-  // acc += acc1 * 2^(e1 - lsb) + acc2 * 2^(e2 - lsb)  (integers < 2^53, shifts <= 61)
-  const unsigned long long a1 = __double2ull_rz(__dmul_rn(acc1, pow2(149 - e1)));
-  const unsigned long long a2 = __double2ull_rz(__dmul_rn(acc2, pow2(149 - e2)));
-  const int s1 = e1 - lsb, s2 = e2 - lsb;
-  U128 f1{a1 << s1, s1 ? (a1 >> (64 - s1)) : 0ull};
-  U128 f2{a2 << s2, s2 ? (a2 >> (64 - s2)) : 0ull};
-  add128(acc, f1);
-  add128(acc, f2);
-  colsum[(size_t)t * K + c] = acc;
-  coltiny[(size_t)t * K + c] = tiny;
+  // this range's total per channel, then the ranges in order
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    U128 acc = xs[part][4 * q + j];
+    add_level(acc, a1[j], e1, lsb);
+    add_level(acc, a2[j], e2, lsb);
+    xs[part][4 * q + j] = acc;
+  }
+  __syncthreads();
+  if (part == 0 && c < K) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      U128 acc = xs[0][4 * q + j];
+      unsigned char tiny = tn[0][4 * q + j];
+#pragma unroll
+      for (int r = 1; r < kSplit; ++r) {
+        add128(acc, xs[r][4 * q + j]);
+        tiny |= tn[r][4 * q + j];
+      }
+      colsum[(size_t)t * K + c + j] = acc;
+      coltiny[(size_t)t * K + c + j] = tiny;
+    }
+  }
 }
 
 // ------------------------------------------------------------------ rank sort
@@ -332,7 +426,7 @@ size_t rank_scratch_bytes(int M, int K, int T) {
 namespace {
 
 // V and the tile maxima (one launch after clearing the maxima).
-cudaError_t launch_vector_scores(const float* I, int M, int K, int T, double* V, int* tile_pmax,
+cudaError_t launch_vector_scores(const ImpSrc& I, int M, int K, int T, double* V, int* tile_pmax,
                                  cudaStream_t s) {
   const int nt = M / T;
   cudaError_t e = cudaMemsetAsync(tile_pmax, 0, (size_t)nt * sizeof(int), s);
@@ -394,7 +488,7 @@ cudaError_t side_stream(SideStream** out) {
 
 }  // namespace
 
-cudaError_t launch_vector_rank(const float* I, const int32_t* perm, long long perm_stride, int M,
+cudaError_t launch_vector_rank(const ImpSrc& I, const int32_t* perm, long long perm_stride, int M,
                                int K, int T,
                                double* V, int32_t* rank, int* tile_pmax, void* scratch,
                                cudaStream_t s) {
@@ -494,7 +588,7 @@ struct CandidateList {
 // vectors' column sums -> rdense[t][m] (values below the tile's scale go to the buckets).
 template <int kPerMax>
 __global__ void __launch_bounds__(512, 2) candidate_lists_kernel(
-    const float* __restrict__ I, const int32_t* __restrict__ perm_all, long long perm_stride,
+    const ImpSrc src, const int32_t* __restrict__ perm_all, long long perm_stride,
     const int32_t* __restrict__ rank,
     const int* __restrict__ tile_pmax, const U128* __restrict__ colsum,
     const unsigned char* __restrict__ coltiny, int K, int T, CandidateList cl, int ncand,
@@ -509,7 +603,7 @@ __global__ void __launch_bounds__(512, 2) candidate_lists_kernel(
   const int32_t* rk = rank + (size_t)t * K;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int lsb = tile_lsb(tile_pmax[t]);
-  const float* It = I + (size_t)t * T * K;
+  const size_t row0 = (size_t)t * T;
   unsigned long long* bkt = bucket + ((size_t)t * ncand + m) * 256;
   unsigned short* out = band + ((size_t)t * ncand + m) * K;
   U128 acc{0ull, 0ull};
@@ -557,10 +651,11 @@ __global__ void __launch_bounds__(512, 2) candidate_lists_kernel(
       if (r < n4) {
         add128(acc, cs[q]);
         if (tn[q]) {  // values below the tile's scale: exact buckets
+          const ImpColumn col = imp_column(src, K, c[q]);
           for (int i = 0; i < T; ++i) {
             uint32_t mm;
             int e;
-            split_f32(__ldg(It + (size_t)i * K + c[q]), mm, e);
+            split_f32(col.at(row0 + i), mm, e);
             if (mm && e < lsb) {
               atomicAdd(bkt + e, (unsigned long long)mm);
               used = true;
@@ -624,6 +719,32 @@ __device__ __forceinline__ void band_slow(float v, U128& ex, int lsb, unsigned l
   }
 }
 
+// A group whose smaller top-2 value on some row lies below the fast path: each of its values
+// to the fast sum or, below thr, to band_slow.  Out of line (rare), so that the common path
+// stays short.
+template <int RB>
+struct GroupTop2 {
+  float t1[RB], t2[RB];
+};
+struct BandSlowState {
+  double acc;
+  U128 ex;
+  bool used;
+};
+template <int RB>
+__device__ __noinline__ BandSlowState band_group_slow(const GroupTop2<RB> g, float thr,
+                                                      BandSlowState st, int lsb,
+                                                      unsigned long long* bkt) {
+#pragma unroll
+  for (int r = 0; r < RB; ++r) {
+    if (g.t1[r] >= thr) st.acc = __dadd_rn(st.acc, (double)g.t1[r]);
+    else band_slow(g.t1[r], st.ex, lsb, bkt, st.used);
+    if (g.t2[r] >= thr) st.acc = __dadd_rn(st.acc, (double)g.t2[r]);
+    else band_slow(g.t2[r], st.ex, lsb, bkt, st.used);
+  }
+  return st;
+}
+
 // Per (tile, chunk of RB rows), 512 threads.  The chunk's rows of I are staged in shared
 // memory channel-major (the RB values of channel c contiguous at slot stage_slot(c), one
 // vector load each).  Then, candidate by candidate, the candidate's 2:4 groups are dealt to
@@ -638,7 +759,7 @@ __device__ __forceinline__ void band_slow(float v, U128& ex, int lsb, unsigned l
 // sums with three 21-bit-piece reductions and one shared atomic.
 template <int RB, int kThreads>
 __global__ void __launch_bounds__(kThreads) band_sum_kernel(
-    const float* __restrict__ I, const unsigned short* __restrict__ band,
+    const ImpSrc src, const unsigned short* __restrict__ band,
     const int* __restrict__ tile_pmax, int K, int T, CandidateList cl, int ncand,
     U128* __restrict__ part, unsigned long long* __restrict__ bucket,
     int* __restrict__ bucket_used) {
@@ -656,7 +777,7 @@ __global__ void __launch_bounds__(kThreads) band_sum_kernel(
   const double unit_scale = pow2(149 - eb);                      // fp64 sum -> integer units
   for (int x = threadIdx.x; x < kMaxCandidates; x += kThreads) fast_sum[x] = 0ull;
   for (int x = threadIdx.x; x < kMaxCandidates * 4; x += kThreads) (&digits[0][0])[x] = 0ull;
-  stage_rows<RB, kThreads>(I + ((size_t)t * T + (size_t)chunk * RB) * K, K, rows_s);
+  stage_rows_imp<RB, kThreads>(src, (size_t)t * T + (size_t)chunk * RB, K, rows_s);
   __syncthreads();
 
   const unsigned short* band_t = band + (size_t)t * ncand * K;
@@ -694,29 +815,27 @@ __global__ void __launch_bounds__(kThreads) band_sum_kernel(
         load_rows<RB>(rows_s + min((int)cq[j].y, K8 - 1) * RB, v1);
         load_rows<RB>(rows_s + min((int)cq[j].z, K8 - 1) * RB, v2);
         load_rows<RB>(rows_s + min((int)cq[j].w, K8 - 1) * RB, v3);
-        float t1[RB], t2[RB];
+        GroupTop2<RB> g2;
         float lo = INFINITY;
 #pragma unroll
         for (int r = 0; r < RB; ++r) {
           const float a = fmaxf(v0[r], v1[r]), b = fminf(v0[r], v1[r]);
           const float cc = fmaxf(v2[r], v3[r]), d = fminf(v2[r], v3[r]);
-          t1[r] = fmaxf(a, cc);
-          t2[r] = fmaxf(fminf(a, cc), fmaxf(b, d));
-          lo = fminf(lo, t2[r]);
+          g2.t1[r] = fmaxf(a, cc);
+          g2.t2[r] = fmaxf(fminf(a, cc), fmaxf(b, d));
+          lo = fminf(lo, g2.t2[r]);
         }
         if (lo >= thr) {  // every value of the group on the fast path (t1 >= t2 >= thr)
           double g = 0.0;
 #pragma unroll
-          for (int r = 0; r < RB; ++r) g = __dadd_rn(g, __dadd_rn((double)t1[r], (double)t2[r]));
+          for (int r = 0; r < RB; ++r)
+            g = __dadd_rn(g, __dadd_rn((double)g2.t1[r], (double)g2.t2[r]));
           acc = __dadd_rn(acc, g);
         } else {
-#pragma unroll
-          for (int r = 0; r < RB; ++r) {
-            if (t1[r] >= thr) acc = __dadd_rn(acc, (double)t1[r]);
-            else band_slow(t1[r], ex, lsb, bkt, used);
-            if (t2[r] >= thr) acc = __dadd_rn(acc, (double)t2[r]);
-            else band_slow(t2[r], ex, lsb, bkt, used);
-          }
+          const BandSlowState st = band_group_slow<RB>(g2, thr, BandSlowState{acc, ex, used}, lsb, bkt);
+          acc = st.acc;
+          ex = st.ex;
+          used = st.used;
         }
       }
     }
@@ -848,7 +967,7 @@ size_t search_workspace_bytes(int M, int K, int T, int ncand) {
   return (c.off + 255) & ~size_t(255);
 }
 
-cudaError_t launch_boundary_search(const float* I, const void* stats, const int32_t* perm,
+cudaError_t launch_boundary_search(const ImpSrc& I, const void* stats, const int32_t* perm,
                                    long long perm_stride,
                                    int M, int K, int T, double t_s, double alpha,
                                    const Candidate* cands, int ncand, int32_t* counts_out,
@@ -898,8 +1017,19 @@ cudaError_t launch_boundary_search(const float* I, const void* stats, const int3
     if (e != cudaSuccess) return e;
     e = cudaStreamWaitEvent(ss->stream, ss->fork, 0);
     if (e != cudaSuccess) return e;
-    dim3 gc((K + 255) / 256, nt);
-    column_sum_kernel<<<gc, 256, 0, ss->stream>>>(I, K, T, pmax, colsum, coltiny);
+    // a CTA per (tile, 256 channels); T = 64 splits its rows in 2, T = 128 in 4
+    const dim3 gc((K + 255) / 256, nt);
+    if (I.I) {  // from I: 16-byte loads, 4 rows in flight
+      if (T == 128)
+        column_sum_kernel<4, 4, false><<<gc, kColThreads, 0, ss->stream>>>(I, K, T, pmax, colsum, coltiny);
+      else
+        column_sum_kernel<4, 2, false><<<gc, kColThreads, 0, ss->stream>>>(I, K, T, pmax, colsum, coltiny);
+    } else {  // from W: 8-byte loads, 8 rows in flight
+      if (T == 128)
+        column_sum_kernel<8, 4, true><<<gc, kColThreads, 0, ss->stream>>>(I, K, T, pmax, colsum, coltiny);
+      else
+        column_sum_kernel<8, 2, true><<<gc, kColThreads, 0, ss->stream>>>(I, K, T, pmax, colsum, coltiny);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     e = cudaEventRecord(ss->join, ss->stream);

@@ -145,6 +145,24 @@ def test_validation_rejects_before_launch(H):
     assert lib.hinm_boundary_search_stats(fake, fake, 8, None, 256, 256, 128, 0.5, 1 / 32, fake,
                                           fake, None, None, fake, 1 << 30,
                                           None) == H.HINM_ERR_INVALID_ARG
+    # importance recomputed from W: without I, both W and stats are needed, stats must be
+    # large enough, W aligned
+    def search_ex(I, W, st, st_bytes):
+        return lib.hinm_boundary_search_ex(I, W, st, st_bytes, None, 0, 256, 256, 128, 0.5,
+                                           1 / 32, fake, fake, None, None, fake, 1 << 30, None)
+    assert search_ex(None, None, fake, sz.value) == H.HINM_ERR_INVALID_ARG
+    assert search_ex(None, fake, None, sz.value) == H.HINM_ERR_INVALID_ARG
+    assert search_ex(None, fake, fake, sz.value - 1) == H.HINM_ERR_INVALID_ARG
+    assert search_ex(None, fake + 2, fake, sz.value) == H.HINM_ERR_ALIGNMENT
+
+    def mask_ex(I, W, st, st_bytes, per_tile=0):
+        return lib.hinm_mask_ex(I, W, st, st_bytes, None, per_tile, fake, None, 256, 256, 128,
+                                fake, fake, fake, 1 << 30, None)
+    assert mask_ex(None, None, fake, sz.value) == H.HINM_ERR_INVALID_ARG
+    assert mask_ex(None, fake, None, sz.value) == H.HINM_ERR_INVALID_ARG
+    assert mask_ex(None, fake, fake, sz.value - 1) == H.HINM_ERR_INVALID_ARG
+    assert mask_ex(None, fake + 2, fake, sz.value) == H.HINM_ERR_ALIGNMENT
+    assert mask_ex(fake, None, None, 0, per_tile=2) == H.HINM_ERR_INVALID_ARG
     # the fused epilogue: an unknown activation is refused; the flags are checked first
     assert lib.hinm_spmm_epilogue(ctypes.byref(L), fake, 16, fake, None, 4, 0, 0,
                                   None) == H.HINM_ERR_INVALID_ARG

@@ -6,6 +6,8 @@ benchmark times, and layer 0 of the LLaMA-2-7B-shaped sweep in all 27 (linear sh
 t_s) cases with the boundary from the search.  Against the CPU oracle:
 
 * I (every element, bit for bit);
+* the benchmark's path does not materialize I (the search and the mask recompute it from W
+  and the channel energies); the sweep runs both ways and they agree bit for bit;
 * the boundary search (counts, v_s, rank and every candidate's R(m), bit for bit) on
   sampled tiles -- the oracle's exact scan costs about a second per tile;
 * the mask and the regions of every tile (bit for bit), with the counts the GPU used (its
@@ -34,10 +36,10 @@ def H():
 
 
 def _check_against_oracle(H, w, hp, Y, counts_used, tiles, R_gpu=None, search_counts=None,
-                          search_vs=None, search_rank=None):
+                          search_vs=None, search_rank=None, I=None):
     M, K, T = w.M, w.K, w.T
     I_ref = O.importance(w.W_bits, w.X_bits)
-    I_gpu = hp.I.cpu().numpy()
+    I_gpu = (hp.I if I is None else I).cpu().numpy()
     np.testing.assert_array_equal(I_gpu.view(np.uint32), I_ref.view(np.uint32))
     del I_gpu
     sr = O.boundary_search(I_ref, w.perm, T, w.t_s, w.alpha, tiles=tiles)
@@ -71,16 +73,17 @@ def test_benchmark_workloads_full(H, name, make, v_s):
     M, K, N, T = w.M, w.K, w.N, w.T
     nt = M // T
     W, X, perm = dev_bf16(w.W_bits), dev_bf16(w.X_bits), dev_i32(w.perm)
-    hp = H.HotPath(M, K, N, T, w.t_s, w.alpha)
+    hp = H.HotPath(M, K, N, T, w.t_s, w.alpha, materialize_importance=False)
     c = np.array(H.hinm_counts_from_vs(K, w.t_s, v_s), dtype=np.int32)
     counts = np.tile(c, (nt, 1))
     Y = hp.run(W, X, perm, fixed_counts=dev_i32(counts),
                tile_pairs=H.tile_pairs_hint(c, w.perm, K))
+    I = H.hinm_importance(W, X)        # for the element-wise check of the importance alone
     torch.cuda.synchronize()
     status_ok(H)
     tiles = sorted({0, nt // 2, nt - 1})
     _check_against_oracle(H, w, hp, Y, counts, tiles, search_counts=hp.counts.cpu().numpy(),
-                          search_rank=hp.rank.cpu().numpy(), search_vs=hp.vs.cpu().numpy())
+                          search_rank=hp.rank.cpu().numpy(), search_vs=hp.vs.cpu().numpy(), I=I)
 
 
 # Layer 0 of the sweep: the three linear shapes (q/k/v/o 4096x4096, gate/up 11008x4096,
@@ -100,8 +103,17 @@ def test_llama_sweep_layer0_full(H, linear, t_s, N):
     n_c = H.hinm_search_num_candidates(K, t_s, w.alpha)
     R_gpu = torch.empty((nt, n_c), dtype=torch.float64, device="cuda")
     H.hinm_boundary_search(hp.I, perm, T, t_s, w.alpha, want_rank=False, retained_out=R_gpu)
+    # the same pass without materializing I: every result bit for bit
+    hq = H.HotPath(M, K, N, T, w.t_s, w.alpha, materialize_importance=False)
+    Yq = hq.run(W, X, perm)
     torch.cuda.synchronize()
     status_ok(H)
+    for a, b in ((hp.counts, hq.counts), (hp.vs, hq.vs), (hp.rank, hq.rank),
+                 (hp.bitmask, hq.bitmask), (hp.region, hq.region),
+                 *zip(H.tile_stats_views(hp.stats, M, K, T), H.tile_stats_views(hq.stats, M, K, T))):
+        assert torch.equal(a, b)
+    assert torch.equal(Y.view(torch.int32), Yq.view(torch.int32))
+    del hq, Yq
     counts = hp.counts.cpu().numpy()
     _check_against_oracle(H, w, hp, Y, counts, [0, nt - 1], R_gpu=R_gpu.cpu().numpy(),
                           search_counts=counts, search_vs=hp.vs.cpu().numpy(),
