@@ -8,18 +8,20 @@
 // less than half of the SMs, a cluster of up to 8 CTAs shares each unit's K-blocks and the
 // leader adds the others' partial accumulators (received over DSMEM) in rank order.
 //
-//   warps 0-3  gather producers: for a K-block whose index is not one contiguous run, the
-//              X rows it selects, 16-byte cp.async into the swizzled MN-major B tile
+// Warp roles (G = 8 gather warps in the persistent kernel at BN >= 128, else 4):
+//   warps 0..G-1  gather producers: for a K-block whose index is not one contiguous run,
+//              the X rows it selects, 16-byte cp.async into the swizzled MN-major B tile
 //              (coalesced 2*BN-byte row segments); arrival on the stage's barrier when
 //              they land.
-//   warp 4     MMA: one thread; 2:4 block -> tcgen05.cp of the metadata into tensor memory,
+//   warp G     MMA: one thread; 2:4 block -> tcgen05.cp of the metadata into tensor memory,
 //              then 4 x tcgen05.mma.sp (K = 32 each); dense block -> 4 x tcgen05.mma
 //              (K = 16 each); tcgen05.commit frees the stage / publishes the accumulator.
-//   warps 5-8  epilogue: tcgen05.ld of the 128 x BN fp32 accumulator (a lane holds one
-//              row), 32 columns at a time transposed through a per-warp swizzled 4 KB
-//              shared tile so that each store instruction writes 128-byte row segments of
-//              four rows of Y (or, in a split-K cluster, to the leader's reduction buffer).
-//   warp 9     bulk copies: one thread runs ahead by up to a full ring; per K-block it
+//   warps G+1..G+4  epilogue: tcgen05.ld of the 128 x BN fp32 accumulator (a lane holds one
+//              row; warp w reads lane quadrant w mod 4), 32 columns at a time transposed
+//              through a per-warp swizzled 4 KB shared tile so that each store instruction
+//              writes 128-byte row segments of four rows of Y (or, in a split-K cluster, to
+//              the leader's reduction buffer).
+//   warp G+5   bulk copies: one thread runs ahead by up to a full ring; per K-block it
 //              publishes the block's run flag and index list and bulk-copies the
 //              pre-swizzled 16 KB A block, its 2 KB metadata and, for a contiguous run,
 //              the X rows as 3-D tiled TMA boxes (one per 64 K-rows).
@@ -31,8 +33,8 @@
 //
 // Shared memory holds STAGES stages of [A 16 KB | B 128 x BN bf16 | E 2 KB]; the stage ring
 // runs across work units.  At wide N the second 64 K-rows of a stage complete a barrier of
-// their own, so that the first two MMAs of a 2:4 block do not wait for them.  No load uses
-// cluster multicast.  Every wait is bounded (2 s), after which the CTA records
+// their own, so that the first two MMAs of a 2:4 block do not wait for them.  Every load
+// brings data to its own CTA only.  Every wait is bounded (2 s), after which the CTA records
 // HINM_ERR_DEVICE_TIMEOUT, stops all roles, drains what it issued, frees tensor memory and
 // returns.
 #include <cuda.h>
@@ -87,10 +89,13 @@ struct SpmmCfg {
   // wide N: the second 64 K-rows of a 2:4 block's B land on a barrier of their own, so the
   // MMAs on the first 64 rows start before the second half arrives
   static constexpr bool kSplitB = BN >= 128;
-  static constexpr int kProducers = 128;
-  static constexpr int kMmaWarp = 4;
-  static constexpr int kBulkWarp = 9;
-  static constexpr int kThreads = 320;  // 10 warps: 4 gather, 1 MMA, 4 epilogue, 1 bulk copies
+  // 8 gather warps for the persistent kernel at BN >= 128 (more 16-byte copies in flight:
+  // measured 2 % faster on the up-proj and gate shapes than 4), else 4; then one MMA warp,
+  // 4 epilogue warps and one bulk-copy warp
+  static constexpr int kProducers = (!SPLIT && BN >= 128) ? 256 : 128;
+  static constexpr int kMmaWarp = kProducers / 32;
+  static constexpr int kBulkWarp = kMmaWarp + 5;
+  static constexpr int kThreads = kProducers + 192;
   static_assert(BN == 16 || BN == 32 || (BN % 64 == 0 && BN <= 256), "BN");
   static_assert(kStages >= 2, "stages");
   static_assert(kTmemNeed <= 512, "tmem");
@@ -253,7 +258,7 @@ __device__ __forceinline__ void store_row(const SpmmArgs& a, const uint32_t (&v)
 }
 
 template <int BN, bool SPLIT>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(SpmmCfg<BN, SPLIT>::kThreads, 1)
     spmm_kernel(const __grid_constant__ CUtensorMap tmX, const SpmmArgs a) {
   using C = SpmmCfg<BN, SPLIT>;
   extern __shared__ uint8_t smem_raw[];
@@ -276,6 +281,36 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t drain_bar = ptx::smem_u32(bars + 2 * C::kStages + 4);
   auto idx_bar = [&](int s) { return ptx::smem_u32(bars + 2 * C::kStages + 5 + s); };
   auto full2_bar = [&](int s) { return ptx::smem_u32(bars + 3 * C::kStages + 5 + s); };
+
+  // Work: persistent CTAs stride over the units; split-K CTAs take one unit each and the
+  // K-block range [kb0, kb1) of their cluster rank.
+  const int u_first = SPLIT ? (int)blockIdx.x / a.split : (int)blockIdx.x;
+  const int u_step = SPLIT ? a.num_units : (int)gridDim.x;
+  const int rank = SPLIT ? (int)(blockIdx.x % a.split) : 0;
+  auto k_range = [&](int nblk, int& kb0, int& kb1) {
+    kb0 = SPLIT ? (int)((long long)nblk * rank / a.split) : 0;
+    kb1 = SPLIT ? (int)((long long)nblk * (rank + 1) / a.split) : nblk;
+  };
+  // The first unit's tile record, and for the bulk-copy thread its first block's run flag,
+  // are loaded before the set-up below, so that their latency overlaps it.
+  int4 info_first = make_int4(0, 0, 0, 0);
+  int run_first = -1;
+  if (u_first < a.num_units) {
+    info_first = __ldg(reinterpret_cast<const int4*>(a.tile_info) + u_first / a.nblk_n);
+    if (warp == C::kBulkWarp && lane == 0) {
+      int kb0, kb1;
+      k_range(info_first.x + info_first.y, kb0, kb1);
+      if (kb0 < kb1) {
+        const bool sparse = kb0 >= info_first.x;
+        const size_t blk = sparse ? (size_t)(info_first.w + kb0 - info_first.x)
+                                  : (size_t)(info_first.z + kb0);
+        run_first = __ldg(sparse ? a.run_sparse + blk : a.run_dense + blk);
+      }
+    }
+  }
+  auto tile_info_of = [&](int u, int tile) {
+    return u == u_first ? info_first : __ldg(reinterpret_cast<const int4*>(a.tile_info) + tile);
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -304,21 +339,12 @@ __global__ void __launch_bounds__(320, 1)
   float* red = reinterpret_cast<float*>(idx_region + C::kStages * C::kIdxBytes + 512);
   // [4 warps][32 rows][8 x 16-byte pieces], piece p of row r at slot p ^ (r & 7)
   uint8_t* epi_stage = reinterpret_cast<uint8_t*>(red) + C::kRedBytes;
-  // Work: persistent CTAs stride over the units; split-K CTAs take one unit each and the
-  // K-block range [kb0, kb1) of their cluster rank.
-  const int u_first = SPLIT ? (int)blockIdx.x / a.split : (int)blockIdx.x;
-  const int u_step = SPLIT ? a.num_units : (int)gridDim.x;
-  const int rank = SPLIT ? (int)(blockIdx.x % a.split) : 0;
-  auto k_range = [&](int nblk, int& kb0, int& kb1) {
-    kb0 = SPLIT ? (int)((long long)nblk * rank / a.split) : 0;
-    kb1 = SPLIT ? (int)((long long)nblk * (rank + 1) / a.split) : nblk;
-  };
 
   // split-K: what the leader's epilogue needs after the cluster barrier
   bool split_ready = false, split_has = false;
   int split_tile = 0, split_n0 = 0, split_b = 0;
 
-  if (warp < 4) {
+  if (warp < C::kProducers / 32) {
     // ------------------------------------------------------------ gather producers
     // Per K-block: wait until the bulk-copy warp has the stage (its index-ready barrier),
     // then either gather the X rows the block's index selects (16-byte cp.async, arrival
@@ -332,7 +358,7 @@ __global__ void __launch_bounds__(320, 1)
     bool stop = false;
     for (int u = u_first; u < a.num_units && !stop; u += u_step) {
       const int tile = u / a.nblk_n, n0 = (u - tile * a.nblk_n) * BN;
-      const int4 info = __ldg(reinterpret_cast<const int4*>(a.tile_info) + tile);
+      const int4 info = tile_info_of(u, tile);
       const int nd = info.x, nblk = info.x + info.y;
       int kb0, kb1;
       k_range(nblk, kb0, kb1);
@@ -387,14 +413,16 @@ __global__ void __launch_bounds__(320, 1)
       bool stop = false;
       for (int u = u_first; u < a.num_units && !stop; u += u_step) {
         const int tile = u / a.nblk_n, n0 = (u - tile * a.nblk_n) * BN;
-        const int4 info = __ldg(reinterpret_cast<const int4*>(a.tile_info) + tile);
+        const int4 info = tile_info_of(u, tile);
         const int nd = info.x, nblk = info.x + info.y;
         int kb0, kb1;
         k_range(nblk, kb0, kb1);
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const bool sparse = kb >= nd;
           const size_t blk = sparse ? (size_t)(info.w + kb - nd) : (size_t)(info.z + kb);
-          const int run = __ldg(sparse ? a.run_sparse + blk : a.run_dense + blk);
+          const int run = (u == u_first && kb == kb0)
+                              ? run_first
+                              : __ldg(sparse ? a.run_sparse + blk : a.run_dense + blk);
           const int s = it % C::kStages;
           const uint32_t ph = (it / C::kStages) & 1;
           if (!ptx::mbar_wait(empty_bar(s), ph ^ 1, a.status, abort_flag)) {
@@ -465,7 +493,7 @@ __global__ void __launch_bounds__(320, 1)
       bool stop = false;
       for (int u = u_first; u < a.num_units && !stop; u += u_step, ++lu) {
         const int tile = u / a.nblk_n;
-        const int4 info = __ldg(reinterpret_cast<const int4*>(a.tile_info) + tile);
+        const int4 info = tile_info_of(u, tile);
         const int nd = info.x, nblk = info.x + info.y;
         int kb0, kb1;
         k_range(nblk, kb0, kb1);
@@ -543,7 +571,7 @@ __global__ void __launch_bounds__(320, 1)
     uint32_t lu = 0;
     for (int u = u_first; u < a.num_units; u += u_step, ++lu) {
       const int tile = u / a.nblk_n, n0 = (u - tile * a.nblk_n) * BN;
-      const int4 info = __ldg(reinterpret_cast<const int4*>(a.tile_info) + tile);
+      const int4 info = tile_info_of(u, tile);
       int kb0, kb1;
       k_range(info.x + info.y, kb0, kb1);
       const bool has = kb1 > kb0;  // else the accumulator was never written: zeros
