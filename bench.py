@@ -278,7 +278,8 @@ def run_sweep(args):
                 W = torch.from_numpy(w.W_bits.view(np.int16)).to(dev).view(torch.bfloat16)
                 X = torch.from_numpy(w.X_bits.view(np.int16)).to(dev).view(torch.bfloat16)
                 perm = torch.from_numpy(w.perm).to(dev)
-                hp = H.HotPath(M, K, N, T, w.t_s, w.alpha, device=dev)
+                hp = H.HotPath(M, K, N, T, w.t_s, w.alpha, device=dev,
+                               materialize_importance=False)
                 for _ in range(args.warmup):
                     hp.run(W, X, perm)
                 torch.cuda.synchronize()
