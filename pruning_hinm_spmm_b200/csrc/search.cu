@@ -747,16 +747,16 @@ __device__ __noinline__ BandSlowState band_group_slow(const GroupTop2<RB> g, flo
 
 // Per (tile, chunk of RB rows), 512 threads.  The chunk's rows of I are staged in shared
 // memory channel-major (the RB values of channel c contiguous at slot stage_slot(c), one
-// vector load each).  Then, candidate by candidate, the candidate's 2:4 groups are dealt to
-// the warps in chunks (the starting warp rotates, so the work stays even over the scan)
-// and, for every row, the top 2 of the group's 4 values are summed.
+// vector load each).  Then every candidate's 2:4 groups, as one candidate-major list, are
+// split into equal contiguous slices, one per warp, and for every row the top 2 of each
+// group's 4 values are summed.
 //
 // The sums are exact.  With eb = max(P - 24, lsb) every value with p >= eb is a multiple of
-// u = 2^(eb - 149) below 2^48 u, and a thread adds at most 32 of them per candidate (for any
-// K <= 16384 with the rows per CTA of band_config), so its fp64 sum never rounds (it stays
-// an integer multiple of u below 2^53 u), in any order.  Values with p < eb (rare: 2^24 below
-// the tile's largest) go to band_slow.  Per candidate, each warp adds its threads' integer
-// sums with three 21-bit-piece reductions and one shared atomic.
+// u = 2^(eb - 149) below 2^48 u.  A lane adds at most 2 kG RB = 32 of them in fp64 per pass
+// (kG groups), so that sum never rounds (an integer multiple of u below 2^53 u), in any
+// order, and then moves it into a 64-bit integer.  Values with p < eb (rare: 2^24 below
+// the tile's largest) go to band_slow.  Per (warp, candidate) the lanes' integers meet in
+// three 21-bit-piece reductions and one shared atomic.
 template <int RB, int kThreads>
 __global__ void __launch_bounds__(kThreads) band_sum_kernel(
     const ImpSrc src, const unsigned short* __restrict__ band,
@@ -781,34 +781,39 @@ __global__ void __launch_bounds__(kThreads) band_sum_kernel(
   __syncthreads();
 
   const unsigned short* band_t = band + (size_t)t * ncand * K;
-  // A candidate's groups go out in warp chunks of 32 * kG consecutive groups (kG per thread);
-  // chunk k of candidate m goes to warp (woff + k) mod nwarps, and woff advances by the
-  // candidate's chunk count, so the warps' work stays even over the scan.
+  // All candidates' groups form one list (candidate-major); warp w takes the contiguous
+  // slice [w n / nwarps, (w + 1) n / nwarps) of it, so the warps' work is even and a warp
+  // meets only the few candidates its slice spans.  Per candidate piece of the slice the
+  // lanes take kG groups each per pass; after every pass a lane's fp64 sum (at most
+  // 2 kG RB <= 32 values, exact) moves into its 64-bit integer sum, and at the end of the
+  // piece the warp adds those with three 21-bit-piece reductions and one shared atomic.
   constexpr int kG = 4;
   constexpr int nwarps = kThreads / 32;
   const int warp = threadIdx.x >> 5;
-  int woff = 0;
-  for (int m = 0; m < ncand; ++m) {
+  int total = 0;
+  for (int m = 0; m < ncand; ++m) total += cl.c[m].n24 / 4;
+  const int w0 = (int)((long long)total * warp / nwarps);
+  const int w1 = (int)((long long)total * (warp + 1) / nwarps);
+  int base = 0;  // first list index of candidate m
+  for (int m = 0; m < ncand && base < w1; ++m) {
     const int ng = cl.c[m].n24 / 4;
-    const int nchunk = (ng + 32 * kG - 1) / (32 * kG);
-    int k0 = (warp - woff) % nwarps;
-    if (k0 < 0) k0 += nwarps;
-    woff = (woff + nchunk) % nwarps;
-    if (k0 >= nchunk) continue;  // warp-uniform: no chunk of this candidate here
+    const int g0 = max(w0, base) - base, g1 = min(w1, base + ng) - base;
+    base += ng;
+    if (g0 >= g1) continue;  // warp-uniform: this candidate is outside the slice
     const ushort4* bl = reinterpret_cast<const ushort4*>(band_t + (size_t)m * K);
     unsigned long long* bkt = bucket + ((size_t)t * ncand + m) * 256;
-    double acc = 0.0;
+    unsigned long long isum = 0ull;  // this lane's fast sum, integer units of 2^(eb - 149)
     U128 ex{0ull, 0ull};
     bool used = false;
-    for (int k = k0; k < nchunk; k += nwarps) {
-      const int gb = k * 32 * kG + lane;
+    for (int gb = g0 + lane; gb < g1; gb += 32 * kG) {
       ushort4 cq[kG];
 #pragma unroll
       for (int j = 0; j < kG; ++j)
-        cq[j] = gb + 32 * j < ng ? __ldg(bl + gb + 32 * j) : make_ushort4(0, 0, 0, 0);
+        cq[j] = gb + 32 * j < g1 ? __ldg(bl + gb + 32 * j) : make_ushort4(0, 0, 0, 0);
+      double acc = 0.0;
 #pragma unroll
       for (int j = 0; j < kG; ++j) {
-        if (gb + 32 * j >= ng) break;
+        if (gb + 32 * j >= g1) break;
         // the lists hold shared-memory slots (stage_slot of the channel), below K rounded up to 8
         float v0[RB], v1[RB], v2[RB], v3[RB];
         load_rows<RB>(rows_s + min((int)cq[j].x, K8 - 1) * RB, v0);
@@ -838,13 +843,14 @@ __global__ void __launch_bounds__(kThreads) band_sum_kernel(
           used = st.used;
         }
       }
+      isum += __double2ull_rz(__dmul_rn(acc, unit_scale));  // an integer below 2^53
     }
     if (used) atomicOr(bucket_used + (size_t)t * ncand + m, 1);
-    // this thread's fast sum as an integer number of units (< 2^53)
-    const unsigned long long ai = __double2ull_rz(__dmul_rn(acc, unit_scale));
-    const unsigned s0 = __reduce_add_sync(0xffffffffu, (unsigned)(ai & 0x1FFFFFull));
-    const unsigned s1 = __reduce_add_sync(0xffffffffu, (unsigned)((ai >> 21) & 0x1FFFFFull));
-    const unsigned s2 = __reduce_add_sync(0xffffffffu, (unsigned)(ai >> 42));
+    // the warp's fast sum (a lane's isum: at most 64 passes of < 2^53 each, < 2^59), in
+    // three 21-bit pieces
+    const unsigned s0 = __reduce_add_sync(0xffffffffu, (unsigned)(isum & 0x1FFFFFull));
+    const unsigned s1 = __reduce_add_sync(0xffffffffu, (unsigned)((isum >> 21) & 0x1FFFFFull));
+    const unsigned s2 = __reduce_add_sync(0xffffffffu, (unsigned)(isum >> 42));
     if (lane == 0) {
       const unsigned long long w = (unsigned long long)s0 + ((unsigned long long)s1 << 21) +
                                    ((unsigned long long)s2 << 42);
@@ -876,7 +882,8 @@ __global__ void __launch_bounds__(kThreads) band_sum_kernel(
     U128 tot;
     tot.lo = (d0 & 0xFFFFFFFFull) | (d1 << 32);
     tot.hi = (d2 & 0xFFFFFFFFull) | (d3 << 32);
-    // + fast_sum * 2^(eb - lsb): fast_sum < 2^63 (32 warps x 32 threads x 2^53), eb - lsb <= 59
+    // + fast_sum * 2^(eb - lsb): fast_sum < 2^62 (a candidate has at most RB K / 2 <= 12288
+    // values per CTA by band_config, each below 2^48 units), eb - lsb <= 59
     const unsigned long long f = fast_sum[threadIdx.x];
     const int sh = eb - lsb;
     U128 fx;
