@@ -421,18 +421,10 @@ __host__ __device__ inline PackSmem pack_smem(int K, int rows) {
   return p;
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
+using ptx::cp_async16;
+using ptx::cp_async4;
+using ptx::cp_async8;
+using ptx::cp_async_commit_wait_all;
 
 constexpr int kPackThreads = 512;
 constexpr int kPackWarps = kPackThreads / 32;

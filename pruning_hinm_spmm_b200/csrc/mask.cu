@@ -129,23 +129,35 @@ __device__ __forceinline__ void mask_load_rows(const float* p, float (&v)[RB]) {
   }
 }
 
+// Keep bits of a 2:4 group's four members over RB rows (v[k][r]: member k's value in row r).
+// g_kl bit r: member l beats member k (k < l) in row r, i.e. v_l > v_k (equal values: the
+// lower position k wins).  Member k is kept iff at most one member beats it: the negated
+// majority of its three "beaten by" words, all rows at once.
 template <int RB>
-__global__ void __launch_bounds__(kMaskThreads) bitmask_kernel(
-    const ImpSrc src, const int8_t* __restrict__ region, const int32_t* __restrict__ counts,
-    const int32_t* __restrict__ member, int K, int T, uint32_t* __restrict__ bitmask) {
-  extern __shared__ __align__(16) uint8_t mask_smem[];
-  const int K8 = (K + 7) & ~7;
-  float* rows_s = reinterpret_cast<float*>(mask_smem);  // [K8][RB], stage_slot order
-  uint8_t* keep = mask_smem + (size_t)K8 * RB * sizeof(float);
-  const int words = (K + 31) >> 5;
-  const int t = blockIdx.y;
-  const int r0 = blockIdx.x * RB;  // first row of the chunk within the tile
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  constexpr int nwarps = kMaskThreads / 32;
-  const int8_t* reg = region + (size_t)t * K;
+__device__ __forceinline__ void group_keep(const float (&v)[4][RB], uint32_t (&kb)[4]) {
+  uint32_t g01 = 0u, g02 = 0u, g03 = 0u, g12 = 0u, g13 = 0u, g23 = 0u;
+#pragma unroll
+  for (int r = 0; r < RB; ++r) {
+    g01 |= (uint32_t)(v[1][r] > v[0][r]) << r;
+    g02 |= (uint32_t)(v[2][r] > v[0][r]) << r;
+    g03 |= (uint32_t)(v[3][r] > v[0][r]) << r;
+    g12 |= (uint32_t)(v[2][r] > v[1][r]) << r;
+    g13 |= (uint32_t)(v[3][r] > v[1][r]) << r;
+    g23 |= (uint32_t)(v[3][r] > v[2][r]) << r;
+  }
+  auto maj = [](uint32_t a, uint32_t b, uint32_t c) { return (a & b) | (a & c) | (b & c); };
+  constexpr uint32_t kRows = (1u << RB) - 1u;
+  kb[0] = ~maj(g01, g02, g03) & kRows;
+  kb[1] = ~maj(~g01, g12, g13) & kRows;
+  kb[2] = ~maj(~g02, ~g12, g23) & kRows;
+  kb[3] = ~maj(~g03, ~g13, ~g23) & kRows;
+}
+
+// Dense channels keep every row: keep[c] = all ones for them, 0 for the others (4 channels
+// per thread, K % 4 == 0).
+template <int RB>
+__device__ __forceinline__ void keep_dense(const int8_t* __restrict__ reg, int K, uint8_t* keep) {
   constexpr uint8_t kAll = (uint8_t)((1u << RB) - 1u);
-  stage_rows_imp<RB, kMaskThreads>(src, (size_t)t * T + r0, K, rows_s);
-  // dense channels keep every row; 4 channels per thread (K % 4 == 0)
   for (int q = threadIdx.x; q < (K >> 2); q += kMaskThreads) {
     const char4 rq = __ldg(reinterpret_cast<const char4*>(reg) + q);
     const uint32_t k4 = (rq.x == HINM_REGION_DENSE ? (uint32_t)kAll : 0u) |
@@ -154,47 +166,23 @@ __global__ void __launch_bounds__(kMaskThreads) bitmask_kernel(
                         (rq.w == HINM_REGION_DENSE ? (uint32_t)kAll << 24 : 0u);
     reinterpret_cast<uint32_t*>(keep)[q] = k4;
   }
-  __syncthreads();
+}
 
+// The tile's 2:4 group count from the counts (0 when they are not a valid split of K).
+__device__ __forceinline__ int groups_24(const int32_t* counts, int t, int K) {
   int n24 = counts[3 * t + 1];
   const int n0 = counts[3 * t], n4 = counts[3 * t + 2];
   if (n0 < 0 || n24 < 0 || n4 < 0 || n0 + n24 + n4 != K || (n24 & 3)) n24 = 0;
-  const int ng = n24 / 4;
-  const int32_t* mem = member + (size_t)t * K;
-  for (int g = threadIdx.x; g < ng; g += kMaskThreads) {
-    // the group's input channels, in ascending working position (k = 0..3)
-    const int4 cq = __ldg(reinterpret_cast<const int4*>(mem) + g);
-    const int cc[4] = {cq.x, cq.y, cq.z, cq.w};
-    int c[4];
-    float v[4][RB];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      c[k] = ((unsigned)cc[k] < (unsigned)K) ? cc[k] : 0;  // never index outside I
-      mask_load_rows<RB>(rows_s + (size_t)stage_slot(c[k]) * RB, v[k]);
-    }
-    // g_kl bit r: member l beats member k (k < l) in row r, i.e. v_l > v_k (equal values:
-    // the lower position k wins).  Member k is kept iff at most one member beats it: the
-    // negated majority of its three "beaten by" words, all rows at once.
-    uint32_t g01 = 0u, g02 = 0u, g03 = 0u, g12 = 0u, g13 = 0u, g23 = 0u;
-#pragma unroll
-    for (int r = 0; r < RB; ++r) {
-      g01 |= (uint32_t)(v[1][r] > v[0][r]) << r;
-      g02 |= (uint32_t)(v[2][r] > v[0][r]) << r;
-      g03 |= (uint32_t)(v[3][r] > v[0][r]) << r;
-      g12 |= (uint32_t)(v[2][r] > v[1][r]) << r;
-      g13 |= (uint32_t)(v[3][r] > v[1][r]) << r;
-      g23 |= (uint32_t)(v[3][r] > v[2][r]) << r;
-    }
-    auto maj = [](uint32_t a, uint32_t b, uint32_t c) { return (a & b) | (a & c) | (b & c); };
-    constexpr uint32_t kRows = (1u << RB) - 1u;
-    const uint32_t kb[4] = {~maj(g01, g02, g03) & kRows, ~maj(~g01, g12, g13) & kRows,
-                            ~maj(~g02, ~g12, g23) & kRows, ~maj(~g03, ~g13, ~g23) & kRows};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) keep[c[k]] = (uint8_t)kb[k];
-  }
-  __syncthreads();
+  return n24 / 4;
+}
 
-  uint32_t* out = bitmask + ((size_t)t * T + r0) * words;
+// The mask words of RB rows from their keep bytes (bit r of keep[c] = row r keeps channel
+// c): 32 words per warp and row by ballots, stored coalesced.
+template <int RB>
+__device__ __forceinline__ void write_words(const uint8_t* keep, int K, uint32_t* out) {
+  const int words = (K + 31) >> 5;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int nwarps = kMaskThreads / 32;
   for (int wb = warp * 32; wb < words; wb += nwarps * 32) {
     uint32_t mine[RB];
 #pragma unroll
@@ -216,12 +204,118 @@ __global__ void __launch_bounds__(kMaskThreads) bitmask_kernel(
   }
 }
 
+template <int RB>
+__global__ void __launch_bounds__(kMaskThreads) bitmask_kernel(
+    const ImpSrc src, const int8_t* __restrict__ region, const int32_t* __restrict__ counts,
+    const int32_t* __restrict__ member, int K, int T, uint32_t* __restrict__ bitmask) {
+  extern __shared__ __align__(16) uint8_t mask_smem[];
+  const int K8 = (K + 7) & ~7;
+  float* rows_s = reinterpret_cast<float*>(mask_smem);  // [K8][RB], stage_slot order
+  uint8_t* keep = mask_smem + (size_t)K8 * RB * sizeof(float);
+  const int words = (K + 31) >> 5;
+  const int t = blockIdx.y;
+  const int r0 = blockIdx.x * RB;  // first row of the chunk within the tile
+  const int8_t* reg = region + (size_t)t * K;
+  stage_rows_imp<RB, kMaskThreads>(src, (size_t)t * T + r0, K, rows_s);
+  keep_dense<RB>(reg, K, keep);
+  __syncthreads();
+
+  const int ng = groups_24(counts, t, K);
+  const int32_t* mem = member + (size_t)t * K;
+  for (int g = threadIdx.x; g < ng; g += kMaskThreads) {
+    // the group's input channels, in ascending working position (k = 0..3)
+    const int4 cq = __ldg(reinterpret_cast<const int4*>(mem) + g);
+    const int cc[4] = {cq.x, cq.y, cq.z, cq.w};
+    int c[4];
+    float v[4][RB];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      c[k] = ((unsigned)cc[k] < (unsigned)K) ? cc[k] : 0;  // never index outside I
+      mask_load_rows<RB>(rows_s + (size_t)stage_slot(c[k]) * RB, v[k]);
+    }
+    uint32_t kb[4];
+    group_keep<RB>(v, kb);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) keep[c[k]] = (uint8_t)kb[k];
+  }
+  __syncthreads();
+  write_words<RB>(keep, K, bitmask + ((size_t)t * T + r0) * words);
+}
+
+// The same mask from W without a materialized I: the chunk's RB rows of W (bf16) are copied
+// into shared memory as they are (cp.async, no conversion), and only the 2:4 groups'
+// members are turned into importances, fl32(fl32(w^2) s_c) as the importance kernels round
+// them, where they are compared; dense and pruned channels need no value.
+template <int RB>
+__global__ void __launch_bounds__(kMaskThreads) bitmask_w_kernel(
+    const uint16_t* __restrict__ W, const float* __restrict__ s_c,
+    const int8_t* __restrict__ region, const int32_t* __restrict__ counts,
+    const int32_t* __restrict__ member, int K, int T, uint32_t* __restrict__ bitmask) {
+  extern __shared__ __align__(16) uint8_t mask_smem[];
+  const int K8 = (K + 7) & ~7;  // row stride in shared memory (16-byte rows)
+  uint16_t* w_s = reinterpret_cast<uint16_t*>(mask_smem);  // [RB][K8]
+  uint8_t* keep = mask_smem + (size_t)RB * K8 * sizeof(uint16_t);
+  const int words = (K + 31) >> 5;
+  const int t = blockIdx.y;
+  const int r0 = blockIdx.x * RB;
+  const int8_t* reg = region + (size_t)t * K;
+  {
+    const uint32_t dst = ptx::smem_u32(w_s);
+    for (int a = 0; a < RB; ++a) {
+      const uint16_t* src = W + ((size_t)t * T + r0 + a) * K;
+      const uint32_t rd = dst + (uint32_t)(a * K8 * 2);
+      if ((K & 7) == 0) {
+        for (int q = threadIdx.x; q < (K >> 3); q += kMaskThreads) ptx::cp_async16(rd + 16 * q, src + 8 * q);
+      } else {
+        for (int q = threadIdx.x; q < (K >> 2); q += kMaskThreads) ptx::cp_async8(rd + 8 * q, src + 4 * q);
+      }
+    }
+  }
+  keep_dense<RB>(reg, K, keep);  // while the rows land
+  ptx::cp_async_commit_wait_all();
+  __syncthreads();
+
+  const int ng = groups_24(counts, t, K);
+  const int32_t* mem = member + (size_t)t * K;
+  for (int g = threadIdx.x; g < ng; g += kMaskThreads) {
+    const int4 cq = __ldg(reinterpret_cast<const int4*>(mem) + g);
+    const int cc[4] = {cq.x, cq.y, cq.z, cq.w};
+    int c[4];
+    float sk[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      c[k] = ((unsigned)cc[k] < (unsigned)K) ? cc[k] : 0;  // never index outside W
+      sk[k] = __ldg(s_c + c[k]);
+    }
+    float v[4][RB];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int r = 0; r < RB; ++r) v[k][r] = imp_from_w(w_s[r * K8 + c[k]], sk[k]);
+    uint32_t kb[4];
+    group_keep<RB>(v, kb);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) keep[c[k]] = (uint8_t)kb[k];
+  }
+  __syncthreads();
+  write_words<RB>(keep, K, bitmask + ((size_t)t * T + r0) * words);
+}
+
 // Rows per bitmask CTA: the largest power of two <= 8 whose rows fit in 96 KB of shared
 // memory (T is a multiple of it), so that wide rows (K ~ 11008) still get two per CTA.
 static int mask_rows(int K) {
   const size_t K8 = ((size_t)K + 7) & ~size_t(7);
   int rb = 8;
   while (rb > 1 && (size_t)rb * K8 * sizeof(float) > 96u * 1024u) rb >>= 1;
+  return rb;
+}
+
+// Rows per CTA of the W-path mask: the largest of 8, 4, 2 whose bf16 rows fit in 96 KB of
+// shared memory (K <= 16384 always fits 2).
+static int mask_rows_w(int K) {
+  const size_t K8 = ((size_t)K + 7) & ~size_t(7);
+  int rb = 8;
+  while (rb > 2 && (size_t)rb * K8 * sizeof(uint16_t) > 96u * 1024u) rb >>= 1;
   return rb;
 }
 
@@ -257,6 +351,23 @@ cudaError_t launch_mask(const ImpSrc& I, const int32_t* perm, long long perm_str
                                       status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (!I.I) {  // from W: rows copied as bf16, importances only for the compared members
+    const int RB = mask_rows_w(K);
+    const size_t smem = (size_t)RB * (((size_t)K + 7) & ~size_t(7)) * sizeof(uint16_t) + (size_t)K;
+    for (const void* fn : {(const void*)bitmask_w_kernel<2>, (const void*)bitmask_w_kernel<4>,
+                           (const void*)bitmask_w_kernel<8>}) {
+      e = set_max_dynamic_smem(fn, 96 * 1024 + kMaxK);
+      if (e != cudaSuccess) return e;
+    }
+    const dim3 g(T / RB, nt);
+    if (RB == 8)
+      bitmask_w_kernel<8><<<g, kMaskThreads, smem, s>>>(I.W, I.s, region, counts, member, K, T, bitmask);
+    else if (RB == 4)
+      bitmask_w_kernel<4><<<g, kMaskThreads, smem, s>>>(I.W, I.s, region, counts, member, K, T, bitmask);
+    else
+      bitmask_w_kernel<2><<<g, kMaskThreads, smem, s>>>(I.W, I.s, region, counts, member, K, T, bitmask);
+    return cudaGetLastError();
+  }
   const int RB = mask_rows(K);
   const size_t smem = (size_t)RB * (((size_t)K + 7) & ~size_t(7)) * sizeof(float) + (size_t)K;
   for (const void* fn : {(const void*)bitmask_kernel<1>, (const void*)bitmask_kernel<2>,
