@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include "hinm_internal.h"
+#include "ptx.cuh"
 
 namespace hinm {
 namespace {
@@ -112,48 +113,79 @@ __global__ void importance_kernel(const uint16_t* __restrict__ W, const float* _
 // I as importance_kernel computes it, and with it the boundary search's tile statistics:
 // V[t, c] = the fp64 sum of the tile's I[., c] over its rows in ascending order (the same
 // additions in the same order as the search's own vector scores), and tile_pmax[t] = the
-// exponent index p (value = m 2^(p-149)) of the tile's largest importance.  One thread per
-// (tile, 2 channels) walks the tile's rows; 32 rows' loads are in flight ahead of the
-// dependent fp64 chains.  tile_pmax must be 0 before the launch.
-constexpr int kStatRows = 32;  // T is a multiple of 32 (64 or 128)
+// exponent index p (value = m 2^(p-149)) of the tile's largest importance.  A CTA of 256
+// threads takes 512 channels of one tile; the tile's rows of W for them come into shared
+// memory 32 at a time by cp.async (two buffers: the next 32 rows land while these are
+// summed), and each thread walks its 2 channels down the rows in ascending order.
+// tile_pmax must be 0 before the launch.
+constexpr int kStatRows = 32;      // rows per buffer; T is a multiple of 32 (64 or 128)
+constexpr int kStatThreads = 256;  // 2 channels each: 512 channels (1 KB of a row) per CTA
+constexpr int kStatChans = 2 * kStatThreads;
+constexpr size_t kStatBufBytes = (size_t)kStatRows * kStatChans * sizeof(uint16_t);  // 32 KB
 
-__global__ void importance_stats_kernel(const uint16_t* __restrict__ W,
-                                        const float* __restrict__ s, int K, int T,
-                                        float* __restrict__ I, double* __restrict__ V,
-                                        int* __restrict__ tile_pmax) {
-  const int cp = blockIdx.x * blockDim.x + threadIdx.x;  // channel pair
+__global__ void __launch_bounds__(kStatThreads) importance_stats_kernel(
+    const uint16_t* __restrict__ W, const float* __restrict__ s, int K, int T,
+    float* __restrict__ I, double* __restrict__ V, int* __restrict__ tile_pmax) {
+  extern __shared__ __align__(16) uint8_t stat_smem[];  // [2][kStatRows][kStatChans] bf16
+  const int c_base = blockIdx.x * kStatChans;
   const int t = blockIdx.y;
-  uint32_t mb = 0;  // largest bit pattern = largest value (non-negative floats)
-  if (2 * cp < K) {
-    const int c0 = 2 * cp;
-    const float s0 = __ldg(s + c0), s1 = __ldg(s + c0 + 1);
-    const uint32_t* wp = reinterpret_cast<const uint32_t*>(W + (size_t)t * T * K + c0);
-    float2* ip = I ? reinterpret_cast<float2*>(I + (size_t)t * T * K + c0) : nullptr;
-    const size_t step = (size_t)K / 2;  // one row, in channel pairs
-    double v0 = 0.0, v1 = 0.0;
-    uint32_t wv[kStatRows], nx[kStatRows];
-#pragma unroll
-    for (int k = 0; k < kStatRows; ++k) wv[k] = __ldg(wp + (size_t)k * step);
-    for (int r0 = 0; r0 < T; r0 += kStatRows) {
-      if (r0 + kStatRows < T) {  // the next rows' loads in flight during these rows
-#pragma unroll
-        for (int k = 0; k < kStatRows; ++k) nx[k] = __ldg(wp + (size_t)(r0 + kStatRows + k) * step);
+  const int nch = min(kStatChans, K - c_base);  // channels of this CTA (a multiple of 4)
+  const uint16_t* wt = W + (size_t)t * T * K + c_base;
+  const uint32_t buf0 = ptx::smem_u32(stat_smem);
+  auto issue = [&](int r0, int b) {  // rows r0 .. r0 + 31 of the tile -> buffer b
+    const uint32_t dst = buf0 + (uint32_t)(b * kStatBufBytes);
+    if ((K & 7) == 0) {  // 16-byte pieces (8 channels), never straddling K
+      const int per_row = nch >> 3;
+      for (int q = threadIdx.x; q < kStatRows * per_row; q += kStatThreads) {
+        const int r = q / per_row, x = q - r * per_row;
+        ptx::cp_async16(dst + (uint32_t)(r * kStatChans * 2 + 16 * x),
+                        wt + (size_t)(r0 + r) * K + 8 * x);
       }
-#pragma unroll
+    } else {  // 8-byte pieces (4 channels)
+      const int per_row = nch >> 2;
+      for (int q = threadIdx.x; q < kStatRows * per_row; q += kStatThreads) {
+        const int r = q / per_row, x = q - r * per_row;
+        ptx::cp_async8(dst + (uint32_t)(r * kStatChans * 2 + 8 * x),
+                       wt + (size_t)(r0 + r) * K + 4 * x);
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  issue(0, 0);
+  if (kStatRows < T) issue(kStatRows, 1);
+
+  const int c0 = 2 * threadIdx.x;  // this thread's channel pair within the CTA
+  const bool mine = c0 < nch;
+  const float s0 = mine ? __ldg(s + c_base + c0) : 0.0f, s1 = mine ? __ldg(s + c_base + c0 + 1) : 0.0f;
+  float2* ip = (I && mine) ? reinterpret_cast<float2*>(I + (size_t)t * T * K + c_base + c0) : nullptr;
+  const size_t step = (size_t)K / 2;  // one row, in channel pairs
+  double v0 = 0.0, v1 = 0.0;
+  uint32_t mb = 0;  // largest bit pattern = largest value (non-negative floats)
+  for (int r0 = 0, b = 0; r0 < T; r0 += kStatRows, b ^= 1) {
+    // this buffer's copies have landed when at most the next buffer's group is pending
+    if (r0 + kStatRows < T) asm volatile("cp.async.wait_group 1;" ::: "memory");
+    else asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+    if (mine) {
+      const uint32_t* rows = reinterpret_cast<const uint32_t*>(stat_smem + b * kStatBufBytes) + threadIdx.x;
+#pragma unroll 8
       for (int k = 0; k < kStatRows; ++k) {  // rows ascending
-        const float w0 = __uint_as_float(wv[k] << 16), w1 = __uint_as_float(wv[k] & 0xFFFF0000u);
+        const uint32_t wv = rows[k * kStatThreads];
+        const float w0 = __uint_as_float(wv << 16), w1 = __uint_as_float(wv & 0xFFFF0000u);
         const float i0 = __fmul_rn(__fmul_rn(w0, w0), s0);
         const float i1 = __fmul_rn(__fmul_rn(w1, w1), s1);
-        if (I) __stcs(ip + (size_t)(r0 + k) * step, make_float2(i0, i1));
+        if (ip) __stcs(ip + (size_t)(r0 + k) * step, make_float2(i0, i1));
         v0 = __dadd_rn(v0, (double)i0);
         v1 = __dadd_rn(v1, (double)i1);
         mb = max(mb, max(__float_as_uint(i0), __float_as_uint(i1)));
       }
-#pragma unroll
-      for (int k = 0; k < kStatRows; ++k) wv[k] = nx[k];
     }
-    V[(size_t)t * K + c0] = v0;
-    V[(size_t)t * K + c0 + 1] = v1;
+    __syncthreads();  // buffer b is refilled next
+    if (r0 + 2 * kStatRows < T) issue(r0 + 2 * kStatRows, b);
+  }
+  if (mine) {
+    V[(size_t)t * K + c_base + c0] = v0;
+    V[(size_t)t * K + c_base + c0 + 1] = v1;
   }
   int pm = 0;
   if (mb) {
@@ -217,8 +249,11 @@ cudaError_t launch_importance_stats(const uint16_t* W, const uint16_t* X, int M,
       X, K, N, s_scratch, pmax, nt);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const dim3 g((K / 2 + 255) / 256, nt);
-  importance_stats_kernel<<<g, 256, 0, st>>>(W, s_scratch, K, T, I, V, pmax);
+  const size_t smem = 2 * kStatBufBytes;
+  e = set_max_dynamic_smem((const void*)importance_stats_kernel, (int)smem);
+  if (e != cudaSuccess) return e;
+  const dim3 g((K + kStatChans - 1) / kStatChans, nt);
+  importance_stats_kernel<<<g, kStatThreads, smem, st>>>(W, s_scratch, K, T, I, V, pmax);
   return cudaGetLastError();
 }
 
