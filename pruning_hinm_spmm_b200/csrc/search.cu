@@ -173,27 +173,31 @@ __global__ void vector_score_kernel(const ImpSrc src, int K, int T,
 // sums and the loads.
 constexpr int kColThreads = 256;
 
-// The rare values of a column (below the second level): exactly into the column's 128-bit
-// sum in shared memory (p >= lsb, owner thread only), else the flag.  Out of line, so that
-// the common path stays short.
-__device__ __noinline__ void col_rare(float x, int lsb, U128* xs, unsigned char* tn) {
-  uint32_t m;
-  int e;
-  split_f32(x, m, e);
-  if (!m) return;
-  if (e >= lsb) {
-    U128 v = *xs;
-    add_shifted(v, m, e - lsb);
-    *xs = v;
-  } else {
-    *tn = 1;
+// The rare values of a column (nonzero, below the second level) are only marked in the
+// main pass; a second, out-of-line pass over the column's rows adds them exactly into its
+// 128-bit sum in shared memory (p >= lsb, owner thread only) or sets the flag.  Both passes
+// take the same values, so each value is counted once.
+template <bool kW>
+struct ImpQuad;
+template <bool kW>
+__device__ __noinline__ void col_rare_pass(const ImpQuad<kW> col, size_t row0, int rows, int j,
+                                           float thr2, int lsb, U128* xs, unsigned char* tn) {
+  U128 v = *xs;
+  for (int i = 0; i < rows; ++i) {
+    const float x = col.value(col.load(row0 + i), j);
+    if (x >= thr2 || x == 0.0f) continue;
+    uint32_t m;
+    int e;
+    split_f32(x, m, e);
+    if (!m) continue;
+    if (e >= lsb) add_shifted(v, m, e - lsb);
+    else *tn = 1;
   }
+  *xs = v;
 }
 
 // Channels c .. c + 3 (c a multiple of 4) of one row: the raw load (kW: 4 bf16 of W, else
 // 4 fp32 of I), and value j of it as the importance.
-template <bool kW>
-struct ImpQuad;
 template <>
 struct ImpQuad<false> {
   using Raw = float4;
@@ -251,6 +255,7 @@ __global__ void __launch_bounds__(kColThreads, 3) column_sum_kernel(
   const float thr1 = __uint_as_float((uint32_t)(e1 + 1) << 23);  // smallest fp32 with p >= e1
   const float thr2 = __uint_as_float((uint32_t)(e2 + 1) << 23);
   double a1[4] = {0.0, 0.0, 0.0, 0.0}, a2[4] = {0.0, 0.0, 0.0, 0.0};
+  unsigned rare = 0u;  // bit j: channel c + j has values below the second level
   if (c < K) {  // K is a multiple of 4
     ImpQuad<kW> col;
     if constexpr (kW) {
@@ -279,12 +284,17 @@ __global__ void __launch_bounds__(kColThreads, 3) column_sum_kernel(
           } else if (x >= thr2) {
             a2[j] = __dadd_rn(a2[j], (double)x);
           } else if (x != 0.0f) {
-            col_rare(x, lsb, &xs[part][4 * q + j], &tn[part][4 * q + j]);
+            rare |= 1u << j;
           }
         }
       }
 #pragma unroll
       for (int k = 0; k < kBatch; ++k) v[k] = nx[k];
+    }
+    if (rare) {
+      for (int j = 0; j < 4; ++j)
+        if ((rare >> j) & 1u)
+          col_rare_pass<kW>(col, row0, rows, j, thr2, lsb, &xs[part][4 * q + j], &tn[part][4 * q + j]);
     }
   }
   // this range's total per channel, then the ranges in order
@@ -384,32 +394,35 @@ __global__ void __launch_bounds__(kRankChunk) chunk_sort_kernel(
 }
 
 // rank[t][j] = number of (key, index) pairs of the tile below position j's.  One CTA per
-// (tile, sorted chunk): thread i takes the i-th pair of its own sorted chunk (its rank within
-// the chunk is i) and adds, for every other chunk staged in shared memory, the number of that
-// chunk's pairs below it (binary search; consecutive threads hold increasing pairs, so their
-// searches follow nearly the same path).  The rank is then written at position j.
+// (tile, sorted chunk): all the tile's sorted chunks are copied into shared memory at once
+// (every load in flight together); thread i takes the i-th pair of its own chunk (its rank
+// within the chunk is i) and adds, for every other chunk, the number of that chunk's pairs
+// below it (binary search; consecutive threads hold increasing pairs, so their searches
+// follow nearly the same path).  The rank is then written at position j.
 __global__ void __launch_bounds__(kRankChunk) merge_rank_kernel(
     const unsigned long long* __restrict__ skey, const unsigned short* __restrict__ sidx, int K,
     int Kp, int32_t* __restrict__ rank) {
-  __shared__ unsigned long long ck[kRankChunk];
-  __shared__ unsigned short ci[kRankChunk];
+  extern __shared__ __align__(16) unsigned char merge_smem[];
+  unsigned long long* ck = reinterpret_cast<unsigned long long*>(merge_smem);  // [Kp]
+  unsigned short* ci = reinterpret_cast<unsigned short*>(ck + Kp);             // [Kp]
   const int t = blockIdx.y, own = blockIdx.x * kRankChunk;
-  const unsigned long long kj = __ldg(skey + (size_t)t * Kp + own + threadIdx.x);
-  const unsigned ij = __ldg(sidx + (size_t)t * Kp + own + threadIdx.x);
+  for (int q = threadIdx.x; q < Kp; q += kRankChunk) {
+    ck[q] = __ldg(skey + (size_t)t * Kp + q);
+    ci[q] = __ldg(sidx + (size_t)t * Kp + q);
+  }
+  __syncthreads();
+  const unsigned long long kj = ck[own + threadIdx.x];
+  const unsigned ij = ci[own + threadIdx.x];
   int r = threadIdx.x;
   for (int base = 0; base < Kp; base += kRankChunk) {
     if (base == own) continue;  // uniform over the CTA
-    ck[threadIdx.x] = __ldg(skey + (size_t)t * Kp + base + threadIdx.x);
-    ci[threadIdx.x] = __ldg(sidx + (size_t)t * Kp + base + threadIdx.x);
-    __syncthreads();
     int lo = 0, hi = kRankChunk;  // count of pairs < (kj, ij) in this sorted chunk
     while (lo < hi) {
       const int mid = (lo + hi) >> 1;
-      if (pair_less(ck[mid], ci[mid], kj, ij)) lo = mid + 1;
+      if (pair_less(ck[base + mid], ci[base + mid], kj, ij)) lo = mid + 1;
       else hi = mid;
     }
     r += lo;
-    __syncthreads();
   }
   if (ij < (unsigned)K) rank[(size_t)t * K + ij] = r;  // padding pairs carry index 0xFFFF
 }
@@ -454,7 +467,10 @@ cudaError_t launch_rank_sort(const double* V, const int32_t* perm, long long per
                                                             n64, zero32, n32);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  merge_rank_kernel<<<dim3(nchunk, nt), kRankChunk, 0, s>>>(skey, sidx, K, Kp, rank);
+  const size_t msmem = (size_t)Kp * (sizeof(unsigned long long) + sizeof(unsigned short));
+  e = set_max_dynamic_smem((const void*)merge_rank_kernel, (int)msmem);
+  if (e != cudaSuccess) return e;
+  merge_rank_kernel<<<dim3(nchunk, nt), kRankChunk, msmem, s>>>(skey, sidx, K, Kp, rank);
   return cudaGetLastError();
 }
 

@@ -135,3 +135,25 @@ def _same_used_blocks(La, Lb):
                  ("vals_sparse", ns_used), ("meta", ns_used), ("idx_sparse", ns_used),
                  ("run_sparse", ns_used)):
         assert torch.equal(getattr(La, f)[:n], getattr(Lb, f)[:n]), f
+
+
+def test_w_path_extreme_dynamic_range(H):
+    """Importances spanning more than 2^100 within a tile (weights near 1e-20): the values
+    below the column sums' two fp64 levels and below band_sum's fast path take the exact
+    128-bit and exponent-bucket paths, recomputed from W, and every R(m), the counts, the
+    ranks and the mask still match the oracle bit for bit."""
+    rng = np.random.default_rng(5)
+    M, K, N, T = 256, 256, 16, 128
+    scale = np.where(rng.random(K) < 0.3, 1e-20, 1.0).astype(np.float32)
+    Wf = (rng.standard_normal((M, K)).astype(np.float32) * scale[None, :])
+    Wf[:, :8] *= np.float32(1e-19)  # a few columns entirely in the tiny range
+    Wf[::7, 8:40] *= np.float32(1e-15)  # scattered values below the tile's window
+    Wf[::5, 40:72] *= np.float32(1e-9)  # and some 2^50-2^80 below the largest: 128-bit path
+    w = hi.Workload(name="extreme_w", M=M, K=K, N=N, T=T, W_bits=hi.f32_to_bf16_bits(Wf),
+                    X_bits=hi.f32_to_bf16_bits(rng.standard_normal((K, N)).astype(np.float32)),
+                    perm=rng.permutation(K).astype(np.int32), t_s=0.5, v_s=None)
+    I_ref = O.importance(w.W_bits, w.X_bits)
+    nz = I_ref[I_ref > 0].astype(np.float64)
+    assert np.log2(nz.max() / nz.min()) > 100   # really exercises the slow paths
+    g = _w_path(H, w, w.perm, None)
+    _against_oracle(w, w.perm, g)
