@@ -406,6 +406,37 @@ def time_dense_context(M, K, N, flush, stream, reps=10):
             "note": "dense W (no pruning) through cuBLAS, same M, K, N; context only"}
 
 
+def time_sparse24_context(M, K, N, flush, stream, reps=10):
+    """Context, not a target: torch's own 2:4 semi-structured product (torch.sparse's
+    to_sparse_semi_structured, whatever backend this torch build uses) on a random W with the
+    2:4 pattern, same M, K, N, one call per timing after the L2 flush, the median of `reps`.
+    Reported as unavailable, with the reason, when this torch build has no such kernel here."""
+    import torch
+    try:
+        from torch.sparse import to_sparse_semi_structured
+        keep = torch.tensor([1, 1, 0, 0], dtype=torch.bfloat16, device="cuda").repeat(M, K // 4)
+        A = to_sparse_semi_structured((torch.randn(M, K, device="cuda") * keep).to(torch.bfloat16))
+        B = torch.randn(K, N, device="cuda").to(torch.bfloat16)
+        torch.mm(A, B)
+        torch.cuda.synchronize()
+        ts = []
+        for i in range(reps + 2):
+            flush.fill_(i & 0xFF)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            torch.mm(A, B)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if i >= 2:
+                ts.append(e0.elapsed_time(e1) * 1e3)
+        t = float(np.median(ts))
+        return {"torch_semi_structured_24_us": t, "tflops_eff": 2.0 * M * K * N / (t * 1e-6) / 1e12,
+                "note": "torch's 2:4 semi-structured matmul, same M, K, N; context only"}
+    except Exception as ex:  # this torch build has no 2:4 kernel for this GPU
+        return {"torch_semi_structured_24": "unavailable",
+                "reason": f"{type(ex).__name__}: {str(ex)[:200]}"}
+
+
 def time_gyro(H, hp, W, X, perm, T, K, G=16, k=2, rounds=4):
     """The library's in-tile gyro rounds (host) on tile 0 of this step: its importance rows,
     its 2:4 band in working order (from the step's regions), `rounds` rounds of G sampled
@@ -479,7 +510,7 @@ def spmm_plan(N: int, T: int, tile_pairs: bool):
         return "spmm_kernel<128>", 128
     if tile_pairs and T == 128 and N >= 1024:
         return "spmm_pair_kernel", 240
-    return "spmm_kernel<256>", 256
+    return "spmm_kernel<192>", 192
 
 
 def l2_to_sm_bytes(M: int, N: int, T: int, counts, tile_pairs: bool) -> float:
@@ -862,6 +893,10 @@ def main():
                 "launches_per_step": mo["launches_per_step"],
                 "config": {"M": wo.M, "K": wo.K, "N": wo.N, "T": wo.T, "t_s": wo.t_s,
                            "v_s_used": wo.v_s, "counts_tile0": mo["counts"][0].tolist()}}
+            if oname == "pure24" and not args.no_next_rows:
+                others[wo.name]["context"] = {
+                    "dense": time_dense_context(wo.M, wo.K, wo.N, flush, stream),
+                    "semi_structured_24": time_sparse24_context(wo.M, wo.K, wo.N, flush, stream)}
             del mo
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
