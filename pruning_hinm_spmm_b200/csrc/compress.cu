@@ -15,6 +15,7 @@
 #include <cuda_runtime.h>
 
 #include "hinm_internal.h"
+#include "launch.cuh"
 #include "ptx.cuh"
 
 namespace hinm {
@@ -40,6 +41,7 @@ __device__ __forceinline__ void tile_blocks(const int32_t* counts, int t, int K,
 __global__ void __launch_bounds__(kTileInfoThreads) tile_info_kernel(
     const int32_t* __restrict__ counts, int nt, int K, int max_dense, int max_sparse,
     int32_t* __restrict__ info, int* status) {
+  ptx::enter_dependent();
   __shared__ int wd[32], ws[32];
   __shared__ int tot_d, tot_s;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -135,6 +137,7 @@ __global__ void __launch_bounds__(1024) slots_kernel(const int8_t* __restrict__ 
                                                      long long perm_stride,
                                                      const int32_t* __restrict__ counts, int K,
                                                      uint16_t* __restrict__ slots, int* status) {
+  ptx::enter_dependent();
   __shared__ int warp_tot[2][32];
   const int t = blockIdx.x;
   const int32_t* perm = perm_all ? perm_all + t * perm_stride : perm_all;  // this tile's order
@@ -248,6 +251,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint16_t* __restrict__ 
                                                    const uint32_t* __restrict__ bitmask,
                                                    const uint16_t* __restrict__ slots, int K,
                                                    int T, hinm_layout L, int* status) {
+  ptx::enter_dependent();
   __shared__ uint8_t nib[128][32];
   __shared__ int chan[kSparseBK];  // input channel of every vector of the block, -1 = padding
   const int t = blockIdx.y;
@@ -432,6 +436,7 @@ constexpr int kPackWarps = kPackThreads / 32;
 __global__ void __launch_bounds__(kPackThreads, 2) pack_rows_kernel(
     const uint16_t* __restrict__ W, const uint32_t* __restrict__ bitmask,
     const uint16_t* __restrict__ slots, int K, int T, int R, hinm_layout L, int* status) {
+  ptx::enter_dependent();
   extern __shared__ __align__(16) uint8_t sm[];
   const PackSmem lay = pack_smem(K, R);
   const uint16_t* chan = reinterpret_cast<const uint16_t*>(sm + lay.chan);
@@ -610,6 +615,7 @@ size_t compress_workspace_bytes(int M, int K, int T) {
 // outside [0, K) is reported as HINM_ERR_INVALID_ARG and written as 0.
 __global__ void __launch_bounds__(kSparseBK) translate_index_kernel(
     const int32_t* __restrict__ row_of_channel, int K, hinm_layout L, int* status) {
+  ptx::enter_dependent();
   __shared__ int first;
   const int t = blockIdx.y, b = blockIdx.x;
   const int nd = L.tile_info[4 * t + 0], ns = L.tile_info[4 * t + 1];
@@ -645,8 +651,8 @@ cudaError_t launch_translate_index(const hinm_layout& L, const int32_t* row_of_c
   const int nt = L.num_tiles, K = L.K;
   if (nt <= 0) return cudaSuccess;
   const int max_blocks = (K + kDenseBK - 1) / kDenseBK + (K + kSparseBK - 1) / kSparseBK;
-  translate_index_kernel<<<dim3(max_blocks, nt), kSparseBK, 0, s>>>(row_of_channel, K, L, status);
-  return cudaGetLastError();
+  return launch_kernel(translate_index_kernel, dim3(max_blocks, nt), kSparseBK, 0, s, nullptr,
+                       row_of_channel, K, L, status);
 }
 
 cudaError_t launch_compress(const uint16_t* W, const uint32_t* bitmask, const int8_t* region,
@@ -655,12 +661,11 @@ cudaError_t launch_compress(const uint16_t* W, const uint32_t* bitmask, const in
                             const hinm_layout& L, void* ws, int* status, cudaStream_t s) {
   const int nt = M / T;
   uint16_t* slots = static_cast<uint16_t*>(ws);
-  tile_info_kernel<<<1, kTileInfoThreads, 0, s>>>(counts, nt, K, L.max_dense_blocks,
-                                                  L.max_sparse_blocks, L.tile_info, status);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_kernel(tile_info_kernel, 1, kTileInfoThreads, 0, s, nullptr, counts, nt,
+                                K, L.max_dense_blocks, L.max_sparse_blocks, L.tile_info, status);
   if (e != cudaSuccess) return e;
-  slots_kernel<<<nt, 1024, 0, s>>>(region, perm, perm_stride, counts, K, slots, status);
-  e = cudaGetLastError();
+  e = launch_kernel(slots_kernel, nt, 1024, 0, s, nullptr, region, perm, perm_stride, counts, K,
+                    slots, status);
   if (e != cudaSuccess) return e;
   // Long rows (K > 8192) leave room for fewer rows per CTA than the staging needs to pay
   // off; there one CTA per (block, tile) gathers from L2 (measured on B200, K = 11008:
@@ -669,17 +674,15 @@ cudaError_t launch_compress(const uint16_t* W, const uint32_t* bitmask, const in
   if (K > 8192) {
     const int max_blocks = (K + kDenseBK - 1) / kDenseBK + (K + kSparseBK - 1) / kSparseBK;
     dim3 g(max_blocks, nt);
-    pack_kernel<<<g, 256, 0, s>>>(W, bitmask, slots, K, T, L, status);
-    return cudaGetLastError();
+    return launch_kernel(pack_kernel, g, 256, 0, s, nullptr, W, bitmask, slots, K, T, L, status);
   }
   const int R = pack_rows_per_cta(K);
   const size_t smem = pack_smem(K, R).total;
   e = set_max_dynamic_smem((const void*)pack_rows_kernel, (int)smem);
   if (e != cudaSuccess) return e;
   const dim3 g((kSparseBK + R - 1) / R, nt);  // every block row, also those past T
-  pack_rows_kernel<<<g, kPackThreads, smem, s>>>(W, bitmask, slots, K, T, R, L, status);
-  e = cudaGetLastError();
-  return e;
+  return launch_kernel(pack_rows_kernel, g, kPackThreads, smem, s, nullptr, W, bitmask, slots, K,
+                       T, R, L, status);
 }
 
 }  // namespace hinm

@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include "hinm_internal.h"
+#include "launch.cuh"
 #include "ptx.cuh"
 
 namespace hinm {
@@ -34,7 +35,8 @@ constexpr int kEnergyWarps = 8;
 // (the tile maxima that importance_stats_kernel raises with atomicMax)
 __global__ void __launch_bounds__(kEnergyWarps * 32) channel_energy_kernel(
     const uint16_t* __restrict__ X, int K, int N, float* __restrict__ s,
-    int* __restrict__ zero_int = nullptr, int n_zero = 0) {
+    int* __restrict__ zero_int, int n_zero) {
+  ptx::enter_dependent();
   if (zero_int)
     for (int x = blockIdx.x * blockDim.x + threadIdx.x; x < n_zero; x += gridDim.x * blockDim.x)
       zero_int[x] = 0;
@@ -79,6 +81,7 @@ constexpr int kQuads = 4;
 
 __global__ void importance_kernel(const uint16_t* __restrict__ W, const float* __restrict__ s,
                                   int M, int K, float* __restrict__ I) {
+  ptx::enter_dependent();
   const long long total4 = (long long)M * K / 4;
   const int k4 = K / 4;
   const long long stride = (long long)gridDim.x * blockDim.x;
@@ -127,6 +130,7 @@ __global__ void __launch_bounds__(kStatThreads) importance_stats_kernel(
     const uint16_t* __restrict__ W, const float* __restrict__ s, int K, int T,
     float* __restrict__ I, double* __restrict__ V, int* __restrict__ tile_pmax) {
   extern __shared__ __align__(16) uint8_t stat_smem[];  // [2][kStatRows][kStatChans] bf16
+  ptx::enter_dependent();
   const int c_base = blockIdx.x * kStatChans;
   const int t = blockIdx.y;
   const int nch = min(kStatChans, K - c_base);  // channels of this CTA (a multiple of 4)
@@ -245,32 +249,32 @@ cudaError_t launch_importance_stats(const uint16_t* W, const uint16_t* X, int M,
   double* V = static_cast<double*>(stats);
   int* pmax = reinterpret_cast<int*>(static_cast<char*>(stats) + tile_stats_v_bytes(M, K, T));
   // the energies' grid also clears the tile maxima (raised by importance_stats_kernel next)
-  channel_energy_kernel<<<(K + kEnergyWarps - 1) / kEnergyWarps, kEnergyWarps * 32, 0, st>>>(
-      X, K, N, s_scratch, pmax, nt);
-  cudaError_t e = cudaGetLastError();
+  const unsigned ge = (K + kEnergyWarps - 1) / kEnergyWarps;
+  cudaError_t e = launch_kernel(channel_energy_kernel, ge, kEnergyWarps * 32, 0, st, nullptr, X,
+                                K, N, s_scratch, pmax, nt);
   if (e != cudaSuccess) return e;
   const size_t smem = 2 * kStatBufBytes;
   e = set_max_dynamic_smem((const void*)importance_stats_kernel, (int)smem);
   if (e != cudaSuccess) return e;
   const dim3 g((K + kStatChans - 1) / kStatChans, nt);
-  importance_stats_kernel<<<g, kStatThreads, smem, st>>>(W, s_scratch, K, T, I, V, pmax);
-  return cudaGetLastError();
+  return launch_kernel(importance_stats_kernel, g, kStatThreads, smem, st, nullptr, W, s_scratch,
+                       K, T, I, V, pmax);
 }
 
 size_t importance_workspace_bytes(int K) { return ((size_t)K * sizeof(float) + 255) & ~size_t(255); }
 
 cudaError_t launch_importance(const uint16_t* W, const uint16_t* X, int M, int K, int N,
                               float* I, float* s_scratch, cudaStream_t st) {
-  channel_energy_kernel<<<(K + kEnergyWarps - 1) / kEnergyWarps, kEnergyWarps * 32, 0, st>>>(
-      X, K, N, s_scratch);
-  cudaError_t e = cudaGetLastError();
+  const unsigned ge = (K + kEnergyWarps - 1) / kEnergyWarps;
+  cudaError_t e = launch_kernel(channel_energy_kernel, ge, kEnergyWarps * 32, 0, st, nullptr, X,
+                                K, N, s_scratch, nullptr, 0);
   if (e != cudaSuccess) return e;
   const long long total4 = (long long)M * K / 4;
   long long blocks = (total4 + 255) / 256;
   const long long cap = (long long)sm_count() * 8;
   if (blocks > cap) blocks = cap;
-  importance_kernel<<<(unsigned)blocks, 256, 0, st>>>(W, s_scratch, M, K, I);
-  return cudaGetLastError();
+  return launch_kernel(importance_kernel, (unsigned)blocks, 256, 0, st, nullptr, W, s_scratch, M,
+                       K, I);
 }
 
 }  // namespace hinm

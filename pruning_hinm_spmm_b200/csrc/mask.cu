@@ -13,6 +13,7 @@
 #include <cuda_runtime.h>
 
 #include "hinm_internal.h"
+#include "launch.cuh"
 #include "ptx.cuh"
 #include "stage_rows.cuh"
 
@@ -52,6 +53,7 @@ __global__ void __launch_bounds__(1024) classify_kernel(const int32_t* __restric
                                                         int8_t* __restrict__ region,
                                                         int32_t* __restrict__ member,
                                                         int* status) {
+  ptx::enter_dependent();
   __shared__ int warp_tot[32];
   __shared__ int total;
   __shared__ uint32_t seen[kMaxK / 32];  // which channels this tile's order has named
@@ -208,6 +210,7 @@ template <int RB>
 __global__ void __launch_bounds__(kMaskThreads) bitmask_kernel(
     const ImpSrc src, const int8_t* __restrict__ region, const int32_t* __restrict__ counts,
     const int32_t* __restrict__ member, int K, int T, uint32_t* __restrict__ bitmask) {
+  ptx::enter_dependent();
   extern __shared__ __align__(16) uint8_t mask_smem[];
   const int K8 = (K + 7) & ~7;
   float* rows_s = reinterpret_cast<float*>(mask_smem);  // [K8][RB], stage_slot order
@@ -251,6 +254,7 @@ __global__ void __launch_bounds__(kMaskThreads) bitmask_w_kernel(
     const uint16_t* __restrict__ W, const float* __restrict__ s_c,
     const int8_t* __restrict__ region, const int32_t* __restrict__ counts,
     const int32_t* __restrict__ member, int K, int T, uint32_t* __restrict__ bitmask) {
+  ptx::enter_dependent();
   extern __shared__ __align__(16) uint8_t mask_smem[];
   const int K8 = (K + 7) & ~7;  // row stride in shared memory (16-byte rows)
   uint16_t* w_s = reinterpret_cast<uint16_t*>(mask_smem);  // [RB][K8]
@@ -347,9 +351,8 @@ cudaError_t launch_mask(const ImpSrc& I, const int32_t* perm, long long perm_str
     if (e != cudaSuccess) return e;
     rank = rank_ws;
   }
-  classify_kernel<<<nt, 1024, 0, s>>>(rank, perm, perm_stride, counts, K, region, member,
-                                      status);
-  e = cudaGetLastError();
+  e = launch_kernel(classify_kernel, nt, 1024, 0, s, nullptr, rank, perm, perm_stride, counts, K,
+                    region, member, status);
   if (e != cudaSuccess) return e;
   if (!I.I) {  // from W: rows copied as bf16, importances only for the compared members
     const int RB = mask_rows_w(K);
@@ -360,13 +363,9 @@ cudaError_t launch_mask(const ImpSrc& I, const int32_t* perm, long long perm_str
       if (e != cudaSuccess) return e;
     }
     const dim3 g(T / RB, nt);
-    if (RB == 8)
-      bitmask_w_kernel<8><<<g, kMaskThreads, smem, s>>>(I.W, I.s, region, counts, member, K, T, bitmask);
-    else if (RB == 4)
-      bitmask_w_kernel<4><<<g, kMaskThreads, smem, s>>>(I.W, I.s, region, counts, member, K, T, bitmask);
-    else
-      bitmask_w_kernel<2><<<g, kMaskThreads, smem, s>>>(I.W, I.s, region, counts, member, K, T, bitmask);
-    return cudaGetLastError();
+    auto kw = RB == 8 ? bitmask_w_kernel<8> : (RB == 4 ? bitmask_w_kernel<4> : bitmask_w_kernel<2>);
+    return launch_kernel(kw, g, kMaskThreads, smem, s, nullptr, I.W, I.s, region, counts, member,
+                         K, T, bitmask);
   }
   const int RB = mask_rows(K);
   const size_t smem = (size_t)RB * (((size_t)K + 7) & ~size_t(7)) * sizeof(float) + (size_t)K;
@@ -376,15 +375,10 @@ cudaError_t launch_mask(const ImpSrc& I, const int32_t* perm, long long perm_str
     if (e != cudaSuccess) return e;
   }
   const dim3 g(T / RB, nt);
-  if (RB == 8)
-    bitmask_kernel<8><<<g, kMaskThreads, smem, s>>>(I, region, counts, member, K, T, bitmask);
-  else if (RB == 4)
-    bitmask_kernel<4><<<g, kMaskThreads, smem, s>>>(I, region, counts, member, K, T, bitmask);
-  else if (RB == 2)
-    bitmask_kernel<2><<<g, kMaskThreads, smem, s>>>(I, region, counts, member, K, T, bitmask);
-  else
-    bitmask_kernel<1><<<g, kMaskThreads, smem, s>>>(I, region, counts, member, K, T, bitmask);
-  return cudaGetLastError();
+  auto ki = RB == 8 ? bitmask_kernel<8>
+                    : (RB == 4 ? bitmask_kernel<4> : (RB == 2 ? bitmask_kernel<2> : bitmask_kernel<1>));
+  return launch_kernel(ki, g, kMaskThreads, smem, s, nullptr, I, region, counts, member, K, T,
+                       bitmask);
 }
 
 }  // namespace hinm

@@ -36,6 +36,19 @@ __device__ __forceinline__ int perm_at(const int32_t* perm, int j, int K) {
   return (unsigned)c < (unsigned)K ? c : 0;
 }
 
+// ---------------------------------------------------------------- dependent launches
+// First statement of every kernel of the path (they are launched with programmatic stream
+// serialization, launch.cuh): wait until the kernels this one depends on have finished and
+// their writes are visible.  Every global access of the kernel comes after the wait, so the
+// accesses keep plain stream order; what overlaps is the launch of this kernel with the end
+// of the previous one.  Without a programmatic dependency the wait returns at once.
+// No kernel triggers its dependents early (griddepcontrol.launch_dependents): blocks of
+// the next kernel placed during this one's last wave crowd onto the SMs that are free at
+// that moment, which made the decode step slower (measured on B200: 414 -> 437 us).
+__device__ __forceinline__ void enter_dependent() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- cp.async (16-, 8-, 4-byte)
 // dst: shared-memory address, src: global; both aligned to the size.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {

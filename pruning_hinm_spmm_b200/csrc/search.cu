@@ -22,6 +22,7 @@
 #include <mutex>
 
 #include "hinm_internal.h"
+#include "launch.cuh"
 #include "ptx.cuh"
 #include "stage_rows.cuh"
 
@@ -122,6 +123,7 @@ __device__ __forceinline__ double pow2(int e) {
 // I (fp64), and the tile's largest exponent P.
 __global__ void vector_score_kernel(const ImpSrc src, int K, int T,
                                     double* __restrict__ Vc, int* __restrict__ tile_pmax) {
+  ptx::enter_dependent();
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   const int t = blockIdx.y;
   int pm = 0;
@@ -238,6 +240,7 @@ template <int kBatch, int kSplit, bool kW>
 __global__ void __launch_bounds__(kColThreads, 3) column_sum_kernel(
     const ImpSrc src, int K, int T, const int* __restrict__ tile_pmax,
     U128* __restrict__ colsum, unsigned char* __restrict__ coltiny) {
+  ptx::enter_dependent();
   constexpr int kQuads = kColThreads / kSplit;  // channel quads per CTA
   __shared__ U128 xs[kSplit][kQuads * 4];
   __shared__ unsigned char tn[kSplit][kQuads * 4];
@@ -344,6 +347,7 @@ __global__ void __launch_bounds__(kRankChunk) chunk_sort_kernel(
     int K, int Kp,
     unsigned long long* __restrict__ skey, unsigned short* __restrict__ sidx,
     unsigned long long* __restrict__ zero64, size_t n64, int* __restrict__ zero32, size_t n32) {
+  ptx::enter_dependent();
   __shared__ unsigned long long key_s[kRankChunk];
   __shared__ unsigned short idx_s[kRankChunk];
   {
@@ -402,6 +406,7 @@ __global__ void __launch_bounds__(kRankChunk) chunk_sort_kernel(
 __global__ void __launch_bounds__(kRankChunk) merge_rank_kernel(
     const unsigned long long* __restrict__ skey, const unsigned short* __restrict__ sidx, int K,
     int Kp, int32_t* __restrict__ rank) {
+  ptx::enter_dependent();
   extern __shared__ __align__(16) unsigned char merge_smem[];
   unsigned long long* ck = reinterpret_cast<unsigned long long*>(merge_smem);  // [Kp]
   unsigned short* ci = reinterpret_cast<unsigned short*>(ck + Kp);             // [Kp]
@@ -445,8 +450,7 @@ cudaError_t launch_vector_scores(const ImpSrc& I, int M, int K, int T, double* V
   cudaError_t e = cudaMemsetAsync(tile_pmax, 0, (size_t)nt * sizeof(int), s);
   if (e != cudaSuccess) return e;
   dim3 g1((K + 255) / 256, nt);
-  vector_score_kernel<<<g1, 256, 0, s>>>(I, K, T, V, tile_pmax);
-  return cudaGetLastError();
+  return launch_kernel(vector_score_kernel, g1, 256, 0, s, nullptr, I, K, T, V, tile_pmax);
 }
 
 // The ranking from V: chunk sort, then merge.
@@ -462,16 +466,14 @@ cudaError_t launch_rank_sort(const double* V, const int32_t* perm, long long per
   Carve c{static_cast<char*>(scratch), 0};
   unsigned long long* skey = c.take<unsigned long long>((size_t)nt * Kp);
   unsigned short* sidx = c.take<unsigned short>((size_t)nt * Kp);
-  chunk_sort_kernel<<<dim3(nchunk, nt), kRankChunk, 0, s>>>(V, perm, perm_stride, K, Kp, skey,
-                                                             sidx, zero64,
-                                                            n64, zero32, n32);
-  e = cudaGetLastError();
+  e = launch_kernel(chunk_sort_kernel, dim3(nchunk, nt), kRankChunk, 0, s, nullptr, V, perm,
+                    perm_stride, K, Kp, skey, sidx, zero64, n64, zero32, n32);
   if (e != cudaSuccess) return e;
   const size_t msmem = (size_t)Kp * (sizeof(unsigned long long) + sizeof(unsigned short));
   e = set_max_dynamic_smem((const void*)merge_rank_kernel, (int)msmem);
   if (e != cudaSuccess) return e;
-  merge_rank_kernel<<<dim3(nchunk, nt), kRankChunk, msmem, s>>>(skey, sidx, K, Kp, rank);
-  return cudaGetLastError();
+  return launch_kernel(merge_rank_kernel, dim3(nchunk, nt), kRankChunk, msmem, s, nullptr, skey,
+                       sidx, K, Kp, rank);
 }
 
 // A second stream per device for work that can run beside the caller's stream (forked and
@@ -610,6 +612,7 @@ __global__ void __launch_bounds__(512, 2) candidate_lists_kernel(
     const unsigned char* __restrict__ coltiny, int K, int T, CandidateList cl, int ncand,
     unsigned short* __restrict__ band, U128* __restrict__ rdense,
     unsigned long long* __restrict__ bucket, int* __restrict__ bucket_used) {
+  ptx::enter_dependent();
   __shared__ int warp_tot[16];
   __shared__ U128 warp_acc[16];
   const int m = blockIdx.x, t = blockIdx.y;
@@ -779,6 +782,7 @@ __global__ void __launch_bounds__(kThreads) band_sum_kernel(
     const int* __restrict__ tile_pmax, int K, int T, CandidateList cl, int ncand,
     U128* __restrict__ part, unsigned long long* __restrict__ bucket,
     int* __restrict__ bucket_used) {
+  ptx::enter_dependent();
   extern __shared__ __align__(16) float rows_s[];  // [K rounded up to 8][RB], stage_slot order
   __shared__ unsigned long long fast_sum[kMaxCandidates];   // units of 2^(eb - 149)
   __shared__ unsigned long long digits[kMaxCandidates][4];  // slow path, units of 2^(lsb - 149)
@@ -918,6 +922,7 @@ __global__ void finalize_kernel(const U128* __restrict__ rdense, const U128* __r
                                 const int* __restrict__ tile_pmax, int ncand, CandidateList cl,
                                 double t_s, double alpha, double* __restrict__ R,
                                 int32_t* __restrict__ counts, double* __restrict__ vs) {
+  ptx::enter_dependent();
   __shared__ double Rs[kMaxCandidates];
   const int t = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -1042,18 +1047,11 @@ cudaError_t launch_boundary_search(const ImpSrc& I, const void* stats, const int
     if (e != cudaSuccess) return e;
     // a CTA per (tile, 256 channels); T = 64 splits its rows in 2, T = 128 in 4
     const dim3 gc((K + 255) / 256, nt);
-    if (I.I) {  // from I: 16-byte loads, 4 rows in flight
-      if (T == 128)
-        column_sum_kernel<4, 4, false><<<gc, kColThreads, 0, ss->stream>>>(I, K, T, pmax, colsum, coltiny);
-      else
-        column_sum_kernel<4, 2, false><<<gc, kColThreads, 0, ss->stream>>>(I, K, T, pmax, colsum, coltiny);
-    } else {  // from W: 8-byte loads, 8 rows in flight
-      if (T == 128)
-        column_sum_kernel<8, 4, true><<<gc, kColThreads, 0, ss->stream>>>(I, K, T, pmax, colsum, coltiny);
-      else
-        column_sum_kernel<8, 2, true><<<gc, kColThreads, 0, ss->stream>>>(I, K, T, pmax, colsum, coltiny);
-    }
-    e = cudaGetLastError();
+    auto col = I.I ? (T == 128 ? column_sum_kernel<4, 4, false> : column_sum_kernel<4, 2, false>)
+                   : (T == 128 ? column_sum_kernel<8, 4, true> : column_sum_kernel<8, 2, true>);
+    // from I: 16-byte loads, 4 rows in flight; from W: 8-byte loads, 8 rows in flight
+    e = launch_kernel(col, gc, kColThreads, 0, ss->stream, nullptr, I, K, T, pmax, colsum,
+                      coltiny);
     if (e != cudaSuccess) return e;
     e = cudaEventRecord(ss->join, ss->stream);
     if (e != cudaSuccess) return e;
@@ -1069,17 +1067,11 @@ cudaError_t launch_boundary_search(const ImpSrc& I, const void* stats, const int
   {
     const dim3 gl(ncand, nt);
     const int per = (K + 511) / 512;
-    if (per <= 8)
-      candidate_lists_kernel<8><<<gl, 512, 0, s>>>(I, perm, perm_stride, rank, pmax, colsum, coltiny, K, T, cl,
-                                                   ncand, band, rdense, bucket, bucket_used);
-    else if (per <= 16)
-      candidate_lists_kernel<16><<<gl, 512, 0, s>>>(I, perm, perm_stride, rank, pmax, colsum, coltiny, K, T, cl,
-                                                    ncand, band, rdense, bucket, bucket_used);
-    else
-      candidate_lists_kernel<32><<<gl, 512, 0, s>>>(I, perm, perm_stride, rank, pmax, colsum, coltiny, K, T, cl,
-                                                    ncand, band, rdense, bucket, bucket_used);
+    auto lists = per <= 8 ? candidate_lists_kernel<8>
+                          : (per <= 16 ? candidate_lists_kernel<16> : candidate_lists_kernel<32>);
+    e = launch_kernel(lists, gl, 512, 0, s, nullptr, I, perm, perm_stride, rank, pmax, colsum,
+                      coltiny, K, T, cl, ncand, band, rdense, bucket, bucket_used);
   }
-  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t smem = (size_t)RB * (((size_t)K + 7) & ~size_t(7)) * sizeof(float);
   for (const void* fn : {(const void*)band_sum_kernel<1, 512>, (const void*)band_sum_kernel<2, 512>,
@@ -1088,20 +1080,13 @@ cudaError_t launch_boundary_search(const ImpSrc& I, const void* stats, const int
     if (e != cudaSuccess) return e;
   }
   const dim3 gb(nchunks, nt);
-  if (RB == 4)
-    band_sum_kernel<4, 512><<<gb, 512, smem, s>>>(I, band, pmax, K, T, cl, ncand, part, bucket,
-                                                  bucket_used);
-  else if (RB == 2)
-    band_sum_kernel<2, 512><<<gb, 512, smem, s>>>(I, band, pmax, K, T, cl, ncand, part, bucket,
-                                                  bucket_used);
-  else
-    band_sum_kernel<1, 512><<<gb, 512, smem, s>>>(I, band, pmax, K, T, cl, ncand, part, bucket,
-                                                  bucket_used);
-  e = cudaGetLastError();
+  auto sum = RB == 4 ? band_sum_kernel<4, 512>
+                     : (RB == 2 ? band_sum_kernel<2, 512> : band_sum_kernel<1, 512>);
+  e = launch_kernel(sum, gb, 512, smem, s, nullptr, I, band, pmax, K, T, cl, ncand, part, bucket,
+                    bucket_used);
   if (e != cudaSuccess) return e;
-  finalize_kernel<<<nt, 1024, 0, s>>>(rdense, part, nchunks, bucket, bucket_used, pmax, ncand, cl,
-                                    t_s, alpha, R, counts_out, vs_out);
-  return cudaGetLastError();
+  return launch_kernel(finalize_kernel, nt, 1024, 0, s, nullptr, rdense, part, nchunks, bucket,
+                       bucket_used, pmax, ncand, cl, t_s, alpha, R, counts_out, vs_out);
 }
 
 }  // namespace hinm

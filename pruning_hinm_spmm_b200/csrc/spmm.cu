@@ -45,6 +45,7 @@
 #include <mutex>
 
 #include "hinm_internal.h"
+#include "launch.cuh"
 #include "ptx.cuh"
 
 namespace hinm {
@@ -262,6 +263,7 @@ __global__ void __launch_bounds__(SpmmCfg<BN, SPLIT>::kThreads, 1)
     spmm_kernel(const __grid_constant__ CUtensorMap tmX, const SpmmArgs a) {
   using C = SpmmCfg<BN, SPLIT>;
   extern __shared__ uint8_t smem_raw[];
+  ptx::enter_dependent();
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* idx_region = smem + C::kStages * C::kStageBytes;  // [S][kIdxBytes]
@@ -789,6 +791,7 @@ __global__ void __launch_bounds__(320, 1)
   using C = PairCfg;
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
+  ptx::enter_dependent();
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* idx_region = smem + C::kStages * C::kStageBytes;  // [S][kIdxBytes]
@@ -1242,23 +1245,17 @@ cudaError_t run(const hinm_layout& L, const uint16_t* X, int N, const SpmmOut& o
              status,      o.bias,       o.act,         o.Yb};
   if constexpr (!SPLIT) {
     const int grid = units < num_sms() ? units : num_sms();
-    spmm_kernel<BN, false><<<grid, C::kThreads, C::kSmemBytes, s>>>(map, a);
-    return cudaGetLastError();
+    return launch_kernel(spmm_kernel<BN, false>, grid, C::kThreads, C::kSmemBytes, s, nullptr,
+                         map, a);
   } else {
     // one cluster of `split` CTAs per unit
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(units * split), 1, 1);
-    cfg.blockDim = dim3(C::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = C::kSmemBytes;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)split;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, spmm_kernel<BN, true>, map, a);
+    cudaLaunchAttribute cluster;
+    cluster.id = cudaLaunchAttributeClusterDimension;
+    cluster.val.clusterDim.x = (unsigned)split;
+    cluster.val.clusterDim.y = 1;
+    cluster.val.clusterDim.z = 1;
+    return launch_kernel(spmm_kernel<BN, true>, (unsigned)(units * split), C::kThreads,
+                         C::kSmemBytes, s, &cluster, map, a);
   }
 }
 
@@ -1280,8 +1277,8 @@ cudaError_t run_pair(const hinm_layout& L, const uint16_t* X, int N, const SpmmO
              L.num_tiles, nblk_n,       units,         1,        x3d ? 1 : 0, status,
              o.bias,      o.act,        o.Yb};
   const int grid = units < num_sms() ? units : num_sms();
-  spmm_pair_kernel<<<grid, C::kThreads, C::kSmemBytes, s>>>(map3, map2, a);
-  return cudaGetLastError();
+  return launch_kernel(spmm_pair_kernel, grid, C::kThreads, C::kSmemBytes, s, nullptr, map3, map2,
+                       a);
 }
 
 // Split-K when the units (tile x column block) fill less than half of the SMs: each unit's
