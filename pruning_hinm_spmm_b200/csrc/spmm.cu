@@ -293,21 +293,24 @@ __global__ void __launch_bounds__(SpmmCfg<BN, SPLIT>::kThreads, 1)
     kb0 = SPLIT ? (int)((long long)nblk * rank / a.split) : 0;
     kb1 = SPLIT ? (int)((long long)nblk * (rank + 1) / a.split) : nblk;
   };
-  // The first unit's tile record, and for the bulk-copy thread its first block's run flag,
-  // are loaded before the set-up below, so that their latency overlaps it.
+  // Run flag of K-block kb of a tile with record info (the bulk-copy warp's lanes load 32
+  // consecutive blocks' flags at once).
+  auto run_flag = [&](const int4& info, int kb) {
+    const bool sparse = kb >= info.x;
+    const size_t blk = sparse ? (size_t)(info.w + kb - info.x) : (size_t)(info.z + kb);
+    return __ldg(sparse ? a.run_sparse + blk : a.run_dense + blk);
+  };
+  // The first unit's tile record, and for the bulk-copy warp the run flags of its first 32
+  // K-blocks (one per lane), are loaded before the set-up below, so that their latency
+  // overlaps it.
   int4 info_first = make_int4(0, 0, 0, 0);
   int run_first = -1;
   if (u_first < a.num_units) {
     info_first = __ldg(reinterpret_cast<const int4*>(a.tile_info) + u_first / a.nblk_n);
-    if (warp == C::kBulkWarp && lane == 0) {
+    if (warp == C::kBulkWarp) {
       int kb0, kb1;
       k_range(info_first.x + info_first.y, kb0, kb1);
-      if (kb0 < kb1) {
-        const bool sparse = kb0 >= info_first.x;
-        const size_t blk = sparse ? (size_t)(info_first.w + kb0 - info_first.x)
-                                  : (size_t)(info_first.z + kb0);
-        run_first = __ldg(sparse ? a.run_sparse + blk : a.run_dense + blk);
-      }
+      if (kb0 + lane < kb1) run_first = run_flag(info_first, kb0 + lane);
     }
   }
   auto tile_info_of = [&](int u, int tile) {
@@ -409,80 +412,93 @@ __global__ void __launch_bounds__(SpmmCfg<BN, SPLIT>::kThreads, 1)
     // One thread runs ahead of the gather warps by up to a full ring: per K-block, once the
     // stage is free, it publishes the block's run flag and index list (index-ready barrier)
     // and bulk-copies the pre-swizzled A block, its metadata and, for a contiguous run, the
-    // X rows by TMA (full barrier).
-    if (lane == 0) {
-      uint32_t it = 0;
-      bool stop = false;
-      for (int u = u_first; u < a.num_units && !stop; u += u_step) {
-        const int tile = u / a.nblk_n, n0 = (u - tile * a.nblk_n) * BN;
-        const int4 info = tile_info_of(u, tile);
-        const int nd = info.x, nblk = info.x + info.y;
-        int kb0, kb1;
-        k_range(nblk, kb0, kb1);
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const bool sparse = kb >= nd;
-          const size_t blk = sparse ? (size_t)(info.w + kb - nd) : (size_t)(info.z + kb);
-          const int run = (u == u_first && kb == kb0)
-                              ? run_first
-                              : __ldg(sparse ? a.run_sparse + blk : a.run_dense + blk);
-          const int s = it % C::kStages;
-          const uint32_t ph = (it / C::kStages) & 1;
-          if (!ptx::mbar_wait(empty_bar(s), ph ^ 1, a.status, abort_flag)) {
-            stop = true;
-            break;
-          }
-          const uint32_t A_s = ptx::smem_u32(smem + s * C::kStageBytes);
-          const uint32_t B_s = A_s + C::kABytes;
-          const uint32_t E_s = B_s + C::kBBytes;
-          const uint32_t I_s = ptx::smem_u32(idx_region + s * C::kIdxBytes);
-          const int rows = sparse ? kSparseBK : kDenseBK;
-          run_s[s] = run;  // published by the arrive below (release)
-          if (run < 0) {
-            ptx::mbar_arrive_expect_tx(idx_bar(s), (uint32_t)rows * 4u);
-            ptx::bulk_g2s(I_s, sparse ? a.idx_sparse + blk * kSparseBK : a.idx_dense + blk * kDenseBK,
-                          (uint32_t)rows * 4u, idx_bar(s));
-          } else {
-            ptx::mbar_arrive(idx_bar(s));
-          }
-          // with kSplitB the full barrier takes A, metadata and the first 64 rows of X; the
-          // second-half barrier the rest of a run's rows (none for a dense block or a gather)
-          const int rows1 = C::kSplitB ? 64 : rows;
-          const uint32_t bytes = C::kABytes + (sparse ? C::kEBytes : 0) +
-                                 (run >= 0 ? (uint32_t)rows1 * BN * 2u : 0u);
-          ptx::mbar_arrive_expect_tx(full_bar(s), bytes);
-          if constexpr (C::kSplitB)
-            ptx::mbar_arrive_expect_tx(full2_bar(s),
-                                       run >= 0 ? (uint32_t)(rows - rows1) * BN * 2u : 0u);
-          ptx::bulk_g2s(A_s, (sparse ? a.vals_sparse : a.vals_dense) + blk * 8192, C::kABytes,
-                        full_bar(s));
-          if (sparse) ptx::bulk_g2s(E_s, a.meta + blk * kMetaWords, C::kEBytes, full_bar(s));
-          if (run >= 0) {
-            // one ascending run of X rows: per half of 64 rows, one 3-D box over all the
-            // column atoms, or one 2-D box per atom
-#pragma unroll 1
-            for (int h = 0; h < rows / 64; ++h) {
-              const uint32_t fb = (C::kSplitB && h == 1) ? full2_bar(s) : full_bar(s);
-              if (a.x3d) {
-                ptx::tma_load_3d(B_s + h * C::kBHalfBytes, &tmX, 0, run + h * 64, n0 / C::kAtom,
-                                 fb);
+    // X rows by TMA (full barrier).  The warp's lanes load the run flags of 32 blocks at a
+    // time, so the issuing thread does not wait for one global load per block (with few
+    // MMAs per stage, as at N = 16, that wait bounded the rate at which stages refilled).
+    uint32_t it = 0;
+    bool stop = false;
+    for (int u = u_first; u < a.num_units && !stop; u += u_step) {
+      const int tile = u / a.nblk_n, n0 = (u - tile * a.nblk_n) * BN;
+      const int4 info = tile_info_of(u, tile);
+      const int nd = info.x, nblk = info.x + info.y;
+      int kb0, kb1;
+      k_range(nblk, kb0, kb1);
+      for (int base = kb0; base < kb1 && !stop; base += 32) {
+        int run_l = -1;
+        if (u == u_first && base == kb0)
+          run_l = run_first;
+        else if (base + lane < kb1)
+          run_l = run_flag(info, base + lane);
+        const int nb = min(32, kb1 - base);
+        for (int q = 0; q < nb; ++q, ++it) {
+          const int run = __shfl_sync(0xffffffffu, run_l, q);
+          int ok = 1;
+          if (lane == 0) {
+            const int kb = base + q;
+            const bool sparse = kb >= nd;
+            const size_t blk = sparse ? (size_t)(info.w + kb - nd) : (size_t)(info.z + kb);
+            const int s = it % C::kStages;
+            const uint32_t ph = (it / C::kStages) & 1;
+            ok = ptx::mbar_wait(empty_bar(s), ph ^ 1, a.status, abort_flag) ? 1 : 0;
+            if (ok) {
+              const uint32_t A_s = ptx::smem_u32(smem + s * C::kStageBytes);
+              const uint32_t B_s = A_s + C::kABytes;
+              const uint32_t E_s = B_s + C::kBBytes;
+              const uint32_t I_s = ptx::smem_u32(idx_region + s * C::kIdxBytes);
+              const int rows = sparse ? kSparseBK : kDenseBK;
+              run_s[s] = run;  // published by the arrive below (release)
+              if (run < 0) {
+                ptx::mbar_arrive_expect_tx(idx_bar(s), (uint32_t)rows * 4u);
+                ptx::bulk_g2s(I_s, sparse ? a.idx_sparse + blk * kSparseBK : a.idx_dense + blk * kDenseBK,
+                              (uint32_t)rows * 4u, idx_bar(s));
               } else {
+                ptx::mbar_arrive(idx_bar(s));
+              }
+              // with kSplitB the full barrier takes A, metadata and the first 64 rows of X; the
+              // second-half barrier the rest of a run's rows (none for a dense block or a gather)
+              const int rows1 = C::kSplitB ? 64 : rows;
+              const uint32_t bytes = C::kABytes + (sparse ? C::kEBytes : 0) +
+                                     (run >= 0 ? (uint32_t)rows1 * BN * 2u : 0u);
+              ptx::mbar_arrive_expect_tx(full_bar(s), bytes);
+              if constexpr (C::kSplitB)
+                ptx::mbar_arrive_expect_tx(full2_bar(s),
+                                           run >= 0 ? (uint32_t)(rows - rows1) * BN * 2u : 0u);
+              ptx::bulk_g2s(A_s, (sparse ? a.vals_sparse : a.vals_dense) + blk * 8192, C::kABytes,
+                            full_bar(s));
+              if (sparse) ptx::bulk_g2s(E_s, a.meta + blk * kMetaWords, C::kEBytes, full_bar(s));
+              if (run >= 0) {
+                // one ascending run of X rows: per half of 64 rows, one 3-D box over all the
+                // column atoms, or one 2-D box per atom
 #pragma unroll 1
-                for (int at = 0; at < BN / C::kAtom; ++at)
-                  ptx::tma_load_2d(B_s + h * C::kBHalfBytes + at * C::kBAtomStride, &tmX,
-                                   n0 + at * C::kAtom, run + h * 64, fb);
+                for (int h = 0; h < rows / 64; ++h) {
+                  const uint32_t fb = (C::kSplitB && h == 1) ? full2_bar(s) : full_bar(s);
+                  if (a.x3d) {
+                    ptx::tma_load_3d(B_s + h * C::kBHalfBytes, &tmX, 0, run + h * 64, n0 / C::kAtom,
+                                     fb);
+                  } else {
+#pragma unroll 1
+                    for (int at = 0; at < BN / C::kAtom; ++at)
+                      ptx::tma_load_2d(B_s + h * C::kBHalfBytes + at * C::kBAtomStride, &tmX,
+                                       n0 + at * C::kAtom, run + h * 64, fb);
+                  }
+                }
               }
             }
           }
+          if (!__shfl_sync(0xffffffffu, ok, 0)) {
+            stop = true;
+            break;
+          }
         }
       }
-      if (*abort_flag) {
-        // wait (bounded) for the bulk / tensor copies of the last stages
-        for (uint32_t k = (it > (uint32_t)C::kStages ? it - C::kStages : 0u); k < it; ++k) {
-          ptx::mbar_wait(idx_bar(k % C::kStages), (k / C::kStages) & 1, a.status, nullptr);
-          ptx::mbar_wait(full_bar(k % C::kStages), (k / C::kStages) & 1, a.status, nullptr);
-          if constexpr (C::kSplitB)
-            ptx::mbar_wait(full2_bar(k % C::kStages), (k / C::kStages) & 1, a.status, nullptr);
-        }
+    }
+    if (lane == 0 && *abort_flag) {
+      // wait (bounded) for the bulk / tensor copies of the last stages
+      for (uint32_t k = (it > (uint32_t)C::kStages ? it - C::kStages : 0u); k < it; ++k) {
+        ptx::mbar_wait(idx_bar(k % C::kStages), (k / C::kStages) & 1, a.status, nullptr);
+        ptx::mbar_wait(full_bar(k % C::kStages), (k / C::kStages) & 1, a.status, nullptr);
+        if constexpr (C::kSplitB)
+          ptx::mbar_wait(full2_bar(k % C::kStages), (k / C::kStages) & 1, a.status, nullptr);
       }
     }
     __syncwarp();
