@@ -179,8 +179,11 @@ int* device_status_ptr() {
 }
 
 namespace {
+// A function attribute lives in the module of one context: a re-created context (after
+// cudaDeviceReset) starts without it, so the record is kept per device and context.
 struct SmemAttr {
   int dev;
+  void* ctx;
   const void* fn;
   int bytes;  // the largest limit set so far
 };
@@ -194,15 +197,18 @@ cudaError_t set_max_dynamic_smem(const void* fn, int bytes) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lk(g_attr_mu);
+  void* ctx = current_context();
   int slot = -1;
   for (int i = 0; i < g_attr_count; ++i)
-    if (g_attr_done[i].dev == dev && g_attr_done[i].fn == fn) slot = i;
-  if (slot >= 0 && g_attr_done[slot].bytes >= bytes) return cudaSuccess;
+    if (g_attr_done[i].dev == dev && g_attr_done[i].ctx == ctx && g_attr_done[i].fn == fn)
+      slot = i;
+  if (ctx && slot >= 0 && g_attr_done[slot].bytes >= bytes) return cudaSuccess;
   e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
+  if (!ctx) return cudaSuccess;  // no context known: set again on every call
   if (slot >= 0) g_attr_done[slot].bytes = bytes;
   else if (g_attr_count < (int)(sizeof(g_attr_done) / sizeof(g_attr_done[0])))
-    g_attr_done[g_attr_count++] = SmemAttr{dev, fn, bytes};
+    g_attr_done[g_attr_count++] = SmemAttr{dev, ctx, fn, bytes};
   return cudaSuccess;
 }
 
