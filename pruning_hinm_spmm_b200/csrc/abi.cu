@@ -108,6 +108,8 @@ void* current_context() {
 
 namespace hinm {
 
+void* current_cuda_context() { return current_context(); }
+
 // The address of a __device__ symbol belongs to the module loaded in one context: after
 // cudaDeviceReset (or any re-creation of the primary context) the module is loaded again
 // and the symbol can move.  The cache keeps, per device, the context the address was

@@ -55,10 +55,16 @@ cudaError_t resolve_symbol(SymbolCache& c, const void* symbol, void** out);
 // Address of the library's status word on the current device (resolve_symbol).
 int* device_status_ptr();
 
+// The CUDA context current on this thread (cuCtxGetCurrent), or nullptr when none is or the
+// driver entry point is unavailable.  Handles the library keeps (symbol addresses, function
+// attributes, the search's side stream) belong to one context and are made again when it
+// changes.
+void* current_cuda_context();
+
 // Raises kernel `fn`'s maximum dynamic shared memory on the current device to at least
-// `bytes`, calling the runtime only when the limit grows (the attribute belongs to the device,
-// and a process may drive several).  Thread-safe; call it before the first launch on each
-// device (and before stream capture).
+// `bytes`, calling the runtime only when the limit grows in the current context (the
+// attribute belongs to the context's module, and a process may drive several devices).
+// Thread-safe; call it before the first launch on each device (and before stream capture).
 cudaError_t set_max_dynamic_smem(const void* fn, int bytes);
 
 // Workspace carving helper: 256-byte aligned sub-buffers.

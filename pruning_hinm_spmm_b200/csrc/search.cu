@@ -481,6 +481,7 @@ cudaError_t launch_rank_sort(const double* V, const int32_t* perm, long long per
 struct SideStream {
   cudaStream_t stream = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
+  void* ctx = nullptr;  // the context they were made in
 };
 constexpr int kMaxSideDevices = 64;
 std::mutex g_side_mu;  // also orders the fork / join records of concurrent host threads
@@ -492,6 +493,10 @@ cudaError_t side_stream(SideStream** out) {
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxSideDevices) return cudaErrorInvalidDevice;
   SideStream& ss = g_side[dev];
+  void* ctx = current_cuda_context();
+  // handles made in another context (the device's context was made again, e.g. after
+  // cudaDeviceReset) went with it: make new ones in the current context
+  if (ss.stream && ctx && ss.ctx && ctx != ss.ctx) ss = SideStream{};
   if (!ss.stream) {
     e = cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking);
     if (e != cudaSuccess) return e;
@@ -499,6 +504,7 @@ cudaError_t side_stream(SideStream** out) {
     if (e != cudaSuccess) return e;
     e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming);
     if (e != cudaSuccess) return e;
+    ss.ctx = ctx ? ctx : current_cuda_context();
   }
   *out = &ss;
   return cudaSuccess;
