@@ -238,7 +238,7 @@ def run_reference(args, w):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": t * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "scaling": "strong", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "T": w.T,
                        "t_s": w.t_s, "alpha": w.alpha},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -902,7 +902,7 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True,
         "ms_per_step_eager": m["t_eager"] * 1e3,
-        "scaling": "strong" if world > 1 else "weak", "vs_baseline": None, "dtype": "bf16",
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": w.name, "M": M, "K": K, "N": N, "T": T, "t_s": w.t_s,
                    "alpha": w.alpha, "v_s_searched": sorted(set(np.round(m["vs"], 6).tolist())),
