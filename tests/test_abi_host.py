@@ -290,3 +290,31 @@ def test_gyro_host_validation():
     I[5, 3] = np.nan
     with pytest.raises(H.HinmError):      # non-finite in a sampled tile
         H.hinm_gyro_output_round_host(I, 4, [1, 1], np.arange(8), [1], [[0]])
+
+
+@pytest.mark.parametrize("shared", [True, False], ids=["shared_order", "per_tile_orders"])
+def test_tile_orders_with_bands_matches_oracle(H, shared):
+    """The binding's per-tile working orders after refined 2:4 bands equal the oracle's
+    tile_perm_with_band tile by tile: each row stays a permutation, the positions of
+    dense and pruned channels keep them, and the 2:4 positions hold the band in order."""
+    rng = np.random.default_rng(41)
+    nt, K = 5, 96
+    region = rng.choice([O.REGION_PRUNED, O.REGION_24, O.REGION_DENSE], size=(nt, K),
+                        p=[0.3, 0.5, 0.2]).astype(np.int8)
+    perm = (rng.permutation(K).astype(np.int32) if shared else
+            np.stack([rng.permutation(K) for _ in range(nt)]).astype(np.int32))
+    bands = []
+    for t in range(nt):
+        pt = perm if shared else perm[t]
+        members = [int(c) for c in pt if region[t][c] == O.REGION_24]
+        bands.append(rng.permutation(np.array(members, dtype=np.int32)))
+    got = H.tile_orders_with_bands(perm, region, bands)
+    assert got.shape == (nt, K) and got.dtype == np.int32
+    for t in range(nt):
+        pt = perm if shared else perm[t]
+        want = O.tile_perm_with_band(pt, region[t], bands[t])
+        np.testing.assert_array_equal(got[t], want)
+        assert sorted(got[t].tolist()) == list(range(K))
+        keep = region[t][pt] != O.REGION_24
+        np.testing.assert_array_equal(got[t][keep], pt[keep])
+        np.testing.assert_array_equal(got[t][~keep], bands[t])
