@@ -29,7 +29,14 @@
  *     memory; the library never allocates, frees or synchronises, except the *_size
  *     helpers and hinm_counts_from_vs, which run on the host only.
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
- *     Work is enqueued asynchronously on it.
+ *     Work is enqueued asynchronously on it.  The first boundary search on a device also
+ *     creates one stream and two events of the library's own (remade if the device's
+ *     context is made again); part of every search runs there, forked from and joined
+ *     back to `stream` with events, so stream capture sees one graph.
+ *   - Kernels are launched with programmatic stream serialization: a launch may begin
+ *     while the previous kernel in the stream is still running, but each kernel waits for
+ *     the stream's earlier work to finish before it touches memory, so stream order holds
+ *     as usual.
  *   - Argument checks run on the host before any launch; a failed check returns an error
  *     status and launches nothing.  hinm_last_error() then describes it.
  *   - Faults detected on the device (a malformed mask in hinm_compress, a wait that
