@@ -110,6 +110,12 @@ def test_closed_form_triples(golden_dir):
     (4096, 0.5, 0.5, (2048, 0, 2048)),      # p_s = 0: pure column pruning
     (4096, 0.0, 0.0, (0, 0, 4096)),         # dense
     (4096, 1.0, 1.0, (4096, 0, 0)),         # everything pruned
+    # the rounding of the group count (R5): 2 (t_s - v_s) K / 4 = 24.5 groups, exactly
+    # representable, rounds up to 25 (a truncation would give 24)
+    (196, 0.5, 0.25, (48, 100, 48)),
+    # t_s - v_s = 0.625 - 0.4 is 0.22499999999999998 in binary64, so the count is just
+    # below 22.5 groups and rounds to 22 (R5: evaluated in double, left to right)
+    (200, 0.625, 0.4, (81, 88, 31)),
 ])
 def test_counts_table(K, t_s, v_s, want):
     assert O.counts_from_vs(K, t_s, v_s) == want
@@ -399,6 +405,65 @@ def test_swizzle_and_meta_bijections():
     assert offs == set(range(0, 16384, 2))
     slots = {O.meta_word_index(m, g) for m in range(128) for g in range(32)}
     assert slots == {(w, 4 * n) for w in range(512) for n in range(8)}
+
+
+def test_layout_worked_examples():
+    """Positions worked by hand from the layout's definitions (a bijection test alone would
+    pass a consistent mistake in both the writer and the reader).
+
+    Values: rows are 128 bytes apart, and the 16-byte chunk of column k of row r sits at
+    chunk (k // 8) XOR (r mod 8), the 128-byte swizzle.  Metadata: word w of lane L, bits
+    [16 s + 4 q, +4), holds group 8 w + 4 ((L // 8) mod 2) + q of row
+    16 (L // 16) + 8 s + (L mod 8)."""
+    # (r, k) -> byte offset
+    for (r, k), off in {(0, 0): 0, (0, 9): 16 + 2, (1, 0): 128 + 16, (1, 8): 128 + 0,
+                        (3, 17): 3 * 128 + (2 ^ 3) * 16 + 2,
+                        (7, 63): 7 * 128 + 0 + 7 * 2}.items():
+        assert O.swizzled_offset(r, k) == off, (r, k)
+    # (row m, group g) -> (lane * 4 + word, bit shift)
+    for (m, g), slot in {(0, 0): (0, 0),            # lane 0, word 0, s = 0, q = 0
+                         (0, 1): (0, 4),            # q = 1
+                         (1, 4): (9 * 4, 0),        # group 4 is in lane half h = 1: lane 8 + 1
+                         (8, 0): (0, 16),           # row 8 is s = 1 of lane 0
+                         (9, 13): (9 * 4 + 1, 20),  # word 1, h = 1, q = 1; s = 1, lane 9
+                         (16, 0): (16 * 4, 0),      # rows 16.. are lanes 16..
+                         (5, 9): (5 * 4 + 1, 4),    # word 1, h = 0, q = 1
+                         (127, 31): (127 * 4 + 3, 28)}.items():
+        assert O.meta_word_index(m, g) == slot, (m, g)
+
+
+@pytest.mark.parametrize("perm", [False, True], ids=["identity", "permuted"])
+def test_all_equal_importances_follow_the_tie_rules(perm):
+    """Every importance equal (W = X = 1): every vector score ties, so the ranking is the
+    working order (R4: the lower working position ranks higher) -- the first n_4 working
+    positions dense, the next n_24 in 2:4, the rest pruned -- and in every 2:4 group every
+    row keeps its first two members (R7: equal values, the lower position wins)."""
+    T, K, N = 64, 64, 8
+    W = bf(np.ones((2 * T, K)))
+    X = bf(np.ones((K, N)))
+    p = np.random.default_rng(4).permutation(K).astype(np.int32) if perm else np.arange(K, dtype=np.int32)
+    n0, n24, n4 = O.counts_from_vs(K, 0.5, 0.25)
+    I = O.importance(W, X)
+    sr = O.boundary_search(I, p, T, 0.5, 1 / 32)
+    for t in range(2):
+        np.testing.assert_array_equal(sr.rank[t], np.arange(K))
+    counts = np.tile(np.array([n0, n24, n4], dtype=np.int32), (2, 1))
+    bm, reg = O.mask(I, p, T, counts)
+    keep = O.unpack_bits(bm, K)
+    for t in range(2):
+        want_reg = np.empty(K, dtype=np.int8)
+        want_keep = np.zeros(K, dtype=bool)
+        for j in range(K):
+            c = p[j]
+            if j < n4:
+                want_reg[c], want_keep[c] = O.REGION_DENSE, True
+            elif j < n4 + n24:
+                want_reg[c], want_keep[c] = O.REGION_24, (j - n4) % 4 < 2
+            else:
+                want_reg[c] = O.REGION_PRUNED
+        np.testing.assert_array_equal(reg[t], want_reg)
+        for r in range(t * T, (t + 1) * T):
+            np.testing.assert_array_equal(keep[r], want_keep)
 
 
 @pytest.mark.parametrize("T,K,t_s,v_s,perm", [
