@@ -369,6 +369,53 @@ def _gyro_round_keeps_worse(I_tile, band, groups, slots, kmeans_iters=8):
     return new, (before, after)
 
 
+# ------------------------------------------------------------------ orders and signs
+def _energy_descending(X_bits):
+    X = O._bf16_to_f64(X_bits)
+    acc = np.zeros(X.shape[0])
+    for n in reversed(range(X.shape[1])):
+        acc += X[:, n] * X[:, n]
+    return acc.astype(np.float32)
+
+
+def _scores_fp32(I, perm, T):
+    M, K = I.shape
+    nt = M // T
+    Iw = (I[:, perm].reshape(nt, T, K) if np.asarray(perm).ndim == 1 else
+          np.stack([I[t * T:(t + 1) * T][:, O.tile_perm(perm, t)] for t in range(nt)]))
+    V = np.zeros((nt, K), dtype=np.float32)
+    for i in range(T):
+        V = (V + Iw[:, i, :].astype(np.float32)).astype(np.float32)
+    return V.astype(np.float64)
+
+
+def _scan_from_the_other_end(R):
+    """The scan starts at the last candidate (v_s lowest) and walks up."""
+    for m in range(len(R) - 1, 0, -1):
+        if R[m - 1] < R[m]:
+            return m
+    return 0
+
+
+def _spmm_bound_signed(W_bits, bitmask, X_bits, rows=None):
+    y, _ = _orig["spmm_reference"](W_bits, bitmask, X_bits, rows)
+    Wm = O.masked_weight(W_bits if rows is None else W_bits[rows],
+                         bitmask if rows is None else bitmask[rows])
+    return y, Wm @ O._bf16_to_f64(X_bits)
+
+
+def _hc_logit_sign(log_alpha, eps, tau):
+    e = np.asarray(eps, dtype=np.float64)
+    return _orig["hard_concrete"](log_alpha, 1.0 - e, tau)
+
+
+def _silu_wrong_sign(x, act):
+    if act == O.ACT_SILU:
+        x = np.asarray(x, dtype=np.float64)
+        return x / (1.0 + np.exp(x))
+    return _orig["activation"](x, act)
+
+
 MUTANTS = {
     "energy_drops_square": {"channel_energy": _energy_drops_square},
     "energy_over_wrong_axis": {"channel_energy": _energy_over_wrong_axis},
@@ -405,6 +452,12 @@ MUTANTS = {
     "index_without_permutation": {"compress": _compress_index_not_permuted},
     "retained_in_fp32": {"retained_importance": _retained_fp32},
     "gyro_keeps_worse_rounds": {"gyro_input_round": _gyro_round_keeps_worse},
+    "energy_sums_descending": {"channel_energy": _energy_descending},
+    "scores_in_fp32": {"vector_scores": _scores_fp32},
+    "scan_from_the_other_end": {"boundary_search": _search_with(_scan_from_the_other_end)},
+    "bound_signed": {"spmm_reference": _spmm_bound_signed},
+    "hard_concrete_logit_sign": {"hard_concrete": _hc_logit_sign},
+    "silu_wrong_sign": {"activation": _silu_wrong_sign},
 }
 
 

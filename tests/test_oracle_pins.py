@@ -77,6 +77,22 @@ def test_importance_rows_hand_example():
                                   np.array([[27, 1], [3, 16]], dtype=np.float32))
 
 
+def test_vector_scores_accumulate_in_fp64():
+    """R3: a vector's score is the fp64 sum of its importances.  Column a holds 1 and then
+    63 values of 2^-25 (exact sum 1 + 63 * 2^-25, exact in fp64; an fp32 running sum would
+    stay at 1), column b holds 1 + 2^-23 and zeros: a outranks b only with the fp64 sum."""
+    T = 64
+    I = np.zeros((T, 4), dtype=np.float32)
+    I[0, 0] = 1.0
+    I[1:, 0] = np.float32(2.0 ** -25)
+    I[0, 1] = np.float32(1.0 + 2.0 ** -23)
+    I[:, 2] = np.float32(2.0 ** -30)
+    V = O.vector_scores(I, np.arange(4, dtype=np.int32), T)
+    assert Fraction(float(V[0, 0])) == 1 + 63 * Fraction(1, 2 ** 25)
+    assert float(V[0, 1]) == 1.0 + 2.0 ** -23
+    np.testing.assert_array_equal(O.vector_order(V[0]), [0, 1, 2, 3])
+
+
 def test_importance_exact_rational():
     rng = np.random.default_rng(3)
     M, K, N = 5, 6, 9
@@ -598,6 +614,16 @@ def test_hard_concrete_closed_forms():
     z2, _, s2 = O.hard_concrete(np.array([50.0, -50.0, 50.0, -50.0] * 3), np.full(12, 0.5), tau)
     np.testing.assert_array_equal(z2, [1.0, 0.0] * 6)
     np.testing.assert_array_equal(s2, [6.0, 0.0])
+
+
+def test_hard_concrete_noise_enters_as_log_eps_minus_log_one_minus_eps():
+    """A worked value at an asymmetric noise draw: eps = 3/4, log alpha = 0, tau = 1 give
+    the logit log 3, s = 3/4 and z = 1.2 * 3/4 - 0.1 = 0.8; eps = 1/4 gives s = 1/4 and
+    z = 0.2.  (The mirror identity and the clip masses are symmetric in eps <-> 1 - eps,
+    so they alone would not tell the two apart.)"""
+    z, hard, _ = O.hard_concrete(np.zeros(4), np.array([0.75, 0.25, 0.75, 0.25]), 1.0)
+    np.testing.assert_allclose(z, [0.8, 0.2, 0.8, 0.2], rtol=0, atol=1e-15)
+    np.testing.assert_array_equal(hard, [1, 0, 1, 0])
 
 
 def test_hard_concrete_mirror_and_regularisers():
