@@ -318,3 +318,23 @@ def test_tile_orders_with_bands_matches_oracle(H, shared):
         keep = region[t][pt] != O.REGION_24
         np.testing.assert_array_equal(got[t][keep], pt[keep])
         np.testing.assert_array_equal(got[t][~keep], bands[t])
+
+
+def test_empty_inputs_are_refused_before_launch(H):
+    """Empty problems (no rows, no channels, no columns) are shape errors reported on the
+    host: nothing is launched and no pointer is read."""
+    lib = H.lib()
+    fake = 0x10000
+    for M, K, N in [(0, 64, 16), (64, 0, 16), (64, 64, 0)]:
+        assert lib.hinm_importance(fake, fake, M, K, N, fake, fake, 1 << 20,
+                                   None) == H.HINM_ERR_SHAPE, (M, K, N)
+    for M, K in [(0, 64), (128, 0)]:
+        assert lib.hinm_boundary_search(fake, None, M, K, 64, 0.5, 1 / 32, fake, fake, None,
+                                        None, fake, 1 << 30, None) == H.HINM_ERR_SHAPE, (M, K)
+        assert lib.hinm_mask(fake, None, fake, None, M, K, 64, fake, fake, fake, 1 << 30,
+                             None) == H.HINM_ERR_SHAPE, (M, K)
+    ws = ctypes.c_size_t(0)
+    assert lib.hinm_search_workspace_size(0, 64, 64, 0.5, 1 / 32, ctypes.byref(ws)) == H.HINM_ERR_SHAPE
+    L = H.hinm_layout(H.HINM_LAYOUT_VERSION, 256, 256, 64, 4, 1, 1, fake, fake, fake, fake, fake,
+                      fake, fake, fake)
+    assert lib.hinm_spmm(ctypes.byref(L), fake, 0, fake, None) == H.HINM_ERR_SHAPE
