@@ -416,6 +416,28 @@ def _silu_wrong_sign(x, act):
     return _orig["activation"](x, act)
 
 
+# ------------------------------------------------------------------ layout bookkeeping
+def _tile_blocks_floor(counts):
+    nt = counts.shape[0]
+    info = np.zeros((nt, 4), dtype=np.int32)
+    d0 = s0 = 0
+    for t in range(nt):
+        n0, n24, n4 = (int(x) for x in counts[t])
+        nd, ns = n4 // O.DENSE_BK, n24 // O.SPARSE_BK
+        info[t] = (nd, ns, d0, s0)
+        d0 += nd
+        s0 += ns
+    return info
+
+
+def _runs_any_ascending(idx):
+    out = np.full(idx.shape[0], -1, dtype=np.int32)
+    if idx.shape[0]:
+        run = (np.diff(idx, axis=1) > 0).all(axis=1)
+        out[run] = idx[run, 0]
+    return out
+
+
 MUTANTS = {
     "energy_drops_square": {"channel_energy": _energy_drops_square},
     "energy_over_wrong_axis": {"channel_energy": _energy_over_wrong_axis},
@@ -458,6 +480,8 @@ MUTANTS = {
     "bound_signed": {"spmm_reference": _spmm_bound_signed},
     "hard_concrete_logit_sign": {"hard_concrete": _hc_logit_sign},
     "silu_wrong_sign": {"activation": _silu_wrong_sign},
+    "tile_blocks_round_down": {"tile_blocks": _tile_blocks_floor},
+    "runs_accept_any_ascending_indices": {"contiguous_runs": _runs_any_ascending},
 }
 
 
